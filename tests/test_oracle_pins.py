@@ -1,0 +1,419 @@
+"""Pins of the CPU oracle to things other than itself.
+
+Each test checks an oracle function against a closed form, a hand-computed
+golden case (tests/golden/), a library routine that computes the same
+quantity by another route, a brute-force enumeration on tiny inputs, or an
+invariant of the mathematics -- chosen so that a dropped term, a wrong sign or
+index, or a transposed operand fails at least one of them.
+"""
+import itertools
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import ssa_oracle as O
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def golden(name):
+    with open(os.path.join(GOLDEN, name)) as f:
+        return json.load(f)
+
+
+def small_problem(**kw):
+    base = dict(batch=1, n_q=32, n_kv=32, h_q=1, h_kv=1, d=4, block=4, topk=2, window=4,
+                dtype=O.F32, sigma=O.FULL, beta=2.0)
+    base.update(kw)
+    return O.Problem(**base)
+
+
+# ------------------------------------------------------------------ rounding
+
+def test_round_bf16_matches_torch_and_ties_to_even():
+    rng = np.random.default_rng(1)
+    x = np.concatenate([rng.standard_normal(20000).astype(np.float32) * 10.0 ** rng.integers(-6, 6, 20000),
+                        np.float32([1.0, 1.0 + 2 ** -8, 1.0 + 3 * 2 ** -8, -1.0 - 2 ** -8, 0.0, -0.0, 3.0e38])])
+    ours = O.round_bf16(x)
+    ref = torch.from_numpy(x.astype(np.float32)).to(torch.bfloat16).to(torch.float64).numpy()
+    assert np.array_equal(ours, ref)
+    # exact halfway cases round to the even neighbour
+    assert O.round_bf16(np.float32(1.0 + 2 ** -8)) == 1.0
+    assert O.round_bf16(np.float32(1.0 + 3 * 2 ** -8)) == 1.0 + 2 ** -6
+
+
+def test_round_f32_matches_numpy_cast():
+    x = np.random.default_rng(2).standard_normal(1000) * 1e3
+    assert np.array_equal(O.round_f32(x), x.astype(np.float32).astype(np.float64))
+
+
+# ------------------------------------------------------------------ summaries
+
+def test_summaries_golden_two_blocks():
+    g = golden("cumulant_routing_outlier.json")
+    K = np.array(g["keys"], dtype=np.float64).reshape(1, 4, 1, 2)
+    pd = small_problem(n_q=4, n_kv=4, d=2, block=2, sigma=O.DIAG)
+    mu, var = O.block_summaries(K, pd)
+    assert np.array_equal(mu[0, 0], np.array(g["mu"], dtype=float))
+    assert np.array_equal(var[0, 0], np.array(g["var"], dtype=float))
+    pf = small_problem(n_q=4, n_kv=4, d=2, block=2, sigma=O.FULL)
+    _, cov = O.block_summaries(K, pf)
+    assert np.array_equal(cov[0, 0], np.array(g["cov"], dtype=float))
+
+
+def test_summaries_match_numpy_mean_and_population_cov():
+    rng = np.random.default_rng(3)
+    K = rng.standard_normal((2, 24, 3, 5))
+    p = small_problem(batch=2, n_q=24, n_kv=24, h_q=3, h_kv=3, d=5, block=8, sigma=O.FULL)
+    mu, cov = O.block_summaries(K, p)
+    _, var = O.block_summaries(K, O.Problem(**{**p.__dict__, "sigma": O.DIAG}))
+    for bi in range(2):
+        for h in range(3):
+            for c in range(3):
+                keys = K[bi, c * 8:(c + 1) * 8, h]
+                np.testing.assert_allclose(mu[bi, h, c], keys.mean(axis=0), rtol=0, atol=1e-14)
+                np.testing.assert_allclose(cov[bi, h, c], np.cov(keys.T, bias=True), rtol=0, atol=1e-13)
+                np.testing.assert_allclose(var[bi, h, c], keys.var(axis=0), rtol=0, atol=1e-14)
+
+
+def test_summary_invariants_shift_scale_psd():
+    rng = np.random.default_rng(4)
+    K = rng.standard_normal((1, 16, 1, 6))
+    p = small_problem(n_q=16, n_kv=16, d=6, block=8, sigma=O.FULL)
+    mu, cov = O.block_summaries(K, p)
+    shift = rng.standard_normal(6)
+    K2 = K.copy()
+    K2[0, :8, 0] += shift                      # shift block 0 only
+    mu2, cov2 = O.block_summaries(K2, p)
+    np.testing.assert_allclose(mu2[0, 0, 0], mu[0, 0, 0] + shift, atol=1e-13)
+    np.testing.assert_allclose(mu2[0, 0, 1], mu[0, 0, 1], atol=0)
+    np.testing.assert_allclose(cov2, cov, atol=1e-13)
+    mu3, cov3 = O.block_summaries(3.0 * K, p)
+    np.testing.assert_allclose(cov3, 9.0 * cov, rtol=1e-13)
+    for c in range(2):
+        S = cov[0, 0, c]
+        assert np.allclose(S, S.T)
+        assert np.linalg.eigvalsh(S).min() > -1e-12
+    # a block of identical keys has zero spread
+    K4 = np.repeat(O.round_bf16(rng.standard_normal((1, 1, 1, 6))), 16, axis=1)
+    _, cov4 = O.block_summaries(K4, p)
+    assert np.abs(cov4).max() == 0
+
+
+def test_stored_table_is_bf16_of_f32():
+    rng = np.random.default_rng(5)
+    K = torch.randn(1, 64, 2, 8, generator=torch.Generator().manual_seed(5)).to(torch.bfloat16).float().numpy()
+    p = small_problem(n_q=64, n_kv=64, h_q=2, h_kv=2, d=8, block=16, dtype=O.BF16, sigma=O.DIAG)
+    mu, var = O.block_summaries(K, p)
+    mu32, var32, tab = O.stored_summaries(mu, var, p)
+    t = torch.from_numpy(np.concatenate([mu, var], axis=-1)).to(torch.float32).to(torch.bfloat16).double().numpy()
+    assert np.array_equal(tab, t)
+    assert tab.shape == (1, 2, 4, 16)
+    del rng
+
+
+# ------------------------------------------------------------------ routing score
+
+def test_routing_golden_outlier_block():
+    g = golden("cumulant_routing_outlier.json")
+    K = np.array(g["keys"], dtype=np.float64).reshape(1, 4, 1, 2)
+    Q = np.array(g["q"], dtype=np.float64).reshape(1, 1, 1, 2)
+    for beta, key_r, key_top in ((2.0, "r_beta2", "top1_beta2"), (0.0, "r_beta0", "top1_beta0")):
+        for sigma in (O.DIAG, O.FULL):
+            p = small_problem(n_q=1, n_kv=4, d=2, block=2, topk=1, window=1, q_offset=3,
+                              beta=beta, sigma=sigma)
+            stored = O.stored_summaries(*O.block_summaries(K, p), p)
+            s = O.route_scores_row(Q, stored, p, 0, 0, 0)
+            assert np.array_equal(s, np.array(g[key_r], dtype=float))
+            sel, _ = O.select_topk(s, 1)
+            assert sel[0] == g[key_top]
+
+
+def _dyadic_keys(rng, shape):
+    return rng.integers(-4, 5, size=shape).astype(np.float64)   # exact in fp32 and after /4, /16
+
+
+def test_full_sigma_score_equals_logit_mean_plus_half_beta_logit_variance():
+    """r_c(q) computed from mu_c / Sigma_c must equal the mean of the block's
+    logits q.k_j plus (beta/2) times their population variance."""
+    rng = np.random.default_rng(6)
+    for beta in (0.0, 0.5, 2.0, -1.0):
+        K = _dyadic_keys(rng, (1, 32, 1, 4))
+        Q = _dyadic_keys(rng, (1, 32, 1, 4))
+        p = small_problem(beta=beta)
+        stored = O.stored_summaries(*O.block_summaries(K, p), p)
+        for i in (3, 17, 31):
+            s = O.route_scores_row(Q, stored, p, 0, i, 0)
+            nv = O.visible_blocks(i, p)
+            for c in range(nv):
+                logits = [float(np.dot(Q[0, i, 0], K[0, c * 4 + j, 0])) for j in range(4)]
+                m = sum(logits) / 4
+                v = sum((x - m) ** 2 for x in logits) / 4
+                assert s[c] == pytest.approx(m + beta / 2 * v, rel=1e-12, abs=1e-12)
+
+
+def test_diag_score_matches_per_dimension_variance_and_full_when_uncorrelated():
+    rng = np.random.default_rng(7)
+    K = _dyadic_keys(rng, (1, 32, 1, 4))
+    Q = _dyadic_keys(rng, (1, 32, 1, 4))
+    p = small_problem(sigma=O.DIAG)
+    stored = O.stored_summaries(*O.block_summaries(K, p), p)
+    s = O.route_scores_row(Q, stored, p, 0, 31, 0)
+    q = Q[0, 31, 0]
+    for c in range(8):
+        keys = K[0, c * 4:(c + 1) * 4, 0]
+        direct = q @ keys.mean(axis=0) + 1.0 * np.sum(q * q * keys.var(axis=0))
+        assert s[c] == pytest.approx(direct, rel=1e-12, abs=1e-12)
+    # keys with exactly diagonal covariance: rows of a Hadamard pattern
+    H = np.array([[1, 1, 1], [1, -1, -1], [-1, 1, -1], [-1, -1, 1]], dtype=np.float64)
+    K2 = np.zeros((1, 8, 1, 3))
+    K2[0, :4, 0] = H * np.array([1.0, 2.0, 0.5]) + 1.0
+    K2[0, 4:, 0] = H * np.array([3.0, 0.25, 1.0]) - 2.0
+    Q2 = np.tile(np.array([0.5, -1.0, 2.0]), (1, 8, 1, 1))
+    pd = small_problem(n_q=8, n_kv=8, d=3, block=4, sigma=O.DIAG)
+    pf = small_problem(n_q=8, n_kv=8, d=3, block=4, sigma=O.FULL)
+    sd = O.route_scores_row(Q2, O.stored_summaries(*O.block_summaries(K2, pd), pd), pd, 0, 7, 0)
+    sf = O.route_scores_row(Q2, O.stored_summaries(*O.block_summaries(K2, pf), pf), pf, 0, 7, 0)
+    np.testing.assert_allclose(sd, sf, rtol=1e-14)
+
+
+def test_beta_zero_is_centroid_routing():
+    rng = np.random.default_rng(8)
+    K = rng.standard_normal((1, 64, 1, 8)).astype(np.float32).astype(np.float64)
+    Q = rng.standard_normal((1, 64, 1, 8)).astype(np.float32).astype(np.float64)
+    p = small_problem(n_q=64, n_kv=64, d=8, block=8, beta=0.0, sigma=O.FULL)
+    stored = O.stored_summaries(*O.block_summaries(K, p), p)
+    s = O.route_scores_row(Q, stored, p, 0, 63, 0)
+    mean_logit = np.array([np.mean(K[0, c * 8:(c + 1) * 8, 0] @ Q[0, 63, 0]) for c in range(8)])
+    np.testing.assert_allclose(s, mean_logit, rtol=1e-6, atol=1e-6)   # fp32-rounded mu
+
+
+def test_group_score_is_sum_of_head_scores():
+    rng = np.random.default_rng(9)
+    K = _dyadic_keys(rng, (1, 32, 2, 4))
+    Q = _dyadic_keys(rng, (1, 32, 8, 4))
+    for sigma in (O.DIAG, O.FULL):
+        p = small_problem(h_q=8, h_kv=2, sigma=sigma)
+        stored = O.stored_summaries(*O.block_summaries(K, p), p)
+        s = O.route_scores_row(Q, stored, p, 0, 30, 1)
+        per_head = np.zeros_like(s)
+        for h in range(4, 8):
+            ph = small_problem(h_q=1, h_kv=1, sigma=sigma)
+            st = O.stored_summaries(*O.block_summaries(K[:, :, 1:2], ph), ph)
+            per_head += O.route_scores_row(Q[:, :, h:h + 1], st, ph, 0, 30, 0)
+        np.testing.assert_allclose(s, per_head, rtol=1e-13)
+
+
+def test_bf16_features_exact_case_equals_group_score():
+    """With small-integer queries every feature rounding is exact, so the bf16
+    route equals the exact group score on the bf16 table."""
+    rng = np.random.default_rng(10)
+    K = torch.randn(1, 64, 2, 8, generator=torch.Generator().manual_seed(10)).to(torch.bfloat16).float().numpy()
+    Q = rng.integers(-3, 4, size=(1, 64, 4, 8)).astype(np.float64)
+    p = O.Problem(batch=1, n_q=64, n_kv=64, h_q=4, h_kv=2, d=8, block=16, topk=2, window=16,
+                  dtype=O.BF16, sigma=O.DIAG, beta=2.0)
+    stored = O.stored_summaries(*O.block_summaries(K, p), p)
+    tab = stored[2]
+    F = O.route_features(Q, p)
+    for g in range(2):
+        qs = Q[0, 40, 2 * g:2 * g + 2].sum(axis=0)
+        qq = (Q[0, 40, 2 * g:2 * g + 2] ** 2).sum(axis=0)
+        np.testing.assert_array_equal(F[0, g, 40], np.concatenate([qs, qq]))
+        s = O.route_scores_row(Q, stored, p, 0, 40, g)
+        direct = sum(Q[0, 40, h] @ tab[0, g, :, :8].T + (Q[0, 40, h] ** 2) @ tab[0, g, :, 8:].T
+                     for h in (2 * g, 2 * g + 1))[:2]
+        np.testing.assert_allclose(s, direct, rtol=1e-14)
+    # the full-row and the per-row route agree
+    S = O.route_scores(Q, stored, p, 0, 1)
+    np.testing.assert_allclose(S[40, :2], O.route_scores_row(Q, stored, p, 0, 40, 1), rtol=1e-14)
+
+
+def test_visible_blocks_brute_force():
+    p = small_problem(n_kv=64, block=8)
+    for pos in range(64):
+        brute = sum(1 for c in range(8) if (c + 1) * 8 - 1 <= pos)
+        assert O.visible_blocks(pos, p) == brute
+
+
+# ------------------------------------------------------------------ top-k
+
+def test_topk_brute_force_with_ties():
+    rng = np.random.default_rng(11)
+    for trial in range(300):
+        nv = int(rng.integers(1, 8))
+        k = int(rng.integers(1, 6))
+        s = rng.integers(-3, 3, size=nv).astype(np.float64)      # many exact ties
+        sel, gap = O.select_topk(s, k)
+        take = min(k, nv)
+        # brute force: the unique subset whose every member beats every non-member
+        # under (higher score, then lower index)
+        beats = lambda a, b: s[a] > s[b] or (s[a] == s[b] and a < b)
+        found = None
+        for sub in itertools.combinations(range(nv), take):
+            rest = [c for c in range(nv) if c not in sub]
+            if all(beats(a, b) for a in sub for b in rest):
+                assert found is None
+                found = sub
+        assert list(sel[:take]) == sorted(found)
+        assert all(x == -1 for x in sel[take:])
+        if nv > k:
+            srt = sorted(s, reverse=True)
+            expect = (srt[k - 1] - srt[k]) / abs(srt[k - 1]) if srt[k - 1] != 0 else (
+                np.inf if srt[k - 1] > srt[k] else 0.0)
+            assert gap == expect
+
+
+# ------------------------------------------------------------------ key set
+
+def test_key_set_brute_force():
+    p = small_problem(n_kv=64, block=8, window=11)
+    rng = np.random.default_rng(12)
+    for _ in range(100):
+        pos = int(rng.integers(0, 64))
+        nv = O.visible_blocks(pos, p)
+        cand = list(range(nv))
+        rng.shuffle(cand)
+        sel = np.array(sorted(cand[:3]) + [-1] * (3 - min(3, nv)))
+        S = O.key_set(pos, sel, p)
+        brute = [j for j in range(64) if (j // 8 in set(sel[sel >= 0])) or (pos - 11 < j <= pos)]
+        assert list(S) == brute
+        assert all(j <= pos for j in S)
+
+
+# ------------------------------------------------------------------ attention
+
+def test_softmax_golden_three_keys():
+    g = golden("softmax_three_keys.json")
+    q = np.array([g["q"]])
+    Ks = np.array(g["keys"])[:, None]
+    Vs = np.array(g["values"])[:, None]
+    o, lse = O.softmax_attend(q, Ks, Vs, 1.0)
+    assert o[0, 0] == pytest.approx(g["o"], rel=1e-15)
+    assert lse[0] == pytest.approx(g["lse"], rel=1e-15)
+
+
+def test_full_budget_equals_dense_causal_attention():
+    """With k >= number of blocks and W >= B every earlier key is attended,
+    so the layer must reduce to dense causal softmax attention."""
+    rng = np.random.default_rng(13)
+    for G, sigma in ((1, O.FULL), (4, O.DIAG)):
+        p = O.Problem(batch=2, n_q=48, n_kv=48, h_q=2 * G, h_kv=2, d=8, block=8, topk=6, window=8,
+                      dtype=O.F32, sigma=sigma)
+        Q = rng.standard_normal((2, 48, 2 * G, 8))
+        K = rng.standard_normal((2, 48, 2, 8))
+        V = rng.standard_normal((2, 48, 2, 8))
+        out = O.forward(Q, K, V, p)
+        Od, Ld = O.dense_causal_attention(Q, K, V, p)
+        np.testing.assert_allclose(out["O"], Od, rtol=0, atol=1e-12)
+        np.testing.assert_allclose(out["lse"], Ld, rtol=0, atol=1e-12)
+    # decode: the single query at the last position equals the dense last row
+    p = O.Problem(batch=1, n_q=1, n_kv=48, h_q=4, h_kv=2, d=8, block=8, topk=6, window=8,
+                  q_offset=47, dtype=O.F32, sigma=O.DIAG)
+    Qd = rng.standard_normal((1, 1, 4, 8))
+    out = O.forward(Qd, K[:1], V[:1], p)
+    Od, _ = O.dense_causal_attention(Qd, K[:1], V[:1], p)
+    np.testing.assert_allclose(out["O"], Od, atol=1e-12)
+
+
+def test_recovery_law_golden_and_exact_construction():
+    for c in golden("recovery_law.json")["cases"]:
+        assert O.recovery_weight(c["beta"], c["delta"], c["mu"]) == pytest.approx(c["w"], rel=1e-12)
+    # exact construction: q = a e1, mu distractors orthogonal to e1, one target
+    # at first coordinate Delta/a; V = e1 on the target only.  The attention
+    # output's first coordinate is the target weight w* at beta = scale.
+    d, a = 8, 2.0
+    rng = np.random.default_rng(14)
+    for mu, delta in ((7, 1.5), (63, 4.0), (255, 6.0)):
+        Ks = np.zeros((mu + 1, d))
+        Ks[:mu, 1:] = rng.standard_normal((mu, d - 1))
+        Ks[mu, 0] = delta / a
+        Vs = np.zeros((mu + 1, d))
+        Vs[mu, 0] = 1.0
+        q = np.zeros((1, d))
+        q[0, 0] = a
+        scale = 1 / math.sqrt(d)
+        o, _ = O.softmax_attend(q, Ks, Vs, scale)
+        assert o[0, 0] == pytest.approx(O.recovery_weight(scale, delta, mu), rel=1e-12)
+
+
+def test_selection_cuts_distractors_recovery_improves():
+    """Selection cuts mu from the causal prefix to the budget: the recovered
+    target weight under SSA equals w* with mu = |S|-1, which is larger than
+    dense attention's w* with mu = pos."""
+    d, B = 8, 8
+    n = 256
+    K = np.zeros((1, n, 1, d))
+    rng = np.random.default_rng(15)
+    K[0, :, 0, 1:] = rng.standard_normal((n, d - 1)) * 0.0     # all distractor logits 0
+    tgt = 40
+    delta = 12.0
+    K[0, tgt, 0, 0] = delta / 2.0
+    V = np.zeros((1, n, 1, d))
+    V[0, tgt, 0, 0] = 1.0
+    Q = np.zeros((1, n, 1, d))
+    Q[0, :, 0, 0] = 2.0
+    p = O.Problem(batch=1, n_q=n, n_kv=n, h_q=1, h_kv=1, d=d, block=B, topk=2, window=8,
+                  dtype=O.F32, sigma=O.DIAG)
+    out = O.forward(Q, K, V, p, rows=[(0, 255)])
+    Od, _ = O.dense_causal_attention(Q, K, V, p)
+    S = O.key_set(255, out["block_idx"][0, 255, 0], p)
+    assert tgt in S
+    w_sparse = out["O"][0, 255, 0, 0]
+    assert w_sparse == pytest.approx(O.recovery_weight(p.scale, delta, len(S) - 1), rel=1e-12)
+    assert Od[0, 255, 0, 0] == pytest.approx(O.recovery_weight(p.scale, delta, 255), rel=1e-12)
+    assert w_sparse > Od[0, 255, 0, 0]
+
+
+def test_dropped_mass_identity_and_bound():
+    """o_S - o_dense = eps (o_S - o_D), eps = dense softmax mass outside S and
+    o_D the dense-normalised average of the dropped values; hence
+    |o_S - o_dense|_inf <= eps * max_t (max_j v_jt - min_j v_jt)."""
+    rng = np.random.default_rng(16)
+    p = O.Problem(batch=1, n_q=128, n_kv=128, h_q=2, h_kv=1, d=8, block=8, topk=3, window=8,
+                  dtype=O.F32, sigma=O.DIAG)
+    Q = rng.standard_normal((1, 128, 2, 8)) * 1.5
+    K = rng.standard_normal((1, 128, 1, 8))
+    V = rng.standard_normal((1, 128, 1, 8))
+    rows = [(0, i) for i in (40, 77, 127)]
+    out = O.forward(Q, K, V, p, rows=rows)
+    Od, _ = O.dense_causal_attention(Q, K, V, p)
+    for _, i in rows:
+        S = O.key_set(i, out["block_idx"][0, i, 0], p)
+        D = np.setdiff1d(np.arange(i + 1), S)
+        for h in range(2):
+            logits = (K[0, :i + 1, 0] @ Q[0, i, h]) * p.scale
+            w = np.exp(logits - logits.max())
+            w /= w.sum()
+            eps = w[D].sum()
+            oD = (w[D, None] * V[0, D, 0]).sum(axis=0) / eps
+            oS = out["O"][0, i, h]
+            np.testing.assert_allclose(oS - Od[0, i, h], eps * (oS - oD), atol=1e-10)
+            spread = V[0, :i + 1, 0].max(axis=0) - V[0, :i + 1, 0].min(axis=0)
+            assert np.abs(oS - Od[0, i, h]).max() <= eps * spread.max() + 1e-12
+
+
+def test_cumulant_routing_recovers_needles_centroid_misses():
+    """On clustered keys with planted needles, second-cumulant routing (beta=2)
+    puts the needle's block in the budget far more often than centroid
+    routing (beta=0)."""
+    from content_routed_block_ssa_b200.workload import WORKLOADS, make_inputs
+    w = WORKLOADS["gqa_bf16_128k"].scaled(n=4096, needles=48, topk=4)
+    Q, K, V, plan = make_inputs(w)
+    Q, K = Q.float().numpy(), K.float().numpy()
+    hits = {}
+    for beta in (2.0, 0.0):
+        p = O.Problem(batch=1, n_q=w.n, n_kv=w.n, h_q=w.h_q, h_kv=w.h_kv, d=w.d, block=w.block,
+                      topk=w.topk, window=w.window, beta=beta, dtype=O.BF16, sigma=O.DIAG)
+        stored = O.stored_summaries(*O.block_summaries(K, p), p)
+        h = 0
+        for (bi, i, head, j) in plan:
+            s = O.route_scores_row(Q, stored, p, bi, i, head // p.group)
+            sel, _ = O.select_topk(s, p.topk)
+            h += int(j // p.block in set(sel))
+        hits[beta] = h / len(plan)
+    assert hits[2.0] >= 0.95
+    assert hits[2.0] > hits[0.0] + 0.3
