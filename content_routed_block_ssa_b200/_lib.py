@@ -1,0 +1,181 @@
+"""ctypes binding of libssa (include/ssa.h): argument marshalling only.
+
+Every function takes torch tensors (device or, for ``ssa_forward_hostio``,
+host) or None, passes their data pointers and the CUDA stream to the C ABI,
+and raises ``SSAError`` on a non-zero status.  All computation happens in the
+CUDA kernels behind the ABI; there is no other implementation to fall back
+to, and importing this module fails if ``libssa.so`` has not been built.
+"""
+from __future__ import annotations
+
+import ctypes as C
+import math
+import os
+
+import torch
+
+_LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libssa.so")
+
+SSA_OK, SSA_ERR_INVALID_ARG, SSA_ERR_UNSUPPORTED, SSA_ERR_WORKSPACE, SSA_ERR_CUDA, SSA_ERR_DEVICE = range(6)
+SSA_F32, SSA_BF16 = 0, 1
+SSA_SIGMA_DIAG, SSA_SIGMA_FULL = 0, 1
+SSA_ROUTE_AUTO, SSA_ROUTE_TILED, SSA_ROUTE_ROWWISE = 0, 1, 2
+
+
+class SSAError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        super().__init__(f"{what}: {status_string(status)} ({status})")
+        self.status = status
+
+
+class ssa_params(C.Structure):
+    _fields_ = [("batch", C.c_int32), ("n_q", C.c_int32), ("n_kv", C.c_int32), ("h_q", C.c_int32),
+                ("h_kv", C.c_int32), ("d", C.c_int32), ("block", C.c_int32), ("topk", C.c_int32),
+                ("window", C.c_int32), ("dtype", C.c_int32), ("sigma", C.c_int32),
+                ("route_impl", C.c_int32), ("q_offset", C.c_int64), ("beta", C.c_float),
+                ("scale", C.c_float)]
+
+
+assert C.sizeof(ssa_params) == 64
+
+
+def _load():
+    if not os.path.exists(_LIB_PATH):
+        raise ImportError(f"{_LIB_PATH} is missing: build it with "
+                          "`python -m content_routed_block_ssa_b200.build` (nvcc, sm_100a)")
+    lib = C.CDLL(_LIB_PATH)
+    P = C.POINTER(ssa_params)
+    vp, sz, i32 = C.c_void_p, C.c_size_t, C.c_int32
+    sig = {
+        "ssa_status_string": (C.c_char_p, [i32]),
+        "ssa_version": (i32, []),
+        "ssa_launch_count": (C.c_uint64, []),
+        "ssa_device_error": (i32, [C.POINTER(C.c_uint32)]),
+        "ssa_block_summary": (i32, [P, vp, vp, vp, vp, vp]),
+        "ssa_route_workspace_size": (sz, [P]),
+        "ssa_route_topk": (i32, [P, vp, vp, vp, vp, vp, vp, vp, sz, vp]),
+        "ssa_sparse_attn": (i32, [P, vp, vp, vp, vp, vp, vp, vp, vp]),
+        "ssa_workspace_size": (sz, [P]),
+        "ssa_forward": (i32, [P, vp, vp, vp, vp, vp, vp, sz, vp]),
+        "ssa_hostio_buffer_size": (sz, [P]),
+        "ssa_forward_hostio": (i32, [P, vp, vp, vp, vp, vp, vp, sz, vp]),
+    }
+    for name, (res, args) in sig.items():
+        f = getattr(lib, name)
+        f.restype = res
+        f.argtypes = args
+    return lib
+
+
+lib = _load()
+LIB_PATH = _LIB_PATH
+EXPORTED = ("ssa_status_string", "ssa_version", "ssa_launch_count", "ssa_device_error",
+            "ssa_block_summary", "ssa_route_workspace_size", "ssa_route_topk", "ssa_sparse_attn",
+            "ssa_workspace_size", "ssa_forward", "ssa_hostio_buffer_size", "ssa_forward_hostio")
+
+
+def status_string(s: int) -> str:
+    return lib.ssa_status_string(int(s)).decode()
+
+
+def make_params(batch, n_q, n_kv, h_q, h_kv, d, block, topk, window, q_offset=0, beta=2.0,
+                scale=None, dtype="bf16", sigma="diag", route_impl=SSA_ROUTE_AUTO) -> ssa_params:
+    """An ssa_params struct from plain values (dtype 'f32'|'bf16', sigma 'diag'|'full')."""
+    return ssa_params(batch=batch, n_q=n_q, n_kv=n_kv, h_q=h_q, h_kv=h_kv, d=d, block=block, topk=topk,
+                      window=window, dtype={"f32": SSA_F32, "bf16": SSA_BF16}.get(dtype, dtype),
+                      sigma={"diag": SSA_SIGMA_DIAG, "full": SSA_SIGMA_FULL}.get(sigma, sigma),
+                      route_impl=route_impl, q_offset=q_offset, beta=beta,
+                      scale=(1.0 / math.sqrt(d)) if scale is None else scale)
+
+
+def _ptr(t):
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return t
+    return t.data_ptr()
+
+
+def _stream(stream):
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+def _check(status, what):
+    if status != SSA_OK:
+        raise SSAError(status, what)
+
+
+def ssa_launch_count() -> int:
+    return int(lib.ssa_launch_count())
+
+
+def ssa_device_error() -> int:
+    code = C.c_uint32(0)
+    st = lib.ssa_device_error(C.byref(code))
+    if st not in (SSA_OK, SSA_ERR_DEVICE):
+        raise SSAError(st, "ssa_device_error")
+    return int(code.value)
+
+
+def ssa_block_summary(p, K, mu=None, sigma=None, route_table=None, stream=None):
+    _check(lib.ssa_block_summary(C.byref(p), _ptr(K), _ptr(mu), _ptr(sigma), _ptr(route_table),
+                                 _stream(stream)), "ssa_block_summary")
+
+
+def ssa_route_workspace_size(p) -> int:
+    return int(lib.ssa_route_workspace_size(C.byref(p)))
+
+
+def ssa_route_topk(p, Q, mu, sigma, route_table, block_idx, top_scores=None, ws=None, stream=None):
+    nbytes = ws.numel() * ws.element_size() if ws is not None else 0
+    _check(lib.ssa_route_topk(C.byref(p), _ptr(Q), _ptr(mu), _ptr(sigma), _ptr(route_table),
+                              _ptr(block_idx), _ptr(top_scores), _ptr(ws), nbytes, _stream(stream)),
+           "ssa_route_topk")
+
+
+def ssa_sparse_attn(p, Q, K, V, block_idx, O, lse=None, bad_index_count=None, stream=None):
+    _check(lib.ssa_sparse_attn(C.byref(p), _ptr(Q), _ptr(K), _ptr(V), _ptr(block_idx), _ptr(O),
+                               _ptr(lse), _ptr(bad_index_count), _stream(stream)), "ssa_sparse_attn")
+
+
+def ssa_workspace_size(p) -> int:
+    return int(lib.ssa_workspace_size(C.byref(p)))
+
+
+def ssa_forward(p, Q, K, V, O, lse=None, ws=None, stream=None):
+    nbytes = ws.numel() * ws.element_size() if ws is not None else 0
+    _check(lib.ssa_forward(C.byref(p), _ptr(Q), _ptr(K), _ptr(V), _ptr(O), _ptr(lse), _ptr(ws), nbytes,
+                           _stream(stream)), "ssa_forward")
+
+
+def ssa_hostio_buffer_size(p) -> int:
+    return int(lib.ssa_hostio_buffer_size(C.byref(p)))
+
+
+def ssa_forward_hostio(p, hQ, hK, hV, hO, hlse=None, dev_buf=None, stream=None):
+    nbytes = dev_buf.numel() * dev_buf.element_size() if dev_buf is not None else 0
+    _check(lib.ssa_forward_hostio(C.byref(p), _ptr(hQ), _ptr(hK), _ptr(hV), _ptr(hO), _ptr(hlse),
+                                  _ptr(dev_buf), nbytes, _stream(stream)), "ssa_forward_hostio")
+
+
+# ---------------------------------------------------------------- buffers
+
+def summary_shapes(p):
+    nb = p.n_kv // p.block
+    mu = (p.batch, p.h_kv, nb, p.d)
+    sig = mu + ((p.d,) if p.sigma == SSA_SIGMA_FULL else ())
+    tab = (p.batch, p.h_kv, nb, 2 * p.d)
+    return mu, sig, tab
+
+
+def idx_shape(p):
+    return (p.batch, p.n_q, p.h_kv, p.topk)
+
+
+def byte_buffer(nbytes: int, device="cuda"):
+    """A caller-owned uint8 buffer (workspaces are allocated by the caller)."""
+    return torch.empty(max(int(nbytes), 16), dtype=torch.uint8, device=device)

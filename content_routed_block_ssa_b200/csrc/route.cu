@@ -1,0 +1,708 @@
+// Step (i) of the layer: route every query row to its top-k key blocks.
+//
+// Score of fully visible block c for the query heads h of kv-head g:
+//   s_c = sum_h r_c(q_h),  r_c(q) = <q, mu_c> + (beta/2) q^T Sigma_c q
+// ["Subquadratic Sparse Attention (SSA)", "The idea in one screen",
+// routing-score equation], with a fixed budget of k blocks per row
+// ["fixed budget kappa << n", opening section].  Ties go to the lower block
+// index.
+//
+// For bf16 problems with a diagonal Sigma the score is the dot product of
+// the feature row f = [sum_h q_h ; (beta/2) sum_h q_h*q_h] with the table
+// row [mu_c ; sigma_c^2], so routing a tile of query rows is a dense
+// contraction (rows x 2d) . (2d x blocks).  The tiled router runs it on the
+// tcgen05 tensor cores with TMEM accumulators and selects the top-k in the
+// epilogue while the next chunk is being multiplied: scores never leave the
+// SM.
+#include <cuda_bf16.h>
+#include <math.h>
+
+#include "common.cuh"
+#include "kernels.h"
+
+namespace ssa {
+namespace {
+
+// ------------------------------------------------------------------ features
+
+// F[b, g, i, :] = [bf16(qs), bf16(hb * qq)], qs / qq accumulated in float32
+// in head order.  Thread = (row, 8 consecutive dimensions).
+template <int D, int G>
+__global__ void __launch_bounds__(256) features_kernel(const __nv_bfloat16* __restrict__ Q,
+                                                       __nv_bfloat16* __restrict__ F,
+                                                       int64_t rows, int n_q, int h_kv,
+                                                       float half_beta) {
+  constexpr int CG = D / 8;
+  constexpr int RPC = 256 / CG;
+  const int64_t row = static_cast<int64_t>(blockIdx.x) * RPC + threadIdx.x / CG;
+  const int cg = threadIdx.x % CG;
+  if (row >= rows) return;
+  const int i = static_cast<int>(row % n_q);
+  const int64_t bg = row / n_q;
+  const int g = static_cast<int>(bg % h_kv);
+  const int64_t b = bg / h_kv;
+  const int h_q = h_kv * G;
+  const __nv_bfloat16* q = Q + ((b * n_q + i) * h_q + static_cast<int64_t>(g) * G) * D + cg * 8;
+  float qs[8], qq[8];
+#pragma unroll
+  for (int v = 0; v < 8; ++v) { qs[v] = 0.f; qq[v] = 0.f; }
+#pragma unroll
+  for (int h = 0; h < G; ++h) {
+    const uint4 raw = __ldg(reinterpret_cast<const uint4*>(q + h * D));
+    const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const float lo = __uint_as_float(w[j] << 16), hi = __uint_as_float(w[j] & 0xFFFF0000u);
+      qs[2 * j] = __fadd_rn(qs[2 * j], lo);
+      qs[2 * j + 1] = __fadd_rn(qs[2 * j + 1], hi);
+      qq[2 * j] = __fmaf_rn(lo, lo, qq[2 * j]);         // lo*lo is exact in float32
+      qq[2 * j + 1] = __fmaf_rn(hi, hi, qq[2 * j + 1]);
+    }
+  }
+  uint4 o1, o2;
+  uint32_t* p1 = reinterpret_cast<uint32_t*>(&o1);
+  uint32_t* p2 = reinterpret_cast<uint32_t*>(&o2);
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    p1[j] = pack_bf16(qs[2 * j], qs[2 * j + 1]);
+    p2[j] = pack_bf16(__fmul_rn(half_beta, qq[2 * j]), __fmul_rn(half_beta, qq[2 * j + 1]));
+  }
+  __nv_bfloat16* f = F + row * (2 * D) + cg * 8;
+  *reinterpret_cast<uint4*>(f) = o1;
+  *reinterpret_cast<uint4*>(f + D) = o2;
+}
+
+// ------------------------------------------------------------------ tiled router
+
+struct RouteTiledArgs {
+  int32_t batch, n_q, h_kv, nb, block, topk;
+  int32_t n_tiles, n_units;
+  int64_t q_offset;
+  int32_t* block_idx;
+  float* top_scores;
+  uint32_t* err;
+};
+
+template <int KF>
+struct TiledCfg {
+  static constexpr int A_BOXES = KF / 64;                 // 64-wide K slices
+  static constexpr int BOX_BYTES = 128 * 128;             // 128 rows x 64 bf16
+  static constexpr int A_BYTES = A_BOXES * BOX_BYTES;     // one 128-row feature tile
+  static constexpr int NS = (KF == 256) ? 4 : 6;          // table-slice ring
+  static constexpr int CAP = 32;                          // candidates per row
+  static constexpr int NACC = 4;                          // TMEM accumulators (128 cols)
+  static constexpr int NBAR = 4 + 2 * NS + 2 * NACC + 1;
+  static constexpr int SMEM = 1024 + 2 * A_BYTES + NS * BOX_BYTES + CAP * 128 * 8 + NBAR * 8 + 16;
+};
+
+__device__ __forceinline__ void route_unit(const RouteTiledArgs& a, int r, int& bg, int& row0,
+                                           int& nch) {
+  const int BG = a.batch * a.h_kv;
+  bg = r % BG;
+  const int tile = a.n_tiles - 1 - r / BG;   // heaviest tiles first
+  row0 = tile * 128;
+  const int rows = min(128, a.n_q - row0);
+  const int64_t pos = a.q_offset + row0 + rows - 1;
+  const int nv = static_cast<int>(min(static_cast<int64_t>(a.nb), (pos + 1) / a.block));
+  nch = (nv + 127) / 128;
+}
+
+// Snake order over rounds keeps every CTA's total work close to the mean.
+__device__ __forceinline__ int route_unit_rank(int q) {
+  return q * gridDim.x + ((q & 1) ? (gridDim.x - 1 - blockIdx.x) : blockIdx.x);
+}
+
+// Bounded wait on a phase that must already be in flight (teardown drain).
+__device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity, uint32_t* err) {
+  const uint64_t t0 = global_timer_ns();
+  while (!mbar_try_wait(bar, parity)) {
+    if (global_timer_ns() - t0 > kWaitLimitNs) {
+      atomicCAS(err, 0u, SITE_DRAIN);
+      return;
+    }
+  }
+}
+
+template <int KSEL>
+__device__ __forceinline__ void compact(uint64_t (&L)[KSEL], int& cnt, float& thr,
+                                        const uint2* my_cand, int k) {
+  uint64_t Bk[32];
+#pragma unroll
+  for (int t = 0; t < 32; ++t) {
+    uint64_t key = 0;
+    if (t < cnt) {
+      const uint2 e = my_cand[t * 128];
+      key = make_key(e.x, e.y);
+    }
+    Bk[t] = key;
+  }
+  bitonic_sort_desc<32>(Bk);
+#pragma unroll
+  for (int j = 0; j < KSEL; ++j) {
+    const uint64_t y = Bk[KSEL - 1 - j];
+    L[j] = L[j] < y ? y : L[j];
+  }
+  bitonic_merge_desc<KSEL>(L);
+  cnt = 0;
+  uint64_t kth = 0;
+#pragma unroll
+  for (int j = 0; j < KSEL; ++j)
+    if (j == k - 1) kth = L[j];
+  thr = kth ? key_score(kth) : -INFINITY;
+}
+
+template <bool MASK>
+__device__ __forceinline__ void filter16(const uint32_t (&v)[16], int c0, int nvis, float thr,
+                                         int& cnt, uint2* my_cand) {
+#pragma unroll
+  for (int t = 0; t < 16; ++t) {
+    const float s = __uint_as_float(v[t]);
+    bool take = s >= thr;
+    if (MASK) take = take && (c0 + t < nvis);
+    if (take) {
+      my_cand[cnt * 128] = make_uint2(v[t], static_cast<uint32_t>(c0 + t));
+      ++cnt;
+    }
+  }
+}
+
+// Warp roles: 0 = TMA producer, 1 = MMA issuer (and TMEM owner),
+// 2..5 = epilogue (TMEM lane quadrant = warp % 4, one query row per thread).
+template <int KF, int KSEL>
+__global__ void __launch_bounds__(192, 1)
+    route_tiled_kernel(const __grid_constant__ CUtensorMap tmF, const __grid_constant__ CUtensorMap tmT,
+                       const RouteTiledArgs a) {
+  using C = TiledCfg<KF>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sA = smem;
+  uint8_t* sB = sA + 2 * C::A_BYTES;
+  uint2* cand = reinterpret_cast<uint2*>(sB + C::NS * C::BOX_BYTES);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(cand + C::CAP * 128);
+  uint64_t* a_full = bars;
+  uint64_t* a_empty = bars + 2;
+  uint64_t* b_full = bars + 4;
+  uint64_t* b_empty = b_full + C::NS;
+  uint64_t* acc_full = b_empty + C::NS;
+  uint64_t* acc_empty = acc_full + C::NACC;
+  uint64_t* mma_done = acc_empty + C::NACC;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
+
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < 2; ++i) { mbar_init(&a_full[i], 1); mbar_init(&a_empty[i], 1); }
+    for (int i = 0; i < C::NS; ++i) { mbar_init(&b_full[i], 1); mbar_init(&b_empty[i], 1); }
+    for (int i = 0; i < C::NACC; ++i) { mbar_init(&acc_full[i], 1); mbar_init(&acc_empty[i], 4); }
+    mbar_init(mma_done, 1);
+    fence_barrier_init();
+    tma_prefetch_desc(&tmF);
+    tma_prefetch_desc(&tmT);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      uint32_t a_cnt = 0, b_cnt = 0;
+      bool ok = true;
+      for (int q = 0; ok; ++q) {
+        const int r = route_unit_rank(q);
+        if (r >= a.n_units) break;
+        int bg, row0, nch;
+        route_unit(a, r, bg, row0, nch);
+        if (nch == 0) continue;
+        const int ab = a_cnt & 1;
+        if (!mbar_wait(&a_empty[ab], ((a_cnt >> 1) & 1) ^ 1, a.err, SITE_ROUTE_PRODUCER)) { ok = false; break; }
+        mbar_arrive_expect_tx(&a_full[ab], C::A_BYTES);
+        const int frow = bg * a.n_q + row0;
+#pragma unroll
+        for (int ks = 0; ks < C::A_BOXES; ++ks)
+          tma_load_2d(sA + ab * C::A_BYTES + ks * C::BOX_BYTES, &tmF, &a_full[ab], ks * 64, frow);
+        ++a_cnt;
+        const int trow = bg * a.nb;
+        for (int j = 0; j < nch && ok; ++j) {
+#pragma unroll
+          for (int ks = 0; ks < C::A_BOXES; ++ks) {
+            const int s = b_cnt % C::NS;
+            if (!mbar_wait(&b_empty[s], ((b_cnt / C::NS) & 1) ^ 1, a.err, SITE_ROUTE_PRODUCER)) { ok = false; break; }
+            mbar_arrive_expect_tx(&b_full[s], C::BOX_BYTES);
+            tma_load_2d(sB + s * C::BOX_BYTES, &tmT, &b_full[s], ks * 64, trow + j * 128);
+            ++b_cnt;
+          }
+        }
+      }
+      if (!ok) {   // make sure no copy is still landing in shared memory
+        for (uint32_t n = (b_cnt > C::NS ? b_cnt - C::NS : 0); n < b_cnt; ++n)
+          drain_wait(&b_full[n % C::NS], (n / C::NS) & 1, a.err);
+        for (uint32_t n = (a_cnt > 2 ? a_cnt - 2 : 0); n < a_cnt; ++n)
+          drain_wait(&a_full[n & 1], (n >> 1) & 1, a.err);
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      constexpr uint32_t IDESC = umma_idesc_bf16(128, 128);
+      uint32_t a_cnt = 0, b_cnt = 0, acc_cnt = 0;
+      bool ok = true;
+      const uint32_t sA_u = smem_u32(sA), sB_u = smem_u32(sB);
+      for (int q = 0; ok; ++q) {
+        const int r = route_unit_rank(q);
+        if (r >= a.n_units) break;
+        int bg, row0, nch;
+        route_unit(a, r, bg, row0, nch);
+        if (nch == 0) continue;
+        const int ab = a_cnt & 1;
+        if (!mbar_wait(&a_full[ab], (a_cnt >> 1) & 1, a.err, SITE_ROUTE_MMA)) { ok = false; break; }
+        tc_fence_after();
+        for (int j = 0; j < nch && ok; ++j) {
+          const int acc = acc_cnt % C::NACC;
+          if (!mbar_wait(&acc_empty[acc], ((acc_cnt / C::NACC) & 1) ^ 1, a.err, SITE_ROUTE_MMA)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t d_tmem = tmem_base + acc * 128;
+#pragma unroll
+          for (int ks = 0; ks < C::A_BOXES; ++ks) {
+            const int s = b_cnt % C::NS;
+            if (!mbar_wait(&b_full[s], (b_cnt / C::NS) & 1, a.err, SITE_ROUTE_MMA)) { ok = false; break; }
+            tc_fence_after();
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk) {
+              const uint64_t ad = umma_desc_sw128(sA_u + ab * C::A_BYTES + ks * C::BOX_BYTES + kk * 32);
+              const uint64_t bd = umma_desc_sw128(sB_u + s * C::BOX_BYTES + kk * 32);
+              umma_bf16(d_tmem, ad, bd, IDESC, (ks | kk) != 0 ? 1u : 0u);
+            }
+            umma_commit(&b_empty[s]);
+            ++b_cnt;
+          }
+          if (!ok) break;
+          umma_commit(&acc_full[acc]);
+          ++acc_cnt;
+        }
+        if (!ok) break;
+        umma_commit(&a_empty[ab]);
+        ++a_cnt;
+      }
+      umma_commit(mma_done);        // all issued MMAs complete before TMEM is freed
+      drain_wait(mma_done, 0, a.err);
+    }
+  } else {
+    const int eq = warp & 3;
+    const int row = eq * 32 + lane;
+    uint2* my_cand = cand + row;
+    uint32_t acc_cnt = 0;
+    bool ok = true;
+    for (int q = 0; ok; ++q) {
+      const int r = route_unit_rank(q);
+      if (r >= a.n_units) break;
+      int bg, row0, nch;
+      route_unit(a, r, bg, row0, nch);
+      const int i = row0 + row;
+      const bool valid = i < a.n_q;
+      const int nvis = valid ? static_cast<int>(min(static_cast<int64_t>(a.nb), (a.q_offset + i + 1) / a.block)) : 0;
+      uint64_t L[KSEL];
+#pragma unroll
+      for (int j = 0; j < KSEL; ++j) L[j] = 0;
+      float thr = -INFINITY;
+      int cnt = 0;
+      for (int j = 0; j < nch; ++j) {
+        const int acc = acc_cnt % C::NACC;
+        ok = __all_sync(0xFFFFFFFFu, mbar_wait(&acc_full[acc], (acc_cnt / C::NACC) & 1, a.err, SITE_ROUTE_EPILOGUE));
+        if (!ok) break;
+        tc_fence_after();
+        const uint32_t taddr = tmem_base + (static_cast<uint32_t>(eq * 32) << 16) + acc * 128;
+#pragma unroll 1
+        for (int sub = 0; sub < 8; ++sub) {
+          uint32_t v[16];
+          tmem_ld16(taddr + sub * 16, v);
+          tmem_wait_ld();
+          if (sub == 7) {
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&acc_empty[acc]);
+          }
+          const int c0 = j * 128 + sub * 16;
+          if (__all_sync(0xFFFFFFFFu, c0 + 16 <= nvis))
+            filter16<false>(v, c0, nvis, thr, cnt, my_cand);
+          else
+            filter16<true>(v, c0, nvis, thr, cnt, my_cand);
+          if (__any_sync(0xFFFFFFFFu, cnt > C::CAP - 16)) compact<KSEL>(L, cnt, thr, my_cand, a.topk);
+        }
+        ++acc_cnt;
+      }
+      if (!ok) break;
+      if (__any_sync(0xFFFFFFFFu, cnt > 0)) compact<KSEL>(L, cnt, thr, my_cand, a.topk);
+      if (valid) {
+        uint32_t ob[KSEL];
+        float os[KSEL];
+#pragma unroll
+        for (int j = 0; j < KSEL; ++j) {
+          const bool use = (j < a.topk) && L[j] != 0;
+          ob[j] = use ? key_block(L[j]) : 0xFFFFFFFFu;
+          os[j] = use ? key_score(L[j]) : -INFINITY;
+        }
+        bitonic_sort_asc_u32<KSEL>(ob, os);
+        const int b = bg / a.h_kv, g = bg % a.h_kv;
+        const int64_t o = ((static_cast<int64_t>(b) * a.n_q + i) * a.h_kv + g) * a.topk;
+#pragma unroll
+        for (int j = 0; j < KSEL; ++j) {
+          if (j < a.topk) {
+            a.block_idx[o + j] = ob[j] == 0xFFFFFFFFu ? -1 : static_cast<int32_t>(ob[j]);
+            if (a.top_scores) a.top_scores[o + j] = os[j];
+          }
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem_base, 512);
+  }
+}
+
+template <int KF, int KSEL>
+cudaError_t run_tiled(const ssa_params& p, const CUtensorMap& tmF, const CUtensorMap& tmT,
+                      int32_t* idx, float* scores, const LaunchCtx& c) {
+  using C = TiledCfg<KF>;
+  RouteTiledArgs a;
+  a.batch = p.batch; a.n_q = p.n_q; a.h_kv = p.h_kv; a.nb = p.n_kv / p.block;
+  a.block = p.block; a.topk = p.topk;
+  a.n_tiles = (p.n_q + 127) / 128;
+  a.n_units = p.batch * p.h_kv * a.n_tiles;
+  a.q_offset = p.q_offset;
+  a.block_idx = idx; a.top_scores = scores; a.err = c.err;
+  cudaError_t e = cudaFuncSetAttribute(route_tiled_kernel<KF, KSEL>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+  if (e != cudaSuccess) return e;
+  const int grid = a.n_units < c.sm_count ? a.n_units : c.sm_count;
+  route_tiled_kernel<KF, KSEL><<<grid, 192, C::SMEM, c.stream>>>(tmF, tmT, a);
+  note_launch();
+  return cudaGetLastError();
+}
+
+// ------------------------------------------------------------------ row-wise routers
+
+struct RowArgs {
+  int32_t n_q, h_kv, nb, block, topk;
+  int64_t q_offset;
+  float half_beta;
+  int32_t* block_idx;
+  float* top_scores;
+};
+
+__device__ __forceinline__ int next_pow2(int x) {
+  int p = 1;
+  while (p < x) p <<= 1;
+  return p;
+}
+
+// Sorts keys[0..n2) descending in shared memory (n2 a power of two) and
+// writes the top-k blocks of the row in ascending block order.
+__device__ void select_and_write(uint64_t* keys, int nvis, int n2, const RowArgs& a, int64_t out) {
+  for (int c = nvis + threadIdx.x; c < n2; c += blockDim.x) keys[c] = 0;
+  __syncthreads();
+  for (int size = 2; size <= n2; size <<= 1) {
+    for (int stride = size >> 1; stride > 0; stride >>= 1) {
+      for (int t = threadIdx.x; t < n2 / 2; t += blockDim.x) {
+        const int i = 2 * t - (t & (stride - 1));   // lower index of the pair
+        const int j = i + stride;
+        const bool desc = (i & size) == 0;
+        const uint64_t x = keys[i], y = keys[j];
+        if (desc ? (x < y) : (x > y)) { keys[i] = y; keys[j] = x; }
+      }
+      __syncthreads();
+    }
+  }
+  if (threadIdx.x < 32) {
+    const int lane = threadIdx.x;
+    const uint64_t key = (lane < a.topk && lane < n2) ? keys[lane] : 0;
+    const uint32_t blk = key ? key_block(key) : 0xFFFFFFFFu;
+    int rank = 0;
+    for (int o = 0; o < 32; ++o) {
+      const uint32_t other = __shfl_sync(0xFFFFFFFFu, blk, o);
+      rank += (other < blk) ? 1 : 0;
+    }
+    if (lane < a.topk) {
+      a.block_idx[out + rank] = key ? static_cast<int32_t>(blk) : -1;
+      if (a.top_scores) a.top_scores[out + rank] = key ? key_score(key) : -INFINITY;
+    }
+  }
+}
+
+// bf16 table, one CTA per (query row, kv-head, batch).  Lane l of every warp
+// holds features [FPL*l, FPL*l + FPL) of the row and dots them with the
+// matching slice of a table row; a warp reduction gives the block score.
+template <int D, int G>
+__global__ void __launch_bounds__(256) route_rowwise_bf16_kernel(const __nv_bfloat16* __restrict__ Q,
+                                                                 const __nv_bfloat16* __restrict__ T,
+                                                                 const RowArgs a) {
+  constexpr int FPL = 2 * D / 32;   // features per lane: 8 (d=128) or 4 (d=64)
+  extern __shared__ uint64_t keys[];
+  const int i = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
+  const int lane = threadIdx.x % 32, warp = threadIdx.x / 32;
+  const int64_t pos = a.q_offset + i;
+  const int nvis = static_cast<int>(min(static_cast<int64_t>(a.nb), (pos + 1) / a.block));
+  const int h_q = a.h_kv * G;
+  const bool second = lane >= 16;
+  const int dim0 = (lane % 16) * FPL;
+  float f[FPL];
+  {
+    float qs[FPL], qq[FPL];
+#pragma unroll
+    for (int v = 0; v < FPL; ++v) { qs[v] = 0.f; qq[v] = 0.f; }
+    const __nv_bfloat16* q = Q + ((static_cast<int64_t>(b) * a.n_q + i) * h_q + static_cast<int64_t>(g) * G) * D + dim0;
+#pragma unroll
+    for (int h = 0; h < G; ++h) {
+#pragma unroll
+      for (int v = 0; v < FPL; ++v) {
+        const float x = __bfloat162float(q[h * D + v]);
+        qs[v] = __fadd_rn(qs[v], x);
+        qq[v] = __fmaf_rn(x, x, qq[v]);
+      }
+    }
+#pragma unroll
+    for (int v = 0; v < FPL; ++v) {
+      const float raw = second ? __fmul_rn(a.half_beta, qq[v]) : qs[v];
+      f[v] = __bfloat162float(__float2bfloat16_rn(raw));
+    }
+  }
+  const __nv_bfloat16* trow = T + (static_cast<int64_t>(b) * a.h_kv + g) * a.nb * (2 * D) + lane * FPL;
+  for (int c0 = warp * 4; c0 < nvis; c0 += 32) {
+    float part[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int c = c0 + u;
+      part[u] = 0.f;
+      if (c < nvis) {
+        const __nv_bfloat16* t = trow + static_cast<int64_t>(c) * (2 * D);
+        float tv[FPL];
+        if (FPL == 8) {
+          const uint4 raw = __ldg(reinterpret_cast<const uint4*>(t));
+          const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            tv[2 * j] = __uint_as_float(w[j] << 16);
+            tv[2 * j + 1] = __uint_as_float(w[j] & 0xFFFF0000u);
+          }
+        } else {
+          const uint2 raw = __ldg(reinterpret_cast<const uint2*>(t));
+          const uint32_t w[2] = {raw.x, raw.y};
+#pragma unroll
+          for (int j = 0; j < 2; ++j) {
+            tv[2 * j] = __uint_as_float(w[j] << 16);
+            tv[2 * j + 1] = __uint_as_float(w[j] & 0xFFFF0000u);
+          }
+        }
+#pragma unroll
+        for (int v = 0; v < FPL; ++v) part[u] = __fmaf_rn(f[v], tv[v], part[u]);
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) part[u] += __shfl_xor_sync(0xFFFFFFFFu, part[u], o);
+      const int c = c0 + u;
+      if (lane == 0 && c < nvis) keys[c] = make_key(__float_as_uint(part[u]), c);
+    }
+  }
+  const int n2 = next_pow2(max(nvis, 1));
+  const int64_t out = ((static_cast<int64_t>(b) * a.n_q + i) * a.h_kv + g) * a.topk;
+  select_and_write(keys, nvis, n2, a, out);
+}
+
+// float32 summaries: s_c = sum_h (<q_h, mu_c> + (beta/2) q_h^T Sigma_c q_h).
+// One warp per block; lane l owns rows s = l, l+32, ... of Sigma_c (full)
+// or dimensions l, l+32, ... (diagonal).
+template <int D, int G, bool FULL>
+__global__ void __launch_bounds__(256) route_rowwise_f32_kernel(const float* __restrict__ Q,
+                                                                const float* __restrict__ MU,
+                                                                const float* __restrict__ SG,
+                                                                const RowArgs a) {
+  extern __shared__ uint64_t keys[];
+  __shared__ float qsm[G][D];
+  const int i = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
+  const int lane = threadIdx.x % 32, warp = threadIdx.x / 32;
+  const int64_t pos = a.q_offset + i;
+  const int nvis = static_cast<int>(min(static_cast<int64_t>(a.nb), (pos + 1) / a.block));
+  const int h_q = a.h_kv * G;
+  const float* q = Q + ((static_cast<int64_t>(b) * a.n_q + i) * h_q + static_cast<int64_t>(g) * G) * D;
+  for (int e = threadIdx.x; e < G * D; e += blockDim.x) qsm[e / D][e % D] = q[e];
+  __syncthreads();
+  const int64_t bgrow = (static_cast<int64_t>(b) * a.h_kv + g) * a.nb;
+  for (int c = warp; c < nvis; c += 8) {
+    const float* mu = MU + (bgrow + c) * D;
+    float acc = 0.f;
+#pragma unroll
+    for (int h = 0; h < G; ++h) {
+      float lin = 0.f, quad = 0.f;
+#pragma unroll
+      for (int ss = 0; ss < D / 32; ++ss) {
+        const int s = lane + 32 * ss;
+        const float qv = qsm[h][s];
+        lin = __fmaf_rn(qv, __ldg(mu + s), lin);
+        if (FULL) {
+          const float* srow = SG + ((bgrow + c) * D + s) * D;
+          float u = 0.f;
+#pragma unroll 8
+          for (int t = 0; t < D; ++t) u = __fmaf_rn(__ldg(srow + t), qsm[h][t], u);
+          quad = __fmaf_rn(qv, u, quad);
+        } else {
+          quad = __fmaf_rn(qv * qv, __ldg(SG + (bgrow + c) * D + s), quad);
+        }
+      }
+      acc += lin + a.half_beta * quad;
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xFFFFFFFFu, acc, o);
+    if (lane == 0) keys[c] = make_key(__float_as_uint(acc), c);
+  }
+  const int n2 = next_pow2(max(nvis, 1));
+  const int64_t out = ((static_cast<int64_t>(b) * a.n_q + i) * a.h_kv + g) * a.topk;
+  __syncthreads();
+  select_and_write(keys, nvis, n2, a, out);
+}
+
+RowArgs row_args(const ssa_params& p, int32_t* idx, float* scores) {
+  RowArgs a;
+  a.n_q = p.n_q; a.h_kv = p.h_kv; a.nb = p.n_kv / p.block; a.block = p.block; a.topk = p.topk;
+  a.q_offset = p.q_offset;
+  a.half_beta = p.beta * 0.5f;   // exact
+  a.block_idx = idx; a.top_scores = scores;
+  return a;
+}
+
+template <int D, int G>
+cudaError_t run_features(const ssa_params& p, const void* Q, void* F, const LaunchCtx& c) {
+  constexpr int RPC = 256 / (D / 8);
+  const int64_t rows = static_cast<int64_t>(p.batch) * p.h_kv * p.n_q;
+  const int64_t grid = (rows + RPC - 1) / RPC;
+  features_kernel<D, G><<<static_cast<unsigned>(grid), 256, 0, c.stream>>>(
+      static_cast<const __nv_bfloat16*>(Q), static_cast<__nv_bfloat16*>(F), rows, p.n_q, p.h_kv,
+      p.beta * 0.5f);
+  note_launch();
+  return cudaGetLastError();
+}
+
+template <int D>
+cudaError_t features_g(const ssa_params& p, const void* Q, void* F, const LaunchCtx& c) {
+  switch (p.h_q / p.h_kv) {
+    case 1: return run_features<D, 1>(p, Q, F, c);
+    case 2: return run_features<D, 2>(p, Q, F, c);
+    case 4: return run_features<D, 4>(p, Q, F, c);
+    case 8: return run_features<D, 8>(p, Q, F, c);
+  }
+  return cudaErrorInvalidValue;
+}
+
+int row_smem_bytes(const ssa_params& p) {
+  int n2 = 1;
+  while (n2 < p.n_kv / p.block) n2 <<= 1;
+  return n2 * 8;
+}
+
+template <int D, int G>
+cudaError_t run_rowwise_bf16(const ssa_params& p, const void* Q, const void* T, int32_t* idx,
+                             float* scores, const LaunchCtx& c) {
+  const int smem = row_smem_bytes(p);
+  cudaError_t e = cudaFuncSetAttribute(route_rowwise_bf16_kernel<D, G>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  dim3 grid(p.n_q, p.h_kv, p.batch);
+  route_rowwise_bf16_kernel<D, G><<<grid, 256, smem, c.stream>>>(
+      static_cast<const __nv_bfloat16*>(Q), static_cast<const __nv_bfloat16*>(T), row_args(p, idx, scores));
+  note_launch();
+  return cudaGetLastError();
+}
+
+template <int D>
+cudaError_t rowwise_bf16_g(const ssa_params& p, const void* Q, const void* T, int32_t* idx,
+                           float* scores, const LaunchCtx& c) {
+  switch (p.h_q / p.h_kv) {
+    case 1: return run_rowwise_bf16<D, 1>(p, Q, T, idx, scores, c);
+    case 2: return run_rowwise_bf16<D, 2>(p, Q, T, idx, scores, c);
+    case 4: return run_rowwise_bf16<D, 4>(p, Q, T, idx, scores, c);
+    case 8: return run_rowwise_bf16<D, 8>(p, Q, T, idx, scores, c);
+  }
+  return cudaErrorInvalidValue;
+}
+
+template <int D, int G, bool FULL>
+cudaError_t run_rowwise_f32(const ssa_params& p, const void* Q, const float* mu, const float* sg,
+                            int32_t* idx, float* scores, const LaunchCtx& c) {
+  const int smem = row_smem_bytes(p);
+  cudaError_t e = cudaFuncSetAttribute(route_rowwise_f32_kernel<D, G, FULL>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  dim3 grid(p.n_q, p.h_kv, p.batch);
+  route_rowwise_f32_kernel<D, G, FULL><<<grid, 256, smem, c.stream>>>(
+      static_cast<const float*>(Q), mu, sg, row_args(p, idx, scores));
+  note_launch();
+  return cudaGetLastError();
+}
+
+template <int D, bool FULL>
+cudaError_t rowwise_f32_g(const ssa_params& p, const void* Q, const float* mu, const float* sg,
+                          int32_t* idx, float* scores, const LaunchCtx& c) {
+  switch (p.h_q / p.h_kv) {
+    case 1: return run_rowwise_f32<D, 1, FULL>(p, Q, mu, sg, idx, scores, c);
+    case 2: return run_rowwise_f32<D, 2, FULL>(p, Q, mu, sg, idx, scores, c);
+    case 4: return run_rowwise_f32<D, 4, FULL>(p, Q, mu, sg, idx, scores, c);
+    case 8: return run_rowwise_f32<D, 8, FULL>(p, Q, mu, sg, idx, scores, c);
+  }
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace
+
+int route_tiled_smem_bytes(int d, int /*topk*/) {
+  return d == 128 ? TiledCfg<256>::SMEM : TiledCfg<128>::SMEM;
+}
+
+cudaError_t launch_features(const ssa_params& p, const void* Q, void* F, const LaunchCtx& c) {
+  if (p.d == 128) return features_g<128>(p, Q, F, c);
+  if (p.d == 64) return features_g<64>(p, Q, F, c);
+  return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_route_tiled(const ssa_params& p, const CUtensorMap& tmF, const CUtensorMap& tmT,
+                               int32_t* idx, float* scores, const LaunchCtx& c) {
+  const int ksel = p.topk <= 8 ? 8 : (p.topk <= 16 ? 16 : 32);
+  if (p.d == 128) {
+    if (ksel == 8) return run_tiled<256, 8>(p, tmF, tmT, idx, scores, c);
+    if (ksel == 16) return run_tiled<256, 16>(p, tmF, tmT, idx, scores, c);
+    return run_tiled<256, 32>(p, tmF, tmT, idx, scores, c);
+  }
+  if (p.d == 64) {
+    if (ksel == 8) return run_tiled<128, 8>(p, tmF, tmT, idx, scores, c);
+    if (ksel == 16) return run_tiled<128, 16>(p, tmF, tmT, idx, scores, c);
+    return run_tiled<128, 32>(p, tmF, tmT, idx, scores, c);
+  }
+  return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_route_rowwise_bf16(const ssa_params& p, const void* Q, const void* table,
+                                      int32_t* idx, float* scores, const LaunchCtx& c) {
+  if (p.d == 128) return rowwise_bf16_g<128>(p, Q, table, idx, scores, c);
+  if (p.d == 64) return rowwise_bf16_g<64>(p, Q, table, idx, scores, c);
+  return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_route_rowwise_f32(const ssa_params& p, const void* Q, const float* mu,
+                                     const float* sigma, int32_t* idx, float* scores,
+                                     const LaunchCtx& c) {
+  const bool full = p.sigma == SSA_SIGMA_FULL;
+  if (p.d == 128) return full ? rowwise_f32_g<128, true>(p, Q, mu, sigma, idx, scores, c)
+                              : rowwise_f32_g<128, false>(p, Q, mu, sigma, idx, scores, c);
+  if (p.d == 64) return full ? rowwise_f32_g<64, true>(p, Q, mu, sigma, idx, scores, c)
+                             : rowwise_f32_g<64, false>(p, Q, mu, sigma, idx, scores, c);
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace ssa

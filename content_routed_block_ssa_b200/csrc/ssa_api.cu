@@ -1,0 +1,400 @@
+// C ABI of libssa: argument validation, workspace carving, TMA descriptor
+// encoding and kernel dispatch.  See include/ssa.h for the contract.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <math.h>
+#include <stdint.h>
+#include <string.h>
+
+#include <atomic>
+#include <mutex>
+
+#include "kernels.h"
+#include "ssa.h"
+
+namespace ssa {
+
+static std::atomic<uint64_t> g_launches{0};
+void note_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
+
+}  // namespace ssa
+
+// Device failure word (one per device that loads the library).
+__device__ uint32_t g_ssa_device_error;
+
+namespace {
+
+using ssa::LaunchCtx;
+
+constexpr int kMaxDevices = 64;
+
+struct DeviceInfo {
+  bool ready = false;
+  int sm_count = 0;
+  uint32_t* err = nullptr;
+};
+
+std::mutex g_dev_mu;
+DeviceInfo g_dev[kMaxDevices];
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+ssa_status make_ctx(void* stream, LaunchCtx& c) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return SSA_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_dev_mu);
+  DeviceInfo& d = g_dev[dev];
+  if (!d.ready) {
+    if (cudaDeviceGetAttribute(&d.sm_count, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+      return SSA_ERR_CUDA;
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_ssa_device_error) != cudaSuccess) return SSA_ERR_CUDA;
+    d.err = static_cast<uint32_t*>(p);
+    d.ready = true;
+  }
+  c.stream = static_cast<cudaStream_t>(stream);
+  c.device = dev;
+  c.sm_count = d.sm_count;
+  c.err = d.err;
+  return SSA_OK;
+}
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+inline size_t round_up(size_t x) { return (x + 255) & ~size_t(255); }
+
+int64_t nb_of(const ssa_params& p) { return p.block > 0 ? p.n_kv / p.block : 0; }
+size_t esize(const ssa_params& p) { return p.dtype == SSA_BF16 ? 2 : 4; }
+
+bool is_empty(const ssa_params& p) { return p.batch == 0 || p.n_q == 0; }
+
+// Shape / support checks shared by every call.
+ssa_status check_params(const ssa_params* pp) {
+  if (!pp) return SSA_ERR_INVALID_ARG;
+  const ssa_params& p = *pp;
+  if (p.batch < 0 || p.n_q < 0 || p.n_kv < 0 || p.h_q < 1 || p.h_kv < 1 || p.d < 1 || p.block < 1 ||
+      p.topk < 1 || p.window < 1)
+    return SSA_ERR_INVALID_ARG;
+  if (p.h_q % p.h_kv != 0 || p.n_kv % p.block != 0) return SSA_ERR_INVALID_ARG;
+  if (p.q_offset < 0 || p.q_offset + p.n_q > p.n_kv) return SSA_ERR_INVALID_ARG;
+  if ((p.dtype != SSA_F32 && p.dtype != SSA_BF16) || (p.sigma != SSA_SIGMA_DIAG && p.sigma != SSA_SIGMA_FULL) ||
+      p.route_impl < SSA_ROUTE_AUTO || p.route_impl > SSA_ROUTE_ROWWISE)
+    return SSA_ERR_INVALID_ARG;
+  if (!isfinite(p.beta) || !isfinite(p.scale) || !(p.scale > 0.f)) return SSA_ERR_INVALID_ARG;
+  const int G = p.h_q / p.h_kv;
+  if (p.d != 64 && p.d != 128) return SSA_ERR_UNSUPPORTED;
+  if (p.block != 64 && p.block != 128) return SSA_ERR_UNSUPPORTED;
+  if (G != 1 && G != 2 && G != 4 && G != 8) return SSA_ERR_UNSUPPORTED;
+  if (p.topk > 32 || p.window > 4032) return SSA_ERR_UNSUPPORTED;
+  if (p.dtype == SSA_BF16 && p.sigma != SSA_SIGMA_DIAG) return SSA_ERR_UNSUPPORTED;
+  // index ranges used by the kernels and the TMA coordinates
+  const int64_t rows_kv = static_cast<int64_t>(p.batch) * p.n_kv;
+  const int64_t rows_q = static_cast<int64_t>(p.batch) * p.h_kv * p.n_q;
+  const int64_t rows_t = static_cast<int64_t>(p.batch) * p.h_kv * nb_of(p);
+  if (rows_kv > INT32_MAX || rows_q > INT32_MAX || rows_t > INT32_MAX) return SSA_ERR_UNSUPPORTED;
+  if (p.batch > 65535 || p.h_kv > 65535 || nb_of(p) > 2147483647) return SSA_ERR_UNSUPPORTED;
+  return SSA_OK;
+}
+
+bool use_tiled(const ssa_params& p) {
+  if (p.dtype != SSA_BF16) return false;
+  if (p.route_impl == SSA_ROUTE_TILED) return true;
+  if (p.route_impl == SSA_ROUTE_ROWWISE) return false;
+  return p.n_q >= 128;
+}
+
+bool rowwise_fits(const ssa_params& p) {
+  int64_t n2 = 1;
+  while (n2 < nb_of(p)) n2 <<= 1;
+  return n2 * 8 <= 200 * 1024 && p.n_q <= 2147483647 && p.h_kv <= 65535;
+}
+
+size_t features_bytes(const ssa_params& p) {
+  return use_tiled(p) ? round_up(static_cast<size_t>(p.batch) * p.h_kv * p.n_q * 2 * p.d * 2) : 0;
+}
+size_t table_bytes(const ssa_params& p) {
+  return p.dtype == SSA_BF16 ? round_up(static_cast<size_t>(p.batch) * p.h_kv * nb_of(p) * 2 * p.d * 2) : 0;
+}
+size_t mu_bytes(const ssa_params& p) {
+  return p.dtype == SSA_F32 ? round_up(static_cast<size_t>(p.batch) * p.h_kv * nb_of(p) * p.d * 4) : 0;
+}
+size_t sigma_bytes(const ssa_params& p) {
+  if (p.dtype != SSA_F32) return 0;
+  const size_t per = p.sigma == SSA_SIGMA_FULL ? static_cast<size_t>(p.d) * p.d : p.d;
+  return round_up(static_cast<size_t>(p.batch) * p.h_kv * nb_of(p) * per * 4);
+}
+size_t idx_bytes(const ssa_params& p) {
+  return round_up(static_cast<size_t>(p.batch) * p.n_q * p.h_kv * p.topk * 4);
+}
+
+ssa_status from_cuda(cudaError_t e) { return e == cudaSuccess ? SSA_OK : SSA_ERR_CUDA; }
+
+// 2D bf16 map of a [rows, cols] row-major matrix, 64 x box_rows boxes, 128B swizzle.
+bool encode_2d(CUtensorMap* m, const void* base, uint64_t cols, uint64_t rows, uint32_t box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[2] = {cols, rows};
+  const cuuint64_t strides[1] = {cols * 2};
+  const cuuint32_t box[2] = {64, box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// 3D bf16 map of K or V viewed as [b*n_kv, h_kv, d]; boxes of 64 keys x 1 head x 64 dims.
+bool encode_kv(CUtensorMap* m, const void* base, const ssa_params& p) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[3] = {static_cast<cuuint64_t>(p.d), static_cast<cuuint64_t>(p.h_kv),
+                              static_cast<cuuint64_t>(p.batch) * p.n_kv};
+  const cuuint64_t strides[2] = {static_cast<cuuint64_t>(p.d) * 2, static_cast<cuuint64_t>(p.h_kv) * p.d * 2};
+  const cuuint32_t box[3] = {64, 1, 64};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+ssa_status do_summary(const ssa_params& p, const void* K, float* mu, float* sigma, void* table,
+                      const LaunchCtx& c) {
+  if (p.batch == 0 || p.n_kv == 0) return SSA_OK;
+  if (!mu && !sigma && !table) return SSA_OK;
+  return from_cuda(ssa::launch_summary(p, K, mu, sigma, table, c));
+}
+
+ssa_status do_route(const ssa_params& p, const void* Q, const float* mu, const float* sigma,
+                    const void* table, int32_t* idx, float* scores, void* ws, size_t ws_bytes,
+                    const LaunchCtx& c) {
+  if (is_empty(p)) return SSA_OK;
+  if (p.dtype == SSA_F32) {
+    if (!rowwise_fits(p)) return SSA_ERR_UNSUPPORTED;
+    return from_cuda(ssa::launch_route_rowwise_f32(p, Q, mu, sigma, idx, scores, c));
+  }
+  if (!use_tiled(p)) {
+    if (!rowwise_fits(p)) return SSA_ERR_UNSUPPORTED;
+    return from_cuda(ssa::launch_route_rowwise_bf16(p, Q, table, idx, scores, c));
+  }
+  const size_t need = features_bytes(p);
+  if (ws_bytes < need || (need && !ws) || !aligned16(ws)) return SSA_ERR_WORKSPACE;
+  ssa_status st = from_cuda(ssa::launch_features(p, Q, ws, c));
+  if (st != SSA_OK) return st;
+  CUtensorMap tmF, tmT;
+  const uint64_t kf = 2 * static_cast<uint64_t>(p.d);
+  if (!encode_2d(&tmF, ws, kf, static_cast<uint64_t>(p.batch) * p.h_kv * p.n_q, 128) ||
+      !encode_2d(&tmT, table, kf, static_cast<uint64_t>(p.batch) * p.h_kv * nb_of(p), 128))
+    return SSA_ERR_CUDA;
+  return from_cuda(ssa::launch_route_tiled(p, tmF, tmT, idx, scores, c));
+}
+
+ssa_status do_attn(const ssa_params& p, const void* Q, const void* K, const void* V,
+                   const int32_t* idx, void* O, float* lse, int32_t* bad, const LaunchCtx& c) {
+  if (is_empty(p)) return SSA_OK;
+  if (p.dtype == SSA_F32) return from_cuda(ssa::launch_attn_f32(p, Q, K, V, idx, O, lse, bad, c));
+  CUtensorMap tmK, tmV;
+  if (!encode_kv(&tmK, K, p) || !encode_kv(&tmV, V, p)) return SSA_ERR_CUDA;
+  return from_cuda(ssa::launch_attn_bf16(p, tmK, tmV, Q, idx, O, lse, bad, c));
+}
+
+struct ForwardLayout {
+  size_t table, mu, sigma, feat, idx, total;
+};
+
+ForwardLayout forward_layout(const ssa_params& p) {
+  ForwardLayout L;
+  size_t off = 0;
+  L.table = off; off += table_bytes(p);
+  L.mu = off; off += mu_bytes(p);
+  L.sigma = off; off += sigma_bytes(p);
+  L.feat = off; off += features_bytes(p);
+  L.idx = off; off += idx_bytes(p);
+  L.total = off;
+  return L;
+}
+
+struct HostioLayout {
+  size_t q, k, v, o, lse, ws, total;
+};
+
+HostioLayout hostio_layout(const ssa_params& p) {
+  HostioLayout L;
+  const size_t es = esize(p);
+  size_t off = 0;
+  L.q = off; off += round_up(static_cast<size_t>(p.batch) * p.n_q * p.h_q * p.d * es);
+  L.k = off; off += round_up(static_cast<size_t>(p.batch) * p.n_kv * p.h_kv * p.d * es);
+  L.v = off; off += round_up(static_cast<size_t>(p.batch) * p.n_kv * p.h_kv * p.d * es);
+  L.o = off; off += round_up(static_cast<size_t>(p.batch) * p.n_q * p.h_q * p.d * es);
+  L.lse = off; off += round_up(static_cast<size_t>(p.batch) * p.n_q * p.h_q * 4);
+  L.ws = off; off += forward_layout(p).total;
+  L.total = off;
+  return L;
+}
+
+ssa_status forward_impl(const ssa_params& p, const void* Q, const void* K, const void* V, void* O,
+                        float* lse, uint8_t* ws, size_t ws_bytes, const LaunchCtx& c) {
+  const ForwardLayout L = forward_layout(p);
+  if (ws_bytes < L.total || (L.total && !ws) || !aligned16(ws)) return SSA_ERR_WORKSPACE;
+  void* table = table_bytes(p) ? ws + L.table : nullptr;
+  float* mu = mu_bytes(p) ? reinterpret_cast<float*>(ws + L.mu) : nullptr;
+  float* sg = sigma_bytes(p) ? reinterpret_cast<float*>(ws + L.sigma) : nullptr;
+  int32_t* idx = reinterpret_cast<int32_t*>(ws + L.idx);
+  ssa_status st = do_summary(p, K, mu, sg, table, c);
+  if (st != SSA_OK) return st;
+  st = do_route(p, Q, mu, sg, table, idx, nullptr, features_bytes(p) ? ws + L.feat : nullptr,
+                features_bytes(p), c);
+  if (st != SSA_OK) return st;
+  return do_attn(p, Q, K, V, idx, O, lse, nullptr, c);
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* ssa_status_string(int32_t s) {
+  switch (s) {
+    case SSA_OK: return "SSA_OK";
+    case SSA_ERR_INVALID_ARG: return "SSA_ERR_INVALID_ARG";
+    case SSA_ERR_UNSUPPORTED: return "SSA_ERR_UNSUPPORTED";
+    case SSA_ERR_WORKSPACE: return "SSA_ERR_WORKSPACE";
+    case SSA_ERR_CUDA: return "SSA_ERR_CUDA";
+    case SSA_ERR_DEVICE: return "SSA_ERR_DEVICE";
+  }
+  return "SSA_ERR_UNKNOWN";
+}
+
+int32_t ssa_version(void) { return 1000; }
+
+uint64_t ssa_launch_count(void) { return ssa::g_launches.load(std::memory_order_relaxed); }
+
+ssa_status ssa_device_error(uint32_t* code) {
+  if (!code) return SSA_ERR_INVALID_ARG;
+  *code = 0;
+  if (cudaDeviceSynchronize() != cudaSuccess) return SSA_ERR_CUDA;
+  uint32_t v = 0;
+  if (cudaMemcpyFromSymbol(&v, g_ssa_device_error, sizeof(v)) != cudaSuccess) return SSA_ERR_CUDA;
+  const uint32_t zero = 0;
+  if (cudaMemcpyToSymbol(g_ssa_device_error, &zero, sizeof(zero)) != cudaSuccess) return SSA_ERR_CUDA;
+  *code = v;
+  return v ? SSA_ERR_DEVICE : SSA_OK;
+}
+
+ssa_status ssa_block_summary(const ssa_params* pp, const void* K, float* mu, float* sigma,
+                             void* route_table, void* stream) {
+  ssa_status st = check_params(pp);
+  if (st != SSA_OK) return st;
+  const ssa_params& p = *pp;
+  if (p.dtype == SSA_F32 && route_table) return SSA_ERR_INVALID_ARG;
+  if (p.batch == 0 || p.n_kv == 0) return SSA_OK;
+  if (!K || !aligned16(K) || !aligned16(mu) || !aligned16(sigma) || !aligned16(route_table))
+    return SSA_ERR_INVALID_ARG;
+  LaunchCtx c;
+  if ((st = make_ctx(stream, c)) != SSA_OK) return st;
+  return do_summary(p, K, mu, sigma, route_table, c);
+}
+
+size_t ssa_route_workspace_size(const ssa_params* p) {
+  if (check_params(p) != SSA_OK) return 0;
+  return features_bytes(*p);
+}
+
+ssa_status ssa_route_topk(const ssa_params* pp, const void* Q, const float* mu, const float* sigma,
+                          const void* route_table, int32_t* block_idx, float* top_scores, void* ws,
+                          size_t ws_bytes, void* stream) {
+  ssa_status st = check_params(pp);
+  if (st != SSA_OK) return st;
+  const ssa_params& p = *pp;
+  if (is_empty(p)) return SSA_OK;
+  if (!Q || !block_idx || !aligned16(Q) || !aligned16(block_idx) || !aligned16(top_scores))
+    return SSA_ERR_INVALID_ARG;
+  if (p.dtype == SSA_F32 && (!mu || !sigma || !aligned16(mu) || !aligned16(sigma))) return SSA_ERR_INVALID_ARG;
+  if (p.dtype == SSA_BF16 && (!route_table || !aligned16(route_table))) return SSA_ERR_INVALID_ARG;
+  LaunchCtx c;
+  if ((st = make_ctx(stream, c)) != SSA_OK) return st;
+  return do_route(p, Q, mu, sigma, route_table, block_idx, top_scores, ws, ws_bytes, c);
+}
+
+ssa_status ssa_sparse_attn(const ssa_params* pp, const void* Q, const void* K, const void* V,
+                           const int32_t* block_idx, void* O, float* lse, int32_t* bad_index_count,
+                           void* stream) {
+  ssa_status st = check_params(pp);
+  if (st != SSA_OK) return st;
+  const ssa_params& p = *pp;
+  if (is_empty(p)) return SSA_OK;
+  if (!Q || !K || !V || !block_idx || !O) return SSA_ERR_INVALID_ARG;
+  if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(block_idx) || !aligned16(O) ||
+      (reinterpret_cast<uintptr_t>(lse) & 3u) || (reinterpret_cast<uintptr_t>(bad_index_count) & 3u))
+    return SSA_ERR_INVALID_ARG;
+  LaunchCtx c;
+  if ((st = make_ctx(stream, c)) != SSA_OK) return st;
+  return do_attn(p, Q, K, V, block_idx, O, lse, bad_index_count, c);
+}
+
+size_t ssa_workspace_size(const ssa_params* p) {
+  if (check_params(p) != SSA_OK) return 0;
+  return forward_layout(*p).total;
+}
+
+ssa_status ssa_forward(const ssa_params* pp, const void* Q, const void* K, const void* V, void* O,
+                       float* lse, void* ws, size_t ws_bytes, void* stream) {
+  ssa_status st = check_params(pp);
+  if (st != SSA_OK) return st;
+  const ssa_params& p = *pp;
+  if (is_empty(p)) return SSA_OK;
+  if (!Q || !K || !V || !O || !aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O) ||
+      (reinterpret_cast<uintptr_t>(lse) & 3u))
+    return SSA_ERR_INVALID_ARG;
+  LaunchCtx c;
+  if ((st = make_ctx(stream, c)) != SSA_OK) return st;
+  return forward_impl(p, Q, K, V, O, lse, static_cast<uint8_t*>(ws), ws_bytes, c);
+}
+
+size_t ssa_hostio_buffer_size(const ssa_params* p) {
+  if (check_params(p) != SSA_OK) return 0;
+  return hostio_layout(*p).total;
+}
+
+ssa_status ssa_forward_hostio(const ssa_params* pp, const void* hQ, const void* hK, const void* hV,
+                              void* hO, float* hlse, void* dev_buf, size_t dev_bytes, void* stream) {
+  ssa_status st = check_params(pp);
+  if (st != SSA_OK) return st;
+  const ssa_params& p = *pp;
+  if (is_empty(p)) return SSA_OK;
+  if (!hQ || !hK || !hV || !hO) return SSA_ERR_INVALID_ARG;
+  const HostioLayout L = hostio_layout(p);
+  if (!dev_buf || dev_bytes < L.total || !aligned16(dev_buf)) return SSA_ERR_WORKSPACE;
+  LaunchCtx c;
+  if ((st = make_ctx(stream, c)) != SSA_OK) return st;
+  uint8_t* d = static_cast<uint8_t*>(dev_buf);
+  const size_t es = esize(p);
+  const size_t qb = static_cast<size_t>(p.batch) * p.n_q * p.h_q * p.d * es;
+  const size_t kb = static_cast<size_t>(p.batch) * p.n_kv * p.h_kv * p.d * es;
+  const size_t lb = static_cast<size_t>(p.batch) * p.n_q * p.h_q * 4;
+  if (cudaMemcpyAsync(d + L.q, hQ, qb, cudaMemcpyHostToDevice, c.stream) != cudaSuccess ||
+      cudaMemcpyAsync(d + L.k, hK, kb, cudaMemcpyHostToDevice, c.stream) != cudaSuccess ||
+      cudaMemcpyAsync(d + L.v, hV, kb, cudaMemcpyHostToDevice, c.stream) != cudaSuccess)
+    return SSA_ERR_CUDA;
+  st = forward_impl(p, d + L.q, d + L.k, d + L.v, d + L.o, reinterpret_cast<float*>(d + L.lse), d + L.ws,
+                    L.total - L.ws, c);
+  if (st != SSA_OK) return st;
+  if (cudaMemcpyAsync(hO, d + L.o, qb, cudaMemcpyDeviceToHost, c.stream) != cudaSuccess) return SSA_ERR_CUDA;
+  if (hlse && cudaMemcpyAsync(hlse, d + L.lse, lb, cudaMemcpyDeviceToHost, c.stream) != cudaSuccess)
+    return SSA_ERR_CUDA;
+  return SSA_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,204 @@
+/*
+ * libssa: forward pass of one content-routed block-sparse attention (SSA)
+ * layer on NVIDIA B200 (sm_100a).
+ *
+ * The layer, as stated on "Subquadratic Sparse Attention (SSA)" (opening
+ * section and "The idea in one screen"):
+ *   (i)   summarise every block of B consecutive keys by its mean mu_c and
+ *         covariance Sigma_c (full, or its diagonal sigma_c^2), and route each
+ *         query with the second-cumulant score
+ *             r_c(q) = <q, mu_c> + (beta/2) q^T Sigma_c q ,
+ *         keeping a fixed budget of the top-k blocks;
+ *   (ii)  add a causal local window of W keys;
+ *   (iii) compute exact softmax attention over the selected keys.
+ *
+ * Conventions shared by every call
+ * --------------------------------
+ *  * All tensors are dense, row-major, caller-owned DEVICE buffers unless a
+ *    call says otherwise, and must be 16-byte aligned.  The library allocates
+ *    no memory and keeps no per-call state; scratch comes from the caller's
+ *    workspace.
+ *  * Layouts (b = batch, nb = n_kv / block, G = h_q / h_kv):
+ *      Q, O        [b, n_q,  h_q,  d]   elements of `dtype`
+ *      K, V        [b, n_kv, h_kv, d]   elements of `dtype`
+ *      mu          [b, h_kv, nb, d]     float32
+ *      sigma       [b, h_kv, nb, d]     float32   (SSA_SIGMA_DIAG: sigma_c^2)
+ *                  [b, h_kv, nb, d, d]  float32   (SSA_SIGMA_FULL: Sigma_c)
+ *      route_table [b, h_kv, nb, 2d]    bfloat16  row c = [mu_c ; sigma_c^2]
+ *                                       (bf16 problems only)
+ *      block_idx   [b, n_q, h_kv, topk] int32, ascending, padded with -1
+ *      top_scores  [b, n_q, h_kv, topk] float32 score of each block_idx entry
+ *      lse         [b, n_q, h_q]        float32, log sum_j exp(scale q.k_j)
+ *  * Query row i sits at key position pos = q_offset + i (prefill: 0;
+ *    one decode token: n_kv - 1).  Block c is a routing candidate only when
+ *    fully visible, (c+1)*block - 1 <= pos.  The window is the keys
+ *    pos-W+1 .. pos.  The attended set is the union of the selected blocks'
+ *    keys and the window keys.  Ties in the routing score go to the lower
+ *    block index.  With grouped-query attention the G query heads of a
+ *    kv-head share one selection, ranked by the sum of their scores.
+ *  * bf16 problems route on bf16 features f = [bf16(sum_h q_h),
+ *    bf16((beta/2) sum_h q_h*q_h)] (float32 sums in head order) against the
+ *    bf16 route table; float32 problems route in float32 on mu / sigma.
+ *  * Every call validates its arguments before launching anything and
+ *    returns SSA_ERR_INVALID_ARG / SSA_ERR_UNSUPPORTED / SSA_ERR_WORKSPACE
+ *    without side effects.  Work is enqueued asynchronously on `stream`
+ *    (a cudaStream_t; NULL = legacy default stream).  A failed launch returns
+ *    SSA_ERR_CUDA.  A kernel whose internal wait exceeds its time limit stops
+ *    early and records a code read by ssa_device_error().  No C++ exception
+ *    crosses this interface.  Calls are reentrant.
+ *  * Supported: d in {64, 128}; block in {64, 128}; G in {1, 2, 4, 8};
+ *    1 <= topk <= 32; 1 <= window <= 4032; n_kv % block == 0;
+ *    0 <= q_offset and q_offset + n_q <= n_kv; bf16 requires SSA_SIGMA_DIAG.
+ *    batch == 0 or n_q == 0 is a valid empty problem (nothing is launched).
+ */
+#ifndef SSA_H_
+#define SSA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define SSA_API __attribute__((visibility("default")))
+#else
+#define SSA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  SSA_OK = 0,
+  SSA_ERR_INVALID_ARG = 1,   /* null / misaligned pointer, inconsistent shape  */
+  SSA_ERR_UNSUPPORTED = 2,   /* valid problem outside the supported set         */
+  SSA_ERR_WORKSPACE = 3,     /* workspace pointer or size too small             */
+  SSA_ERR_CUDA = 4,          /* a CUDA runtime call or kernel launch failed     */
+  SSA_ERR_DEVICE = 5         /* a kernel recorded a device-side failure          */
+} ssa_status;
+
+typedef enum { SSA_F32 = 0, SSA_BF16 = 1 } ssa_dtype;
+typedef enum { SSA_SIGMA_DIAG = 0, SSA_SIGMA_FULL = 1 } ssa_sigma;
+
+/* Routing kernel choice for bf16 problems (ssa_params.route_impl). */
+typedef enum {
+  SSA_ROUTE_AUTO = 0,   /* tensor-core tiles when n_q >= 128, else per row    */
+  SSA_ROUTE_TILED = 1,  /* tcgen05 128-row tiles with fused streaming top-k    */
+  SSA_ROUTE_ROWWISE = 2 /* one CTA per query row (decode-shaped work)          */
+} ssa_route_impl;
+
+/* 64 bytes, no padding: twelve int32, one int64, two float32. */
+typedef struct {
+  int32_t batch;      /* b                                               */
+  int32_t n_q;        /* query rows per sequence                         */
+  int32_t n_kv;       /* keys per sequence (multiple of block)           */
+  int32_t h_q;        /* query heads                                     */
+  int32_t h_kv;       /* key/value heads (h_q % h_kv == 0)               */
+  int32_t d;          /* head dimension                                  */
+  int32_t block;      /* B, keys per routing block                       */
+  int32_t topk;       /* k, routed blocks per (query row, kv-head)       */
+  int32_t window;     /* W, causal local window in keys                  */
+  int32_t dtype;      /* ssa_dtype of Q, K, V, O                          */
+  int32_t sigma;      /* ssa_sigma                                        */
+  int32_t route_impl; /* ssa_route_impl                                   */
+  int64_t q_offset;   /* key position of query row 0                      */
+  float beta;         /* routing inverse temperature                      */
+  float scale;        /* attention logit scale (normally 1/sqrt(d))        */
+} ssa_params;
+
+/* Human-readable name of a status code (static string, never NULL). */
+SSA_API const char* ssa_status_string(int32_t status);
+
+/* Library ABI version (major*1000 + minor). */
+SSA_API int32_t ssa_version(void);
+
+/* Number of kernels this process has launched through libssa so far. */
+SSA_API uint64_t ssa_launch_count(void);
+
+/*
+ * Reads and clears the device-side failure word of the current device
+ * (synchronises the device).  *code is 0 when no kernel recorded a failure,
+ * else an identifier of the wait that timed out.  Returns SSA_ERR_DEVICE when
+ * *code != 0.
+ */
+SSA_API ssa_status ssa_device_error(uint32_t* code);
+
+/*
+ * Step (i), summaries: "routes ... using only per-block summary statistics"
+ * [Subquadratic Sparse Attention (SSA), opening section] with
+ * mu_c = (1/B) sum_{j in c} k_j and the population covariance
+ * Sigma_c = (1/B) sum_{j in c} (k_j - mu_c)(k_j - mu_c)^T (or its diagonal).
+ * Sums are accumulated in float64; mu / sigma are the float32 roundings and
+ * route_table holds their bfloat16 roundings.
+ *   K            device, [b, n_kv, h_kv, d] of dtype (read)
+ *   mu, sigma    device float32 outputs, may each be NULL (not written)
+ *   route_table  device bf16 output [b, h_kv, nb, 2d]; bf16 problems only,
+ *                may be NULL; must be NULL for float32 problems
+ */
+SSA_API ssa_status ssa_block_summary(const ssa_params* p, const void* K, float* mu, float* sigma,
+                             void* route_table, void* stream);
+
+/* Bytes of device workspace ssa_route_topk needs (0 when none). */
+SSA_API size_t ssa_route_workspace_size(const ssa_params* p);
+
+/*
+ * Step (i), routing and selection: r_c(q) = <q, mu_c> + (beta/2) q^T Sigma_c q
+ * ["The idea in one screen", routing-score equation] for every fully visible
+ * block, then the top-k blocks under (higher score, lower index) with a fixed
+ * budget k ["fixed budget kappa << n", opening section].  The score matrix is
+ * never written to memory: selection runs in the scoring kernel's epilogue.
+ *   Q            device [b, n_q, h_q, d] of dtype
+ *   mu, sigma    device float32 summaries (float32 problems; else ignored)
+ *   route_table  device bf16 table (bf16 problems; else ignored)
+ *   block_idx    device int32 output
+ *   top_scores   device float32 output, may be NULL
+ *   ws, ws_bytes device workspace of at least ssa_route_workspace_size(p)
+ */
+SSA_API ssa_status ssa_route_topk(const ssa_params* p, const void* Q, const float* mu,
+                          const float* sigma, const void* route_table, int32_t* block_idx,
+                          float* top_scores, void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * Steps (ii)+(iii): exact softmax attention of every query head over the
+ * union of its kv-head's selected blocks and the causal window
+ * [opening section, (ii) and (iii)], with an online (running max / running
+ * sum) softmax.  block_idx entries that are not -1 must be ascending,
+ * distinct and fully visible; any other entry is skipped and, when
+ * bad_index_count is not NULL, counted into that device int32 (atomically
+ * added, not reset).
+ *   O            device output [b, n_q, h_q, d] of dtype
+ *   lse          device float32 output, may be NULL
+ */
+SSA_API ssa_status ssa_sparse_attn(const ssa_params* p, const void* Q, const void* K, const void* V,
+                           const int32_t* block_idx, void* O, float* lse,
+                           int32_t* bad_index_count, void* stream);
+
+/* Bytes of device workspace ssa_forward needs. */
+SSA_API size_t ssa_workspace_size(const ssa_params* p);
+
+/*
+ * The whole layer: ssa_block_summary, ssa_route_topk and ssa_sparse_attn on
+ * `stream`, with the summaries, routing features and block indices carved
+ * from the caller's workspace (at least ssa_workspace_size(p) bytes).
+ */
+SSA_API ssa_status ssa_forward(const ssa_params* p, const void* Q, const void* K, const void* V,
+                       void* O, float* lse, void* ws, size_t ws_bytes, void* stream);
+
+/* Bytes of device buffer ssa_forward_hostio needs. */
+SSA_API size_t ssa_hostio_buffer_size(const ssa_params* p);
+
+/*
+ * ssa_forward on HOST inputs and outputs: copies hQ, hK, hV into dev_buf,
+ * runs the layer and copies O (and lse when hlse is not NULL) back, all
+ * enqueued on `stream`; the caller synchronises.  Host buffers should be
+ * page-locked for the copies to be asynchronous.  dev_buf must hold
+ * ssa_hostio_buffer_size(p) bytes of device memory.
+ */
+SSA_API ssa_status ssa_forward_hostio(const ssa_params* p, const void* hQ, const void* hK,
+                              const void* hV, void* hO, float* hlse, void* dev_buf,
+                              size_t dev_bytes, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SSA_H_ */

@@ -1,0 +1,288 @@
+"""GPU parity: every stage of the CUDA path, called through the C ABI, against
+the CPU oracle on the same seeded inputs.
+
+Stages are isolated by feeding the CUDA kernel the oracle's output of the
+previous stage (oracle summaries -> CUDA router; oracle block indices ->
+CUDA attention), then the whole layer is compared end to end.  Sizes span
+several row tiles, a ragged last tile and several blocks per window.
+"""
+import ctypes as C
+
+import numpy as np
+import pytest
+import torch
+
+from content_routed_block_ssa_b200 import ssa
+from content_routed_block_ssa_b200.workload import Workload, make_inputs, problem_dict
+from oracle import ssa_oracle as O
+
+from parity_util import (as_np, check_no_device_error, compare_idx, compare_out, gpu_attn, gpu_route,
+                         gpu_summary, params, NEAR_TIE_BAND)
+
+pytestmark = pytest.mark.gpu
+
+CASES = {
+    "bf16_gqa4_d128_b64": Workload("c", 101, 2, 1152, 8, 2, 128, "bf16", 64, "diag", 8, 256, 6, "total",
+                                   clustered=True),
+    "bf16_mha_d128_b64_k32": Workload("c", 102, 1, 2112, 2, 2, 128, "bf16", 64, "diag", 32, 128, 8, "per_head"),
+    "bf16_gqa8_d128_b128_k16": Workload("c", 103, 1, 3072, 8, 1, 128, "bf16", 128, "diag", 16, 256, 12, "total",
+                                        clustered=True),
+    "bf16_gqa2_d64_b64": Workload("c", 104, 1, 1024, 4, 2, 64, "bf16", 64, "diag", 4, 64, 6, "total"),
+    "bf16_mha_d64_b128_w200": Workload("c", 105, 1, 1280, 1, 1, 64, "bf16", 128, "diag", 8, 200, 4, "total"),
+    "f32_full_d64": Workload("c", 106, 1, 1024, 1, 1, 64, "f32", 64, "full", 8, 64, 8, "total"),
+    "f32_diag_d128_gqa4_w100": Workload("c", 107, 1, 512, 4, 1, 128, "f32", 64, "diag", 4, 100, 4, "total"),
+    "f32_full_gqa2_d64_b128": Workload("c", 108, 1, 768, 2, 1, 64, "f32", 128, "full", 2, 64, 2, "total"),
+}
+
+_cache = {}
+
+
+def case(name):
+    if name not in _cache:
+        w = CASES[name]
+        Q, K, V, plan = make_inputs(w, "cpu")
+        pd = problem_dict(w)
+        op = O.Problem(**pd)
+        Qn, Kn, Vn = Q.float().numpy(), K.float().numpy(), V.float().numpy()
+        ref = O.forward(Qn, Kn, Vn, op)
+        _cache[name] = dict(w=w, pd=pd, op=op, Q=Q, K=K, V=V, Qn=Qn, Kn=Kn, Vn=Vn, ref=ref)
+    return _cache[name]
+
+
+def to_dev(*ts):
+    return [t.cuda() for t in ts]
+
+
+@pytest.mark.parametrize("name", list(CASES))
+def test_summary_bit_exact(name):
+    c = case(name)
+    p = params(c["pd"])
+    (K,) = to_dev(c["K"])
+    mu, sig, tab = gpu_summary(p, K)
+    check_no_device_error()
+    mu32, sig32, table = c["ref"]["stored"]
+    assert np.array_equal(mu.cpu().numpy().astype(np.float64), mu32)
+    g = sig.cpu().numpy()
+    r = sig32.astype(np.float32)
+    ulp = np.abs(g.view(np.int32).astype(np.int64) - r.view(np.int32).astype(np.int64))
+    assert ulp.max() <= 1 and np.mean(ulp > 0) < 1e-4
+    if tab is not None:
+        assert np.array_equal(tab.float().cpu().numpy().astype(np.float64), table)
+
+
+def _stored_on_device(c):
+    mu32, sig32, table = c["ref"]["stored"]
+    mu = torch.from_numpy(mu32.astype(np.float32)).cuda()
+    sig = torch.from_numpy(sig32.astype(np.float32)).cuda()
+    tab = torch.from_numpy(table).to(torch.bfloat16).cuda() if table is not None else None
+    return mu, sig, tab
+
+
+ROUTE_IMPLS = [(n, impl) for n in CASES for impl in
+               ((ssa.SSA_ROUTE_TILED, ssa.SSA_ROUTE_ROWWISE) if CASES[n].dtype == "bf16" else (ssa.SSA_ROUTE_AUTO,))]
+
+
+@pytest.mark.parametrize("name,impl", ROUTE_IMPLS)
+def test_route_matches_oracle_selection(name, impl):
+    c = case(name)
+    p = params(c["pd"], impl)
+    (Q,) = to_dev(c["Q"])
+    mu, sig, tab = _stored_on_device(c)
+    idx, sc = gpu_route(p, Q, mu, sig, tab)
+    check_no_device_error()
+    gi = idx.cpu().numpy()
+    n, strict, literal, in_band = compare_idx(gi, c["ref"]["block_idx"], c["ref"]["gaps"])
+    assert strict == 0, f"{strict} of {n} rows differ outside the {NEAR_TIE_BAND} near-tie band"
+    # scores of the selected blocks agree with the oracle's to float32 accumulation error
+    stored = c["ref"]["stored"]
+    op = c["op"]
+    gs = sc.cpu().numpy()
+    rng = np.random.default_rng(0)
+    for bi in range(op.batch):
+        for g in range(op.h_kv):
+            S = O.route_scores(c["Qn"], stored, op, bi, g)
+            for i in rng.choice(op.n_q, size=min(64, op.n_q), replace=False):
+                for j in range(op.topk):
+                    blk = gi[bi, i, g, j]
+                    if blk >= 0:
+                        assert abs(gs[bi, i, g, j] - S[i, blk]) <= 2e-5 * abs(S[i, blk]) + 1e-4
+                    else:
+                        assert gs[bi, i, g, j] == -np.inf
+    # rows with fewer visible blocks than k keep all of them, then -1
+    for i in range(min(op.n_q, 3 * op.block)):
+        nv = O.visible_blocks(op.q_offset + i, op)
+        if nv <= op.topk:
+            assert list(gi[0, i, 0, :nv]) == list(range(nv))
+            assert np.all(gi[0, i, 0, nv:] == -1)
+
+
+@pytest.mark.parametrize("name", list(CASES))
+def test_attention_matches_oracle_on_oracle_selection(name):
+    c = case(name)
+    p = params(c["pd"])
+    Q, K, V = to_dev(c["Q"], c["K"], c["V"])
+    idx = torch.from_numpy(c["ref"]["block_idx"].astype(np.int32)).cuda()
+    O_, lse, bad = gpu_attn(p, Q, K, V, idx)
+    check_no_device_error()
+    assert int(bad.item()) == 0
+    max_abs, rel, ok = compare_out(as_np(O_), c["ref"]["O"], c["w"].dtype)
+    assert ok, (max_abs, rel)
+    np.testing.assert_allclose(lse.cpu().numpy(), c["ref"]["lse"], rtol=0, atol=2e-3 if c["w"].dtype == "bf16" else 1e-4)
+
+
+@pytest.mark.parametrize("name", list(CASES))
+def test_forward_end_to_end(name):
+    c = case(name)
+    p = params(c["pd"])
+    Q, K, V = to_dev(c["Q"], c["K"], c["V"])
+    ws = ssa.byte_buffer(ssa.ssa_workspace_size(p))
+    O_ = torch.empty_like(Q)
+    lse = torch.empty(Q.shape[:3], dtype=torch.float32, device="cuda")
+    ssa.ssa_forward(p, Q, K, V, O_, lse, ws)
+    check_no_device_error()
+    gaps = c["ref"]["gaps"]                      # [b, n_q, h_kv]
+    keep = np.all(gaps >= NEAR_TIE_BAND, axis=2)   # rows with no near-tie in any kv-head
+    got = as_np(O_)
+    max_abs, rel, ok = compare_out(got[keep], c["ref"]["O"][keep], c["w"].dtype)
+    assert ok, (max_abs, rel)
+    # the staged calls run the same kernels: identical bytes
+    mu, sig, tab = gpu_summary(p, K)
+    idx, _ = gpu_route(p, Q, mu, sig, tab)
+    O2, lse2, _ = gpu_attn(p, Q, K, V, idx)
+    assert torch.equal(O_, O2) and torch.equal(lse, lse2)
+
+
+def test_hostio_matches_device_forward():
+    c = case("bf16_gqa4_d128_b64")
+    p = params(c["pd"])
+    Q, K, V = to_dev(c["Q"], c["K"], c["V"])
+    ws = ssa.byte_buffer(ssa.ssa_workspace_size(p))
+    O_ = torch.empty_like(Q)
+    ssa.ssa_forward(p, Q, K, V, O_, None, ws)
+    hQ, hK, hV = (t.pin_memory() for t in (c["Q"], c["K"], c["V"]))
+    hO = torch.empty_like(c["Q"]).pin_memory()
+    hl = torch.empty(c["Q"].shape[:3], dtype=torch.float32).pin_memory()
+    buf = ssa.byte_buffer(ssa.ssa_hostio_buffer_size(p))
+    ssa.ssa_forward_hostio(p, hQ, hK, hV, hO, hl, buf)
+    torch.cuda.synchronize()
+    assert torch.equal(hO, O_.cpu())
+
+
+def test_decode_row_equals_last_prefill_row():
+    w = Workload("c", 110, 3, 2048, 8, 2, 128, "bf16", 64, "diag", 8, 256, 4, "per_seq", decode=True)
+    Q, K, V, _ = make_inputs(w, "cpu")
+    pd = problem_dict(w)
+    op = O.Problem(**pd)
+    ref = O.forward(Q.float().numpy(), K.float().numpy(), V.float().numpy(), op)
+    p = params(pd)
+    Qd, Kd, Vd = to_dev(Q, K, V)
+    mu, sig, tab = gpu_summary(p, Kd)
+    idx, _ = gpu_route(p, Qd, mu, sig, tab)
+    O_, lse, _ = gpu_attn(p, Qd, Kd, Vd, idx)
+    check_no_device_error()
+    n, strict, _, _ = compare_idx(idx.cpu().numpy(), ref["block_idx"], ref["gaps"])
+    assert strict == 0
+    _, _, ok = compare_out(as_np(O_), ref["O"], "bf16")
+    assert ok
+    # the decode row is the prefill definition's last row
+    pp = O.Problem(**{**pd, "n_q": w.n, "q_offset": 0})
+    Qfull = np.zeros((w.batch, w.n, w.h_q, w.d))
+    Qfull[:, -1] = Q.float().numpy()[:, 0]
+    last = O.forward(Qfull, K.float().numpy(), V.float().numpy(), pp, rows=[(b, w.n - 1) for b in range(w.batch)])
+    np.testing.assert_allclose(last["O"][:, -1], ref["O"][:, 0], atol=1e-12)
+
+
+def test_full_budget_is_dense_causal_attention():
+    w = Workload("c", 111, 1, 1024, 8, 2, 128, "bf16", 64, "diag", 16, 64, 0, "total")
+    Q, K, V, _ = make_inputs(w, "cpu")
+    pd = problem_dict(w)
+    op = O.Problem(**pd)
+    Od, _ = O.dense_causal_attention(Q.float().numpy(), K.float().numpy(), V.float().numpy(), op)
+    p = params(pd)
+    Qd, Kd, Vd = to_dev(Q, K, V)
+    ws = ssa.byte_buffer(ssa.ssa_workspace_size(p))
+    O_ = torch.empty_like(Qd)
+    ssa.ssa_forward(p, Qd, Kd, Vd, O_, None, ws)
+    check_no_device_error()
+    _, _, ok = compare_out(as_np(O_), Od, "bf16")
+    assert ok
+
+
+def _clean_row(row, nvis):
+    out, run = [], -1
+    for v in row:
+        if 0 <= v < nvis:
+            if v > run:
+                out.append(v)
+            run = max(run, v)
+    return out
+
+
+def test_invalid_block_indices_are_skipped_and_counted():
+    c = case("bf16_gqa4_d128_b64")
+    op = c["op"]
+    p = params(c["pd"])
+    rng = np.random.default_rng(5)
+    idx = c["ref"]["block_idx"].copy()
+    n_bad = 0
+    for _ in range(300):
+        b, i, g = rng.integers(0, op.batch), rng.integers(0, op.n_q), rng.integers(0, op.h_kv)
+        j = rng.integers(0, op.topk)
+        idx[b, i, g, j] = rng.choice([op.nb + 3, -5, 10 ** 6, idx[b, i, g, max(j - 1, 0)], 0])
+    expect_bad = 0
+    clean = np.full_like(idx, -1)
+    for b in range(op.batch):
+        for i in range(op.n_q):
+            nv = O.visible_blocks(i, op)
+            for g in range(op.h_kv):
+                row = list(idx[b, i, g])
+                kept = _clean_row(row, nv)
+                expect_bad += sum(1 for v in row if v != -1) - len(kept)
+                clean[b, i, g, :len(kept)] = kept
+    Q, K, V = to_dev(c["Q"], c["K"], c["V"])
+    O_, _, bad = gpu_attn(p, Q, K, V, torch.from_numpy(idx.astype(np.int32)).cuda())
+    check_no_device_error()
+    assert int(bad.item()) == expect_bad and expect_bad > 0
+    rows = [(b, i) for b in range(op.batch) for i in range(0, op.n_q, 7)]
+    Oref, _ = O.attention(c["Qn"], c["Kn"], c["Vn"], clean, op, rows=rows)
+    got = as_np(O_)
+    for b, i in rows:
+        assert np.abs(got[b, i] - Oref[b, i]).max() < 2e-2
+    del n_bad
+
+
+def test_window_of_one_key_and_early_rows():
+    w = Workload("c", 112, 1, 640, 4, 4, 64, "bf16", 64, "diag", 4, 1, 0, "total")
+    Q, K, V, _ = make_inputs(w, "cpu")
+    pd = problem_dict(w)
+    op = O.Problem(**pd)
+    ref = O.forward(Q.float().numpy(), K.float().numpy(), V.float().numpy(), op)
+    p = params(pd)
+    Qd, Kd, Vd = to_dev(Q, K, V)
+    ws = ssa.byte_buffer(ssa.ssa_workspace_size(p))
+    O_ = torch.empty_like(Qd)
+    ssa.ssa_forward(p, Qd, Kd, Vd, O_, None, ws)
+    check_no_device_error()
+    keep = np.all(ref["gaps"] >= NEAR_TIE_BAND, axis=2)
+    _, _, ok = compare_out(as_np(O_)[keep], ref["O"][keep], "bf16")
+    assert ok
+    # rows before the first full block attend only to themselves: o = v_pos
+    got = as_np(O_)
+    for i in range(63):
+        np.testing.assert_allclose(got[0, i], np.repeat(V.float().numpy()[0, i], 1, axis=0), atol=1e-2)
+
+
+def test_empty_problem_launches_nothing_and_small_workspace_is_rejected():
+    before = ssa.ssa_launch_count()
+    p = ssa.make_params(0, 128, 128, 2, 2, 128, 64, 4, 64)
+    ssa.ssa_forward(p, None, None, None, None, None, None)
+    assert ssa.ssa_launch_count() == before
+    c = case("bf16_gqa4_d128_b64")
+    p = params(c["pd"])
+    Q, K, V = to_dev(c["Q"], c["K"], c["V"])
+    O_ = torch.empty_like(Q)
+    small = ssa.byte_buffer(ssa.ssa_workspace_size(p) - 4096)
+    with pytest.raises(ssa.SSAError) as e:
+        ssa.ssa_forward(p, Q, K, V, O_, None, small)
+    assert e.value.status == ssa.SSA_ERR_WORKSPACE
+    assert ssa.ssa_launch_count() == before

@@ -1,0 +1,122 @@
+"""Host-side checks of the C ABI: no kernel is launched here.
+
+The library must load, export every entry point ``include/ssa.h`` declares,
+lay ``ssa_params`` out as the header says, and reject invalid or unsupported
+arguments with the documented status codes before touching the GPU.
+"""
+import ctypes as C
+import os
+import re
+
+import pytest
+
+from content_routed_block_ssa_b200 import ssa
+
+HEADER = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include", "ssa.h")
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"SSA_API\s+[\w\s\*]+?\b(ssa_\w+)\s*\(", text)))
+
+
+def test_library_exports_every_declared_symbol():
+    names = declared_functions()
+    assert len(names) >= 12
+    lib = C.CDLL(ssa.LIB_PATH)
+    for n in names:
+        assert hasattr(lib, n), n
+    assert sorted(ssa.EXPORTED) == names
+
+
+def test_params_layout_matches_header():
+    assert C.sizeof(ssa.ssa_params) == 64
+    assert ssa.ssa_params.q_offset.offset == 48
+    assert ssa.ssa_params.beta.offset == 56
+    assert ssa.ssa_params.scale.offset == 60
+    text = open(HEADER).read()
+    body = text[text.index("typedef struct {"):text.index("} ssa_params;")]
+    fields = re.findall(r"\b(int32_t|int64_t|float)\s+(\w+);", body)
+    assert [f for _, f in fields] == [f for f, _ in ssa.ssa_params._fields_]
+
+
+def test_status_strings():
+    assert ssa.status_string(0) == "SSA_OK"
+    assert ssa.status_string(3) == "SSA_ERR_WORKSPACE"
+    assert ssa.status_string(99) == "SSA_ERR_UNKNOWN"
+    assert ssa.lib.ssa_version() == 1000
+
+
+def good(**kw):
+    base = dict(batch=1, n_q=256, n_kv=256, h_q=4, h_kv=2, d=128, block=64, topk=4, window=64)
+    base.update(kw)
+    return ssa.make_params(**base)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(n_kv=250), ssa.SSA_ERR_INVALID_ARG),              # n_kv % block
+    (dict(h_q=3), ssa.SSA_ERR_INVALID_ARG),                 # h_q % h_kv
+    (dict(topk=0), ssa.SSA_ERR_INVALID_ARG),
+    (dict(window=0), ssa.SSA_ERR_INVALID_ARG),
+    (dict(q_offset=1), ssa.SSA_ERR_INVALID_ARG),            # queries past the last key
+    (dict(q_offset=-1), ssa.SSA_ERR_INVALID_ARG),
+    (dict(batch=-1), ssa.SSA_ERR_INVALID_ARG),
+    (dict(scale=0.0), ssa.SSA_ERR_INVALID_ARG),
+    (dict(beta=float("nan")), ssa.SSA_ERR_INVALID_ARG),
+    (dict(dtype=7), ssa.SSA_ERR_INVALID_ARG),
+    (dict(route_impl=5), ssa.SSA_ERR_INVALID_ARG),
+    (dict(d=96), ssa.SSA_ERR_UNSUPPORTED),
+    (dict(block=32, n_kv=256), ssa.SSA_ERR_UNSUPPORTED),
+    (dict(h_q=6, h_kv=2), ssa.SSA_ERR_UNSUPPORTED),         # G = 3
+    (dict(topk=33), ssa.SSA_ERR_UNSUPPORTED),
+    (dict(window=5000), ssa.SSA_ERR_UNSUPPORTED),
+    (dict(sigma="full"), ssa.SSA_ERR_UNSUPPORTED),          # bf16 routes on a diagonal Sigma
+])
+def test_invalid_and_unsupported_params(kw, code):
+    p = good(**kw)
+    dummy = 256   # any non-null, 16-byte-aligned value: validation fails first
+    assert ssa.lib.ssa_block_summary(C.byref(p), dummy, None, None, dummy, None) == code
+    assert ssa.lib.ssa_forward(C.byref(p), dummy, dummy, dummy, dummy, None, dummy, 1 << 30, None) == code
+    assert ssa.lib.ssa_sparse_attn(C.byref(p), dummy, dummy, dummy, dummy, dummy, None, None, None) == code
+    assert ssa.lib.ssa_workspace_size(C.byref(p)) == 0
+
+
+def test_null_and_misaligned_pointers_rejected():
+    p = good()
+    assert ssa.lib.ssa_block_summary(None, 256, None, None, None, None) == ssa.SSA_ERR_INVALID_ARG
+    assert ssa.lib.ssa_block_summary(C.byref(p), None, None, None, 256, None) == ssa.SSA_ERR_INVALID_ARG
+    assert ssa.lib.ssa_block_summary(C.byref(p), 258, None, None, 256, None) == ssa.SSA_ERR_INVALID_ARG
+    assert ssa.lib.ssa_route_topk(C.byref(p), 256, None, None, None, 256, None, None, 0, None) == \
+        ssa.SSA_ERR_INVALID_ARG                           # bf16 needs the route table
+    assert ssa.lib.ssa_sparse_attn(C.byref(p), 256, 256, 256, None, 256, None, None, None) == \
+        ssa.SSA_ERR_INVALID_ARG
+    assert ssa.lib.ssa_forward(C.byref(p), 256, 256, 264, 256, None, 256, 1 << 30, None) == \
+        ssa.SSA_ERR_INVALID_ARG
+    f32 = good(dtype="f32")
+    assert ssa.lib.ssa_block_summary(C.byref(f32), 256, 256, 256, 256, None) == ssa.SSA_ERR_INVALID_ARG
+
+
+def test_empty_problems_are_valid_noops():
+    for kw in (dict(batch=0), dict(n_q=0, q_offset=0)):
+        p = good(**kw)
+        assert ssa.lib.ssa_forward(C.byref(p), None, None, None, None, None, None, 0, None) == ssa.SSA_OK
+        assert ssa.lib.ssa_sparse_attn(C.byref(p), None, None, None, None, None, None, None, None) == ssa.SSA_OK
+        assert ssa.lib.ssa_route_topk(C.byref(p), None, None, None, None, None, None, None, 0, None) == ssa.SSA_OK
+
+
+def test_workspace_sizes():
+    p = good(n_q=1000, n_kv=1024)
+    nb = 1024 // 64
+    tab = 1 * 2 * nb * 256 * 2
+    feat = 1 * 2 * 1000 * 256 * 2
+    idx = 1 * 1000 * 2 * 4 * 4
+    rnd = lambda x: (x + 255) // 256 * 256
+    assert ssa.ssa_route_workspace_size(p) == rnd(feat)
+    assert ssa.ssa_workspace_size(p) == rnd(tab) + rnd(feat) + rnd(idx)
+    row = good(n_q=1, n_kv=1024, q_offset=1023)           # decode routes per row: no features
+    assert ssa.ssa_route_workspace_size(row) == 0
+    f32 = good(dtype="f32", sigma="full", d=64, h_q=2, n_q=128, n_kv=128)
+    nb = 2
+    assert ssa.ssa_workspace_size(f32) == rnd(2 * nb * 64 * 4) + rnd(2 * nb * 64 * 64 * 4) + rnd(128 * 2 * 4 * 4)
+    h = ssa.ssa_hostio_buffer_size(p)
+    assert h > ssa.ssa_workspace_size(p)
