@@ -1,0 +1,418 @@
+"""Benchmark of the SSA forward on B200: query-heads/s at 128K (and 1M) tokens.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload NAME] [--no-secondary]
+
+One step is one pass of the whole layer over the workload's synthetic input:
+block summaries -> routing features + tensor-core route with fused top-k ->
+gathered exact attention, each a call of the libssa C ABI on the current
+stream (ssa_forward issues the same three calls).  Inputs are resident in HBM
+when the timed region starts; L2 is flushed between steps.  Step time is the
+sum of CUDA-event intervals around the step's kernels, the reported time the
+max over ranks.  With N > 1 every rank runs its own replica of the workload
+(independent problems, no collective on the data path): weak scaling.
+
+`e2e` repeats the step through ssa_forward_hostio with page-locked host
+inputs and outputs, host<->device copies inside the timed region.
+
+`--impl reference` times the CPU oracle (float64 NumPy) on a bounded sample of
+the same workload on the host cores.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+from content_routed_block_ssa_b200.workload import WORKLOADS, make_inputs, problem_dict  # noqa: E402
+
+METRIC = "SSA fwd query-heads/s at 128K and 1M; % HBM BW (gather) / % TC peak (route)"
+UNIT = "query-heads/s"
+PRIMARY = "gqa_bf16_128k"
+SECONDARY = "gqa_bf16_1m"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return {k: float(d[k]) for k in FALLBACK_PEAKS}, "of measured"
+    except Exception:
+        return dict(FALLBACK_PEAKS), "of fallback"
+
+
+def load_traffic():
+    """Per-launch DRAM bytes of the dominant kernels from the committed ncu summary."""
+    out = {}
+    path = os.path.join(ROOT, "profiles", "dram_traffic.txt")
+    if not os.path.exists(path):
+        return out
+    for line in open(path):
+        parts = line.split()
+        if len(parts) == 3 and not line.startswith("#"):
+            out[(parts[0], parts[1])] = float(parts[2])
+    return out
+
+
+# ------------------------------------------------------------------ distributed
+
+def dist_setup(n_gpus):
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if ws > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=600),
+                                device_id=torch.device("cuda", local))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(0)
+    return ws, rank, local
+
+
+def barrier(ws):
+    if ws > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x, ws):
+    if ws == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ------------------------------------------------------------------ clocks
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except Exception:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self):
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in self.lines:
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx.append(float(f[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ------------------------------------------------------------------ algorithmic work
+
+def attended_keys(idx, w):
+    """|S_i| per (batch, row, kv-head): selected blocks' keys plus window keys
+    outside them (bookkeeping for the roofline, not part of the layer)."""
+    B, W = w.block, w.window
+    pos = torch.arange(w.n_q, device=idx.device, dtype=torch.int64).view(1, -1, 1, 1) + w.q_offset
+    lo = torch.clamp(pos - W + 1, min=0)
+    valid = idx >= 0
+    c = idx.to(torch.int64)
+    ov_lo = torch.maximum(c * B, lo)
+    ov_hi = torch.minimum(c * B + B - 1, pos)
+    overlap = torch.where(valid, torch.clamp(ov_hi - ov_lo + 1, min=0), torch.zeros_like(c)).sum(-1)
+    n_sel = valid.sum(-1).to(torch.int64)
+    wcount = (pos - lo + 1).squeeze(-1)
+    return n_sel * B + wcount - overlap
+
+
+def algorithmic_work(w, idx):
+    es = 4 if w.dtype == "f32" else 2
+    nb = w.n // w.block
+    G = w.h_q // w.h_kv
+    pos = np.arange(w.n_q) + w.q_offset
+    nvis = np.minimum(nb, (pos + 1) // w.block).sum()
+    summary_bytes = w.batch * w.n * w.h_kv * w.d * es + w.batch * w.h_kv * nb * 2 * w.d * 2
+    route_flops = 2.0 * (2 * w.d) * float(nvis) * w.h_kv * w.batch
+    S = attended_keys(idx, w)
+    gathered = float(S.sum().item()) * w.d * 2 * es
+    qo = 2.0 * w.batch * w.n_q * w.h_q * w.d * es
+    attn_flops = 4.0 * float(S.sum().item()) * G * w.d
+    return dict(summary_bytes=summary_bytes, route_flops=route_flops, attn_bytes=gathered + qo,
+                gathered_bytes=gathered, attn_flops=attn_flops, mean_keys=float(S.float().mean().item()))
+
+
+# ------------------------------------------------------------------ our arm
+
+def run_ours(w, steps, warmup, ws, rank, with_e2e=True):
+    from content_routed_block_ssa_b200 import ssa
+    dev = torch.device("cuda", torch.cuda.current_device())
+    Q, K, V, _ = make_inputs(w, dev)
+    p = ssa.make_params(**problem_dict(w))
+    mu_s, sig_s, tab_s = ssa.summary_shapes(p)
+    tab = torch.empty(tab_s, dtype=torch.bfloat16, device=dev)
+    idx = torch.empty(ssa.idx_shape(p), dtype=torch.int32, device=dev)
+    rws = ssa.byte_buffer(ssa.ssa_route_workspace_size(p), dev)
+    O = torch.empty_like(Q)
+    lse = torch.empty(Q.shape[:3], dtype=torch.float32, device=dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step(ev=None):
+        if ev:
+            ev[0].record(stream)
+        ssa.ssa_block_summary(p, K, None, None, tab)
+        if ev:
+            ev[1].record(stream)
+        ssa.ssa_route_topk(p, Q, None, None, tab, idx, None, rws)
+        if ev:
+            ev[2].record(stream)
+        ssa.ssa_sparse_attn(p, Q, K, V, idx, O, lse)
+        if ev:
+            ev[3].record(stream)
+
+    for _ in range(warmup):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(steps)]
+    barrier(ws)
+    torch.cuda.synchronize()
+    l0 = ssa.ssa_launch_count()
+    with ClockSampler(torch.cuda.current_device()) as clk:
+        for k in range(steps):
+            flush.zero_()
+            step(evs[k])
+        torch.cuda.synchronize()
+    launches = ssa.ssa_launch_count() - l0
+    barrier(ws)
+    assert ssa.ssa_device_error() == 0
+    per = np.array([[e[0].elapsed_time(e[1]), e[1].elapsed_time(e[2]), e[2].elapsed_time(e[3])] for e in evs])
+    ms_kernels = per.mean(axis=0)
+    ms_step_local = float(per.sum(axis=1).mean())
+    ms_step = max_over_ranks(ms_step_local, ws)
+    work = algorithmic_work(w, idx)
+
+    e2e = None
+    if with_e2e:
+        hQ, hK, hV = Q.cpu().pin_memory(), K.cpu().pin_memory(), V.cpu().pin_memory()
+        hO = torch.empty(Q.shape, dtype=Q.dtype).pin_memory()
+        hl = torch.empty(Q.shape[:3], dtype=torch.float32).pin_memory()
+        del O, lse
+        buf = ssa.byte_buffer(ssa.ssa_hostio_buffer_size(p), dev)
+        for _ in range(max(1, warmup)):
+            ssa.ssa_forward_hostio(p, hQ, hK, hV, hO, hl, buf)
+        torch.cuda.synchronize()
+        barrier(ws)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        n_e2e = max(1, min(steps, 5))
+        for _ in range(n_e2e):
+            ssa.ssa_forward_hostio(p, hQ, hK, hV, hO, hl, buf)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        ms_e2e = max_over_ranks(e0.elapsed_time(e1) / n_e2e, ws)
+        h2d = hQ.numel() * hQ.element_size() + 2 * hK.numel() * hK.element_size()
+        d2h = hO.numel() * hO.element_size() + hl.numel() * hl.element_size()
+        e2e = {"value": ws * w.batch * w.n_q * w.h_q / (ms_e2e / 1e3), "unit": UNIT,
+               "ms_per_step": ms_e2e, "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
+               "steps": n_e2e}
+        del buf
+    return dict(ms_step=ms_step, ms_kernels=ms_kernels, work=work, launches=int(launches),
+                clocks=clk.summary(), e2e=e2e)
+
+
+def kernel_report(w, res, peaks, traffic):
+    ms_s, ms_r, ms_a = (float(x) for x in res["ms_kernels"])
+    wk = res["work"]
+    hbm = peaks["hbm_gbs"]
+    tc = peaks["bf16_tflops_sustained"]
+    s_gbs = wk["summary_bytes"] / (ms_s * 1e-3) / 1e9
+    r_tf = wk["route_flops"] / (ms_r * 1e-3) / 1e12
+    a_gbs = wk["attn_bytes"] / (ms_a * 1e-3) / 1e9
+    return {
+        "summary": {"ms": ms_s, "bound": "hbm", "achieved": s_gbs, "unit": "GB/s", "frac": s_gbs / hbm,
+                    "algorithmic_bytes": wk["summary_bytes"]},
+        "route": {"ms": ms_r, "bound": "tensor", "achieved": r_tf, "unit": "TFLOP/s", "frac": r_tf / tc,
+                  "algorithmic_flops": wk["route_flops"], "peak": tc},
+        "attention": {"ms": ms_a, "bound": "hbm", "achieved": a_gbs, "unit": "GB/s", "frac": a_gbs / hbm,
+                      "algorithmic_bytes": wk["attn_bytes"], "mean_keys_per_row": wk["mean_keys"],
+                      "traffic": traffic.get(("attn_bf16", w.name))},
+    }
+
+
+# ------------------------------------------------------------------ oracle (CPU)
+
+def run_oracle_sample(w, rows_per_step, steps, warmup, seed=7):
+    """Times the oracle on the host: full block summaries once (amortised per
+    step by the sampled fraction), then route + attention of `rows_per_step`
+    query rows (all heads) per step.  Returns (query-heads/s, seconds, info)."""
+    from oracle import ssa_oracle as O
+    Q, K, V, _ = make_inputs(w, "cuda" if torch.cuda.is_available() else "cpu")
+    Kn = K.float().cpu().numpy()
+    Vn = V.float().cpu().numpy()
+    rng = np.random.default_rng(seed)
+    op = O.Problem(**problem_dict(w))
+    t0 = time.perf_counter()
+    mu, sig = O.block_summaries(Kn, op)
+    stored = O.stored_summaries(mu, sig, op)
+    t_sum = time.perf_counter() - t0
+    times = []
+    G = w.h_q // w.h_kv
+    for k in range(warmup + steps):
+        rows_i = np.sort(rng.choice(w.n_q, size=rows_per_step, replace=False))
+        Qs = Q[:, torch.from_numpy(rows_i).to(Q.device)].float().cpu().numpy()   # [b, rows, h_q, d]
+        t1 = time.perf_counter()
+        for bi in range(w.batch):
+            for r, i in enumerate(rows_i):
+                pos = w.q_offset + int(i)
+                pr = O.Problem(**{**problem_dict(w), "n_q": rows_per_step, "q_offset": pos - r})
+                for g in range(w.h_kv):
+                    s = O.route_scores_row(Qs, stored, pr, bi, r, g)
+                    sel, _ = O.select_topk(s, w.topk)
+                    S = O.key_set(pos, sel, op)
+                    O.softmax_attend(Qs[bi, r, g * G:(g + 1) * G], Kn[bi, S, g], Vn[bi, S, g], op.scale)
+        dt = time.perf_counter() - t1
+        if k >= warmup:
+            times.append(dt + t_sum * rows_per_step / w.n_q)
+    sec = float(np.mean(times))
+    qh = w.batch * rows_per_step * w.h_q
+    info = {"summary_s": t_sum, "rows_per_step": rows_per_step}
+    return qh / sec, sec, info
+
+
+def cores():
+    try:
+        return len(os.sched_getaffinity(0))
+    except Exception:
+        return os.cpu_count()
+
+
+# ------------------------------------------------------------------ main
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default=PRIMARY, choices=list(WORKLOADS))
+    ap.add_argument("--no-secondary", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--n", type=int, default=None,
+                    help="shorter sequence of the same workload (profiling captures); not a bench line")
+    a = ap.parse_args()
+    w = WORKLOADS[a.workload]
+    if a.n is not None:
+        w = w.scaled(n=a.n, needles=max(1, w.needles * a.n // w.n))
+    ws, rank, local = dist_setup(a.gpus)
+    peaks, peak_src = load_peaks()
+
+    config = {"workload": w.name, "batch": w.batch, "n": w.n, "n_q": w.n_q, "h_q": w.h_q, "h_kv": w.h_kv,
+              "d": w.d, "block": w.block, "topk": w.topk, "window": w.window, "sigma": w.sigma,
+              "beta": w.beta, "keys": "block-clustered + planted needles" if w.clustered else "iid + planted needles",
+              "l2": "flushed between steps (256 MiB write); inputs larger than L2",
+              "parallelism": f"replicas x{ws} (independent problems)"}
+
+    if a.impl == "reference":
+        if rank != 0:
+            return
+        rows = 4
+        val, sec, info = run_oracle_sample(w, rows, a.steps, a.warmup)
+        line = {"impl": "reference", "metric": METRIC, "value": val, "unit": UNIT, "n_gpus": a.gpus,
+                "steps": a.steps, "warmup": a.warmup, "ms_per_step": sec * 1e3, "higher_is_better": True,
+                "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic", "config": config,
+                "cpu_baseline": {"value": val, "unit": UNIT, "cores": cores(), "kind": "oracle",
+                                 "sample": f"{rows} query rows x {w.h_q} heads per step, block summaries of all "
+                                           f"{w.n} keys amortised by {rows}/{w.n_q}"},
+                "e2e": {"value": val, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+        print(json.dumps(line), flush=True)
+        return
+
+    traffic = load_traffic()
+    res = run_ours(w, a.steps, a.warmup, ws, rank, with_e2e=not a.no_e2e)
+    kern = kernel_report(w, res, peaks, traffic)
+    value = ws * w.batch * w.n_q * w.h_q / (res["ms_step"] / 1e3)
+    att = kern["attention"]
+    roof = {"bound": "hbm", "achieved": att["achieved"], "peak": peaks["hbm_gbs"], "unit": "GB/s",
+            "frac": att["frac"], "traffic": att["traffic"], "kernel": "attn_bf16_kernel",
+            "peak_source": peak_src, "algorithmic_bytes_per_launch": att["algorithmic_bytes"]}
+    secondary = None
+    if not a.no_secondary and w.name == PRIMARY and a.n is None:
+        torch.cuda.empty_cache()
+        w2 = WORKLOADS[SECONDARY]
+        r2 = run_ours(w2, max(3, a.steps // 2), a.warmup, ws, rank, with_e2e=False)
+        k2 = kernel_report(w2, r2, peaks, traffic)
+        secondary = {"workload": w2.name, "value": ws * w2.batch * w2.n_q * w2.h_q / (r2["ms_step"] / 1e3),
+                     "unit": UNIT, "ms_per_step": r2["ms_step"], "kernels": k2, "gpu_launches": r2["launches"],
+                     "clocks": r2["clocks"]}
+    cpu = None
+    if rank == 0 and ws == 1 and not a.no_cpu_baseline:
+        rows = 16
+        val, sec, info = run_oracle_sample(w, rows, 2, 1)
+        cpu = {"value": val, "unit": UNIT, "cores": cores(), "kind": "oracle",
+               "sample": f"{rows} query rows x {w.h_q} heads per step, block summaries of all {w.n} keys "
+                         f"amortised by {rows}/{w.n_q}; 2 steps after 1 warm-up"}
+    if rank == 0:
+        line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws, "steps": a.steps, "warmup": a.warmup,
+                "ms_per_step": res["ms_step"], "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+                "dtype": "bf16", "data": "synthetic", "config": config, "roofline": roof, "cpu_baseline": cpu,
+                "e2e": res["e2e"], "gpu_launches": res["launches"], "clocks": res["clocks"], "kernels": kern,
+                "secondary": secondary}
+        print(json.dumps(line), flush=True)
+    if ws > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

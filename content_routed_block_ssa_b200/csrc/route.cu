@@ -424,11 +424,14 @@ __device__ void select_and_write(uint64_t* keys, int nvis, int n2, const RowArgs
     const int lane = threadIdx.x;
     const uint64_t key = (lane < a.topk && lane < n2) ? keys[lane] : 0;
     const uint32_t blk = key ? key_block(key) : 0xFFFFFFFFu;
+    // valid entries are ranked by block index; empty slots follow, in lane order
+    const uint32_t vmask = __ballot_sync(0xFFFFFFFFu, key != 0);
     int rank = 0;
     for (int o = 0; o < 32; ++o) {
       const uint32_t other = __shfl_sync(0xFFFFFFFFu, blk, o);
       rank += (other < blk) ? 1 : 0;
     }
+    if (!key) rank = __popc(vmask) + __popc(~vmask & ((1u << lane) - 1u));
     if (lane < a.topk) {
       a.block_idx[out + rank] = key ? static_cast<int32_t>(blk) : -1;
       if (a.top_scores) a.top_scores[out + rank] = key ? key_score(key) : -INFINITY;

@@ -82,7 +82,10 @@ ROUTE_IMPLS = [(n, impl) for n in CASES for impl in
                ((ssa.SSA_ROUTE_TILED, ssa.SSA_ROUTE_ROWWISE) if CASES[n].dtype == "bf16" else (ssa.SSA_ROUTE_AUTO,))]
 
 
-@pytest.mark.parametrize("name,impl", ROUTE_IMPLS)
+IMPL_NAME = {ssa.SSA_ROUTE_AUTO: "auto", ssa.SSA_ROUTE_TILED: "tiled", ssa.SSA_ROUTE_ROWWISE: "rowwise"}
+
+
+@pytest.mark.parametrize("name,impl", ROUTE_IMPLS, ids=[f"{n}-{IMPL_NAME[i]}" for n, i in ROUTE_IMPLS])
 def test_route_matches_oracle_selection(name, impl):
     c = case(name)
     p = params(c["pd"], impl)
