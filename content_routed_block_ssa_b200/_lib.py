@@ -54,6 +54,7 @@ def _load():
         "ssa_block_summary": (i32, [P, vp, vp, vp, vp, vp]),
         "ssa_route_workspace_size": (sz, [P]),
         "ssa_route_topk": (i32, [P, vp, vp, vp, vp, vp, vp, vp, sz, vp]),
+        "ssa_route_topk_static": (i32, [P, vp, vp, vp, vp, vp, vp, vp]),
         "ssa_sparse_attn": (i32, [P, vp, vp, vp, vp, vp, vp, vp, vp]),
         "ssa_workspace_size": (sz, [P]),
         "ssa_forward": (i32, [P, vp, vp, vp, vp, vp, vp, sz, vp]),
@@ -70,7 +71,8 @@ def _load():
 lib = _load()
 LIB_PATH = _LIB_PATH
 EXPORTED = ("ssa_status_string", "ssa_version", "ssa_launch_count", "ssa_device_error",
-            "ssa_block_summary", "ssa_route_workspace_size", "ssa_route_topk", "ssa_sparse_attn",
+            "ssa_block_summary", "ssa_route_workspace_size", "ssa_route_topk", "ssa_route_topk_static",
+            "ssa_sparse_attn",
             "ssa_workspace_size", "ssa_forward", "ssa_hostio_buffer_size", "ssa_forward_hostio")
 
 
@@ -135,6 +137,16 @@ def ssa_route_topk(p, Q, mu, sigma, route_table, block_idx, top_scores=None, ws=
     _check(lib.ssa_route_topk(C.byref(p), _ptr(Q), _ptr(mu), _ptr(sigma), _ptr(route_table),
                               _ptr(block_idx), _ptr(top_scores), _ptr(ws), nbytes, _stream(stream)),
            "ssa_route_topk")
+
+
+ROUTE_STATIC_SCRATCH_BYTES = 16 << 20
+
+
+def ssa_route_topk_static(p, Q, mu, sigma, route_table, block_idx, top_scores=None, stream=None):
+    """ssa_route_topk with the library's fixed scratch array instead of a workspace."""
+    _check(lib.ssa_route_topk_static(C.byref(p), _ptr(Q), _ptr(mu), _ptr(sigma), _ptr(route_table),
+                                     _ptr(block_idx), _ptr(top_scores), _stream(stream)),
+           "ssa_route_topk_static")
 
 
 def ssa_sparse_attn(p, Q, K, V, block_idx, O, lse=None, bad_index_count=None, stream=None):

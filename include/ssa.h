@@ -172,6 +172,25 @@ SSA_API ssa_status ssa_sparse_attn(const ssa_params* p, const void* Q, const voi
                            const int32_t* block_idx, void* O, float* lse,
                            int32_t* bad_index_count, void* stream);
 
+/*
+ * ssa_route_topk without a caller workspace.  No counterpart in the paper:
+ * this is an interface convenience for callers that cannot allocate device
+ * memory when they route (a host framework whose allocator owns the whole
+ * device pool, or a loop that cannot afford cudaMalloc's implicit device
+ * synchronisation).  The routing-feature scratch lives in a fixed array of
+ * SSA_ROUTE_STATIC_SCRATCH_BYTES inside the library, present on every device
+ * that loads it until the process exits; problems that need more return
+ * SSA_ERR_WORKSPACE before any launch.  The first call on a device looks up
+ * the array's address with that device current; make it before any stream
+ * capture.  All calls share the array, so calls whose kernels overlap on the
+ * GPU race on it and must be serialised.  Arguments and results are those of
+ * ssa_route_topk.  Allocates nothing.
+ */
+#define SSA_ROUTE_STATIC_SCRATCH_BYTES (16u << 20)
+SSA_API ssa_status ssa_route_topk_static(const ssa_params* p, const void* Q, const float* mu,
+                                         const float* sigma, const void* route_table,
+                                         int32_t* block_idx, float* top_scores, void* stream);
+
 /* Bytes of device workspace ssa_forward needs. */
 SSA_API size_t ssa_workspace_size(const ssa_params* p);
 
