@@ -47,80 +47,137 @@ template <int D>
 struct AttnCfg {
   static constexpr int HALF = 64 * 64 * 2;            // 64 keys x 64 dims bf16 (8 KB)
   static constexpr int KBYTES = (D / 64) * HALF;
-  static constexpr int STAGE = 2 * KBYTES;            // K then V
-  static constexpr int NS = (D == 128) ? 6 : 10;
+  static constexpr int STAGE = 2 * KBYTES;            // K then V of one 64-key tile
+  static constexpr int NS = (D == 128) ? 6 : 12;      // tile ring
+  static constexpr int MAXT = 32 * 2 + 66;            // selected tiles (k <= 32, <= 2 per block) + window tiles
+  // item slot: Q tile (<= 8 heads, as D/64 boxes of G x 64), tile list, meta
+  static constexpr int QBYTES = 8 * D * 2;
+  static constexpr int SLOT = 4096;
   static constexpr int MERGE = 4 * 8 * D * 4 + 4 * 8 * 2 * 4;
-  static constexpr int SMEM = 1024 + NS * STAGE + MERGE + 2 * NS * 8 + 16;
+  static constexpr int NBAR = 2 * NS + 4;
+  static constexpr int SMEM = 1024 + NS * STAGE + 2 * SLOT + MERGE + NBAR * 8 + 32;
+  static_assert(QBYTES + MAXT * 4 + 64 <= SLOT, "item slot too small");
+};
+
+struct ItemMeta {
+  int64_t pos, lo, qrow;
+  int32_t n_sub, ns;
 };
 
 __device__ __forceinline__ void named_bar_consumers() {
-  asm volatile("bar.sync 1, 128;" ::: "memory");
+  asm volatile("bar.sync 1, 256;" ::: "memory");
 }
 
+// Warp roles: warp 8 = producer (item setup one item ahead: block list,
+// tile list and Q into an item slot; then TMA gathers of the item's tiles
+// into the ring), warps 0-7 = consumers in two groups of four; group 0 takes
+// the even tiles of an item, group 1 the odd ones.  Within a group every
+// 64-key tile is shared by the four warps, 16 keys each, so a ring stage is
+// released after a quarter of the tile's work and the rest of the ring stays
+// in flight; two groups give each SM sub-partition two warps to overlap.
 template <int D, int G>
-__global__ void __launch_bounds__(160, 1)
+__global__ void __launch_bounds__(288, 1)
     attn_bf16_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
-                     const AttnArgs a) {
+                     const __grid_constant__ CUtensorMap tmQ, const AttnArgs a) {
   using C = AttnCfg<D>;
   constexpr int KS = D / 16;    // k-steps over dims
   constexpr int MT = D / 16;    // dim m-tiles of O^T
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* stages = smem;
-  float* mO = reinterpret_cast<float*>(stages + C::NS * C::STAGE);   // [4][8][D]
+  uint8_t* slots = stages + C::NS * C::STAGE;                        // 2 item slots
+  float* mO = reinterpret_cast<float*>(slots + 2 * C::SLOT);          // [4][8][D]
   float* mM = mO + 4 * 8 * D;                                         // [4][8]
   float* mL = mM + 4 * 8;                                             // [4][8]
   uint64_t* full = reinterpret_cast<uint64_t*>(mL + 4 * 8);
   uint64_t* empty = full + C::NS;
-  int* abort_flag = reinterpret_cast<int*>(empty + C::NS);   // [4]
+  uint64_t* item_full = empty + C::NS;
+  uint64_t* item_empty = item_full + 2;
+  int* abort_flag = reinterpret_cast<int*>(item_empty + 2);          // [8]
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   if (threadIdx.x == 0) {
-    for (int s = 0; s < C::NS; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
+    for (int s = 0; s < C::NS; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 4); }
+    for (int s = 0; s < 2; ++s) { mbar_init(&item_full[s], 1); mbar_init(&item_empty[s], 8); }
     fence_barrier_init();
     tma_prefetch_desc(&tmK);
     tma_prefetch_desc(&tmV);
+    tma_prefetch_desc(&tmQ);
   }
   __syncthreads();
 
-  const __nv_bfloat16* Q = static_cast<const __nv_bfloat16*>(a.Q);
   __nv_bfloat16* Out = static_cast<__nv_bfloat16*>(a.O);
+  auto slot_q = [&](int sl) { return slots + sl * C::SLOT; };
+  auto slot_tiles = [&](int sl) { return reinterpret_cast<int32_t*>(slots + sl * C::SLOT + C::QBYTES); };
+  auto slot_meta = [&](int sl) {
+    return reinterpret_cast<ItemMeta*>(slots + sl * C::SLOT + C::QBYTES + C::MAXT * 4);
+  };
 
-  if (warp == 4) {
+  if (warp == 8) {
     // ------------------------------------------------------------ producer
     uint32_t cnt = 0;
     bool ok = true;
-    for (int64_t u = blockIdx.x; u < a.n_items && ok; u += gridDim.x) {
+    int local = 0;
+    auto sel_ptr = [&](int64_t u) {
       const int i = static_cast<int>(u % a.n_q);
       const int64_t bg = u / a.n_q;
       const int g = static_cast<int>(bg % a.h_kv);
       const int64_t b = bg / a.h_kv;
-      const int32_t* sel = a.idx + ((b * a.n_q + i) * a.h_kv + g) * a.topk;
-      const ItemTiles it = item_tiles(sel, a.topk, a.q_offset + i, a.nb, a.block, a.window);
-      if (lane == 0 && a.bad && it.n_bad) atomicAdd(a.bad, it.n_bad);
-      for (int j = 0; j < it.n_sub; ++j) {
-        bool wt;
-        const int64_t key0 = tile_key0(it, j, a.block, wt);
-        if (lane == 0) {
-          const int s = cnt % C::NS;
-          ok = mbar_wait(&empty[s], ((cnt / C::NS) & 1) ^ 1, a.err, SITE_ATTN_PRODUCER);
-          if (ok) {
-            uint8_t* st = stages + s * C::STAGE;
-            mbar_arrive_expect_tx(&full[s], C::STAGE);
-            const int z = static_cast<int>(b * a.n_kv + key0);
-#pragma unroll
-            for (int hf = 0; hf < D / 64; ++hf) {
-              tma_load_3d(st + hf * C::HALF, &tmK, &full[s], hf * 64, g, z);
-              tma_load_3d(st + C::KBYTES + hf * C::HALF, &tmV, &full[s], hf * 64, g, z);
-            }
-          }
-        }
-        ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
-        if (!ok) break;
-        ++cnt;
+      return a.idx + ((b * a.n_q + i) * a.h_kv + g) * a.topk;
+    };
+    int vnext = (static_cast<int64_t>(blockIdx.x) < a.n_items && lane < a.topk) ? __ldg(sel_ptr(blockIdx.x) + lane) : -1;
+    for (int64_t u = blockIdx.x; u < a.n_items && ok; u += gridDim.x, ++local) {
+      const int v = vnext;
+      const int64_t un = u + gridDim.x;
+      vnext = (un < a.n_items && lane < a.topk) ? __ldg(sel_ptr(un) + lane) : -1;   // prefetch
+      const int i = static_cast<int>(u % a.n_q);
+      const int64_t bg = u / a.n_q;
+      const int g = static_cast<int>(bg % a.h_kv);
+      const int64_t b = bg / a.h_kv;
+      const ItemTiles it = item_tiles_v(v, a.topk, a.q_offset + i, a.nb, a.block, a.window);
+      const int sl = local & 1;
+      if (lane == 0) ok = mbar_wait(&item_empty[sl], ((local >> 1) & 1) ^ 1, a.err, SITE_ATTN_PRODUCER);
+      ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
+      if (!ok) break;
+      int32_t* tl = slot_tiles(sl);
+      for (int j0 = 0; j0 < it.n_sub; j0 += 32) {
+        const int j = j0 + lane;
+        const int64_t k0 = tile_key0_lane(it, j, a.block);
+        if (j < it.n_sub) tl[j] = static_cast<int32_t>(k0);
       }
+      if (lane == 0) {
+        ItemMeta* m = slot_meta(sl);
+        m->pos = it.pos;
+        m->lo = it.lo;
+        m->qrow = (b * a.n_q + i) * a.h_q + static_cast<int64_t>(g) * G;
+        m->n_sub = it.n_sub;
+        m->ns = it.n_sel * it.spb;
+        if (a.bad && it.n_bad) atomicAdd(a.bad, it.n_bad);
+      }
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive_expect_tx(&item_full[sl], G * D * 2);
+        const int qrow = static_cast<int>((b * a.n_q + i) * a.h_q + static_cast<int64_t>(g) * G);
+#pragma unroll
+        for (int hf = 0; hf < D / 64; ++hf) tma_load_2d(slot_q(sl) + hf * G * 128, &tmQ, &item_full[sl], hf * 64, qrow);
+        for (int j = 0; j < it.n_sub; ++j) {
+          const int s = cnt % C::NS;
+          if (!mbar_wait(&empty[s], ((cnt / C::NS) & 1) ^ 1, a.err, SITE_ATTN_PRODUCER)) { ok = false; break; }
+          uint8_t* st = stages + s * C::STAGE;
+          mbar_arrive_expect_tx(&full[s], C::STAGE);
+          const int z = static_cast<int>(b * a.n_kv + tl[j]);
+#pragma unroll
+          for (int hf = 0; hf < D / 64; ++hf) {
+            tma_load_3d(st + hf * C::HALF, &tmK, &full[s], hf * 64, g, z);
+            tma_load_3d(st + C::KBYTES + hf * C::HALF, &tmV, &full[s], hf * 64, g, z);
+          }
+          ++cnt;
+        }
+      }
+      cnt = __shfl_sync(0xFFFFFFFFu, cnt, 0);
+      ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
     }
-    if (!ok && lane == 0) {
+    if (!ok && lane == 0) {   // let copies already issued land before the CTA exits
       for (uint32_t n = (cnt > C::NS ? cnt - C::NS : 0); n < cnt; ++n) {
         const uint64_t t0 = global_timer_ns();
         while (!mbar_try_wait(&full[n % C::NS], (n / C::NS) & 1))
@@ -131,153 +188,191 @@ __global__ void __launch_bounds__(160, 1)
     // ------------------------------------------------------------ consumers
     const int gq = lane >> 2, tq = lane & 3;   // fragment row group / column pair
     uint32_t cnt = 0;
-    bool ok = true;
-    for (int64_t u = blockIdx.x; u < a.n_items && ok; u += gridDim.x) {
-      const int i = static_cast<int>(u % a.n_q);
-      const int64_t bg = u / a.n_q;
-      const int g = static_cast<int>(bg % a.h_kv);
-      const int64_t b = bg / a.h_kv;
-      const int32_t* sel = a.idx + ((b * a.n_q + i) * a.h_kv + g) * a.topk;
-      const ItemTiles it = item_tiles(sel, a.topk, a.q_offset + i, a.nb, a.block, a.window);
-      const int64_t qrow = (b * a.n_q + i) * a.h_q + static_cast<int64_t>(g) * G;
-
-      // Q^T as the n8 operand: (dims 2t..2t+1 (+8), head gq), zero for gq >= G
-      uint32_t qf[KS][2];
-#pragma unroll
-      for (int ks = 0; ks < KS; ++ks) {
-        if (gq < G) {
-          const uint32_t* qp = reinterpret_cast<const uint32_t*>(Q + (qrow + gq) * D + ks * 16 + 2 * tq);
-          qf[ks][0] = __ldg(qp);
-          qf[ks][1] = __ldg(qp + 4);
-        } else {
-          qf[ks][0] = 0u;
-          qf[ks][1] = 0u;
-        }
-      }
+    int local = 0;
+    const int wq = warp & 3, grp = warp >> 2;
+    const int krow = wq * 16;                  // this warp's 16 keys of each of its tiles
+    for (int64_t u = blockIdx.x; u < a.n_items; u += gridDim.x, ++local) {
+      const int sl = local & 1;
+      bool ok = __all_sync(0xFFFFFFFFu, mbar_wait(&item_full[sl], (local >> 1) & 1, a.err, SITE_ATTN_CONSUMER));
       float m_run[2] = {-INFINITY, -INFINITY}, l_run[2] = {0.f, 0.f};
       float oacc[MT][4];
 #pragma unroll
       for (int mm = 0; mm < MT; ++mm)
 #pragma unroll
         for (int r = 0; r < 4; ++r) oacc[mm][r] = 0.f;
-
-      for (int j = warp; j < it.n_sub; j += 4) {
-        bool wt;
-        const int64_t key0 = tile_key0(it, j, a.block, wt);
-        const uint32_t n = cnt + j;
-        const int s = n % C::NS;
-        ok = __all_sync(0xFFFFFFFFu, mbar_wait(&full[s], (n / C::NS) & 1, a.err, SITE_ATTN_CONSUMER));
-        if (!ok) break;
-        const uint32_t kb = smem_u32(stages + s * C::STAGE);
-        const uint32_t vb = kb + C::KBYTES;
-
-        // S^T = K Q^T for 4 tiles of 16 keys
-        float sacc[4][4];
+      ItemMeta meta{};
+      if (ok) {
+        meta = *slot_meta(sl);
+        const int32_t* tl = slot_tiles(sl);
+        // Q^T as the n8 operand: (dims 2t..2t+1 (+8), head gq), zero for gq >= G
+        uint32_t qf[KS][2];
+        const uint8_t* qs = slot_q(sl);
 #pragma unroll
-        for (int m = 0; m < 4; ++m) {
-#pragma unroll
-          for (int r = 0; r < 4; ++r) sacc[m][r] = 0.f;
-          const int row = m * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
-#pragma unroll
-          for (int ks = 0; ks < KS; ++ks) {
-            const int chunk = (ks & 3) * 2 + (lane >> 4);
-            const uint32_t addr = kb + (ks >> 2) * C::HALF + row * 128 + ((chunk ^ (row & 7)) << 4);
-            uint32_t af[4];
-            ldmatrix_x4(af, addr);
-            mma_16816(sacc[m], af, qf[ks][0], qf[ks][1]);
+        for (int ks = 0; ks < KS; ++ks) {
+          if (gq < G) {
+            const uint32_t* qp = reinterpret_cast<const uint32_t*>(
+                qs + (ks >> 2) * G * 128 + gq * 128 + ((ks & 3) * 16 + 2 * tq) * 2);
+            qf[ks][0] = qp[0];
+            qf[ks][1] = qp[4];
+          } else {
+            qf[ks][0] = 0u;
+            qf[ks][1] = 0u;
           }
         }
-        // scale, mask, running max per head (heads 2tq, 2tq+1)
-        float mx[2] = {-INFINITY, -INFINITY};
+        for (int j = grp; j < meta.n_sub; j += 2) {
+          const uint32_t n = cnt + j;
+          const int s = n % C::NS;
+          ok = __all_sync(0xFFFFFFFFu, mbar_wait(&full[s], (n / C::NS) & 1, a.err, SITE_ATTN_CONSUMER));
+          if (!ok) break;
+          const int64_t key0 = tl[j];
+          const bool wt = j >= meta.ns;
+          const uint32_t kb = smem_u32(stages + s * C::STAGE);
+          const uint32_t vb = kb + C::KBYTES;
+
+          // S^T = K Q^T for this warp's 16 keys (two independent accumulators)
+          float sacc[4] = {0.f, 0.f, 0.f, 0.f};
+          {
+            float sacc2[4] = {0.f, 0.f, 0.f, 0.f};
+            const int row = krow + (lane & 7) + ((lane >> 3) & 1) * 8;
 #pragma unroll
-        for (int m = 0; m < 4; ++m) {
+            for (int ks = 0; ks < KS; ++ks) {
+              const int chunk = (ks & 3) * 2 + (lane >> 4);
+              const uint32_t addr = kb + (ks >> 2) * C::HALF + row * 128 + ((chunk ^ (row & 7)) << 4);
+              uint32_t af[4];
+              ldmatrix_x4(af, addr);
+              if (ks & 1)
+                mma_16816(sacc2, af, qf[ks][0], qf[ks][1]);
+              else
+                mma_16816(sacc, af, qf[ks][0], qf[ks][1]);
+            }
+#pragma unroll
+            for (int r = 0; r < 4; ++r) sacc[r] += sacc2[r];
+          }
+          // scale, mask, running max per head (heads 2tq, 2tq+1)
+          float mx[2] = {-INFINITY, -INFINITY};
 #pragma unroll
           for (int r = 0; r < 4; ++r) {
-            const int64_t key = key0 + m * 16 + gq + (r >= 2 ? 8 : 0);
-            const bool in = !wt || (key >= it.lo && key <= it.pos);
-            const float sv = in ? sacc[m][r] * a.scale_log2 : -INFINITY;
-            sacc[m][r] = sv;
+            const int64_t key = key0 + krow + gq + (r >= 2 ? 8 : 0);
+            const bool in = !wt || (key >= meta.lo && key <= meta.pos);
+            const float sv = in ? sacc[r] * a.scale_log2 : -INFINITY;
+            sacc[r] = sv;
             mx[r & 1] = fmaxf(mx[r & 1], sv);
           }
-        }
-        float alpha[2];
+          bool grow = false;
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          mx[h] = fmaxf(mx[h], __shfl_xor_sync(0xFFFFFFFFu, mx[h], 4));
-          mx[h] = fmaxf(mx[h], __shfl_xor_sync(0xFFFFFFFFu, mx[h], 8));
-          mx[h] = fmaxf(mx[h], __shfl_xor_sync(0xFFFFFFFFu, mx[h], 16));
-          const float mnew = fmaxf(m_run[h], mx[h]);
-          alpha[h] = (mnew == -INFINITY) ? 1.f : fast_exp2(m_run[h] - mnew);
-          m_run[h] = mnew;
-        }
-        uint32_t pb[4][2];
+          for (int h = 0; h < 2; ++h) {
+            mx[h] = fmaxf(mx[h], __shfl_xor_sync(0xFFFFFFFFu, mx[h], 4));
+            mx[h] = fmaxf(mx[h], __shfl_xor_sync(0xFFFFFFFFu, mx[h], 8));
+            mx[h] = fmaxf(mx[h], __shfl_xor_sync(0xFFFFFFFFu, mx[h], 16));
+            grow |= mx[h] > m_run[h];
+          }
+          // rescale only when some head's running max rose (exact either way)
+          if (__any_sync(0xFFFFFFFFu, grow)) {
+            float alpha[2];
 #pragma unroll
-        for (int m = 0; m < 4; ++m) {
+            for (int h = 0; h < 2; ++h) {
+              const float mnew = fmaxf(m_run[h], mx[h]);
+              alpha[h] = (m_run[h] == -INFINITY) ? 0.f : fast_exp2(m_run[h] - mnew);
+              m_run[h] = mnew;
+              l_run[h] *= alpha[h];
+            }
+#pragma unroll
+            for (int mm = 0; mm < MT; ++mm) {
+              oacc[mm][0] *= alpha[0];
+              oacc[mm][1] *= alpha[1];
+              oacc[mm][2] *= alpha[0];
+              oacc[mm][3] *= alpha[1];
+            }
+          }
           float p[4];
 #pragma unroll
-          for (int r = 0; r < 4; ++r) {
-            const float mr = m_run[r & 1];
-            p[r] = (mr == -INFINITY) ? 0.f : fast_exp2(sacc[m][r] - mr);
+          for (int r = 0; r < 4; ++r) p[r] = (sacc[r] == -INFINITY) ? 0.f : fast_exp2(sacc[r] - m_run[r & 1]);
+          l_run[0] += p[0] + p[2];
+          l_run[1] += p[1] + p[3];
+          const uint32_t pb0 = movmatrix_trans(pack_bf16(p[0], p[1]));
+          const uint32_t pb1 = movmatrix_trans(pack_bf16(p[2], p[3]));
+          // O^T += V^T P^T over this warp's 16 keys
+          {
+            const int mi = lane >> 3;
+            const int row = krow + (lane & 7) + (mi >> 1) * 8;
+#pragma unroll
+            for (int mm = 0; mm < MT; ++mm) {
+              const int dchunk = mm * 2 + (mi & 1);
+              const uint32_t addr = vb + (dchunk >> 3) * C::HALF + row * 128 + (((dchunk & 7) ^ (row & 7)) << 4);
+              uint32_t af[4];
+              ldmatrix_x4_trans(af, addr);
+              mma_16816(oacc[mm], af, pb0, pb1);
+            }
           }
-          l_run[0] = l_run[0] * (m == 0 ? alpha[0] : 1.f) + p[0] + p[2];
-          l_run[1] = l_run[1] * (m == 0 ? alpha[1] : 1.f) + p[1] + p[3];
-          pb[m][0] = movmatrix_trans(pack_bf16(p[0], p[1]));
-          pb[m][1] = movmatrix_trans(pack_bf16(p[2], p[3]));
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&empty[s]);
         }
-#pragma unroll
-        for (int mm = 0; mm < MT; ++mm) {
-          oacc[mm][0] *= alpha[0];
-          oacc[mm][1] *= alpha[1];
-          oacc[mm][2] *= alpha[0];
-          oacc[mm][3] *= alpha[1];
-        }
-        // O^T += V^T P^T
-#pragma unroll
-        for (int m = 0; m < 4; ++m) {
-          const int mi = lane >> 3;
-          const int row = m * 16 + (lane & 7) + (mi >> 1) * 8;
-#pragma unroll
-          for (int mm = 0; mm < MT; ++mm) {
-            const int dchunk = mm * 2 + (mi & 1);
-            const uint32_t addr = vb + (dchunk >> 3) * C::HALF + row * 128 + (((dchunk & 7) ^ (row & 7)) << 4);
-            uint32_t af[4];
-            ldmatrix_x4_trans(af, addr);
-            mma_16816(oacc[mm], af, pb[m][0], pb[m][1]);
-          }
-        }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&empty[s]);
+        cnt += meta.n_sub;
       }
-      cnt += it.n_sub;
 
-      // per-warp partials -> shared memory
+      // per-warp partials; all eight consumer warps meet here every item
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
         l_run[h] += __shfl_xor_sync(0xFFFFFFFFu, l_run[h], 4);
         l_run[h] += __shfl_xor_sync(0xFFFFFFFFu, l_run[h], 8);
         l_run[h] += __shfl_xor_sync(0xFFFFFFFFu, l_run[h], 16);
       }
-      float* myO = mO + warp * 8 * D;
-#pragma unroll
-      for (int mm = 0; mm < MT; ++mm) {
-        const int d0 = mm * 16 + gq;
-        myO[(2 * tq) * D + d0] = oacc[mm][0];
-        myO[(2 * tq + 1) * D + d0] = oacc[mm][1];
-        myO[(2 * tq) * D + d0 + 8] = oacc[mm][2];
-        myO[(2 * tq + 1) * D + d0 + 8] = oacc[mm][3];
-      }
       if (lane == 0) abort_flag[warp] = ok ? 0 : 1;
-      if (gq == 0) {
-        mM[warp * 8 + 2 * tq] = m_run[0];
-        mM[warp * 8 + 2 * tq + 1] = m_run[1];
-        mL[warp * 8 + 2 * tq] = l_run[0];
-        mL[warp * 8 + 2 * tq + 1] = l_run[1];
+      float* myO = mO + wq * 8 * D;
+      // group 1 hands its partials to the group-0 warp with the same key slice
+      if (grp == 1) {
+#pragma unroll
+        for (int mm = 0; mm < MT; ++mm) {
+          const int d0 = mm * 16 + gq;
+          myO[(2 * tq) * D + d0] = oacc[mm][0];
+          myO[(2 * tq + 1) * D + d0] = oacc[mm][1];
+          myO[(2 * tq) * D + d0 + 8] = oacc[mm][2];
+          myO[(2 * tq + 1) * D + d0 + 8] = oacc[mm][3];
+        }
+        if (gq == 0) {
+          mM[wq * 8 + 2 * tq] = m_run[0];
+          mM[wq * 8 + 2 * tq + 1] = m_run[1];
+          mL[wq * 8 + 2 * tq] = l_run[0];
+          mL[wq * 8 + 2 * tq + 1] = l_run[1];
+        }
       }
       named_bar_consumers();
-      // every consumer warp reaches both barriers of an item, so a failed
-      // wait in one warp stops all four together after the first
-      const bool any_abort = (abort_flag[0] | abort_flag[1] | abort_flag[2] | abort_flag[3]) != 0;
-      for (int e = threadIdx.x; e < G * D && !any_abort; e += 128) {
+      if (grp == 0) {
+        float f0[2], f1[2];
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const float mo = mM[wq * 8 + 2 * tq + h], lo_ = mL[wq * 8 + 2 * tq + h];
+          const float M = fmaxf(m_run[h], mo);
+          f0[h] = (m_run[h] == -INFINITY) ? 0.f : fast_exp2(m_run[h] - M);
+          f1[h] = (mo == -INFINITY) ? 0.f : fast_exp2(mo - M);
+          l_run[h] = f0[h] * l_run[h] + f1[h] * lo_;
+          m_run[h] = M;
+        }
+#pragma unroll
+        for (int mm = 0; mm < MT; ++mm) {
+          const int d0 = mm * 16 + gq;
+          float* o0 = &myO[(2 * tq) * D + d0];
+          float* o1 = &myO[(2 * tq + 1) * D + d0];
+          o0[0] = f0[0] * oacc[mm][0] + f1[0] * o0[0];
+          o1[0] = f0[1] * oacc[mm][1] + f1[1] * o1[0];
+          o0[8] = f0[0] * oacc[mm][2] + f1[0] * o0[8];
+          o1[8] = f0[1] * oacc[mm][3] + f1[1] * o1[8];
+        }
+        __syncwarp();
+        if (gq == 0) {
+          mM[wq * 8 + 2 * tq] = m_run[0];
+          mM[wq * 8 + 2 * tq + 1] = m_run[1];
+          mL[wq * 8 + 2 * tq] = l_run[0];
+          mL[wq * 8 + 2 * tq + 1] = l_run[1];
+        }
+      }
+      named_bar_consumers();
+      // a failed wait in any warp stops all eight together
+      int ab = 0;
+#pragma unroll
+      for (int w = 0; w < 8; ++w) ab |= abort_flag[w];
+      const bool any_abort = ab != 0;
+      for (int e = threadIdx.x; e < G * D && !any_abort; e += 256) {
         const int h = e / D, dd = e % D;
         float M = -INFINITY;
 #pragma unroll
@@ -290,10 +385,11 @@ __global__ void __launch_bounds__(160, 1)
           num += f * mO[(w * 8 + h) * D + dd];
           den += f * mL[w * 8 + h];
         }
-        Out[(qrow + h) * D + dd] = __float2bfloat16_rn(num / den);
-        if (dd == 0 && a.lse) a.lse[qrow + h] = (M + log2f(den)) * 0.69314718055994531f;
+        Out[(meta.qrow + h) * D + dd] = __float2bfloat16_rn(num / den);
+        if (dd == 0 && a.lse) a.lse[meta.qrow + h] = (M + log2f(den)) * 0.69314718055994531f;
       }
       named_bar_consumers();
+      if (lane == 0) mbar_arrive(&item_empty[sl]);
       if (any_abort) break;
     }
   }
@@ -427,30 +523,30 @@ AttnArgs attn_args(const ssa_params& p, const void* Q, const void* K, const void
 
 template <int D, int G>
 cudaError_t run_bf16(const ssa_params& p, const CUtensorMap& tmK, const CUtensorMap& tmV,
-                     const AttnArgs& a, const LaunchCtx& c) {
+                     const CUtensorMap& tmQ, const AttnArgs& a, const LaunchCtx& c) {
   using C = AttnCfg<D>;
   cudaError_t e = cudaFuncSetAttribute(attn_bf16_kernel<D, G>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
   if (e != cudaSuccess) return e;
   int per_sm = 1;
-  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, attn_bf16_kernel<D, G>, 160, C::SMEM);
+  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, attn_bf16_kernel<D, G>, 288, C::SMEM);
   if (e != cudaSuccess) return e;
   if (per_sm < 1) per_sm = 1;
   int64_t grid = static_cast<int64_t>(per_sm) * c.sm_count;
   if (grid > a.n_items) grid = a.n_items;
-  attn_bf16_kernel<D, G><<<static_cast<unsigned>(grid), 160, C::SMEM, c.stream>>>(tmK, tmV, a);
+  attn_bf16_kernel<D, G><<<static_cast<unsigned>(grid), 288, C::SMEM, c.stream>>>(tmK, tmV, tmQ, a);
   note_launch();
   return cudaGetLastError();
 }
 
 template <int D>
 cudaError_t bf16_g(const ssa_params& p, const CUtensorMap& tmK, const CUtensorMap& tmV,
-                   const AttnArgs& a, const LaunchCtx& c) {
+                   const CUtensorMap& tmQ, const AttnArgs& a, const LaunchCtx& c) {
   switch (p.h_q / p.h_kv) {
-    case 1: return run_bf16<D, 1>(p, tmK, tmV, a, c);
-    case 2: return run_bf16<D, 2>(p, tmK, tmV, a, c);
-    case 4: return run_bf16<D, 4>(p, tmK, tmV, a, c);
-    case 8: return run_bf16<D, 8>(p, tmK, tmV, a, c);
+    case 1: return run_bf16<D, 1>(p, tmK, tmV, tmQ, a, c);
+    case 2: return run_bf16<D, 2>(p, tmK, tmV, tmQ, a, c);
+    case 4: return run_bf16<D, 4>(p, tmK, tmV, tmQ, a, c);
+    case 8: return run_bf16<D, 8>(p, tmK, tmV, tmQ, a, c);
   }
   return cudaErrorInvalidValue;
 }
@@ -482,11 +578,11 @@ cudaError_t f32_g(const ssa_params& p, const AttnArgs& a, const LaunchCtx& c) {
 int attn_bf16_smem_bytes(int d) { return d == 128 ? AttnCfg<128>::SMEM : AttnCfg<64>::SMEM; }
 
 cudaError_t launch_attn_bf16(const ssa_params& p, const CUtensorMap& tmK, const CUtensorMap& tmV,
-                             const void* Q, const int32_t* block_idx, void* O, float* lse,
-                             int32_t* bad, const LaunchCtx& c) {
+                             const CUtensorMap& tmQ, const void* Q, const int32_t* block_idx, void* O,
+                             float* lse, int32_t* bad, const LaunchCtx& c) {
   const AttnArgs a = attn_args(p, Q, nullptr, nullptr, block_idx, O, lse, bad, c.err);
-  if (p.d == 128) return bf16_g<128>(p, tmK, tmV, a, c);
-  if (p.d == 64) return bf16_g<64>(p, tmK, tmV, a, c);
+  if (p.d == 128) return bf16_g<128>(p, tmK, tmV, tmQ, a, c);
+  if (p.d == 64) return bf16_g<64>(p, tmK, tmV, tmQ, a, c);
   return cudaErrorInvalidValue;
 }
 

@@ -42,8 +42,8 @@ cudaError_t launch_route_rowwise_f32(const ssa_params& p, const void* Q, const f
 
 // steps (ii)+(iii): TMA tile-gather attention, bf16
 cudaError_t launch_attn_bf16(const ssa_params& p, const CUtensorMap& tmK, const CUtensorMap& tmV,
-                             const void* Q, const int32_t* block_idx, void* O, float* lse,
-                             int32_t* bad, const LaunchCtx& c);
+                             const CUtensorMap& tmQ, const void* Q, const int32_t* block_idx, void* O,
+                             float* lse, int32_t* bad, const LaunchCtx& c);
 
 // steps (ii)+(iii): float32 attention
 cudaError_t launch_attn_f32(const ssa_params& p, const void* Q, const void* K, const void* V,

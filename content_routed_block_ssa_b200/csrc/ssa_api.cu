@@ -157,6 +157,19 @@ bool encode_2d(CUtensorMap* m, const void* base, uint64_t cols, uint64_t rows, u
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// 2D bf16 map of a [rows, cols] row-major matrix, unswizzled boxes of 64 x box_rows.
+bool encode_rows(CUtensorMap* m, const void* base, uint64_t cols, uint64_t rows, uint32_t box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[2] = {cols, rows};
+  const cuuint64_t strides[1] = {cols * 2};
+  const cuuint32_t box[2] = {64, box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // 3D bf16 map of K or V viewed as [b*n_kv, h_kv, d]; boxes of 64 keys x 1 head x 64 dims.
 bool encode_kv(CUtensorMap* m, const void* base, const ssa_params& p) {
   EncodeTiledFn fn = encode_fn();
@@ -206,9 +219,12 @@ ssa_status do_attn(const ssa_params& p, const void* Q, const void* K, const void
                    const int32_t* idx, void* O, float* lse, int32_t* bad, const LaunchCtx& c) {
   if (is_empty(p)) return SSA_OK;
   if (p.dtype == SSA_F32) return from_cuda(ssa::launch_attn_f32(p, Q, K, V, idx, O, lse, bad, c));
-  CUtensorMap tmK, tmV;
-  if (!encode_kv(&tmK, K, p) || !encode_kv(&tmV, V, p)) return SSA_ERR_CUDA;
-  return from_cuda(ssa::launch_attn_bf16(p, tmK, tmV, Q, idx, O, lse, bad, c));
+  CUtensorMap tmK, tmV, tmQ;
+  const uint32_t G = static_cast<uint32_t>(p.h_q / p.h_kv);
+  if (!encode_kv(&tmK, K, p) || !encode_kv(&tmV, V, p) ||
+      !encode_rows(&tmQ, Q, p.d, static_cast<uint64_t>(p.batch) * p.n_q * p.h_q, G))
+    return SSA_ERR_CUDA;
+  return from_cuda(ssa::launch_attn_bf16(p, tmK, tmV, tmQ, Q, idx, O, lse, bad, c));
 }
 
 struct ForwardLayout {

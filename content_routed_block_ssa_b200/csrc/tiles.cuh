@@ -28,14 +28,13 @@ struct ItemTiles {
   int n_bad;          // block_idx entries skipped as invalid
 };
 
-// sel: the item's block_idx row (topk entries).
-__device__ __forceinline__ ItemTiles item_tiles(const int32_t* __restrict__ sel, int topk,
-                                                int64_t pos, int nb, int block, int window) {
+// v: this lane's entry of the item's block_idx row (-1 for lanes >= topk).
+__device__ __forceinline__ ItemTiles item_tiles_v(int v, int topk, int64_t pos, int nb, int block,
+                                                  int window) {
   const int lane = threadIdx.x & 31;
   ItemTiles it;
   it.pos = pos;
   const int nvis = static_cast<int>(min(static_cast<int64_t>(nb), (pos + 1) / block));
-  const int v = lane < topk ? __ldg(sel + lane) : -1;
   const bool inrange = v >= 0 && v < nvis;
   // strictly ascending among the in-range entries: compare with the running
   // maximum of the in-range entries on lower lanes
@@ -67,6 +66,14 @@ __device__ __forceinline__ ItemTiles item_tiles(const int32_t* __restrict__ sel,
   return it;
 }
 
+// sel: the item's block_idx row (topk entries).
+__device__ __forceinline__ ItemTiles item_tiles(const int32_t* __restrict__ sel, int topk,
+                                                int64_t pos, int nb, int block, int window) {
+  const int lane = threadIdx.x & 31;
+  const int v = lane < topk ? __ldg(sel + lane) : -1;
+  return item_tiles_v(v, topk, pos, nb, block, window);
+}
+
 // n-th set bit (0-based) of a 32-bit mask.
 __device__ __forceinline__ int nth_bit32(uint32_t m, int n) {
   for (int k = 0; k < n; ++k) m &= m - 1;
@@ -77,6 +84,19 @@ __device__ __forceinline__ int nth_bit32(uint32_t m, int n) {
 __device__ __forceinline__ int nth_bit64(uint64_t m, int n) {
   for (int k = 0; k < n; ++k) m &= m - 1;
   return __ffsll(static_cast<long long>(m)) - 1;
+}
+
+// First key of tile j, computed by each lane for its own j (any j per lane;
+// every lane must call).  Tiles j < n_sel*spb are selected-block tiles.
+__device__ __forceinline__ int64_t tile_key0_lane(const ItemTiles& it, int j, int block) {
+  const int ns = it.n_sel * it.spb;
+  const int which = (j < ns) ? j / it.spb : 0;
+  int src = (j < ns) ? nth_bit32(it.selmask, which) : 0;
+  src = src < 0 ? 0 : src;
+  const int blk = __shfl_sync(0xFFFFFFFFu, it.my_blk, src);
+  if (j < ns) return static_cast<int64_t>(blk) * block + (j % it.spb) * 64;
+  const int wbit = nth_bit64(it.winmask, j - ns);
+  return (it.win_t0 + (wbit < 0 ? 0 : wbit)) * 64;
 }
 
 // Tile j of the list: first key and whether it is a (masked) window tile.
