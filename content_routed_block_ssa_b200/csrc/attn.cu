@@ -54,8 +54,9 @@ struct AttnCfg {
   static constexpr int QBYTES = 8 * D * 2;
   static constexpr int SLOT = 4096;
   static constexpr int MERGE = 4 * 8 * D * 4 + 4 * 8 * 2 * 4;
-  static constexpr int NBAR = 2 * NS + 4;
-  static constexpr int SMEM = 1024 + NS * STAGE + 2 * SLOT + MERGE + NBAR * 8 + 32;
+  static constexpr int NSLOT = 3;
+  static constexpr int NBAR = 2 * NS + 2 * NSLOT;
+  static constexpr int SMEM = 1024 + NS * STAGE + NSLOT * SLOT + MERGE + NBAR * 8 + 32;
   static_assert(QBYTES + MAXT * 4 + 64 <= SLOT, "item slot too small");
 };
 
@@ -85,20 +86,20 @@ __global__ void __launch_bounds__(288, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* stages = smem;
-  uint8_t* slots = stages + C::NS * C::STAGE;                        // 2 item slots
-  float* mO = reinterpret_cast<float*>(slots + 2 * C::SLOT);          // [4][8][D]
+  uint8_t* slots = stages + C::NS * C::STAGE;                        // item slots
+  float* mO = reinterpret_cast<float*>(slots + C::NSLOT * C::SLOT);   // [4][8][D]
   float* mM = mO + 4 * 8 * D;                                         // [4][8]
   float* mL = mM + 4 * 8;                                             // [4][8]
   uint64_t* full = reinterpret_cast<uint64_t*>(mL + 4 * 8);
   uint64_t* empty = full + C::NS;
   uint64_t* item_full = empty + C::NS;
-  uint64_t* item_empty = item_full + 2;
-  int* abort_flag = reinterpret_cast<int*>(item_empty + 2);          // [8]
+  uint64_t* item_empty = item_full + C::NSLOT;
+  int* abort_flag = reinterpret_cast<int*>(item_empty + C::NSLOT);   // [8]
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::NS; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 4); }
-    for (int s = 0; s < 2; ++s) { mbar_init(&item_full[s], 1); mbar_init(&item_empty[s], 8); }
+    for (int s = 0; s < C::NSLOT; ++s) { mbar_init(&item_full[s], 1); mbar_init(&item_empty[s], 8); }
     fence_barrier_init();
     tma_prefetch_desc(&tmK);
     tma_prefetch_desc(&tmV);
@@ -115,9 +116,10 @@ __global__ void __launch_bounds__(288, 1)
 
   if (warp == 8) {
     // ------------------------------------------------------------ producer
+    // Item setup (tile list + Q) runs one item ahead of the tile gathers, so
+    // the consumers find the next item ready when they finish the current one.
     uint32_t cnt = 0;
     bool ok = true;
-    int local = 0;
     auto sel_ptr = [&](int64_t u) {
       const int i = static_cast<int>(u % a.n_q);
       const int64_t bg = u / a.n_q;
@@ -125,20 +127,19 @@ __global__ void __launch_bounds__(288, 1)
       const int64_t b = bg / a.h_kv;
       return a.idx + ((b * a.n_q + i) * a.h_kv + g) * a.topk;
     };
-    int vnext = (static_cast<int64_t>(blockIdx.x) < a.n_items && lane < a.topk) ? __ldg(sel_ptr(blockIdx.x) + lane) : -1;
-    for (int64_t u = blockIdx.x; u < a.n_items && ok; u += gridDim.x, ++local) {
-      const int v = vnext;
-      const int64_t un = u + gridDim.x;
-      vnext = (un < a.n_items && lane < a.topk) ? __ldg(sel_ptr(un) + lane) : -1;   // prefetch
+    // set up item number `local` (u = blockIdx.x + local * gridDim.x) in slot local % NSLOT
+    auto setup = [&](int local, int v) -> bool {
+      const int64_t u = blockIdx.x + static_cast<int64_t>(local) * gridDim.x;
       const int i = static_cast<int>(u % a.n_q);
       const int64_t bg = u / a.n_q;
       const int g = static_cast<int>(bg % a.h_kv);
       const int64_t b = bg / a.h_kv;
       const ItemTiles it = item_tiles_v(v, a.topk, a.q_offset + i, a.nb, a.block, a.window);
-      const int sl = local & 1;
-      if (lane == 0) ok = mbar_wait(&item_empty[sl], ((local >> 1) & 1) ^ 1, a.err, SITE_ATTN_PRODUCER);
-      ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
-      if (!ok) break;
+      const int sl = local % C::NSLOT;
+      bool w_ok = true;
+      if (lane == 0) w_ok = mbar_wait(&item_empty[sl], ((local / C::NSLOT) & 1) ^ 1, a.err, SITE_ATTN_PRODUCER);
+      w_ok = __shfl_sync(0xFFFFFFFFu, w_ok, 0);
+      if (!w_ok) return false;
       int32_t* tl = slot_tiles(sl);
       for (int j0 = 0; j0 < it.n_sub; j0 += 32) {
         const int j = j0 + lane;
@@ -160,7 +161,32 @@ __global__ void __launch_bounds__(288, 1)
         const int qrow = static_cast<int>((b * a.n_q + i) * a.h_q + static_cast<int64_t>(g) * G);
 #pragma unroll
         for (int hf = 0; hf < D / 64; ++hf) tma_load_2d(slot_q(sl) + hf * G * 128, &tmQ, &item_full[sl], hf * 64, qrow);
-        for (int j = 0; j < it.n_sub; ++j) {
+      }
+      return true;
+    };
+    const int n_local = static_cast<int>((a.n_items - blockIdx.x + gridDim.x - 1) / gridDim.x);
+    int vnext = (n_local > 1 && lane < a.topk) ? __ldg(sel_ptr(blockIdx.x + gridDim.x) + lane) : -1;
+    if (n_local > 0) {
+      const int v0 = lane < a.topk ? __ldg(sel_ptr(blockIdx.x) + lane) : -1;
+      ok = setup(0, v0);
+    }
+    for (int local = 0; local < n_local && ok; ++local) {
+      if (local + 1 < n_local) {
+        const int v = vnext;
+        vnext = (local + 2 < n_local && lane < a.topk)
+                    ? __ldg(sel_ptr(blockIdx.x + static_cast<int64_t>(local + 2) * gridDim.x) + lane) : -1;
+        ok = setup(local + 1, v);
+        if (!ok) break;
+      }
+      const int64_t u = blockIdx.x + static_cast<int64_t>(local) * gridDim.x;
+      const int64_t bg = u / a.n_q;
+      const int g = static_cast<int>(bg % a.h_kv);
+      const int64_t b = bg / a.h_kv;
+      const int sl = local % C::NSLOT;
+      const int32_t* tl = slot_tiles(sl);
+      const int n_sub = slot_meta(sl)->n_sub;
+      if (lane == 0) {
+        for (int j = 0; j < n_sub; ++j) {
           const int s = cnt % C::NS;
           if (!mbar_wait(&empty[s], ((cnt / C::NS) & 1) ^ 1, a.err, SITE_ATTN_PRODUCER)) { ok = false; break; }
           uint8_t* st = stages + s * C::STAGE;
@@ -192,8 +218,8 @@ __global__ void __launch_bounds__(288, 1)
     const int wq = warp & 3, grp = warp >> 2;
     const int krow = wq * 16;                  // this warp's 16 keys of each of its tiles
     for (int64_t u = blockIdx.x; u < a.n_items; u += gridDim.x, ++local) {
-      const int sl = local & 1;
-      bool ok = __all_sync(0xFFFFFFFFu, mbar_wait(&item_full[sl], (local >> 1) & 1, a.err, SITE_ATTN_CONSUMER));
+      const int sl = local % C::NSLOT;
+      bool ok = __all_sync(0xFFFFFFFFu, mbar_wait(&item_full[sl], (local / C::NSLOT) & 1, a.err, SITE_ATTN_CONSUMER));
       float m_run[2] = {-INFINITY, -INFINITY}, l_run[2] = {0.f, 0.f};
       float oacc[MT][4];
 #pragma unroll
@@ -224,40 +250,60 @@ __global__ void __launch_bounds__(288, 1)
           const int s = n % C::NS;
           ok = __all_sync(0xFFFFFFFFu, mbar_wait(&full[s], (n / C::NS) & 1, a.err, SITE_ATTN_CONSUMER));
           if (!ok) break;
-          const int64_t key0 = tl[j];
+          const int key0 = tl[j];
           const bool wt = j >= meta.ns;
           const uint32_t kb = smem_u32(stages + s * C::STAGE);
           const uint32_t vb = kb + C::KBYTES;
-
-          // S^T = K Q^T for this warp's 16 keys (two independent accumulators)
-          float sacc[4] = {0.f, 0.f, 0.f, 0.f};
+          // copy this warp's 16-key slice of K and V into registers and give
+          // the stage back at once, so the ring refills while we compute
+          uint32_t kf[KS][4], vf[MT][4];
           {
-            float sacc2[4] = {0.f, 0.f, 0.f, 0.f};
             const int row = krow + (lane & 7) + ((lane >> 3) & 1) * 8;
 #pragma unroll
             for (int ks = 0; ks < KS; ++ks) {
               const int chunk = (ks & 3) * 2 + (lane >> 4);
-              const uint32_t addr = kb + (ks >> 2) * C::HALF + row * 128 + ((chunk ^ (row & 7)) << 4);
-              uint32_t af[4];
-              ldmatrix_x4(af, addr);
-              if (ks & 1)
-                mma_16816(sacc2, af, qf[ks][0], qf[ks][1]);
-              else
-                mma_16816(sacc, af, qf[ks][0], qf[ks][1]);
+              ldmatrix_x4(kf[ks], kb + (ks >> 2) * C::HALF + row * 128 + ((chunk ^ (row & 7)) << 4));
             }
+            const int mi = lane >> 3;
+            const int vrow = krow + (lane & 7) + (mi >> 1) * 8;
 #pragma unroll
-            for (int r = 0; r < 4; ++r) sacc[r] += sacc2[r];
+            for (int mm = 0; mm < MT; ++mm) {
+              const int dchunk = mm * 2 + (mi & 1);
+              ldmatrix_x4_trans(vf[mm], vb + (dchunk >> 3) * C::HALF + vrow * 128 + (((dchunk & 7) ^ (vrow & 7)) << 4));
+            }
           }
-          // scale, mask, running max per head (heads 2tq, 2tq+1)
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&empty[s]);
+
+          // S^T = K Q^T for this warp's 16 keys (two independent accumulators)
+          float sacc[4];
+          {
+            float part[4][4];
+#pragma unroll
+            for (int c = 0; c < 4; ++c)
+#pragma unroll
+              for (int r = 0; r < 4; ++r) part[c][r] = 0.f;
+#pragma unroll
+            for (int ks = 0; ks < KS; ++ks) mma_16816(part[ks & 3], kf[ks], qf[ks][0], qf[ks][1]);
+#pragma unroll
+            for (int r = 0; r < 4; ++r) sacc[r] = (part[0][r] + part[1][r]) + (part[2][r] + part[3][r]);
+          }
+          // scale, mask (window tiles only), running max per head (heads 2tq, 2tq+1)
           float mx[2] = {-INFINITY, -INFINITY};
+          if (wt) {
+            const int klo = static_cast<int>(meta.lo) - key0 - krow - gq;
+            const int khi = static_cast<int>(meta.pos) - key0 - krow - gq;
 #pragma unroll
-          for (int r = 0; r < 4; ++r) {
-            const int64_t key = key0 + krow + gq + (r >= 2 ? 8 : 0);
-            const bool in = !wt || (key >= meta.lo && key <= meta.pos);
-            const float sv = in ? sacc[r] * a.scale_log2 : -INFINITY;
-            sacc[r] = sv;
-            mx[r & 1] = fmaxf(mx[r & 1], sv);
+            for (int r = 0; r < 4; ++r) {
+              const int kk = (r >= 2 ? 8 : 0);
+              sacc[r] = (kk >= klo && kk <= khi) ? sacc[r] * a.scale_log2 : -INFINITY;
+            }
+          } else {
+#pragma unroll
+            for (int r = 0; r < 4; ++r) sacc[r] *= a.scale_log2;
           }
+#pragma unroll
+          for (int r = 0; r < 4; ++r) mx[r & 1] = fmaxf(mx[r & 1], sacc[r]);
           bool grow = false;
 #pragma unroll
           for (int h = 0; h < 2; ++h) {
@@ -292,20 +338,8 @@ __global__ void __launch_bounds__(288, 1)
           const uint32_t pb0 = movmatrix_trans(pack_bf16(p[0], p[1]));
           const uint32_t pb1 = movmatrix_trans(pack_bf16(p[2], p[3]));
           // O^T += V^T P^T over this warp's 16 keys
-          {
-            const int mi = lane >> 3;
-            const int row = krow + (lane & 7) + (mi >> 1) * 8;
 #pragma unroll
-            for (int mm = 0; mm < MT; ++mm) {
-              const int dchunk = mm * 2 + (mi & 1);
-              const uint32_t addr = vb + (dchunk >> 3) * C::HALF + row * 128 + (((dchunk & 7) ^ (row & 7)) << 4);
-              uint32_t af[4];
-              ldmatrix_x4_trans(af, addr);
-              mma_16816(oacc[mm], af, pb0, pb1);
-            }
-          }
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&empty[s]);
+          for (int mm = 0; mm < MT; ++mm) mma_16816(oacc[mm], vf[mm], pb0, pb1);
         }
         cnt += meta.n_sub;
       }

@@ -54,14 +54,21 @@ __device__ __forceinline__ ItemTiles item_tiles_v(int v, int topk, int64_t pos, 
   it.spb = block / 64;
   it.lo = pos - window + 1 > 0 ? pos - window + 1 : 0;
   it.win_t0 = it.lo / 64;
-  const int64_t win_t1 = pos / 64;
-  uint64_t wm = 0;
-  for (int64_t t = it.win_t0; t <= win_t1; ++t) {
-    const int blk = static_cast<int>((t * 64) / block);
-    const bool covered = __ballot_sync(0xFFFFFFFFu, valid && v == blk) != 0;
-    if (!covered) wm |= 1ull << (t - it.win_t0);
+  const int ntw = static_cast<int>(pos / 64 - it.win_t0) + 1;     // window tiles, <= 64
+  // window tiles covered by this lane's selected block, then OR over the warp
+  uint32_t cov_lo = 0, cov_hi = 0;
+  if (valid) {
+    for (int q = 0; q < it.spb; ++q) {
+      const int64_t r = static_cast<int64_t>(v) * it.spb + q - it.win_t0;
+      if (r >= 0 && r < 32) cov_lo |= 1u << r;
+      else if (r >= 32 && r < 64) cov_hi |= 1u << (r - 32);
+    }
   }
-  it.winmask = wm;
+  cov_lo = __reduce_or_sync(0xFFFFFFFFu, cov_lo);
+  cov_hi = __reduce_or_sync(0xFFFFFFFFu, cov_hi);
+  const uint64_t all = ntw >= 64 ? ~0ull : ((1ull << ntw) - 1ull);
+  it.winmask = all & ~((static_cast<uint64_t>(cov_hi) << 32) | cov_lo);
+  const uint64_t wm = it.winmask;
   it.n_sub = it.n_sel * it.spb + __popcll(wm);
   return it;
 }
