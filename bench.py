@@ -174,6 +174,25 @@ def attended_keys(idx, w):
     return n_sel * B + wcount - overlap
 
 
+def block_major_counts(idx, w):
+    """Valid (query, kv-head, slot) selections and distinct selected
+    (batch, kv-head, block) pairs, by the same validity rule as the kernels
+    (in range, larger than every earlier in-range entry of the row)."""
+    nb = w.n // w.block
+    pos = torch.arange(w.n_q, device=idx.device, dtype=torch.int64).view(1, -1, 1, 1) + w.q_offset
+    nvis = torch.clamp((pos + 1) // w.block, max=nb)
+    v = idx.to(torch.int64)
+    inr = (v >= 0) & (v < nvis)
+    run = torch.cummax(torch.where(inr, v, torch.full_like(v, -1)), dim=-1).values
+    prev = torch.cat([torch.full_like(run[..., :1], -1), run[..., :-1]], dim=-1)
+    valid = inr & (v > prev)
+    n_entries = int(valid.sum().item())
+    b_, i_, g_, j_ = torch.nonzero(valid, as_tuple=True)
+    key = (b_ * w.h_kv + g_) * nb + v[b_, i_, g_, j_]
+    n_blocks = int(torch.unique(key).numel())
+    return n_entries, n_blocks
+
+
 def algorithmic_work(w, idx):
     es = 4 if w.dtype == "f32" else 2
     nb = w.n // w.block
@@ -186,8 +205,25 @@ def algorithmic_work(w, idx):
     gathered = float(S.sum().item()) * w.d * 2 * es
     qo = 2.0 * w.batch * w.n_q * w.h_q * w.d * es
     attn_flops = 4.0 * float(S.sum().item()) * G * w.d
-    return dict(summary_bytes=summary_bytes, route_flops=route_flops, attn_bytes=gathered + qo,
-                gathered_bytes=gathered, attn_flops=attn_flops, mean_keys=float(S.float().mean().item()))
+    out = dict(summary_bytes=summary_bytes, route_flops=route_flops, attn_bytes=gathered + qo,
+               gathered_bytes=gathered, attn_flops=attn_flops, mean_keys=float(S.float().mean().item()))
+    if w.dtype == "bf16":
+        # block-major stages: per valid selection the tile kernel reads the
+        # query heads' rows and writes one partial row + log-sum-exp per head,
+        # and reads each distinct selected block's K_c, V_c once; the merge
+        # reads Q, the partials and the window keys outside the selected
+        # blocks and writes O and lse
+        ne, nblk = block_major_counts(idx, w)
+        items = w.batch * w.n_q * w.h_kv
+        window_keys = float(S.sum().item()) - ne * w.block
+        out["blocks_bytes"] = ne * G * (w.d * 2 * 2 + 8) + nblk * 2 * w.block * w.d * 2
+        out["blocks_flops"] = 4.0 * ne * G * w.block * w.d
+        out["merge_bytes"] = (items * (G * w.d * 2 * 2 + G * 4 + w.topk * 4) + ne * G * (w.d * 2 + 8)
+                              + window_keys * 2 * w.d * 2)
+        out["plan_bytes"] = items * w.topk * 4 * 2 + ne * 4 * 2
+        out["n_entries"] = ne
+        out["n_blocks"] = nblk
+    return out
 
 
 # ------------------------------------------------------------------ our arm
@@ -201,29 +237,40 @@ def run_ours(w, steps, warmup, ws, rank, with_e2e=True):
     tab = torch.empty(tab_s, dtype=torch.bfloat16, device=dev)
     idx = torch.empty(ssa.idx_shape(p), dtype=torch.int32, device=dev)
     rws = ssa.byte_buffer(ssa.ssa_route_workspace_size(p), dev)
+    aw_bytes = ssa.ssa_attn_workspace_size(p)
+    aws = ssa.byte_buffer(aw_bytes, dev) if aw_bytes else None
     O = torch.empty_like(Q)
     lse = torch.empty(Q.shape[:3], dtype=torch.float32, device=dev)
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream()
 
+    # stages of one step, each bracketed by events on the launching stream;
+    # block-major attention runs as its three staged calls
+    if aws is not None:
+        stages = [("summary", lambda: ssa.ssa_block_summary(p, K, None, None, tab)),
+                  ("route", lambda: ssa.ssa_route_topk(p, Q, None, None, tab, idx, None, rws)),
+                  ("attn_plan", lambda: ssa.ssa_attn_plan(p, idx, aws)),
+                  ("attn_blocks", lambda: ssa.ssa_attn_blocks(p, Q, K, V, aws)),
+                  ("attn_merge", lambda: ssa.ssa_attn_merge(p, Q, K, V, idx, O, lse, None, aws))]
+    else:
+        stages = [("summary", lambda: ssa.ssa_block_summary(p, K, None, None, tab)),
+                  ("route", lambda: ssa.ssa_route_topk(p, Q, None, None, tab, idx, None, rws)),
+                  ("attn_gather", lambda: ssa.ssa_sparse_attn(p, Q, K, V, idx, O, lse))]
+    ns = len(stages)
+
     def step(ev=None):
+        for k, (_, fn) in enumerate(stages):
+            if ev:
+                ev[k].record(stream)
+            fn()
         if ev:
-            ev[0].record(stream)
-        ssa.ssa_block_summary(p, K, None, None, tab)
-        if ev:
-            ev[1].record(stream)
-        ssa.ssa_route_topk(p, Q, None, None, tab, idx, None, rws)
-        if ev:
-            ev[2].record(stream)
-        ssa.ssa_sparse_attn(p, Q, K, V, idx, O, lse)
-        if ev:
-            ev[3].record(stream)
+            ev[ns].record(stream)
 
     for _ in range(warmup):
         flush.zero_()
         step()
     torch.cuda.synchronize()
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(steps)]
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(ns + 1)] for _ in range(steps)]
     barrier(ws)
     torch.cuda.synchronize()
     l0 = ssa.ssa_launch_count()
@@ -235,8 +282,8 @@ def run_ours(w, steps, warmup, ws, rank, with_e2e=True):
     launches = ssa.ssa_launch_count() - l0
     barrier(ws)
     assert ssa.ssa_device_error() == 0
-    per = np.array([[e[0].elapsed_time(e[1]), e[1].elapsed_time(e[2]), e[2].elapsed_time(e[3])] for e in evs])
-    ms_kernels = per.mean(axis=0)
+    per = np.array([[e[k].elapsed_time(e[k + 1]) for k in range(ns)] for e in evs])
+    ms_kernels = {name: float(x) for (name, _), x in zip(stages, per.mean(axis=0))}
     ms_step_local = float(per.sum(axis=1).mean())
     ms_step = max_over_ranks(ms_step_local, ws)
     work = algorithmic_work(w, idx)
@@ -246,7 +293,7 @@ def run_ours(w, steps, warmup, ws, rank, with_e2e=True):
         hQ, hK, hV = Q.cpu().pin_memory(), K.cpu().pin_memory(), V.cpu().pin_memory()
         hO = torch.empty(Q.shape, dtype=Q.dtype).pin_memory()
         hl = torch.empty(Q.shape[:3], dtype=torch.float32).pin_memory()
-        del O, lse
+        del O, lse, aws, stages
         buf = ssa.byte_buffer(ssa.ssa_hostio_buffer_size(p), dev)
         for _ in range(max(1, warmup)):
             ssa.ssa_forward_hostio(p, hQ, hK, hV, hO, hl, buf)
@@ -270,23 +317,58 @@ def run_ours(w, steps, warmup, ws, rank, with_e2e=True):
                 clocks=clk.summary(), e2e=e2e)
 
 
+KERNEL_NAMES = {"summary": "summary_diag_kernel", "route": "route_tiled_kernel", "attn_plan": "inv_*_kernel (5)",
+                "attn_blocks": "attn_block_kernel", "attn_merge": "attn_bf16_kernel (merge)",
+                "attn_gather": "attn_bf16_kernel"}
+
+
 def kernel_report(w, res, peaks, traffic):
-    ms_s, ms_r, ms_a = (float(x) for x in res["ms_kernels"])
+    """Per stage: time, algorithmic work and the fraction of the measured
+    peak of the unit that bounds it (the larger of the HBM and tensor
+    fractions where both apply)."""
+    ms = res["ms_kernels"]
     wk = res["work"]
     hbm = peaks["hbm_gbs"]
     tc = peaks["bf16_tflops_sustained"]
-    s_gbs = wk["summary_bytes"] / (ms_s * 1e-3) / 1e9
-    r_tf = wk["route_flops"] / (ms_r * 1e-3) / 1e12
-    a_gbs = wk["attn_bytes"] / (ms_a * 1e-3) / 1e9
-    return {
-        "summary": {"ms": ms_s, "bound": "hbm", "achieved": s_gbs, "unit": "GB/s", "frac": s_gbs / hbm,
-                    "algorithmic_bytes": wk["summary_bytes"]},
-        "route": {"ms": ms_r, "bound": "tensor", "achieved": r_tf, "unit": "TFLOP/s", "frac": r_tf / tc,
-                  "algorithmic_flops": wk["route_flops"], "peak": tc},
-        "attention": {"ms": ms_a, "bound": "hbm", "achieved": a_gbs, "unit": "GB/s", "frac": a_gbs / hbm,
-                      "algorithmic_bytes": wk["attn_bytes"], "mean_keys_per_row": wk["mean_keys"],
-                      "traffic": traffic.get(("attn_bf16", w.name))},
-    }
+    rep = {}
+
+    def hbm_entry(name, nbytes, extra=None):
+        t = ms[name] * 1e-3
+        gbs = nbytes / t / 1e9
+        e = {"ms": ms[name], "bound": "hbm", "achieved": gbs, "unit": "GB/s", "frac": gbs / hbm, "peak": hbm,
+             "algorithmic_bytes": nbytes, "kernel": KERNEL_NAMES[name],
+             "traffic": traffic.get((KERNEL_NAMES[name].split()[0], w.name))}
+        e.update(extra or {})
+        rep[name] = e
+
+    hbm_entry("summary", wk["summary_bytes"])
+    r_tf = wk["route_flops"] / (ms["route"] * 1e-3) / 1e12
+    rep["route"] = {"ms": ms["route"], "bound": "tensor", "achieved": r_tf, "unit": "TFLOP/s", "frac": r_tf / tc,
+                    "peak": tc, "algorithmic_flops": wk["route_flops"], "kernel": KERNEL_NAMES["route"],
+                    "traffic": traffic.get(("route_tiled_kernel", w.name))}
+    if "attn_gather" in ms:
+        hbm_entry("attn_gather", wk["attn_bytes"], {"mean_keys_per_row": wk["mean_keys"]})
+    else:
+        hbm_entry("attn_plan", wk["plan_bytes"])
+        hbm_entry("attn_blocks", wk["blocks_bytes"], {"n_entries": wk["n_entries"], "n_blocks": wk["n_blocks"]})
+        b_tf = wk["blocks_flops"] / (ms["attn_blocks"] * 1e-3) / 1e12
+        rep["attn_blocks"]["tensor"] = {"achieved": b_tf, "unit": "TFLOP/s", "frac": b_tf / tc, "peak": tc,
+                                        "algorithmic_flops": wk["blocks_flops"]}
+        if b_tf / tc > rep["attn_blocks"]["frac"]:
+            rep["attn_blocks"].update(bound="tensor", achieved=b_tf, unit="TFLOP/s", frac=b_tf / tc, peak=tc)
+        hbm_entry("attn_merge", wk["merge_bytes"])
+    # the pages' attention figure: algorithmic gathered K+V (+ q, o) bytes over
+    # the whole attention time, whichever way it is evaluated
+    t_att = sum(v for k, v in ms.items() if k.startswith("attn_")) * 1e-3
+    rep["attention_gather_equivalent"] = {"ms": t_att * 1e3, "achieved": wk["attn_bytes"] / t_att / 1e9,
+                                          "unit": "GB/s", "algorithmic_bytes": wk["attn_bytes"],
+                                          "mean_keys_per_row": wk["mean_keys"]}
+    return rep
+
+
+def dominant(rep):
+    name = max((k for k in rep if "bound" in rep[k]), key=lambda k: rep[k]["ms"])
+    return name, rep[name]
 
 
 # ------------------------------------------------------------------ oracle (CPU)
@@ -382,10 +464,12 @@ def main():
     res = run_ours(w, a.steps, a.warmup, ws, rank, with_e2e=not a.no_e2e)
     kern = kernel_report(w, res, peaks, traffic)
     value = ws * w.batch * w.n_q * w.h_q / (res["ms_step"] / 1e3)
-    att = kern["attention"]
-    roof = {"bound": "hbm", "achieved": att["achieved"], "peak": peaks["hbm_gbs"], "unit": "GB/s",
-            "frac": att["frac"], "traffic": att["traffic"], "kernel": "attn_bf16_kernel",
-            "peak_source": peak_src, "algorithmic_bytes_per_launch": att["algorithmic_bytes"]}
+    dname, dk = dominant(kern)
+    roof = {"bound": dk["bound"], "achieved": dk["achieved"], "peak": dk["peak"], "unit": dk["unit"],
+            "frac": dk["frac"], "traffic": dk["traffic"], "kernel": dk["kernel"], "stage": dname,
+            "peak_source": peak_src,
+            "algorithmic_per_launch": dk.get("algorithmic_flops") if dk["bound"] == "tensor"
+            else dk["algorithmic_bytes"]}
     secondary = None
     if not a.no_secondary and w.name == PRIMARY and a.n is None:
         torch.cuda.empty_cache()

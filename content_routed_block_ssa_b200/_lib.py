@@ -55,7 +55,11 @@ def _load():
         "ssa_route_workspace_size": (sz, [P]),
         "ssa_route_topk": (i32, [P, vp, vp, vp, vp, vp, vp, vp, sz, vp]),
         "ssa_route_topk_static": (i32, [P, vp, vp, vp, vp, vp, vp, vp]),
-        "ssa_sparse_attn": (i32, [P, vp, vp, vp, vp, vp, vp, vp, vp]),
+        "ssa_attn_workspace_size": (sz, [P]),
+        "ssa_attn_plan": (i32, [P, vp, vp, sz, vp]),
+        "ssa_attn_blocks": (i32, [P, vp, vp, vp, vp, sz, vp]),
+        "ssa_attn_merge": (i32, [P, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]),
+        "ssa_sparse_attn": (i32, [P, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]),
         "ssa_workspace_size": (sz, [P]),
         "ssa_forward": (i32, [P, vp, vp, vp, vp, vp, vp, sz, vp]),
         "ssa_hostio_buffer_size": (sz, [P]),
@@ -72,7 +76,8 @@ lib = _load()
 LIB_PATH = _LIB_PATH
 EXPORTED = ("ssa_status_string", "ssa_version", "ssa_launch_count", "ssa_device_error",
             "ssa_block_summary", "ssa_route_workspace_size", "ssa_route_topk", "ssa_route_topk_static",
-            "ssa_sparse_attn",
+            "ssa_attn_workspace_size", "ssa_sparse_attn", "ssa_attn_plan", "ssa_attn_blocks",
+            "ssa_attn_merge",
             "ssa_workspace_size", "ssa_forward", "ssa_hostio_buffer_size", "ssa_forward_hostio")
 
 
@@ -149,9 +154,33 @@ def ssa_route_topk_static(p, Q, mu, sigma, route_table, block_idx, top_scores=No
            "ssa_route_topk_static")
 
 
-def ssa_sparse_attn(p, Q, K, V, block_idx, O, lse=None, bad_index_count=None, stream=None):
+def ssa_attn_workspace_size(p) -> int:
+    return int(lib.ssa_attn_workspace_size(C.byref(p)))
+
+
+def _nbytes(t):
+    return t.numel() * t.element_size() if t is not None else 0
+
+
+def ssa_attn_plan(p, block_idx, ws, stream=None):
+    _check(lib.ssa_attn_plan(C.byref(p), _ptr(block_idx), _ptr(ws), _nbytes(ws), _stream(stream)), "ssa_attn_plan")
+
+
+def ssa_attn_blocks(p, Q, K, V, ws, stream=None):
+    _check(lib.ssa_attn_blocks(C.byref(p), _ptr(Q), _ptr(K), _ptr(V), _ptr(ws), _nbytes(ws), _stream(stream)),
+           "ssa_attn_blocks")
+
+
+def ssa_attn_merge(p, Q, K, V, block_idx, O, lse, bad_index_count, ws, stream=None):
+    _check(lib.ssa_attn_merge(C.byref(p), _ptr(Q), _ptr(K), _ptr(V), _ptr(block_idx), _ptr(O), _ptr(lse),
+                              _ptr(bad_index_count), _ptr(ws), _nbytes(ws), _stream(stream)), "ssa_attn_merge")
+
+
+def ssa_sparse_attn(p, Q, K, V, block_idx, O, lse=None, bad_index_count=None, ws=None, stream=None):
+    nbytes = ws.numel() * ws.element_size() if ws is not None else 0
     _check(lib.ssa_sparse_attn(C.byref(p), _ptr(Q), _ptr(K), _ptr(V), _ptr(block_idx), _ptr(O),
-                               _ptr(lse), _ptr(bad_index_count), _stream(stream)), "ssa_sparse_attn")
+                               _ptr(lse), _ptr(bad_index_count), _ptr(ws), nbytes, _stream(stream)),
+           "ssa_sparse_attn")
 
 
 def ssa_workspace_size(p) -> int:

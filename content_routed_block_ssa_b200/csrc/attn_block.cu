@@ -1,0 +1,598 @@
+// Block-major evaluation of the routed part of the attention (steps (ii) and
+// (iii) of "Subquadratic Sparse Attention (SSA)", opening section): instead of
+// every query gathering its selected key blocks, every selected block is
+// read once and multiplied against the queries that selected it.
+//
+//  1. inversion: count the selections per key block, scan, scatter the
+//     (query, slot) entries into per-block lists and cut each list into
+//     tiles of 128 / G queries (128 tensor-core rows with the G query heads);
+//  2. block tiles on tcgen05: the tile's Q rows are gathered with 16-byte
+//     asynchronous copies into the 128-byte-swizzled operand layout, K_c and
+//     V_c arrive by TMA, S = Q K_c^T and O = P V_c run on the tensor cores with TMEM
+//     accumulators, the softmax over the block's keys runs in between, and
+//     each (query, head, slot) gets a normalised partial output (float16
+//     with a power-of-two row scale) and its log-sum-exp (base 2, of the
+//     scaled logits);
+//  3. the window keys and the merge of the partials into the final output
+//     run in the gather kernel (attn.cu, merge mode), one query row at a time.
+//
+// Exact: the merge of normalised partials with their log-sum-exps is the
+// same softmax over the union of the selected blocks and the window.
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <math.h>
+
+#include "common.cuh"
+#include "invert.cuh"
+#include "kernels.h"
+
+namespace ssa {
+namespace {
+
+// ------------------------------------------------------------------ inversion
+
+__global__ void __launch_bounds__(256) inv_count_kernel(const BlockPlan pl, const int32_t* __restrict__ idx) {
+  const int64_t row = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  if (row >= static_cast<int64_t>(pl.bgs) * pl.n_q) return;   // warp-uniform
+  const int lane = threadIdx.x & 31;
+  const int i = static_cast<int>(row % pl.n_q);
+  const int bg = static_cast<int>(row / pl.n_q);
+  const int b = bg / pl.h_kv, g = bg % pl.h_kv;
+  const int64_t pos = pl.q_offset + i;
+  const int nvis = static_cast<int>(min(static_cast<int64_t>(pl.nb), (pos + 1) / pl.block));
+  const int v = lane < pl.topk ? __ldg(idx + ((static_cast<int64_t>(b) * pl.n_q + i) * pl.h_kv + g) * pl.topk + lane) : -1;
+  if (selection_valid(v, nvis)) atomicAdd(&pl.count[static_cast<int64_t>(bg) * pl.nb + v], 1);
+}
+
+// One CTA per (batch, kv-head): exclusive scans of the per-block entry and
+// tile counts.
+__global__ void __launch_bounds__(1024) inv_scan_kernel(const BlockPlan pl) {
+  __shared__ int32_t wsum_e[32], wsum_t[32];
+  const int bg = blockIdx.x;
+  const int32_t* cnt = pl.count + static_cast<int64_t>(bg) * pl.nb;
+  const int per = (pl.nb + 1023) / 1024;
+  const int c0 = threadIdx.x * per;
+  int se = 0, st = 0;
+  for (int c = c0; c < min(c0 + per, pl.nb); ++c) {
+    se += cnt[c];
+    st += (cnt[c] + pl.qpt - 1) / pl.qpt;
+  }
+  // block-wide exclusive scan of (se, st)
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  int ie = se, it = st;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int ye = __shfl_up_sync(0xFFFFFFFFu, ie, o), yt = __shfl_up_sync(0xFFFFFFFFu, it, o);
+    if (lane >= o) { ie += ye; it += yt; }
+  }
+  if (lane == 31) { wsum_e[warp] = ie; wsum_t[warp] = it; }
+  __syncthreads();
+  if (warp == 0) {
+    int ve = wsum_e[lane], vt = wsum_t[lane];
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int ye = __shfl_up_sync(0xFFFFFFFFu, ve, o), yt = __shfl_up_sync(0xFFFFFFFFu, vt, o);
+      if (lane >= o) { ve += ye; vt += yt; }
+    }
+    wsum_e[lane] = ve;
+    wsum_t[lane] = vt;
+  }
+  __syncthreads();
+  int base_e = (warp ? wsum_e[warp - 1] : 0) + ie - se;
+  int base_t = (warp ? wsum_t[warp - 1] : 0) + it - st;
+  for (int c = c0; c < min(c0 + per, pl.nb); ++c) {
+    pl.blk_off[static_cast<int64_t>(bg) * pl.nb + c] = base_e;
+    pl.tile_off[static_cast<int64_t>(bg) * pl.nb + c] = base_t;
+    base_e += cnt[c];
+    base_t += (cnt[c] + pl.qpt - 1) / pl.qpt;
+  }
+  if (threadIdx.x == 1023) {
+    pl.bg_ents[bg] = base_e;
+    pl.bg_tiles[bg] = base_t;
+  }
+}
+
+// One CTA: exclusive scans over (batch, kv-head); slot [bgs] holds the totals.
+__global__ void __launch_bounds__(1024) inv_scan_bg_kernel(const BlockPlan pl) {
+  if (threadIdx.x != 0) return;
+  int e = 0, t = 0;
+  for (int bg = 0; bg < pl.bgs; ++bg) {
+    pl.ent_base[bg] = e;
+    pl.tile_base[bg] = t;
+    e += pl.bg_ents[bg];
+    t += pl.bg_tiles[bg];
+  }
+  pl.ent_base[pl.bgs] = e;
+  pl.tile_base[pl.bgs] = t;
+}
+
+__global__ void __launch_bounds__(256) inv_scatter_kernel(const BlockPlan pl, const int32_t* __restrict__ idx) {
+  const int64_t row = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  if (row >= static_cast<int64_t>(pl.bgs) * pl.n_q) return;   // warp-uniform
+  const int lane = threadIdx.x & 31;
+  const int i = static_cast<int>(row % pl.n_q);
+  const int bg = static_cast<int>(row / pl.n_q);
+  const int b = bg / pl.h_kv, g = bg % pl.h_kv;
+  const int64_t pos = pl.q_offset + i;
+  const int nvis = static_cast<int>(min(static_cast<int64_t>(pl.nb), (pos + 1) / pl.block));
+  const int v = lane < pl.topk ? __ldg(idx + ((static_cast<int64_t>(b) * pl.n_q + i) * pl.h_kv + g) * pl.topk + lane) : -1;
+  if (selection_valid(v, nvis)) {
+    const int64_t cb = static_cast<int64_t>(bg) * pl.nb + v;
+    const int slot = pl.ent_base[bg] + pl.blk_off[cb] + atomicAdd(&pl.cursor[cb], 1);
+    pl.entries[slot] = (i << 5) | lane;
+  }
+}
+
+__global__ void __launch_bounds__(256) inv_tiles_kernel(const BlockPlan pl) {
+  const int64_t x = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (x >= static_cast<int64_t>(pl.bgs) * pl.nb) return;
+  const int bg = static_cast<int>(x / pl.nb), c = static_cast<int>(x % pl.nb);
+  const int n = pl.count[x];
+  const int e0 = pl.ent_base[bg] + pl.blk_off[x];
+  const int t0 = pl.tile_base[bg] + pl.tile_off[x];
+  for (int t = 0; t * pl.qpt < n; ++t)
+    pl.tiles[t0 + t] = make_int4(bg, c, e0 + t * pl.qpt, min(pl.qpt, n - t * pl.qpt));
+}
+
+// ------------------------------------------------------------------ block tiles
+
+template <int BLK>
+struct BlkCfg {
+  static constexpr int D = 128;
+  static constexpr int ROW = 128;                       // bytes per 64-wide swizzled row
+  static constexpr int A_HALF = 128 * ROW;              // 128 rows x 64 dims
+  static constexpr int A_BYTES = 2 * A_HALF;            // Q tile
+  static constexpr int KV_HALF = BLK * ROW;             // BLK keys x 64 dims
+  static constexpr int KV_BYTES = 4 * KV_HALF;          // K lo, K hi, V lo, V hi
+  static constexpr int P_HALF = 128 * ROW;              // 128 rows x 64 keys
+  static constexpr int P_BYTES = (BLK / 64) * P_HALF;
+  static constexpr int NKV = (BLK == 64) ? 2 : 1;       // K/V buffers
+  static constexpr int SMEM = 1024 + 2 * A_BYTES + NKV * KV_BYTES + 2 * P_BYTES + 24 * 8 + 16;
+  static constexpr int S_COL = 0;                       // TMEM: S[2] then O[2]
+  static constexpr int O_COL = 2 * BLK;
+};
+
+struct BlkArgs {
+  const __nv_bfloat16* Q;
+  const int4* tiles;
+  const int32_t* n_tiles;    // device: total tiles
+  const int32_t* entries;
+  int32_t n_q, n_kv, h_q, h_kv, topk;
+  float scale_log2;
+  __half* partO;             // [items][topk][G][D], o / 2^e
+  float2* partL;             // [items][partL_stride]: (log2-sum-exp, 2^e); slot j head h at j*G + h
+  int32_t partL_stride;
+  uint32_t* err;
+};
+
+__device__ __forceinline__ void tile_range(int T, int& t0, int& t1) {
+  t0 = static_cast<int>((static_cast<int64_t>(T) * blockIdx.x) / gridDim.x);
+  t1 = static_cast<int>((static_cast<int64_t>(T) * (blockIdx.x + 1)) / gridDim.x);
+}
+
+__device__ __forceinline__ void fence_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// Shared-memory descriptor of an MN-major operand written by TMA with the
+// 128-byte swizzle: rows of 64 MN-elements (128 B), 8-row groups `sbo` apart
+// along K, 64-element MN groups `lbo` apart.
+__device__ __forceinline__ uint64_t umma_desc_sw128_mn(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+  uint64_t d = 0;
+  d |= static_cast<uint64_t>((saddr & 0x3FFFFu) >> 4);
+  d |= static_cast<uint64_t>((lbo >> 4) & 0x3FFFu) << 16;
+  d |= static_cast<uint64_t>((sbo >> 4) & 0x3FFFu) << 32;
+  d |= static_cast<uint64_t>(1) << 46;
+  d |= static_cast<uint64_t>(2) << 61;
+  return d;
+}
+
+// Warp roles: 0 = TMA producer (Q rows of each tile, K/V of each block),
+// 1 = MMA issuer and TMEM owner, 2..5 = softmax and epilogue (one tensor-core
+// row = one (query, head) pair per thread).
+template <int G, int BLK>
+__global__ void __launch_bounds__(192, 1)
+    attn_block_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+                      const BlkArgs a) {
+  using C = BlkCfg<BLK>;
+  constexpr int D = C::D;
+  constexpr int QPT = 128 / G;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sA = smem;                                   // [2][A_BYTES]
+  uint8_t* sKV = sA + 2 * C::A_BYTES;                   // [NKV][KV_BYTES]
+  uint8_t* sP = sKV + C::NKV * C::KV_BYTES;             // [2][P_BYTES]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sP + 2 * C::P_BYTES);
+  uint64_t* a_full = bars;          // [2] (producer arrives once the tile's copies landed)
+  uint64_t* a_empty = bars + 2;     // [2]
+  uint64_t* kv_full = bars + 4;     // [2]
+  uint64_t* kv_empty = bars + 6;    // [2]
+  uint64_t* s_full = bars + 8;      // [2]
+  uint64_t* s_empty = bars + 10;    // [2]
+  uint64_t* p_full = bars + 12;     // [2]
+  uint64_t* o_full = bars + 14;     // [2]
+  uint64_t* o_empty = bars + 16;    // [2]
+  uint64_t* mma_done = bars + 18;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 19);
+
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&a_full[i], 1); mbar_init(&a_empty[i], 1);
+      mbar_init(&kv_full[i], 1); mbar_init(&kv_empty[i], 1);
+      mbar_init(&s_full[i], 1); mbar_init(&s_empty[i], 4);
+      mbar_init(&p_full[i], 4); mbar_init(&o_full[i], 1); mbar_init(&o_empty[i], 4);
+    }
+    mbar_init(mma_done, 1);
+    fence_barrier_init();
+    tma_prefetch_desc(&tmK);
+    tma_prefetch_desc(&tmV);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  int t0, t1;
+  tile_range(*a.n_tiles, t0, t1);
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    bool ok = true;
+    int kv_ord = -1;
+    int64_t prev = -1;
+    uint32_t a_loads = 0, kv_loads = 0;
+    // the next tile's descriptor and entries (one per lane, two for G = 2)
+    // are loaded while this tile's copies are issued
+    const int4 none = make_int4(0, 0, 0, 0);
+    int4 nxt = t0 < t1 ? a.tiles[t0] : none;
+    int4 nxt2 = t0 + 1 < t1 ? a.tiles[t0 + 1] : none;
+    int nen0 = lane < nxt.w ? __ldg(a.entries + nxt.z + lane) : 0;
+    int nen1 = (QPT > 32 && lane + 32 < nxt.w) ? __ldg(a.entries + nxt.z + 32 + lane) : 0;
+    for (int t = t0; t < t1 && ok; ++t) {
+      const int lt = t - t0;
+      const int4 td = nxt;   // bg, c, entry start, entries
+      const int en0 = nen0, en1 = nen1;
+      nxt = nxt2;
+      nxt2 = t + 2 < t1 ? a.tiles[t + 2] : none;
+      nen0 = lane < nxt.w ? __ldg(a.entries + nxt.z + lane) : 0;
+      nen1 = (QPT > 32 && lane + 32 < nxt.w) ? __ldg(a.entries + nxt.z + 32 + lane) : 0;
+      const int bg = td.x, c = td.y, ne = td.w;
+      const int b = bg / a.h_kv, g = bg % a.h_kv;
+      // Q rows of the tile: 16-byte cp.async copies placed at their 128-byte
+      // swizzled positions
+      const int ab = lt & 1;
+      if (lane == 0) ok = mbar_wait(&a_empty[ab], ((lt >> 1) & 1) ^ 1, a.err, SITE_BLK_A_EMPTY);
+      ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
+      if (!ok) break;
+      const uint32_t abase = smem_u32(sA + ab * C::A_BYTES);
+      for (int ee = 0; ee < ne; ++ee) {
+        const int ent = ee < 32 ? __shfl_sync(0xFFFFFFFFu, en0, ee) : __shfl_sync(0xFFFFFFFFu, en1, ee - 32);
+        const int i = ent >> 5;
+        const __nv_bfloat16* qrow = a.Q + ((static_cast<int64_t>(b) * a.n_q + i) * a.h_q +
+                                           static_cast<int64_t>(g) * G) * D;
+#pragma unroll
+        for (int x = lane; x < G * 16; x += 32) {   // G heads x 16 chunks of 8 dims
+          const int hh = x >> 4, ch = x & 15;
+          const int r = ee * G + hh;
+          const uint32_t dst = abase + (ch >> 3) * C::A_HALF + r * C::ROW + (((ch & 7) ^ (r & 7)) << 4);
+          asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(qrow + hh * D + ch * 8)
+                       : "memory");
+        }
+      }
+      asm volatile("cp.async.commit_group;" ::: "memory");
+      ++a_loads;
+      // tile t-1 is published once tile t is in flight, and before any wait
+      // on the K/V buffers: freeing a K/V buffer can need tile t-1's MMAs
+      if (lt > 0) {
+        asm volatile("cp.async.wait_group 1;" ::: "memory");
+        fence_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&a_full[(lt - 1) & 1]);
+      }
+      const int64_t key = static_cast<int64_t>(bg) * 0x7FFFFFFF + c;
+      if (key != prev) {
+        ++kv_ord;
+        prev = key;
+        const int kb = kv_ord % C::NKV;
+        if (lane == 0) {
+          ok = mbar_wait(&kv_empty[kb], ((kv_ord / C::NKV) & 1) ^ 1, a.err, SITE_BLK_KV_EMPTY);
+          if (ok) {
+            uint8_t* kv = sKV + kb * C::KV_BYTES;
+            mbar_arrive_expect_tx(&kv_full[kb], C::KV_BYTES);
+            const int z = static_cast<int>(static_cast<int64_t>(b) * a.n_kv + static_cast<int64_t>(c) * BLK);
+#pragma unroll
+            for (int sub = 0; sub < BLK / 64; ++sub) {
+#pragma unroll
+              for (int hf = 0; hf < 2; ++hf) {
+                tma_load_3d(kv + hf * C::KV_HALF + sub * 64 * C::ROW, &tmK, &kv_full[kb], hf * 64, g, z + sub * 64);
+                tma_load_3d(kv + (2 + hf) * C::KV_HALF + sub * 64 * C::ROW, &tmV, &kv_full[kb], hf * 64, g, z + sub * 64);
+              }
+            }
+            ++kv_loads;
+          }
+        }
+        ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
+        kv_loads = __shfl_sync(0xFFFFFFFFu, kv_loads, 0);
+        if (!ok) break;
+      }
+    }
+    if (ok && a_loads > 0) {
+      asm volatile("cp.async.wait_group 0;" ::: "memory");
+      fence_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&a_full[(a_loads - 1) & 1]);
+    }
+    if (!ok) {   // let issued copies land before the CTA exits
+      asm volatile("cp.async.wait_group 0;" ::: "memory");
+      if (lane == 0) {
+        const uint64_t tq = global_timer_ns();
+        for (uint32_t n = (kv_loads > C::NKV ? kv_loads - C::NKV : 0); n < kv_loads; ++n)
+          while (!mbar_try_wait(&kv_full[n % C::NKV], (n / C::NKV) & 1) && global_timer_ns() - tq < kWaitLimitNs) {}
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t IDESC1 = umma_idesc_bf16(128, BLK);
+      constexpr uint32_t IDESC2 = umma_idesc_bf16(128, D) | (1u << 16);   // B (V) is MN-major
+      const uint32_t sA_u = smem_u32(sA), sKV_u = smem_u32(sKV), sP_u = smem_u32(sP);
+      bool ok = true;
+      int kv_ord = -1;
+      int64_t prev = -1;
+      int pend_l = -1, pend_kb = 0;
+      bool pend_last = false;
+      auto mma2 = [&](int l, int kb, bool last_of_block) -> bool {
+        const int ob = l & 1;
+        if (!mbar_wait(&p_full[ob], (l >> 1) & 1, a.err, SITE_BLK_P_FULL)) return false;
+        if (!mbar_wait(&o_empty[ob], ((l >> 1) & 1) ^ 1, a.err, SITE_BLK_O_EMPTY)) return false;
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + C::O_COL + ob * D;
+        const uint32_t vbase = sKV_u + kb * C::KV_BYTES + 2 * C::KV_HALF;
+#pragma unroll
+        for (int kk = 0; kk < BLK / 16; ++kk) {
+          const uint64_t ad = umma_desc_sw128(sP_u + ob * C::P_BYTES + (kk >> 2) * C::P_HALF + (kk & 3) * 32);
+          const uint64_t bd = umma_desc_sw128_mn(vbase + kk * 16 * C::ROW, C::KV_HALF, 1024);
+          umma_bf16(d_tmem, ad, bd, IDESC2, kk != 0 ? 1u : 0u);
+        }
+        umma_commit(&o_full[ob]);
+        if (last_of_block) umma_commit(&kv_empty[kb]);
+        return true;
+      };
+      // tile descriptors two ahead, so no global load sits on the issue path
+      int4 cur = t0 < t1 ? a.tiles[t0] : make_int4(0, 0, 0, 0);
+      int4 nxt = t0 + 1 < t1 ? a.tiles[t0 + 1] : make_int4(-1, -1, 0, 0);
+      for (int t = t0; t < t1 && ok; ++t) {
+        const int lt = t - t0;
+        const int4 td = cur;
+        const int4 tn = nxt;
+        cur = nxt;
+        nxt = t + 2 < t1 ? a.tiles[t + 2] : make_int4(-1, -1, 0, 0);
+        const int64_t key = static_cast<int64_t>(td.x) * 0x7FFFFFFF + td.y;
+        bool fresh = false;
+        if (key != prev) { ++kv_ord; prev = key; fresh = true; }
+        const int kb = kv_ord % C::NKV;
+        const bool last = (t + 1 == t1) || (static_cast<int64_t>(tn.x) * 0x7FFFFFFF + tn.y) != key;
+        // a new block reusing the pending tile's K/V buffer: finish that
+        // tile's P V first, its commit frees the buffer for the producer
+        if (fresh && pend_l >= 0 && pend_kb == kb) {
+          if (!mma2(pend_l, pend_kb, pend_last)) { ok = false; break; }
+          pend_l = -1;
+        }
+        if (fresh && !mbar_wait(&kv_full[kb], (kv_ord / C::NKV) & 1, a.err, SITE_BLK_KV_FULL)) { ok = false; break; }
+        const int ab = lt & 1;
+        if (!mbar_wait(&a_full[ab], (lt >> 1) & 1, a.err, SITE_BLK_A_FULL)) { ok = false; break; }
+        if (!mbar_wait(&s_empty[ab], ((lt >> 1) & 1) ^ 1, a.err, SITE_BLK_S_EMPTY)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t s_tmem = tmem_base + C::S_COL + ab * BLK;
+        const uint32_t kbase = sKV_u + kb * C::KV_BYTES;
+#pragma unroll
+        for (int ks = 0; ks < D / 16; ++ks) {
+          const uint64_t ad = umma_desc_sw128(sA_u + ab * C::A_BYTES + (ks >> 2) * C::A_HALF + (ks & 3) * 32);
+          const uint64_t bd = umma_desc_sw128(kbase + (ks >> 2) * C::KV_HALF + (ks & 3) * 32);
+          umma_bf16(s_tmem, ad, bd, IDESC1, ks != 0 ? 1u : 0u);
+        }
+        umma_commit(&s_full[ab]);
+        umma_commit(&a_empty[ab]);
+        if (pend_l >= 0 && !mma2(pend_l, pend_kb, pend_last)) { ok = false; break; }
+        pend_l = lt;
+        pend_kb = kb;
+        pend_last = last;
+      }
+      if (ok && pend_l >= 0) mma2(pend_l, pend_kb, pend_last);
+      umma_commit(mma_done);
+      const uint64_t tq = global_timer_ns();
+      while (!mbar_try_wait(mma_done, 0) && global_timer_ns() - tq < kWaitLimitNs) {}
+    }
+  } else {
+    // ------------------------------------------------------------ softmax + epilogue
+    const int eq = warp & 3;
+    const int row = eq * 32 + lane;
+    const int e = row / G, h = row % G;
+    const uint32_t lane_base = static_cast<uint32_t>(eq * 32) << 16;
+    bool ok = true;
+    // tile descriptors two ahead and this thread's entry one ahead of use
+    const int4 none = make_int4(0, 0, 0, 0);
+    int4 nxt = t0 < t1 ? a.tiles[t0] : none;
+    int4 nxt2 = t0 + 1 < t1 ? a.tiles[t0 + 1] : none;
+    int nxt_ent = e < nxt.w ? __ldg(a.entries + nxt.z + e) : 0;
+    for (int t = t0; t < t1 && ok; ++t) {
+      const int lt = t - t0;
+      const int sb = lt & 1;
+      const int4 td = nxt;
+      const int ent = nxt_ent;
+      nxt = nxt2;
+      nxt2 = t + 2 < t1 ? a.tiles[t + 2] : none;
+      nxt_ent = e < nxt.w ? __ldg(a.entries + nxt.z + e) : 0;
+      const int bg = td.x, ne = td.w;
+      ok = __all_sync(0xFFFFFFFFu, mbar_wait(&s_full[sb], (lt >> 1) & 1, a.err, SITE_BLK_S_FULL));
+      if (!ok) break;
+      tc_fence_after();
+      float sv[BLK];
+      {
+        uint32_t r[BLK];
+#pragma unroll
+        for (int q = 0; q < BLK / 16; ++q)
+          tmem_ld16(tmem_base + lane_base + C::S_COL + sb * BLK + q * 16,
+                    *reinterpret_cast<uint32_t(*)[16]>(&r[q * 16]));
+        tmem_wait_ld();
+        tmem_regs_ready(r);
+#pragma unroll
+        for (int u = 0; u < BLK; ++u) sv[u] = __uint_as_float(r[u]) * a.scale_log2;
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&s_empty[sb]);
+      float m = -INFINITY;
+#pragma unroll
+      for (int j = 0; j < BLK; ++j) m = fmaxf(m, sv[j]);
+      float l = 0.f;
+      uint8_t* prow = sP + sb * C::P_BYTES;
+#pragma unroll
+      for (int ch = 0; ch < BLK / 8; ++ch) {
+        uint32_t w[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const float p0 = fast_exp2(sv[ch * 8 + 2 * u] - m), p1 = fast_exp2(sv[ch * 8 + 2 * u + 1] - m);
+          l += p0 + p1;
+          w[u] = pack_bf16(p0, p1);
+        }
+        const int half = ch >> 3, cc = ch & 7;
+        *reinterpret_cast<uint4*>(prow + half * C::P_HALF + row * C::ROW + ((cc ^ (row & 7)) << 4)) =
+            make_uint4(w[0], w[1], w[2], w[3]);
+      }
+      fence_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&p_full[sb]);
+      ok = __all_sync(0xFFFFFFFFu, mbar_wait(&o_full[sb], (lt >> 1) & 1, a.err, SITE_BLK_O_FULL));
+      if (!ok) break;
+      tc_fence_after();
+      const bool valid = e < ne;
+      const int i = ent >> 5, j = ent & 31;
+      const int64_t item = static_cast<int64_t>(bg) * a.n_q + i;
+      const int64_t slot = (item * a.topk + j) * G + h;
+      const int64_t lslot = item * a.partL_stride + j * G + h;
+      float ov[D];
+      {
+        uint32_t r[D];
+#pragma unroll
+        for (int q = 0; q < D / 16; ++q)
+          tmem_ld16(tmem_base + lane_base + C::O_COL + sb * D + q * 16,
+                    *reinterpret_cast<uint32_t(*)[16]>(&r[q * 16]));
+        tmem_wait_ld();
+        tmem_regs_ready(r);
+#pragma unroll
+        for (int u = 0; u < D; ++u) ov[u] = __uint_as_float(r[u]);
+      }
+      if (valid) {
+        // the normalised row o = O / l, stored as float16 times 2^-e with the
+        // power of two 2^e chosen so the row's largest entry lands in
+        // [2^14, 2^15): 11 significant bits whatever the scale of V
+        float amax = 0.f;
+#pragma unroll
+        for (int dd = 0; dd < D; ++dd) amax = fmaxf(amax, fabsf(ov[dd]));
+        const float inv_l = 1.f / l;
+        const float x = amax * inv_l;
+        int e = x > 0.f ? static_cast<int>((__float_as_uint(x) >> 23) & 0xFFu) - 127 - 14 : 0;
+        e = min(max(e, -100), 100);
+        const float mul = inv_l * __uint_as_float(static_cast<uint32_t>(127 - e) << 23);
+        uint4* dst = reinterpret_cast<uint4*>(a.partO + slot * D);
+#pragma unroll
+        for (int q = 0; q < D / 8; ++q) {
+          uint32_t w[4];
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            const __half2 hv = __floats2half2_rn(ov[q * 8 + 2 * u] * mul, ov[q * 8 + 2 * u + 1] * mul);
+            w[u] = *reinterpret_cast<const uint32_t*>(&hv);
+          }
+          dst[q] = make_uint4(w[0], w[1], w[2], w[3]);
+        }
+        a.partL[lslot] = make_float2(m + log2f(l), __uint_as_float(static_cast<uint32_t>(127 + e) << 23));
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&o_empty[sb]);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem_base, 512);
+  }
+}
+
+template <int G, int BLK>
+cudaError_t run_block(const BlockPlan& pl, const CUtensorMap& tmK, const CUtensorMap& tmV,
+                      const BlkArgs& a, const LaunchCtx& c) {
+  using C = BlkCfg<BLK>;
+  cudaError_t e = cudaFuncSetAttribute(attn_block_kernel<G, BLK>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+  if (e != cudaSuccess) return e;
+  attn_block_kernel<G, BLK><<<c.sm_count, 192, C::SMEM, c.stream>>>(tmK, tmV, a);
+  note_launch();
+  (void)pl;
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+int attn_block_smem_bytes(int block) { return block == 64 ? BlkCfg<64>::SMEM : BlkCfg<128>::SMEM; }
+
+cudaError_t launch_block_plan(const ssa_params& p, const int32_t* block_idx, const BlockPlan& pl,
+                              const LaunchCtx& c) {
+  const size_t cnt_bytes = static_cast<size_t>(pl.bgs) * pl.nb * sizeof(int32_t);
+  cudaError_t e = cudaMemsetAsync(pl.count, 0, cnt_bytes, c.stream);
+  if (e == cudaSuccess) e = cudaMemsetAsync(pl.cursor, 0, cnt_bytes, c.stream);
+  if (e != cudaSuccess) return e;
+  const int64_t rows = static_cast<int64_t>(pl.bgs) * pl.n_q;
+  const unsigned gw = static_cast<unsigned>((rows * 32 + 255) / 256);
+  inv_count_kernel<<<gw, 256, 0, c.stream>>>(pl, block_idx);
+  note_launch();
+  inv_scan_kernel<<<pl.bgs, 1024, 0, c.stream>>>(pl);
+  note_launch();
+  inv_scan_bg_kernel<<<1, 32, 0, c.stream>>>(pl);
+  note_launch();
+  inv_scatter_kernel<<<gw, 256, 0, c.stream>>>(pl, block_idx);
+  note_launch();
+  const unsigned gt = static_cast<unsigned>((static_cast<int64_t>(pl.bgs) * pl.nb + 255) / 256);
+  inv_tiles_kernel<<<gt, 256, 0, c.stream>>>(pl);
+  note_launch();
+  (void)p;
+  return cudaGetLastError();
+}
+
+cudaError_t launch_attn_block(const ssa_params& p, const BlockPlan& pl, const void* Q,
+                              const CUtensorMap& tmK, const CUtensorMap& tmV, void* partO, void* partL,
+                              const LaunchCtx& c) {
+  BlkArgs a;
+  a.Q = static_cast<const __nv_bfloat16*>(Q);
+  a.tiles = pl.tiles;
+  a.n_tiles = pl.tile_base + pl.bgs;
+  a.entries = pl.entries;
+  a.n_q = p.n_q; a.n_kv = p.n_kv; a.h_q = p.h_q; a.h_kv = p.h_kv; a.topk = p.topk;
+  a.scale_log2 = p.scale * 1.4426950408889634f;
+  a.partO = static_cast<__half*>(partO);
+  a.partL = static_cast<float2*>(partL);
+  a.err = c.err;
+  const int G = p.h_q / p.h_kv;
+  a.partL_stride = (p.topk * G + 3) / 4 * 4;
+  if (p.d != 128) return cudaErrorInvalidValue;
+  if (p.block == 64) {
+    if (G == 2) return run_block<2, 64>(pl, tmK, tmV, a, c);
+    if (G == 4) return run_block<4, 64>(pl, tmK, tmV, a, c);
+    if (G == 8) return run_block<8, 64>(pl, tmK, tmV, a, c);
+  } else if (p.block == 128) {
+    if (G == 2) return run_block<2, 128>(pl, tmK, tmV, a, c);
+    if (G == 4) return run_block<4, 128>(pl, tmK, tmV, a, c);
+    if (G == 8) return run_block<8, 128>(pl, tmK, tmV, a, c);
+  }
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace ssa

@@ -17,7 +17,18 @@ enum WaitSite : uint32_t {
   SITE_ROUTE_EPILOGUE = 0x103,
   SITE_ATTN_PRODUCER = 0x201,
   SITE_ATTN_CONSUMER = 0x202,
+  SITE_MERGE_PRODUCER = 0x211,
+  SITE_MERGE_CONSUMER = 0x212,
   SITE_DRAIN = 0x301,
+  SITE_BLK_A_EMPTY = 0x401,    // block-major tiles: producer
+  SITE_BLK_KV_EMPTY = 0x402,
+  SITE_BLK_KV_FULL = 0x411,    // MMA issuer
+  SITE_BLK_A_FULL = 0x412,
+  SITE_BLK_S_EMPTY = 0x413,
+  SITE_BLK_P_FULL = 0x414,
+  SITE_BLK_O_EMPTY = 0x415,
+  SITE_BLK_S_FULL = 0x421,     // softmax / epilogue
+  SITE_BLK_O_FULL = 0x422,
 };
 
 // A single wait gives up after this long (legitimate waits last microseconds).
@@ -165,6 +176,14 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
 
 __device__ __forceinline__ void tmem_wait_ld() {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+// Orders later uses of registers filled by tcgen05.ld after the preceding
+// tcgen05.wait::ld (both volatile asm, so they keep their relative order).
+template <int N>
+__device__ __forceinline__ void tmem_regs_ready(uint32_t (&r)[N]) {
+#pragma unroll
+  for (int i = 0; i < N; ++i) asm volatile("" : "+r"(r[i]));
 }
 
 // Shared-memory matrix descriptor for a K-major tile written by TMA with

@@ -50,6 +50,41 @@ cudaError_t launch_attn_f32(const ssa_params& p, const void* Q, const void* K, c
                             const int32_t* block_idx, void* O, float* lse, int32_t* bad,
                             const LaunchCtx& c);
 
+// Block-major attention plan: per-block lists of the (query, slot) entries
+// that selected each key block, cut into tiles of 128 / G queries.
+struct BlockPlan {
+  int32_t bgs, n_q, h_kv, nb, block, topk, qpt;
+  int64_t q_offset;
+  int32_t* count;      // [bgs][nb] selections per block
+  int32_t* cursor;     // [bgs][nb] scatter cursors
+  int32_t* blk_off;    // [bgs][nb] first entry of each block within its (batch, kv-head)
+  int32_t* tile_off;   // [bgs][nb] first tile of each block within its (batch, kv-head)
+  int32_t* bg_ents;    // [bgs]
+  int32_t* bg_tiles;   // [bgs]
+  int32_t* ent_base;   // [bgs + 1]
+  int32_t* tile_base;  // [bgs + 1]; tile_base[bgs] = number of tiles
+  int32_t* entries;    // [selections] (query << 5) | slot
+  int4* tiles;         // [max tiles] {batch*h_kv + kv-head, block, first entry, entries}
+};
+
+cudaError_t launch_block_plan(const ssa_params& p, const int32_t* block_idx, const BlockPlan& pl,
+                              const LaunchCtx& c);
+
+// tcgen05 block tiles -> per-(query, head, slot) normalised partial outputs
+// partO [items][topk][G][d] (float16, row-scaled by 2^-e) and partL
+// [items][stride] of (base-2 log-sum-exp, 2^e).
+cudaError_t launch_attn_block(const ssa_params& p, const BlockPlan& pl, const void* Q,
+                              const CUtensorMap& tmK, const CUtensorMap& tmV, void* partO, void* partL,
+                              const LaunchCtx& c);
+
+// Gather attention over the window keys only, merged with the block partials.
+cudaError_t launch_attn_bf16_merge(const ssa_params& p, const CUtensorMap& tmK, const CUtensorMap& tmV,
+                                   const CUtensorMap& tmQ, const void* Q, const int32_t* block_idx,
+                                   const void* partO, const void* partL, void* O, float* lse,
+                                   int32_t* bad, const LaunchCtx& c);
+
+int attn_block_smem_bytes(int block);
+
 // Shared-memory bytes of the tiled router / gather attention (for checks).
 int route_tiled_smem_bytes(int d, int topk);
 int attn_bf16_smem_bytes(int d);

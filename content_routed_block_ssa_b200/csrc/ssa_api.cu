@@ -144,6 +144,48 @@ size_t idx_bytes(const ssa_params& p) {
 
 ssa_status from_cuda(cudaError_t e) { return e == cudaSuccess ? SSA_OK : SSA_ERR_CUDA; }
 
+// Block-major attention applies to long bf16 problems whose query heads
+// fill a 128-row tensor-core tile in groups of G and whose per-row partials
+// fit the merge kernel's item slot.
+bool use_block_attn(const ssa_params& p) {
+  const int G = p.h_q / p.h_kv;
+  return p.dtype == SSA_BF16 && p.d == 128 && (G == 2 || G == 4 || G == 8) && p.topk * G <= 128 &&
+         p.n_q >= 1024 && p.n_q < (1 << 26);
+}
+
+struct AttnLayout {
+  size_t count, cursor, blk_off, tile_off, bg_ents, bg_tiles, ent_base, tile_base, entries, tiles, part_o,
+      part_l, total;
+};
+
+AttnLayout attn_layout(const ssa_params& p) {
+  AttnLayout L{};
+  if (!use_block_attn(p)) return L;
+  const size_t bgs = static_cast<size_t>(p.batch) * p.h_kv;
+  const size_t nb = static_cast<size_t>(nb_of(p));
+  const size_t G = static_cast<size_t>(p.h_q / p.h_kv);
+  const size_t qpt = 128 / G;
+  const size_t sel = bgs * p.n_q * p.topk;
+  const size_t max_tiles = (sel + qpt - 1) / qpt + bgs * nb;
+  const size_t items = bgs * p.n_q;
+  const size_t ls = (p.topk * G + 3) / 4 * 4;
+  size_t off = 0;
+  L.count = off; off += round_up(bgs * nb * 4);
+  L.cursor = off; off += round_up(bgs * nb * 4);
+  L.blk_off = off; off += round_up(bgs * nb * 4);
+  L.tile_off = off; off += round_up(bgs * nb * 4);
+  L.bg_ents = off; off += round_up(bgs * 4);
+  L.bg_tiles = off; off += round_up(bgs * 4);
+  L.ent_base = off; off += round_up((bgs + 1) * 4);
+  L.tile_base = off; off += round_up((bgs + 1) * 4);
+  L.entries = off; off += round_up(sel * 4);
+  L.tiles = off; off += round_up(max_tiles * 16);
+  L.part_o = off; off += round_up(items * p.topk * G * p.d * 2);
+  L.part_l = off; off += round_up(items * ls * 8);
+  L.total = off;
+  return L;
+}
+
 // 2D bf16 map of a [rows, cols] row-major matrix, 64 x box_rows boxes, 128B swizzle.
 bool encode_2d(CUtensorMap* m, const void* base, uint64_t cols, uint64_t rows, uint32_t box_rows) {
   EncodeTiledFn fn = encode_fn();
@@ -215,20 +257,77 @@ ssa_status do_route(const ssa_params& p, const void* Q, const float* mu, const f
   return from_cuda(ssa::launch_route_tiled(p, tmF, tmT, idx, scores, c));
 }
 
+ssa::BlockPlan block_plan(const ssa_params& p, const AttnLayout& L, uint8_t* w) {
+  ssa::BlockPlan pl;
+  pl.bgs = p.batch * p.h_kv;
+  pl.n_q = p.n_q;
+  pl.h_kv = p.h_kv;
+  pl.nb = static_cast<int32_t>(nb_of(p));
+  pl.block = p.block;
+  pl.topk = p.topk;
+  pl.qpt = 128 / (p.h_q / p.h_kv);
+  pl.q_offset = p.q_offset;
+  pl.count = reinterpret_cast<int32_t*>(w + L.count);
+  pl.cursor = reinterpret_cast<int32_t*>(w + L.cursor);
+  pl.blk_off = reinterpret_cast<int32_t*>(w + L.blk_off);
+  pl.tile_off = reinterpret_cast<int32_t*>(w + L.tile_off);
+  pl.bg_ents = reinterpret_cast<int32_t*>(w + L.bg_ents);
+  pl.bg_tiles = reinterpret_cast<int32_t*>(w + L.bg_tiles);
+  pl.ent_base = reinterpret_cast<int32_t*>(w + L.ent_base);
+  pl.tile_base = reinterpret_cast<int32_t*>(w + L.tile_base);
+  pl.entries = reinterpret_cast<int32_t*>(w + L.entries);
+  pl.tiles = reinterpret_cast<int4*>(w + L.tiles);
+  return pl;
+}
+
+struct AttnMaps {
+  CUtensorMap K, V, Q;
+};
+
+bool encode_attn_maps(AttnMaps& m, const ssa_params& p, const void* Q, const void* K, const void* V) {
+  const uint32_t G = static_cast<uint32_t>(p.h_q / p.h_kv);
+  return encode_kv(&m.K, K, p) && encode_kv(&m.V, V, p) &&
+         encode_rows(&m.Q, Q, p.d, static_cast<uint64_t>(p.batch) * p.n_q * p.h_q, G);
+}
+
+// Block-major stages; the caller has checked that the problem qualifies and
+// that `w` holds attn_layout(p).total bytes.
+ssa_status attn_stage_plan(const ssa_params& p, const int32_t* idx, uint8_t* w, const LaunchCtx& c) {
+  const AttnLayout L = attn_layout(p);
+  return from_cuda(ssa::launch_block_plan(p, idx, block_plan(p, L, w), c));
+}
+
+ssa_status attn_stage_blocks(const ssa_params& p, const void* Q, const AttnMaps& m, uint8_t* w, const LaunchCtx& c) {
+  const AttnLayout L = attn_layout(p);
+  return from_cuda(ssa::launch_attn_block(p, block_plan(p, L, w), Q, m.K, m.V, w + L.part_o, w + L.part_l, c));
+}
+
+ssa_status attn_stage_merge(const ssa_params& p, const void* Q, const AttnMaps& m, const int32_t* idx, void* O,
+                            float* lse, int32_t* bad, const uint8_t* w, const LaunchCtx& c) {
+  const AttnLayout L = attn_layout(p);
+  return from_cuda(ssa::launch_attn_bf16_merge(p, m.K, m.V, m.Q, Q, idx, w + L.part_o, w + L.part_l, O, lse,
+                                               bad, c));
+}
+
 ssa_status do_attn(const ssa_params& p, const void* Q, const void* K, const void* V,
-                   const int32_t* idx, void* O, float* lse, int32_t* bad, const LaunchCtx& c) {
+                   const int32_t* idx, void* O, float* lse, int32_t* bad, void* ws, size_t ws_bytes,
+                   const LaunchCtx& c) {
   if (is_empty(p)) return SSA_OK;
   if (p.dtype == SSA_F32) return from_cuda(ssa::launch_attn_f32(p, Q, K, V, idx, O, lse, bad, c));
-  CUtensorMap tmK, tmV, tmQ;
-  const uint32_t G = static_cast<uint32_t>(p.h_q / p.h_kv);
-  if (!encode_kv(&tmK, K, p) || !encode_kv(&tmV, V, p) ||
-      !encode_rows(&tmQ, Q, p.d, static_cast<uint64_t>(p.batch) * p.n_q * p.h_q, G))
-    return SSA_ERR_CUDA;
-  return from_cuda(ssa::launch_attn_bf16(p, tmK, tmV, tmQ, Q, idx, O, lse, bad, c));
+  AttnMaps m;
+  if (!encode_attn_maps(m, p, Q, K, V)) return SSA_ERR_CUDA;
+  const AttnLayout L = attn_layout(p);
+  if (L.total == 0 || !ws || ws_bytes < L.total || !aligned16(ws))
+    return from_cuda(ssa::launch_attn_bf16(p, m.K, m.V, m.Q, Q, idx, O, lse, bad, c));
+  uint8_t* w = static_cast<uint8_t*>(ws);
+  ssa_status st = attn_stage_plan(p, idx, w, c);
+  if (st == SSA_OK) st = attn_stage_blocks(p, Q, m, w, c);
+  if (st == SSA_OK) st = attn_stage_merge(p, Q, m, idx, O, lse, bad, w, c);
+  return st;
 }
 
 struct ForwardLayout {
-  size_t table, mu, sigma, feat, idx, total;
+  size_t table, mu, sigma, feat, idx, attn, total;
 };
 
 ForwardLayout forward_layout(const ssa_params& p) {
@@ -239,6 +338,7 @@ ForwardLayout forward_layout(const ssa_params& p) {
   L.sigma = off; off += sigma_bytes(p);
   L.feat = off; off += features_bytes(p);
   L.idx = off; off += idx_bytes(p);
+  L.attn = off; off += attn_layout(p).total;
   L.total = off;
   return L;
 }
@@ -274,7 +374,8 @@ ssa_status forward_impl(const ssa_params& p, const void* Q, const void* K, const
   st = do_route(p, Q, mu, sg, table, idx, nullptr, features_bytes(p) ? ws + L.feat : nullptr,
                 features_bytes(p), c);
   if (st != SSA_OK) return st;
-  return do_attn(p, Q, K, V, idx, O, lse, nullptr, c);
+  const size_t aw = attn_layout(p).total;
+  return do_attn(p, Q, K, V, idx, O, lse, nullptr, aw ? ws + L.attn : nullptr, aw, c);
 }
 
 }  // namespace
@@ -344,9 +445,14 @@ ssa_status ssa_route_topk(const ssa_params* pp, const void* Q, const float* mu, 
   return do_route(p, Q, mu, sigma, route_table, block_idx, top_scores, ws, ws_bytes, c);
 }
 
+size_t ssa_attn_workspace_size(const ssa_params* p) {
+  if (check_params(p) != SSA_OK) return 0;
+  return attn_layout(*p).total;
+}
+
 ssa_status ssa_sparse_attn(const ssa_params* pp, const void* Q, const void* K, const void* V,
                            const int32_t* block_idx, void* O, float* lse, int32_t* bad_index_count,
-                           void* stream) {
+                           void* ws, size_t ws_bytes, void* stream) {
   ssa_status st = check_params(pp);
   if (st != SSA_OK) return st;
   const ssa_params& p = *pp;
@@ -357,7 +463,55 @@ ssa_status ssa_sparse_attn(const ssa_params* pp, const void* Q, const void* K, c
     return SSA_ERR_INVALID_ARG;
   LaunchCtx c;
   if ((st = make_ctx(stream, c)) != SSA_OK) return st;
-  return do_attn(p, Q, K, V, block_idx, O, lse, bad_index_count, c);
+  return do_attn(p, Q, K, V, block_idx, O, lse, bad_index_count, ws, ws_bytes, c);
+}
+
+// Common checks of the three block-major stage calls.
+ssa_status check_stage(const ssa_params* pp, const void* ws, size_t ws_bytes) {
+  ssa_status st = check_params(pp);
+  if (st != SSA_OK) return st;
+  if (is_empty(*pp)) return SSA_OK;
+  const AttnLayout L = attn_layout(*pp);
+  if (L.total == 0) return SSA_ERR_UNSUPPORTED;
+  if (!ws || ws_bytes < L.total || !aligned16(ws)) return SSA_ERR_WORKSPACE;
+  return SSA_OK;
+}
+
+ssa_status ssa_attn_plan(const ssa_params* pp, const int32_t* block_idx, void* ws, size_t ws_bytes, void* stream) {
+  ssa_status st = check_stage(pp, ws, ws_bytes);
+  if (st != SSA_OK || is_empty(*pp)) return st;
+  if (!block_idx || !aligned16(block_idx)) return SSA_ERR_INVALID_ARG;
+  LaunchCtx c;
+  if ((st = make_ctx(stream, c)) != SSA_OK) return st;
+  return attn_stage_plan(*pp, block_idx, static_cast<uint8_t*>(ws), c);
+}
+
+ssa_status ssa_attn_blocks(const ssa_params* pp, const void* Q, const void* K, const void* V, void* ws,
+                           size_t ws_bytes, void* stream) {
+  ssa_status st = check_stage(pp, ws, ws_bytes);
+  if (st != SSA_OK || is_empty(*pp)) return st;
+  if (!Q || !K || !V || !aligned16(Q) || !aligned16(K) || !aligned16(V)) return SSA_ERR_INVALID_ARG;
+  LaunchCtx c;
+  if ((st = make_ctx(stream, c)) != SSA_OK) return st;
+  AttnMaps m;
+  if (!encode_attn_maps(m, *pp, Q, K, V)) return SSA_ERR_CUDA;
+  return attn_stage_blocks(*pp, Q, m, static_cast<uint8_t*>(ws), c);
+}
+
+ssa_status ssa_attn_merge(const ssa_params* pp, const void* Q, const void* K, const void* V,
+                          const int32_t* block_idx, void* O, float* lse, int32_t* bad_index_count, const void* ws,
+                          size_t ws_bytes, void* stream) {
+  ssa_status st = check_stage(pp, ws, ws_bytes);
+  if (st != SSA_OK || is_empty(*pp)) return st;
+  if (!Q || !K || !V || !block_idx || !O || !aligned16(Q) || !aligned16(K) || !aligned16(V) ||
+      !aligned16(block_idx) || !aligned16(O) || (reinterpret_cast<uintptr_t>(lse) & 3u) ||
+      (reinterpret_cast<uintptr_t>(bad_index_count) & 3u))
+    return SSA_ERR_INVALID_ARG;
+  LaunchCtx c;
+  if ((st = make_ctx(stream, c)) != SSA_OK) return st;
+  AttnMaps m;
+  if (!encode_attn_maps(m, *pp, Q, K, V)) return SSA_ERR_CUDA;
+  return attn_stage_merge(*pp, Q, m, block_idx, O, lse, bad_index_count, static_cast<const uint8_t*>(ws), c);
 }
 
 size_t ssa_workspace_size(const ssa_params* p) {

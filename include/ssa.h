@@ -157,20 +157,58 @@ SSA_API ssa_status ssa_route_topk(const ssa_params* p, const void* Q, const floa
                           const float* sigma, const void* route_table, int32_t* block_idx,
                           float* top_scores, void* ws, size_t ws_bytes, void* stream);
 
+/* Bytes of device workspace that lets ssa_sparse_attn run block-major (0 when
+ * the problem always runs the per-query gather). */
+SSA_API size_t ssa_attn_workspace_size(const ssa_params* p);
+
 /*
  * Steps (ii)+(iii): exact softmax attention of every query head over the
  * union of its kv-head's selected blocks and the causal window
- * [opening section, (ii) and (iii)], with an online (running max / running
- * sum) softmax.  block_idx entries that are not -1 must be ascending,
- * distinct and fully visible; any other entry is skipped and, when
- * bad_index_count is not NULL, counted into that device int32 (atomically
- * added, not reset).
+ * [opening section, (ii) and (iii)].  block_idx entries that are not -1 are
+ * used when they are fully visible and larger than every earlier in-range
+ * entry of their row (ascending, distinct); any other entry is skipped and,
+ * when bad_index_count is not NULL, counted into that device int32
+ * (atomically added, not reset).
+ * Two evaluations give the same result up to rounding: with a workspace of
+ * ssa_attn_workspace_size(p) bytes (bf16 problems with n_q >= 1024, d = 128,
+ * G in {2, 4, 8}, topk * G <= 128) the selections are inverted and every
+ * selected key block is multiplied once against all queries that chose it
+ * on the tensor cores, then merged with the window per query; with ws NULL
+ * (or too small) every (query, kv-head) gathers its own blocks.
  *   O            device output [b, n_q, h_q, d] of dtype
  *   lse          device float32 output, may be NULL
+ *   ws, ws_bytes device workspace, may be NULL / 0
  */
 SSA_API ssa_status ssa_sparse_attn(const ssa_params* p, const void* Q, const void* K, const void* V,
-                           const int32_t* block_idx, void* O, float* lse,
-                           int32_t* bad_index_count, void* stream);
+                                   const int32_t* block_idx, void* O, float* lse,
+                                   int32_t* bad_index_count, void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * The block-major evaluation of ssa_sparse_attn as three calls, for callers
+ * that schedule or time the stages themselves.  Made in this order on one
+ * stream with one workspace (ssa_attn_workspace_size(p) bytes, 16-byte
+ * aligned; its contents are private to the library and live from the plan
+ * call to the merge call), they give exactly the bytes ssa_sparse_attn gives
+ * with that workspace.
+ *   ssa_attn_plan    inverts block_idx: the valid (query, slot) entries of
+ *                    every (batch, kv-head, key block), in tiles of 128 / G
+ *                    queries;
+ *   ssa_attn_blocks  per tile, S = Q_tile K_c^T and O = P V_c on the tensor
+ *                    cores; writes each entry's normalised partial output
+ *                    and base-2 log-sum-exp into the workspace;
+ *   ssa_attn_merge   per (query, kv-head): the window keys outside the
+ *                    selected blocks, merged with the block partials into O
+ *                    and lse; counts skipped entries as ssa_sparse_attn does.
+ * Problems that do not qualify return SSA_ERR_UNSUPPORTED, a missing or
+ * short workspace SSA_ERR_WORKSPACE; both before any launch.
+ */
+SSA_API ssa_status ssa_attn_plan(const ssa_params* p, const int32_t* block_idx, void* ws, size_t ws_bytes,
+                                 void* stream);
+SSA_API ssa_status ssa_attn_blocks(const ssa_params* p, const void* Q, const void* K, const void* V,
+                                   void* ws, size_t ws_bytes, void* stream);
+SSA_API ssa_status ssa_attn_merge(const ssa_params* p, const void* Q, const void* K, const void* V,
+                                  const int32_t* block_idx, void* O, float* lse, int32_t* bad_index_count,
+                                  const void* ws, size_t ws_bytes, void* stream);
 
 /*
  * ssa_route_topk without a caller workspace.  No counterpart in the paper:
@@ -196,8 +234,9 @@ SSA_API size_t ssa_workspace_size(const ssa_params* p);
 
 /*
  * The whole layer: ssa_block_summary, ssa_route_topk and ssa_sparse_attn on
- * `stream`, with the summaries, routing features and block indices carved
- * from the caller's workspace (at least ssa_workspace_size(p) bytes).
+ * `stream`, with the summaries, routing features, block indices and the
+ * attention workspace carved from the caller's workspace (at least
+ * ssa_workspace_size(p) bytes).
  */
 SSA_API ssa_status ssa_forward(const ssa_params* p, const void* Q, const void* K, const void* V,
                        void* O, float* lse, void* ws, size_t ws_bytes, void* stream);

@@ -48,11 +48,16 @@ def gpu_route(p, Q, mu, sig, tab):
     return idx, sc
 
 
-def gpu_attn(p, Q, K, V, idx):
+def gpu_attn(p, Q, K, V, idx, workspace=True):
+    """Sparse attention through the C ABI.  With ``workspace`` the call gets
+    the attention workspace, so problems that qualify run block-major;
+    without it every problem takes the per-row gather path."""
     O_ = torch.empty_like(Q)
     lse = torch.empty(Q.shape[:3], dtype=torch.float32, device=Q.device)
     bad = torch.zeros(1, dtype=torch.int32, device=Q.device)
-    ssa.ssa_sparse_attn(p, Q, K, V, idx, O_, lse, bad)
+    nbytes = ssa.ssa_attn_workspace_size(p) if workspace else 0
+    ws = ssa.byte_buffer(nbytes, Q.device) if nbytes else None
+    ssa.ssa_sparse_attn(p, Q, K, V, idx, O_, lse, bad, ws)
     return O_, lse, bad
 
 

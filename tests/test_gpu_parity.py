@@ -27,6 +27,9 @@ CASES = {
     "bf16_mha_d128_b64_k32": Workload("c", 102, 1, 2112, 2, 2, 128, "bf16", 64, "diag", 32, 128, 8, "per_head"),
     "bf16_gqa8_d128_b128_k16": Workload("c", 103, 1, 3072, 8, 1, 128, "bf16", 128, "diag", 16, 256, 12, "total",
                                         clustered=True),
+    "bf16_gqa4_d128_b64_k32_b2": Workload("c", 109, 2, 2560, 8, 2, 128, "bf16", 64, "diag", 32, 256, 8, "total",
+                                          clustered=True),
+    "bf16_gqa2_d128_b64_w100": Workload("c", 113, 1, 2304, 4, 2, 128, "bf16", 64, "diag", 16, 100, 6, "per_head"),
     "bf16_gqa2_d64_b64": Workload("c", 104, 1, 1024, 4, 2, 64, "bf16", 64, "diag", 4, 64, 6, "total"),
     "bf16_mha_d64_b128_w200": Workload("c", 105, 1, 1280, 1, 1, 64, "bf16", 128, "diag", 8, 200, 4, "total"),
     "f32_full_d64": Workload("c", 106, 1, 1024, 1, 1, 64, "f32", 64, "full", 8, 64, 8, "total"),
@@ -289,3 +292,95 @@ def test_empty_problem_launches_nothing_and_small_workspace_is_rejected():
         ssa.ssa_forward(p, Q, K, V, O_, None, small)
     assert e.value.status == ssa.SSA_ERR_WORKSPACE
     assert ssa.ssa_launch_count() == before
+
+
+# Problems the block-major attention takes (bf16, d = 128, G in {2, 4, 8},
+# k * G <= 128, at least 1024 query rows) when it is given its workspace.
+BLOCK_MAJOR = [n for n, w in CASES.items()
+               if w.dtype == "bf16" and w.d == 128 and w.h_q // w.h_kv in (2, 4, 8)
+               and w.topk * (w.h_q // w.h_kv) <= 128 and w.n_q >= 1024]
+
+
+def test_block_major_cases_exist():
+    assert len(BLOCK_MAJOR) >= 3
+    for n in BLOCK_MAJOR:
+        assert ssa.ssa_attn_workspace_size(params(problem_dict(CASES[n]))) > 0
+    assert ssa.ssa_attn_workspace_size(params(problem_dict(CASES["bf16_mha_d128_b64_k32"]))) == 0
+
+
+@pytest.mark.parametrize("name", BLOCK_MAJOR)
+def test_block_major_attention_matches_oracle_and_gather(name):
+    c = case(name)
+    p = params(c["pd"])
+    Q, K, V = to_dev(c["Q"], c["K"], c["V"])
+    idx = torch.from_numpy(c["ref"]["block_idx"].astype(np.int32)).cuda()
+    n0 = ssa.ssa_launch_count()
+    Ob, lb, bad_b = gpu_attn(p, Q, K, V, idx, workspace=True)
+    n1 = ssa.ssa_launch_count()
+    Og, lg, bad_g = gpu_attn(p, Q, K, V, idx, workspace=False)
+    n2 = ssa.ssa_launch_count()
+    check_no_device_error()
+    assert n2 - n1 == 1 and n1 - n0 > 1        # gather: one kernel; block-major: plan, tiles, merge
+    assert int(bad_b.item()) == 0 and int(bad_g.item()) == 0
+    for got, lse in ((Ob, lb), (Og, lg)):
+        max_abs, rel, ok = compare_out(as_np(got), c["ref"]["O"], "bf16")
+        assert ok, (max_abs, rel)
+        np.testing.assert_allclose(lse.cpu().numpy(), c["ref"]["lse"], rtol=0, atol=2e-3)
+    # each path is within the bf16 bound of the oracle, so the two are within twice it
+    assert float((Ob.float() - Og.float()).abs().max()) <= 2 * 2e-2
+
+
+def test_block_major_with_query_offset():
+    """A chunk of query rows [n - 1024, n) at q_offset = n - 1024 gives the
+    full problem's last 1024 rows."""
+    c = case("bf16_gqa4_d128_b64_k32_b2")
+    w = c["w"]
+    m = 1024
+    pd = {**c["pd"], "n_q": m, "q_offset": w.n - m}
+    p = params(pd)
+    Q = c["Q"][:, w.n - m:].contiguous()
+    Qd, K, V = to_dev(Q, c["K"], c["V"])
+    idx = torch.from_numpy(np.ascontiguousarray(c["ref"]["block_idx"][:, w.n - m:]).astype(np.int32)).cuda()
+    assert ssa.ssa_attn_workspace_size(p) > 0
+    O_, lse, bad = gpu_attn(p, Qd, K, V, idx)
+    check_no_device_error()
+    assert int(bad.item()) == 0
+    max_abs, rel, ok = compare_out(as_np(O_), c["ref"]["O"][:, w.n - m:], "bf16")
+    assert ok, (max_abs, rel)
+    np.testing.assert_allclose(lse.cpu().numpy(), c["ref"]["lse"][:, w.n - m:], rtol=0, atol=2e-3)
+
+
+def test_block_major_without_selections_is_window_attention():
+    """Every block_idx entry -1: no block tile runs and each row attends to
+    its causal window alone."""
+    c = case("bf16_gqa8_d128_b128_k16")
+    op = c["op"]
+    p = params(c["pd"])
+    Q, K, V = to_dev(c["Q"], c["K"], c["V"])
+    none = np.full(c["ref"]["block_idx"].shape, -1, dtype=np.int32)
+    O_, lse, bad = gpu_attn(p, Q, K, V, torch.from_numpy(none).cuda())
+    check_no_device_error()
+    assert int(bad.item()) == 0
+    rows = [(0, i) for i in range(0, op.n_q, 5)]
+    Oref, Lref = O.attention(c["Qn"], c["Kn"], c["Vn"], none, op, rows=rows)
+    got = as_np(O_)
+    ri = [i for _, i in rows]
+    max_abs, rel, ok = compare_out(got[0, ri], Oref[0, ri], "bf16")
+    assert ok, (max_abs, rel)
+
+
+def test_block_major_stages_equal_single_call():
+    c = case("bf16_gqa4_d128_b64_k32_b2")
+    p = params(c["pd"])
+    Q, K, V = to_dev(c["Q"], c["K"], c["V"])
+    idx = torch.from_numpy(c["ref"]["block_idx"].astype(np.int32)).cuda()
+    O1, l1, b1 = gpu_attn(p, Q, K, V, idx)
+    ws = ssa.byte_buffer(ssa.ssa_attn_workspace_size(p))
+    O2 = torch.empty_like(Q)
+    l2 = torch.empty(Q.shape[:3], dtype=torch.float32, device="cuda")
+    b2 = torch.zeros(1, dtype=torch.int32, device="cuda")
+    ssa.ssa_attn_plan(p, idx, ws)
+    ssa.ssa_attn_blocks(p, Q, K, V, ws)
+    ssa.ssa_attn_merge(p, Q, K, V, idx, O2, l2, b2, ws)
+    check_no_device_error()
+    assert torch.equal(O1, O2) and torch.equal(l1, l2) and int(b2.item()) == int(b1.item()) == 0

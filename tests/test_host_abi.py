@@ -77,7 +77,7 @@ def test_invalid_and_unsupported_params(kw, code):
     dummy = 256   # any non-null, 16-byte-aligned value: validation fails first
     assert ssa.lib.ssa_block_summary(C.byref(p), dummy, None, None, dummy, None) == code
     assert ssa.lib.ssa_forward(C.byref(p), dummy, dummy, dummy, dummy, None, dummy, 1 << 30, None) == code
-    assert ssa.lib.ssa_sparse_attn(C.byref(p), dummy, dummy, dummy, dummy, dummy, None, None, None) == code
+    assert ssa.lib.ssa_sparse_attn(C.byref(p), dummy, dummy, dummy, dummy, dummy, None, None, None, 0, None) == code
     assert ssa.lib.ssa_workspace_size(C.byref(p)) == 0
 
 
@@ -88,7 +88,7 @@ def test_null_and_misaligned_pointers_rejected():
     assert ssa.lib.ssa_block_summary(C.byref(p), 258, None, None, 256, None) == ssa.SSA_ERR_INVALID_ARG
     assert ssa.lib.ssa_route_topk(C.byref(p), 256, None, None, None, 256, None, None, 0, None) == \
         ssa.SSA_ERR_INVALID_ARG                           # bf16 needs the route table
-    assert ssa.lib.ssa_sparse_attn(C.byref(p), 256, 256, 256, None, 256, None, None, None) == \
+    assert ssa.lib.ssa_sparse_attn(C.byref(p), 256, 256, 256, None, 256, None, None, None, 0, None) == \
         ssa.SSA_ERR_INVALID_ARG
     assert ssa.lib.ssa_forward(C.byref(p), 256, 256, 264, 256, None, 256, 1 << 30, None) == \
         ssa.SSA_ERR_INVALID_ARG
@@ -100,7 +100,7 @@ def test_empty_problems_are_valid_noops():
     for kw in (dict(batch=0), dict(n_q=0, q_offset=0)):
         p = good(**kw)
         assert ssa.lib.ssa_forward(C.byref(p), None, None, None, None, None, None, 0, None) == ssa.SSA_OK
-        assert ssa.lib.ssa_sparse_attn(C.byref(p), None, None, None, None, None, None, None, None) == ssa.SSA_OK
+        assert ssa.lib.ssa_sparse_attn(C.byref(p), None, None, None, None, None, None, None, None, 0, None) == ssa.SSA_OK
         assert ssa.lib.ssa_route_topk(C.byref(p), None, None, None, None, None, None, None, 0, None) == ssa.SSA_OK
 
 
@@ -120,3 +120,32 @@ def test_workspace_sizes():
     assert ssa.ssa_workspace_size(f32) == rnd(2 * nb * 64 * 4) + rnd(2 * nb * 64 * 64 * 4) + rnd(128 * 2 * 4 * 4)
     h = ssa.ssa_hostio_buffer_size(p)
     assert h > ssa.ssa_workspace_size(p)
+
+
+def test_block_major_workspace_and_stage_checks():
+    # qualifies: bf16, d = 128, G = 4, k * G = 32, n_q >= 1024
+    p = good(n_q=2048, n_kv=2048, topk=8, h_q=8, h_kv=2)
+    aw = ssa.ssa_attn_workspace_size(p)
+    assert aw > 0
+    base = ssa.ssa_workspace_size(good(n_q=2048, n_kv=2048, topk=8, h_q=8, h_kv=2, d=64))
+    assert ssa.ssa_workspace_size(p) >= aw
+    # the partial outputs dominate: one bf16 row of d per (query, kv-head, slot, head)
+    assert aw >= 2048 * 2 * 8 * 4 * 128 * 2
+    del base
+    # does not qualify: too few rows, G = 1, d = 64, k * G > 128, float32
+    for kw in (dict(n_q=1000, n_kv=1024), dict(h_q=2, h_kv=2), dict(d=64),
+               dict(topk=32, h_q=16, h_kv=2), dict(dtype="f32", h_q=2, h_kv=1)):
+        q = good(**{**dict(n_q=2048, n_kv=2048), **kw})
+        assert ssa.ssa_attn_workspace_size(q) == 0, kw
+        assert ssa.lib.ssa_attn_plan(C.byref(q), 256, 256, 1 << 40, None) == ssa.SSA_ERR_UNSUPPORTED
+    # staged calls without (or with too little) workspace are refused before any launch
+    before = ssa.ssa_launch_count()
+    assert ssa.lib.ssa_attn_plan(C.byref(p), 256, None, 0, None) == ssa.SSA_ERR_WORKSPACE
+    assert ssa.lib.ssa_attn_blocks(C.byref(p), 256, 256, 256, 256, aw - 16, None) == ssa.SSA_ERR_WORKSPACE
+    assert ssa.lib.ssa_attn_merge(C.byref(p), 256, 256, 256, 256, 256, None, None, 264, aw, None) == \
+        ssa.SSA_ERR_WORKSPACE                                  # misaligned
+    assert ssa.lib.ssa_attn_plan(C.byref(p), None, 256, aw, None) == ssa.SSA_ERR_INVALID_ARG
+    assert ssa.ssa_launch_count() == before
+    # empty problems are no-ops for every stage
+    e = good(n_q=0, q_offset=0)
+    assert ssa.lib.ssa_attn_merge(C.byref(e), None, None, None, None, None, None, None, None, 0, None) == ssa.SSA_OK
