@@ -175,21 +175,31 @@ def attended_keys(idx, w):
 
 
 def block_major_counts(idx, w):
-    """Valid (query, kv-head, slot) selections and distinct selected
-    (batch, kv-head, block) pairs, by the same validity rule as the kernels
-    (in range, larger than every earlier in-range entry of the row)."""
+    """Slots of the block-major attention, by the kernels' rule: the used
+    block_idx entries (in range, larger than every earlier in-range entry of
+    the row) plus the window blocks no used entry selects.  Returns the number
+    of slots and of distinct (batch, kv-head, block) lists they fall in."""
     nb = w.n // w.block
+    B = w.block
     pos = torch.arange(w.n_q, device=idx.device, dtype=torch.int64).view(1, -1, 1, 1) + w.q_offset
-    nvis = torch.clamp((pos + 1) // w.block, max=nb)
+    nvis = torch.clamp((pos + 1) // B, max=nb)
     v = idx.to(torch.int64)
     inr = (v >= 0) & (v < nvis)
     run = torch.cummax(torch.where(inr, v, torch.full_like(v, -1)), dim=-1).values
     prev = torch.cat([torch.full_like(run[..., :1], -1), run[..., :-1]], dim=-1)
     valid = inr & (v > prev)
-    n_entries = int(valid.sum().item())
-    b_, i_, g_, j_ = torch.nonzero(valid, as_tuple=True)
-    key = (b_ * w.h_kv + g_) * nb + v[b_, i_, g_, j_]
-    n_blocks = int(torch.unique(key).numel())
+    wt = (w.window - 1 + B - 1) // B + 1
+    lo = torch.clamp(pos - w.window + 1, min=0)
+    wb = lo // B + torch.arange(wt, device=idx.device).view(1, 1, 1, -1)          # [1, n, 1, wt]
+    in_win = wb <= pos // B
+    sel = torch.where(valid, v, torch.full_like(v, -1))
+    covered = (sel.unsqueeze(-1) == wb.unsqueeze(-2)).any(-2)                    # [b, n, h, wt]
+    win = in_win & ~covered
+    n_entries = int(valid.sum().item()) + int(win.sum().item())
+    bgi = (torch.arange(w.batch, device=idx.device).view(-1, 1, 1, 1) * w.h_kv
+           + torch.arange(w.h_kv, device=idx.device).view(1, 1, -1, 1))
+    keys = torch.cat([(bgi * nb + sel)[valid], (bgi * nb + wb.expand_as(win))[win]])
+    n_blocks = int(torch.unique(keys).numel())
     return n_entries, n_blocks
 
 
@@ -208,19 +218,17 @@ def algorithmic_work(w, idx):
     out = dict(summary_bytes=summary_bytes, route_flops=route_flops, attn_bytes=gathered + qo,
                gathered_bytes=gathered, attn_flops=attn_flops, mean_keys=float(S.float().mean().item()))
     if w.dtype == "bf16":
-        # block-major stages: per valid selection the tile kernel reads the
-        # query heads' rows and writes one partial row + log-sum-exp per head,
-        # and reads each distinct selected block's K_c, V_c once; the merge
-        # reads Q, the partials and the window keys outside the selected
-        # blocks and writes O and lse
+        # block-major stages, per slot (a used selected block or an uncovered
+        # window block of a row): the tile kernel reads the G query rows and
+        # writes G partial rows + (log-sum-exp, scale), and reads each distinct
+        # key block's K, V once; the merge reads the slot partials and writes
+        # O and lse per row
         ne, nblk = block_major_counts(idx, w)
         items = w.batch * w.n_q * w.h_kv
-        window_keys = float(S.sum().item()) - ne * w.block
         out["blocks_bytes"] = ne * G * (w.d * 2 * 2 + 8) + nblk * 2 * w.block * w.d * 2
         out["blocks_flops"] = 4.0 * ne * G * w.block * w.d
-        out["merge_bytes"] = (items * (G * w.d * 2 * 2 + G * 4 + w.topk * 4) + ne * G * (w.d * 2 + 8)
-                              + window_keys * 2 * w.d * 2)
-        out["plan_bytes"] = items * w.topk * 4 * 2 + ne * 4 * 2
+        out["merge_bytes"] = items * (G * w.d * 2 + G * 4 + w.topk * 4) + ne * G * (w.d * 2 + 8)
+        out["plan_bytes"] = items * w.topk * 4 * 2 + ne * 4
         out["n_entries"] = ne
         out["n_blocks"] = nblk
     return out
@@ -251,7 +259,7 @@ def run_ours(w, steps, warmup, ws, rank, with_e2e=True):
                   ("route", lambda: ssa.ssa_route_topk(p, Q, None, None, tab, idx, None, rws)),
                   ("attn_plan", lambda: ssa.ssa_attn_plan(p, idx, aws)),
                   ("attn_blocks", lambda: ssa.ssa_attn_blocks(p, Q, K, V, aws)),
-                  ("attn_merge", lambda: ssa.ssa_attn_merge(p, Q, K, V, idx, O, lse, None, aws))]
+                  ("attn_merge", lambda: ssa.ssa_attn_merge(p, idx, O, lse, None, aws))]
     else:
         stages = [("summary", lambda: ssa.ssa_block_summary(p, K, None, None, tab)),
                   ("route", lambda: ssa.ssa_route_topk(p, Q, None, None, tab, idx, None, rws)),
@@ -317,8 +325,8 @@ def run_ours(w, steps, warmup, ws, rank, with_e2e=True):
                 clocks=clk.summary(), e2e=e2e)
 
 
-KERNEL_NAMES = {"summary": "summary_diag_kernel", "route": "route_tiled_kernel", "attn_plan": "inv_*_kernel (5)",
-                "attn_blocks": "attn_block_kernel", "attn_merge": "attn_bf16_kernel (merge)",
+KERNEL_NAMES = {"summary": "summary_diag_kernel", "route": "route_tiled_kernel", "attn_plan": "inv_*_kernel (6)",
+                "attn_blocks": "attn_block_kernel", "attn_merge": "attn_merge_kernel",
                 "attn_gather": "attn_bf16_kernel"}
 
 

@@ -58,7 +58,7 @@ def _load():
         "ssa_attn_workspace_size": (sz, [P]),
         "ssa_attn_plan": (i32, [P, vp, vp, sz, vp]),
         "ssa_attn_blocks": (i32, [P, vp, vp, vp, vp, sz, vp]),
-        "ssa_attn_merge": (i32, [P, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]),
+        "ssa_attn_merge": (i32, [P, vp, vp, vp, vp, vp, sz, vp]),
         "ssa_sparse_attn": (i32, [P, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]),
         "ssa_workspace_size": (sz, [P]),
         "ssa_forward": (i32, [P, vp, vp, vp, vp, vp, vp, sz, vp]),
@@ -171,9 +171,9 @@ def ssa_attn_blocks(p, Q, K, V, ws, stream=None):
            "ssa_attn_blocks")
 
 
-def ssa_attn_merge(p, Q, K, V, block_idx, O, lse, bad_index_count, ws, stream=None):
-    _check(lib.ssa_attn_merge(C.byref(p), _ptr(Q), _ptr(K), _ptr(V), _ptr(block_idx), _ptr(O), _ptr(lse),
-                              _ptr(bad_index_count), _ptr(ws), _nbytes(ws), _stream(stream)), "ssa_attn_merge")
+def ssa_attn_merge(p, block_idx, O, lse, bad_index_count, ws, stream=None):
+    _check(lib.ssa_attn_merge(C.byref(p), _ptr(block_idx), _ptr(O), _ptr(lse), _ptr(bad_index_count), _ptr(ws),
+                              _nbytes(ws), _stream(stream)), "ssa_attn_merge")
 
 
 def ssa_sparse_attn(p, Q, K, V, block_idx, O, lse=None, bad_index_count=None, ws=None, stream=None):

@@ -18,7 +18,6 @@
 //
 // float32 kernel: one CTA per item, SIMT, same tile list.
 #include <cuda_bf16.h>
-#include <cuda_fp16.h>
 #include <math.h>
 
 #include "common.cuh"
@@ -42,30 +41,20 @@ struct AttnArgs {
   float scale_log2;   // scale * log2(e)
   float scale;
   uint32_t* err;
-  // merge mode: per-(item, slot, head) partials of the selected blocks
-  const __half* partO;          // [items][topk][G][d], normalised, times 2^-e
-  const float2* partL;          // [items][partL_stride]: (base-2 log-sum-exp, 2^e)
-  int32_t partL_stride;
 };
 
-template <int D, bool MRG = false>
+template <int D>
 struct AttnCfg {
   static constexpr int HALF = 64 * 64 * 2;            // 64 keys x 64 dims bf16 (8 KB)
   static constexpr int KBYTES = (D / 64) * HALF;
   static constexpr int STAGE = 2 * KBYTES;            // K then V of one 64-key tile
-  static constexpr int NS = MRG ? 3 : ((D == 128) ? 6 : 12);   // tile ring
+  static constexpr int NS = (D == 128) ? 6 : 12;      // tile ring
   static constexpr int MAXT = 32 * 2 + 66;            // selected tiles (k <= 32, <= 2 per block) + window tiles
-  // item slot: Q tile (<= 8 heads, as D/64 boxes of G x 64), tile list, meta;
-  // merge mode adds the item's block partials (topk * G <= 128 rows of d)
+  // item slot: Q tile (<= 8 heads, as D/64 boxes of G x 64), tile list, meta
   static constexpr int QBYTES = 8 * D * 2;
-  static constexpr int PART_O = 4096;                 // offset of the partial outputs
-  static constexpr int PART_OBYTES = 128 * D * 2;
-  static constexpr int PART_L = PART_O + PART_OBYTES;
-  static constexpr int PART_LBYTES = 128 * 8;
-  static constexpr int MERGE_W = (128 + 32 + 8) * 4;   // merge weights (slot tail)
-  static constexpr int SLOT = MRG ? (PART_L + PART_LBYTES + MERGE_W + 1023) / 1024 * 1024 : 4096;
+  static constexpr int SLOT = 4096;
   static constexpr int MERGE = 4 * 8 * D * 4 + 4 * 8 * 2 * 4;
-  static constexpr int NSLOT = MRG ? 2 : 3;
+  static constexpr int NSLOT = 3;
   static constexpr int NBAR = 2 * NS + 2 * NSLOT;
   static constexpr int SMEM = 1024 + NS * STAGE + NSLOT * SLOT + MERGE + NBAR * 8 + 32;
   static_assert(QBYTES + MAXT * 4 + 64 <= SLOT, "item slot too small");
@@ -74,7 +63,6 @@ struct AttnCfg {
 struct ItemMeta {
   int64_t pos, lo, qrow;
   int32_t n_sub, ns;
-  uint32_t selmask;   // merge mode: slots holding a block partial
 };
 
 __device__ __forceinline__ void named_bar_consumers() {
@@ -88,15 +76,13 @@ __device__ __forceinline__ void named_bar_consumers() {
 // 64-key tile is shared by the four warps, 16 keys each, so a ring stage is
 // released after a quarter of the tile's work and the rest of the ring stays
 // in flight; two groups give each SM sub-partition two warps to overlap.
-template <int D, int G, bool MRG>
+template <int D, int G>
 __global__ void __launch_bounds__(288, 1)
     attn_bf16_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                      const __grid_constant__ CUtensorMap tmQ, const AttnArgs a) {
-  using C = AttnCfg<D, MRG>;
+  using C = AttnCfg<D>;
   constexpr int KS = D / 16;    // k-steps over dims
   constexpr int MT = D / 16;    // dim m-tiles of O^T
-  constexpr uint32_t kSiteP = MRG ? SITE_MERGE_PRODUCER : SITE_ATTN_PRODUCER;
-  constexpr uint32_t kSiteC = MRG ? SITE_MERGE_CONSUMER : SITE_ATTN_CONSUMER;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* stages = smem;
@@ -151,48 +137,27 @@ __global__ void __launch_bounds__(288, 1)
       const ItemTiles it = item_tiles_v(v, a.topk, a.q_offset + i, a.nb, a.block, a.window);
       const int sl = local % C::NSLOT;
       bool w_ok = true;
-      if (lane == 0) w_ok = mbar_wait(&item_empty[sl], ((local / C::NSLOT) & 1) ^ 1, a.err, kSiteP);
+      if (lane == 0) w_ok = mbar_wait(&item_empty[sl], ((local / C::NSLOT) & 1) ^ 1, a.err, SITE_ATTN_PRODUCER);
       w_ok = __shfl_sync(0xFFFFFFFFu, w_ok, 0);
       if (!w_ok) return false;
       int32_t* tl = slot_tiles(sl);
-      // merge mode lists only the window tiles; the selected blocks arrive
-      // as partials
-      const int n_list = MRG ? __popcll(it.winmask) : it.n_sub;
-      for (int j0 = 0; j0 < n_list; j0 += 32) {
+      for (int j0 = 0; j0 < it.n_sub; j0 += 32) {
         const int j = j0 + lane;
-        int64_t k0;
-        if (MRG) {
-          const int wb = nth_bit64(it.winmask, j);
-          k0 = (it.win_t0 + (wb < 0 ? 0 : wb)) * 64;
-        } else {
-          k0 = tile_key0_lane(it, j, a.block);
-        }
-        if (j < n_list) tl[j] = static_cast<int32_t>(k0);
+        const int64_t k0 = tile_key0_lane(it, j, a.block);
+        if (j < it.n_sub) tl[j] = static_cast<int32_t>(k0);
       }
       if (lane == 0) {
         ItemMeta* m = slot_meta(sl);
         m->pos = it.pos;
         m->lo = it.lo;
         m->qrow = (b * a.n_q + i) * a.h_q + static_cast<int64_t>(g) * G;
-        m->n_sub = n_list;
-        m->ns = MRG ? 0 : it.n_sel * it.spb;
-        m->selmask = it.selmask;
+        m->n_sub = it.n_sub;
+        m->ns = it.n_sel * it.spb;
         if (a.bad && it.n_bad) atomicAdd(a.bad, it.n_bad);
       }
       __syncwarp();
       if (lane == 0) {
-        const int pbytes = MRG ? a.topk * G * D * 2 : 0;
-        const int lbytes = MRG ? a.partL_stride * 8 : 0;
-        mbar_arrive_expect_tx(&item_full[sl], G * D * 2 + pbytes + lbytes);
-        if (MRG) {
-          const int64_t item = u;
-          const __half* po = a.partO + item * a.topk * G * D;
-          const float2* pl = a.partL + item * a.partL_stride;
-          asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
-                       ::"r"(smem_u32(slot_q(sl) + C::PART_O)), "l"(po), "r"(pbytes), "r"(smem_u32(&item_full[sl])) : "memory");
-          asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
-                       ::"r"(smem_u32(slot_q(sl) + C::PART_L)), "l"(pl), "r"(lbytes), "r"(smem_u32(&item_full[sl])) : "memory");
-        }
+        mbar_arrive_expect_tx(&item_full[sl], G * D * 2);
         const int qrow = static_cast<int>((b * a.n_q + i) * a.h_q + static_cast<int64_t>(g) * G);
 #pragma unroll
         for (int hf = 0; hf < D / 64; ++hf) tma_load_2d(slot_q(sl) + hf * G * 128, &tmQ, &item_full[sl], hf * 64, qrow);
@@ -205,8 +170,14 @@ __global__ void __launch_bounds__(288, 1)
       const int v0 = lane < a.topk ? __ldg(sel_ptr(blockIdx.x) + lane) : -1;
       ok = setup(0, v0);
     }
-    // the tile gathers of item `local`
-    auto gather = [&](int local) -> bool {
+    for (int local = 0; local < n_local && ok; ++local) {
+      if (local + 1 < n_local) {
+        const int v = vnext;
+        vnext = (local + 2 < n_local && lane < a.topk)
+                    ? __ldg(sel_ptr(blockIdx.x + static_cast<int64_t>(local + 2) * gridDim.x) + lane) : -1;
+        ok = setup(local + 1, v);
+        if (!ok) break;
+      }
       const int64_t u = blockIdx.x + static_cast<int64_t>(local) * gridDim.x;
       const int64_t bg = u / a.n_q;
       const int g = static_cast<int>(bg % a.h_kv);
@@ -214,11 +185,10 @@ __global__ void __launch_bounds__(288, 1)
       const int sl = local % C::NSLOT;
       const int32_t* tl = slot_tiles(sl);
       const int n_sub = slot_meta(sl)->n_sub;
-      bool g_ok = true;
       if (lane == 0) {
         for (int j = 0; j < n_sub; ++j) {
           const int s = cnt % C::NS;
-          if (!mbar_wait(&empty[s], ((cnt / C::NS) & 1) ^ 1, a.err, kSiteP)) { g_ok = false; break; }
+          if (!mbar_wait(&empty[s], ((cnt / C::NS) & 1) ^ 1, a.err, SITE_ATTN_PRODUCER)) { ok = false; break; }
           uint8_t* st = stages + s * C::STAGE;
           mbar_arrive_expect_tx(&full[s], C::STAGE);
           const int z = static_cast<int>(b * a.n_kv + tl[j]);
@@ -231,26 +201,7 @@ __global__ void __launch_bounds__(288, 1)
         }
       }
       cnt = __shfl_sync(0xFFFFFFFFu, cnt, 0);
-      return __shfl_sync(0xFFFFFFFFu, g_ok, 0);
-    };
-    auto setup_next = [&](int local) -> bool {   // sets up item local + 1
-      if (local + 1 >= n_local) return true;
-      const int v = vnext;
-      vnext = (local + 2 < n_local && lane < a.topk)
-                  ? __ldg(sel_ptr(blockIdx.x + static_cast<int64_t>(local + 2) * gridDim.x) + lane) : -1;
-      return setup(local + 1, v);
-    };
-    for (int local = 0; local < n_local && ok; ++local) {
-      if (MRG) {
-        // few window tiles per item and two item slots: gather this item's
-        // tiles first, so they are in flight while the previous item ends;
-        // setting up the next item waits for that end (slot reuse)
-        ok = gather(local);
-        if (ok) ok = setup_next(local);
-      } else {
-        ok = setup_next(local);
-        if (ok) ok = gather(local);
-      }
+      ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
     }
     if (!ok && lane == 0) {   // let copies already issued land before the CTA exits
       for (uint32_t n = (cnt > C::NS ? cnt - C::NS : 0); n < cnt; ++n) {
@@ -268,7 +219,7 @@ __global__ void __launch_bounds__(288, 1)
     const int krow = wq * 16;                  // this warp's 16 keys of each of its tiles
     for (int64_t u = blockIdx.x; u < a.n_items; u += gridDim.x, ++local) {
       const int sl = local % C::NSLOT;
-      bool ok = __all_sync(0xFFFFFFFFu, mbar_wait(&item_full[sl], (local / C::NSLOT) & 1, a.err, kSiteC));
+      bool ok = __all_sync(0xFFFFFFFFu, mbar_wait(&item_full[sl], (local / C::NSLOT) & 1, a.err, SITE_ATTN_CONSUMER));
       float m_run[2] = {-INFINITY, -INFINITY}, l_run[2] = {0.f, 0.f};
       float oacc[MT][4];
 #pragma unroll
@@ -297,7 +248,7 @@ __global__ void __launch_bounds__(288, 1)
         for (int j = grp; j < meta.n_sub; j += 2) {
           const uint32_t n = cnt + j;
           const int s = n % C::NS;
-          ok = __all_sync(0xFFFFFFFFu, mbar_wait(&full[s], (n / C::NS) & 1, a.err, kSiteC));
+          ok = __all_sync(0xFFFFFFFFu, mbar_wait(&full[s], (n / C::NS) & 1, a.err, SITE_ATTN_CONSUMER));
           if (!ok) break;
           const int key0 = tl[j];
           const bool wt = j >= meta.ns;
@@ -455,68 +406,21 @@ __global__ void __launch_bounds__(288, 1)
 #pragma unroll
       for (int w = 0; w < 8; ++w) ab |= abort_flag[w];
       const bool any_abort = ab != 0;
-      const uint8_t* pslot = slot_q(sl);
-      if (!MRG) {
-        for (int e = threadIdx.x; e < G * D && !any_abort; e += 256) {
-          const int h = e / D, dd = e % D;
-          float M = -INFINITY;
+      for (int e = threadIdx.x; e < G * D && !any_abort; e += 256) {
+        const int h = e / D, dd = e % D;
+        float M = -INFINITY;
 #pragma unroll
-          for (int w = 0; w < 4; ++w) M = fmaxf(M, mM[w * 8 + h]);
-          float num = 0.f, den = 0.f;
+        for (int w = 0; w < 4; ++w) M = fmaxf(M, mM[w * 8 + h]);
+        float num = 0.f, den = 0.f;
 #pragma unroll
-          for (int w = 0; w < 4; ++w) {
-            const float mw = mM[w * 8 + h];
-            const float f = (mw == -INFINITY) ? 0.f : fast_exp2(mw - M);
-            num += f * mO[(w * 8 + h) * D + dd];
-            den += f * mL[w * 8 + h];
-          }
-          Out[(meta.qrow + h) * D + dd] = __float2bfloat16_rn(num / den);
-          if (dd == 0 && a.lse) a.lse[meta.qrow + h] = (M + log2f(den)) * 0.69314718055994531f;
+        for (int w = 0; w < 4; ++w) {
+          const float mw = mM[w * 8 + h];
+          const float f = (mw == -INFINITY) ? 0.f : fast_exp2(mw - M);
+          num += f * mO[(w * 8 + h) * D + dd];
+          den += f * mL[w * 8 + h];
         }
-      } else if (!any_abort) {
-        // merge with the block partials: one thread per head finds the
-        // common maximum and every weight, then all threads combine rows
-        const float2* pL = reinterpret_cast<const float2*>(pslot + C::PART_L);
-        const __half* pO = reinterpret_cast<const __half*>(pslot + C::PART_O);
-        float* wts = reinterpret_cast<float*>(slot_q(sl) + C::PART_L + C::PART_LBYTES);   // [topk * G]
-        float* fwin = wts + 128;                                                          // [4][8]
-        float* hinv = fwin + 32;                                                          // [8]
-        if (threadIdx.x < G) {
-          const int h = threadIdx.x;
-          float M = -INFINITY;
-#pragma unroll
-          for (int w = 0; w < 4; ++w) M = fmaxf(M, mM[w * 8 + h]);
-          for (uint32_t sm = meta.selmask; sm; sm &= sm - 1) M = fmaxf(M, pL[(__ffs(sm) - 1) * G + h].x);
-          float den = 0.f;
-#pragma unroll
-          for (int w = 0; w < 4; ++w) {
-            const float mw = mM[w * 8 + h];
-            const float f = (mw == -INFINITY) ? 0.f : fast_exp2(mw - M);
-            fwin[w * 8 + h] = f;
-            den += f * mL[w * 8 + h];
-          }
-          for (uint32_t sm = meta.selmask; sm; sm &= sm - 1) {
-            const int jj = __ffs(sm) - 1;
-            const float2 ls = pL[jj * G + h];
-            const float f = fast_exp2(ls.x - M);
-            wts[jj * G + h] = f * ls.y;   // the row was stored times 2^-e
-            den += f;
-          }
-          hinv[h] = 1.f / den;
-          if (a.lse) a.lse[meta.qrow + h] = (M + log2f(den)) * 0.69314718055994531f;
-        }
-        named_bar_consumers();
-        for (int e = threadIdx.x; e < G * D; e += 256) {
-          const int h = e / D, dd = e % D;
-          float num = 0.f;
-#pragma unroll
-          for (int w = 0; w < 4; ++w) num += fwin[w * 8 + h] * mO[(w * 8 + h) * D + dd];
-          for (uint32_t sm = meta.selmask; sm; sm &= sm - 1) {
-            const int jj = __ffs(sm) - 1;
-            num += wts[jj * G + h] * __half2float(pO[(jj * G + h) * D + dd]);
-          }
-          Out[(meta.qrow + h) * D + dd] = __float2bfloat16_rn(num * hinv[h]);
-        }
+        Out[(meta.qrow + h) * D + dd] = __float2bfloat16_rn(num / den);
+        if (dd == 0 && a.lse) a.lse[meta.qrow + h] = (M + log2f(den)) * 0.69314718055994531f;
       }
       named_bar_consumers();
       if (lane == 0) mbar_arrive(&item_empty[sl]);
@@ -648,38 +552,35 @@ AttnArgs attn_args(const ssa_params& p, const void* Q, const void* K, const void
   a.scale = p.scale;
   a.scale_log2 = p.scale * 1.4426950408889634f;
   a.err = err;
-  a.partO = nullptr;
-  a.partL = nullptr;
-  a.partL_stride = 0;
   return a;
 }
 
-template <int D, int G, bool MRG>
+template <int D, int G>
 cudaError_t run_bf16(const ssa_params& p, const CUtensorMap& tmK, const CUtensorMap& tmV,
                      const CUtensorMap& tmQ, const AttnArgs& a, const LaunchCtx& c) {
-  using C = AttnCfg<D, MRG>;
-  cudaError_t e = cudaFuncSetAttribute(attn_bf16_kernel<D, G, MRG>,
+  using C = AttnCfg<D>;
+  cudaError_t e = cudaFuncSetAttribute(attn_bf16_kernel<D, G>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
   if (e != cudaSuccess) return e;
   int per_sm = 1;
-  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, attn_bf16_kernel<D, G, MRG>, 288, C::SMEM);
+  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, attn_bf16_kernel<D, G>, 288, C::SMEM);
   if (e != cudaSuccess) return e;
   if (per_sm < 1) per_sm = 1;
   int64_t grid = static_cast<int64_t>(per_sm) * c.sm_count;
   if (grid > a.n_items) grid = a.n_items;
-  attn_bf16_kernel<D, G, MRG><<<static_cast<unsigned>(grid), 288, C::SMEM, c.stream>>>(tmK, tmV, tmQ, a);
+  attn_bf16_kernel<D, G><<<static_cast<unsigned>(grid), 288, C::SMEM, c.stream>>>(tmK, tmV, tmQ, a);
   note_launch();
   return cudaGetLastError();
 }
 
-template <int D, bool MRG = false>
+template <int D>
 cudaError_t bf16_g(const ssa_params& p, const CUtensorMap& tmK, const CUtensorMap& tmV,
                    const CUtensorMap& tmQ, const AttnArgs& a, const LaunchCtx& c) {
   switch (p.h_q / p.h_kv) {
-    case 1: return run_bf16<D, 1, MRG>(p, tmK, tmV, tmQ, a, c);
-    case 2: return run_bf16<D, 2, MRG>(p, tmK, tmV, tmQ, a, c);
-    case 4: return run_bf16<D, 4, MRG>(p, tmK, tmV, tmQ, a, c);
-    case 8: return run_bf16<D, 8, MRG>(p, tmK, tmV, tmQ, a, c);
+    case 1: return run_bf16<D, 1>(p, tmK, tmV, tmQ, a, c);
+    case 2: return run_bf16<D, 2>(p, tmK, tmV, tmQ, a, c);
+    case 4: return run_bf16<D, 4>(p, tmK, tmV, tmQ, a, c);
+    case 8: return run_bf16<D, 8>(p, tmK, tmV, tmQ, a, c);
   }
   return cudaErrorInvalidValue;
 }
@@ -709,18 +610,6 @@ cudaError_t f32_g(const ssa_params& p, const AttnArgs& a, const LaunchCtx& c) {
 }  // namespace
 
 int attn_bf16_smem_bytes(int d) { return d == 128 ? AttnCfg<128>::SMEM : AttnCfg<64>::SMEM; }
-
-cudaError_t launch_attn_bf16_merge(const ssa_params& p, const CUtensorMap& tmK, const CUtensorMap& tmV,
-                                   const CUtensorMap& tmQ, const void* Q, const int32_t* block_idx,
-                                   const void* partO, const void* partL, void* O, float* lse,
-                                   int32_t* bad, const LaunchCtx& c) {
-  AttnArgs a = attn_args(p, Q, nullptr, nullptr, block_idx, O, lse, bad, c.err);
-  a.partO = static_cast<const __half*>(partO);
-  a.partL = static_cast<const float2*>(partL);
-  a.partL_stride = (p.topk * (p.h_q / p.h_kv) + 3) / 4 * 4;
-  if (p.d == 128) return bf16_g<128, true>(p, tmK, tmV, tmQ, a, c);
-  return cudaErrorInvalidValue;
-}
 
 cudaError_t launch_attn_bf16(const ssa_params& p, const CUtensorMap& tmK, const CUtensorMap& tmV,
                              const CUtensorMap& tmQ, const void* Q, const int32_t* block_idx, void* O,

@@ -30,18 +30,51 @@ namespace ssa {
 namespace {
 
 // ------------------------------------------------------------------ inversion
+//
+// The rows of one (batch, kv-head) are cut into chunks of kPlanRows.  A CTA
+// per chunk counts its slots per key block in shared memory; a column scan
+// over the chunks then gives every (chunk, block) its place in the block's
+// entry list, so the scatter again needs only shared-memory atomics.
 
-__global__ void __launch_bounds__(256) inv_count_kernel(const BlockPlan pl, const int32_t* __restrict__ idx) {
-  const int64_t row = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
-  if (row >= static_cast<int64_t>(pl.bgs) * pl.n_q) return;   // warp-uniform
-  const int lane = threadIdx.x & 31;
-  const int i = static_cast<int>(row % pl.n_q);
-  const int bg = static_cast<int>(row / pl.n_q);
+constexpr int kPlanThreads = 512;
+
+__device__ __forceinline__ int slot_block(const SlotSet& s, int j, int topk) {
+  return j < topk ? s.v : static_cast<int>(s.b0) + (j - topk);   // lane j's own entry for j < topk
+}
+
+__global__ void __launch_bounds__(kPlanThreads) inv_hist_kernel(const BlockPlan pl, const int32_t* __restrict__ idx) {
+  extern __shared__ int32_t hist[];
+  const int k = blockIdx.x, bg = blockIdx.y;
+  for (int c = threadIdx.x; c < pl.nb; c += blockDim.x) hist[c] = 0;
+  __syncthreads();
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
   const int b = bg / pl.h_kv, g = bg % pl.h_kv;
-  const int64_t pos = pl.q_offset + i;
-  const int nvis = static_cast<int>(min(static_cast<int64_t>(pl.nb), (pos + 1) / pl.block));
-  const int v = lane < pl.topk ? __ldg(idx + ((static_cast<int64_t>(b) * pl.n_q + i) * pl.h_kv + g) * pl.topk + lane) : -1;
-  if (selection_valid(v, nvis)) atomicAdd(&pl.count[static_cast<int64_t>(bg) * pl.nb + v], 1);
+  const int r1 = min((k + 1) * kPlanRows, pl.n_q);
+  for (int i = k * kPlanRows + warp; i < r1; i += nw) {
+    const int v = lane < pl.topk ? __ldg(idx + ((static_cast<int64_t>(b) * pl.n_q + i) * pl.h_kv + g) * pl.topk + lane) : -1;
+    const SlotSet s = row_slots(v, pl.topk, pl.q_offset + i, pl.nb, pl.block, pl.window);
+    if ((s.mask >> lane) & 1) atomicAdd(&hist[slot_block(s, lane, pl.topk)], 1);
+    if ((s.mask >> (lane + 32)) & 1) atomicAdd(&hist[static_cast<int>(s.b0) + lane + 32 - pl.topk], 1);
+  }
+  __syncthreads();
+  int32_t* out = pl.chist + (static_cast<int64_t>(bg) * pl.nchunk + k) * pl.nb;
+  for (int c = threadIdx.x; c < pl.nb; c += blockDim.x) out[c] = hist[c];
+}
+
+// Thread per (batch, kv-head, block): exclusive scan of the chunk counts in
+// place, and the block's total.
+__global__ void __launch_bounds__(256) inv_colscan_kernel(const BlockPlan pl) {
+  const int64_t x = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (x >= static_cast<int64_t>(pl.bgs) * pl.nb) return;
+  const int bg = static_cast<int>(x / pl.nb), c = static_cast<int>(x % pl.nb);
+  int32_t* col = pl.chist + static_cast<int64_t>(bg) * pl.nchunk * pl.nb + c;
+  int run = 0;
+  for (int k = 0; k < pl.nchunk; ++k) {
+    const int v = col[static_cast<int64_t>(k) * pl.nb];
+    col[static_cast<int64_t>(k) * pl.nb] = run;
+    run += v;
+  }
+  pl.count[x] = run;
 }
 
 // One CTA per (batch, kv-head): exclusive scans of the per-block entry and
@@ -92,8 +125,8 @@ __global__ void __launch_bounds__(1024) inv_scan_kernel(const BlockPlan pl) {
   }
 }
 
-// One CTA: exclusive scans over (batch, kv-head); slot [bgs] holds the totals.
-__global__ void __launch_bounds__(1024) inv_scan_bg_kernel(const BlockPlan pl) {
+// One thread: exclusive scans over (batch, kv-head); slot [bgs] holds the totals.
+__global__ void __launch_bounds__(32) inv_scan_bg_kernel(const BlockPlan pl) {
   if (threadIdx.x != 0) return;
   int e = 0, t = 0;
   for (int bg = 0; bg < pl.bgs; ++bg) {
@@ -106,20 +139,25 @@ __global__ void __launch_bounds__(1024) inv_scan_bg_kernel(const BlockPlan pl) {
   pl.tile_base[pl.bgs] = t;
 }
 
-__global__ void __launch_bounds__(256) inv_scatter_kernel(const BlockPlan pl, const int32_t* __restrict__ idx) {
-  const int64_t row = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
-  if (row >= static_cast<int64_t>(pl.bgs) * pl.n_q) return;   // warp-uniform
-  const int lane = threadIdx.x & 31;
-  const int i = static_cast<int>(row % pl.n_q);
-  const int bg = static_cast<int>(row / pl.n_q);
+// Same rows as inv_hist_kernel: every used slot becomes the entry
+// make_entry(query row, slot) in its block's list.
+__global__ void __launch_bounds__(kPlanThreads) inv_scatter_kernel(const BlockPlan pl, const int32_t* __restrict__ idx) {
+  extern __shared__ int32_t cur[];
+  const int k = blockIdx.x, bg = blockIdx.y;
+  const int32_t* col = pl.chist + (static_cast<int64_t>(bg) * pl.nchunk + k) * pl.nb;
+  const int32_t* boff = pl.blk_off + static_cast<int64_t>(bg) * pl.nb;
+  const int ebase = pl.ent_base[bg];
+  for (int c = threadIdx.x; c < pl.nb; c += blockDim.x) cur[c] = ebase + boff[c] + col[c];
+  __syncthreads();
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
   const int b = bg / pl.h_kv, g = bg % pl.h_kv;
-  const int64_t pos = pl.q_offset + i;
-  const int nvis = static_cast<int>(min(static_cast<int64_t>(pl.nb), (pos + 1) / pl.block));
-  const int v = lane < pl.topk ? __ldg(idx + ((static_cast<int64_t>(b) * pl.n_q + i) * pl.h_kv + g) * pl.topk + lane) : -1;
-  if (selection_valid(v, nvis)) {
-    const int64_t cb = static_cast<int64_t>(bg) * pl.nb + v;
-    const int slot = pl.ent_base[bg] + pl.blk_off[cb] + atomicAdd(&pl.cursor[cb], 1);
-    pl.entries[slot] = (i << 5) | lane;
+  const int r1 = min((k + 1) * kPlanRows, pl.n_q);
+  for (int i = k * kPlanRows + warp; i < r1; i += nw) {
+    const int v = lane < pl.topk ? __ldg(idx + ((static_cast<int64_t>(b) * pl.n_q + i) * pl.h_kv + g) * pl.topk + lane) : -1;
+    const SlotSet s = row_slots(v, pl.topk, pl.q_offset + i, pl.nb, pl.block, pl.window);
+    if ((s.mask >> lane) & 1) pl.entries[atomicAdd(&cur[slot_block(s, lane, pl.topk)], 1)] = make_entry(i, lane);
+    if ((s.mask >> (lane + 32)) & 1)
+      pl.entries[atomicAdd(&cur[static_cast<int>(s.b0) + lane + 32 - pl.topk], 1)] = make_entry(i, lane + 32);
   }
 }
 
@@ -156,12 +194,12 @@ struct BlkArgs {
   const __nv_bfloat16* Q;
   const int4* tiles;
   const int32_t* n_tiles;    // device: total tiles
-  const int32_t* entries;
-  int32_t n_q, n_kv, h_q, h_kv, topk;
+  const int32_t* entries;    // make_entry(query row, slot)
+  int32_t n_q, n_kv, h_q, h_kv, topk, window, nsl;
+  int64_t q_offset;
   float scale_log2;
-  __half* partO;             // [items][topk][G][D], o / 2^e
-  float2* partL;             // [items][partL_stride]: (log2-sum-exp, 2^e); slot j head h at j*G + h
-  int32_t partL_stride;
+  __half* partO;             // [items][nsl][G][D], o / 2^e
+  float2* partL;             // [items][nsl][G]: (log2-sum-exp, 2^e)
   uint32_t* err;
 };
 
@@ -272,7 +310,11 @@ __global__ void __launch_bounds__(192, 1)
       const uint32_t abase = smem_u32(sA + ab * C::A_BYTES);
       for (int ee = 0; ee < ne; ++ee) {
         const int ent = ee < 32 ? __shfl_sync(0xFFFFFFFFu, en0, ee) : __shfl_sync(0xFFFFFFFFu, en1, ee - 32);
-        const int i = ent >> 5;
+        const int i = entry_row(ent);
+        if (static_cast<unsigned>(i) >= static_cast<unsigned>(a.n_q)) {   // never for a consistent plan
+          if (lane == 0) atomicCAS(a.err, 0u, static_cast<uint32_t>(SITE_BLK_BAD_ENTRY));
+          continue;
+        }
         const __nv_bfloat16* qrow = a.Q + ((static_cast<int64_t>(b) * a.n_q + i) * a.h_q +
                                            static_cast<int64_t>(g) * G) * D;
 #pragma unroll
@@ -429,6 +471,16 @@ __global__ void __launch_bounds__(192, 1)
       nxt2 = t + 2 < t1 ? a.tiles[t + 2] : none;
       nxt_ent = e < nxt.w ? __ldg(a.entries + nxt.z + e) : 0;
       const int bg = td.x, ne = td.w;
+      const int i = entry_row(ent), j = entry_slot(ent);
+      const bool valid = e < ne && static_cast<unsigned>(i) < static_cast<unsigned>(a.n_q) && j < a.nsl;
+      // a window slot keeps the block's keys inside pos-W+1 .. pos
+      int klo = 0, khi = BLK - 1;
+      if (valid && j >= a.topk) {
+        const int64_t pos = a.q_offset + i, base = static_cast<int64_t>(td.y) * BLK;
+        const int64_t lo = pos - a.window + 1;
+        klo = static_cast<int>(max(lo - base, static_cast<int64_t>(0)));
+        khi = static_cast<int>(min(pos - base, static_cast<int64_t>(BLK - 1)));
+      }
       ok = __all_sync(0xFFFFFFFFu, mbar_wait(&s_full[sb], (lt >> 1) & 1, a.err, SITE_BLK_S_FULL));
       if (!ok) break;
       tc_fence_after();
@@ -442,7 +494,8 @@ __global__ void __launch_bounds__(192, 1)
         tmem_wait_ld();
         tmem_regs_ready(r);
 #pragma unroll
-        for (int u = 0; u < BLK; ++u) sv[u] = __uint_as_float(r[u]) * a.scale_log2;
+        for (int u = 0; u < BLK; ++u)
+          sv[u] = (u >= klo && u <= khi) ? __uint_as_float(r[u]) * a.scale_log2 : -INFINITY;
       }
       tc_fence_before();
       __syncwarp();
@@ -471,11 +524,8 @@ __global__ void __launch_bounds__(192, 1)
       ok = __all_sync(0xFFFFFFFFu, mbar_wait(&o_full[sb], (lt >> 1) & 1, a.err, SITE_BLK_O_FULL));
       if (!ok) break;
       tc_fence_after();
-      const bool valid = e < ne;
-      const int i = ent >> 5, j = ent & 31;
       const int64_t item = static_cast<int64_t>(bg) * a.n_q + i;
-      const int64_t slot = (item * a.topk + j) * G + h;
-      const int64_t lslot = item * a.partL_stride + j * G + h;
+      const int64_t slot = (item * a.nsl + j) * G + h;
       float ov[D];
       {
         uint32_t r[D];
@@ -497,9 +547,9 @@ __global__ void __launch_bounds__(192, 1)
         for (int dd = 0; dd < D; ++dd) amax = fmaxf(amax, fabsf(ov[dd]));
         const float inv_l = 1.f / l;
         const float x = amax * inv_l;
-        int e = x > 0.f ? static_cast<int>((__float_as_uint(x) >> 23) & 0xFFu) - 127 - 14 : 0;
-        e = min(max(e, -100), 100);
-        const float mul = inv_l * __uint_as_float(static_cast<uint32_t>(127 - e) << 23);
+        int ex = x > 0.f ? static_cast<int>((__float_as_uint(x) >> 23) & 0xFFu) - 127 - 14 : 0;
+        ex = min(max(ex, -100), 100);
+        const float mul = inv_l * __uint_as_float(static_cast<uint32_t>(127 - ex) << 23);
         uint4* dst = reinterpret_cast<uint4*>(a.partO + slot * D);
 #pragma unroll
         for (int q = 0; q < D / 8; ++q) {
@@ -511,7 +561,7 @@ __global__ void __launch_bounds__(192, 1)
           }
           dst[q] = make_uint4(w[0], w[1], w[2], w[3]);
         }
-        a.partL[lslot] = make_float2(m + log2f(l), __uint_as_float(static_cast<uint32_t>(127 + e) << 23));
+        a.partL[slot] = make_float2(m + log2f(l), __uint_as_float(static_cast<uint32_t>(127 + ex) << 23));
       }
       tc_fence_before();
       __syncwarp();
@@ -525,6 +575,111 @@ __global__ void __launch_bounds__(192, 1)
     __syncwarp();
     tc_fence_after();
     tmem_dealloc(tmem_base, 512);
+  }
+}
+
+// ------------------------------------------------------------------ merge
+//
+// One warp per (query, kv-head) item: the item's slots are recomputed from
+// its block_idx row (same rule as the inversion), and the normalised slot
+// partials o_j with base-2 log-sum-exps L_j combine into the softmax over
+// the union of their keys: o = sum_j 2^(L_j - M) o_j / sum_j 2^(L_j - M),
+// lse = (M + log2 sum_j 2^(L_j - M)) ln 2, with M the largest L_j.
+
+struct MergeArgs {
+  const int32_t* idx;
+  const __half* partO;
+  const float2* partL;
+  __nv_bfloat16* O;
+  float* lse;
+  int32_t* bad;
+  int32_t n_q, h_q, h_kv, nb, block, topk, window, nsl;
+  int64_t q_offset, n_items;
+};
+
+template <int G>
+__global__ void __launch_bounds__(256) attn_merge_kernel(const MergeArgs a) {
+  constexpr int D = 128;
+  const int lane = threadIdx.x & 31;
+  const int64_t item = static_cast<int64_t>(blockIdx.x) * 8 + (threadIdx.x >> 5);
+  if (item >= a.n_items) return;   // warp-uniform
+  const int i = static_cast<int>(item % a.n_q);
+  const int bg = static_cast<int>(item / a.n_q);
+  const int b = bg / a.h_kv, g = bg % a.h_kv;
+  const int v = lane < a.topk ? __ldg(a.idx + ((static_cast<int64_t>(b) * a.n_q + i) * a.h_kv + g) * a.topk + lane) : -1;
+  const SlotSet s = row_slots(v, a.topk, a.q_offset + i, a.nb, a.block, a.window);
+  if (lane == 0 && a.bad && s.n_bad) atomicAdd(a.bad, s.n_bad);
+  const float2* pl = a.partL + item * a.nsl * G;
+  const __half* po = a.partO + item * a.nsl * G * D;
+  // per head: this lane's slots lane and lane + 32, their weights 2^(L-M) 2^e
+  float w0[G], w1[G], inv_den[G], lse2[G];
+  const bool has0 = (s.mask >> lane) & 1, has1 = (s.mask >> (lane + 32)) & 1;
+#pragma unroll
+  for (int h = 0; h < G; ++h) {
+    const float2 l0 = has0 ? pl[lane * G + h] : make_float2(-INFINITY, 0.f);
+    const float2 l1 = has1 ? pl[(lane + 32) * G + h] : make_float2(-INFINITY, 0.f);
+    float M = fmaxf(l0.x, l1.x);
+#pragma unroll
+    for (int o = 16; o; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xFFFFFFFFu, M, o));
+    const float f0 = has0 ? fast_exp2(l0.x - M) : 0.f, f1 = has1 ? fast_exp2(l1.x - M) : 0.f;
+    float den = f0 + f1;
+#pragma unroll
+    for (int o = 16; o; o >>= 1) den += __shfl_xor_sync(0xFFFFFFFFu, den, o);
+    w0[h] = f0 * l0.y;
+    w1[h] = f1 * l1.y;
+    inv_den[h] = 1.f / den;
+    lse2[h] = M + log2f(den);
+  }
+  // every lane accumulates dims 4 lane .. 4 lane + 3 of every head, four
+  // slots at a time
+  float acc[G][4];
+#pragma unroll
+  for (int h = 0; h < G; ++h)
+#pragma unroll
+    for (int u = 0; u < 4; ++u) acc[h][u] = 0.f;
+  uint64_t m = s.mask;
+  while (m) {
+    int js[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      js[q] = m ? __ffsll(static_cast<long long>(m)) - 1 : -1;
+      m &= m - 1;
+    }
+    uint2 raw[4][G];
+#pragma unroll
+    for (int q = 0; q < 4; ++q)
+#pragma unroll
+      for (int h = 0; h < G; ++h)
+        raw[q][h] = js[q] >= 0 ? __ldg(reinterpret_cast<const uint2*>(po + (js[q] * G + h) * D) + lane)
+                               : make_uint2(0u, 0u);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      if (js[q] < 0) break;   // warp-uniform
+      const int src = js[q] & 31;
+#pragma unroll
+      for (int h = 0; h < G; ++h) {
+        const float wj = __shfl_sync(0xFFFFFFFFu, js[q] < 32 ? w0[h] : w1[h], src);
+        const float2 o01 = __half22float2(*reinterpret_cast<const __half2*>(&raw[q][h].x));
+        const float2 o23 = __half22float2(*reinterpret_cast<const __half2*>(&raw[q][h].y));
+        acc[h][0] += wj * o01.x;
+        acc[h][1] += wj * o01.y;
+        acc[h][2] += wj * o23.x;
+        acc[h][3] += wj * o23.y;
+      }
+    }
+  }
+  const int64_t qrow = (static_cast<int64_t>(b) * a.n_q + i) * a.h_q + static_cast<int64_t>(g) * G;
+#pragma unroll
+  for (int h = 0; h < G; ++h) {
+    const uint32_t lo = pack_bf16(acc[h][0] * inv_den[h], acc[h][1] * inv_den[h]);
+    const uint32_t hi = pack_bf16(acc[h][2] * inv_den[h], acc[h][3] * inv_den[h]);
+    reinterpret_cast<uint2*>(a.O + (qrow + h) * D)[lane] = make_uint2(lo, hi);
+  }
+  if (a.lse && lane < G) {
+    float x = lse2[0];
+#pragma unroll
+    for (int h = 1; h < G; ++h) x = lane == h ? lse2[h] : x;
+    a.lse[qrow + lane] = x * 0.69314718055994531f;
   }
 }
 
@@ -542,26 +697,56 @@ cudaError_t run_block(const BlockPlan& pl, const CUtensorMap& tmK, const CUtenso
 
 }  // namespace
 
+cudaError_t launch_attn_merge(const ssa_params& p, const int32_t* block_idx, const void* partO, const void* partL,
+                              void* O, float* lse, int32_t* bad, const LaunchCtx& c) {
+  MergeArgs a;
+  a.idx = block_idx;
+  a.partO = static_cast<const __half*>(partO);
+  a.partL = static_cast<const float2*>(partL);
+  a.O = static_cast<__nv_bfloat16*>(O);
+  a.lse = lse;
+  a.bad = bad;
+  a.n_q = p.n_q; a.h_q = p.h_q; a.h_kv = p.h_kv; a.nb = p.n_kv / p.block; a.block = p.block; a.topk = p.topk;
+  a.window = p.window;
+  a.nsl = p.topk + window_slots(p.window, p.block);
+  a.q_offset = p.q_offset;
+  a.n_items = static_cast<int64_t>(p.batch) * p.h_kv * p.n_q;
+  if (p.d != 128) return cudaErrorInvalidValue;
+  const unsigned grid = static_cast<unsigned>((a.n_items + 7) / 8);
+  switch (p.h_q / p.h_kv) {
+    case 2: attn_merge_kernel<2><<<grid, 256, 0, c.stream>>>(a); break;
+    case 4: attn_merge_kernel<4><<<grid, 256, 0, c.stream>>>(a); break;
+    case 8: attn_merge_kernel<8><<<grid, 256, 0, c.stream>>>(a); break;
+    default: return cudaErrorInvalidValue;
+  }
+  note_launch();
+  return cudaGetLastError();
+}
+
 int attn_block_smem_bytes(int block) { return block == 64 ? BlkCfg<64>::SMEM : BlkCfg<128>::SMEM; }
 
 cudaError_t launch_block_plan(const ssa_params& p, const int32_t* block_idx, const BlockPlan& pl,
                               const LaunchCtx& c) {
-  const size_t cnt_bytes = static_cast<size_t>(pl.bgs) * pl.nb * sizeof(int32_t);
-  cudaError_t e = cudaMemsetAsync(pl.count, 0, cnt_bytes, c.stream);
-  if (e == cudaSuccess) e = cudaMemsetAsync(pl.cursor, 0, cnt_bytes, c.stream);
+  const size_t hist_smem = static_cast<size_t>(pl.nb) * sizeof(int32_t);
+  cudaError_t e = cudaFuncSetAttribute(inv_hist_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(hist_smem));
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(inv_scatter_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(hist_smem));
   if (e != cudaSuccess) return e;
-  const int64_t rows = static_cast<int64_t>(pl.bgs) * pl.n_q;
-  const unsigned gw = static_cast<unsigned>((rows * 32 + 255) / 256);
-  inv_count_kernel<<<gw, 256, 0, c.stream>>>(pl, block_idx);
+  const dim3 rows(static_cast<unsigned>(pl.nchunk), static_cast<unsigned>(pl.bgs));
+  const unsigned cols = static_cast<unsigned>((static_cast<int64_t>(pl.bgs) * pl.nb + 255) / 256);
+  inv_hist_kernel<<<rows, kPlanThreads, hist_smem, c.stream>>>(pl, block_idx);
+  note_launch();
+  inv_colscan_kernel<<<cols, 256, 0, c.stream>>>(pl);
   note_launch();
   inv_scan_kernel<<<pl.bgs, 1024, 0, c.stream>>>(pl);
   note_launch();
   inv_scan_bg_kernel<<<1, 32, 0, c.stream>>>(pl);
   note_launch();
-  inv_scatter_kernel<<<gw, 256, 0, c.stream>>>(pl, block_idx);
+  inv_scatter_kernel<<<rows, kPlanThreads, hist_smem, c.stream>>>(pl, block_idx);
   note_launch();
-  const unsigned gt = static_cast<unsigned>((static_cast<int64_t>(pl.bgs) * pl.nb + 255) / 256);
-  inv_tiles_kernel<<<gt, 256, 0, c.stream>>>(pl);
+  inv_tiles_kernel<<<cols, 256, 0, c.stream>>>(pl);
   note_launch();
   (void)p;
   return cudaGetLastError();
@@ -575,13 +760,14 @@ cudaError_t launch_attn_block(const ssa_params& p, const BlockPlan& pl, const vo
   a.tiles = pl.tiles;
   a.n_tiles = pl.tile_base + pl.bgs;
   a.entries = pl.entries;
-  a.n_q = p.n_q; a.n_kv = p.n_kv; a.h_q = p.h_q; a.h_kv = p.h_kv; a.topk = p.topk;
+  a.n_q = p.n_q; a.n_kv = p.n_kv; a.h_q = p.h_q; a.h_kv = p.h_kv; a.topk = p.topk; a.window = p.window;
+  a.nsl = p.topk + window_slots(p.window, p.block);
+  a.q_offset = p.q_offset;
   a.scale_log2 = p.scale * 1.4426950408889634f;
   a.partO = static_cast<__half*>(partO);
   a.partL = static_cast<float2*>(partL);
   a.err = c.err;
   const int G = p.h_q / p.h_kv;
-  a.partL_stride = (p.topk * G + 3) / 4 * 4;
   if (p.d != 128) return cudaErrorInvalidValue;
   if (p.block == 64) {
     if (G == 2) return run_block<2, 64>(pl, tmK, tmV, a, c);

@@ -29,6 +29,7 @@ enum WaitSite : uint32_t {
   SITE_BLK_O_EMPTY = 0x415,
   SITE_BLK_S_FULL = 0x421,     // softmax / epilogue
   SITE_BLK_O_FULL = 0x422,
+  SITE_BLK_BAD_ENTRY = 0x431,  // an entry outside the query rows (inconsistent plan)
 };
 
 // A single wait gives up after this long (legitimate waits last microseconds).

@@ -1,17 +1,44 @@
-// Validity of one block_idx row entry, shared by the kernels that read the
-// selections.  An entry is used when it is a fully visible block index and
-// larger than every earlier in-range entry of its row (so the used entries
-// are ascending and distinct); anything else is skipped.
+// The attended key set of one (query, kv-head) item as a set of partial
+// "slots", shared by the kernels of the block-major attention.
+//
+// The keys are the union of the selected blocks and the causal window
+// pos-W+1 .. pos ["Subquadratic Sparse Attention (SSA)", opening section, (i)
+// and (ii)].  Slot j < topk is the row's j-th block_idx entry when it is
+// used: a fully visible block index larger than every earlier in-range entry
+// (so the used entries are ascending and distinct; anything else is skipped
+// and counted).  Slot topk + w is the w-th key block overlapping the window,
+// block lo/B + w, when no used entry selects it; it contributes only its keys
+// inside the window.  Every key of the set is thus in exactly one slot.
 #pragma once
 
 #include <stdint.h>
 
 namespace ssa {
 
-// Warp-collective: lane j holds entry v of the row (-1 for lanes >= topk).
-// Returns whether this lane's entry is used.
-__device__ __forceinline__ bool selection_valid(int v, int nvis) {
+// An inverted entry: the query row and the slot of that row.
+__device__ __forceinline__ int32_t make_entry(int row, int slot) { return (row << 6) | slot; }
+__device__ __forceinline__ int entry_row(int32_t e) { return e >> 6; }
+__device__ __forceinline__ int entry_slot(int32_t e) { return e & 63; }
+
+// Most key blocks a window of W keys overlaps (blocks lo/B .. pos/B).
+__host__ __device__ constexpr int window_slots(int window, int block) {
+  return (window - 1 + block - 1) / block + 1;
+}
+
+struct SlotSet {
+  uint64_t mask;   // bit j: slot j holds keys
+  int n_bad;       // block_idx entries skipped as invalid
+  int v;           // this lane's block_idx entry (-1 past topk)
+  int64_t lo;      // first window key
+  int64_t b0;      // first window block
+};
+
+// Warp-collective: lane l < topk passes entry l of the row (any value past
+// topk is ignored).  topk + window_slots(window, block) <= 64.
+__device__ __forceinline__ SlotSet row_slots(int v_in, int topk, int64_t pos, int nb, int block, int window) {
   const int lane = threadIdx.x & 31;
+  const int v = lane < topk ? v_in : -1;
+  const int nvis = static_cast<int>(min(static_cast<int64_t>(nb), (pos + 1) / block));
   const bool inrange = v >= 0 && v < nvis;
   int run = inrange ? v : -1;
 #pragma unroll
@@ -21,7 +48,25 @@ __device__ __forceinline__ bool selection_valid(int v, int nvis) {
   }
   int prev = __shfl_up_sync(0xFFFFFFFFu, run, 1);
   if (lane == 0) prev = -1;
-  return inrange && v > prev;
+  const bool valid = inrange && v > prev;
+  SlotSet s;
+  s.v = v;
+  s.mask = __ballot_sync(0xFFFFFFFFu, valid);
+  s.n_bad = __popc(__ballot_sync(0xFFFFFFFFu, v != -1 && !valid));
+  s.lo = pos - window + 1 > 0 ? pos - window + 1 : 0;
+  s.b0 = s.lo / block;
+  const int nwb = static_cast<int>(pos / block - s.b0) + 1;
+  // window block w is uncovered unless some used entry selects it; lane w
+  // checks block b0 + w against every used entry
+  const int64_t wb = s.b0 + lane;
+  bool covered = false;
+  for (uint32_t m = static_cast<uint32_t>(s.mask); m; m &= m - 1) {
+    const int src = __ffs(static_cast<int>(m)) - 1;
+    covered |= __shfl_sync(0xFFFFFFFFu, v, src) == wb;
+  }
+  const uint32_t win = __ballot_sync(0xFFFFFFFFu, lane < nwb && !covered);
+  s.mask |= static_cast<uint64_t>(win) << topk;
+  return s;
 }
 
 }  // namespace ssa

@@ -52,19 +52,18 @@ cudaError_t launch_attn_f32(const ssa_params& p, const void* Q, const void* K, c
 
 // Block-major attention plan: per-block lists of the (query, slot) entries
 // that selected each key block, cut into tiles of 128 / G queries.
+// Query rows per CTA of the selection inversion.
+constexpr int kPlanRows = 1024;
+
 struct BlockPlan {
-  int32_t bgs, n_q, h_kv, nb, block, topk, qpt;
+  int32_t bgs, n_q, h_kv, nb, block, topk, window, qpt, nchunk;
   int64_t q_offset;
-  int32_t* count;      // [bgs][nb] selections per block
-  int32_t* cursor;     // [bgs][nb] scatter cursors
-  int32_t* blk_off;    // [bgs][nb] first entry of each block within its (batch, kv-head)
-  int32_t* tile_off;   // [bgs][nb] first tile of each block within its (batch, kv-head)
-  int32_t* bg_ents;    // [bgs]
-  int32_t* bg_tiles;   // [bgs]
-  int32_t* ent_base;   // [bgs + 1]
-  int32_t* tile_base;  // [bgs + 1]; tile_base[bgs] = number of tiles
-  int32_t* entries;    // [selections] (query << 5) | slot
-  int4* tiles;         // [max tiles] {batch*h_kv + kv-head, block, first entry, entries}
+  int32_t* chist;      // [bgs][nchunk][nb] slot counts, then their column scans
+  int32_t *count, *blk_off, *tile_off;   // [bgs][nb]
+  int32_t *bg_ents, *bg_tiles;           // [bgs]
+  int32_t *ent_base, *tile_base;         // [bgs + 1]
+  int32_t* entries;                      // make_entry(query row, slot)
+  int4* tiles;                           // {bg, block, first entry, entries}
 };
 
 cudaError_t launch_block_plan(const ssa_params& p, const int32_t* block_idx, const BlockPlan& pl,
@@ -77,11 +76,9 @@ cudaError_t launch_attn_block(const ssa_params& p, const BlockPlan& pl, const vo
                               const CUtensorMap& tmK, const CUtensorMap& tmV, void* partO, void* partL,
                               const LaunchCtx& c);
 
-// Gather attention over the window keys only, merged with the block partials.
-cudaError_t launch_attn_bf16_merge(const ssa_params& p, const CUtensorMap& tmK, const CUtensorMap& tmV,
-                                   const CUtensorMap& tmQ, const void* Q, const int32_t* block_idx,
-                                   const void* partO, const void* partL, void* O, float* lse,
-                                   int32_t* bad, const LaunchCtx& c);
+// Per (query, kv-head): the softmax merge of the slot partials into O, lse.
+cudaError_t launch_attn_merge(const ssa_params& p, const int32_t* block_idx, const void* partO, const void* partL,
+                              void* O, float* lse, int32_t* bad, const LaunchCtx& c);
 
 int attn_block_smem_bytes(int block);
 

@@ -9,6 +9,7 @@
 #include <atomic>
 #include <mutex>
 
+#include "invert.cuh"
 #include "kernels.h"
 #include "ssa.h"
 
@@ -145,17 +146,20 @@ size_t idx_bytes(const ssa_params& p) {
 ssa_status from_cuda(cudaError_t e) { return e == cudaSuccess ? SSA_OK : SSA_ERR_CUDA; }
 
 // Block-major attention applies to long bf16 problems whose query heads
-// fill a 128-row tensor-core tile in groups of G and whose per-row partials
-// fit the merge kernel's item slot.
+// fill a 128-row tensor-core tile in groups of G, whose row slots (selected
+// blocks plus window blocks) fit the 6-bit slot field of an entry, and whose
+// per-block counters fit the inversion's shared memory.
 bool use_block_attn(const ssa_params& p) {
   const int G = p.h_q / p.h_kv;
+  const int64_t nb = p.n_kv / p.block;
   return p.dtype == SSA_BF16 && p.d == 128 && (G == 2 || G == 4 || G == 8) && p.topk * G <= 128 &&
-         p.n_q >= 1024 && p.n_q < (1 << 26);
+         ssa::window_slots(p.window, p.block) <= 32 && nb <= 16384 && p.n_q >= 1024 && p.n_q < (1 << 25);
 }
 
 struct AttnLayout {
-  size_t count, cursor, blk_off, tile_off, bg_ents, bg_tiles, ent_base, tile_base, entries, tiles, part_o,
-      part_l, total;
+  size_t chist, count, blk_off, tile_off, bg_ents, bg_tiles, ent_base, tile_base, entries, tiles, part_o, part_l,
+      total;
+  int nchunk, nsl;
 };
 
 AttnLayout attn_layout(const ssa_params& p) {
@@ -165,13 +169,14 @@ AttnLayout attn_layout(const ssa_params& p) {
   const size_t nb = static_cast<size_t>(nb_of(p));
   const size_t G = static_cast<size_t>(p.h_q / p.h_kv);
   const size_t qpt = 128 / G;
-  const size_t sel = bgs * p.n_q * p.topk;
-  const size_t max_tiles = (sel + qpt - 1) / qpt + bgs * nb;
+  L.nchunk = (p.n_q + ssa::kPlanRows - 1) / ssa::kPlanRows;
+  L.nsl = p.topk + ssa::window_slots(p.window, p.block);
   const size_t items = bgs * p.n_q;
-  const size_t ls = (p.topk * G + 3) / 4 * 4;
+  const size_t sel = items * L.nsl;                       // entries, at most
+  const size_t max_tiles = (sel + qpt - 1) / qpt + bgs * nb;
   size_t off = 0;
+  L.chist = off; off += round_up(bgs * L.nchunk * nb * 4);
   L.count = off; off += round_up(bgs * nb * 4);
-  L.cursor = off; off += round_up(bgs * nb * 4);
   L.blk_off = off; off += round_up(bgs * nb * 4);
   L.tile_off = off; off += round_up(bgs * nb * 4);
   L.bg_ents = off; off += round_up(bgs * 4);
@@ -180,8 +185,8 @@ AttnLayout attn_layout(const ssa_params& p) {
   L.tile_base = off; off += round_up((bgs + 1) * 4);
   L.entries = off; off += round_up(sel * 4);
   L.tiles = off; off += round_up(max_tiles * 16);
-  L.part_o = off; off += round_up(items * p.topk * G * p.d * 2);
-  L.part_l = off; off += round_up(items * ls * 8);
+  L.part_o = off; off += round_up(sel * G * p.d * 2);
+  L.part_l = off; off += round_up(sel * G * 8);
   L.total = off;
   return L;
 }
@@ -265,10 +270,12 @@ ssa::BlockPlan block_plan(const ssa_params& p, const AttnLayout& L, uint8_t* w) 
   pl.nb = static_cast<int32_t>(nb_of(p));
   pl.block = p.block;
   pl.topk = p.topk;
+  pl.window = p.window;
   pl.qpt = 128 / (p.h_q / p.h_kv);
+  pl.nchunk = L.nchunk;
   pl.q_offset = p.q_offset;
+  pl.chist = reinterpret_cast<int32_t*>(w + L.chist);
   pl.count = reinterpret_cast<int32_t*>(w + L.count);
-  pl.cursor = reinterpret_cast<int32_t*>(w + L.cursor);
   pl.blk_off = reinterpret_cast<int32_t*>(w + L.blk_off);
   pl.tile_off = reinterpret_cast<int32_t*>(w + L.tile_off);
   pl.bg_ents = reinterpret_cast<int32_t*>(w + L.bg_ents);
@@ -302,11 +309,10 @@ ssa_status attn_stage_blocks(const ssa_params& p, const void* Q, const AttnMaps&
   return from_cuda(ssa::launch_attn_block(p, block_plan(p, L, w), Q, m.K, m.V, w + L.part_o, w + L.part_l, c));
 }
 
-ssa_status attn_stage_merge(const ssa_params& p, const void* Q, const AttnMaps& m, const int32_t* idx, void* O,
-                            float* lse, int32_t* bad, const uint8_t* w, const LaunchCtx& c) {
+ssa_status attn_stage_merge(const ssa_params& p, const int32_t* idx, void* O, float* lse, int32_t* bad,
+                            const uint8_t* w, const LaunchCtx& c) {
   const AttnLayout L = attn_layout(p);
-  return from_cuda(ssa::launch_attn_bf16_merge(p, m.K, m.V, m.Q, Q, idx, w + L.part_o, w + L.part_l, O, lse,
-                                               bad, c));
+  return from_cuda(ssa::launch_attn_merge(p, idx, w + L.part_o, w + L.part_l, O, lse, bad, c));
 }
 
 ssa_status do_attn(const ssa_params& p, const void* Q, const void* K, const void* V,
@@ -322,7 +328,7 @@ ssa_status do_attn(const ssa_params& p, const void* Q, const void* K, const void
   uint8_t* w = static_cast<uint8_t*>(ws);
   ssa_status st = attn_stage_plan(p, idx, w, c);
   if (st == SSA_OK) st = attn_stage_blocks(p, Q, m, w, c);
-  if (st == SSA_OK) st = attn_stage_merge(p, Q, m, idx, O, lse, bad, w, c);
+  if (st == SSA_OK) st = attn_stage_merge(p, idx, O, lse, bad, w, c);
   return st;
 }
 
@@ -498,20 +504,16 @@ ssa_status ssa_attn_blocks(const ssa_params* pp, const void* Q, const void* K, c
   return attn_stage_blocks(*pp, Q, m, static_cast<uint8_t*>(ws), c);
 }
 
-ssa_status ssa_attn_merge(const ssa_params* pp, const void* Q, const void* K, const void* V,
-                          const int32_t* block_idx, void* O, float* lse, int32_t* bad_index_count, const void* ws,
-                          size_t ws_bytes, void* stream) {
+ssa_status ssa_attn_merge(const ssa_params* pp, const int32_t* block_idx, void* O, float* lse,
+                          int32_t* bad_index_count, const void* ws, size_t ws_bytes, void* stream) {
   ssa_status st = check_stage(pp, ws, ws_bytes);
   if (st != SSA_OK || is_empty(*pp)) return st;
-  if (!Q || !K || !V || !block_idx || !O || !aligned16(Q) || !aligned16(K) || !aligned16(V) ||
-      !aligned16(block_idx) || !aligned16(O) || (reinterpret_cast<uintptr_t>(lse) & 3u) ||
+  if (!block_idx || !O || !aligned16(block_idx) || !aligned16(O) || (reinterpret_cast<uintptr_t>(lse) & 3u) ||
       (reinterpret_cast<uintptr_t>(bad_index_count) & 3u))
     return SSA_ERR_INVALID_ARG;
   LaunchCtx c;
   if ((st = make_ctx(stream, c)) != SSA_OK) return st;
-  AttnMaps m;
-  if (!encode_attn_maps(m, *pp, Q, K, V)) return SSA_ERR_CUDA;
-  return attn_stage_merge(*pp, Q, m, block_idx, O, lse, bad_index_count, static_cast<const uint8_t*>(ws), c);
+  return attn_stage_merge(*pp, block_idx, O, lse, bad_index_count, static_cast<const uint8_t*>(ws), c);
 }
 
 size_t ssa_workspace_size(const ssa_params* p) {

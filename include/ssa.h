@@ -169,12 +169,16 @@ SSA_API size_t ssa_attn_workspace_size(const ssa_params* p);
  * entry of their row (ascending, distinct); any other entry is skipped and,
  * when bad_index_count is not NULL, counted into that device int32
  * (atomically added, not reset).
- * Two evaluations give the same result up to rounding: with a workspace of
- * ssa_attn_workspace_size(p) bytes (bf16 problems with n_q >= 1024, d = 128,
- * G in {2, 4, 8}, topk * G <= 128) the selections are inverted and every
- * selected key block is multiplied once against all queries that chose it
- * on the tensor cores, then merged with the window per query; with ws NULL
- * (or too small) every (query, kv-head) gathers its own blocks.
+ * Two evaluations give the same result up to rounding.  With a workspace
+ * of ssa_attn_workspace_size(p) bytes (bf16 problems with n_q >= 1024,
+ * d = 128, G in {2, 4, 8}, topk * G <= 128, at most 32 key blocks per
+ * window and 16384 key blocks) the evaluation is block-major: every
+ * (query, kv-head) row is split into slots, one per used selected block and
+ * one per window block not selected, the slots are inverted into per-block
+ * lists, each key block is multiplied once against all its slots' queries on
+ * the tensor cores (window slots masked to the window), and the slot
+ * partials are merged per row.  With ws NULL (or too small) every
+ * (query, kv-head) gathers its own keys.
  *   O            device output [b, n_q, h_q, d] of dtype
  *   lse          device float32 output, may be NULL
  *   ws, ws_bytes device workspace, may be NULL / 0
@@ -190,15 +194,17 @@ SSA_API ssa_status ssa_sparse_attn(const ssa_params* p, const void* Q, const voi
  * aligned; its contents are private to the library and live from the plan
  * call to the merge call), they give exactly the bytes ssa_sparse_attn gives
  * with that workspace.
- *   ssa_attn_plan    inverts block_idx: the valid (query, slot) entries of
- *                    every (batch, kv-head, key block), in tiles of 128 / G
- *                    queries;
+ *   ssa_attn_plan    inverts block_idx: the slots of every row (used
+ *                    selected blocks, then window blocks not selected) as
+ *                    per-(batch, kv-head, key block) lists, in tiles of
+ *                    128 / G queries;
  *   ssa_attn_blocks  per tile, S = Q_tile K_c^T and O = P V_c on the tensor
- *                    cores; writes each entry's normalised partial output
- *                    and base-2 log-sum-exp into the workspace;
- *   ssa_attn_merge   per (query, kv-head): the window keys outside the
- *                    selected blocks, merged with the block partials into O
- *                    and lse; counts skipped entries as ssa_sparse_attn does.
+ *                    cores, window slots masked to pos-W+1 .. pos; writes each
+ *                    slot's normalised partial output and base-2
+ *                    log-sum-exp into the workspace;
+ *   ssa_attn_merge   per (query, kv-head): the softmax merge of the row's
+ *                    slot partials into O and lse; counts skipped block_idx
+ *                    entries as ssa_sparse_attn does.
  * Problems that do not qualify return SSA_ERR_UNSUPPORTED, a missing or
  * short workspace SSA_ERR_WORKSPACE; both before any launch.
  */
@@ -206,9 +212,8 @@ SSA_API ssa_status ssa_attn_plan(const ssa_params* p, const int32_t* block_idx, 
                                  void* stream);
 SSA_API ssa_status ssa_attn_blocks(const ssa_params* p, const void* Q, const void* K, const void* V,
                                    void* ws, size_t ws_bytes, void* stream);
-SSA_API ssa_status ssa_attn_merge(const ssa_params* p, const void* Q, const void* K, const void* V,
-                                  const int32_t* block_idx, void* O, float* lse, int32_t* bad_index_count,
-                                  const void* ws, size_t ws_bytes, void* stream);
+SSA_API ssa_status ssa_attn_merge(const ssa_params* p, const int32_t* block_idx, void* O, float* lse,
+                                  int32_t* bad_index_count, const void* ws, size_t ws_bytes, void* stream);
 
 /*
  * ssa_route_topk without a caller workspace.  No counterpart in the paper:

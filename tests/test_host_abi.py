@@ -142,10 +142,10 @@ def test_block_major_workspace_and_stage_checks():
     before = ssa.ssa_launch_count()
     assert ssa.lib.ssa_attn_plan(C.byref(p), 256, None, 0, None) == ssa.SSA_ERR_WORKSPACE
     assert ssa.lib.ssa_attn_blocks(C.byref(p), 256, 256, 256, 256, aw - 16, None) == ssa.SSA_ERR_WORKSPACE
-    assert ssa.lib.ssa_attn_merge(C.byref(p), 256, 256, 256, 256, 256, None, None, 264, aw, None) == \
+    assert ssa.lib.ssa_attn_merge(C.byref(p), 256, 256, None, None, 264, aw, None) == \
         ssa.SSA_ERR_WORKSPACE                                  # misaligned
     assert ssa.lib.ssa_attn_plan(C.byref(p), None, 256, aw, None) == ssa.SSA_ERR_INVALID_ARG
     assert ssa.ssa_launch_count() == before
     # empty problems are no-ops for every stage
     e = good(n_q=0, q_offset=0)
-    assert ssa.lib.ssa_attn_merge(C.byref(e), None, None, None, None, None, None, None, None, 0, None) == ssa.SSA_OK
+    assert ssa.lib.ssa_attn_merge(C.byref(e), None, None, None, None, None, 0, None) == ssa.SSA_OK
