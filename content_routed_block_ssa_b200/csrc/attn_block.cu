@@ -180,14 +180,18 @@ struct BlkCfg {
   static constexpr int ROW = 128;                       // bytes per 64-wide swizzled row
   static constexpr int A_HALF = 128 * ROW;              // 128 rows x 64 dims
   static constexpr int A_BYTES = 2 * A_HALF;            // Q tile
+  static constexpr int NA = (BLK == 64) ? 4 : 3;        // Q tile buffers = gather warps
   static constexpr int KV_HALF = BLK * ROW;             // BLK keys x 64 dims
   static constexpr int KV_BYTES = 4 * KV_HALF;          // K lo, K hi, V lo, V hi
+  static constexpr int NKV = (BLK == 64) ? 2 : 1;       // K/V buffers (at most 2)
   static constexpr int P_HALF = 128 * ROW;              // 128 rows x 64 keys
   static constexpr int P_BYTES = (BLK / 64) * P_HALF;
-  static constexpr int NKV = (BLK == 64) ? 2 : 1;       // K/V buffers
-  static constexpr int SMEM = 1024 + 2 * A_BYTES + NKV * KV_BYTES + 2 * P_BYTES + 24 * 8 + 16;
+  static constexpr int NBAR = 2 * NA + 2 * NKV + 2 * 5 + 1;
+  static constexpr int SMEM = 1024 + NA * A_BYTES + NKV * KV_BYTES + 2 * P_BYTES + NBAR * 8 + 16;
+  static constexpr int THREADS = 32 * (6 + NA);         // KV, MMA, 4 softmax, NA gather warps
   static constexpr int S_COL = 0;                       // TMEM: S[2] then O[2]
   static constexpr int O_COL = 2 * BLK;
+  static_assert(SMEM <= 232448, "shared memory");
 };
 
 struct BlkArgs {
@@ -212,6 +216,8 @@ __device__ __forceinline__ void fence_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
+__device__ __forceinline__ int64_t tile_key(const int4& t) { return static_cast<int64_t>(t.x) * 0x7FFFFFFF + t.y; }
+
 // Shared-memory descriptor of an MN-major operand written by TMA with the
 // 128-byte swizzle: rows of 64 MN-elements (128 B), 8-row groups `sbo` apart
 // along K, 64-element MN groups `lbo` apart.
@@ -225,39 +231,61 @@ __device__ __forceinline__ uint64_t umma_desc_sw128_mn(uint32_t saddr, uint32_t 
   return d;
 }
 
-// Warp roles: 0 = TMA producer (Q rows of each tile, K/V of each block),
-// 1 = MMA issuer and TMEM owner, 2..5 = softmax and epilogue (one tensor-core
-// row = one (query, head) pair per thread).
+__device__ __forceinline__ float max8(const float (&v)[8]) {
+  return fmaxf(fmaxf(fmaxf(v[0], v[1]), fmaxf(v[2], v[3])), fmaxf(fmaxf(v[4], v[5]), fmaxf(v[6], v[7])));
+}
+
+// 64 consecutive TMEM columns of this warp's 32 lanes into registers.
+__device__ __forceinline__ void tmem_ld64(uint32_t taddr, uint32_t (&r)[64]) {
+#pragma unroll
+  for (int q = 0; q < 4; ++q) tmem_ld16(taddr + q * 16, *reinterpret_cast<uint32_t(*)[16]>(&r[q * 16]));
+  tmem_wait_ld();
+  tmem_regs_ready(r);
+}
+
+// One CTA per SM walks a contiguous range of tiles (ordered by key block, so
+// a block's K_c, V_c are loaded once per CTA).  Warp roles:
+//   0          K/V producer: TMA of each new block's K_c, V_c;
+//   1          MMA issuer and TMEM owner: a non-blocking loop that issues
+//              S = Q K_c^T for the next tile whose Q rows have landed and
+//              O = P V_c for the oldest tile whose P is written, whichever
+//              is ready first;
+//   2..5       softmax and epilogue, one tensor-core row = one
+//              (query, head) pair per thread;
+//   6..6+NA-1  Q gather: warp q fills Q buffer q with the rows of tiles
+//              q, q + NA, ... (16-byte asynchronous copies to their
+//              128-byte-swizzled positions), so NA tiles are in flight.
 template <int G, int BLK>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(BlkCfg<BLK>::THREADS, 1)
     attn_block_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                       const BlkArgs a) {
   using C = BlkCfg<BLK>;
   constexpr int D = C::D;
   constexpr int QPT = 128 / G;
+  constexpr int NA = C::NA;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* sA = smem;                                   // [2][A_BYTES]
-  uint8_t* sKV = sA + 2 * C::A_BYTES;                   // [NKV][KV_BYTES]
+  uint8_t* sA = smem;                                   // [NA][A_BYTES]
+  uint8_t* sKV = sA + NA * C::A_BYTES;                  // [NKV][KV_BYTES]
   uint8_t* sP = sKV + C::NKV * C::KV_BYTES;             // [2][P_BYTES]
   uint64_t* bars = reinterpret_cast<uint64_t*>(sP + 2 * C::P_BYTES);
-  uint64_t* a_full = bars;          // [2] (producer arrives once the tile's copies landed)
-  uint64_t* a_empty = bars + 2;     // [2]
-  uint64_t* kv_full = bars + 4;     // [2]
-  uint64_t* kv_empty = bars + 6;    // [2]
-  uint64_t* s_full = bars + 8;      // [2]
-  uint64_t* s_empty = bars + 10;    // [2]
-  uint64_t* p_full = bars + 12;     // [2]
-  uint64_t* o_full = bars + 14;     // [2]
-  uint64_t* o_empty = bars + 16;    // [2]
-  uint64_t* mma_done = bars + 18;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 19);
+  uint64_t* a_full = bars;                  // [NA] gather warp arrives once its copies landed
+  uint64_t* a_empty = a_full + NA;          // [NA]
+  uint64_t* kv_full = a_empty + NA;         // [NKV]
+  uint64_t* kv_empty = kv_full + C::NKV;    // [NKV]
+  uint64_t* s_full = kv_empty + C::NKV;     // [2]
+  uint64_t* s_empty = s_full + 2;           // [2]
+  uint64_t* p_full = s_empty + 2;           // [2]
+  uint64_t* o_full = p_full + 2;            // [2]
+  uint64_t* o_empty = o_full + 2;           // [2]
+  uint64_t* mma_done = o_empty + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   if (threadIdx.x == 0) {
+    for (int i = 0; i < NA; ++i) { mbar_init(&a_full[i], 1); mbar_init(&a_empty[i], 1); }
+    for (int i = 0; i < C::NKV; ++i) { mbar_init(&kv_full[i], 1); mbar_init(&kv_empty[i], 1); }
     for (int i = 0; i < 2; ++i) {
-      mbar_init(&a_full[i], 1); mbar_init(&a_empty[i], 1);
-      mbar_init(&kv_full[i], 1); mbar_init(&kv_empty[i], 1);
       mbar_init(&s_full[i], 1); mbar_init(&s_empty[i], 4);
       mbar_init(&p_full[i], 4); mbar_init(&o_full[i], 1); mbar_init(&o_empty[i], 4);
     }
@@ -277,101 +305,42 @@ __global__ void __launch_bounds__(192, 1)
 
   int t0, t1;
   tile_range(*a.n_tiles, t0, t1);
+  const int T = t1 - t0;
+  const int4 none = make_int4(-1, -1, 0, 0);
 
   if (warp == 0) {
-    // ------------------------------------------------------------ producer
-    bool ok = true;
-    int kv_ord = -1;
-    int64_t prev = -1;
-    uint32_t a_loads = 0, kv_loads = 0;
-    // the next tile's descriptor and entries (one per lane, two for G = 2)
-    // are loaded while this tile's copies are issued
-    const int4 none = make_int4(0, 0, 0, 0);
-    int4 nxt = t0 < t1 ? a.tiles[t0] : none;
-    int4 nxt2 = t0 + 1 < t1 ? a.tiles[t0 + 1] : none;
-    int nen0 = lane < nxt.w ? __ldg(a.entries + nxt.z + lane) : 0;
-    int nen1 = (QPT > 32 && lane + 32 < nxt.w) ? __ldg(a.entries + nxt.z + 32 + lane) : 0;
-    for (int t = t0; t < t1 && ok; ++t) {
-      const int lt = t - t0;
-      const int4 td = nxt;   // bg, c, entry start, entries
-      const int en0 = nen0, en1 = nen1;
-      nxt = nxt2;
-      nxt2 = t + 2 < t1 ? a.tiles[t + 2] : none;
-      nen0 = lane < nxt.w ? __ldg(a.entries + nxt.z + lane) : 0;
-      nen1 = (QPT > 32 && lane + 32 < nxt.w) ? __ldg(a.entries + nxt.z + 32 + lane) : 0;
-      const int bg = td.x, c = td.y, ne = td.w;
-      const int b = bg / a.h_kv, g = bg % a.h_kv;
-      // Q rows of the tile: 16-byte cp.async copies placed at their 128-byte
-      // swizzled positions
-      const int ab = lt & 1;
-      if (lane == 0) ok = mbar_wait(&a_empty[ab], ((lt >> 1) & 1) ^ 1, a.err, SITE_BLK_A_EMPTY);
-      ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
-      if (!ok) break;
-      const uint32_t abase = smem_u32(sA + ab * C::A_BYTES);
-      for (int ee = 0; ee < ne; ++ee) {
-        const int ent = ee < 32 ? __shfl_sync(0xFFFFFFFFu, en0, ee) : __shfl_sync(0xFFFFFFFFu, en1, ee - 32);
-        const int i = entry_row(ent);
-        if (static_cast<unsigned>(i) >= static_cast<unsigned>(a.n_q)) {   // never for a consistent plan
-          if (lane == 0) atomicCAS(a.err, 0u, static_cast<uint32_t>(SITE_BLK_BAD_ENTRY));
-          continue;
-        }
-        const __nv_bfloat16* qrow = a.Q + ((static_cast<int64_t>(b) * a.n_q + i) * a.h_q +
-                                           static_cast<int64_t>(g) * G) * D;
-#pragma unroll
-        for (int x = lane; x < G * 16; x += 32) {   // G heads x 16 chunks of 8 dims
-          const int hh = x >> 4, ch = x & 15;
-          const int r = ee * G + hh;
-          const uint32_t dst = abase + (ch >> 3) * C::A_HALF + r * C::ROW + (((ch & 7) ^ (r & 7)) << 4);
-          asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(qrow + hh * D + ch * 8)
-                       : "memory");
-        }
-      }
-      asm volatile("cp.async.commit_group;" ::: "memory");
-      ++a_loads;
-      // tile t-1 is published once tile t is in flight, and before any wait
-      // on the K/V buffers: freeing a K/V buffer can need tile t-1's MMAs
-      if (lt > 0) {
-        asm volatile("cp.async.wait_group 1;" ::: "memory");
-        fence_async_smem();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&a_full[(lt - 1) & 1]);
-      }
-      const int64_t key = static_cast<int64_t>(bg) * 0x7FFFFFFF + c;
-      if (key != prev) {
+    // ------------------------------------------------------------ K/V producer
+    if (lane == 0) {
+      bool ok = true;
+      int kv_ord = -1;
+      int64_t prev = -1;
+      uint32_t kv_loads = 0;
+      int4 nxt = T > 0 ? a.tiles[t0] : none;
+      for (int t = t0; t < t1 && ok; ++t) {
+        const int4 td = nxt;
+        nxt = t + 1 < t1 ? a.tiles[t + 1] : none;
+        const int64_t key = tile_key(td);
+        if (key == prev) continue;
         ++kv_ord;
         prev = key;
         const int kb = kv_ord % C::NKV;
-        if (lane == 0) {
-          ok = mbar_wait(&kv_empty[kb], ((kv_ord / C::NKV) & 1) ^ 1, a.err, SITE_BLK_KV_EMPTY);
-          if (ok) {
-            uint8_t* kv = sKV + kb * C::KV_BYTES;
-            mbar_arrive_expect_tx(&kv_full[kb], C::KV_BYTES);
-            const int z = static_cast<int>(static_cast<int64_t>(b) * a.n_kv + static_cast<int64_t>(c) * BLK);
+        ok = mbar_wait(&kv_empty[kb], ((kv_ord / C::NKV) & 1) ^ 1, a.err, SITE_BLK_KV_EMPTY);
+        if (!ok) break;
+        const int b = td.x / a.h_kv, g = td.x % a.h_kv;
+        uint8_t* kv = sKV + kb * C::KV_BYTES;
+        mbar_arrive_expect_tx(&kv_full[kb], C::KV_BYTES);
+        const int z = static_cast<int>(static_cast<int64_t>(b) * a.n_kv + static_cast<int64_t>(td.y) * BLK);
 #pragma unroll
-            for (int sub = 0; sub < BLK / 64; ++sub) {
+        for (int sub = 0; sub < BLK / 64; ++sub) {
 #pragma unroll
-              for (int hf = 0; hf < 2; ++hf) {
-                tma_load_3d(kv + hf * C::KV_HALF + sub * 64 * C::ROW, &tmK, &kv_full[kb], hf * 64, g, z + sub * 64);
-                tma_load_3d(kv + (2 + hf) * C::KV_HALF + sub * 64 * C::ROW, &tmV, &kv_full[kb], hf * 64, g, z + sub * 64);
-              }
-            }
-            ++kv_loads;
+          for (int hf = 0; hf < 2; ++hf) {
+            tma_load_3d(kv + hf * C::KV_HALF + sub * 64 * C::ROW, &tmK, &kv_full[kb], hf * 64, g, z + sub * 64);
+            tma_load_3d(kv + (2 + hf) * C::KV_HALF + sub * 64 * C::ROW, &tmV, &kv_full[kb], hf * 64, g, z + sub * 64);
           }
         }
-        ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
-        kv_loads = __shfl_sync(0xFFFFFFFFu, kv_loads, 0);
-        if (!ok) break;
+        ++kv_loads;
       }
-    }
-    if (ok && a_loads > 0) {
-      asm volatile("cp.async.wait_group 0;" ::: "memory");
-      fence_async_smem();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&a_full[(a_loads - 1) & 1]);
-    }
-    if (!ok) {   // let issued copies land before the CTA exits
-      asm volatile("cp.async.wait_group 0;" ::: "memory");
-      if (lane == 0) {
+      if (!ok) {   // let issued copies land before the CTA exits
         const uint64_t tq = global_timer_ns();
         for (uint32_t n = (kv_loads > C::NKV ? kv_loads - C::NKV : 0); n < kv_loads; ++n)
           while (!mbar_try_wait(&kv_full[n % C::NKV], (n / C::NKV) & 1) && global_timer_ns() - tq < kWaitLimitNs) {}
@@ -383,85 +352,156 @@ __global__ void __launch_bounds__(192, 1)
       constexpr uint32_t IDESC1 = umma_idesc_bf16(128, BLK);
       constexpr uint32_t IDESC2 = umma_idesc_bf16(128, D) | (1u << 16);   // B (V) is MN-major
       const uint32_t sA_u = smem_u32(sA), sKV_u = smem_u32(sKV), sP_u = smem_u32(sP);
-      bool ok = true;
+      int n1 = 0, n2 = 0;               // tiles whose S = Q K^T / O = P V are issued
       int kv_ord = -1;
       int64_t prev = -1;
-      int pend_l = -1, pend_kb = 0;
-      bool pend_last = false;
-      auto mma2 = [&](int l, int kb, bool last_of_block) -> bool {
-        const int ob = l & 1;
-        if (!mbar_wait(&p_full[ob], (l >> 1) & 1, a.err, SITE_BLK_P_FULL)) return false;
-        if (!mbar_wait(&o_empty[ob], ((l >> 1) & 1) ^ 1, a.err, SITE_BLK_O_EMPTY)) return false;
-        tc_fence_after();
-        const uint32_t d_tmem = tmem_base + C::O_COL + ob * D;
-        const uint32_t vbase = sKV_u + kb * C::KV_BYTES + 2 * C::KV_HALF;
+      uint32_t ring_kb = 0, ring_last = 0;   // bit (n & 3) per issued S, read by its P V
+      int4 cur = T > 0 ? a.tiles[t0] : none;
+      int4 nxt = T > 1 ? a.tiles[t0 + 1] : none;
+      int4 nxt2 = T > 2 ? a.tiles[t0 + 2] : none;
+      bool fresh = tile_key(cur) != prev;
+      int kb = (kv_ord + (fresh ? 1 : 0)) % C::NKV;
+      uint64_t last_progress = global_timer_ns();
+      uint32_t spins = 0;
+      bool ok = true;
+      while (n2 < T) {
+        bool progressed = false;
+        if (n1 < T && n1 - n2 < 4) {
+          const int ab = n1 % NA;
+          const int ord = kv_ord + (fresh ? 1 : 0);
+          if ((!fresh || mbar_test_wait(&kv_full[kb], (ord / C::NKV) & 1)) &&
+              mbar_test_wait(&a_full[ab], (n1 / NA) & 1) && mbar_test_wait(&s_empty[n1 & 1], ((n1 >> 1) & 1) ^ 1)) {
+            tc_fence_after();
+            const uint32_t s_tmem = tmem_base + C::S_COL + (n1 & 1) * BLK;
+            const uint32_t kbase = sKV_u + kb * C::KV_BYTES;
 #pragma unroll
-        for (int kk = 0; kk < BLK / 16; ++kk) {
-          const uint64_t ad = umma_desc_sw128(sP_u + ob * C::P_BYTES + (kk >> 2) * C::P_HALF + (kk & 3) * 32);
-          const uint64_t bd = umma_desc_sw128_mn(vbase + kk * 16 * C::ROW, C::KV_HALF, 1024);
-          umma_bf16(d_tmem, ad, bd, IDESC2, kk != 0 ? 1u : 0u);
+            for (int ks = 0; ks < D / 16; ++ks) {
+              const uint64_t ad = umma_desc_sw128(sA_u + ab * C::A_BYTES + (ks >> 2) * C::A_HALF + (ks & 3) * 32);
+              const uint64_t bd = umma_desc_sw128(kbase + (ks >> 2) * C::KV_HALF + (ks & 3) * 32);
+              umma_bf16(s_tmem, ad, bd, IDESC1, ks != 0 ? 1u : 0u);
+            }
+            umma_commit(&s_full[n1 & 1]);
+            umma_commit(&a_empty[ab]);
+            if (fresh) { kv_ord = ord; prev = tile_key(cur); }
+            const uint32_t bit = 1u << (n1 & 3);
+            ring_kb = kb ? (ring_kb | bit) : (ring_kb & ~bit);
+            ring_last = (n1 + 1 == T || tile_key(nxt) != tile_key(cur)) ? (ring_last | bit) : (ring_last & ~bit);
+            ++n1;
+            cur = nxt;
+            nxt = nxt2;
+            nxt2 = n1 + 2 < T ? a.tiles[t0 + n1 + 2] : none;
+            fresh = tile_key(cur) != prev;
+            kb = (kv_ord + (fresh ? 1 : 0)) % C::NKV;
+            progressed = true;
+          }
         }
-        umma_commit(&o_full[ob]);
-        if (last_of_block) umma_commit(&kv_empty[kb]);
-        return true;
-      };
-      // tile descriptors two ahead, so no global load sits on the issue path
-      int4 cur = t0 < t1 ? a.tiles[t0] : make_int4(0, 0, 0, 0);
-      int4 nxt = t0 + 1 < t1 ? a.tiles[t0 + 1] : make_int4(-1, -1, 0, 0);
-      for (int t = t0; t < t1 && ok; ++t) {
-        const int lt = t - t0;
-        const int4 td = cur;
-        const int4 tn = nxt;
-        cur = nxt;
-        nxt = t + 2 < t1 ? a.tiles[t + 2] : make_int4(-1, -1, 0, 0);
-        const int64_t key = static_cast<int64_t>(td.x) * 0x7FFFFFFF + td.y;
-        bool fresh = false;
-        if (key != prev) { ++kv_ord; prev = key; fresh = true; }
-        const int kb = kv_ord % C::NKV;
-        const bool last = (t + 1 == t1) || (static_cast<int64_t>(tn.x) * 0x7FFFFFFF + tn.y) != key;
-        // a new block reusing the pending tile's K/V buffer: finish that
-        // tile's P V first, its commit frees the buffer for the producer
-        if (fresh && pend_l >= 0 && pend_kb == kb) {
-          if (!mma2(pend_l, pend_kb, pend_last)) { ok = false; break; }
-          pend_l = -1;
-        }
-        if (fresh && !mbar_wait(&kv_full[kb], (kv_ord / C::NKV) & 1, a.err, SITE_BLK_KV_FULL)) { ok = false; break; }
-        const int ab = lt & 1;
-        if (!mbar_wait(&a_full[ab], (lt >> 1) & 1, a.err, SITE_BLK_A_FULL)) { ok = false; break; }
-        if (!mbar_wait(&s_empty[ab], ((lt >> 1) & 1) ^ 1, a.err, SITE_BLK_S_EMPTY)) { ok = false; break; }
-        tc_fence_after();
-        const uint32_t s_tmem = tmem_base + C::S_COL + ab * BLK;
-        const uint32_t kbase = sKV_u + kb * C::KV_BYTES;
+        if (n2 < n1) {
+          const int ob = n2 & 1;
+          if (mbar_test_wait(&p_full[ob], (n2 >> 1) & 1) && mbar_test_wait(&o_empty[ob], ((n2 >> 1) & 1) ^ 1)) {
+            tc_fence_after();
+            const int kb2 = (ring_kb >> (n2 & 3)) & 1;
+            const uint32_t d_tmem = tmem_base + C::O_COL + ob * D;
+            const uint32_t vbase = sKV_u + kb2 * C::KV_BYTES + 2 * C::KV_HALF;
 #pragma unroll
-        for (int ks = 0; ks < D / 16; ++ks) {
-          const uint64_t ad = umma_desc_sw128(sA_u + ab * C::A_BYTES + (ks >> 2) * C::A_HALF + (ks & 3) * 32);
-          const uint64_t bd = umma_desc_sw128(kbase + (ks >> 2) * C::KV_HALF + (ks & 3) * 32);
-          umma_bf16(s_tmem, ad, bd, IDESC1, ks != 0 ? 1u : 0u);
+            for (int kk = 0; kk < BLK / 16; ++kk) {
+              const uint64_t ad = umma_desc_sw128(sP_u + ob * C::P_BYTES + (kk >> 2) * C::P_HALF + (kk & 3) * 32);
+              const uint64_t bd = umma_desc_sw128_mn(vbase + kk * 16 * C::ROW, C::KV_HALF, 1024);
+              umma_bf16(d_tmem, ad, bd, IDESC2, kk != 0 ? 1u : 0u);
+            }
+            umma_commit(&o_full[ob]);
+            if ((ring_last >> (n2 & 3)) & 1) umma_commit(&kv_empty[kb2]);
+            ++n2;
+            progressed = true;
+          }
         }
-        umma_commit(&s_full[ab]);
-        umma_commit(&a_empty[ab]);
-        if (pend_l >= 0 && !mma2(pend_l, pend_kb, pend_last)) { ok = false; break; }
-        pend_l = lt;
-        pend_kb = kb;
-        pend_last = last;
+        if (progressed) {
+          spins = 0;
+        } else if ((++spins & 255u) == 0) {
+          const uint64_t now = global_timer_ns();
+          if (spins == 256u) last_progress = now;
+          if (*reinterpret_cast<volatile uint32_t*>(a.err) != 0) { ok = false; break; }
+          if (now - last_progress > kWaitLimitNs) {
+            atomicCAS(a.err, 0u, static_cast<uint32_t>(SITE_BLK_MMA_STALL));
+            ok = false;
+            break;
+          }
+        }
       }
-      if (ok && pend_l >= 0) mma2(pend_l, pend_kb, pend_last);
+      (void)ok;
       umma_commit(mma_done);
       const uint64_t tq = global_timer_ns();
       while (!mbar_try_wait(mma_done, 0) && global_timer_ns() - tq < kWaitLimitNs) {}
     }
-  } else {
+  } else if (warp < 6) {
     // ------------------------------------------------------------ softmax + epilogue
+    // Software-pipelined: the softmax of tile t, then the epilogue of tile
+    // t - 1 (O is double-buffered in TMEM), so P V of tile t runs while the
+    // previous tile's output is stored.
     const int eq = warp & 3;
     const int row = eq * 32 + lane;
     const int e = row / G, h = row % G;
     const uint32_t lane_base = static_cast<uint32_t>(eq * 32) << 16;
     bool ok = true;
     // tile descriptors two ahead and this thread's entry one ahead of use
-    const int4 none = make_int4(0, 0, 0, 0);
-    int4 nxt = t0 < t1 ? a.tiles[t0] : none;
-    int4 nxt2 = t0 + 1 < t1 ? a.tiles[t0 + 1] : none;
+    int4 nxt = T > 0 ? a.tiles[t0] : none;
+    int4 nxt2 = T > 1 ? a.tiles[t0 + 1] : none;
     int nxt_ent = e < nxt.w ? __ldg(a.entries + nxt.z + e) : 0;
+    // the pending epilogue: its slot row, validity and softmax statistics
+    int64_t pend_slot = 0;
+    bool pend_valid = false;
+    float pend_m = 0.f, pend_l = 1.f;
+    auto epilogue = [&](int lt) -> bool {
+      const int sb = lt & 1;
+      if (!__all_sync(0xFFFFFFFFu, mbar_wait(&o_full[sb], (lt >> 1) & 1, a.err, SITE_BLK_O_FULL))) return false;
+      tc_fence_after();
+      // two passes over the row in halves of 64 columns: its largest
+      // magnitude, then the scaled float16 conversion
+      const uint32_t ocol = tmem_base + lane_base + C::O_COL + sb * D;
+      float am[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};   // eight independent chains
+#pragma unroll
+      for (int hf = 0; hf < D / 64; ++hf) {
+        uint32_t r[64];
+        tmem_ld64(ocol + hf * 64, r);
+#pragma unroll
+        for (int u = 0; u < 64; ++u) am[u & 7] = fmaxf(am[u & 7], fabsf(__uint_as_float(r[u])));
+      }
+      const float amax = max8(am);
+      // the normalised row o = O / l, stored as float16 times 2^-e with the
+      // power of two 2^e chosen so the row's largest entry lands in
+      // [2^14, 2^15): 11 significant bits whatever the scale of V.  Every
+      // lane runs the (warp-collective) TMEM loads; only valid rows store.
+      const float inv_l = 1.f / pend_l;
+      const float x = amax * inv_l;
+      int ex = x > 0.f ? static_cast<int>((__float_as_uint(x) >> 23) & 0xFFu) - 127 - 14 : 0;
+      ex = min(max(ex, -100), 100);
+      const float mul = inv_l * __uint_as_float(static_cast<uint32_t>(127 - ex) << 23);
+      uint4* dst = reinterpret_cast<uint4*>(a.partO + pend_slot * D);
+#pragma unroll
+      for (int hf = 0; hf < D / 64; ++hf) {
+        uint32_t r[64];
+        tmem_ld64(ocol + hf * 64, r);
+        if (pend_valid) {
+#pragma unroll
+          for (int q = 0; q < 8; ++q) {
+            uint32_t w[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+              const __half2 hv = __floats2half2_rn(__uint_as_float(r[q * 8 + 2 * u]) * mul,
+                                                   __uint_as_float(r[q * 8 + 2 * u + 1]) * mul);
+              w[u] = *reinterpret_cast<const uint32_t*>(&hv);
+            }
+            dst[hf * 8 + q] = make_uint4(w[0], w[1], w[2], w[3]);
+          }
+        }
+      }
+      if (pend_valid)
+        a.partL[pend_slot] = make_float2(pend_m + log2f(pend_l),
+                                         __uint_as_float(static_cast<uint32_t>(127 + ex) << 23));
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&o_empty[sb]);
+      return true;
+    };
     for (int t = t0; t < t1 && ok; ++t) {
       const int lt = t - t0;
       const int sb = lt & 1;
@@ -484,89 +524,124 @@ __global__ void __launch_bounds__(192, 1)
       ok = __all_sync(0xFFFFFFFFu, mbar_wait(&s_full[sb], (lt >> 1) & 1, a.err, SITE_BLK_S_FULL));
       if (!ok) break;
       tc_fence_after();
-      float sv[BLK];
-      {
-        uint32_t r[BLK];
+      // the row's scaled logits in halves of 64 columns: the maximum, then
+      // P = 2^(s - m) in bfloat16 into the swizzled P tile (one pass when
+      // the block is 64 keys)
+      const uint32_t scol = tmem_base + lane_base + C::S_COL + sb * BLK;
+      // a half of S, loaded with the columns outside [klo, khi] set to -inf;
+      // most tiles hold no window slot, and their warps skip the masking
+      const bool any_mask = __any_sync(0xFFFFFFFFu, klo > 0 || khi < BLK - 1);
+      auto load_half = [&](int hf, uint32_t (&r)[64]) {
+        tmem_ld64(scol + hf * 64, r);
+        if (any_mask) {
+          const int lo = klo - hf * 64, hi = khi - hf * 64;
 #pragma unroll
-        for (int q = 0; q < BLK / 16; ++q)
-          tmem_ld16(tmem_base + lane_base + C::S_COL + sb * BLK + q * 16,
-                    *reinterpret_cast<uint32_t(*)[16]>(&r[q * 16]));
-        tmem_wait_ld();
-        tmem_regs_ready(r);
-#pragma unroll
-        for (int u = 0; u < BLK; ++u)
-          sv[u] = (u >= klo && u <= khi) ? __uint_as_float(r[u]) * a.scale_log2 : -INFINITY;
-      }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&s_empty[sb]);
-      float m = -INFINITY;
-#pragma unroll
-      for (int j = 0; j < BLK; ++j) m = fmaxf(m, sv[j]);
-      float l = 0.f;
-      uint8_t* prow = sP + sb * C::P_BYTES;
-#pragma unroll
-      for (int ch = 0; ch < BLK / 8; ++ch) {
-        uint32_t w[4];
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const float p0 = fast_exp2(sv[ch * 8 + 2 * u] - m), p1 = fast_exp2(sv[ch * 8 + 2 * u + 1] - m);
-          l += p0 + p1;
-          w[u] = pack_bf16(p0, p1);
+          for (int u = 0; u < 64; ++u) r[u] = (u >= lo && u <= hi) ? r[u] : 0xFF800000u;
         }
-        const int half = ch >> 3, cc = ch & 7;
-        *reinterpret_cast<uint4*>(prow + half * C::P_HALF + row * C::ROW + ((cc ^ (row & 7)) << 4)) =
-            make_uint4(w[0], w[1], w[2], w[3]);
+      };
+      auto logit = [&](uint32_t raw, int) { return __uint_as_float(raw) * a.scale_log2; };
+      // maxima and sums in eight independent chains (one warp per SMSP runs
+      // this, so dependent chains would cost their full latency)
+      float mx[8] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY, -INFINITY, -INFINITY, -INFINITY, -INFINITY};
+      float ls[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+      float m = -INFINITY;
+      uint8_t* prow = sP + sb * C::P_BYTES;
+      if (BLK > 64) {   // first pass: the maximum over both halves
+#pragma unroll
+        for (int hf = 0; hf < BLK / 64; ++hf) {
+          uint32_t r[64];
+          load_half(hf, r);
+#pragma unroll
+          for (int u = 0; u < 64; ++u) mx[u & 7] = fmaxf(mx[u & 7], logit(r[u], hf * 64 + u));
+        }
+        m = max8(mx);
       }
-      fence_async_smem();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&p_full[sb]);
-      ok = __all_sync(0xFFFFFFFFu, mbar_wait(&o_full[sb], (lt >> 1) & 1, a.err, SITE_BLK_O_FULL));
-      if (!ok) break;
-      tc_fence_after();
-      const int64_t item = static_cast<int64_t>(bg) * a.n_q + i;
-      const int64_t slot = (item * a.nsl + j) * G + h;
-      float ov[D];
-      {
-        uint32_t r[D];
 #pragma unroll
-        for (int q = 0; q < D / 16; ++q)
-          tmem_ld16(tmem_base + lane_base + C::O_COL + sb * D + q * 16,
-                    *reinterpret_cast<uint32_t(*)[16]>(&r[q * 16]));
-        tmem_wait_ld();
-        tmem_regs_ready(r);
+      for (int hf = 0; hf < BLK / 64; ++hf) {
+        uint32_t r[64];
+        load_half(hf, r);
+        if (BLK == 64) {
 #pragma unroll
-        for (int u = 0; u < D; ++u) ov[u] = __uint_as_float(r[u]);
-      }
-      if (valid) {
-        // the normalised row o = O / l, stored as float16 times 2^-e with the
-        // power of two 2^e chosen so the row's largest entry lands in
-        // [2^14, 2^15): 11 significant bits whatever the scale of V
-        float amax = 0.f;
+          for (int u = 0; u < 64; ++u) mx[u & 7] = fmaxf(mx[u & 7], logit(r[u], u));
+          m = max8(mx);
+        }
+        if (hf == BLK / 64 - 1) {   // all of S is in registers or consumed: free the buffer
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&s_empty[sb]);
+        }
 #pragma unroll
-        for (int dd = 0; dd < D; ++dd) amax = fmaxf(amax, fabsf(ov[dd]));
-        const float inv_l = 1.f / l;
-        const float x = amax * inv_l;
-        int ex = x > 0.f ? static_cast<int>((__float_as_uint(x) >> 23) & 0xFFu) - 127 - 14 : 0;
-        ex = min(max(ex, -100), 100);
-        const float mul = inv_l * __uint_as_float(static_cast<uint32_t>(127 - ex) << 23);
-        uint4* dst = reinterpret_cast<uint4*>(a.partO + slot * D);
-#pragma unroll
-        for (int q = 0; q < D / 8; ++q) {
+        for (int ch = 0; ch < 8; ++ch) {
           uint32_t w[4];
 #pragma unroll
           for (int u = 0; u < 4; ++u) {
-            const __half2 hv = __floats2half2_rn(ov[q * 8 + 2 * u] * mul, ov[q * 8 + 2 * u + 1] * mul);
-            w[u] = *reinterpret_cast<const uint32_t*>(&hv);
+            const int c0 = hf * 64 + ch * 8 + 2 * u;
+            const float p0 = fast_exp2(logit(r[ch * 8 + 2 * u], c0) - m);
+            const float p1 = fast_exp2(logit(r[ch * 8 + 2 * u + 1], c0 + 1) - m);
+            ls[2 * u] += p0;
+            ls[2 * u + 1] += p1;
+            w[u] = pack_bf16(p0, p1);
           }
-          dst[q] = make_uint4(w[0], w[1], w[2], w[3]);
+          *reinterpret_cast<uint4*>(prow + hf * C::P_HALF + row * C::ROW + ((ch ^ (row & 7)) << 4)) =
+              make_uint4(w[0], w[1], w[2], w[3]);
         }
-        a.partL[slot] = make_float2(m + log2f(l), __uint_as_float(static_cast<uint32_t>(127 + ex) << 23));
       }
-      tc_fence_before();
+      const float l = ((ls[0] + ls[1]) + (ls[2] + ls[3])) + ((ls[4] + ls[5]) + (ls[6] + ls[7]));
+      fence_async_smem();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&o_empty[sb]);
+      if (lane == 0) mbar_arrive(&p_full[sb]);
+      if (lt > 0 && !epilogue(lt - 1)) { ok = false; break; }
+      pend_slot = ((static_cast<int64_t>(bg) * a.n_q + i) * a.nsl + j) * G + h;
+      pend_valid = valid;
+      pend_m = m;
+      pend_l = l;
     }
+    if (ok && T > 0) epilogue(T - 1);
+  } else {
+    // ------------------------------------------------------------ Q gather
+    const int q = warp - 6;   // buffer q: tiles q, q + NA, ...
+    const uint32_t abase = smem_u32(sA + q * C::A_BYTES);
+    bool ok = true;
+    int4 nxt = q < T ? a.tiles[t0 + q] : none;
+    int nen0 = lane < nxt.w ? __ldg(a.entries + nxt.z + lane) : 0;
+    int nen1 = (QPT > 32 && lane + 32 < nxt.w) ? __ldg(a.entries + nxt.z + 32 + lane) : 0;
+    uint32_t uses = 0;
+    for (int lt = q; lt < T && ok; lt += NA, ++uses) {
+      const int4 td = nxt;
+      const int en0 = nen0, en1 = nen1;
+      const int b = td.x / a.h_kv, g = td.x % a.h_kv, ne = td.w;
+      if (lane == 0) ok = mbar_wait(&a_empty[q], (uses & 1) ^ 1, a.err, SITE_BLK_A_EMPTY);
+      ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
+      if (!ok) break;
+      for (int ee = 0; ee < ne; ++ee) {
+        const int ent = ee < 32 ? __shfl_sync(0xFFFFFFFFu, en0, ee) : __shfl_sync(0xFFFFFFFFu, en1, ee - 32);
+        const int i = entry_row(ent);
+        if (static_cast<unsigned>(i) >= static_cast<unsigned>(a.n_q)) {   // never for a consistent plan
+          if (lane == 0) atomicCAS(a.err, 0u, static_cast<uint32_t>(SITE_BLK_BAD_ENTRY));
+          continue;
+        }
+        const __nv_bfloat16* qrow = a.Q + ((static_cast<int64_t>(b) * a.n_q + i) * a.h_q +
+                                           static_cast<int64_t>(g) * G) * D;
+#pragma unroll
+        for (int x = lane; x < G * 16; x += 32) {   // G heads x 16 chunks of 8 dims
+          const int hh = x >> 4, ch = x & 15;
+          const int r = ee * G + hh;
+          const uint32_t dst = abase + (ch >> 3) * C::A_HALF + r * C::ROW + (((ch & 7) ^ (r & 7)) << 4);
+          asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(qrow + hh * D + ch * 8)
+                       : "memory");
+        }
+      }
+      asm volatile("cp.async.commit_group;" ::: "memory");
+      // this warp's next tile: descriptor and entries load while the copies fly
+      nxt = lt + NA < T ? a.tiles[t0 + lt + NA] : none;
+      nen0 = lane < nxt.w ? __ldg(a.entries + nxt.z + lane) : 0;
+      nen1 = (QPT > 32 && lane + 32 < nxt.w) ? __ldg(a.entries + nxt.z + 32 + lane) : 0;
+      asm volatile("cp.async.wait_group 0;" ::: "memory");
+      fence_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&a_full[q]);
+    }
+    asm volatile("cp.async.wait_group 0;" ::: "memory");
   }
 
   tc_fence_before();
@@ -689,7 +764,7 @@ cudaError_t run_block(const BlockPlan& pl, const CUtensorMap& tmK, const CUtenso
   using C = BlkCfg<BLK>;
   cudaError_t e = cudaFuncSetAttribute(attn_block_kernel<G, BLK>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
   if (e != cudaSuccess) return e;
-  attn_block_kernel<G, BLK><<<c.sm_count, 192, C::SMEM, c.stream>>>(tmK, tmV, a);
+  attn_block_kernel<G, BLK><<<c.sm_count, C::THREADS, C::SMEM, c.stream>>>(tmK, tmV, a);
   note_launch();
   (void)pl;
   return cudaGetLastError();

@@ -29,6 +29,7 @@ enum WaitSite : uint32_t {
   SITE_BLK_O_EMPTY = 0x415,
   SITE_BLK_S_FULL = 0x421,     // softmax / epilogue
   SITE_BLK_O_FULL = 0x422,
+  SITE_BLK_MMA_STALL = 0x416,  // the MMA issuer saw no progress
   SITE_BLK_BAD_ENTRY = 0x431,  // an entry outside the query rows (inconsistent plan)
 };
 
@@ -70,6 +71,19 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
       "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Non-blocking test of a phase (returns at once, unlike try_wait).
+__device__ __forceinline__ bool mbar_test_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
       "selp.u32 %0, 1, 0, p;\n\t}"
       : "=r"(ok)
       : "r"(smem_u32(bar)), "r"(parity)
