@@ -174,13 +174,17 @@ __global__ void __launch_bounds__(256) inv_tiles_kernel(const BlockPlan pl) {
 
 // ------------------------------------------------------------------ block tiles
 
-template <int BLK>
+template <int G, int BLK>
 struct BlkCfg {
   static constexpr int D = 128;
   static constexpr int ROW = 128;                       // bytes per 64-wide swizzled row
   static constexpr int A_HALF = 128 * ROW;              // 128 rows x 64 dims
   static constexpr int A_BYTES = 2 * A_HALF;            // Q tile
-  static constexpr int NA = (BLK == 64) ? 4 : 3;        // Q tile buffers = gather warps
+  // Q tile buffers: with G = 8 one warp fills them all by TMA; otherwise one
+  // cp.async warp per buffer
+  static constexpr bool TMA_Q = (G == 8);
+  static constexpr int NA = (BLK == 64) ? 4 : (TMA_Q ? 3 : 2);
+  static constexpr int NGW = TMA_Q ? 1 : NA;            // gather warps
   static constexpr int KV_HALF = BLK * ROW;             // BLK keys x 64 dims
   static constexpr int KV_BYTES = 4 * KV_HALF;          // K lo, K hi, V lo, V hi
   static constexpr int NKV = (BLK == 64) ? 2 : 1;       // K/V buffers (at most 2)
@@ -188,7 +192,11 @@ struct BlkCfg {
   static constexpr int P_BYTES = (BLK / 64) * P_HALF;
   static constexpr int NBAR = 2 * NA + 2 * NKV + 2 * 5 + 1;
   static constexpr int SMEM = 1024 + NA * A_BYTES + NKV * KV_BYTES + 2 * P_BYTES + NBAR * 8 + 16;
-  static constexpr int THREADS = 32 * (6 + NA);         // KV, MMA, 4 softmax, NA gather warps
+  static constexpr int SW0 = 2 + NGW;                   // first softmax warp
+  static constexpr int THREADS = 32 * (SW0 + 8);        // KV, MMA, gather, 2 x 4 softmax warps
+  // registers per thread: a sub-partition (SMSP) holds ceil(warps / 4) warps
+  // of its 16384 registers
+  static constexpr int MAXREG = (16384 / (32 * ((SW0 + 8 + 3) / 4))) & ~7;
   static constexpr int S_COL = 0;                       // TMEM: S[2] then O[2]
   static constexpr int O_COL = 2 * BLK;
   static_assert(SMEM <= 232448, "shared memory");
@@ -245,21 +253,23 @@ __device__ __forceinline__ void tmem_ld64(uint32_t taddr, uint32_t (&r)[64]) {
 
 // One CTA per SM walks a contiguous range of tiles (ordered by key block, so
 // a block's K_c, V_c are loaded once per CTA).  Warp roles:
-//   0          K/V producer: TMA of each new block's K_c, V_c;
-//   1          MMA issuer and TMEM owner: a non-blocking loop that issues
-//              S = Q K_c^T for the next tile whose Q rows have landed and
-//              O = P V_c for the oldest tile whose P is written, whichever
-//              is ready first;
-//   2..5       softmax and epilogue, one tensor-core row = one
-//              (query, head) pair per thread;
-//   6..6+NA-1  Q gather: warp q fills Q buffer q with the rows of tiles
-//              q, q + NA, ... (16-byte asynchronous copies to their
-//              128-byte-swizzled positions), so NA tiles are in flight.
+//   0      K/V producer: TMA of each new block's K_c, V_c;
+//   1      MMA issuer and TMEM owner: a non-blocking loop that issues
+//          S = Q K_c^T for the next tile whose Q rows have landed and
+//          O = P V_c for the oldest tile whose P is written, whichever is
+//          ready first;
+//   2 ..   Q gather into NA buffers: with G = 8 one warp issues two TMA
+//          boxes per entry for every tile; otherwise warp 2 + q fills
+//          buffer q with the rows of tiles q, q + NA, ... (16-byte
+//          asynchronous copies to their 128-byte-swizzled positions);
+//   SW0 .. softmax and epilogue in two groups of four warps that take
+//          alternate tiles (S, P and O are double-buffered by tile parity),
+//          one tensor-core row = one (query, head) pair per thread.
 template <int G, int BLK>
-__global__ void __launch_bounds__(BlkCfg<BLK>::THREADS, 1)
+__global__ void __maxnreg__((BlkCfg<G, BLK>::MAXREG))
     attn_block_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
-                      const BlkArgs a) {
-  using C = BlkCfg<BLK>;
+                      const __grid_constant__ CUtensorMap tmQ, const BlkArgs a) {
+  using C = BlkCfg<G, BLK>;
   constexpr int D = C::D;
   constexpr int QPT = 128 / G;
   constexpr int NA = C::NA;
@@ -293,6 +303,7 @@ __global__ void __launch_bounds__(BlkCfg<BLK>::THREADS, 1)
     fence_barrier_init();
     tma_prefetch_desc(&tmK);
     tma_prefetch_desc(&tmV);
+    if (C::TMA_Q) tma_prefetch_desc(&tmQ);
   }
   if (warp == 1) {
     tmem_alloc(tmem_slot, 512);
@@ -432,83 +443,23 @@ __global__ void __launch_bounds__(BlkCfg<BLK>::THREADS, 1)
       const uint64_t tq = global_timer_ns();
       while (!mbar_try_wait(mma_done, 0) && global_timer_ns() - tq < kWaitLimitNs) {}
     }
-  } else if (warp < 6) {
+  } else if (warp >= C::SW0) {
     // ------------------------------------------------------------ softmax + epilogue
-    // Software-pipelined: the softmax of tile t, then the epilogue of tile
-    // t - 1 (O is double-buffered in TMEM), so P V of tile t runs while the
-    // previous tile's output is stored.
+    const int grp = (warp - C::SW0) >> 2;     // tiles grp, grp + 2, ...
     const int eq = warp & 3;
     const int row = eq * 32 + lane;
     const int e = row / G, h = row % G;
     const uint32_t lane_base = static_cast<uint32_t>(eq * 32) << 16;
+    const int sb = grp;                        // this group's S, P and O buffers
     bool ok = true;
-    // tile descriptors two ahead and this thread's entry one ahead of use
-    int4 nxt = T > 0 ? a.tiles[t0] : none;
-    int4 nxt2 = T > 1 ? a.tiles[t0 + 1] : none;
+    // this group's tile descriptors one ahead and this thread's entry with it
+    int4 nxt = grp < T ? a.tiles[t0 + grp] : none;
     int nxt_ent = e < nxt.w ? __ldg(a.entries + nxt.z + e) : 0;
-    // the pending epilogue: its slot row, validity and softmax statistics
-    int64_t pend_slot = 0;
-    bool pend_valid = false;
-    float pend_m = 0.f, pend_l = 1.f;
-    auto epilogue = [&](int lt) -> bool {
-      const int sb = lt & 1;
-      if (!__all_sync(0xFFFFFFFFu, mbar_wait(&o_full[sb], (lt >> 1) & 1, a.err, SITE_BLK_O_FULL))) return false;
-      tc_fence_after();
-      // two passes over the row in halves of 64 columns: its largest
-      // magnitude, then the scaled float16 conversion
-      const uint32_t ocol = tmem_base + lane_base + C::O_COL + sb * D;
-      float am[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};   // eight independent chains
-#pragma unroll
-      for (int hf = 0; hf < D / 64; ++hf) {
-        uint32_t r[64];
-        tmem_ld64(ocol + hf * 64, r);
-#pragma unroll
-        for (int u = 0; u < 64; ++u) am[u & 7] = fmaxf(am[u & 7], fabsf(__uint_as_float(r[u])));
-      }
-      const float amax = max8(am);
-      // the normalised row o = O / l, stored as float16 times 2^-e with the
-      // power of two 2^e chosen so the row's largest entry lands in
-      // [2^14, 2^15): 11 significant bits whatever the scale of V.  Every
-      // lane runs the (warp-collective) TMEM loads; only valid rows store.
-      const float inv_l = 1.f / pend_l;
-      const float x = amax * inv_l;
-      int ex = x > 0.f ? static_cast<int>((__float_as_uint(x) >> 23) & 0xFFu) - 127 - 14 : 0;
-      ex = min(max(ex, -100), 100);
-      const float mul = inv_l * __uint_as_float(static_cast<uint32_t>(127 - ex) << 23);
-      uint4* dst = reinterpret_cast<uint4*>(a.partO + pend_slot * D);
-#pragma unroll
-      for (int hf = 0; hf < D / 64; ++hf) {
-        uint32_t r[64];
-        tmem_ld64(ocol + hf * 64, r);
-        if (pend_valid) {
-#pragma unroll
-          for (int q = 0; q < 8; ++q) {
-            uint32_t w[4];
-#pragma unroll
-            for (int u = 0; u < 4; ++u) {
-              const __half2 hv = __floats2half2_rn(__uint_as_float(r[q * 8 + 2 * u]) * mul,
-                                                   __uint_as_float(r[q * 8 + 2 * u + 1]) * mul);
-              w[u] = *reinterpret_cast<const uint32_t*>(&hv);
-            }
-            dst[hf * 8 + q] = make_uint4(w[0], w[1], w[2], w[3]);
-          }
-        }
-      }
-      if (pend_valid)
-        a.partL[pend_slot] = make_float2(pend_m + log2f(pend_l),
-                                         __uint_as_float(static_cast<uint32_t>(127 + ex) << 23));
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&o_empty[sb]);
-      return true;
-    };
-    for (int t = t0; t < t1 && ok; ++t) {
-      const int lt = t - t0;
-      const int sb = lt & 1;
+    for (int lt = grp; lt < T && ok; lt += 2) {
+      const int use = lt >> 1;                 // this buffer's use count
       const int4 td = nxt;
       const int ent = nxt_ent;
-      nxt = nxt2;
-      nxt2 = t + 2 < t1 ? a.tiles[t + 2] : none;
+      nxt = lt + 2 < T ? a.tiles[t0 + lt + 2] : none;
       nxt_ent = e < nxt.w ? __ldg(a.entries + nxt.z + e) : 0;
       const int bg = td.x, ne = td.w;
       const int i = entry_row(ent), j = entry_slot(ent);
@@ -521,12 +472,11 @@ __global__ void __launch_bounds__(BlkCfg<BLK>::THREADS, 1)
         klo = static_cast<int>(max(lo - base, static_cast<int64_t>(0)));
         khi = static_cast<int>(min(pos - base, static_cast<int64_t>(BLK - 1)));
       }
-      ok = __all_sync(0xFFFFFFFFu, mbar_wait(&s_full[sb], (lt >> 1) & 1, a.err, SITE_BLK_S_FULL));
+      ok = __all_sync(0xFFFFFFFFu, mbar_wait(&s_full[sb], use & 1, a.err, SITE_BLK_S_FULL));
       if (!ok) break;
       tc_fence_after();
       // the row's scaled logits in halves of 64 columns: the maximum, then
-      // P = 2^(s - m) in bfloat16 into the swizzled P tile (one pass when
-      // the block is 64 keys)
+      // P = 2^(s - m) in bfloat16 into the swizzled P tile
       const uint32_t scol = tmem_base + lane_base + C::S_COL + sb * BLK;
       // a half of S, loaded with the columns outside [klo, khi] set to -inf;
       // most tiles hold no window slot, and their warps skip the masking
@@ -539,9 +489,7 @@ __global__ void __launch_bounds__(BlkCfg<BLK>::THREADS, 1)
           for (int u = 0; u < 64; ++u) r[u] = (u >= lo && u <= hi) ? r[u] : 0xFF800000u;
         }
       };
-      auto logit = [&](uint32_t raw, int) { return __uint_as_float(raw) * a.scale_log2; };
-      // maxima and sums in eight independent chains (one warp per SMSP runs
-      // this, so dependent chains would cost their full latency)
+      // maxima and sums in eight independent chains
       float mx[8] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY, -INFINITY, -INFINITY, -INFINITY, -INFINITY};
       float ls[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
       float m = -INFINITY;
@@ -552,9 +500,9 @@ __global__ void __launch_bounds__(BlkCfg<BLK>::THREADS, 1)
           uint32_t r[64];
           load_half(hf, r);
 #pragma unroll
-          for (int u = 0; u < 64; ++u) mx[u & 7] = fmaxf(mx[u & 7], logit(r[u], hf * 64 + u));
+          for (int u = 0; u < 64; ++u) mx[u & 7] = fmaxf(mx[u & 7], __uint_as_float(r[u]));
         }
-        m = max8(mx);
+        m = max8(mx) * a.scale_log2;
       }
 #pragma unroll
       for (int hf = 0; hf < BLK / 64; ++hf) {
@@ -562,8 +510,8 @@ __global__ void __launch_bounds__(BlkCfg<BLK>::THREADS, 1)
         load_half(hf, r);
         if (BLK == 64) {
 #pragma unroll
-          for (int u = 0; u < 64; ++u) mx[u & 7] = fmaxf(mx[u & 7], logit(r[u], u));
-          m = max8(mx);
+          for (int u = 0; u < 64; ++u) mx[u & 7] = fmaxf(mx[u & 7], __uint_as_float(r[u]));
+          m = max8(mx) * a.scale_log2;
         }
         if (hf == BLK / 64 - 1) {   // all of S is in registers or consumed: free the buffer
           tc_fence_before();
@@ -575,9 +523,8 @@ __global__ void __launch_bounds__(BlkCfg<BLK>::THREADS, 1)
           uint32_t w[4];
 #pragma unroll
           for (int u = 0; u < 4; ++u) {
-            const int c0 = hf * 64 + ch * 8 + 2 * u;
-            const float p0 = fast_exp2(logit(r[ch * 8 + 2 * u], c0) - m);
-            const float p1 = fast_exp2(logit(r[ch * 8 + 2 * u + 1], c0 + 1) - m);
+            const float p0 = fast_exp2(fmaf(__uint_as_float(r[ch * 8 + 2 * u]), a.scale_log2, -m));
+            const float p1 = fast_exp2(fmaf(__uint_as_float(r[ch * 8 + 2 * u + 1]), a.scale_log2, -m));
             ls[2 * u] += p0;
             ls[2 * u + 1] += p1;
             w[u] = pack_bf16(p0, p1);
@@ -590,58 +537,151 @@ __global__ void __launch_bounds__(BlkCfg<BLK>::THREADS, 1)
       fence_async_smem();
       __syncwarp();
       if (lane == 0) mbar_arrive(&p_full[sb]);
-      if (lt > 0 && !epilogue(lt - 1)) { ok = false; break; }
-      pend_slot = ((static_cast<int64_t>(bg) * a.n_q + i) * a.nsl + j) * G + h;
-      pend_valid = valid;
-      pend_m = m;
-      pend_l = l;
+      // epilogue: O of this tile (the other group's softmax runs meanwhile)
+      ok = __all_sync(0xFFFFFFFFu, mbar_wait(&o_full[sb], use & 1, a.err, SITE_BLK_O_FULL));
+      if (!ok) break;
+      tc_fence_after();
+      // two passes over the row in halves of 64 columns: its largest
+      // magnitude, then the scaled float16 conversion
+      const uint32_t ocol = tmem_base + lane_base + C::O_COL + sb * D;
+      float am[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int hf = 0; hf < D / 64; ++hf) {
+        uint32_t r[64];
+        tmem_ld64(ocol + hf * 64, r);
+#pragma unroll
+        for (int u = 0; u < 64; ++u) am[u & 7] = fmaxf(am[u & 7], fabsf(__uint_as_float(r[u])));
+      }
+      const float amax = max8(am);
+      // the normalised row o = O / l, stored as float16 times 2^-e with the
+      // power of two 2^e chosen so the row's largest entry lands in
+      // [2^14, 2^15): 11 significant bits whatever the scale of V.  Every
+      // lane runs the (warp-collective) TMEM loads; only valid rows store.
+      const float inv_l = 1.f / l;
+      const float x = amax * inv_l;
+      int ex = x > 0.f ? static_cast<int>((__float_as_uint(x) >> 23) & 0xFFu) - 127 - 14 : 0;
+      ex = min(max(ex, -100), 100);
+      const float mul = inv_l * __uint_as_float(static_cast<uint32_t>(127 - ex) << 23);
+      const int64_t slot = ((static_cast<int64_t>(bg) * a.n_q + i) * a.nsl + j) * G + h;
+      // Coalesced stores: each warp passes its 32 rows through its own 32
+      // rows of this group's P tile (free once P V has run), 16-byte chunks
+      // XOR-swizzled by row against bank conflicts, then writes four whole
+      // 128-byte half-rows per instruction.
+      uint8_t* stage = sP + sb * C::P_BYTES + eq * 32 * C::ROW;
+      const int srow = lane >> 3, sch = lane & 7;   // store phase: row k*4 + srow, chunk sch
+#pragma unroll
+      for (int hf = 0; hf < D / 64; ++hf) {
+        uint32_t r[64];
+        tmem_ld64(ocol + hf * 64, r);
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+          uint32_t w[4];
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            const __half2 hv = __floats2half2_rn(__uint_as_float(r[q * 8 + 2 * u]) * mul,
+                                                 __uint_as_float(r[q * 8 + 2 * u + 1]) * mul);
+            w[u] = *reinterpret_cast<const uint32_t*>(&hv);
+          }
+          *reinterpret_cast<uint4*>(stage + lane * C::ROW + ((q ^ (lane & 7)) << 4)) = make_uint4(w[0], w[1], w[2], w[3]);
+        }
+        __syncwarp();
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          const int rr = k * 4 + srow;   // the warp lane whose row this is
+          const int64_t rslot = __shfl_sync(0xFFFFFFFFu, slot, rr);
+          const bool rvalid = __shfl_sync(0xFFFFFFFFu, valid ? 1 : 0, rr) != 0;
+          const uint4 v = *reinterpret_cast<const uint4*>(stage + rr * C::ROW + ((sch ^ (rr & 7)) << 4));
+          if (rvalid) reinterpret_cast<uint4*>(a.partO + rslot * D + hf * 64)[sch] = v;
+        }
+        __syncwarp();
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&o_empty[sb]);
+      if (valid) a.partL[slot] = make_float2(m + log2f(l), __uint_as_float(static_cast<uint32_t>(127 + ex) << 23));
     }
-    if (ok && T > 0) epilogue(T - 1);
   } else {
     // ------------------------------------------------------------ Q gather
-    const int q = warp - 6;   // buffer q: tiles q, q + NA, ...
-    const uint32_t abase = smem_u32(sA + q * C::A_BYTES);
+    const int q = warp - 2;   // tiles q, q + NGW, ... into buffers lt % NA
     bool ok = true;
     int4 nxt = q < T ? a.tiles[t0 + q] : none;
     int nen0 = lane < nxt.w ? __ldg(a.entries + nxt.z + lane) : 0;
     int nen1 = (QPT > 32 && lane + 32 < nxt.w) ? __ldg(a.entries + nxt.z + 32 + lane) : 0;
-    uint32_t uses = 0;
-    for (int lt = q; lt < T && ok; lt += NA, ++uses) {
+    int last_lt = -1;
+    for (int lt = q; lt < T && ok; lt += C::NGW) {
+      const int ab = lt % NA;
+      const uint32_t use = static_cast<uint32_t>(lt / NA);
       const int4 td = nxt;
       const int en0 = nen0, en1 = nen1;
       const int b = td.x / a.h_kv, g = td.x % a.h_kv, ne = td.w;
-      if (lane == 0) ok = mbar_wait(&a_empty[q], (uses & 1) ^ 1, a.err, SITE_BLK_A_EMPTY);
+      if (lane == 0) ok = mbar_wait(&a_empty[ab], (use & 1) ^ 1, a.err, SITE_BLK_A_EMPTY);
       ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
       if (!ok) break;
-      for (int ee = 0; ee < ne; ++ee) {
-        const int ent = ee < 32 ? __shfl_sync(0xFFFFFFFFu, en0, ee) : __shfl_sync(0xFFFFFFFFu, en1, ee - 32);
-        const int i = entry_row(ent);
-        if (static_cast<unsigned>(i) >= static_cast<unsigned>(a.n_q)) {   // never for a consistent plan
-          if (lane == 0) atomicCAS(a.err, 0u, static_cast<uint32_t>(SITE_BLK_BAD_ENTRY));
-          continue;
-        }
-        const __nv_bfloat16* qrow = a.Q + ((static_cast<int64_t>(b) * a.n_q + i) * a.h_q +
-                                           static_cast<int64_t>(g) * G) * D;
+      last_lt = lt;
+      uint8_t* abuf = sA + ab * C::A_BYTES;
+      if (C::TMA_Q) {
+        // an entry's 8 query heads are 8 tensor-core rows = one 1024-byte
+        // swizzle atom per 64-dim half: two TMA boxes per entry
+        if (lane == 0) mbar_arrive_expect_tx(&a_full[ab], static_cast<uint32_t>(ne) * G * D * 2);
+        for (int ee = 0; ee < ne; ++ee) {
+          const int ent = __shfl_sync(0xFFFFFFFFu, en0, ee);
+          const int i = entry_row(ent);
+          if (static_cast<unsigned>(i) >= static_cast<unsigned>(a.n_q)) {   // never for a consistent plan
+            if (lane == 0) atomicCAS(a.err, 0u, static_cast<uint32_t>(SITE_BLK_BAD_ENTRY));
+            ok = false;
+            break;
+          }
+          if (lane == 0) {
+            const int z = static_cast<int>(static_cast<int64_t>(b) * a.n_q + i);
 #pragma unroll
-        for (int x = lane; x < G * 16; x += 32) {   // G heads x 16 chunks of 8 dims
-          const int hh = x >> 4, ch = x & 15;
-          const int r = ee * G + hh;
-          const uint32_t dst = abase + (ch >> 3) * C::A_HALF + r * C::ROW + (((ch & 7) ^ (r & 7)) << 4);
-          asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(qrow + hh * D + ch * 8)
-                       : "memory");
+            for (int hf = 0; hf < 2; ++hf)
+              tma_load_3d(abuf + hf * C::A_HALF + ee * (G * C::ROW), &tmQ, &a_full[ab], hf * 64, g * G, z);
+          }
         }
+        nxt = lt + C::NGW < T ? a.tiles[t0 + lt + C::NGW] : none;
+        nen0 = lane < nxt.w ? __ldg(a.entries + nxt.z + lane) : 0;
+      } else {
+        const uint32_t abase = smem_u32(abuf);
+        for (int ee = 0; ee < ne; ++ee) {
+          const int ent = ee < 32 ? __shfl_sync(0xFFFFFFFFu, en0, ee) : __shfl_sync(0xFFFFFFFFu, en1, ee - 32);
+          const int i = entry_row(ent);
+          if (static_cast<unsigned>(i) >= static_cast<unsigned>(a.n_q)) {   // never for a consistent plan
+            if (lane == 0) atomicCAS(a.err, 0u, static_cast<uint32_t>(SITE_BLK_BAD_ENTRY));
+            continue;
+          }
+          const __nv_bfloat16* qrow = a.Q + ((static_cast<int64_t>(b) * a.n_q + i) * a.h_q +
+                                             static_cast<int64_t>(g) * G) * D;
+#pragma unroll
+          for (int x = lane; x < G * 16; x += 32) {   // G heads x 16 chunks of 8 dims
+            const int hh = x >> 4, ch = x & 15;
+            const int r = ee * G + hh;
+            const uint32_t dst = abase + (ch >> 3) * C::A_HALF + r * C::ROW + (((ch & 7) ^ (r & 7)) << 4);
+            asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(qrow + hh * D + ch * 8)
+                         : "memory");
+          }
+        }
+        asm volatile("cp.async.commit_group;" ::: "memory");
+        // this warp's next tile: descriptor and entries load while the copies fly
+        nxt = lt + C::NGW < T ? a.tiles[t0 + lt + C::NGW] : none;
+        nen0 = lane < nxt.w ? __ldg(a.entries + nxt.z + lane) : 0;
+        nen1 = (QPT > 32 && lane + 32 < nxt.w) ? __ldg(a.entries + nxt.z + 32 + lane) : 0;
+        asm volatile("cp.async.wait_group 0;" ::: "memory");
+        fence_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&a_full[ab]);
       }
-      asm volatile("cp.async.commit_group;" ::: "memory");
-      // this warp's next tile: descriptor and entries load while the copies fly
-      nxt = lt + NA < T ? a.tiles[t0 + lt + NA] : none;
-      nen0 = lane < nxt.w ? __ldg(a.entries + nxt.z + lane) : 0;
-      nen1 = (QPT > 32 && lane + 32 < nxt.w) ? __ldg(a.entries + nxt.z + 32 + lane) : 0;
-      asm volatile("cp.async.wait_group 0;" ::: "memory");
-      fence_async_smem();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&a_full[q]);
     }
-    asm volatile("cp.async.wait_group 0;" ::: "memory");
+    if (C::TMA_Q) {
+      // after a failure, let the TMA boxes of the buffers in flight land before
+      // the CTA exits
+      if (!ok && lane == 0) {
+        const uint64_t tq = global_timer_ns();
+        for (int lt = (last_lt - NA + 1 > 0 ? last_lt - NA + 1 : 0); lt <= last_lt; ++lt)
+          while (!mbar_try_wait(&a_full[lt % NA], (lt / NA) & 1) && global_timer_ns() - tq < kWaitLimitNs) {}
+      }
+    } else {
+      asm volatile("cp.async.wait_group 0;" ::: "memory");
+    }
   }
 
   tc_fence_before();
@@ -759,12 +799,12 @@ __global__ void __launch_bounds__(256) attn_merge_kernel(const MergeArgs a) {
 }
 
 template <int G, int BLK>
-cudaError_t run_block(const BlockPlan& pl, const CUtensorMap& tmK, const CUtensorMap& tmV,
+cudaError_t run_block(const BlockPlan& pl, const CUtensorMap& tmK, const CUtensorMap& tmV, const CUtensorMap& tmQ,
                       const BlkArgs& a, const LaunchCtx& c) {
-  using C = BlkCfg<BLK>;
+  using C = BlkCfg<G, BLK>;
   cudaError_t e = cudaFuncSetAttribute(attn_block_kernel<G, BLK>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
   if (e != cudaSuccess) return e;
-  attn_block_kernel<G, BLK><<<c.sm_count, C::THREADS, C::SMEM, c.stream>>>(tmK, tmV, a);
+  attn_block_kernel<G, BLK><<<c.sm_count, C::THREADS, C::SMEM, c.stream>>>(tmK, tmV, tmQ, a);
   note_launch();
   (void)pl;
   return cudaGetLastError();
@@ -798,7 +838,7 @@ cudaError_t launch_attn_merge(const ssa_params& p, const int32_t* block_idx, con
   return cudaGetLastError();
 }
 
-int attn_block_smem_bytes(int block) { return block == 64 ? BlkCfg<64>::SMEM : BlkCfg<128>::SMEM; }
+int attn_block_smem_bytes(int block) { return block == 64 ? BlkCfg<4, 64>::SMEM : BlkCfg<4, 128>::SMEM; }
 
 cudaError_t launch_block_plan(const ssa_params& p, const int32_t* block_idx, const BlockPlan& pl,
                               const LaunchCtx& c) {
@@ -828,8 +868,8 @@ cudaError_t launch_block_plan(const ssa_params& p, const int32_t* block_idx, con
 }
 
 cudaError_t launch_attn_block(const ssa_params& p, const BlockPlan& pl, const void* Q,
-                              const CUtensorMap& tmK, const CUtensorMap& tmV, void* partO, void* partL,
-                              const LaunchCtx& c) {
+                              const CUtensorMap& tmK, const CUtensorMap& tmV, const CUtensorMap& tmQ,
+                              void* partO, void* partL, const LaunchCtx& c) {
   BlkArgs a;
   a.Q = static_cast<const __nv_bfloat16*>(Q);
   a.tiles = pl.tiles;
@@ -845,13 +885,13 @@ cudaError_t launch_attn_block(const ssa_params& p, const BlockPlan& pl, const vo
   const int G = p.h_q / p.h_kv;
   if (p.d != 128) return cudaErrorInvalidValue;
   if (p.block == 64) {
-    if (G == 2) return run_block<2, 64>(pl, tmK, tmV, a, c);
-    if (G == 4) return run_block<4, 64>(pl, tmK, tmV, a, c);
-    if (G == 8) return run_block<8, 64>(pl, tmK, tmV, a, c);
+    if (G == 2) return run_block<2, 64>(pl, tmK, tmV, tmQ, a, c);
+    if (G == 4) return run_block<4, 64>(pl, tmK, tmV, tmQ, a, c);
+    if (G == 8) return run_block<8, 64>(pl, tmK, tmV, tmQ, a, c);
   } else if (p.block == 128) {
-    if (G == 2) return run_block<2, 128>(pl, tmK, tmV, a, c);
-    if (G == 4) return run_block<4, 128>(pl, tmK, tmV, a, c);
-    if (G == 8) return run_block<8, 128>(pl, tmK, tmV, a, c);
+    if (G == 2) return run_block<2, 128>(pl, tmK, tmV, tmQ, a, c);
+    if (G == 4) return run_block<4, 128>(pl, tmK, tmV, tmQ, a, c);
+    if (G == 8) return run_block<8, 128>(pl, tmK, tmV, tmQ, a, c);
   }
   return cudaErrorInvalidValue;
 }

@@ -72,9 +72,11 @@ cudaError_t launch_block_plan(const ssa_params& p, const int32_t* block_idx, con
 // tcgen05 block tiles -> per-(query, head, slot) normalised partial outputs
 // partO [items][topk][G][d] (float16, row-scaled by 2^-e) and partL
 // [items][stride] of (base-2 log-sum-exp, 2^e).
+// tmQ: Q as [b * n_q, h_q, d], 128-byte-swizzled boxes of 64 dims x 8 heads
+// (used when G = 8).
 cudaError_t launch_attn_block(const ssa_params& p, const BlockPlan& pl, const void* Q,
-                              const CUtensorMap& tmK, const CUtensorMap& tmV, void* partO, void* partL,
-                              const LaunchCtx& c);
+                              const CUtensorMap& tmK, const CUtensorMap& tmV, const CUtensorMap& tmQ,
+                              void* partO, void* partL, const LaunchCtx& c);
 
 // Per (query, kv-head): the softmax merge of the slot partials into O, lse.
 cudaError_t launch_attn_merge(const ssa_params& p, const int32_t* block_idx, const void* partO, const void* partL,

@@ -231,6 +231,21 @@ bool encode_kv(CUtensorMap* m, const void* base, const ssa_params& p) {
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// 3D bf16 map of Q viewed as [b*n_q, h_q, d]; 128-byte-swizzled boxes of
+// 64 dims x 8 heads x 1 query row.
+bool encode_q_heads(CUtensorMap* m, const void* base, const ssa_params& p) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[3] = {static_cast<cuuint64_t>(p.d), static_cast<cuuint64_t>(p.h_q),
+                              static_cast<cuuint64_t>(p.batch) * p.n_q};
+  const cuuint64_t strides[2] = {static_cast<cuuint64_t>(p.d) * 2, static_cast<cuuint64_t>(p.h_q) * p.d * 2};
+  const cuuint32_t box[3] = {64, 8, 1};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 ssa_status do_summary(const ssa_params& p, const void* K, float* mu, float* sigma, void* table,
                       const LaunchCtx& c) {
   if (p.batch == 0 || p.n_kv == 0) return SSA_OK;
@@ -288,13 +303,17 @@ ssa::BlockPlan block_plan(const ssa_params& p, const AttnLayout& L, uint8_t* w) 
 }
 
 struct AttnMaps {
-  CUtensorMap K, V, Q;
+  CUtensorMap K, V, Q, Qh;   // Q: unswizzled G-row boxes (gather path); Qh: 8-head boxes (G = 8 tiles)
 };
 
 bool encode_attn_maps(AttnMaps& m, const ssa_params& p, const void* Q, const void* K, const void* V) {
   const uint32_t G = static_cast<uint32_t>(p.h_q / p.h_kv);
-  return encode_kv(&m.K, K, p) && encode_kv(&m.V, V, p) &&
-         encode_rows(&m.Q, Q, p.d, static_cast<uint64_t>(p.batch) * p.n_q * p.h_q, G);
+  if (!encode_kv(&m.K, K, p) || !encode_kv(&m.V, V, p) ||
+      !encode_rows(&m.Q, Q, p.d, static_cast<uint64_t>(p.batch) * p.n_q * p.h_q, G))
+    return false;
+  if (G == 8 && p.d == 128) return encode_q_heads(&m.Qh, Q, p);
+  m.Qh = m.Q;
+  return true;
 }
 
 // Block-major stages; the caller has checked that the problem qualifies and
@@ -306,7 +325,7 @@ ssa_status attn_stage_plan(const ssa_params& p, const int32_t* idx, uint8_t* w, 
 
 ssa_status attn_stage_blocks(const ssa_params& p, const void* Q, const AttnMaps& m, uint8_t* w, const LaunchCtx& c) {
   const AttnLayout L = attn_layout(p);
-  return from_cuda(ssa::launch_attn_block(p, block_plan(p, L, w), Q, m.K, m.V, w + L.part_o, w + L.part_l, c));
+  return from_cuda(ssa::launch_attn_block(p, block_plan(p, L, w), Q, m.K, m.V, m.Qh, w + L.part_o, w + L.part_l, c));
 }
 
 ssa_status attn_stage_merge(const ssa_params& p, const int32_t* idx, void* O, float* lse, int32_t* bad,
