@@ -123,46 +123,70 @@ __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity, uint3
   }
 }
 
+// Merges this row's buffered candidates into its top list: a descending
+// register list of (score, block), KSEL long, of which the first k count.
+// Candidates are inserted one at a time in arrival order (ascending block
+// index) and an equal score is placed after the entries already held, so a
+// lower block index wins ties.  Each insertion is a branchless shift over the
+// list with independent compares; the loop runs to the warp's largest count
+// (lanes past their own count insert -inf, which changes nothing).
 template <int KSEL>
-__device__ __forceinline__ void compact(uint64_t (&L)[KSEL], int& cnt, float& thr,
-                                        const uint2* my_cand, int k) {
-  uint64_t Bk[32];
+__device__ __forceinline__ void merge_candidates(float (&Ls)[KSEL], int (&Li)[KSEL], int& cnt, float& thr,
+                                                 const uint2* my_cand, int k) {
+  int n = cnt;
 #pragma unroll
-  for (int t = 0; t < 32; ++t) {
-    uint64_t key = 0;
+  for (int o = 16; o; o >>= 1) n = max(n, __shfl_xor_sync(0xFFFFFFFFu, n, o));
+#pragma unroll 1
+  for (int t = 0; t < n; ++t) {
+    float x = -INFINITY;
+    int xi = 0;
     if (t < cnt) {
       const uint2 e = my_cand[t * 128];
-      key = make_key(e.x, e.y);
+      x = __uint_as_float(e.x);
+      xi = static_cast<int>(e.y);
     }
-    Bk[t] = key;
-  }
-  bitonic_sort_desc<32>(Bk);
+    bool gt[KSEL];
 #pragma unroll
-  for (int j = 0; j < KSEL; ++j) {
-    const uint64_t y = Bk[KSEL - 1 - j];
-    L[j] = L[j] < y ? y : L[j];
+    for (int j = 0; j < KSEL; ++j) gt[j] = x > Ls[j];
+#pragma unroll
+    for (int j = KSEL - 1; j >= 1; --j) {
+      Ls[j] = gt[j - 1] ? Ls[j - 1] : (gt[j] ? x : Ls[j]);
+      Li[j] = gt[j - 1] ? Li[j - 1] : (gt[j] ? xi : Li[j]);
+    }
+    Ls[0] = gt[0] ? x : Ls[0];
+    Li[0] = gt[0] ? xi : Li[0];
   }
-  bitonic_merge_desc<KSEL>(L);
   cnt = 0;
-  uint64_t kth = 0;
+  // the k-th best (the list is descending: the least of its first k)
+  float kth = INFINITY;
 #pragma unroll
   for (int j = 0; j < KSEL; ++j)
-    if (j == k - 1) kth = L[j];
-  thr = kth ? key_score(kth) : -INFINITY;
+    if (j < k) kth = fminf(kth, Ls[j]);
+  thr = kth;
 }
 
+// Appends the scores above the threshold (strictly: an equal score comes
+// from a higher block index and would rank below the k-th) to the row's
+// candidate buffer, in block order: independent compares build a take mask,
+// then one store per set bit.
 template <bool MASK>
 __device__ __forceinline__ void filter16(const uint32_t (&v)[16], int c0, int nvis, float thr,
                                          int& cnt, uint2* my_cand) {
+  uint32_t take = 0;
 #pragma unroll
   for (int t = 0; t < 16; ++t) {
-    const float s = __uint_as_float(v[t]);
-    bool take = s >= thr;
-    if (MASK) take = take && (c0 + t < nvis);
-    if (take) {
-      my_cand[cnt * 128] = make_uint2(v[t], static_cast<uint32_t>(c0 + t));
-      ++cnt;
-    }
+    bool tk = __uint_as_float(v[t]) > thr;
+    if (MASK) tk = tk && (c0 + t < nvis);
+    take |= tk ? (1u << t) : 0u;
+  }
+  // one store per taken score, lowest column first (block order)
+  for (uint32_t m = take; m; m &= m - 1u) {
+    const int t = __ffs(static_cast<int>(m)) - 1;
+    uint32_t vt = v[0];
+#pragma unroll
+    for (int u = 1; u < 16; ++u) vt = (t == u) ? v[u] : vt;
+    my_cand[cnt * 128] = make_uint2(vt, static_cast<uint32_t>(c0 + t));
+    ++cnt;
   }
 }
 
@@ -303,9 +327,10 @@ __global__ void __launch_bounds__(192, 1)
       const int i = row0 + row;
       const bool valid = i < a.n_q;
       const int nvis = valid ? static_cast<int>(min(static_cast<int64_t>(a.nb), (a.q_offset + i + 1) / a.block)) : 0;
-      uint64_t L[KSEL];
+      float Ls[KSEL];
+      int Li[KSEL];
 #pragma unroll
-      for (int j = 0; j < KSEL; ++j) L[j] = 0;
+      for (int j = 0; j < KSEL; ++j) { Ls[j] = -INFINITY; Li[j] = -1; }
       float thr = -INFINITY;
       int cnt = 0;
       for (int j = 0; j < nch; ++j) {
@@ -329,20 +354,20 @@ __global__ void __launch_bounds__(192, 1)
             filter16<false>(v, c0, nvis, thr, cnt, my_cand);
           else
             filter16<true>(v, c0, nvis, thr, cnt, my_cand);
-          if (__any_sync(0xFFFFFFFFu, cnt > C::CAP - 16)) compact<KSEL>(L, cnt, thr, my_cand, a.topk);
+          if (__any_sync(0xFFFFFFFFu, cnt > C::CAP - 16)) merge_candidates<KSEL>(Ls, Li, cnt, thr, my_cand, a.topk);
         }
         ++acc_cnt;
       }
       if (!ok) break;
-      if (__any_sync(0xFFFFFFFFu, cnt > 0)) compact<KSEL>(L, cnt, thr, my_cand, a.topk);
+      if (__any_sync(0xFFFFFFFFu, cnt > 0)) merge_candidates<KSEL>(Ls, Li, cnt, thr, my_cand, a.topk);
       if (valid) {
         uint32_t ob[KSEL];
         float os[KSEL];
 #pragma unroll
         for (int j = 0; j < KSEL; ++j) {
-          const bool use = (j < a.topk) && L[j] != 0;
-          ob[j] = use ? key_block(L[j]) : 0xFFFFFFFFu;
-          os[j] = use ? key_score(L[j]) : -INFINITY;
+          const bool use = (j < a.topk) && Li[j] >= 0;
+          ob[j] = use ? static_cast<uint32_t>(Li[j]) : 0xFFFFFFFFu;
+          os[j] = use ? Ls[j] : -INFINITY;
         }
         bitonic_sort_asc_u32<KSEL>(ob, os);
         const int b = bg / a.h_kv, g = bg % a.h_kv;
