@@ -69,7 +69,18 @@ __global__ void __launch_bounds__(256) inv_colscan_kernel(const BlockPlan pl) {
   const int bg = static_cast<int>(x / pl.nb), c = static_cast<int>(x % pl.nb);
   int32_t* col = pl.chist + static_cast<int64_t>(bg) * pl.nchunk * pl.nb + c;
   int run = 0;
-  for (int k = 0; k < pl.nchunk; ++k) {
+  int k = 0;
+  for (; k + 8 <= pl.nchunk; k += 8) {   // eight loads in flight per thread
+    int v[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) v[u] = col[static_cast<int64_t>(k + u) * pl.nb];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      col[static_cast<int64_t>(k + u) * pl.nb] = run;
+      run += v[u];
+    }
+  }
+  for (; k < pl.nchunk; ++k) {
     const int v = col[static_cast<int64_t>(k) * pl.nb];
     col[static_cast<int64_t>(k) * pl.nb] = run;
     run += v;
@@ -712,8 +723,10 @@ struct MergeArgs {
   int64_t q_offset, n_items;
 };
 
+// Latency bound on its partial loads: the register cap keeps at least
+// 16 (G = 8) / 24 / 32 warps per SM resident.
 template <int G>
-__global__ void __launch_bounds__(256) attn_merge_kernel(const MergeArgs a) {
+__global__ void __launch_bounds__(256, (G == 8 ? 2 : (G == 4 ? 3 : 4))) attn_merge_kernel(const MergeArgs a) {
   constexpr int D = 128;
   const int lane = threadIdx.x & 31;
   const int64_t item = static_cast<int64_t>(blockIdx.x) * 8 + (threadIdx.x >> 5);
@@ -745,8 +758,9 @@ __global__ void __launch_bounds__(256) attn_merge_kernel(const MergeArgs a) {
     inv_den[h] = 1.f / den;
     lse2[h] = M + log2f(den);
   }
-  // every lane accumulates dims 4 lane .. 4 lane + 3 of every head, four
-  // slots at a time
+  // every lane accumulates dims 4 lane .. 4 lane + 3 of every head, SU
+  // slots at a time (loads of SU x G rows in flight)
+  constexpr int SU = G == 8 ? 2 : 4;
   float acc[G][4];
 #pragma unroll
   for (int h = 0; h < G; ++h)
@@ -754,21 +768,21 @@ __global__ void __launch_bounds__(256) attn_merge_kernel(const MergeArgs a) {
     for (int u = 0; u < 4; ++u) acc[h][u] = 0.f;
   uint64_t m = s.mask;
   while (m) {
-    int js[4];
+    int js[SU];
 #pragma unroll
-    for (int q = 0; q < 4; ++q) {
+    for (int q = 0; q < SU; ++q) {
       js[q] = m ? __ffsll(static_cast<long long>(m)) - 1 : -1;
       m &= m - 1;
     }
-    uint2 raw[4][G];
+    uint2 raw[SU][G];
 #pragma unroll
-    for (int q = 0; q < 4; ++q)
+    for (int q = 0; q < SU; ++q)
 #pragma unroll
       for (int h = 0; h < G; ++h)
         raw[q][h] = js[q] >= 0 ? __ldg(reinterpret_cast<const uint2*>(po + (js[q] * G + h) * D) + lane)
                                : make_uint2(0u, 0u);
 #pragma unroll
-    for (int q = 0; q < 4; ++q) {
+    for (int q = 0; q < SU; ++q) {
       if (js[q] < 0) break;   // warp-uniform
       const int src = js[q] & 31;
 #pragma unroll

@@ -56,16 +56,12 @@ __device__ __forceinline__ SlotSet row_slots(int v_in, int topk, int64_t pos, in
   s.lo = pos - window + 1 > 0 ? pos - window + 1 : 0;
   s.b0 = s.lo / block;
   const int nwb = static_cast<int>(pos / block - s.b0) + 1;
-  // window block w is uncovered unless some used entry selects it; lane w
-  // checks block b0 + w against every used entry
-  const int64_t wb = s.b0 + lane;
-  bool covered = false;
-  for (uint32_t m = static_cast<uint32_t>(s.mask); m; m &= m - 1) {
-    const int src = __ffs(static_cast<int>(m)) - 1;
-    covered |= __shfl_sync(0xFFFFFFFFu, v, src) == wb;
-  }
-  const uint32_t win = __ballot_sync(0xFFFFFFFFu, lane < nwb && !covered);
-  s.mask |= static_cast<uint64_t>(win) << topk;
+  // window block w is uncovered unless some used entry selects it: each
+  // lane marks the window block its own entry covers, OR over the warp
+  const int64_t w = static_cast<int64_t>(v) - s.b0;
+  const uint32_t cov = __reduce_or_sync(0xFFFFFFFFu, (valid && w >= 0 && w < 32) ? (1u << w) : 0u);
+  const uint32_t all = nwb >= 32 ? 0xFFFFFFFFu : ((1u << nwb) - 1u);
+  s.mask |= static_cast<uint64_t>(all & ~cov) << topk;
   return s;
 }
 
