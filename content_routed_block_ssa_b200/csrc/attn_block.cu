@@ -183,6 +183,112 @@ __global__ void __launch_bounds__(256) inv_tiles_kernel(const BlockPlan pl) {
     pl.tiles[t0 + t] = make_int4(bg, c, e0 + t * pl.qpt, min(pl.qpt, n - t * pl.qpt));
 }
 
+// Work estimate of each tile for the split over CTAs (units of a quarter of
+// an unmasked tile, from per-CTA cycle counts of the block kernel on B200):
+// a tile costs 4, masked_cost when a window slot in it is masked to part of
+// the block (the masked softmax path), plus block_start_cost for the first
+// tile of a block (loading K_c, V_c; with one K/V buffer the pipeline
+// drains).  The per-256-tile sums go to csum.
+__global__ void __launch_bounds__(256) inv_cost_kernel(const BlockPlan pl, int masked_cost, int block_start_cost) {
+  const int t = blockIdx.x * blockDim.x + threadIdx.x;
+  const int T = pl.tile_base[pl.bgs];
+  int cost = 0;
+  if (t < T) {
+    const int4 td = pl.tiles[t];
+    bool masked = false;
+    const int64_t base = static_cast<int64_t>(td.y) * pl.block;
+    for (int e = 0; e < td.w && !masked; ++e) {
+      const int ent = pl.entries[td.z + e];
+      if (entry_slot(ent) >= pl.topk) {
+        const int64_t pos = pl.q_offset + entry_row(ent);
+        masked = (pos - pl.window + 1 > base) || (pos < base + pl.block - 1);
+      }
+    }
+    cost = masked ? masked_cost : 4;
+    if (t == 0) {
+      cost += block_start_cost;
+    } else {
+      const int4 tp = pl.tiles[t - 1];
+      if (tp.x != td.x || tp.y != td.y) cost += block_start_cost;
+    }
+    pl.tcost[t] = static_cast<uint8_t>(cost);
+  }
+  // block sum
+  __shared__ int ws[8];
+  int v = cost;
+#pragma unroll
+  for (int o = 16; o; o >>= 1) v += __shfl_xor_sync(0xFFFFFFFFu, v, o);
+  if ((threadIdx.x & 31) == 0) ws[threadIdx.x >> 5] = v;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    int sum = 0;
+    for (int w = 0; w < 8; ++w) sum += ws[w];
+    pl.csum[blockIdx.x] = sum;
+  }
+}
+
+// One CTA: exclusive scan of the 256-tile sums, then for every split point
+// b * total / grid the first tile whose cost prefix reaches it.
+__global__ void __launch_bounds__(1024) inv_split_kernel(const BlockPlan pl, int n_chunks) {
+  __shared__ int wsum[32];
+  __shared__ int total_s;
+  const int per = (n_chunks + 1023) / 1024;
+  const int c0 = threadIdx.x * per;
+  int local = 0;
+  for (int c = c0; c < min(c0 + per, n_chunks); ++c) local += pl.csum[c];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  int inc = local;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xFFFFFFFFu, inc, o);
+    if (lane >= o) inc += y;
+  }
+  if (lane == 31) wsum[warp] = inc;
+  __syncthreads();
+  if (warp == 0) {
+    int v = wsum[lane];
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xFFFFFFFFu, v, o);
+      if (lane >= o) v += y;
+    }
+    wsum[lane] = v;
+    if (lane == 31) total_s = v;
+  }
+  __syncthreads();
+  int run = (warp ? wsum[warp - 1] : 0) + inc - local;
+  for (int c = c0; c < min(c0 + per, n_chunks); ++c) {
+    const int x = pl.csum[c];
+    pl.csum[c] = run;   // exclusive prefix
+    run += x;
+  }
+  __syncthreads();
+  const int total = total_s;
+  const int T = pl.tile_base[pl.bgs];
+  for (int b = threadIdx.x; b <= pl.grid; b += blockDim.x) {
+    int t;
+    if (b == 0) {
+      t = 0;
+    } else if (b == pl.grid) {
+      t = T;
+    } else {
+      const int target = static_cast<int>((static_cast<int64_t>(total) * b) / pl.grid);
+      // last chunk whose prefix is <= target, then walk its tiles
+      int lo = 0, hi = n_chunks - 1;
+      while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (pl.csum[mid] <= target) lo = mid; else hi = mid - 1;
+      }
+      int acc = pl.csum[lo];
+      t = lo * 256;
+      const int tend = min(T, (lo + 1) * 256);
+      while (t < tend && acc + pl.tcost[t] <= target) acc += pl.tcost[t++];
+      t = min(t, T);
+    }
+    pl.t_start[b] = t;
+  }
+}
+
 // ------------------------------------------------------------------ block tiles
 
 template <int G, int BLK>
@@ -216,7 +322,7 @@ struct BlkCfg {
 struct BlkArgs {
   const __nv_bfloat16* Q;
   const int4* tiles;
-  const int32_t* n_tiles;    // device: total tiles
+  const int32_t* t_start;    // device: [grid + 1] first tile of each CTA
   const int32_t* entries;    // make_entry(query row, slot)
   int32_t n_q, n_kv, h_q, h_kv, topk, window, nsl;
   int64_t q_offset;
@@ -225,11 +331,6 @@ struct BlkArgs {
   float2* partL;             // [items][nsl][G]: (log2-sum-exp, 2^e)
   uint32_t* err;
 };
-
-__device__ __forceinline__ void tile_range(int T, int& t0, int& t1) {
-  t0 = static_cast<int>((static_cast<int64_t>(T) * blockIdx.x) / gridDim.x);
-  t1 = static_cast<int>((static_cast<int64_t>(T) * (blockIdx.x + 1)) / gridDim.x);
-}
 
 __device__ __forceinline__ void fence_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
@@ -325,8 +426,7 @@ __global__ void __maxnreg__((BlkCfg<G, BLK>::MAXREG))
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
 
-  int t0, t1;
-  tile_range(*a.n_tiles, t0, t1);
+  const int t0 = a.t_start[blockIdx.x], t1 = a.t_start[blockIdx.x + 1];
   const int T = t1 - t0;
   const int4 none = make_int4(-1, -1, 0, 0);
 
@@ -463,14 +563,18 @@ __global__ void __maxnreg__((BlkCfg<G, BLK>::MAXREG))
     const uint32_t lane_base = static_cast<uint32_t>(eq * 32) << 16;
     const int sb = grp;                        // this group's S, P and O buffers
     bool ok = true;
-    // this group's tile descriptors one ahead and this thread's entry with it
+    // this group's tile descriptors two of its tiles ahead and this thread's
+    // entry one ahead, so neither load stalls the loop (the descriptor of the
+    // next tile has arrived when its entry is fetched)
     int4 nxt = grp < T ? a.tiles[t0 + grp] : none;
+    int4 nxt2 = grp + 2 < T ? a.tiles[t0 + grp + 2] : none;
     int nxt_ent = e < nxt.w ? __ldg(a.entries + nxt.z + e) : 0;
     for (int lt = grp; lt < T && ok; lt += 2) {
       const int use = lt >> 1;                 // this buffer's use count
       const int4 td = nxt;
       const int ent = nxt_ent;
-      nxt = lt + 2 < T ? a.tiles[t0 + lt + 2] : none;
+      nxt = nxt2;
+      nxt2 = lt + 4 < T ? a.tiles[t0 + lt + 4] : none;
       nxt_ent = e < nxt.w ? __ldg(a.entries + nxt.z + e) : 0;
       const int bg = td.x, ne = td.w;
       const int i = entry_row(ent), j = entry_slot(ent);
@@ -616,6 +720,7 @@ __global__ void __maxnreg__((BlkCfg<G, BLK>::MAXREG))
     const int q = warp - 2;   // tiles q, q + NGW, ... into buffers lt % NA
     bool ok = true;
     int4 nxt = q < T ? a.tiles[t0 + q] : none;
+    int4 nxt2 = q + C::NGW < T ? a.tiles[t0 + q + C::NGW] : none;   // two ahead (TMA path)
     int nen0 = lane < nxt.w ? __ldg(a.entries + nxt.z + lane) : 0;
     int nen1 = (QPT > 32 && lane + 32 < nxt.w) ? __ldg(a.entries + nxt.z + 32 + lane) : 0;
     int last_lt = -1;
@@ -632,24 +737,22 @@ __global__ void __maxnreg__((BlkCfg<G, BLK>::MAXREG))
       uint8_t* abuf = sA + ab * C::A_BYTES;
       if (C::TMA_Q) {
         // an entry's 8 query heads are 8 tensor-core rows = one 1024-byte
-        // swizzle atom per 64-dim half: two TMA boxes per entry
+        // swizzle atom per 64-dim half: lane e issues entry e's two TMA boxes
         if (lane == 0) mbar_arrive_expect_tx(&a_full[ab], static_cast<uint32_t>(ne) * G * D * 2);
-        for (int ee = 0; ee < ne; ++ee) {
-          const int ent = __shfl_sync(0xFFFFFFFFu, en0, ee);
-          const int i = entry_row(ent);
-          if (static_cast<unsigned>(i) >= static_cast<unsigned>(a.n_q)) {   // never for a consistent plan
-            if (lane == 0) atomicCAS(a.err, 0u, static_cast<uint32_t>(SITE_BLK_BAD_ENTRY));
-            ok = false;
-            break;
-          }
-          if (lane == 0) {
+        __syncwarp();
+        if (lane < ne) {
+          const int i = entry_row(en0);
+          if (static_cast<unsigned>(i) < static_cast<unsigned>(a.n_q)) {
             const int z = static_cast<int>(static_cast<int64_t>(b) * a.n_q + i);
 #pragma unroll
             for (int hf = 0; hf < 2; ++hf)
-              tma_load_3d(abuf + hf * C::A_HALF + ee * (G * C::ROW), &tmQ, &a_full[ab], hf * 64, g * G, z);
+              tma_load_3d(abuf + hf * C::A_HALF + lane * (G * C::ROW), &tmQ, &a_full[ab], hf * 64, g * G, z);
+          } else {   // never for a consistent plan; the tile's wait then times out
+            atomicCAS(a.err, 0u, static_cast<uint32_t>(SITE_BLK_BAD_ENTRY));
           }
         }
-        nxt = lt + C::NGW < T ? a.tiles[t0 + lt + C::NGW] : none;
+        nxt = nxt2;
+        nxt2 = lt + 2 * C::NGW < T ? a.tiles[t0 + lt + 2 * C::NGW] : none;
         nen0 = lane < nxt.w ? __ldg(a.entries + nxt.z + lane) : 0;
       } else {
         const uint32_t abase = smem_u32(abuf);
@@ -877,7 +980,15 @@ cudaError_t launch_block_plan(const ssa_params& p, const int32_t* block_idx, con
   note_launch();
   inv_tiles_kernel<<<cols, 256, 0, c.stream>>>(pl);
   note_launch();
-  (void)p;
+  if (pl.grid < 1 || pl.grid > kMaxBlockGrid) return cudaErrorInvalidValue;
+  const int n_chunks = (pl.max_tiles + 255) / 256;
+  // 64-key blocks (two K/V buffers): every tile alike — equal counts were
+  // measured as fast as any weighting; 128-key blocks (one K/V buffer): a
+  // masked tile costs about 1.75 tiles and a new block two
+  inv_cost_kernel<<<n_chunks, 256, 0, c.stream>>>(pl, p.block == 64 ? 4 : 7, p.block == 64 ? 0 : 8);
+  note_launch();
+  inv_split_kernel<<<1, 1024, 0, c.stream>>>(pl, n_chunks);
+  note_launch();
   return cudaGetLastError();
 }
 
@@ -887,7 +998,7 @@ cudaError_t launch_attn_block(const ssa_params& p, const BlockPlan& pl, const vo
   BlkArgs a;
   a.Q = static_cast<const __nv_bfloat16*>(Q);
   a.tiles = pl.tiles;
-  a.n_tiles = pl.tile_base + pl.bgs;
+  a.t_start = pl.t_start;
   a.entries = pl.entries;
   a.n_q = p.n_q; a.n_kv = p.n_kv; a.h_q = p.h_q; a.h_kv = p.h_kv; a.topk = p.topk; a.window = p.window;
   a.nsl = p.topk + window_slots(p.window, p.block);

@@ -64,7 +64,15 @@ struct BlockPlan {
   int32_t *ent_base, *tile_base;         // [bgs + 1]
   int32_t* entries;                      // make_entry(query row, slot)
   int4* tiles;                           // {bg, block, first entry, entries}
+  // balanced split of the tiles over the block kernel's CTAs
+  int32_t max_tiles, grid;               // tile capacity; CTAs (<= kMaxBlockGrid)
+  uint8_t* tcost;                        // [max_tiles] estimated cost of each tile
+  int32_t* csum;                         // [ceil(max_tiles / 256)] cost per 256 tiles, then its scan
+  int32_t* t_start;                      // [grid + 1] first tile of each CTA
 };
+
+// Upper bound on the block kernel's grid (one CTA per SM).
+constexpr int kMaxBlockGrid = 1024;
 
 cudaError_t launch_block_plan(const ssa_params& p, const int32_t* block_idx, const BlockPlan& pl,
                               const LaunchCtx& c);

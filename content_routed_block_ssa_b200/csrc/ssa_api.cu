@@ -157,9 +157,10 @@ bool use_block_attn(const ssa_params& p) {
 }
 
 struct AttnLayout {
-  size_t chist, count, blk_off, tile_off, bg_ents, bg_tiles, ent_base, tile_base, entries, tiles, part_o, part_l,
-      total;
+  size_t chist, count, blk_off, tile_off, bg_ents, bg_tiles, ent_base, tile_base, entries, tiles, tcost, csum,
+      t_start, part_o, part_l, total;
   int nchunk, nsl;
+  size_t max_tiles;
 };
 
 AttnLayout attn_layout(const ssa_params& p) {
@@ -185,6 +186,10 @@ AttnLayout attn_layout(const ssa_params& p) {
   L.tile_base = off; off += round_up((bgs + 1) * 4);
   L.entries = off; off += round_up(sel * 4);
   L.tiles = off; off += round_up(max_tiles * 16);
+  L.max_tiles = max_tiles;
+  L.tcost = off; off += round_up(max_tiles);
+  L.csum = off; off += round_up((max_tiles + 255) / 256 * 4);
+  L.t_start = off; off += round_up((ssa::kMaxBlockGrid + 1) * 4);
   L.part_o = off; off += round_up(sel * G * p.d * 2);
   L.part_l = off; off += round_up(sel * G * 8);
   L.total = off;
@@ -299,6 +304,11 @@ ssa::BlockPlan block_plan(const ssa_params& p, const AttnLayout& L, uint8_t* w) 
   pl.tile_base = reinterpret_cast<int32_t*>(w + L.tile_base);
   pl.entries = reinterpret_cast<int32_t*>(w + L.entries);
   pl.tiles = reinterpret_cast<int4*>(w + L.tiles);
+  pl.max_tiles = static_cast<int32_t>(L.max_tiles);
+  pl.grid = 0;   // set by the caller from the device's SM count
+  pl.tcost = w + L.tcost;
+  pl.csum = reinterpret_cast<int32_t*>(w + L.csum);
+  pl.t_start = reinterpret_cast<int32_t*>(w + L.t_start);
   return pl;
 }
 
@@ -320,12 +330,16 @@ bool encode_attn_maps(AttnMaps& m, const ssa_params& p, const void* Q, const voi
 // that `w` holds attn_layout(p).total bytes.
 ssa_status attn_stage_plan(const ssa_params& p, const int32_t* idx, uint8_t* w, const LaunchCtx& c) {
   const AttnLayout L = attn_layout(p);
-  return from_cuda(ssa::launch_block_plan(p, idx, block_plan(p, L, w), c));
+  ssa::BlockPlan pl = block_plan(p, L, w);
+  pl.grid = c.sm_count;
+  return from_cuda(ssa::launch_block_plan(p, idx, pl, c));
 }
 
 ssa_status attn_stage_blocks(const ssa_params& p, const void* Q, const AttnMaps& m, uint8_t* w, const LaunchCtx& c) {
   const AttnLayout L = attn_layout(p);
-  return from_cuda(ssa::launch_attn_block(p, block_plan(p, L, w), Q, m.K, m.V, m.Qh, w + L.part_o, w + L.part_l, c));
+  ssa::BlockPlan pl = block_plan(p, L, w);
+  pl.grid = c.sm_count;
+  return from_cuda(ssa::launch_attn_block(p, pl, Q, m.K, m.V, m.Qh, w + L.part_o, w + L.part_l, c));
 }
 
 ssa_status attn_stage_merge(const ssa_params& p, const int32_t* idx, void* O, float* lse, int32_t* bad,
