@@ -70,16 +70,23 @@ def load_traffic():
 
 # ------------------------------------------------------------------ distributed
 
-def dist_setup(n_gpus):
+def dist_setup(n_gpus, backend=None):
+    """One process per GPU (torchrun sets RANK / LOCAL_RANK / WORLD_SIZE).
+    The layer has no exchange step: ranks run independent replicas and only
+    meet for the barriers and the max-over-ranks of the timings (NCCL on the
+    GPUs; gloo when there is no GPU, which the CPU tests use)."""
     ws = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
     if ws > 1:
         import datetime
         import torch.distributed as dist
-        torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=600),
-                                device_id=torch.device("cuda", local))
+        backend = backend or ("nccl" if torch.cuda.is_available() else "gloo")
+        kw = {}
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+            kw["device_id"] = torch.device("cuda", local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120), **kw)
     elif torch.cuda.is_available():
         torch.cuda.set_device(0)
     return ws, rank, local
@@ -95,9 +102,16 @@ def max_over_ranks(x, ws):
     if ws == 1:
         return x
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def whole_job_rate(units_per_rank, ws, ms_max):
+    """Units all ranks processed per second over the slowest rank's time
+    (weak scaling: every rank runs the full workload)."""
+    return ws * units_per_rank / (ms_max / 1e3)
 
 
 # ------------------------------------------------------------------ clocks
@@ -317,7 +331,7 @@ def run_ours(w, steps, warmup, ws, rank, with_e2e=True):
         ms_e2e = max_over_ranks(e0.elapsed_time(e1) / n_e2e, ws)
         h2d = hQ.numel() * hQ.element_size() + 2 * hK.numel() * hK.element_size()
         d2h = hO.numel() * hO.element_size() + hl.numel() * hl.element_size()
-        e2e = {"value": ws * w.batch * w.n_q * w.h_q / (ms_e2e / 1e3), "unit": UNIT,
+        e2e = {"value": whole_job_rate(w.batch * w.n_q * w.h_q, ws, ms_e2e), "unit": UNIT,
                "ms_per_step": ms_e2e, "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
                "steps": n_e2e}
         del buf
@@ -471,7 +485,7 @@ def main():
     traffic = load_traffic()
     res = run_ours(w, a.steps, a.warmup, ws, rank, with_e2e=not a.no_e2e)
     kern = kernel_report(w, res, peaks, traffic)
-    value = ws * w.batch * w.n_q * w.h_q / (res["ms_step"] / 1e3)
+    value = whole_job_rate(w.batch * w.n_q * w.h_q, ws, res["ms_step"])
     dname, dk = dominant(kern)
     roof = {"bound": dk["bound"], "achieved": dk["achieved"], "peak": dk["peak"], "unit": dk["unit"],
             "frac": dk["frac"], "traffic": dk["traffic"], "kernel": dk["kernel"], "stage": dname,
@@ -484,7 +498,7 @@ def main():
         w2 = WORKLOADS[SECONDARY]
         r2 = run_ours(w2, max(3, a.steps // 2), a.warmup, ws, rank, with_e2e=False)
         k2 = kernel_report(w2, r2, peaks, traffic)
-        secondary = {"workload": w2.name, "value": ws * w2.batch * w2.n_q * w2.h_q / (r2["ms_step"] / 1e3),
+        secondary = {"workload": w2.name, "value": whole_job_rate(w2.batch * w2.n_q * w2.h_q, ws, r2["ms_step"]),
                      "unit": UNIT, "ms_per_step": r2["ms_step"], "kernels": k2, "gpu_launches": r2["launches"],
                      "clocks": r2["clocks"]}
     cpu = None

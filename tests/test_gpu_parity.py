@@ -30,6 +30,14 @@ CASES = {
     "bf16_gqa4_d128_b64_k32_b2": Workload("c", 109, 2, 2560, 8, 2, 128, "bf16", 64, "diag", 32, 256, 8, "total",
                                           clustered=True),
     "bf16_gqa2_d128_b64_w100": Workload("c", 113, 1, 2304, 4, 2, 128, "bf16", 64, "diag", 16, 100, 6, "per_head"),
+    # block-major variants: cp.async Q rows with 128-key blocks (G = 4, 2; a
+    # window of 300 keys, not block aligned) and TMA Q boxes with 64-key
+    # blocks (G = 8)
+    "bf16_gqa4_d128_b128_k16": Workload("c", 114, 1, 2560, 8, 2, 128, "bf16", 128, "diag", 16, 256, 6, "total"),
+    "bf16_gqa2_d128_b128_w300_b2": Workload("c", 116, 2, 1536, 4, 2, 128, "bf16", 128, "diag", 8, 300, 4,
+                                            "per_head"),
+    "bf16_gqa8_d128_b64_k16": Workload("c", 115, 1, 2048, 16, 2, 128, "bf16", 64, "diag", 16, 192, 6, "total",
+                                       clustered=True),
     "bf16_gqa2_d64_b64": Workload("c", 104, 1, 1024, 4, 2, 64, "bf16", 64, "diag", 4, 64, 6, "total"),
     "bf16_mha_d64_b128_w200": Workload("c", 105, 1, 1280, 1, 1, 64, "bf16", 128, "diag", 8, 200, 4, "total"),
     "f32_full_d64": Workload("c", 106, 1, 1024, 1, 1, 64, "f32", 64, "full", 8, 64, 8, "total"),
