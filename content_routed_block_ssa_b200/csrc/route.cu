@@ -85,23 +85,30 @@ struct RouteTiledArgs {
 
 template <int KF>
 struct TiledCfg {
+  static constexpr int RT = 2;                            // 128-row feature tiles per unit
   static constexpr int A_BOXES = KF / 64;                 // 64-wide K slices
   static constexpr int BOX_BYTES = 128 * 128;             // 128 rows x 64 bf16
-  static constexpr int A_BYTES = A_BOXES * BOX_BYTES;     // one 128-row feature tile
-  static constexpr int NS = (KF == 256) ? 4 : 6;          // table-slice ring
-  static constexpr int CAP = 32;                          // candidates per row
-  static constexpr int NACC = 4;                          // TMEM accumulators (128 cols)
-  static constexpr int NBAR = 4 + 2 * NS + 2 * NACC + 1;
-  static constexpr int SMEM = 1024 + 2 * A_BYTES + NS * BOX_BYTES + CAP * 128 * 8 + NBAR * 8 + 16;
+  static constexpr int A_TILE = A_BOXES * BOX_BYTES;      // one 128-row feature tile
+  static constexpr int A_BYTES = RT * A_TILE;             // a unit's feature rows
+  static constexpr int NAB = (KF == 256) ? 1 : 2;         // unit buffers
+  static constexpr int NS = 4;                            // table-slice ring
+  static constexpr int CAP = 16;                          // candidates per row (per epilogue group)
+  static constexpr int NACC = 4;                          // TMEM accumulators: 2 chunks x RT tiles
+  static constexpr int NBAR = 2 * NAB + 2 * NS + 2 * NACC + 1;
+  static constexpr int SMEM = 1024 + NAB * A_BYTES + NS * BOX_BYTES + RT * CAP * 128 * 8 + NBAR * 8 + 16;
+  static constexpr int THREADS = 64 + RT * 128;           // TMA, MMA, RT epilogue groups
+  static_assert(SMEM <= 232448, "shared memory");
 };
 
+// A unit is 256 query rows (two 128-row tensor-core tiles) of one (batch,
+// kv-head): every table slice is loaded once for both tiles.
 __device__ __forceinline__ void route_unit(const RouteTiledArgs& a, int r, int& bg, int& row0,
                                            int& nch) {
   const int BG = a.batch * a.h_kv;
   bg = r % BG;
-  const int tile = a.n_tiles - 1 - r / BG;   // heaviest tiles first
-  row0 = tile * 128;
-  const int rows = min(128, a.n_q - row0);
+  const int unit = a.n_tiles - 1 - r / BG;   // heaviest units first
+  row0 = unit * 256;
+  const int rows = min(256, a.n_q - row0);
   const int64_t pos = a.q_offset + row0 + rows - 1;
   const int nv = static_cast<int>(min(static_cast<int64_t>(a.nb), (pos + 1) / a.block));
   nch = (nv + 127) / 128;
@@ -190,22 +197,23 @@ __device__ __forceinline__ void filter16(const uint32_t (&v)[16], int c0, int nv
   }
 }
 
-// Warp roles: 0 = TMA producer, 1 = MMA issuer (and TMEM owner),
-// 2..5 = epilogue (TMEM lane quadrant = warp % 4, one query row per thread).
+// Warp roles: 0 = TMA producer, 1 = MMA issuer (and TMEM owner), 2..5 and
+// 6..9 = two epilogue groups, group g owning the unit's tile g (TMEM lane
+// quadrant = warp % 4, one query row per thread).
 template <int KF, int KSEL>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(TiledCfg<KF>::THREADS, 1)
     route_tiled_kernel(const __grid_constant__ CUtensorMap tmF, const __grid_constant__ CUtensorMap tmT,
                        const RouteTiledArgs a) {
   using C = TiledCfg<KF>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sA = smem;
-  uint8_t* sB = sA + 2 * C::A_BYTES;
+  uint8_t* sB = sA + C::NAB * C::A_BYTES;
   uint2* cand = reinterpret_cast<uint2*>(sB + C::NS * C::BOX_BYTES);
-  uint64_t* bars = reinterpret_cast<uint64_t*>(cand + C::CAP * 128);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(cand + C::RT * C::CAP * 128);
   uint64_t* a_full = bars;
-  uint64_t* a_empty = bars + 2;
-  uint64_t* b_full = bars + 4;
+  uint64_t* a_empty = a_full + C::NAB;
+  uint64_t* b_full = a_empty + C::NAB;
   uint64_t* b_empty = b_full + C::NS;
   uint64_t* acc_full = b_empty + C::NS;
   uint64_t* acc_empty = acc_full + C::NACC;
@@ -214,7 +222,7 @@ __global__ void __launch_bounds__(192, 1)
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   if (threadIdx.x == 0) {
-    for (int i = 0; i < 2; ++i) { mbar_init(&a_full[i], 1); mbar_init(&a_empty[i], 1); }
+    for (int i = 0; i < C::NAB; ++i) { mbar_init(&a_full[i], 1); mbar_init(&a_empty[i], 1); }
     for (int i = 0; i < C::NS; ++i) { mbar_init(&b_full[i], 1); mbar_init(&b_empty[i], 1); }
     for (int i = 0; i < C::NACC; ++i) { mbar_init(&acc_full[i], 1); mbar_init(&acc_empty[i], 4); }
     mbar_init(mma_done, 1);
@@ -241,13 +249,16 @@ __global__ void __launch_bounds__(192, 1)
         int bg, row0, nch;
         route_unit(a, r, bg, row0, nch);
         if (nch == 0) continue;
-        const int ab = a_cnt & 1;
-        if (!mbar_wait(&a_empty[ab], ((a_cnt >> 1) & 1) ^ 1, a.err, SITE_ROUTE_PRODUCER)) { ok = false; break; }
+        const int ab = a_cnt % C::NAB;
+        if (!mbar_wait(&a_empty[ab], ((a_cnt / C::NAB) & 1) ^ 1, a.err, SITE_ROUTE_PRODUCER)) { ok = false; break; }
         mbar_arrive_expect_tx(&a_full[ab], C::A_BYTES);
-        const int frow = bg * a.n_q + row0;
+        const int frow = bg * a.n_q + row0;   // rows past this (batch, kv-head) are never used
 #pragma unroll
-        for (int ks = 0; ks < C::A_BOXES; ++ks)
-          tma_load_2d(sA + ab * C::A_BYTES + ks * C::BOX_BYTES, &tmF, &a_full[ab], ks * 64, frow);
+        for (int rt = 0; rt < C::RT; ++rt)
+#pragma unroll
+          for (int ks = 0; ks < C::A_BOXES; ++ks)
+            tma_load_2d(sA + ab * C::A_BYTES + rt * C::A_TILE + ks * C::BOX_BYTES, &tmF, &a_full[ab], ks * 64,
+                        frow + rt * 128);
         ++a_cnt;
         const int trow = bg * a.nb;
         for (int j = 0; j < nch && ok; ++j) {
@@ -264,14 +275,14 @@ __global__ void __launch_bounds__(192, 1)
       if (!ok) {   // make sure no copy is still landing in shared memory
         for (uint32_t n = (b_cnt > C::NS ? b_cnt - C::NS : 0); n < b_cnt; ++n)
           drain_wait(&b_full[n % C::NS], (n / C::NS) & 1, a.err);
-        for (uint32_t n = (a_cnt > 2 ? a_cnt - 2 : 0); n < a_cnt; ++n)
-          drain_wait(&a_full[n & 1], (n >> 1) & 1, a.err);
+        for (uint32_t n = (a_cnt > C::NAB ? a_cnt - C::NAB : 0); n < a_cnt; ++n)
+          drain_wait(&a_full[n % C::NAB], (n / C::NAB) & 1, a.err);
       }
     }
   } else if (warp == 1) {
     if (lane == 0) {
       constexpr uint32_t IDESC = umma_idesc_bf16(128, 128);
-      uint32_t a_cnt = 0, b_cnt = 0, acc_cnt = 0;
+      uint32_t a_cnt = 0, b_cnt = 0, ch_cnt = 0;
       bool ok = true;
       const uint32_t sA_u = smem_u32(sA), sB_u = smem_u32(sB);
       for (int q = 0; ok; ++q) {
@@ -280,31 +291,38 @@ __global__ void __launch_bounds__(192, 1)
         int bg, row0, nch;
         route_unit(a, r, bg, row0, nch);
         if (nch == 0) continue;
-        const int ab = a_cnt & 1;
-        if (!mbar_wait(&a_full[ab], (a_cnt >> 1) & 1, a.err, SITE_ROUTE_MMA)) { ok = false; break; }
+        const int ab = a_cnt % C::NAB;
+        if (!mbar_wait(&a_full[ab], (a_cnt / C::NAB) & 1, a.err, SITE_ROUTE_MMA)) { ok = false; break; }
         tc_fence_after();
         for (int j = 0; j < nch && ok; ++j) {
-          const int acc = acc_cnt % C::NACC;
-          if (!mbar_wait(&acc_empty[acc], ((acc_cnt / C::NACC) & 1) ^ 1, a.err, SITE_ROUTE_MMA)) { ok = false; break; }
+          // chunk slot: accumulators 2 slot + rt, one per tile
+          const int slot = ch_cnt & 1;
+          const uint32_t par = ((ch_cnt >> 1) & 1) ^ 1;
+          if (!mbar_wait(&acc_empty[2 * slot], par, a.err, SITE_ROUTE_MMA) ||
+              !mbar_wait(&acc_empty[2 * slot + 1], par, a.err, SITE_ROUTE_MMA)) { ok = false; break; }
           tc_fence_after();
-          const uint32_t d_tmem = tmem_base + acc * 128;
 #pragma unroll
           for (int ks = 0; ks < C::A_BOXES; ++ks) {
             const int s = b_cnt % C::NS;
             if (!mbar_wait(&b_full[s], (b_cnt / C::NS) & 1, a.err, SITE_ROUTE_MMA)) { ok = false; break; }
             tc_fence_after();
+            const uint32_t bslice = sB_u + s * C::BOX_BYTES;
 #pragma unroll
-            for (int kk = 0; kk < 4; ++kk) {
-              const uint64_t ad = umma_desc_sw128(sA_u + ab * C::A_BYTES + ks * C::BOX_BYTES + kk * 32);
-              const uint64_t bd = umma_desc_sw128(sB_u + s * C::BOX_BYTES + kk * 32);
-              umma_bf16(d_tmem, ad, bd, IDESC, (ks | kk) != 0 ? 1u : 0u);
+            for (int rt = 0; rt < C::RT; ++rt) {
+              const uint32_t d_tmem = tmem_base + (2 * slot + rt) * 128;
+              const uint32_t atile = sA_u + ab * C::A_BYTES + rt * C::A_TILE + ks * C::BOX_BYTES;
+#pragma unroll
+              for (int kk = 0; kk < 4; ++kk)
+                umma_bf16(d_tmem, umma_desc_sw128(atile + kk * 32), umma_desc_sw128(bslice + kk * 32), IDESC,
+                          (ks | kk) != 0 ? 1u : 0u);
             }
             umma_commit(&b_empty[s]);
             ++b_cnt;
           }
           if (!ok) break;
-          umma_commit(&acc_full[acc]);
-          ++acc_cnt;
+          umma_commit(&acc_full[2 * slot]);
+          umma_commit(&acc_full[2 * slot + 1]);
+          ++ch_cnt;
         }
         if (!ok) break;
         umma_commit(&a_empty[ab]);
@@ -314,17 +332,18 @@ __global__ void __launch_bounds__(192, 1)
       drain_wait(mma_done, 0, a.err);
     }
   } else {
+    const int grp = (warp - 2) >> 2;   // the unit's tile this group owns
     const int eq = warp & 3;
     const int row = eq * 32 + lane;
-    uint2* my_cand = cand + row;
-    uint32_t acc_cnt = 0;
+    uint2* my_cand = cand + grp * (C::CAP * 128) + row;
+    uint32_t ch_cnt = 0;
     bool ok = true;
     for (int q = 0; ok; ++q) {
       const int r = route_unit_rank(q);
       if (r >= a.n_units) break;
       int bg, row0, nch;
       route_unit(a, r, bg, row0, nch);
-      const int i = row0 + row;
+      const int i = row0 + grp * 128 + row;
       const bool valid = i < a.n_q;
       const int nvis = valid ? static_cast<int>(min(static_cast<int64_t>(a.nb), (a.q_offset + i + 1) / a.block)) : 0;
       float Ls[KSEL];
@@ -334,8 +353,8 @@ __global__ void __launch_bounds__(192, 1)
       float thr = -INFINITY;
       int cnt = 0;
       for (int j = 0; j < nch; ++j) {
-        const int acc = acc_cnt % C::NACC;
-        ok = __all_sync(0xFFFFFFFFu, mbar_wait(&acc_full[acc], (acc_cnt / C::NACC) & 1, a.err, SITE_ROUTE_EPILOGUE));
+        const int acc = 2 * (ch_cnt & 1) + grp;
+        ok = __all_sync(0xFFFFFFFFu, mbar_wait(&acc_full[acc], (ch_cnt >> 1) & 1, a.err, SITE_ROUTE_EPILOGUE));
         if (!ok) break;
         tc_fence_after();
         const uint32_t taddr = tmem_base + (static_cast<uint32_t>(eq * 32) << 16) + acc * 128;
@@ -356,7 +375,7 @@ __global__ void __launch_bounds__(192, 1)
             filter16<true>(v, c0, nvis, thr, cnt, my_cand);
           if (__any_sync(0xFFFFFFFFu, cnt > C::CAP - 16)) merge_candidates<KSEL>(Ls, Li, cnt, thr, my_cand, a.topk);
         }
-        ++acc_cnt;
+        ++ch_cnt;
       }
       if (!ok) break;
       if (__any_sync(0xFFFFFFFFu, cnt > 0)) merge_candidates<KSEL>(Ls, Li, cnt, thr, my_cand, a.topk);
@@ -399,7 +418,7 @@ cudaError_t run_tiled(const ssa_params& p, const CUtensorMap& tmF, const CUtenso
   RouteTiledArgs a;
   a.batch = p.batch; a.n_q = p.n_q; a.h_kv = p.h_kv; a.nb = p.n_kv / p.block;
   a.block = p.block; a.topk = p.topk;
-  a.n_tiles = (p.n_q + 127) / 128;
+  a.n_tiles = (p.n_q + 255) / 256;   // 256-row units per (batch, kv-head)
   a.n_units = p.batch * p.h_kv * a.n_tiles;
   a.q_offset = p.q_offset;
   a.block_idx = idx; a.top_scores = scores; a.err = c.err;
@@ -407,7 +426,7 @@ cudaError_t run_tiled(const ssa_params& p, const CUtensorMap& tmF, const CUtenso
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
   if (e != cudaSuccess) return e;
   const int grid = a.n_units < c.sm_count ? a.n_units : c.sm_count;
-  route_tiled_kernel<KF, KSEL><<<grid, 192, C::SMEM, c.stream>>>(tmF, tmT, a);
+  route_tiled_kernel<KF, KSEL><<<grid, C::THREADS, C::SMEM, c.stream>>>(tmF, tmT, a);
   note_launch();
   return cudaGetLastError();
 }
