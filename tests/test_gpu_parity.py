@@ -392,3 +392,29 @@ def test_block_major_stages_equal_single_call():
     ssa.ssa_attn_merge(p, idx, O2, l2, b2, ws)
     check_no_device_error()
     assert torch.equal(O1, O2) and torch.equal(l1, l2) and int(b2.item()) == int(b1.item()) == 0
+
+
+def test_block_major_one_key_window_and_single_block():
+    """W = 1 and k = 1 on the block-major path: every row's window slot is
+    masked down to its own key, rows before the first full block attend to
+    themselves alone, and the rest add one selected block."""
+    w = Workload("c", 117, 1, 1536, 8, 2, 128, "bf16", 64, "diag", 1, 1, 4, "total", clustered=True)
+    Q, K, V, _ = make_inputs(w, "cpu")
+    pd = problem_dict(w)
+    op = O.Problem(**pd)
+    ref = O.forward(Q.float().numpy(), K.float().numpy(), V.float().numpy(), op)
+    p = params(pd)
+    assert ssa.ssa_attn_workspace_size(p) > 0
+    Qd, Kd, Vd = to_dev(Q, K, V)
+    idx = torch.from_numpy(ref["block_idx"].astype(np.int32)).cuda()
+    O_, lse, bad = gpu_attn(p, Qd, Kd, Vd, idx)
+    check_no_device_error()
+    assert int(bad.item()) == 0
+    max_abs, rel, ok = compare_out(as_np(O_), ref["O"], "bf16")
+    assert ok, (max_abs, rel)
+    np.testing.assert_allclose(lse.cpu().numpy(), ref["lse"], rtol=0, atol=2e-3)
+    got = as_np(O_)
+    Vn = V.float().numpy()
+    for i in range(63):                          # no full block yet: o = v_i for every head
+        for h in range(w.h_q):
+            np.testing.assert_allclose(got[0, i, h], Vn[0, i, h // (w.h_q // w.h_kv)], atol=1e-2)
