@@ -172,14 +172,18 @@ __global__ void __launch_bounds__(kPlanThreads) inv_scatter_kernel(const BlockPl
   }
 }
 
+// A warp per (batch, kv-head, block): its tiles written lane-strided (a
+// block chosen by nearly every query has tens of thousands of tiles).
 __global__ void __launch_bounds__(256) inv_tiles_kernel(const BlockPlan pl) {
-  const int64_t x = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
-  if (x >= static_cast<int64_t>(pl.bgs) * pl.nb) return;
+  const int64_t x = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  if (x >= static_cast<int64_t>(pl.bgs) * pl.nb) return;   // warp-uniform
+  const int lane = threadIdx.x & 31;
   const int bg = static_cast<int>(x / pl.nb), c = static_cast<int>(x % pl.nb);
   const int n = pl.count[x];
   const int e0 = pl.ent_base[bg] + pl.blk_off[x];
   const int t0 = pl.tile_base[bg] + pl.tile_off[x];
-  for (int t = 0; t * pl.qpt < n; ++t)
+  const int nt = (n + pl.qpt - 1) / pl.qpt;
+  for (int t = lane; t < nt; t += 32)
     pl.tiles[t0 + t] = make_int4(bg, c, e0 + t * pl.qpt, min(pl.qpt, n - t * pl.qpt));
 }
 
@@ -978,7 +982,8 @@ cudaError_t launch_block_plan(const ssa_params& p, const int32_t* block_idx, con
   note_launch();
   inv_scatter_kernel<<<rows, kPlanThreads, hist_smem, c.stream>>>(pl, block_idx);
   note_launch();
-  inv_tiles_kernel<<<cols, 256, 0, c.stream>>>(pl);
+  inv_tiles_kernel<<<static_cast<unsigned>((static_cast<int64_t>(pl.bgs) * pl.nb * 32 + 255) / 256), 256, 0,
+                     c.stream>>>(pl);
   note_launch();
   if (pl.grid < 1 || pl.grid > kMaxBlockGrid) return cudaErrorInvalidValue;
   const int n_chunks = (pl.max_tiles + 255) / 256;
