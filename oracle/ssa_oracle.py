@@ -76,6 +76,7 @@ class Problem:
     scale: float = field(default=float("nan"))
     dtype: str = BF16
     sigma: str = DIAG
+    subblocks: int = 1          # sub-block summaries per block (max-pooled routing)
 
     def __post_init__(self):
         if not math.isfinite(self.scale):
@@ -88,6 +89,11 @@ class Problem:
     @property
     def nb(self) -> int:
         return self.n_kv // self.block
+
+    @property
+    def unit(self) -> int:
+        """Keys per summary: the block, or its sub-block when subblocks > 1."""
+        return self.block // self.subblocks
 
 
 # ---------------------------------------------------------------- rounding
@@ -123,9 +129,11 @@ def block_summaries(K: np.ndarray, p: Problem):
       mu  [batch, h_kv, nb, d]       mu_c = (1/B) sum_{j in c} k_j
       sig [batch, h_kv, nb, d]       diagonal: (1/B) sum_j (k_j - mu_c)_t^2
       sig [batch, h_kv, nb, d, d]    full:     (1/B) sum_j (k_j - mu_c)(k_j - mu_c)^T
+    With p.subblocks = S > 1 the summaries are taken per sub-block of B/S
+    consecutive keys instead (nb * S rows, sub-block s of block c at c*S + s).
     """
     b, n, h, d = K.shape
-    B = p.block
+    B = p.unit
     nb = n // B
     Kb = np.asarray(K, dtype=np.float64).reshape(b, nb, B, h, d).transpose(0, 3, 1, 2, 4)
     mu = Kb.sum(axis=3) / B
@@ -188,27 +196,40 @@ def visible_blocks(pos: int, p: Problem) -> int:
 
 # ---------------------------------------------------------------- step 2 (scores)
 
+def pool_subblocks(scores: np.ndarray, p: Problem) -> np.ndarray:
+    """Block scores from sub-block scores (last axis nb * S): the maximum
+    over each block's S sub-blocks (identity for S = 1)."""
+    S = p.subblocks
+    if S == 1:
+        return scores
+    sh = scores.shape
+    return scores.reshape(sh[:-1] + (sh[-1] // S, S)).max(axis=-1)
+
+
 def route_scores_row(Q: np.ndarray, stored, p: Problem, bi: int, i: int, g: int) -> np.ndarray:
     """Routing scores of query row i (batch bi, kv-head g) for all visible blocks.
 
     bf16: s_c = f . [mu_c ; sigma_c^2] with the bf16 features and table.
     fp32: s_c = sum_h ( <q_h, mu_c> + (beta/2) q_h^T Sigma_c q_h ) with the
           float32 summaries (diagonal Sigma: q_h^T diag(sigma^2) q_h).
+    With sub-block summaries each score is taken per sub-block and a block
+    scores the largest of its sub-blocks' (group-summed) scores.
     """
     mu32, sig32, table = stored
     nv = visible_blocks(p.q_offset + i, p)
+    nu = nv * p.subblocks                      # visible summary rows
     if p.dtype == BF16:
         f = route_features(Q[bi:bi + 1, i:i + 1], p)[0, g, 0]
-        return table[bi, g, :nv] @ f
+        return pool_subblocks(table[bi, g, :nu] @ f, p)
     G = p.group
     q = np.asarray(Q[bi, i, g * G:(g + 1) * G], dtype=np.float64)  # [G, d]
-    mu = mu32[bi, g, :nv]                                           # [nv, d]
+    mu = mu32[bi, g, :nu]                                           # [nu, d]
     s = (q @ mu.T).sum(axis=0)
     if p.sigma == FULL:
-        quad = np.einsum("hs,cst,ht->c", q, sig32[bi, g, :nv], q)
+        quad = np.einsum("hs,cst,ht->c", q, sig32[bi, g, :nu], q)
     else:
-        quad = ((q * q) @ sig32[bi, g, :nv].T).sum(axis=0)
-    return s + (p.beta / 2.0) * quad
+        quad = ((q * q) @ sig32[bi, g, :nu].T).sum(axis=0)
+    return pool_subblocks(s + (p.beta / 2.0) * quad, p)
 
 
 def route_scores(Q: np.ndarray, stored, p: Problem, bi: int, g: int) -> np.ndarray:
@@ -226,10 +247,30 @@ def route_scores(Q: np.ndarray, stored, p: Problem, bi: int, g: int) -> np.ndarr
             full = full + (p.beta / 2.0) * np.einsum("ihs,cst,iht->ic", q, sig32[bi, g], q)
         else:
             full = full + (p.beta / 2.0) * np.einsum("ihd,cd->ic", q * q, sig32[bi, g])
+    full = pool_subblocks(full, p)
     for i in range(p.n_q):
         nv = visible_blocks(p.q_offset + i, p)
         out[i, :nv] = full[i, :nv]
     return out
+
+
+def tempered_block_score(q: np.ndarray, Kc: np.ndarray, beta: float) -> float:
+    """The tempered block score  T_beta = (1/beta) log( (1/B) sum_j exp(beta <q, k_j>) )
+    over the B keys of one block (beta = 0: the mean logit).
+
+    The routing score's family ["Subquadratic Sparse Attention (SSA)",
+    artifact list: the temperature family interpolating centroid <->
+    cumulant <-> exact-max]: T_beta is the block's log-mean-exp of the scaled
+    logits; beta -> 0 gives the centroid score <q, mu_c>, its second-order
+    expansion in beta is the cumulant score <q, mu_c> + (beta/2) q^T Sigma_c q,
+    and beta -> infinity gives max_j <q, k_j>.  Needs every key of the block,
+    so it is an analysis reference, not a summary-only router.
+    """
+    s = np.asarray(Kc, dtype=np.float64) @ np.asarray(q, dtype=np.float64)
+    if beta == 0.0:
+        return float(s.mean())
+    m = s.max()
+    return float(m + np.log(np.mean(np.exp(beta * (s - m)))) / beta)
 
 
 # ---------------------------------------------------------------- step 3

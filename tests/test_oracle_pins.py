@@ -417,3 +417,91 @@ def test_cumulant_routing_recovers_needles_centroid_misses():
         hits[beta] = h / len(plan)
     assert hits[2.0] >= 0.95
     assert hits[2.0] > hits[0.0] + 0.3
+
+
+# ---------------------------------------------------------------- sub-block routing, tempered family
+
+def test_subblock_summaries_are_summaries_of_the_smaller_blocks():
+    rng = np.random.default_rng(21)
+    K = O.round_bf16(rng.standard_normal((2, 256, 2, 16)))
+    for S in (2, 4):
+        p = O.Problem(2, 256, 256, 4, 2, 16, 64, 4, 64, subblocks=S, dtype="f32", sigma="full")
+        q = O.Problem(2, 256, 256, 4, 2, 16, 64 // S, 4, 64, dtype="f32", sigma="full")
+        mu_a, sig_a = O.block_summaries(K, p)
+        mu_b, sig_b = O.block_summaries(K, q)
+        assert mu_a.shape == (2, 2, 4 * S, 16)
+        np.testing.assert_array_equal(mu_a, mu_b)
+        np.testing.assert_array_equal(sig_a, sig_b)
+
+
+def _direct_block_score(Qh, Kc, beta):
+    """Sum over query heads of mean + (beta/2) population variance of the
+    logits q_h . k_j over the keys Kc, from the keys themselves."""
+    tot = 0.0
+    for q in Qh:
+        s = Kc @ q
+        tot += s.mean() + 0.5 * beta * s.var()
+    return tot
+
+
+@pytest.mark.parametrize("sigma", ["full", "diag"])
+def test_pooled_score_is_the_best_subblock_score_from_the_keys(sigma):
+    rng = np.random.default_rng(22)
+    B, S, d, G = 64, 4, 8, 2
+    K = O.round_f32(rng.standard_normal((1, 4 * B, 1, d)))
+    Q = O.round_f32(rng.standard_normal((1, 4 * B, G, d)))
+    p = O.Problem(1, 4 * B, 4 * B, G, 1, d, B, 2, 16, subblocks=S, dtype="f32", sigma=sigma, beta=1.5)
+    st = O.stored_summaries(*O.block_summaries(K, p), p)
+    i = 4 * B - 1
+    got = O.route_scores_row(Q, st, p, 0, i, 0)
+    assert got.shape == (4,)
+    Kn = K[0, :, 0]
+    for c in range(4):
+        want = max(_direct_block_score(Q[0, i], Kn[c * B + s * (B // S): c * B + (s + 1) * (B // S)], 1.5)
+                   for s in range(S))
+        if sigma == "diag":   # the diagonal form drops the cross-covariances: compare per-dimension
+            want = max(sum(Q[0, i, h] @ Kn[c * B + s * 16: c * B + (s + 1) * 16].mean(0)
+                           + 0.75 * (Q[0, i, h] ** 2) @ Kn[c * B + s * 16: c * B + (s + 1) * 16].var(0)
+                           for h in range(G)) for s in range(S))
+        assert abs(got[c] - want) <= 1e-5 * max(1.0, abs(want))
+
+
+def test_subblock_pooling_rescues_a_spike_that_the_block_variance_dilutes():
+    """A block whose only signal is one spike key loses to a block of
+    uniformly spread keys under whole-block summaries, and wins once each
+    block is summarised in four sub-blocks (the spike is then 1 key of 16,
+    not 1 of 64)."""
+    B, d = 64, 16
+    K = np.zeros((1, 8 * B, 1, d))
+    K[0, 3 * B:4 * B, 0, 0] = np.where(np.arange(B) % 2 == 0, 1.0, -1.0) * math.sqrt(2.0) / 4.0   # block 3
+    K[0, 5 * B + 37, 0, 0] = 2.0                                                                   # block 5
+    Q = np.zeros((1, 8 * B, 1, d))
+    Q[0, :, 0, 0] = 4.0
+    res = {}
+    for S in (1, 4):
+        p = O.Problem(1, 8 * B, 8 * B, 1, 1, d, B, 1, 1, subblocks=S, dtype="f32", sigma="diag", beta=2.0)
+        st = O.stored_summaries(*O.block_summaries(K, p), p)
+        s = O.route_scores_row(Q, st, p, 0, 8 * B - 1, 0)
+        res[S] = O.select_topk(s, 1)[0][0]
+    assert res[1] == 3 and res[4] == 5
+
+
+def test_tempered_score_limits_and_cumulant_expansion():
+    rng = np.random.default_rng(23)
+    Kc = rng.standard_normal((64, 8))
+    q = rng.standard_normal(8)
+    s = Kc @ q
+    mean, var = s.mean(), s.var()
+    k3 = np.mean((s - mean) ** 3)
+    assert O.tempered_block_score(q, Kc, 0.0) == pytest.approx(mean, rel=1e-12)
+    assert O.tempered_block_score(q, Kc, 1e-6) == pytest.approx(mean, abs=1e-5)
+    # T_beta = mean + (beta/2) var + (beta^2/6) k3 + O(beta^3): the cumulant score is the second-order term
+    for beta in (1e-2, 3e-3):
+        t = O.tempered_block_score(q, Kc, beta)
+        assert (t - (mean + 0.5 * beta * var)) / beta ** 2 == pytest.approx(k3 / 6.0, rel=2e-2)
+    # beta -> infinity: the exact maximum, approached as max - log(B)/beta for a unique max
+    beta = 400.0
+    assert O.tempered_block_score(q, Kc, beta) == pytest.approx(s.max() - math.log(64) / beta, abs=1e-9)
+    # non-decreasing in beta (power-mean inequality)
+    vals = [O.tempered_block_score(q, Kc, b) for b in (0.0, 0.1, 0.5, 1.0, 2.0, 8.0, 50.0)]
+    assert all(a <= b + 1e-12 for a, b in zip(vals, vals[1:]))
