@@ -223,8 +223,9 @@ def algorithmic_work(w, idx):
     G = w.h_q // w.h_kv
     pos = np.arange(w.n_q) + w.q_offset
     nvis = np.minimum(nb, (pos + 1) // w.block).sum()
-    summary_bytes = w.batch * w.n * w.h_kv * w.d * es + w.batch * w.h_kv * nb * 2 * w.d * 2
-    route_flops = 2.0 * (2 * w.d) * float(nvis) * w.h_kv * w.batch
+    # one summary row and one routing dot product per sub-block
+    summary_bytes = w.batch * w.n * w.h_kv * w.d * es + w.batch * w.h_kv * nb * w.subblocks * 2 * w.d * 2
+    route_flops = 2.0 * (2 * w.d) * float(nvis) * w.subblocks * w.h_kv * w.batch
     S = attended_keys(idx, w)
     gathered = float(S.sum().item()) * w.d * 2 * es
     qo = 2.0 * w.batch * w.n_q * w.h_q * w.d * es
@@ -454,15 +455,20 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--n", type=int, default=None,
                     help="shorter sequence of the same workload (profiling captures); not a bench line")
+    ap.add_argument("--subblocks", type=int, default=1,
+                    help="route on S sub-block summaries per block, max-pooled (S in 1, 2, 4; block / S >= 32)")
     a = ap.parse_args()
     w = WORKLOADS[a.workload]
     if a.n is not None:
         w = w.scaled(n=a.n, needles=max(1, w.needles * a.n // w.n))
+    if a.subblocks != 1:
+        w = w.scaled(subblocks=a.subblocks)
     ws, rank, local = dist_setup(a.gpus)
     peaks, peak_src = load_peaks()
 
     config = {"workload": w.name, "batch": w.batch, "n": w.n, "n_q": w.n_q, "h_q": w.h_q, "h_kv": w.h_kv,
               "d": w.d, "block": w.block, "topk": w.topk, "window": w.window, "sigma": w.sigma,
+              "subblocks": w.subblocks,
               "beta": w.beta, "keys": "block-clustered + planted needles" if w.clustered else "iid + planted needles",
               "l2": "flushed between steps (256 MiB write); inputs larger than L2",
               "parallelism": f"replicas x{ws} (independent problems)"}
@@ -482,7 +488,8 @@ def main():
         print(json.dumps(line), flush=True)
         return
 
-    traffic = load_traffic()
+    # the committed DRAM counters were taken with whole-block summaries
+    traffic = load_traffic() if w.subblocks == 1 else {}
     res = run_ours(w, a.steps, a.warmup, ws, rank, with_e2e=not a.no_e2e)
     kern = kernel_report(w, res, peaks, traffic)
     value = whole_job_rate(w.batch * w.n_q * w.h_q, ws, res["ms_step"])
@@ -496,9 +503,12 @@ def main():
     if not a.no_secondary and w.name == PRIMARY and a.n is None:
         torch.cuda.empty_cache()
         w2 = WORKLOADS[SECONDARY]
+        if w.subblocks != 1 and w2.block // w.subblocks >= 32:
+            w2 = w2.scaled(subblocks=w.subblocks)
         r2 = run_ours(w2, max(3, a.steps // 2), a.warmup, ws, rank, with_e2e=False)
         k2 = kernel_report(w2, r2, peaks, traffic)
-        secondary = {"workload": w2.name, "value": whole_job_rate(w2.batch * w2.n_q * w2.h_q, ws, r2["ms_step"]),
+        secondary = {"workload": w2.name, "subblocks": w2.subblocks,
+                     "value": whole_job_rate(w2.batch * w2.n_q * w2.h_q, ws, r2["ms_step"]),
                      "unit": UNIT, "ms_per_step": r2["ms_step"], "kernels": k2, "gpu_launches": r2["launches"],
                      "clocks": r2["clocks"]}
     cpu = None

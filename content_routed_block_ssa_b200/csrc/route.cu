@@ -76,6 +76,8 @@ __global__ void __launch_bounds__(256) features_kernel(const __nv_bfloat16* __re
 
 struct RouteTiledArgs {
   int32_t batch, n_q, h_kv, nb, block, topk;
+  int32_t S;                 // table rows (sub-blocks) per block
+
   int32_t n_tiles, n_units;
   int64_t q_offset;
   int32_t* block_idx;
@@ -111,7 +113,7 @@ __device__ __forceinline__ void route_unit(const RouteTiledArgs& a, int r, int& 
   const int rows = min(256, a.n_q - row0);
   const int64_t pos = a.q_offset + row0 + rows - 1;
   const int nv = static_cast<int>(min(static_cast<int64_t>(a.nb), (pos + 1) / a.block));
-  nch = (nv + 127) / 128;
+  nch = (nv * a.S + 127) / 128;   // 128 table rows (sub-block columns) per chunk
 }
 
 // Snake order over rounds keeps every CTA's total work close to the mean.
@@ -175,13 +177,13 @@ __device__ __forceinline__ void merge_candidates(float (&Ls)[KSEL], int (&Li)[KS
 // Appends the scores above the threshold (strictly: an equal score comes
 // from a higher block index and would rank below the k-th) to the row's
 // candidate buffer, in block order: independent compares build a take mask,
-// then one store per set bit.
-template <bool MASK>
-__device__ __forceinline__ void filter16(const uint32_t (&v)[16], int c0, int nvis, float thr,
+// then one store per set bit.  v holds the scores of blocks c0 .. c0+N-1.
+template <int N, bool MASK>
+__device__ __forceinline__ void filter_n(const uint32_t (&v)[N], int c0, int nvis, float thr,
                                          int& cnt, uint2* my_cand) {
   uint32_t take = 0;
 #pragma unroll
-  for (int t = 0; t < 16; ++t) {
+  for (int t = 0; t < N; ++t) {
     bool tk = __uint_as_float(v[t]) > thr;
     if (MASK) tk = tk && (c0 + t < nvis);
     take |= tk ? (1u << t) : 0u;
@@ -191,10 +193,43 @@ __device__ __forceinline__ void filter16(const uint32_t (&v)[16], int c0, int nv
     const int t = __ffs(static_cast<int>(m)) - 1;
     uint32_t vt = v[0];
 #pragma unroll
-    for (int u = 1; u < 16; ++u) vt = (t == u) ? v[u] : vt;
+    for (int u = 1; u < N; ++u) vt = (t == u) ? v[u] : vt;
     my_cand[cnt * 128] = make_uint2(vt, static_cast<uint32_t>(c0 + t));
     ++cnt;
   }
+}
+
+// Block scores of 16 sub-block columns, S per block: the largest of each
+// block's S sub-block scores (the scores are finite, so fmaxf is the max).
+template <int S>
+__device__ __forceinline__ void pool_columns(const uint32_t (&v)[16], uint32_t (&w)[16 / S]) {
+#pragma unroll
+  for (int t = 0; t < 16 / S; ++t) {
+    float m = __uint_as_float(v[t * S]);
+#pragma unroll
+    for (int s = 1; s < S; ++s) m = fmaxf(m, __uint_as_float(v[t * S + s]));
+    w[t] = __float_as_uint(m);
+  }
+}
+
+// Filters one 16-column TMEM group of a row: c0 is the group's first
+// column, so its blocks start at c0 / S.
+template <int S>
+__device__ __forceinline__ void filter_group(const uint32_t (&v)[16], int c0, int nvis, float thr,
+                                             int& cnt, uint2* my_cand) {
+  constexpr int N = 16 / S;
+  const int b0 = c0 / S;
+  uint32_t w[N];
+  if constexpr (S == 1) {
+#pragma unroll
+    for (int t = 0; t < 16; ++t) w[t] = v[t];
+  } else {
+    pool_columns<S>(v, w);
+  }
+  if (__all_sync(0xFFFFFFFFu, b0 + N <= nvis))
+    filter_n<N, false>(w, b0, nvis, thr, cnt, my_cand);
+  else
+    filter_n<N, true>(w, b0, nvis, thr, cnt, my_cand);
 }
 
 // Warp roles: 0 = TMA producer, 1 = MMA issuer (and TMEM owner), 2..5 and
@@ -260,7 +295,7 @@ __global__ void __launch_bounds__(TiledCfg<KF>::THREADS, 1)
             tma_load_2d(sA + ab * C::A_BYTES + rt * C::A_TILE + ks * C::BOX_BYTES, &tmF, &a_full[ab], ks * 64,
                         frow + rt * 128);
         ++a_cnt;
-        const int trow = bg * a.nb;
+        const int trow = bg * a.nb * a.S;
         for (int j = 0; j < nch && ok; ++j) {
 #pragma unroll
           for (int ks = 0; ks < C::A_BOXES; ++ks) {
@@ -369,10 +404,12 @@ __global__ void __launch_bounds__(TiledCfg<KF>::THREADS, 1)
             if (lane == 0) mbar_arrive(&acc_empty[acc]);
           }
           const int c0 = j * 128 + sub * 16;
-          if (__all_sync(0xFFFFFFFFu, c0 + 16 <= nvis))
-            filter16<false>(v, c0, nvis, thr, cnt, my_cand);
+          if (a.S == 1)
+            filter_group<1>(v, c0, nvis, thr, cnt, my_cand);
+          else if (a.S == 2)
+            filter_group<2>(v, c0, nvis, thr, cnt, my_cand);
           else
-            filter16<true>(v, c0, nvis, thr, cnt, my_cand);
+            filter_group<4>(v, c0, nvis, thr, cnt, my_cand);
           if (__any_sync(0xFFFFFFFFu, cnt > C::CAP - 16)) merge_candidates<KSEL>(Ls, Li, cnt, thr, my_cand, a.topk);
         }
         ++ch_cnt;
@@ -417,7 +454,7 @@ cudaError_t run_tiled(const ssa_params& p, const CUtensorMap& tmF, const CUtenso
   using C = TiledCfg<KF>;
   RouteTiledArgs a;
   a.batch = p.batch; a.n_q = p.n_q; a.h_kv = p.h_kv; a.nb = p.n_kv / p.block;
-  a.block = p.block; a.topk = p.topk;
+  a.block = p.block; a.topk = p.topk; a.S = p.subblocks;
   a.n_tiles = (p.n_q + 255) / 256;   // 256-row units per (batch, kv-head)
   a.n_units = p.batch * p.h_kv * a.n_tiles;
   a.q_offset = p.q_offset;
@@ -435,6 +472,7 @@ cudaError_t run_tiled(const ssa_params& p, const CUtensorMap& tmF, const CUtenso
 
 struct RowArgs {
   int32_t n_q, h_kv, nb, block, topk;
+  int32_t S;                 // summary rows (sub-blocks) per block
   int64_t q_offset;
   float half_beta;
   int32_t* block_idx;
@@ -520,14 +558,17 @@ __global__ void __launch_bounds__(256) route_rowwise_bf16_kernel(const __nv_bflo
       f[v] = __bfloat162float(__float2bfloat16_rn(raw));
     }
   }
-  const __nv_bfloat16* trow = T + (static_cast<int64_t>(b) * a.h_kv + g) * a.nb * (2 * D) + lane * FPL;
-  for (int c0 = warp * 4; c0 < nvis; c0 += 32) {
+  // table rows are sub-blocks (S per block); a warp scores 4 consecutive
+  // rows, which hold 4 / S whole blocks
+  const int nrows = nvis * a.S;
+  const __nv_bfloat16* trow = T + (static_cast<int64_t>(b) * a.h_kv + g) * a.nb * a.S * (2 * D) + lane * FPL;
+  for (int c0 = warp * 4; c0 < nrows; c0 += 32) {
     float part[4];
 #pragma unroll
     for (int u = 0; u < 4; ++u) {
       const int c = c0 + u;
       part[u] = 0.f;
-      if (c < nvis) {
+      if (c < nrows) {
         const __nv_bfloat16* t = trow + static_cast<int64_t>(c) * (2 * D);
         float tv[FPL];
         if (FPL == 8) {
@@ -555,7 +596,13 @@ __global__ void __launch_bounds__(256) route_rowwise_bf16_kernel(const __nv_bflo
     for (int u = 0; u < 4; ++u) {
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1) part[u] += __shfl_xor_sync(0xFFFFFFFFu, part[u], o);
-      const int c = c0 + u;
+    }
+    // a block's score is the largest of its sub-blocks' scores
+    if (a.S >= 2) { part[0] = fmaxf(part[0], part[1]); part[1] = fmaxf(part[2], part[3]); }
+    if (a.S == 4) part[0] = fmaxf(part[0], part[1]);
+    const int nper = 4 / a.S;
+    for (int u = 0; u < nper; ++u) {
+      const int c = c0 / a.S + u;
       if (lane == 0 && c < nvis) keys[c] = make_key(__float_as_uint(part[u]), c);
     }
   }
@@ -582,33 +629,40 @@ __global__ void __launch_bounds__(256) route_rowwise_f32_kernel(const float* __r
   const float* q = Q + ((static_cast<int64_t>(b) * a.n_q + i) * h_q + static_cast<int64_t>(g) * G) * D;
   for (int e = threadIdx.x; e < G * D; e += blockDim.x) qsm[e / D][e % D] = q[e];
   __syncthreads();
-  const int64_t bgrow = (static_cast<int64_t>(b) * a.h_kv + g) * a.nb;
-  for (int c = warp; c < nvis; c += 8) {
-    const float* mu = MU + (bgrow + c) * D;
-    float acc = 0.f;
+  // summary rows are sub-blocks, S per block; a warp scores a block's S
+  // rows and keeps the largest
+  const int64_t bgrow = (static_cast<int64_t>(b) * a.h_kv + g) * a.nb * a.S;
+  for (int cb = warp; cb < nvis; cb += 8) {
+    float best = -INFINITY;
+    for (int sb = 0; sb < a.S; ++sb) {
+      const int64_t c = static_cast<int64_t>(cb) * a.S + sb;
+      const float* mu = MU + (bgrow + c) * D;
+      float acc = 0.f;
 #pragma unroll
-    for (int h = 0; h < G; ++h) {
-      float lin = 0.f, quad = 0.f;
+      for (int h = 0; h < G; ++h) {
+        float lin = 0.f, quad = 0.f;
 #pragma unroll
-      for (int ss = 0; ss < D / 32; ++ss) {
-        const int s = lane + 32 * ss;
-        const float qv = qsm[h][s];
-        lin = __fmaf_rn(qv, __ldg(mu + s), lin);
-        if (FULL) {
-          const float* srow = SG + ((bgrow + c) * D + s) * D;
-          float u = 0.f;
+        for (int ss = 0; ss < D / 32; ++ss) {
+          const int s = lane + 32 * ss;
+          const float qv = qsm[h][s];
+          lin = __fmaf_rn(qv, __ldg(mu + s), lin);
+          if (FULL) {
+            const float* srow = SG + ((bgrow + c) * D + s) * D;
+            float u = 0.f;
 #pragma unroll 8
-          for (int t = 0; t < D; ++t) u = __fmaf_rn(__ldg(srow + t), qsm[h][t], u);
-          quad = __fmaf_rn(qv, u, quad);
-        } else {
-          quad = __fmaf_rn(qv * qv, __ldg(SG + (bgrow + c) * D + s), quad);
+            for (int t = 0; t < D; ++t) u = __fmaf_rn(__ldg(srow + t), qsm[h][t], u);
+            quad = __fmaf_rn(qv, u, quad);
+          } else {
+            quad = __fmaf_rn(qv * qv, __ldg(SG + (bgrow + c) * D + s), quad);
+          }
         }
+        acc += lin + a.half_beta * quad;
       }
-      acc += lin + a.half_beta * quad;
-    }
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xFFFFFFFFu, acc, o);
-    if (lane == 0) keys[c] = make_key(__float_as_uint(acc), c);
+      for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xFFFFFFFFu, acc, o);
+      best = fmaxf(best, acc);
+    }
+    if (lane == 0) keys[cb] = make_key(__float_as_uint(best), cb);
   }
   const int n2 = next_pow2(max(nvis, 1));
   const int64_t out = ((static_cast<int64_t>(b) * a.n_q + i) * a.h_kv + g) * a.topk;
@@ -619,6 +673,7 @@ __global__ void __launch_bounds__(256) route_rowwise_f32_kernel(const float* __r
 RowArgs row_args(const ssa_params& p, int32_t* idx, float* scores) {
   RowArgs a;
   a.n_q = p.n_q; a.h_kv = p.h_kv; a.nb = p.n_kv / p.block; a.block = p.block; a.topk = p.topk;
+  a.S = p.subblocks;
   a.q_offset = p.q_offset;
   a.half_beta = p.beta * 0.5f;   // exact
   a.block_idx = idx; a.top_scores = scores;

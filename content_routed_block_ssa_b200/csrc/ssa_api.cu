@@ -80,6 +80,8 @@ inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 
 inline size_t round_up(size_t x) { return (x + 255) & ~size_t(255); }
 
 int64_t nb_of(const ssa_params& p) { return p.block > 0 ? p.n_kv / p.block : 0; }
+// Summary rows per (batch, kv-head): one per sub-block.
+int64_t summary_rows(const ssa_params& p) { return nb_of(p) * p.subblocks; }
 size_t esize(const ssa_params& p) { return p.dtype == SSA_BF16 ? 2 : 4; }
 
 bool is_empty(const ssa_params& p) { return p.batch == 0 || p.n_q == 0; }
@@ -92,6 +94,7 @@ ssa_status check_params(const ssa_params* pp) {
       p.topk < 1 || p.window < 1)
     return SSA_ERR_INVALID_ARG;
   if (p.h_q % p.h_kv != 0 || p.n_kv % p.block != 0) return SSA_ERR_INVALID_ARG;
+  if (p.subblocks < 1 || p.block % p.subblocks != 0 || p.reserved != 0) return SSA_ERR_INVALID_ARG;
   if (p.q_offset < 0 || p.q_offset + p.n_q > p.n_kv) return SSA_ERR_INVALID_ARG;
   if ((p.dtype != SSA_F32 && p.dtype != SSA_BF16) || (p.sigma != SSA_SIGMA_DIAG && p.sigma != SSA_SIGMA_FULL) ||
       p.route_impl < SSA_ROUTE_AUTO || p.route_impl > SSA_ROUTE_ROWWISE)
@@ -100,13 +103,15 @@ ssa_status check_params(const ssa_params* pp) {
   const int G = p.h_q / p.h_kv;
   if (p.d != 64 && p.d != 128) return SSA_ERR_UNSUPPORTED;
   if (p.block != 64 && p.block != 128) return SSA_ERR_UNSUPPORTED;
+  if ((p.subblocks != 1 && p.subblocks != 2 && p.subblocks != 4) || p.block / p.subblocks < 32)
+    return SSA_ERR_UNSUPPORTED;
   if (G != 1 && G != 2 && G != 4 && G != 8) return SSA_ERR_UNSUPPORTED;
   if (p.topk > 32 || p.window > 4032) return SSA_ERR_UNSUPPORTED;
   if (p.dtype == SSA_BF16 && p.sigma != SSA_SIGMA_DIAG) return SSA_ERR_UNSUPPORTED;
   // index ranges used by the kernels and the TMA coordinates
   const int64_t rows_kv = static_cast<int64_t>(p.batch) * p.n_kv;
   const int64_t rows_q = static_cast<int64_t>(p.batch) * p.h_kv * p.n_q;
-  const int64_t rows_t = static_cast<int64_t>(p.batch) * p.h_kv * nb_of(p);
+  const int64_t rows_t = static_cast<int64_t>(p.batch) * p.h_kv * summary_rows(p);
   if (rows_kv > INT32_MAX || rows_q > INT32_MAX || rows_t > INT32_MAX) return SSA_ERR_UNSUPPORTED;
   if (p.batch > 65535 || p.h_kv > 65535 || nb_of(p) > 2147483647) return SSA_ERR_UNSUPPORTED;
   return SSA_OK;
@@ -129,15 +134,15 @@ size_t features_bytes(const ssa_params& p) {
   return use_tiled(p) ? round_up(static_cast<size_t>(p.batch) * p.h_kv * p.n_q * 2 * p.d * 2) : 0;
 }
 size_t table_bytes(const ssa_params& p) {
-  return p.dtype == SSA_BF16 ? round_up(static_cast<size_t>(p.batch) * p.h_kv * nb_of(p) * 2 * p.d * 2) : 0;
+  return p.dtype == SSA_BF16 ? round_up(static_cast<size_t>(p.batch) * p.h_kv * summary_rows(p) * 2 * p.d * 2) : 0;
 }
 size_t mu_bytes(const ssa_params& p) {
-  return p.dtype == SSA_F32 ? round_up(static_cast<size_t>(p.batch) * p.h_kv * nb_of(p) * p.d * 4) : 0;
+  return p.dtype == SSA_F32 ? round_up(static_cast<size_t>(p.batch) * p.h_kv * summary_rows(p) * p.d * 4) : 0;
 }
 size_t sigma_bytes(const ssa_params& p) {
   if (p.dtype != SSA_F32) return 0;
   const size_t per = p.sigma == SSA_SIGMA_FULL ? static_cast<size_t>(p.d) * p.d : p.d;
-  return round_up(static_cast<size_t>(p.batch) * p.h_kv * nb_of(p) * per * 4);
+  return round_up(static_cast<size_t>(p.batch) * p.h_kv * summary_rows(p) * per * 4);
 }
 size_t idx_bytes(const ssa_params& p) {
   return round_up(static_cast<size_t>(p.batch) * p.n_q * p.h_kv * p.topk * 4);
@@ -277,7 +282,7 @@ ssa_status do_route(const ssa_params& p, const void* Q, const float* mu, const f
   CUtensorMap tmF, tmT;
   const uint64_t kf = 2 * static_cast<uint64_t>(p.d);
   if (!encode_2d(&tmF, ws, kf, static_cast<uint64_t>(p.batch) * p.h_kv * p.n_q, 128) ||
-      !encode_2d(&tmT, table, kf, static_cast<uint64_t>(p.batch) * p.h_kv * nb_of(p), 128))
+      !encode_2d(&tmT, table, kf, static_cast<uint64_t>(p.batch) * p.h_kv * summary_rows(p), 128))
     return SSA_ERR_CUDA;
   return from_cuda(ssa::launch_route_tiled(p, tmF, tmT, idx, scores, c));
 }

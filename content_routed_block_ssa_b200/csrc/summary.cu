@@ -4,9 +4,10 @@
 // [Subquadratic Sparse Attention (SSA), opening section]; the routing score
 // needs the block mean mu_c and the covariance Sigma_c of the block's keys
 // ["The idea in one screen", routing-score equation].  Normalisation is by
-// the block size B (population moments).
+// the number of keys summarised (population moments).
 //
-// One CTA per (batch, kv-head, block).  The block's B x d keys are read once
+// One CTA per (batch, kv-head, unit), a unit being a block of B keys, or a
+// sub-block of B / S keys when each block is summarised S times.  The block's B x d keys are read once
 // with 16-byte coalesced loads into registers; the mean and then the centred
 // second moments are reduced in float64.  For bf16 and float32 keys every
 // partial sum of the mean is exact in float64, so mu is the exact block mean
@@ -145,53 +146,68 @@ __global__ void __launch_bounds__(256) summary_full_kernel(const float* __restri
   }
 }
 
+// A launch summarises units of BLK keys: whole blocks, or the sub-blocks of
+// B / S keys when S > 1 (unit c*S + s is sub-block s of block c, so the rows
+// come out in that order with no index arithmetic of their own).
 template <typename T, int D, int BLK>
 cudaError_t run_diag(const ssa_params& p, const void* K, float* mu, float* sig, void* table,
                      const LaunchCtx& c) {
-  const int nb = p.n_kv / p.block;
-  dim3 grid(nb, p.h_kv, p.batch);
+  const int nu = p.n_kv / BLK;
+  dim3 grid(nu, p.h_kv, p.batch);
   summary_diag_kernel<T, D, BLK><<<grid, 256, 0, c.stream>>>(
-      static_cast<const T*>(K), mu, sig, static_cast<__nv_bfloat16*>(table), p.n_kv, p.h_kv, nb);
+      static_cast<const T*>(K), mu, sig, static_cast<__nv_bfloat16*>(table), p.n_kv, p.h_kv, nu);
   note_launch();
   return cudaGetLastError();
 }
 
 template <int D, int BLK>
 cudaError_t run_full(const ssa_params& p, const void* K, float* mu, float* sig, const LaunchCtx& c) {
-  const int nb = p.n_kv / p.block;
+  const int nu = p.n_kv / BLK;
   const int smem = BLK * D * static_cast<int>(sizeof(double));
   cudaError_t e = cudaFuncSetAttribute(summary_full_kernel<D, BLK>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
-  dim3 grid(nb, p.h_kv, p.batch);
+  dim3 grid(nu, p.h_kv, p.batch);
   summary_full_kernel<D, BLK><<<grid, 256, smem, c.stream>>>(static_cast<const float*>(K), mu, sig,
-                                                             p.n_kv, p.h_kv, nb);
+                                                             p.n_kv, p.h_kv, nu);
   note_launch();
   return cudaGetLastError();
+}
+
+template <int D>
+cudaError_t full_u(int unit, const ssa_params& p, const void* K, float* mu, float* sig, const LaunchCtx& c) {
+  if (unit == 32) return run_full<D, 32>(p, K, mu, sig, c);
+  if (unit == 64) return run_full<D, 64>(p, K, mu, sig, c);
+  if (unit == 128) return run_full<D, 128>(p, K, mu, sig, c);
+  return cudaErrorInvalidValue;
+}
+
+template <typename T, int D>
+cudaError_t diag_u(int unit, const ssa_params& p, const void* K, float* mu, float* sig, void* table,
+                   const LaunchCtx& c) {
+  if (unit == 32) return run_diag<T, D, 32>(p, K, mu, sig, table, c);
+  if (unit == 64) return run_diag<T, D, 64>(p, K, mu, sig, table, c);
+  if (unit == 128) return run_diag<T, D, 128>(p, K, mu, sig, table, c);
+  return cudaErrorInvalidValue;
 }
 
 }  // namespace
 
 cudaError_t launch_summary(const ssa_params& p, const void* K, float* mu, float* sigma,
                            void* table, const LaunchCtx& c) {
-  const bool bf = p.dtype == SSA_BF16;
+  if (p.subblocks < 1 || p.block % p.subblocks != 0) return cudaErrorInvalidValue;
+  const int unit = p.block / p.subblocks;
   if (p.sigma == SSA_SIGMA_FULL) {
-    if (p.d == 64 && p.block == 64) return run_full<64, 64>(p, K, mu, sigma, c);
-    if (p.d == 64 && p.block == 128) return run_full<64, 128>(p, K, mu, sigma, c);
-    if (p.d == 128 && p.block == 64) return run_full<128, 64>(p, K, mu, sigma, c);
-    if (p.d == 128 && p.block == 128) return run_full<128, 128>(p, K, mu, sigma, c);
+    if (p.d == 64) return full_u<64>(unit, p, K, mu, sigma, c);
+    if (p.d == 128) return full_u<128>(unit, p, K, mu, sigma, c);
     return cudaErrorInvalidValue;
   }
-  if (bf) {
-    if (p.d == 128 && p.block == 64) return run_diag<__nv_bfloat16, 128, 64>(p, K, mu, sigma, table, c);
-    if (p.d == 128 && p.block == 128) return run_diag<__nv_bfloat16, 128, 128>(p, K, mu, sigma, table, c);
-    if (p.d == 64 && p.block == 64) return run_diag<__nv_bfloat16, 64, 64>(p, K, mu, sigma, table, c);
-    if (p.d == 64 && p.block == 128) return run_diag<__nv_bfloat16, 64, 128>(p, K, mu, sigma, table, c);
+  if (p.dtype == SSA_BF16) {
+    if (p.d == 128) return diag_u<__nv_bfloat16, 128>(unit, p, K, mu, sigma, table, c);
+    if (p.d == 64) return diag_u<__nv_bfloat16, 64>(unit, p, K, mu, sigma, table, c);
   } else {
-    if (p.d == 128 && p.block == 64) return run_diag<float, 128, 64>(p, K, mu, sigma, nullptr, c);
-    if (p.d == 128 && p.block == 128) return run_diag<float, 128, 128>(p, K, mu, sigma, nullptr, c);
-    if (p.d == 64 && p.block == 64) return run_diag<float, 64, 64>(p, K, mu, sigma, nullptr, c);
-    if (p.d == 64 && p.block == 128) return run_diag<float, 64, 128>(p, K, mu, sigma, nullptr, c);
+    if (p.d == 128) return diag_u<float, 128>(unit, p, K, mu, sigma, nullptr, c);
+    if (p.d == 64) return diag_u<float, 64>(unit, p, K, mu, sigma, nullptr, c);
   }
   return cudaErrorInvalidValue;
 }

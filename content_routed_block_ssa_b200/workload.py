@@ -50,6 +50,7 @@ class Workload:
     clustered: bool = False
     decode: bool = False
     beta: float = 2.0
+    subblocks: int = 1  # summaries per block (sub-block max-pool routing when > 1)
 
     @property
     def n_q(self) -> int:
@@ -162,4 +163,5 @@ def problem_dict(w: Workload) -> dict:
     """Layer parameters of a workload (argument names of the C struct)."""
     return dict(batch=w.batch, n_q=w.n_q, n_kv=w.n, h_q=w.h_q, h_kv=w.h_kv, d=w.d,
                 block=w.block, topk=w.topk, window=w.window, q_offset=w.q_offset,
-                beta=w.beta, scale=1.0 / math.sqrt(w.d), dtype=w.dtype, sigma=w.sigma)
+                beta=w.beta, scale=1.0 / math.sqrt(w.d), dtype=w.dtype, sigma=w.sigma,
+                subblocks=w.subblocks)

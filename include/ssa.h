@@ -103,7 +103,22 @@ typedef struct {
   int64_t q_offset;   /* key position of query row 0                      */
   float beta;         /* routing inverse temperature                      */
   float scale;        /* attention logit scale (normally 1/sqrt(d))        */
+  int32_t subblocks;  /* S in {1, 2, 4}: summaries per block (see below)  */
+  int32_t reserved;   /* must be 0                                        */
 } ssa_params;
+
+/*
+ * Sub-block summaries (subblocks = S > 1): every block of B keys is
+ * summarised as S sub-blocks of B/S consecutive keys (B/S >= 32), and a
+ * block's routing score is the largest of its sub-blocks' scores, each the
+ * second-cumulant score of those keys (summed over the kv-head's query
+ * heads).  The finer summaries keep a single strongly matching key from
+ * being averaged away over the whole block — the sub-block part of the
+ * selector named "Certified Causal Cascade" ("Subquadratic Sparse Attention
+ * (SSA)", artifact list: sub-block max-pool).  Selection, the window and the
+ * attention still work on whole blocks.  Summary outputs then have nb * S
+ * rows per (batch, kv-head), sub-block s of block c at row c * S + s.
+ */
 
 /* Human-readable name of a status code (static string, never NULL). */
 SSA_API const char* ssa_status_string(int32_t status);

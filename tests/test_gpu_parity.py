@@ -43,6 +43,17 @@ CASES = {
     "f32_full_d64": Workload("c", 106, 1, 1024, 1, 1, 64, "f32", 64, "full", 8, 64, 8, "total"),
     "f32_diag_d128_gqa4_w100": Workload("c", 107, 1, 512, 4, 1, 128, "f32", 64, "diag", 4, 100, 4, "total"),
     "f32_full_gqa2_d64_b128": Workload("c", 108, 1, 768, 2, 1, 64, "f32", 128, "full", 2, 64, 2, "total"),
+    # sub-block summaries (max-pooled block scores): 32-key units from 64- and
+    # 128-key blocks, 64-key units at d = 64, float32 full and diagonal
+    "bf16_gqa4_d128_b64_s2": Workload("c", 117, 1, 1280, 8, 2, 128, "bf16", 64, "diag", 8, 128, 6, "total",
+                                      clustered=True, subblocks=2),
+    "bf16_gqa8_d128_b128_s4": Workload("c", 118, 1, 2304, 8, 1, 128, "bf16", 128, "diag", 8, 256, 8, "total",
+                                       subblocks=4),
+    "bf16_mha_d64_b128_s2": Workload("c", 119, 1, 1024, 2, 2, 64, "bf16", 128, "diag", 4, 128, 4, "per_head",
+                                     subblocks=2),
+    "f32_full_d64_s2": Workload("c", 120, 1, 768, 1, 1, 64, "f32", 64, "full", 4, 64, 4, "total", subblocks=2),
+    "f32_diag_gqa2_d128_b128_s4": Workload("c", 121, 1, 512, 2, 1, 128, "f32", 128, "diag", 2, 100, 2, "total",
+                                           subblocks=4),
 }
 
 _cache = {}

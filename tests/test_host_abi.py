@@ -30,10 +30,12 @@ def test_library_exports_every_declared_symbol():
 
 
 def test_params_layout_matches_header():
-    assert C.sizeof(ssa.ssa_params) == 64
+    assert C.sizeof(ssa.ssa_params) == 72
     assert ssa.ssa_params.q_offset.offset == 48
     assert ssa.ssa_params.beta.offset == 56
     assert ssa.ssa_params.scale.offset == 60
+    assert ssa.ssa_params.subblocks.offset == 64
+    assert ssa.ssa_params.reserved.offset == 68
     text = open(HEADER).read()
     body = text[text.index("typedef struct {"):text.index("} ssa_params;")]
     fields = re.findall(r"\b(int32_t|int64_t|float)\s+(\w+);", body)
@@ -71,6 +73,11 @@ def good(**kw):
     (dict(topk=33), ssa.SSA_ERR_UNSUPPORTED),
     (dict(window=5000), ssa.SSA_ERR_UNSUPPORTED),
     (dict(sigma="full"), ssa.SSA_ERR_UNSUPPORTED),          # bf16 routes on a diagonal Sigma
+    (dict(subblocks=0), ssa.SSA_ERR_INVALID_ARG),
+    (dict(subblocks=3), ssa.SSA_ERR_INVALID_ARG),           # does not divide the block
+    (dict(subblocks=4), ssa.SSA_ERR_UNSUPPORTED),           # 16-key sub-blocks
+    (dict(subblocks=8, block=128), ssa.SSA_ERR_UNSUPPORTED),
+    (dict(subblocks=64), ssa.SSA_ERR_UNSUPPORTED),
 ])
 def test_invalid_and_unsupported_params(kw, code):
     p = good(**kw)
@@ -79,6 +86,14 @@ def test_invalid_and_unsupported_params(kw, code):
     assert ssa.lib.ssa_forward(C.byref(p), dummy, dummy, dummy, dummy, None, dummy, 1 << 30, None) == code
     assert ssa.lib.ssa_sparse_attn(C.byref(p), dummy, dummy, dummy, dummy, dummy, None, None, None, 0, None) == code
     assert ssa.lib.ssa_workspace_size(C.byref(p)) == 0
+
+
+def test_reserved_field_must_be_zero():
+    p = good()
+    p.reserved = 1
+    dummy = 256
+    assert ssa.lib.ssa_block_summary(C.byref(p), dummy, None, None, dummy, None) == ssa.SSA_ERR_INVALID_ARG
+    assert ssa.ssa_workspace_size(p) == 0
 
 
 def test_null_and_misaligned_pointers_rejected():
@@ -120,6 +135,13 @@ def test_workspace_sizes():
     assert ssa.ssa_workspace_size(f32) == rnd(2 * nb * 64 * 4) + rnd(2 * nb * 64 * 64 * 4) + rnd(128 * 2 * 4 * 4)
     h = ssa.ssa_hostio_buffer_size(p)
     assert h > ssa.ssa_workspace_size(p)
+    # sub-block summaries: S route-table rows per block
+    s2 = good(n_q=1000, n_kv=1024, subblocks=2)
+    assert ssa.ssa_workspace_size(s2) == rnd(2 * tab) + rnd(feat) + rnd(idx)
+    mu, sig, t = ssa.summary_shapes(s2)
+    assert mu == (1, 2, 2 * 16, 128) and t == (1, 2, 2 * 16, 256)
+    f4 = good(dtype="f32", sigma="full", d=64, h_q=2, n_q=128, n_kv=128, block=128, subblocks=4)
+    assert ssa.ssa_workspace_size(f4) == rnd(2 * 4 * 64 * 4) + rnd(2 * 4 * 64 * 64 * 4) + rnd(128 * 2 * 4 * 4)
 
 
 def test_block_major_workspace_and_stage_checks():
