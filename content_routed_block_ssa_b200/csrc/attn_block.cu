@@ -309,17 +309,22 @@ struct BlkCfg {
   static constexpr int KV_HALF = BLK * ROW;             // BLK keys x 64 dims
   static constexpr int KV_BYTES = 4 * KV_HALF;          // K lo, K hi, V lo, V hi
   static constexpr int NKV = (BLK == 64) ? 2 : 1;       // K/V buffers (at most 2)
-  static constexpr int P_HALF = 128 * ROW;              // 128 rows x 64 keys
-  static constexpr int P_BYTES = (BLK / 64) * P_HALF;
-  static constexpr int NBAR = 2 * NA + 2 * NKV + 2 * 5 + 1;
-  static constexpr int SMEM = 1024 + NA * A_BYTES + NKV * KV_BYTES + 2 * P_BYTES + NBAR * 8 + 16;
+  static constexpr int STG_BYTES = 128 * ROW;           // epilogue staging: 128 rows x 64 dims
+  static constexpr int NBAR = 2 * NA + 2 * NKV + 2 * 6 + 1;
+  // (m, l) of each row from the softmax to the epilogue, by tile parity: in
+  // spare TMEM columns with 64-key blocks, else in shared memory
+  static constexpr bool ML_TMEM = (BLK == 64);
+  static constexpr int ML_BYTES = ML_TMEM ? 0 : 2 * 128 * 8;
+  static constexpr int SMEM = 1024 + NA * A_BYTES + NKV * KV_BYTES + 2 * STG_BYTES + ML_BYTES + NBAR * 8 + 16;
   static constexpr int SW0 = 2 + NGW;                   // first softmax warp
   static constexpr int THREADS = 32 * (SW0 + 8);        // KV, MMA, gather, 2 x 4 softmax warps
   // registers per thread: a sub-partition (SMSP) holds ceil(warps / 4) warps
   // of its 16384 registers
   static constexpr int MAXREG = (16384 / (32 * ((SW0 + 8 + 3) / 4))) & ~7;
-  static constexpr int S_COL = 0;                       // TMEM: S[2] then O[2]
-  static constexpr int O_COL = 2 * BLK;
+  static constexpr int S_COL = 0;                       // TMEM: S[2] (P over the first BLK/2
+  static constexpr int O_COL = 2 * BLK;                 // columns of its S), O[2], (m, l)[2]
+  static constexpr int ML_COL = O_COL + 2 * 128;
+  static_assert(!ML_TMEM || ML_COL + 4 <= 512, "tensor memory");
   static_assert(SMEM <= 232448, "shared memory");
 };
 
@@ -393,8 +398,9 @@ __global__ void __maxnreg__((BlkCfg<G, BLK>::MAXREG))
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sA = smem;                                   // [NA][A_BYTES]
   uint8_t* sKV = sA + NA * C::A_BYTES;                  // [NKV][KV_BYTES]
-  uint8_t* sP = sKV + C::NKV * C::KV_BYTES;             // [2][P_BYTES]
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sP + 2 * C::P_BYTES);
+  uint8_t* sStg = sKV + C::NKV * C::KV_BYTES;           // [2][STG_BYTES] epilogue staging
+  float2* sML = reinterpret_cast<float2*>(sStg + 2 * C::STG_BYTES);   // [2][128] when not in TMEM
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sStg + 2 * C::STG_BYTES + C::ML_BYTES);
   uint64_t* a_full = bars;                  // [NA] gather warp arrives once its copies landed
   uint64_t* a_empty = a_full + NA;          // [NA]
   uint64_t* kv_full = a_empty + NA;         // [NKV]
@@ -404,7 +410,8 @@ __global__ void __maxnreg__((BlkCfg<G, BLK>::MAXREG))
   uint64_t* p_full = s_empty + 2;           // [2]
   uint64_t* o_full = p_full + 2;            // [2]
   uint64_t* o_empty = o_full + 2;           // [2]
-  uint64_t* mma_done = o_empty + 2;
+  uint64_t* ml_empty = o_empty + 2;         // [2] the epilogue has read a tile's (m, l)
+  uint64_t* mma_done = ml_empty + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
@@ -412,8 +419,9 @@ __global__ void __maxnreg__((BlkCfg<G, BLK>::MAXREG))
     for (int i = 0; i < NA; ++i) { mbar_init(&a_full[i], 1); mbar_init(&a_empty[i], 1); }
     for (int i = 0; i < C::NKV; ++i) { mbar_init(&kv_full[i], 1); mbar_init(&kv_empty[i], 1); }
     for (int i = 0; i < 2; ++i) {
-      mbar_init(&s_full[i], 1); mbar_init(&s_empty[i], 4);
+      mbar_init(&s_full[i], 1); mbar_init(&s_empty[i], 1);
       mbar_init(&p_full[i], 4); mbar_init(&o_full[i], 1); mbar_init(&o_empty[i], 4);
+      mbar_init(&ml_empty[i], 4);
     }
     mbar_init(mma_done, 1);
     fence_barrier_init();
@@ -477,7 +485,7 @@ __global__ void __maxnreg__((BlkCfg<G, BLK>::MAXREG))
     if (lane == 0) {
       constexpr uint32_t IDESC1 = umma_idesc_bf16(128, BLK);
       constexpr uint32_t IDESC2 = umma_idesc_bf16(128, D) | (1u << 16);   // B (V) is MN-major
-      const uint32_t sA_u = smem_u32(sA), sKV_u = smem_u32(sKV), sP_u = smem_u32(sP);
+      const uint32_t sA_u = smem_u32(sA), sKV_u = smem_u32(sKV);
       int n1 = 0, n2 = 0;               // tiles whose S = Q K^T / O = P V are issued
       int kv_ord = -1;
       int64_t prev = -1;
@@ -527,14 +535,17 @@ __global__ void __maxnreg__((BlkCfg<G, BLK>::MAXREG))
             tc_fence_after();
             const int kb2 = (ring_kb >> (n2 & 3)) & 1;
             const uint32_t d_tmem = tmem_base + C::O_COL + ob * D;
+            // P (bf16, two per column) sits over the first BLK/2 columns of
+            // this tile's S; 16 keys = 8 columns per step
+            const uint32_t p_tmem = tmem_base + C::S_COL + ob * BLK;
             const uint32_t vbase = sKV_u + kb2 * C::KV_BYTES + 2 * C::KV_HALF;
 #pragma unroll
             for (int kk = 0; kk < BLK / 16; ++kk) {
-              const uint64_t ad = umma_desc_sw128(sP_u + ob * C::P_BYTES + (kk >> 2) * C::P_HALF + (kk & 3) * 32);
               const uint64_t bd = umma_desc_sw128_mn(vbase + kk * 16 * C::ROW, C::KV_HALF, 1024);
-              umma_bf16(d_tmem, ad, bd, IDESC2, kk != 0 ? 1u : 0u);
+              umma_bf16_tmem_a(d_tmem, p_tmem + kk * 8, bd, IDESC2, kk != 0 ? 1u : 0u);
             }
             umma_commit(&o_full[ob]);
+            umma_commit(&s_empty[ob]);   // P read: the S / P columns take the next tile
             if ((ring_last >> (n2 & 3)) & 1) umma_commit(&kv_empty[kb2]);
             ++n2;
             progressed = true;
@@ -560,164 +571,206 @@ __global__ void __maxnreg__((BlkCfg<G, BLK>::MAXREG))
     }
   } else if (warp >= C::SW0) {
     // ------------------------------------------------------------ softmax + epilogue
-    const int grp = (warp - C::SW0) >> 2;     // tiles grp, grp + 2, ...
+    // Group g runs the softmax of tiles g, g + 2, ... and, after each, the
+    // epilogue of the other group's previous tile, whose O is complete by
+    // then: neither group waits on its own tile's P V.  A tile's S columns
+    // take its P, and are free for the next tile of the same parity as soon
+    // as P V has read them.
+    const int grp = (warp - C::SW0) >> 2;
     const int eq = warp & 3;
     const int row = eq * 32 + lane;
     const int e = row / G, h = row % G;
     const uint32_t lane_base = static_cast<uint32_t>(eq * 32) << 16;
-    const int sb = grp;                        // this group's S, P and O buffers
+    // this warp's 32 staging rows (a 64-dim half of each)
+    uint8_t* stage = sStg + grp * C::STG_BYTES + eq * 32 * C::ROW;
+    auto tile_at = [&](int x) { return (x >= 0 && x < T) ? a.tiles[t0 + x] : none; };
+    auto entry_of = [&](const int4& td) { return e < td.w ? __ldg(a.entries + td.z + e) : 0; };
+    // descriptors two tiles ahead and this thread's entry one tile ahead on
+    // both chains (softmax tiles grp + 2k, epilogue tiles grp - 1 + 2k)
+    int4 s_td = tile_at(grp), s_td2 = tile_at(grp + 2);
+    int4 e_td = tile_at(grp - 1), e_td2 = tile_at(grp + 1);
+    int s_ent = entry_of(s_td), e_ent = entry_of(e_td);
     bool ok = true;
-    // this group's tile descriptors two of its tiles ahead and this thread's
-    // entry one ahead, so neither load stalls the loop (the descriptor of the
-    // next tile has arrived when its entry is fetched)
-    int4 nxt = grp < T ? a.tiles[t0 + grp] : none;
-    int4 nxt2 = grp + 2 < T ? a.tiles[t0 + grp + 2] : none;
-    int nxt_ent = e < nxt.w ? __ldg(a.entries + nxt.z + e) : 0;
-    for (int lt = grp; lt < T && ok; lt += 2) {
-      const int use = lt >> 1;                 // this buffer's use count
-      const int4 td = nxt;
-      const int ent = nxt_ent;
-      nxt = nxt2;
-      nxt2 = lt + 4 < T ? a.tiles[t0 + lt + 4] : none;
-      nxt_ent = e < nxt.w ? __ldg(a.entries + nxt.z + e) : 0;
-      const int bg = td.x, ne = td.w;
-      const int i = entry_row(ent), j = entry_slot(ent);
-      const bool valid = e < ne && static_cast<unsigned>(i) < static_cast<unsigned>(a.n_q) && j < a.nsl;
-      // a window slot keeps the block's keys inside pos-W+1 .. pos
-      int klo = 0, khi = BLK - 1;
-      if (valid && j >= a.topk) {
-        const int64_t pos = a.q_offset + i, base = static_cast<int64_t>(td.y) * BLK;
-        const int64_t lo = pos - a.window + 1;
-        klo = static_cast<int>(max(lo - base, static_cast<int64_t>(0)));
-        khi = static_cast<int>(min(pos - base, static_cast<int64_t>(BLK - 1)));
-      }
-      ok = __all_sync(0xFFFFFFFFu, mbar_wait(&s_full[sb], use & 1, a.err, SITE_BLK_S_FULL));
-      if (!ok) break;
-      tc_fence_after();
-      // the row's scaled logits in halves of 64 columns: the maximum, then
-      // P = 2^(s - m) in bfloat16 into the swizzled P tile
-      const uint32_t scol = tmem_base + lane_base + C::S_COL + sb * BLK;
-      // a half of S, loaded with the columns outside [klo, khi] set to -inf;
-      // most tiles hold no window slot, and their warps skip the masking
-      const bool any_mask = __any_sync(0xFFFFFFFFu, klo > 0 || khi < BLK - 1);
-      auto load_half = [&](int hf, uint32_t (&r)[64]) {
-        tmem_ld64(scol + hf * 64, r);
-        if (any_mask) {
-          const int lo = klo - hf * 64, hi = khi - hf * 64;
-#pragma unroll
-          for (int u = 0; u < 64; ++u) r[u] = (u >= lo && u <= hi) ? r[u] : 0xFF800000u;
+    for (int ts = grp; ok; ts += 2) {
+      const int te = ts - 1;
+      if (ts >= T && te >= T) break;
+      const int4 std_ = s_td, etd = e_td;
+      const int sent = s_ent, eent = e_ent;
+      s_td = s_td2; s_td2 = tile_at(ts + 4);
+      e_td = e_td2; e_td2 = tile_at(te + 4);
+      s_ent = entry_of(s_td);
+      e_ent = entry_of(e_td);
+      if (ts < T) {
+        // ---------------- softmax of tile ts: P = 2^(s - m) in bf16 over S
+        const int sb = ts & 1, use = ts >> 1;
+        const int i = entry_row(sent), j = entry_slot(sent);
+        const bool valid = e < std_.w && static_cast<unsigned>(i) < static_cast<unsigned>(a.n_q) && j < a.nsl;
+        // a window slot keeps the block's keys inside pos-W+1 .. pos
+        int klo = 0, khi = BLK - 1;
+        if (valid && j >= a.topk) {
+          const int64_t pos = a.q_offset + i, base = static_cast<int64_t>(std_.y) * BLK;
+          const int64_t lo = pos - a.window + 1;
+          klo = static_cast<int>(max(lo - base, static_cast<int64_t>(0)));
+          khi = static_cast<int>(min(pos - base, static_cast<int64_t>(BLK - 1)));
         }
-      };
-      // maxima and sums in eight independent chains
-      float mx[8] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY, -INFINITY, -INFINITY, -INFINITY, -INFINITY};
-      float ls[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-      float m = -INFINITY;
-      uint8_t* prow = sP + sb * C::P_BYTES;
-      if (BLK > 64) {   // first pass: the maximum over both halves
+        ok = __all_sync(0xFFFFFFFFu, mbar_wait(&s_full[sb], use & 1, a.err, SITE_BLK_S_FULL));
+        if (!ok) break;
+        tc_fence_after();
+        const uint32_t scol = tmem_base + lane_base + C::S_COL + sb * BLK;
+        // a half of S, loaded with the columns outside [klo, khi] set to -inf;
+        // most tiles hold no window slot, and their warps skip the masking
+        const bool any_mask = __any_sync(0xFFFFFFFFu, klo > 0 || khi < BLK - 1);
+        auto load_half = [&](int hf, uint32_t (&r)[64]) {
+          tmem_ld64(scol + hf * 64, r);
+          if (any_mask) {
+            const int lo = klo - hf * 64, hi = khi - hf * 64;
+#pragma unroll
+            for (int u = 0; u < 64; ++u) r[u] = (u >= lo && u <= hi) ? r[u] : 0xFF800000u;
+          }
+        };
+        // maxima and sums in eight independent chains
+        float mx[8] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY, -INFINITY, -INFINITY, -INFINITY, -INFINITY};
+        float ls[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+        float m = -INFINITY;
+        if (BLK > 64) {   // first pass: the maximum over both halves
+#pragma unroll
+          for (int hf = 0; hf < BLK / 64; ++hf) {
+            uint32_t r[64];
+            load_half(hf, r);
+#pragma unroll
+            for (int u = 0; u < 64; ++u) mx[u & 7] = fmaxf(mx[u & 7], __uint_as_float(r[u]));
+          }
+          m = max8(mx) * a.scale_log2;
+        }
+        // P of half hf goes to columns hf*32 .. hf*32+31: the S columns it
+        // covers are already in registers (half 0) or consumed (half 1)
 #pragma unroll
         for (int hf = 0; hf < BLK / 64; ++hf) {
           uint32_t r[64];
           load_half(hf, r);
+          if (BLK == 64) {
 #pragma unroll
-          for (int u = 0; u < 64; ++u) mx[u & 7] = fmaxf(mx[u & 7], __uint_as_float(r[u]));
+            for (int u = 0; u < 64; ++u) mx[u & 7] = fmaxf(mx[u & 7], __uint_as_float(r[u]));
+            m = max8(mx) * a.scale_log2;
+          }
+#pragma unroll
+          for (int qq = 0; qq < 2; ++qq) {   // 32 keys = 16 columns of P per store
+            uint32_t pw[16];
+#pragma unroll
+            for (int u = 0; u < 16; ++u) {
+              const int c = qq * 32 + 2 * u;
+              const float p0 = fast_exp2(fmaf(__uint_as_float(r[c]), a.scale_log2, -m));
+              const float p1 = fast_exp2(fmaf(__uint_as_float(r[c + 1]), a.scale_log2, -m));
+              ls[c & 7] += p0;
+              ls[(c + 1) & 7] += p1;
+              pw[u] = pack_bf16(p0, p1);
+            }
+            tmem_st16(scol + hf * 32 + qq * 16, pw);
+          }
         }
-        m = max8(mx) * a.scale_log2;
+        const float l = ((ls[0] + ls[1]) + (ls[2] + ls[3])) + ((ls[4] + ls[5]) + (ls[6] + ls[7]));
+        // (m, l) into this parity's slot once the epilogue two tiles back read it
+        ok = __all_sync(0xFFFFFFFFu, mbar_wait(&ml_empty[sb], (use & 1) ^ 1, a.err, SITE_BLK_ML_EMPTY));
+        if (!ok) break;
+        tc_fence_after();
+        if (C::ML_TMEM) {
+          const uint32_t mlv[2] = {__float_as_uint(m), __float_as_uint(l)};
+          tmem_st2(tmem_base + lane_base + C::ML_COL + sb * 2, mlv);
+        } else {
+          sML[sb * 128 + row] = make_float2(m, l);
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&p_full[sb]);
       }
-#pragma unroll
-      for (int hf = 0; hf < BLK / 64; ++hf) {
-        uint32_t r[64];
-        load_half(hf, r);
-        if (BLK == 64) {
-#pragma unroll
-          for (int u = 0; u < 64; ++u) mx[u & 7] = fmaxf(mx[u & 7], __uint_as_float(r[u]));
-          m = max8(mx) * a.scale_log2;
+      if (te >= 0 && te < T) {
+        // ---------------- epilogue of tile te: o = O / l as scaled float16
+        const int ob = te & 1, use = te >> 1;
+        const int bg = etd.x, ne = etd.w;
+        const int i = entry_row(eent), j = entry_slot(eent);
+        const bool valid = e < ne && static_cast<unsigned>(i) < static_cast<unsigned>(a.n_q) && j < a.nsl;
+        // the softmax's (m, l) are published with P (p_full); O follows P V
+        ok = __all_sync(0xFFFFFFFFu, mbar_wait(&p_full[ob], use & 1, a.err, SITE_BLK_O_FULL) &&
+                                         mbar_wait(&o_full[ob], use & 1, a.err, SITE_BLK_O_FULL));
+        if (!ok) break;
+        tc_fence_after();
+        float m, l;
+        if (C::ML_TMEM) {
+          uint32_t mlv[2];
+          tmem_ld2(tmem_base + lane_base + C::ML_COL + ob * 2, mlv);
+          tmem_wait_ld();
+          tmem_regs_ready(mlv);
+          m = __uint_as_float(mlv[0]);
+          l = __uint_as_float(mlv[1]);
+        } else {
+          const float2 ml = sML[ob * 128 + row];
+          m = ml.x;
+          l = ml.y;
         }
-        if (hf == BLK / 64 - 1) {   // all of S is in registers or consumed: free the buffer
-          tc_fence_before();
+        // (m, l) read: its slot may take the next tile of this parity
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&ml_empty[ob]);
+        // two passes over the row in halves of 64 columns: its largest
+        // magnitude, then the scaled float16 conversion
+        const uint32_t ocol = tmem_base + lane_base + C::O_COL + ob * D;
+        float am[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int hf = 0; hf < D / 64; ++hf) {
+          uint32_t r[64];
+          tmem_ld64(ocol + hf * 64, r);
+#pragma unroll
+          for (int u = 0; u < 64; ++u) am[u & 7] = fmaxf(am[u & 7], fabsf(__uint_as_float(r[u])));
+        }
+        const float amax = max8(am);
+        // the normalised row o = O / l, stored as float16 times 2^-e with the
+        // power of two 2^e chosen so the row's largest entry lands in
+        // [2^14, 2^15): 11 significant bits whatever the scale of V.  Every
+        // lane runs the (warp-collective) TMEM loads; only valid rows store.
+        const float inv_l = 1.f / l;
+        const float x = amax * inv_l;
+        int ex = x > 0.f ? static_cast<int>((__float_as_uint(x) >> 23) & 0xFFu) - 127 - 14 : 0;
+        ex = min(max(ex, -100), 100);
+        const float mul = inv_l * __uint_as_float(static_cast<uint32_t>(127 - ex) << 23);
+        const int64_t slot = ((static_cast<int64_t>(bg) * a.n_q + i) * a.nsl + j) * G + h;
+        // Coalesced stores: each warp passes its 32 rows through its own 32
+        // staging rows, 16-byte chunks XOR-swizzled by row against bank
+        // conflicts, then writes four whole 128-byte half-rows per instruction.
+        const int srow = lane >> 3, sch = lane & 7;   // store phase: row k*4 + srow, chunk sch
+#pragma unroll
+        for (int hf = 0; hf < D / 64; ++hf) {
+          uint32_t r[64];
+          tmem_ld64(ocol + hf * 64, r);
+          if (hf == D / 64 - 1) {   // all of O is in registers: free the buffer
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&o_empty[ob]);
+          }
+#pragma unroll
+          for (int q = 0; q < 8; ++q) {
+            uint32_t w[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+              const __half2 hv = __floats2half2_rn(__uint_as_float(r[q * 8 + 2 * u]) * mul,
+                                                   __uint_as_float(r[q * 8 + 2 * u + 1]) * mul);
+              w[u] = *reinterpret_cast<const uint32_t*>(&hv);
+            }
+            *reinterpret_cast<uint4*>(stage + lane * C::ROW + ((q ^ (lane & 7)) << 4)) = make_uint4(w[0], w[1], w[2], w[3]);
+          }
           __syncwarp();
-          if (lane == 0) mbar_arrive(&s_empty[sb]);
-        }
 #pragma unroll
-        for (int ch = 0; ch < 8; ++ch) {
-          uint32_t w[4];
-#pragma unroll
-          for (int u = 0; u < 4; ++u) {
-            const float p0 = fast_exp2(fmaf(__uint_as_float(r[ch * 8 + 2 * u]), a.scale_log2, -m));
-            const float p1 = fast_exp2(fmaf(__uint_as_float(r[ch * 8 + 2 * u + 1]), a.scale_log2, -m));
-            ls[2 * u] += p0;
-            ls[2 * u + 1] += p1;
-            w[u] = pack_bf16(p0, p1);
+          for (int k = 0; k < 8; ++k) {
+            const int rr = k * 4 + srow;   // the warp lane whose row this is
+            const int64_t rslot = __shfl_sync(0xFFFFFFFFu, slot, rr);
+            const bool rvalid = __shfl_sync(0xFFFFFFFFu, valid ? 1 : 0, rr) != 0;
+            const uint4 v = *reinterpret_cast<const uint4*>(stage + rr * C::ROW + ((sch ^ (rr & 7)) << 4));
+            if (rvalid) reinterpret_cast<uint4*>(a.partO + rslot * D + hf * 64)[sch] = v;
           }
-          *reinterpret_cast<uint4*>(prow + hf * C::P_HALF + row * C::ROW + ((ch ^ (row & 7)) << 4)) =
-              make_uint4(w[0], w[1], w[2], w[3]);
+          __syncwarp();
         }
+        if (valid) a.partL[slot] = make_float2(m + log2f(l), __uint_as_float(static_cast<uint32_t>(127 + ex) << 23));
       }
-      const float l = ((ls[0] + ls[1]) + (ls[2] + ls[3])) + ((ls[4] + ls[5]) + (ls[6] + ls[7]));
-      fence_async_smem();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&p_full[sb]);
-      // epilogue: O of this tile (the other group's softmax runs meanwhile)
-      ok = __all_sync(0xFFFFFFFFu, mbar_wait(&o_full[sb], use & 1, a.err, SITE_BLK_O_FULL));
-      if (!ok) break;
-      tc_fence_after();
-      // two passes over the row in halves of 64 columns: its largest
-      // magnitude, then the scaled float16 conversion
-      const uint32_t ocol = tmem_base + lane_base + C::O_COL + sb * D;
-      float am[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-      for (int hf = 0; hf < D / 64; ++hf) {
-        uint32_t r[64];
-        tmem_ld64(ocol + hf * 64, r);
-#pragma unroll
-        for (int u = 0; u < 64; ++u) am[u & 7] = fmaxf(am[u & 7], fabsf(__uint_as_float(r[u])));
-      }
-      const float amax = max8(am);
-      // the normalised row o = O / l, stored as float16 times 2^-e with the
-      // power of two 2^e chosen so the row's largest entry lands in
-      // [2^14, 2^15): 11 significant bits whatever the scale of V.  Every
-      // lane runs the (warp-collective) TMEM loads; only valid rows store.
-      const float inv_l = 1.f / l;
-      const float x = amax * inv_l;
-      int ex = x > 0.f ? static_cast<int>((__float_as_uint(x) >> 23) & 0xFFu) - 127 - 14 : 0;
-      ex = min(max(ex, -100), 100);
-      const float mul = inv_l * __uint_as_float(static_cast<uint32_t>(127 - ex) << 23);
-      const int64_t slot = ((static_cast<int64_t>(bg) * a.n_q + i) * a.nsl + j) * G + h;
-      // Coalesced stores: each warp passes its 32 rows through its own 32
-      // rows of this group's P tile (free once P V has run), 16-byte chunks
-      // XOR-swizzled by row against bank conflicts, then writes four whole
-      // 128-byte half-rows per instruction.
-      uint8_t* stage = sP + sb * C::P_BYTES + eq * 32 * C::ROW;
-      const int srow = lane >> 3, sch = lane & 7;   // store phase: row k*4 + srow, chunk sch
-#pragma unroll
-      for (int hf = 0; hf < D / 64; ++hf) {
-        uint32_t r[64];
-        tmem_ld64(ocol + hf * 64, r);
-#pragma unroll
-        for (int q = 0; q < 8; ++q) {
-          uint32_t w[4];
-#pragma unroll
-          for (int u = 0; u < 4; ++u) {
-            const __half2 hv = __floats2half2_rn(__uint_as_float(r[q * 8 + 2 * u]) * mul,
-                                                 __uint_as_float(r[q * 8 + 2 * u + 1]) * mul);
-            w[u] = *reinterpret_cast<const uint32_t*>(&hv);
-          }
-          *reinterpret_cast<uint4*>(stage + lane * C::ROW + ((q ^ (lane & 7)) << 4)) = make_uint4(w[0], w[1], w[2], w[3]);
-        }
-        __syncwarp();
-#pragma unroll
-        for (int k = 0; k < 8; ++k) {
-          const int rr = k * 4 + srow;   // the warp lane whose row this is
-          const int64_t rslot = __shfl_sync(0xFFFFFFFFu, slot, rr);
-          const bool rvalid = __shfl_sync(0xFFFFFFFFu, valid ? 1 : 0, rr) != 0;
-          const uint4 v = *reinterpret_cast<const uint4*>(stage + rr * C::ROW + ((sch ^ (rr & 7)) << 4));
-          if (rvalid) reinterpret_cast<uint4*>(a.partO + rslot * D + hf * 64)[sch] = v;
-        }
-        __syncwarp();
-      }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&o_empty[sb]);
-      if (valid) a.partL[slot] = make_float2(m + log2f(l), __uint_as_float(static_cast<uint32_t>(127 + ex) << 23));
     }
   } else {
     // ------------------------------------------------------------ Q gather
