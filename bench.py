@@ -189,10 +189,10 @@ def attended_keys(idx, w):
 
 
 def block_major_counts(idx, w):
-    """Slots of the block-major attention, by the kernels' rule: the used
-    block_idx entries (in range, larger than every earlier in-range entry of
-    the row) plus the window blocks no used entry selects.  Returns the number
-    of slots and of distinct (batch, kv-head, block) lists they fall in."""
+    """Selected slots of the block-major attention, by the kernels' rule:
+    the used block_idx entries (in range, larger than every earlier in-range
+    entry of the row).  Returns the number of slots and of distinct (batch,
+    kv-head, block) lists they fall in."""
     nb = w.n // w.block
     B = w.block
     pos = torch.arange(w.n_q, device=idx.device, dtype=torch.int64).view(1, -1, 1, 1) + w.q_offset
@@ -202,18 +202,11 @@ def block_major_counts(idx, w):
     run = torch.cummax(torch.where(inr, v, torch.full_like(v, -1)), dim=-1).values
     prev = torch.cat([torch.full_like(run[..., :1], -1), run[..., :-1]], dim=-1)
     valid = inr & (v > prev)
-    wt = (w.window - 1 + B - 1) // B + 1
-    lo = torch.clamp(pos - w.window + 1, min=0)
-    wb = lo // B + torch.arange(wt, device=idx.device).view(1, 1, 1, -1)          # [1, n, 1, wt]
-    in_win = wb <= pos // B
     sel = torch.where(valid, v, torch.full_like(v, -1))
-    covered = (sel.unsqueeze(-1) == wb.unsqueeze(-2)).any(-2)                    # [b, n, h, wt]
-    win = in_win & ~covered
-    n_entries = int(valid.sum().item()) + int(win.sum().item())
+    n_entries = int(valid.sum().item())
     bgi = (torch.arange(w.batch, device=idx.device).view(-1, 1, 1, 1) * w.h_kv
            + torch.arange(w.h_kv, device=idx.device).view(1, 1, -1, 1))
-    keys = torch.cat([(bgi * nb + sel)[valid], (bgi * nb + wb.expand_as(win))[win]])
-    n_blocks = int(torch.unique(keys).numel())
+    n_blocks = int(torch.unique((bgi * nb + sel)[valid]).numel())
     return n_entries, n_blocks
 
 
@@ -233,17 +226,23 @@ def algorithmic_work(w, idx):
     out = dict(summary_bytes=summary_bytes, route_flops=route_flops, attn_bytes=gathered + qo,
                gathered_bytes=gathered, attn_flops=attn_flops, mean_keys=float(S.float().mean().item()))
     if w.dtype == "bf16":
-        # block-major stages, per slot (a used selected block or an uncovered
-        # window block of a row): the tile kernel reads the G query rows and
-        # writes G partial rows + (log-sum-exp, scale), and reads each distinct
-        # key block's K, V once; the merge reads the slot partials and writes
-        # O and lse per row
+        # block-major stages.  Per selected slot (a used selected block of a
+        # row) the tile kernel reads the G query rows and writes G partial rows
+        # + (log-sum-exp, scale), and reads each distinct key block's K, V
+        # once.  Per window chunk of a row the window kernel reads the G query
+        # rows and writes G partial rows; it reads the window's K, V once.
+        # The merge reads all slot partials and writes O and lse per row.
         ne, nblk = block_major_counts(idx, w)
         items = w.batch * w.n_q * w.h_kv
+        nwc = (w.window + 255) // 256
+        nwin = items * nwc
+        wkeys = float(np.minimum(w.window, pos + 1).sum()) * w.batch * w.h_kv
         out["blocks_bytes"] = ne * G * (w.d * 2 * 2 + 8) + nblk * 2 * w.block * w.d * 2
         out["blocks_flops"] = 4.0 * ne * G * w.block * w.d
-        out["merge_bytes"] = items * (G * w.d * 2 + G * 4 + w.topk * 4) + ne * G * (w.d * 2 + 8)
-        out["plan_bytes"] = items * w.topk * 4 * 2 + ne * 4
+        out["window_bytes"] = nwin * G * (w.d * 2 * 2 + 8) + w.batch * w.n * w.h_kv * 2 * w.d * 2
+        out["window_flops"] = 4.0 * wkeys * G * w.d
+        out["merge_bytes"] = items * (G * w.d * 2 + G * 4 + w.topk * 4) + (ne + nwin) * G * (w.d * 2 + 8)
+        out["plan_bytes"] = items * w.topk * 4 * 2 + ne * 4 + items * 4
         out["n_entries"] = ne
         out["n_blocks"] = nblk
     return out
@@ -274,6 +273,7 @@ def run_ours(w, steps, warmup, ws, rank, with_e2e=True):
                   ("route", lambda: ssa.ssa_route_topk(p, Q, None, None, tab, idx, None, rws)),
                   ("attn_plan", lambda: ssa.ssa_attn_plan(p, idx, aws)),
                   ("attn_blocks", lambda: ssa.ssa_attn_blocks(p, Q, K, V, aws)),
+                  ("attn_window", lambda: ssa.ssa_attn_window(p, Q, K, V, aws)),
                   ("attn_merge", lambda: ssa.ssa_attn_merge(p, idx, O, lse, None, aws))]
     else:
         stages = [("summary", lambda: ssa.ssa_block_summary(p, K, None, None, tab)),
@@ -341,7 +341,8 @@ def run_ours(w, steps, warmup, ws, rank, with_e2e=True):
 
 
 KERNEL_NAMES = {"summary": "summary_diag_kernel", "route": "route_tiled_kernel", "attn_plan": "inv_*_kernel (6)",
-                "attn_blocks": "attn_block_kernel", "attn_merge": "attn_merge_kernel",
+                "attn_blocks": "attn_block_kernel", "attn_window": "attn_window_kernel",
+                "attn_merge": "attn_merge_kernel",
                 "attn_gather": "attn_bf16_kernel"}
 
 
@@ -379,6 +380,10 @@ def kernel_report(w, res, peaks, traffic):
                                         "algorithmic_flops": wk["blocks_flops"]}
         if b_tf / tc > rep["attn_blocks"]["frac"]:
             rep["attn_blocks"].update(bound="tensor", achieved=b_tf, unit="TFLOP/s", frac=b_tf / tc, peak=tc)
+        hbm_entry("attn_window", wk["window_bytes"])
+        w_tf = wk["window_flops"] / (ms["attn_window"] * 1e-3) / 1e12
+        rep["attn_window"]["tensor"] = {"achieved": w_tf, "unit": "TFLOP/s", "frac": w_tf / tc, "peak": tc,
+                                        "algorithmic_flops": wk["window_flops"]}
         hbm_entry("attn_merge", wk["merge_bytes"])
     # the pages' attention figure: algorithmic gathered K+V (+ q, o) bytes over
     # the whole attention time, whichever way it is evaluated

@@ -58,6 +58,7 @@ def _load():
         "ssa_attn_workspace_size": (sz, [P]),
         "ssa_attn_plan": (i32, [P, vp, vp, sz, vp]),
         "ssa_attn_blocks": (i32, [P, vp, vp, vp, vp, sz, vp]),
+        "ssa_attn_window": (i32, [P, vp, vp, vp, vp, sz, vp]),
         "ssa_attn_merge": (i32, [P, vp, vp, vp, vp, vp, sz, vp]),
         "ssa_sparse_attn": (i32, [P, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]),
         "ssa_workspace_size": (sz, [P]),
@@ -77,7 +78,7 @@ LIB_PATH = _LIB_PATH
 EXPORTED = ("ssa_status_string", "ssa_version", "ssa_launch_count", "ssa_device_error",
             "ssa_block_summary", "ssa_route_workspace_size", "ssa_route_topk", "ssa_route_topk_static",
             "ssa_attn_workspace_size", "ssa_sparse_attn", "ssa_attn_plan", "ssa_attn_blocks",
-            "ssa_attn_merge",
+            "ssa_attn_window", "ssa_attn_merge",
             "ssa_workspace_size", "ssa_forward", "ssa_hostio_buffer_size", "ssa_forward_hostio")
 
 
@@ -169,6 +170,11 @@ def ssa_attn_plan(p, block_idx, ws, stream=None):
 def ssa_attn_blocks(p, Q, K, V, ws, stream=None):
     _check(lib.ssa_attn_blocks(C.byref(p), _ptr(Q), _ptr(K), _ptr(V), _ptr(ws), _nbytes(ws), _stream(stream)),
            "ssa_attn_blocks")
+
+
+def ssa_attn_window(p, Q, K, V, ws, stream=None):
+    _check(lib.ssa_attn_window(C.byref(p), _ptr(Q), _ptr(K), _ptr(V), _ptr(ws), _nbytes(ws), _stream(stream)),
+           "ssa_attn_window")
 
 
 def ssa_attn_merge(p, block_idx, O, lse, bad_index_count, ws, stream=None):

@@ -32,15 +32,13 @@ namespace {
 // ------------------------------------------------------------------ inversion
 //
 // The rows of one (batch, kv-head) are cut into chunks of kPlanRows.  A CTA
-// per chunk counts its slots per key block in shared memory; a column scan
-// over the chunks then gives every (chunk, block) its place in the block's
-// entry list, so the scatter again needs only shared-memory atomics.
+// per chunk counts its selected slots per key block in shared memory; a
+// column scan over the chunks then gives every (chunk, block) its place in
+// the block's entry list, so the scatter again needs only shared-memory
+// atomics.  The counting pass also records each row's uncovered window
+// blocks for the sliding-window kernel.
 
 constexpr int kPlanThreads = 512;
-
-__device__ __forceinline__ int slot_block(const SlotSet& s, int j, int topk) {
-  return j < topk ? s.v : static_cast<int>(s.b0) + (j - topk);   // lane j's own entry for j < topk
-}
 
 __global__ void __launch_bounds__(kPlanThreads) inv_hist_kernel(const BlockPlan pl, const int32_t* __restrict__ idx) {
   extern __shared__ int32_t hist[];
@@ -53,8 +51,8 @@ __global__ void __launch_bounds__(kPlanThreads) inv_hist_kernel(const BlockPlan 
   for (int i = k * kPlanRows + warp; i < r1; i += nw) {
     const int v = lane < pl.topk ? __ldg(idx + ((static_cast<int64_t>(b) * pl.n_q + i) * pl.h_kv + g) * pl.topk + lane) : -1;
     const SlotSet s = row_slots(v, pl.topk, pl.q_offset + i, pl.nb, pl.block, pl.window);
-    if ((s.mask >> lane) & 1) atomicAdd(&hist[slot_block(s, lane, pl.topk)], 1);
-    if ((s.mask >> (lane + 32)) & 1) atomicAdd(&hist[static_cast<int>(s.b0) + lane + 32 - pl.topk], 1);
+    if ((s.mask >> lane) & 1) atomicAdd(&hist[s.v], 1);
+    if (lane == 0) pl.win[static_cast<int64_t>(bg) * pl.n_q + i] = s.win;
   }
   __syncthreads();
   int32_t* out = pl.chist + (static_cast<int64_t>(bg) * pl.nchunk + k) * pl.nb;
@@ -150,7 +148,7 @@ __global__ void __launch_bounds__(32) inv_scan_bg_kernel(const BlockPlan pl) {
   pl.tile_base[pl.bgs] = t;
 }
 
-// Same rows as inv_hist_kernel: every used slot becomes the entry
+// Same rows as inv_hist_kernel: every used selected slot becomes the entry
 // make_entry(query row, slot) in its block's list.
 __global__ void __launch_bounds__(kPlanThreads) inv_scatter_kernel(const BlockPlan pl, const int32_t* __restrict__ idx) {
   extern __shared__ int32_t cur[];
@@ -166,9 +164,7 @@ __global__ void __launch_bounds__(kPlanThreads) inv_scatter_kernel(const BlockPl
   for (int i = k * kPlanRows + warp; i < r1; i += nw) {
     const int v = lane < pl.topk ? __ldg(idx + ((static_cast<int64_t>(b) * pl.n_q + i) * pl.h_kv + g) * pl.topk + lane) : -1;
     const SlotSet s = row_slots(v, pl.topk, pl.q_offset + i, pl.nb, pl.block, pl.window);
-    if ((s.mask >> lane) & 1) pl.entries[atomicAdd(&cur[slot_block(s, lane, pl.topk)], 1)] = make_entry(i, lane);
-    if ((s.mask >> (lane + 32)) & 1)
-      pl.entries[atomicAdd(&cur[static_cast<int>(s.b0) + lane + 32 - pl.topk], 1)] = make_entry(i, lane + 32);
+    if ((s.mask >> lane) & 1) pl.entries[atomicAdd(&cur[s.v], 1)] = make_entry(i, lane);
   }
 }
 
@@ -188,27 +184,17 @@ __global__ void __launch_bounds__(256) inv_tiles_kernel(const BlockPlan pl) {
 }
 
 // Work estimate of each tile for the split over CTAs (units of a quarter of
-// an unmasked tile, from per-CTA cycle counts of the block kernel on B200):
-// a tile costs 4, masked_cost when a window slot in it is masked to part of
-// the block (the masked softmax path), plus block_start_cost for the first
-// tile of a block (loading K_c, V_c; with one K/V buffer the pipeline
-// drains).  The per-256-tile sums go to csum.
-__global__ void __launch_bounds__(256) inv_cost_kernel(const BlockPlan pl, int masked_cost, int block_start_cost) {
+// a tile, from per-CTA cycle counts of the block kernel on B200): a tile
+// costs 4, plus block_start_cost for the first tile of a block (loading
+// K_c, V_c; with one K/V buffer the pipeline drains).  The per-256-tile
+// sums go to csum.
+__global__ void __launch_bounds__(256) inv_cost_kernel(const BlockPlan pl, int block_start_cost) {
   const int t = blockIdx.x * blockDim.x + threadIdx.x;
   const int T = pl.tile_base[pl.bgs];
   int cost = 0;
   if (t < T) {
     const int4 td = pl.tiles[t];
-    bool masked = false;
-    const int64_t base = static_cast<int64_t>(td.y) * pl.block;
-    for (int e = 0; e < td.w && !masked; ++e) {
-      const int ent = pl.entries[td.z + e];
-      if (entry_slot(ent) >= pl.topk) {
-        const int64_t pos = pl.q_offset + entry_row(ent);
-        masked = (pos - pl.window + 1 > base) || (pos < base + pl.block - 1);
-      }
-    }
-    cost = masked ? masked_cost : 4;
+    cost = 4;
     if (t == 0) {
       cost += block_start_cost;
     } else {
@@ -585,49 +571,27 @@ __global__ void __maxnreg__((BlkCfg<G, BLK>::MAXREG))
     uint8_t* stage = sStg + grp * C::STG_BYTES + eq * 32 * C::ROW;
     auto tile_at = [&](int x) { return (x >= 0 && x < T) ? a.tiles[t0 + x] : none; };
     auto entry_of = [&](const int4& td) { return e < td.w ? __ldg(a.entries + td.z + e) : 0; };
-    // descriptors two tiles ahead and this thread's entry one tile ahead on
-    // both chains (softmax tiles grp + 2k, epilogue tiles grp - 1 + 2k)
-    int4 s_td = tile_at(grp), s_td2 = tile_at(grp + 2);
+    // the epilogue's tile descriptors two tiles ahead and this thread's entry
+    // one tile ahead (epilogue tiles grp - 1 + 2k; the softmax needs neither:
+    // every entry is a selected block, all of whose keys the row attends)
     int4 e_td = tile_at(grp - 1), e_td2 = tile_at(grp + 1);
-    int s_ent = entry_of(s_td), e_ent = entry_of(e_td);
+    int e_ent = entry_of(e_td);
     bool ok = true;
     for (int ts = grp; ok; ts += 2) {
       const int te = ts - 1;
       if (ts >= T && te >= T) break;
-      const int4 std_ = s_td, etd = e_td;
-      const int sent = s_ent, eent = e_ent;
-      s_td = s_td2; s_td2 = tile_at(ts + 4);
+      const int4 etd = e_td;
+      const int eent = e_ent;
       e_td = e_td2; e_td2 = tile_at(te + 4);
-      s_ent = entry_of(s_td);
       e_ent = entry_of(e_td);
       if (ts < T) {
         // ---------------- softmax of tile ts: P = 2^(s - m) in bf16 over S
         const int sb = ts & 1, use = ts >> 1;
-        const int i = entry_row(sent), j = entry_slot(sent);
-        const bool valid = e < std_.w && static_cast<unsigned>(i) < static_cast<unsigned>(a.n_q) && j < a.nsl;
-        // a window slot keeps the block's keys inside pos-W+1 .. pos
-        int klo = 0, khi = BLK - 1;
-        if (valid && j >= a.topk) {
-          const int64_t pos = a.q_offset + i, base = static_cast<int64_t>(std_.y) * BLK;
-          const int64_t lo = pos - a.window + 1;
-          klo = static_cast<int>(max(lo - base, static_cast<int64_t>(0)));
-          khi = static_cast<int>(min(pos - base, static_cast<int64_t>(BLK - 1)));
-        }
         ok = __all_sync(0xFFFFFFFFu, mbar_wait(&s_full[sb], use & 1, a.err, SITE_BLK_S_FULL));
         if (!ok) break;
         tc_fence_after();
         const uint32_t scol = tmem_base + lane_base + C::S_COL + sb * BLK;
-        // a half of S, loaded with the columns outside [klo, khi] set to -inf;
-        // most tiles hold no window slot, and their warps skip the masking
-        const bool any_mask = __any_sync(0xFFFFFFFFu, klo > 0 || khi < BLK - 1);
-        auto load_half = [&](int hf, uint32_t (&r)[64]) {
-          tmem_ld64(scol + hf * 64, r);
-          if (any_mask) {
-            const int lo = klo - hf * 64, hi = khi - hf * 64;
-#pragma unroll
-            for (int u = 0; u < 64; ++u) r[u] = (u >= lo && u <= hi) ? r[u] : 0xFF800000u;
-          }
-        };
+        auto load_half = [&](int hf, uint32_t (&r)[64]) { tmem_ld64(scol + hf * 64, r); };
         // maxima and sums in eight independent chains
         float mx[8] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY, -INFINITY, -INFINITY, -INFINITY, -INFINITY};
         float ls[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
@@ -689,7 +653,7 @@ __global__ void __maxnreg__((BlkCfg<G, BLK>::MAXREG))
         const int ob = te & 1, use = te >> 1;
         const int bg = etd.x, ne = etd.w;
         const int i = entry_row(eent), j = entry_slot(eent);
-        const bool valid = e < ne && static_cast<unsigned>(i) < static_cast<unsigned>(a.n_q) && j < a.nsl;
+        const bool valid = e < ne && static_cast<unsigned>(i) < static_cast<unsigned>(a.n_q) && j < a.topk;
         // the softmax's (m, l) are published with P (p_full); O follows P V
         ok = __all_sync(0xFFFFFFFFu, mbar_wait(&p_full[ob], use & 1, a.err, SITE_BLK_O_FULL) &&
                                          mbar_wait(&o_full[ob], use & 1, a.err, SITE_BLK_O_FULL));
@@ -895,8 +859,12 @@ __global__ void __launch_bounds__(256, (G == 8 ? 2 : (G == 4 ? 3 : 4))) attn_mer
   const int bg = static_cast<int>(item / a.n_q);
   const int b = bg / a.h_kv, g = bg % a.h_kv;
   const int v = lane < a.topk ? __ldg(a.idx + ((static_cast<int64_t>(b) * a.n_q + i) * a.h_kv + g) * a.topk + lane) : -1;
-  const SlotSet s = row_slots(v, a.topk, a.q_offset + i, a.nb, a.block, a.window);
+  SlotSet s = row_slots(v, a.topk, a.q_offset + i, a.nb, a.block, a.window);
   if (lane == 0 && a.bad && s.n_bad) atomicAdd(a.bad, s.n_bad);
+  // the window chunks (slots topk + c) that hold keys, one lane each
+  const uint32_t wch = __ballot_sync(0xFFFFFFFFu, lane < a.nsl - a.topk &&
+                                                      chunk_has_keys(s.win, a.q_offset + i, a.window, a.block, lane));
+  s.mask |= static_cast<uint64_t>(wch) << a.topk;
   const float2* pl = a.partL + item * a.nsl * G;
   const __half* po = a.partO + item * a.nsl * G * D;
   // per head: this lane's slots lane and lane + 32, their weights 2^(L-M) 2^e
@@ -997,7 +965,7 @@ cudaError_t launch_attn_merge(const ssa_params& p, const int32_t* block_idx, con
   a.bad = bad;
   a.n_q = p.n_q; a.h_q = p.h_q; a.h_kv = p.h_kv; a.nb = p.n_kv / p.block; a.block = p.block; a.topk = p.topk;
   a.window = p.window;
-  a.nsl = p.topk + window_slots(p.window, p.block);
+  a.nsl = p.topk + window_chunks(p.window);
   a.q_offset = p.q_offset;
   a.n_items = static_cast<int64_t>(p.batch) * p.h_kv * p.n_q;
   if (p.d != 128) return cudaErrorInvalidValue;
@@ -1042,8 +1010,8 @@ cudaError_t launch_block_plan(const ssa_params& p, const int32_t* block_idx, con
   const int n_chunks = (pl.max_tiles + 255) / 256;
   // 64-key blocks (two K/V buffers): every tile alike — equal counts were
   // measured as fast as any weighting; 128-key blocks (one K/V buffer): a
-  // masked tile costs about 1.75 tiles and a new block two
-  inv_cost_kernel<<<n_chunks, 256, 0, c.stream>>>(pl, p.block == 64 ? 4 : 7, p.block == 64 ? 0 : 8);
+  // new block costs two tiles
+  inv_cost_kernel<<<n_chunks, 256, 0, c.stream>>>(pl, p.block == 64 ? 0 : 8);
   note_launch();
   inv_split_kernel<<<1, 1024, 0, c.stream>>>(pl, n_chunks);
   note_launch();
@@ -1059,7 +1027,7 @@ cudaError_t launch_attn_block(const ssa_params& p, const BlockPlan& pl, const vo
   a.t_start = pl.t_start;
   a.entries = pl.entries;
   a.n_q = p.n_q; a.n_kv = p.n_kv; a.h_q = p.h_q; a.h_kv = p.h_kv; a.topk = p.topk; a.window = p.window;
-  a.nsl = p.topk + window_slots(p.window, p.block);
+  a.nsl = p.topk + window_chunks(p.window);
   a.q_offset = p.q_offset;
   a.scale_log2 = p.scale * 1.4426950408889634f;
   a.partO = static_cast<__half*>(partO);

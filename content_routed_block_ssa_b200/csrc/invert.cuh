@@ -6,14 +6,19 @@
 // and (ii)].  Slot j < topk is the row's j-th block_idx entry when it is
 // used: a fully visible block index larger than every earlier in-range entry
 // (so the used entries are ascending and distinct; anything else is skipped
-// and counted).  Slot topk + w is the w-th key block overlapping the window,
-// block lo/B + w, when no used entry selects it; it contributes only its keys
-// inside the window.  Every key of the set is thus in exactly one slot.
+// and counted).  Slot topk + s is chunk s of the window: its keys
+// pos-W+1 + 256 s .. min(pos, pos-W + 256 (s+1)) that lie in no used block.
+// Every key of the set is thus in exactly one slot.  Selected slots are
+// evaluated block by block (the block kernel), window chunks by a dense
+// sliding-window kernel.
 #pragma once
 
 #include <stdint.h>
 
 namespace ssa {
+
+// Keys per window chunk (one slot each).
+constexpr int kWinChunk = 256;
 
 // An inverted entry: the query row and the slot of that row.
 __device__ __forceinline__ int32_t make_entry(int row, int slot) { return (row << 6) | slot; }
@@ -25,16 +30,20 @@ __host__ __device__ constexpr int window_slots(int window, int block) {
   return (window - 1 + block - 1) / block + 1;
 }
 
+// Window chunks (slots) of a window of W keys.
+__host__ __device__ constexpr int window_chunks(int window) { return (window + kWinChunk - 1) / kWinChunk; }
+
 struct SlotSet {
-  uint64_t mask;   // bit j: slot j holds keys
+  uint64_t mask;   // bit j < topk: selected slot j holds keys
   int n_bad;       // block_idx entries skipped as invalid
   int v;           // this lane's block_idx entry (-1 past topk)
   int64_t lo;      // first window key
   int64_t b0;      // first window block
+  uint32_t win;    // bit w: window block b0 + w is in no used entry
 };
 
 // Warp-collective: lane l < topk passes entry l of the row (any value past
-// topk is ignored).  topk + window_slots(window, block) <= 64.
+// topk is ignored).  window_slots(window, block) <= 32.
 __device__ __forceinline__ SlotSet row_slots(int v_in, int topk, int64_t pos, int nb, int block, int window) {
   const int lane = threadIdx.x & 31;
   const int v = lane < topk ? v_in : -1;
@@ -61,8 +70,23 @@ __device__ __forceinline__ SlotSet row_slots(int v_in, int topk, int64_t pos, in
   const int64_t w = static_cast<int64_t>(v) - s.b0;
   const uint32_t cov = __reduce_or_sync(0xFFFFFFFFu, (valid && w >= 0 && w < 32) ? (1u << w) : 0u);
   const uint32_t all = nwb >= 32 ? 0xFFFFFFFFu : ((1u << nwb) - 1u);
-  s.mask |= static_cast<uint64_t>(all & ~cov) << topk;
+  s.win = all & ~cov;
   return s;
+}
+
+// Whether window chunk s of the row at pos holds keys: some block it
+// overlaps is uncovered.  win as in SlotSet (blocks b0 + w).
+__host__ __device__ inline bool chunk_has_keys(uint32_t win, int64_t pos, int window, int block, int s) {
+  const int64_t w0 = pos - window + 1;                 // unclamped window start
+  int64_t klo = w0 + static_cast<int64_t>(s) * kWinChunk;
+  int64_t khi = w0 + static_cast<int64_t>(s + 1) * kWinChunk - 1;
+  if (khi > pos) khi = pos;
+  if (klo < 0) klo = 0;
+  if (khi < klo) return false;
+  const int64_t b0 = (w0 > 0 ? w0 : 0) / block;
+  const int f = static_cast<int>(klo / block - b0), l = static_cast<int>(khi / block - b0);
+  const uint32_t span = (l - f + 1 >= 32) ? 0xFFFFFFFFu : ((1u << (l - f + 1)) - 1u);
+  return ((win >> f) & span) != 0;
 }
 
 }  // namespace ssa

@@ -64,6 +64,7 @@ struct BlockPlan {
   int32_t *ent_base, *tile_base;         // [bgs + 1]
   int32_t* entries;                      // make_entry(query row, slot)
   int4* tiles;                           // {bg, block, first entry, entries}
+  uint32_t* win;                         // [bgs * n_q] uncovered window blocks of each row
   // balanced split of the tiles over the block kernel's CTAs
   int32_t max_tiles, grid;               // tile capacity; CTAs (<= kMaxBlockGrid)
   uint8_t* tcost;                        // [max_tiles] estimated cost of each tile
@@ -85,6 +86,14 @@ cudaError_t launch_block_plan(const ssa_params& p, const int32_t* block_idx, con
 cudaError_t launch_attn_block(const ssa_params& p, const BlockPlan& pl, const void* Q,
                               const CUtensorMap& tmK, const CUtensorMap& tmV, const CUtensorMap& tmQ,
                               void* partO, void* partL, const LaunchCtx& c);
+
+// The causal window, densely: one partial per (query, head, window chunk)
+// at slot topk + chunk, same format as the block tiles' partials.  tmQ: Q as
+// [b * n_q, h_q, d], 128-byte-swizzled boxes of 64 dims x G heads x 128/G
+// query rows; tmK, tmV as for the block tiles.
+cudaError_t launch_attn_window(const ssa_params& p, const BlockPlan& pl, const CUtensorMap& tmQ,
+                               const CUtensorMap& tmK, const CUtensorMap& tmV, void* partO, void* partL,
+                               const LaunchCtx& c);
 
 // Per (query, kv-head): the softmax merge of the slot partials into O, lse.
 cudaError_t launch_attn_merge(const ssa_params& p, const int32_t* block_idx, const void* partO, const void* partL,

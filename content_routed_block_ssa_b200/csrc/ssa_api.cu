@@ -163,7 +163,7 @@ bool use_block_attn(const ssa_params& p) {
 
 struct AttnLayout {
   size_t chist, count, blk_off, tile_off, bg_ents, bg_tiles, ent_base, tile_base, entries, tiles, tcost, csum,
-      t_start, part_o, part_l, total;
+      t_start, win, part_o, part_l, total;
   int nchunk, nsl;
   size_t max_tiles;
 };
@@ -176,7 +176,7 @@ AttnLayout attn_layout(const ssa_params& p) {
   const size_t G = static_cast<size_t>(p.h_q / p.h_kv);
   const size_t qpt = 128 / G;
   L.nchunk = (p.n_q + ssa::kPlanRows - 1) / ssa::kPlanRows;
-  L.nsl = p.topk + ssa::window_slots(p.window, p.block);
+  L.nsl = p.topk + ssa::window_chunks(p.window);
   const size_t items = bgs * p.n_q;
   const size_t sel = items * L.nsl;                       // entries, at most
   const size_t max_tiles = (sel + qpt - 1) / qpt + bgs * nb;
@@ -195,6 +195,7 @@ AttnLayout attn_layout(const ssa_params& p) {
   L.tcost = off; off += round_up(max_tiles);
   L.csum = off; off += round_up((max_tiles + 255) / 256 * 4);
   L.t_start = off; off += round_up((ssa::kMaxBlockGrid + 1) * 4);
+  L.win = off; off += round_up(items * 4);
   L.part_o = off; off += round_up(sel * G * p.d * 2);
   L.part_l = off; off += round_up(sel * G * 8);
   L.total = off;
@@ -256,6 +257,21 @@ bool encode_q_heads(CUtensorMap* m, const void* base, const ssa_params& p) {
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// 3D bf16 map of Q viewed as [b*n_q, h_q, d]; 128-byte-swizzled boxes of
+// 64 dims x `heads` heads x `rows` query rows.
+bool encode_q_tile(CUtensorMap* m, const void* base, const ssa_params& p, int heads, int rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[3] = {static_cast<cuuint64_t>(p.d), static_cast<cuuint64_t>(p.h_q),
+                              static_cast<cuuint64_t>(p.batch) * p.n_q};
+  const cuuint64_t strides[2] = {static_cast<cuuint64_t>(p.d) * 2, static_cast<cuuint64_t>(p.h_q) * p.d * 2};
+  const cuuint32_t box[3] = {64, static_cast<cuuint32_t>(heads), static_cast<cuuint32_t>(rows)};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 ssa_status do_summary(const ssa_params& p, const void* K, float* mu, float* sigma, void* table,
                       const LaunchCtx& c) {
   if (p.batch == 0 || p.n_kv == 0) return SSA_OK;
@@ -309,6 +325,7 @@ ssa::BlockPlan block_plan(const ssa_params& p, const AttnLayout& L, uint8_t* w) 
   pl.tile_base = reinterpret_cast<int32_t*>(w + L.tile_base);
   pl.entries = reinterpret_cast<int32_t*>(w + L.entries);
   pl.tiles = reinterpret_cast<int4*>(w + L.tiles);
+  pl.win = reinterpret_cast<uint32_t*>(w + L.win);
   pl.max_tiles = static_cast<int32_t>(L.max_tiles);
   pl.grid = 0;   // set by the caller from the device's SM count
   pl.tcost = w + L.tcost;
@@ -319,6 +336,7 @@ ssa::BlockPlan block_plan(const ssa_params& p, const AttnLayout& L, uint8_t* w) 
 
 struct AttnMaps {
   CUtensorMap K, V, Q, Qh;   // Q: unswizzled G-row boxes (gather path); Qh: 8-head boxes (G = 8 tiles)
+  CUtensorMap Qw;            // G heads x 128/G query rows (window tiles)
 };
 
 bool encode_attn_maps(AttnMaps& m, const ssa_params& p, const void* Q, const void* K, const void* V) {
@@ -326,6 +344,7 @@ bool encode_attn_maps(AttnMaps& m, const ssa_params& p, const void* Q, const voi
   if (!encode_kv(&m.K, K, p) || !encode_kv(&m.V, V, p) ||
       !encode_rows(&m.Q, Q, p.d, static_cast<uint64_t>(p.batch) * p.n_q * p.h_q, G))
     return false;
+  if (p.d == 128 && (G == 2 || G == 4 || G == 8) && !encode_q_tile(&m.Qw, Q, p, G, 128 / G)) return false;
   if (G == 8 && p.d == 128) return encode_q_heads(&m.Qh, Q, p);
   m.Qh = m.Q;
   return true;
@@ -347,6 +366,13 @@ ssa_status attn_stage_blocks(const ssa_params& p, const void* Q, const AttnMaps&
   return from_cuda(ssa::launch_attn_block(p, pl, Q, m.K, m.V, m.Qh, w + L.part_o, w + L.part_l, c));
 }
 
+ssa_status attn_stage_window(const ssa_params& p, const AttnMaps& m, uint8_t* w, const LaunchCtx& c) {
+  const AttnLayout L = attn_layout(p);
+  ssa::BlockPlan pl = block_plan(p, L, w);
+  pl.grid = c.sm_count;
+  return from_cuda(ssa::launch_attn_window(p, pl, m.Qw, m.K, m.V, w + L.part_o, w + L.part_l, c));
+}
+
 ssa_status attn_stage_merge(const ssa_params& p, const int32_t* idx, void* O, float* lse, int32_t* bad,
                             const uint8_t* w, const LaunchCtx& c) {
   const AttnLayout L = attn_layout(p);
@@ -366,6 +392,7 @@ ssa_status do_attn(const ssa_params& p, const void* Q, const void* K, const void
   uint8_t* w = static_cast<uint8_t*>(ws);
   ssa_status st = attn_stage_plan(p, idx, w, c);
   if (st == SSA_OK) st = attn_stage_blocks(p, Q, m, w, c);
+  if (st == SSA_OK) st = attn_stage_window(p, m, w, c);
   if (st == SSA_OK) st = attn_stage_merge(p, idx, O, lse, bad, w, c);
   return st;
 }
@@ -540,6 +567,18 @@ ssa_status ssa_attn_blocks(const ssa_params* pp, const void* Q, const void* K, c
   AttnMaps m;
   if (!encode_attn_maps(m, *pp, Q, K, V)) return SSA_ERR_CUDA;
   return attn_stage_blocks(*pp, Q, m, static_cast<uint8_t*>(ws), c);
+}
+
+ssa_status ssa_attn_window(const ssa_params* pp, const void* Q, const void* K, const void* V, void* ws,
+                           size_t ws_bytes, void* stream) {
+  ssa_status st = check_stage(pp, ws, ws_bytes);
+  if (st != SSA_OK || is_empty(*pp)) return st;
+  if (!Q || !K || !V || !aligned16(Q) || !aligned16(K) || !aligned16(V)) return SSA_ERR_INVALID_ARG;
+  LaunchCtx c;
+  if ((st = make_ctx(stream, c)) != SSA_OK) return st;
+  AttnMaps m;
+  if (!encode_attn_maps(m, *pp, Q, K, V)) return SSA_ERR_CUDA;
+  return attn_stage_window(*pp, m, static_cast<uint8_t*>(ws), c);
 }
 
 ssa_status ssa_attn_merge(const ssa_params* pp, const int32_t* block_idx, void* O, float* lse,

@@ -3,5 +3,5 @@ from ._lib import *  # noqa: F401,F403
 from ._lib import (SSAError, lib, make_params, ssa_block_summary, ssa_device_error, ssa_forward,  # noqa: F401
                    ssa_forward_hostio, ssa_hostio_buffer_size, ssa_launch_count, ssa_params,
                    ssa_route_topk, ssa_route_topk_static, ssa_route_workspace_size, ssa_sparse_attn,
-                   ssa_attn_workspace_size, ssa_attn_plan, ssa_attn_blocks, ssa_attn_merge, ssa_workspace_size,
-                   status_string, summary_shapes, idx_shape, byte_buffer, EXPORTED, LIB_PATH)
+                   ssa_attn_workspace_size, ssa_attn_plan, ssa_attn_blocks, ssa_attn_window, ssa_attn_merge,
+                   ssa_workspace_size, status_string, summary_shapes, idx_shape, byte_buffer, EXPORTED, LIB_PATH)

@@ -203,29 +203,38 @@ SSA_API ssa_status ssa_sparse_attn(const ssa_params* p, const void* Q, const voi
                                    int32_t* bad_index_count, void* ws, size_t ws_bytes, void* stream);
 
 /*
- * The block-major evaluation of ssa_sparse_attn as three calls, for callers
+ * The block-major evaluation of ssa_sparse_attn as four calls, for callers
  * that schedule or time the stages themselves.  Made in this order on one
  * stream with one workspace (ssa_attn_workspace_size(p) bytes, 16-byte
  * aligned; its contents are private to the library and live from the plan
  * call to the merge call), they give exactly the bytes ssa_sparse_attn gives
- * with that workspace.
- *   ssa_attn_plan    inverts block_idx: the slots of every row (used
- *                    selected blocks, then window blocks not selected) as
- *                    per-(batch, kv-head, key block) lists, in tiles of
- *                    128 / G queries;
+ * with that workspace.  A row's keys fall in "slots": each used selected
+ * block, and each 256-key chunk of the window (pos-W+1 .. pos) minus the
+ * keys of its used selected blocks.
+ *   ssa_attn_plan    inverts block_idx: the used selected blocks of every
+ *                    row as per-(batch, kv-head, key block) lists, in tiles
+ *                    of 128 / G queries, and each row's window blocks that
+ *                    no used entry selects;
  *   ssa_attn_blocks  per tile, S = Q_tile K_c^T and O = P V_c on the tensor
- *                    cores, window slots masked to pos-W+1 .. pos; writes each
- *                    slot's normalised partial output and base-2
- *                    log-sum-exp into the workspace;
+ *                    cores; writes each selected slot's normalised partial
+ *                    output and base-2 log-sum-exp into the workspace;
+ *   ssa_attn_window  per run of 128 / G consecutive queries and window
+ *                    chunk, the same over the chunk's keys (dense tensor-core
+ *                    tiles masked per row); writes the window slots' partials;
  *   ssa_attn_merge   per (query, kv-head): the softmax merge of the row's
  *                    slot partials into O and lse; counts skipped block_idx
  *                    entries as ssa_sparse_attn does.
+ * ssa_attn_blocks and ssa_attn_window write disjoint parts of the workspace
+ * and may run in either order (or on two streams ordered after the plan and
+ * before the merge).
  * Problems that do not qualify return SSA_ERR_UNSUPPORTED, a missing or
  * short workspace SSA_ERR_WORKSPACE; both before any launch.
  */
 SSA_API ssa_status ssa_attn_plan(const ssa_params* p, const int32_t* block_idx, void* ws, size_t ws_bytes,
                                  void* stream);
 SSA_API ssa_status ssa_attn_blocks(const ssa_params* p, const void* Q, const void* K, const void* V,
+                                   void* ws, size_t ws_bytes, void* stream);
+SSA_API ssa_status ssa_attn_window(const ssa_params* p, const void* Q, const void* K, const void* V,
                                    void* ws, size_t ws_bytes, void* stream);
 SSA_API ssa_status ssa_attn_merge(const ssa_params* p, const int32_t* block_idx, void* O, float* lse,
                                   int32_t* bad_index_count, const void* ws, size_t ws_bytes, void* stream);

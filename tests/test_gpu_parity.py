@@ -400,6 +400,7 @@ def test_block_major_stages_equal_single_call():
     b2 = torch.zeros(1, dtype=torch.int32, device="cuda")
     ssa.ssa_attn_plan(p, idx, ws)
     ssa.ssa_attn_blocks(p, Q, K, V, ws)
+    ssa.ssa_attn_window(p, Q, K, V, ws)
     ssa.ssa_attn_merge(p, idx, O2, l2, b2, ws)
     check_no_device_error()
     assert torch.equal(O1, O2) and torch.equal(l1, l2) and int(b2.item()) == int(b1.item()) == 0
