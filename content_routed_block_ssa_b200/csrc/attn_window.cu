@@ -34,15 +34,16 @@ struct WinCfg {
   static constexpr int K_BLK = 64 * ROW;             // one 64-key block, one 64-dim half
   static constexpr int K_HALF = KB * K_BLK;          // half h of all K blocks, block kb at kb * K_BLK
   static constexpr int V_SLOT = 2 * K_BLK;           // one V block, both halves (LBO = K_BLK)
-  static constexpr int NBAR = 12;
+  static constexpr int NBAR = 14;
   static constexpr int XCH = 2 * 2 * 128 * 4;         // two buffers of one float per (group, row)
   // bytes used from the 1024-byte-aligned base; the allocation adds what
   // alignment may cost, up to the per-block limit (checked in the kernel)
   static constexpr int USED = 2 * Q_HALF + 2 * K_HALF + KB * V_SLOT + XCH + NBAR * 8 + 16;
   static constexpr int SMEM = USED + 1024 < 232448 ? USED + 1024 : 232448;
-  static constexpr int THREADS = 320;                // producer, MMA, 2 x 4 softmax / epilogue warps
+  static constexpr int THREADS = 448;                // producer, MMA, 2 x 4 softmax, 4 epilogue warps
   static constexpr int S_COL = 0;                    // TMEM: S (KB * 64 columns), then O
   static constexpr int O_COL = KB * 64;
+  static constexpr int ML_COL = S_COL + 32;          // (m, l): in the first block's S, past its P
   static_assert(O_COL + D <= 512, "tensor memory");
   static_assert(USED <= 232448, "shared memory");
 };
@@ -99,6 +100,13 @@ __device__ __forceinline__ uint64_t win_desc_mn(uint32_t saddr, uint32_t lbo, ui
   return d;
 }
 
+__device__ __forceinline__ void win_ld32(uint32_t taddr, uint32_t (&r)[32]) {
+#pragma unroll
+  for (int q = 0; q < 2; ++q) tmem_ld16(taddr + q * 16, *reinterpret_cast<uint32_t(*)[16]>(&r[q * 16]));
+  tmem_wait_ld();
+  tmem_regs_ready(r);
+}
+
 __device__ __forceinline__ void win_ld64(uint32_t taddr, uint32_t (&r)[64]) {
 #pragma unroll
   for (int q = 0; q < 4; ++q) tmem_ld16(taddr + q * 16, *reinterpret_cast<uint32_t(*)[16]>(&r[q * 16]));
@@ -107,14 +115,14 @@ __device__ __forceinline__ void win_ld64(uint32_t taddr, uint32_t (&r)[64]) {
 }
 
 // Warp roles: 0 TMA producer (Q, then K, then V of each tile), 1 MMA issuer
-// and TMEM owner, 2..9 softmax and epilogue in two groups of four warps
-// (one tensor-core row = one (query, head) pair per thread of each group):
-// group g takes half of the tile's 64-key blocks and half of O's columns,
-// and the groups swap per-row partials (maximum, sum, largest |o|) through
-// shared memory.  One tile in flight: the next tile's Q and K load during
-// this tile's softmax, its S runs during this tile's epilogue; the epilogue
-// stages its stores through the first two V slots, so the next tile's V
-// loads after it.
+// and TMEM owner, 2..9 softmax in two groups of four warps (one tensor-core
+// row = one (query, head) pair per thread of each group; group g takes half
+// of the tile's 64-key blocks, and the groups swap each row's maximum and
+// sum through shared memory), 10..13 epilogue.  The epilogue of a tile runs
+// while the softmax works on the next: the next tile's Q and K load during
+// this tile's softmax, its S runs once this tile's P V has read P (which
+// lies over S); the epilogue stages its stores through the first V slot, so
+// the next tile's V loads after it.
 template <int G>
 __global__ void __launch_bounds__(WinCfg<G>::THREADS, 1)
     attn_window_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
@@ -139,17 +147,21 @@ __global__ void __launch_bounds__(WinCfg<G>::THREADS, 1)
   uint64_t* s_full = bars + 4;
   uint64_t* p_full = bars + 5;
   uint64_t* o_full = bars + 6;      // P V done
-  uint64_t* epi_done = bars + 7;    // O read and the staging rows written out
-  uint64_t* o_empty = epi_done;     // (the epilogue reads O before it stages)
-  uint64_t* xbar = bars + 8;        // [3] both groups' row partials of a tile written
-  uint64_t* mma_done = bars + 11;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 12);
+  uint64_t* o_empty = bars + 7;     // the epilogue has read O
+  uint64_t* stg_done = bars + 8;    // the epilogue's staging rows are written out (V slot 0 free)
+  uint64_t* xbar = bars + 9;        // [2] both softmax groups' row partials of a tile written
+  uint64_t* ml_full = bars + 11;    // (m, l) of the tile written to TMEM
+  uint64_t* ml_read = bars + 12;    // ... and read by the epilogue (its columns may take S)
+  uint64_t* mma_done = bars + 13;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 14);
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1); mbar_init(q_empty, 1); mbar_init(k_full, 1); mbar_init(v_full, 1);
-    mbar_init(s_full, 1); mbar_init(p_full, 8); mbar_init(o_full, 1); mbar_init(epi_done, 8);
-    for (int k = 0; k < 3; ++k) mbar_init(&xbar[k], 8);
+    mbar_init(s_full, 1); mbar_init(p_full, 8); mbar_init(o_full, 1); mbar_init(o_empty, 4);
+    mbar_init(stg_done, 4);
+    mbar_init(&xbar[0], 8); mbar_init(&xbar[1], 8);
+    mbar_init(ml_full, 4); mbar_init(ml_read, 4);
     mbar_init(mma_done, 1);
     fence_barrier_init();
     tma_prefetch_desc(&tmQ);
@@ -189,7 +201,7 @@ __global__ void __launch_bounds__(WinCfg<G>::THREADS, 1)
             tma_load_3d(sK + hf * C::K_HALF + kb * C::K_BLK, &tmK, k_full, hf * 64, g, kz + kb * 64);
         ++uqk;
         // V once the previous tile's epilogue has left the staging rows
-        if (!mbar_wait(epi_done, par, a.err, SITE_WIN_PRODUCER)) { ok = false; break; }
+        if (!mbar_wait(stg_done, par, a.err, SITE_WIN_PRODUCER)) { ok = false; break; }
         mbar_arrive_expect_tx(v_full, static_cast<uint32_t>(w.nkb) * C::V_SLOT);
         for (int kb = 0; kb < w.nkb; ++kb)
 #pragma unroll
@@ -218,9 +230,10 @@ __global__ void __launch_bounds__(WinCfg<G>::THREADS, 1)
         const WinTile w = win_tile<G>(a, t);
         if (w.kb0 < 0) continue;
         const uint32_t par = u & 1;
-        // S over the span: the previous tile's P V has read its P (over S)
-        if (!mbar_wait(o_full, par ^ 1, a.err, SITE_WIN_MMA) || !mbar_wait(q_full, par, a.err, SITE_WIN_MMA) ||
-            !mbar_wait(k_full, par, a.err, SITE_WIN_MMA))
+        // S over the span: the previous tile's P V has read its P and the
+        // epilogue its (m, l), both over S
+        if (!mbar_wait(o_full, par ^ 1, a.err, SITE_WIN_MMA) || !mbar_wait(ml_read, par ^ 1, a.err, SITE_WIN_MMA) ||
+            !mbar_wait(q_full, par, a.err, SITE_WIN_MMA) || !mbar_wait(k_full, par, a.err, SITE_WIN_MMA))
           break;
         tc_fence_after();
         for (int n0 = 0; n0 < w.nkb; n0 += 4) {
@@ -256,16 +269,14 @@ __global__ void __launch_bounds__(WinCfg<G>::THREADS, 1)
       const uint64_t tq = global_timer_ns();
       while (!mbar_try_wait(mma_done, 0) && global_timer_ns() - tq < kWaitLimitNs) {}
     }
-  } else {
-    // ------------------------------------------------------------ softmax + epilogue
-    const int gs = (warp - 2) >> 2;   // this group's blocks and O columns
+  } else if (warp < 10) {
+    // ------------------------------------------------------------ softmax
+    const int gs = (warp - 2) >> 2;   // this group's half of the tile's blocks
     const int eq = warp & 3;
     const int row = eq * 32 + lane;
-    const int e = row / G, h = row % G;
+    const int e = row / G;
     const uint32_t lane_base = static_cast<uint32_t>(eq * 32) << 16;
     const uint32_t scol = tmem_base + lane_base + C::S_COL;
-    const uint32_t ocol = tmem_base + lane_base + C::O_COL + gs * 64;
-    uint8_t* stage = sV + gs * C::V_SLOT + eq * 32 * C::ROW;   // this warp's 32 staging rows
     // publish this thread's row partial, then read the other group's once
     // both groups have published (bounded waits; the phase is the tile
     // count).  Exchanges alternate between two buffers: a buffer is written
@@ -290,39 +301,52 @@ __global__ void __launch_bounds__(WinCfg<G>::THREADS, 1)
       const int kb_lo = gs ? kbh : 0, kb_hi = gs ? w.nkb : kbh;
       const int i = w.q0 + e;
       const bool valid = i < a.n_q;
-      // this row's keys: its chunk of the window, minus the blocks it selected
-      const int64_t pos = a.q_offset + i;
-      const int64_t w0 = pos - a.window + 1;
-      int64_t klo = w0 + static_cast<int64_t>(w.s) * kWinChunk, khi = w0 + static_cast<int64_t>(w.s + 1) * kWinChunk - 1;
-      if (klo < 0) klo = 0;
-      if (khi > pos) khi = pos;
+      // this row's keys: its chunk of the window, minus the blocks it
+      // selected, as offsets from the span's first key (key positions are
+      // below 2^31: every key index fits the 32-bit TMA coordinates)
+      const int pos = static_cast<int>(a.q_offset) + i;
+      const int w0 = pos - a.window + 1;
+      const int span0 = w.kb0 * 64;
+      int klo = max(w0 + w.s * kWinChunk, 0), khi = min(w0 + (w.s + 1) * kWinChunk - 1, pos);
       if (!valid) { klo = 1; khi = 0; }
-      const int64_t b0 = (w0 > 0 ? w0 : 0) / a.block;
+      klo -= span0;
+      khi -= span0;
+      const int b0 = max(w0, 0) / a.block;
       const uint32_t win = valid ? __ldg(a.win + static_cast<int64_t>(w.bg) * a.n_q + i) : 0u;
       // columns [c_lo, c_hi] of span block kb hold this row's keys (empty
       // when c_lo > c_hi); a selected block contributes none
       auto cols = [&](int kb, int& c_lo, int& c_hi) {
-        const int64_t kbase = static_cast<int64_t>(w.kb0 + kb) * 64;
-        const int64_t wb = kbase / a.block - b0;
+        const int wb = (span0 + kb * 64) / a.block - b0;
         const bool open = wb >= 0 && wb < 32 && ((win >> wb) & 1u);
-        c_lo = static_cast<int>(max(klo - kbase, static_cast<int64_t>(0)));
-        c_hi = static_cast<int>(min(khi - kbase, static_cast<int64_t>(63)));
+        c_lo = max(klo - kb * 64, 0);
+        c_hi = min(khi - kb * 64, 63);
         if (!open) { c_lo = 1; c_hi = 0; }
       };
       ok = __all_sync(0xFFFFFFFFu, mbar_wait(s_full, par, a.err, SITE_WIN_SOFTMAX));
       if (!ok) break;
       tc_fence_after();
-      // the row maximum over its keys (this group's blocks, then both)
+      // the row maximum over its keys (this group's blocks, then both);
+      // blocks whole for every row of the warp skip the masking
       float mx[8] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY, -INFINITY, -INFINITY, -INFINITY, -INFINITY};
       for (int kb = kb_lo; kb < kb_hi; ++kb) {
         int c_lo, c_hi;
         cols(kb, c_lo, c_hi);
         if (!__any_sync(0xFFFFFFFFu, c_lo <= c_hi)) continue;   // warp-uniform
-        uint32_t r[64];
-        win_ld64(scol + kb * 64, r);
+        const bool whole = __all_sync(0xFFFFFFFFu, c_lo == 0 && c_hi == 63);
+#pragma unroll 1
+        for (int qq = 0; qq < 2; ++qq) {
+          uint32_t r[32];
+          win_ld32(scol + kb * 64 + qq * 32, r);
+          if (whole) {
 #pragma unroll
-        for (int u2 = 0; u2 < 64; ++u2)
-          if (u2 >= c_lo && u2 <= c_hi) mx[u2 & 7] = fmaxf(mx[u2 & 7], __uint_as_float(r[u2]));
+            for (int u2 = 0; u2 < 32; ++u2) mx[u2 & 7] = fmaxf(mx[u2 & 7], __uint_as_float(r[u2]));
+          } else {
+            const int lo = c_lo - qq * 32, hi = c_hi - qq * 32;
+#pragma unroll
+            for (int u2 = 0; u2 < 32; ++u2)
+              if (u2 >= lo && u2 <= hi) mx[u2 & 7] = fmaxf(mx[u2 & 7], __uint_as_float(r[u2]));
+          }
+        }
       }
       float m = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])), fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
       m = fmaxf(m, swap(0, m, par, ok));
@@ -335,22 +359,37 @@ __global__ void __launch_bounds__(WinCfg<G>::THREADS, 1)
         int c_lo, c_hi;
         cols(kb, c_lo, c_hi);
         const bool any = __any_sync(0xFFFFFFFFu, c_lo <= c_hi);
-        uint32_t r[64];
-        if (any) win_ld64(scol + kb * 64, r);
-#pragma unroll
+        const bool whole = __all_sync(0xFFFFFFFFu, c_lo == 0 && c_hi == 63);
+        // 32 keys at a time: their S columns in, 16 columns of P out
+#pragma unroll 1
         for (int qq = 0; qq < 2; ++qq) {
-          uint32_t pw[16];
+          uint32_t r[32], pw[16];
+          if (any) win_ld32(scol + kb * 64 + qq * 32, r);
+          if (whole) {
 #pragma unroll
-          for (int u2 = 0; u2 < 16; ++u2) {
-            const int c = qq * 32 + 2 * u2;
-            float p0 = 0.f, p1 = 0.f;
-            if (any) {
-              p0 = (c >= c_lo && c <= c_hi) ? fast_exp2(fmaf(__uint_as_float(r[c]), a.scale_log2, -m)) : 0.f;
-              p1 = (c + 1 >= c_lo && c + 1 <= c_hi) ? fast_exp2(fmaf(__uint_as_float(r[c + 1]), a.scale_log2, -m)) : 0.f;
+            for (int u2 = 0; u2 < 16; ++u2) {
+              const float p0 = fast_exp2(fmaf(__uint_as_float(r[2 * u2]), a.scale_log2, -m));
+              const float p1 = fast_exp2(fmaf(__uint_as_float(r[2 * u2 + 1]), a.scale_log2, -m));
+              ls[(2 * u2) & 7] += p0;
+              ls[(2 * u2 + 1) & 7] += p1;
+              pw[u2] = pack_bf16(p0, p1);
             }
-            ls[c & 7] += p0;
-            ls[(c + 1) & 7] += p1;
-            pw[u2] = pack_bf16(p0, p1);
+          } else {
+            const int lo = c_lo - qq * 32, hi = c_hi - qq * 32;
+#pragma unroll
+            for (int u2 = 0; u2 < 16; ++u2) {
+              float p0 = 0.f, p1 = 0.f;
+              if (any) {
+                p0 = (2 * u2 >= lo && 2 * u2 <= hi) ? fast_exp2(fmaf(__uint_as_float(r[2 * u2]), a.scale_log2, -m))
+                                                      : 0.f;
+                p1 = (2 * u2 + 1 >= lo && 2 * u2 + 1 <= hi)
+                         ? fast_exp2(fmaf(__uint_as_float(r[2 * u2 + 1]), a.scale_log2, -m))
+                         : 0.f;
+              }
+              ls[(2 * u2) & 7] += p0;
+              ls[(2 * u2 + 1) & 7] += p1;
+              pw[u2] = pack_bf16(p0, p1);
+            }
           }
           tmem_st16(scol + kb * 64 + qq * 16, pw);
         }
@@ -366,54 +405,100 @@ __global__ void __launch_bounds__(WinCfg<G>::THREADS, 1)
         l = gs ? other + l : l + other;
       }
       if (!ok) break;
-      // ---------------- epilogue: o = O / l as scaled float16, slot topk + s
-      ok = __all_sync(0xFFFFFFFFu, mbar_wait(o_full, par, a.err, SITE_WIN_SOFTMAX));
-      if (!ok) break;
+      // (m, l) to the epilogue through TMEM columns past the first block's P
+      // (both groups are past their S loads here); the next tile's S waits
+      // until the epilogue has read them
+      if (gs == 0) {
+        const uint32_t mlv[2] = {__float_as_uint(m), __float_as_uint(l)};
+        tmem_st2(scol + (C::ML_COL - C::S_COL), mlv);
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(ml_full);
+      }
+      ++u;
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int eq = warp & 3;
+    const int row = eq * 32 + lane;
+    const int e = row / G, h = row % G;
+    const uint32_t ocol = tmem_base + (static_cast<uint32_t>(eq * 32) << 16) + C::O_COL;
+    uint8_t* stage = sV + eq * 32 * C::ROW;   // this warp's 32 staging rows (first V slot)
+    uint32_t u = 0;
+    for (int t = blockIdx.x; t < a.n_tiles; t += gridDim.x) {
+      const WinTile w = win_tile<G>(a, t);
+      if (w.kb0 < 0) continue;
+      const uint32_t par = u & 1;
+      const int i = w.q0 + e;
+      const bool valid = i < a.n_q;
+      if (!__all_sync(0xFFFFFFFFu, mbar_wait(ml_full, par, a.err, SITE_WIN_SOFTMAX) &&
+                                       mbar_wait(o_full, par, a.err, SITE_WIN_SOFTMAX)))
+        break;
       tc_fence_after();
-      uint32_t r[64];
-      win_ld64(ocol, r);   // this group's 64 columns of O
+      uint32_t mlv[2];
+      tmem_ld2(tmem_base + (static_cast<uint32_t>(eq * 32) << 16) + C::ML_COL, mlv);
+      tmem_wait_ld();
+      tmem_regs_ready(mlv);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(ml_read);
+      const float m = __uint_as_float(mlv[0]), l = __uint_as_float(mlv[1]);
       float am[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-      for (int u2 = 0; u2 < 64; ++u2) am[u2 & 7] = fmaxf(am[u2 & 7], fabsf(__uint_as_float(r[u2])));
-      float amax = fmaxf(fmaxf(fmaxf(am[0], am[1]), fmaxf(am[2], am[3])), fmaxf(fmaxf(am[4], am[5]), fmaxf(am[6], am[7])));
-      amax = fmaxf(amax, swap(2, amax, par, ok));
-      if (!ok) break;
-      // a row with no keys in this chunk (never read by the merge) stores zeros
+      for (int hf = 0; hf < D / 64; ++hf) {
+        uint32_t r[64];
+        win_ld64(ocol + hf * 64, r);
+#pragma unroll
+        for (int u2 = 0; u2 < 64; ++u2) am[u2 & 7] = fmaxf(am[u2 & 7], fabsf(__uint_as_float(r[u2])));
+      }
+      const float amax = fmaxf(fmaxf(fmaxf(am[0], am[1]), fmaxf(am[2], am[3])), fmaxf(fmaxf(am[4], am[5]), fmaxf(am[6], am[7])));
+      // o = O / l as float16 times 2^-e; a row with no keys in this chunk
+      // (never read by the merge) stores zeros
       const float inv_l = l > 0.f ? 1.f / l : 0.f;
       const float x = amax * inv_l;
       int ex = x > 0.f ? static_cast<int>((__float_as_uint(x) >> 23) & 0xFFu) - 127 - 14 : 0;
       ex = min(max(ex, -100), 100);
       const float mul = inv_l * __uint_as_float(static_cast<uint32_t>(127 - ex) << 23);
       const int64_t slot = ((static_cast<int64_t>(w.bg) * a.n_q + i) * a.nsl + a.topk + w.s) * G + h;
-#pragma unroll
-      for (int q = 0; q < 8; ++q) {
-        uint32_t wv[4];
-#pragma unroll
-        for (int u2 = 0; u2 < 4; ++u2) {
-          const __half2 hv = __floats2half2_rn(__uint_as_float(r[q * 8 + 2 * u2]) * mul,
-                                               __uint_as_float(r[q * 8 + 2 * u2 + 1]) * mul);
-          wv[u2] = *reinterpret_cast<const uint32_t*>(&hv);
-        }
-        *reinterpret_cast<uint4*>(stage + lane * C::ROW + ((q ^ (lane & 7)) << 4)) =
-            make_uint4(wv[0], wv[1], wv[2], wv[3]);
-      }
-      __syncwarp();
       const int srow = lane >> 3, sch = lane & 7;
+      // the staging rows are free once the previous tile's stores have read them
 #pragma unroll
-      for (int k = 0; k < 8; ++k) {
-        const int rr = k * 4 + srow;
-        const int64_t rslot = __shfl_sync(0xFFFFFFFFu, slot, rr);
-        const bool rvalid = __shfl_sync(0xFFFFFFFFu, valid ? 1 : 0, rr) != 0;
-        const uint4 v = *reinterpret_cast<const uint4*>(stage + rr * C::ROW + ((sch ^ (rr & 7)) << 4));
-        if (rvalid) reinterpret_cast<uint4*>(a.partO + rslot * D + gs * 64)[sch] = v;
+      for (int hf = 0; hf < D / 64; ++hf) {
+        uint32_t r[64];
+        win_ld64(ocol + hf * 64, r);
+        if (hf == D / 64 - 1) {   // all of O is in registers: free the accumulator
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(o_empty);
+        }
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+          uint32_t wv[4];
+#pragma unroll
+          for (int u2 = 0; u2 < 4; ++u2) {
+            const __half2 hv = __floats2half2_rn(__uint_as_float(r[q * 8 + 2 * u2]) * mul,
+                                                 __uint_as_float(r[q * 8 + 2 * u2 + 1]) * mul);
+            wv[u2] = *reinterpret_cast<const uint32_t*>(&hv);
+          }
+          *reinterpret_cast<uint4*>(stage + lane * C::ROW + ((q ^ (lane & 7)) << 4)) =
+              make_uint4(wv[0], wv[1], wv[2], wv[3]);
+        }
+        __syncwarp();
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          const int rr = k * 4 + srow;
+          const int64_t rslot = __shfl_sync(0xFFFFFFFFu, slot, rr);
+          const bool rvalid = __shfl_sync(0xFFFFFFFFu, valid ? 1 : 0, rr) != 0;
+          const uint4 v = *reinterpret_cast<const uint4*>(stage + rr * C::ROW + ((sch ^ (rr & 7)) << 4));
+          if (rvalid) reinterpret_cast<uint4*>(a.partO + rslot * D + hf * 64)[sch] = v;
+        }
+        __syncwarp();
       }
-      if (valid && gs == 0)
+      if (valid)
         a.partL[slot] = make_float2(l > 0.f ? m + log2f(l) : -INFINITY,
                                     __uint_as_float(static_cast<uint32_t>(127 + ex) << 23));
-      // O read and the staging rows stored: the next tile's P V and V loads
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(epi_done);
+      if (lane == 0) mbar_arrive(stg_done);
       ++u;
     }
   }
