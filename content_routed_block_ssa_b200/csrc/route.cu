@@ -93,8 +93,11 @@ struct TiledCfg {
   static constexpr int A_TILE = A_BOXES * BOX_BYTES;      // one 128-row feature tile
   static constexpr int A_BYTES = RT * A_TILE;             // a unit's feature rows
   static constexpr int NAB = (KF == 256) ? 1 : 2;         // unit buffers
-  static constexpr int NS = 4;                            // table-slice ring
-  static constexpr int CAP = 16;                          // candidates per row (per epilogue group)
+  static constexpr int NS = 2;                            // table-slice ring
+  // candidates per row (per epilogue group); a row's buffered candidates are
+  // merged once some lane holds more than CAP - 16, so a deeper buffer merges
+  // larger batches (the warp runs as many insertions as its fullest lane)
+  static constexpr int CAP = 32;
   static constexpr int NACC = 4;                          // TMEM accumulators: 2 chunks x RT tiles
   static constexpr int NBAR = 2 * NAB + 2 * NS + 2 * NACC + 1;
   static constexpr int SMEM = 1024 + NAB * A_BYTES + NS * BOX_BYTES + RT * CAP * 128 * 8 + NBAR * 8 + 16;
