@@ -45,6 +45,10 @@ SECONDARY = "gqa_bf16_1m"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
+# FP32 FMA peak for ALU-bound kernels: 148 SMs x 128 FP32 lanes x 2 flop x 1.965 GHz.
+FP32_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
+
+
 def load_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -216,14 +220,21 @@ def algorithmic_work(w, idx):
     G = w.h_q // w.h_kv
     pos = np.arange(w.n_q) + w.q_offset
     nvis = np.minimum(nb, (pos + 1) // w.block).sum()
-    # one summary row and one routing dot product per sub-block
+    # one summary row and one routing dot product per sub-block (float32:
+    # mu and Sigma rows, d + d^2 for a full Sigma)
     summary_bytes = w.batch * w.n * w.h_kv * w.d * es + w.batch * w.h_kv * nb * w.subblocks * 2 * w.d * 2
     route_flops = 2.0 * (2 * w.d) * float(nvis) * w.subblocks * w.h_kv * w.batch
+    if w.dtype == "f32":
+        per = w.d + (w.d * w.d if w.sigma == "full" else w.d)
+        route_flops = 2.0 * per * float(nvis) * w.subblocks * w.h_q * w.batch
+        summary_bytes = w.batch * w.n * w.h_kv * w.d * es + w.batch * w.h_kv * nb * per * 4
+    route_table_bytes = float(nvis) * w.subblocks * w.h_kv * w.batch * 2 * w.d * 2
     S = attended_keys(idx, w)
     gathered = float(S.sum().item()) * w.d * 2 * es
     qo = 2.0 * w.batch * w.n_q * w.h_q * w.d * es
     attn_flops = 4.0 * float(S.sum().item()) * G * w.d
-    out = dict(summary_bytes=summary_bytes, route_flops=route_flops, attn_bytes=gathered + qo,
+    out = dict(summary_bytes=summary_bytes, route_flops=route_flops, route_table_bytes=route_table_bytes,
+               attn_bytes=gathered + qo,
                gathered_bytes=gathered, attn_flops=attn_flops, mean_keys=float(S.float().mean().item()))
     if w.dtype == "bf16":
         # block-major stages.  Per selected slot (a used selected block of a
@@ -256,7 +267,13 @@ def run_ours(w, steps, warmup, ws, rank, with_e2e=True):
     Q, K, V, _ = make_inputs(w, dev)
     p = ssa.make_params(**problem_dict(w))
     mu_s, sig_s, tab_s = ssa.summary_shapes(p)
-    tab = torch.empty(tab_s, dtype=torch.bfloat16, device=dev)
+    if w.dtype == "f32":   # float32 problems route on float32 mu / Sigma, no table
+        mu = torch.empty(mu_s, dtype=torch.float32, device=dev)
+        sig = torch.empty(sig_s, dtype=torch.float32, device=dev)
+        tab = None
+    else:
+        mu = sig = None
+        tab = torch.empty(tab_s, dtype=torch.bfloat16, device=dev)
     idx = torch.empty(ssa.idx_shape(p), dtype=torch.int32, device=dev)
     rws = ssa.byte_buffer(ssa.ssa_route_workspace_size(p), dev)
     aw_bytes = ssa.ssa_attn_workspace_size(p)
@@ -276,8 +293,8 @@ def run_ours(w, steps, warmup, ws, rank, with_e2e=True):
                   ("attn_window", lambda: ssa.ssa_attn_window(p, Q, K, V, aws)),
                   ("attn_merge", lambda: ssa.ssa_attn_merge(p, idx, O, lse, None, aws))]
     else:
-        stages = [("summary", lambda: ssa.ssa_block_summary(p, K, None, None, tab)),
-                  ("route", lambda: ssa.ssa_route_topk(p, Q, None, None, tab, idx, None, rws)),
+        stages = [("summary", lambda: ssa.ssa_block_summary(p, K, mu, sig, tab)),
+                  ("route", lambda: ssa.ssa_route_topk(p, Q, mu, sig, tab, idx, None, rws)),
                   ("attn_gather", lambda: ssa.ssa_sparse_attn(p, Q, K, V, idx, O, lse))]
     ns = len(stages)
 
@@ -340,7 +357,7 @@ def run_ours(w, steps, warmup, ws, rank, with_e2e=True):
                 clocks=clk.summary(), e2e=e2e)
 
 
-KERNEL_NAMES = {"summary": "summary_diag_kernel", "route": "route_tiled_kernel", "attn_plan": "inv_*_kernel (6)",
+KERNEL_NAMES = {"summary": "summary_bf16_warp_kernel", "route": "route_tiled_kernel", "attn_plan": "inv_*_kernel (6)",
                 "attn_blocks": "attn_block_kernel", "attn_window": "attn_window_kernel",
                 "attn_merge": "attn_merge_kernel",
                 "attn_gather": "attn_bf16_kernel"}
@@ -366,12 +383,28 @@ def kernel_report(w, res, peaks, traffic):
         rep[name] = e
 
     hbm_entry("summary", wk["summary_bytes"])
-    r_tf = wk["route_flops"] / (ms["route"] * 1e-3) / 1e12
-    rep["route"] = {"ms": ms["route"], "bound": "tensor", "achieved": r_tf, "unit": "TFLOP/s", "frac": r_tf / tc,
-                    "peak": tc, "algorithmic_flops": wk["route_flops"], "kernel": KERNEL_NAMES["route"],
-                    "traffic": traffic.get(("route_tiled_kernel", w.name))}
+    if w.dtype == "f32":
+        rep["summary"]["kernel"] = "summary_diag_kernel" if w.sigma == "diag" else "summary_full_kernel"
+        # float32 rows score their blocks with FMA on the CUDA cores (row-wise router)
+        r_tf = wk["route_flops"] / (ms["route"] * 1e-3) / 1e12
+        rep["route"] = {"ms": ms["route"], "bound": "alu", "achieved": r_tf, "unit": "TFLOP/s",
+                        "frac": r_tf / FP32_TFLOPS, "peak": FP32_TFLOPS, "algorithmic_flops": wk["route_flops"],
+                        "kernel": "route_rowwise_f32_kernel", "traffic": None}
+    elif w.n_q < 128:
+        # decode: each row streams its (batch, kv-head) table once (row-wise router)
+        e = wk["route_table_bytes"] / (ms["route"] * 1e-3) / 1e9
+        rep["route"] = {"ms": ms["route"], "bound": "hbm", "achieved": e, "unit": "GB/s", "frac": e / hbm,
+                        "peak": hbm, "algorithmic_bytes": wk["route_table_bytes"],
+                        "kernel": "route_rowwise_bf16_kernel", "traffic": None}
+    else:
+        r_tf = wk["route_flops"] / (ms["route"] * 1e-3) / 1e12
+        rep["route"] = {"ms": ms["route"], "bound": "tensor", "achieved": r_tf, "unit": "TFLOP/s",
+                        "frac": r_tf / tc, "peak": tc, "algorithmic_flops": wk["route_flops"],
+                        "kernel": KERNEL_NAMES["route"], "traffic": traffic.get(("route_tiled_kernel", w.name))}
     if "attn_gather" in ms:
         hbm_entry("attn_gather", wk["attn_bytes"], {"mean_keys_per_row": wk["mean_keys"]})
+        if w.dtype == "f32":
+            rep["attn_gather"]["kernel"] = "attn_f32_kernel"
     else:
         hbm_entry("attn_plan", wk["plan_bytes"])
         hbm_entry("attn_blocks", wk["blocks_bytes"], {"n_entries": wk["n_entries"], "n_blocks": wk["n_blocks"]})
@@ -502,7 +535,7 @@ def main():
     roof = {"bound": dk["bound"], "achieved": dk["achieved"], "peak": dk["peak"], "unit": dk["unit"],
             "frac": dk["frac"], "traffic": dk["traffic"], "kernel": dk["kernel"], "stage": dname,
             "peak_source": peak_src,
-            "algorithmic_per_launch": dk.get("algorithmic_flops") if dk["bound"] == "tensor"
+            "algorithmic_per_launch": dk.get("algorithmic_flops") if dk["bound"] in ("tensor", "alu")
             else dk["algorithmic_bytes"]}
     secondary = None
     if not a.no_secondary and w.name == PRIMARY and a.n is None:
@@ -526,7 +559,7 @@ def main():
     if rank == 0:
         line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws, "steps": a.steps, "warmup": a.warmup,
                 "ms_per_step": res["ms_step"], "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-                "dtype": "bf16", "data": "synthetic", "config": config, "roofline": roof, "cpu_baseline": cpu,
+                "dtype": w.dtype, "data": "synthetic", "config": config, "roofline": roof, "cpu_baseline": cpu,
                 "e2e": res["e2e"], "gpu_launches": res["launches"], "clocks": res["clocks"], "kernels": kern,
                 "secondary": secondary}
         print(json.dumps(line), flush=True)

@@ -6,12 +6,13 @@
 // ["The idea in one screen", routing-score equation].  Normalisation is by
 // the number of keys summarised (population moments).
 //
-// One CTA per (batch, kv-head, unit), a unit being a block of B keys, or a
-// sub-block of B / S keys when each block is summarised S times.  The block's B x d keys are read once
-// with 16-byte coalesced loads into registers; the mean and then the centred
-// second moments are reduced in float64.  For bf16 and float32 keys every
-// partial sum of the mean is exact in float64, so mu is the exact block mean
-// and its float32 / bfloat16 roundings are reproducible bit for bit.
+// A unit is a block of B keys, or a sub-block of B / S keys when each block
+// is summarised S times.  bf16 keys: one warp per (batch, kv-head, unit),
+// lane l owning dimensions d/32 l .. d/32 (l+1) - 1, one pass over the rows
+// with float64 sums.  float32 keys: one CTA per unit, the mean and then the
+// centred second moments reduced in float64.  Every partial sum of the mean
+// is exact in float64, so mu is the exact block mean and its float32 /
+// bfloat16 roundings are reproducible bit for bit.
 #include <cuda_bf16.h>
 
 #include "common.cuh"
@@ -109,6 +110,84 @@ __global__ void __launch_bounds__(256) summary_diag_kernel(const T* __restrict__
   }
 }
 
+// bf16 diagonal summaries, a warp per unit.  The variance comes from sums
+// of the keys shifted by the unit's first key, sum (x - x0) and
+// sum (x - x0)^2: for bf16 keys each shifted value and its square are exact
+// in float64 and so are their sums over a unit, so the one-pass formula
+// (sum (x-x0)^2 - (sum (x-x0))^2 / n) / n differs from the centred two-pass
+// sum only in the final float64 roundings.
+template <int D, int BLK>
+__global__ void __launch_bounds__(256) summary_bf16_warp_kernel(const __nv_bfloat16* __restrict__ K,
+                                                                 float* __restrict__ mu, float* __restrict__ sig,
+                                                                 __nv_bfloat16* __restrict__ table, int n_kv,
+                                                                 int h_kv, int nu, int64_t units) {
+  constexpr int VPL = D / 32;   // dimensions per lane: 4 (d = 128) or 2 (d = 64)
+  constexpr int UNROLL = 16;    // rows loaded before they are summed
+  static_assert(BLK % UNROLL == 0, "unit size");
+  const int lane = threadIdx.x & 31;
+  const int64_t x = static_cast<int64_t>(blockIdx.x) * 8 + (threadIdx.x >> 5);   // output row
+  if (x >= units) return;   // warp-uniform
+  const int c = static_cast<int>(x % nu);
+  const int64_t bg = x / nu;
+  const int g = static_cast<int>(bg % h_kv), b = static_cast<int>(bg / h_kv);
+  const int64_t row_stride = static_cast<int64_t>(h_kv) * D;
+  const __nv_bfloat16* base = K + ((static_cast<int64_t>(b) * n_kv + static_cast<int64_t>(c) * BLK) * h_kv + g) * D +
+                              lane * VPL;
+  auto load = [&](int r, float (&v)[VPL]) {
+    if (VPL == 4) {
+      const uint2 w = __ldg(reinterpret_cast<const uint2*>(base + r * row_stride));
+      v[0] = __uint_as_float(w.x << 16); v[1] = __uint_as_float(w.x & 0xFFFF0000u);
+      v[2] = __uint_as_float(w.y << 16); v[3] = __uint_as_float(w.y & 0xFFFF0000u);
+    } else {
+      const uint32_t w = __ldg(reinterpret_cast<const uint32_t*>(base + r * row_stride));
+      v[0] = __uint_as_float(w << 16); v[1] = __uint_as_float(w & 0xFFFF0000u);
+    }
+  };
+  float x0[VPL];
+  load(0, x0);
+  double s0[VPL], s1[VPL], s2[VPL];   // sum x, sum (x - x0), sum (x - x0)^2
+#pragma unroll
+  for (int v = 0; v < VPL; ++v) { s0[v] = 0.0; s1[v] = 0.0; s2[v] = 0.0; }
+#pragma unroll 1
+  for (int r0 = 0; r0 < BLK; r0 += UNROLL) {
+    float xv[UNROLL][VPL];
+#pragma unroll
+    for (int u = 0; u < UNROLL; ++u) load(r0 + u, xv[u]);
+#pragma unroll
+    for (int u = 0; u < UNROLL; ++u) {
+#pragma unroll
+      for (int v = 0; v < VPL; ++v) {
+        const double xd = static_cast<double>(xv[u][v]);
+        const double t = xd - static_cast<double>(x0[v]);
+        s0[v] += xd;
+        s1[v] += t;
+        s2[v] = fma(t, t, s2[v]);
+      }
+    }
+  }
+  float m32[VPL], v32[VPL];
+#pragma unroll
+  for (int v = 0; v < VPL; ++v) {
+    m32[v] = __double2float_rn(s0[v] / BLK);
+    v32[v] = __double2float_rn((s2[v] - s1[v] * s1[v] / BLK) / BLK);
+  }
+  if (mu) {
+#pragma unroll
+    for (int v = 0; v < VPL; ++v) mu[x * D + lane * VPL + v] = m32[v];
+  }
+  if (sig) {
+#pragma unroll
+    for (int v = 0; v < VPL; ++v) sig[x * D + lane * VPL + v] = v32[v];
+  }
+  if (table) {
+#pragma unroll
+    for (int v = 0; v < VPL; ++v) {
+      table[x * 2 * D + lane * VPL + v] = __float2bfloat16_rn(m32[v]);
+      table[x * 2 * D + D + lane * VPL + v] = __float2bfloat16_rn(v32[v]);
+    }
+  }
+}
+
 // Full covariance (float32 problems).  The block is staged centred in
 // shared memory as float64; thread e computes entries e, e+256, ...
 template <int D, int BLK>
@@ -153,11 +232,22 @@ template <typename T, int D, int BLK>
 cudaError_t run_diag(const ssa_params& p, const void* K, float* mu, float* sig, void* table,
                      const LaunchCtx& c) {
   const int nu = p.n_kv / BLK;
-  dim3 grid(nu, p.h_kv, p.batch);
-  summary_diag_kernel<T, D, BLK><<<grid, 256, 0, c.stream>>>(
-      static_cast<const T*>(K), mu, sig, static_cast<__nv_bfloat16*>(table), p.n_kv, p.h_kv, nu);
-  note_launch();
-  return cudaGetLastError();
+  if constexpr (sizeof(T) == 2) {   // bf16: a warp per unit
+    const int64_t units = static_cast<int64_t>(p.batch) * p.h_kv * nu;
+    const int64_t grid = (units + 7) / 8;
+    if (grid > 2147483647) return cudaErrorInvalidValue;
+    summary_bf16_warp_kernel<D, BLK><<<static_cast<unsigned>(grid), 256, 0, c.stream>>>(
+        reinterpret_cast<const __nv_bfloat16*>(K), mu, sig, static_cast<__nv_bfloat16*>(table), p.n_kv, p.h_kv, nu,
+        units);
+    note_launch();
+    return cudaGetLastError();
+  } else {   // float32: a CTA per unit
+    dim3 grid(nu, p.h_kv, p.batch);
+    summary_diag_kernel<T, D, BLK><<<grid, 256, 0, c.stream>>>(
+        static_cast<const T*>(K), mu, sig, static_cast<__nv_bfloat16*>(table), p.n_kv, p.h_kv, nu);
+    note_launch();
+    return cudaGetLastError();
+  }
 }
 
 template <int D, int BLK>
