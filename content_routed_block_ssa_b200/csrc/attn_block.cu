@@ -742,14 +742,22 @@ __global__ void __maxnreg__((BlkCfg<G, BLK>::MAXREG))
     bool ok = true;
     int4 nxt = q < T ? a.tiles[t0 + q] : none;
     int4 nxt2 = q + C::NGW < T ? a.tiles[t0 + q + C::NGW] : none;   // two ahead (TMA path)
-    int nen0 = lane < nxt.w ? __ldg(a.entries + nxt.z + lane) : 0;
-    int nen1 = (QPT > 32 && lane + 32 < nxt.w) ? __ldg(a.entries + nxt.z + 32 + lane) : 0;
+    // the next tile's entries, entry j in register j / 32 of lane j % 32
+    constexpr int NEN = (QPT + 31) / 32;
+    int nen[NEN];
+    auto load_entries = [&](const int4& td) {
+#pragma unroll
+      for (int k = 0; k < NEN; ++k) nen[k] = lane + 32 * k < td.w ? __ldg(a.entries + td.z + 32 * k + lane) : 0;
+    };
+    load_entries(nxt);
     int last_lt = -1;
     for (int lt = q; lt < T && ok; lt += C::NGW) {
       const int ab = lt % NA;
       const uint32_t use = static_cast<uint32_t>(lt / NA);
       const int4 td = nxt;
-      const int en0 = nen0, en1 = nen1;
+      int en[NEN];
+#pragma unroll
+      for (int k = 0; k < NEN; ++k) en[k] = nen[k];
       const int b = td.x / a.h_kv, g = td.x % a.h_kv, ne = td.w;
       if (lane == 0) ok = mbar_wait(&a_empty[ab], (use & 1) ^ 1, a.err, SITE_BLK_A_EMPTY);
       ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
@@ -762,7 +770,7 @@ __global__ void __maxnreg__((BlkCfg<G, BLK>::MAXREG))
         if (lane == 0) mbar_arrive_expect_tx(&a_full[ab], static_cast<uint32_t>(ne) * G * D * 2);
         __syncwarp();
         if (lane < ne) {
-          const int i = entry_row(en0);
+          const int i = entry_row(en[0]);
           if (static_cast<unsigned>(i) < static_cast<unsigned>(a.n_q)) {
             const int z = static_cast<int>(static_cast<int64_t>(b) * a.n_q + i);
 #pragma unroll
@@ -774,20 +782,28 @@ __global__ void __maxnreg__((BlkCfg<G, BLK>::MAXREG))
         }
         nxt = nxt2;
         nxt2 = lt + 2 * C::NGW < T ? a.tiles[t0 + lt + 2 * C::NGW] : none;
-        nen0 = lane < nxt.w ? __ldg(a.entries + nxt.z + lane) : 0;
+        load_entries(nxt);
       } else {
         const uint32_t abase = smem_u32(abuf);
-        for (int ee = 0; ee < ne; ++ee) {
-          const int ent = ee < 32 ? __shfl_sync(0xFFFFFFFFu, en0, ee) : __shfl_sync(0xFFFFFFFFu, en1, ee - 32);
+        // an entry is G rows of 16 chunks of 8 dims; a warp instruction
+        // copies 32 chunks: one entry's (G >= 2) or two entries' (G = 1)
+        constexpr int CPE = G * 16;
+        constexpr int EPI = CPE >= 32 ? 1 : 32 / CPE;
+        for (int ee0 = 0; ee0 < ne; ee0 += EPI) {
+          const int ee = ee0 + (EPI > 1 ? lane / CPE : 0);   // ee0 and ee share a register: ee0 is even
+          int reg = en[0];
+#pragma unroll
+          for (int k = 1; k < NEN; ++k) reg = (ee0 >> 5) == k ? en[k] : reg;
+          const int ent = __shfl_sync(0xFFFFFFFFu, reg, ee & 31);
           const int i = entry_row(ent);
-          if (static_cast<unsigned>(i) >= static_cast<unsigned>(a.n_q)) {   // never for a consistent plan
-            if (lane == 0) atomicCAS(a.err, 0u, static_cast<uint32_t>(SITE_BLK_BAD_ENTRY));
-            continue;
-          }
+          const bool live = ee < ne;
+          const bool row_ok = static_cast<unsigned>(i) < static_cast<unsigned>(a.n_q);
+          if (live && !row_ok) atomicCAS(a.err, 0u, static_cast<uint32_t>(SITE_BLK_BAD_ENTRY));   // never for a consistent plan
+          if (!live || !row_ok) continue;
           const __nv_bfloat16* qrow = a.Q + ((static_cast<int64_t>(b) * a.n_q + i) * a.h_q +
                                              static_cast<int64_t>(g) * G) * D;
 #pragma unroll
-          for (int x = lane; x < G * 16; x += 32) {   // G heads x 16 chunks of 8 dims
+          for (int x = (EPI > 1 ? lane % CPE : lane); x < CPE; x += (EPI > 1 ? CPE : 32)) {
             const int hh = x >> 4, ch = x & 15;
             const int r = ee * G + hh;
             const uint32_t dst = abase + (ch >> 3) * C::A_HALF + r * C::ROW + (((ch & 7) ^ (r & 7)) << 4);
@@ -798,8 +814,7 @@ __global__ void __maxnreg__((BlkCfg<G, BLK>::MAXREG))
         asm volatile("cp.async.commit_group;" ::: "memory");
         // this warp's next tile: descriptor and entries load while the copies fly
         nxt = lt + C::NGW < T ? a.tiles[t0 + lt + C::NGW] : none;
-        nen0 = lane < nxt.w ? __ldg(a.entries + nxt.z + lane) : 0;
-        nen1 = (QPT > 32 && lane + 32 < nxt.w) ? __ldg(a.entries + nxt.z + 32 + lane) : 0;
+        load_entries(nxt);
         asm volatile("cp.async.wait_group 0;" ::: "memory");
         fence_async_smem();
         __syncwarp();
@@ -863,7 +878,8 @@ __global__ void __launch_bounds__(256, (G == 8 ? 2 : (G == 4 ? 3 : 4))) attn_mer
   if (lane == 0 && a.bad && s.n_bad) atomicAdd(a.bad, s.n_bad);
   // the window chunks (slots topk + c) that hold keys, one lane each
   const uint32_t wch = __ballot_sync(0xFFFFFFFFu, lane < a.nsl - a.topk &&
-                                                      chunk_has_keys(s.win, a.q_offset + i, a.window, a.block, lane));
+                                                      chunk_has_keys(s.win, a.q_offset + i, a.window, a.block, lane,
+                                                                     win_chunk(G)));
   s.mask |= static_cast<uint64_t>(wch) << a.topk;
   const float2* pl = a.partL + item * a.nsl * G;
   const __half* po = a.partO + item * a.nsl * G * D;
@@ -965,12 +981,13 @@ cudaError_t launch_attn_merge(const ssa_params& p, const int32_t* block_idx, con
   a.bad = bad;
   a.n_q = p.n_q; a.h_q = p.h_q; a.h_kv = p.h_kv; a.nb = p.n_kv / p.block; a.block = p.block; a.topk = p.topk;
   a.window = p.window;
-  a.nsl = p.topk + window_chunks(p.window);
+  a.nsl = p.topk + window_chunks(p.window, p.h_q / p.h_kv);
   a.q_offset = p.q_offset;
   a.n_items = static_cast<int64_t>(p.batch) * p.h_kv * p.n_q;
   if (p.d != 128) return cudaErrorInvalidValue;
   const unsigned grid = static_cast<unsigned>((a.n_items + 7) / 8);
   switch (p.h_q / p.h_kv) {
+    case 1: attn_merge_kernel<1><<<grid, 256, 0, c.stream>>>(a); break;
     case 2: attn_merge_kernel<2><<<grid, 256, 0, c.stream>>>(a); break;
     case 4: attn_merge_kernel<4><<<grid, 256, 0, c.stream>>>(a); break;
     case 8: attn_merge_kernel<8><<<grid, 256, 0, c.stream>>>(a); break;
@@ -1027,7 +1044,7 @@ cudaError_t launch_attn_block(const ssa_params& p, const BlockPlan& pl, const vo
   a.t_start = pl.t_start;
   a.entries = pl.entries;
   a.n_q = p.n_q; a.n_kv = p.n_kv; a.h_q = p.h_q; a.h_kv = p.h_kv; a.topk = p.topk; a.window = p.window;
-  a.nsl = p.topk + window_chunks(p.window);
+  a.nsl = p.topk + window_chunks(p.window, p.h_q / p.h_kv);
   a.q_offset = p.q_offset;
   a.scale_log2 = p.scale * 1.4426950408889634f;
   a.partO = static_cast<__half*>(partO);
@@ -1036,10 +1053,12 @@ cudaError_t launch_attn_block(const ssa_params& p, const BlockPlan& pl, const vo
   const int G = p.h_q / p.h_kv;
   if (p.d != 128) return cudaErrorInvalidValue;
   if (p.block == 64) {
+    if (G == 1) return run_block<1, 64>(pl, tmK, tmV, tmQ, a, c);
     if (G == 2) return run_block<2, 64>(pl, tmK, tmV, tmQ, a, c);
     if (G == 4) return run_block<4, 64>(pl, tmK, tmV, tmQ, a, c);
     if (G == 8) return run_block<8, 64>(pl, tmK, tmV, tmQ, a, c);
   } else if (p.block == 128) {
+    if (G == 1) return run_block<1, 128>(pl, tmK, tmV, tmQ, a, c);
     if (G == 2) return run_block<2, 128>(pl, tmK, tmV, tmQ, a, c);
     if (G == 4) return run_block<4, 128>(pl, tmK, tmV, tmQ, a, c);
     if (G == 8) return run_block<8, 128>(pl, tmK, tmV, tmQ, a, c);

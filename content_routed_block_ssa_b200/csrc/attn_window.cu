@@ -4,9 +4,10 @@
 // queries.
 //
 // A tile is the 128 tensor-core rows of 128/G consecutive queries x the G
-// query heads of one kv-head, for one window chunk s (keys pos-W+1 + 256 s
-// .. min(pos, pos-W + 256 (s+1)) of each row).  The chunks of the tile's rows
-// together span at most 256 + 128/G - 1 keys, six 64-key blocks: S = Q K^T
+// query heads of one kv-head, for one window chunk s (keys pos-W+1 + C s ..
+// min(pos, pos-W + C (s+1)) of each row, C = 256 keys, 128 when G = 1).  The
+// chunks of the tile's rows together span at most C + 128/G - 1 keys, six
+// 64-key blocks: S = Q K^T
 // over the whole span fits 384 TMEM columns next to the 128 of O, so the
 // softmax needs no rescaling.  Each row masks the keys outside its own chunk
 // and the keys of blocks it already attends through its selected slots (the
@@ -76,8 +77,9 @@ __device__ __forceinline__ WinTile win_tile(const WinArgs& a, int t) {
   w.s = r % a.nwc;
   const int64_t p0 = a.q_offset + w.q0;
   const int64_t pl = a.q_offset + min(w.q0 + QT, a.n_q) - 1;
-  int64_t lo = p0 - a.window + 1 + static_cast<int64_t>(w.s) * kWinChunk;
-  int64_t hi = pl - a.window + static_cast<int64_t>(w.s + 1) * kWinChunk;
+  constexpr int CH = win_chunk(G);
+  int64_t lo = p0 - a.window + 1 + static_cast<int64_t>(w.s) * CH;
+  int64_t hi = pl - a.window + static_cast<int64_t>(w.s + 1) * CH;
   if (lo < 0) lo = 0;
   if (hi > pl) hi = pl;
   if (hi < lo) {
@@ -307,7 +309,8 @@ __global__ void __launch_bounds__(WinCfg<G>::THREADS, 1)
       const int pos = static_cast<int>(a.q_offset) + i;
       const int w0 = pos - a.window + 1;
       const int span0 = w.kb0 * 64;
-      int klo = max(w0 + w.s * kWinChunk, 0), khi = min(w0 + (w.s + 1) * kWinChunk - 1, pos);
+      constexpr int CH = win_chunk(G);
+      int klo = max(w0 + w.s * CH, 0), khi = min(w0 + (w.s + 1) * CH - 1, pos);
       if (!valid) { klo = 1; khi = 0; }
       klo -= span0;
       khi -= span0;
@@ -531,12 +534,12 @@ cudaError_t launch_attn_window(const ssa_params& p, const BlockPlan& pl, const C
                                const CUtensorMap& tmK, const CUtensorMap& tmV, void* partO, void* partL,
                                const LaunchCtx& c) {
   const int G = p.h_q / p.h_kv;
-  if (p.d != 128 || (G != 2 && G != 4 && G != 8)) return cudaErrorInvalidValue;
+  if (p.d != 128 || (G != 1 && G != 2 && G != 4 && G != 8)) return cudaErrorInvalidValue;
   WinArgs a;
   a.win = pl.win;
   a.n_q = p.n_q; a.n_kv = p.n_kv; a.h_q = p.h_q; a.h_kv = p.h_kv; a.block = p.block; a.topk = p.topk;
   a.window = p.window;
-  a.nwc = window_chunks(p.window);
+  a.nwc = window_chunks(p.window, G);
   a.nsl = p.topk + a.nwc;
   const int qt = 128 / G;
   a.n_qt = (p.n_q + qt - 1) / qt;
@@ -548,6 +551,7 @@ cudaError_t launch_attn_window(const ssa_params& p, const BlockPlan& pl, const C
   a.partO = static_cast<__half*>(partO);
   a.partL = static_cast<float2*>(partL);
   a.err = c.err;
+  if (G == 1) return run_window<1>(tmQ, tmK, tmV, a, c);
   if (G == 2) return run_window<2>(tmQ, tmK, tmV, a, c);
   if (G == 4) return run_window<4>(tmQ, tmK, tmV, a, c);
   return run_window<8>(tmQ, tmK, tmV, a, c);

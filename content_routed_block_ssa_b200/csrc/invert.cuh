@@ -7,7 +7,8 @@
 // used: a fully visible block index larger than every earlier in-range entry
 // (so the used entries are ascending and distinct; anything else is skipped
 // and counted).  Slot topk + s is chunk s of the window: its keys
-// pos-W+1 + 256 s .. min(pos, pos-W + 256 (s+1)) that lie in no used block.
+// pos-W+1 + C s .. min(pos, pos-W + C (s+1)) that lie in no used block, with
+// C = win_chunk(G) keys per chunk.
 // Every key of the set is thus in exactly one slot.  Selected slots are
 // evaluated block by block (the block kernel), window chunks by a dense
 // sliding-window kernel.
@@ -17,8 +18,10 @@
 
 namespace ssa {
 
-// Keys per window chunk (one slot each).
-constexpr int kWinChunk = 256;
+// Keys per window chunk (one slot each): 256, or 128 when a query has one
+// head per kv-head (a sliding-window tile then spans 128 queries, and its
+// keys must still fit six 64-key blocks).
+__host__ __device__ constexpr int win_chunk(int G) { return G == 1 ? 128 : 256; }
 
 // An inverted entry: the query row and the slot of that row.
 __device__ __forceinline__ int32_t make_entry(int row, int slot) { return (row << 6) | slot; }
@@ -31,7 +34,9 @@ __host__ __device__ constexpr int window_slots(int window, int block) {
 }
 
 // Window chunks (slots) of a window of W keys.
-__host__ __device__ constexpr int window_chunks(int window) { return (window + kWinChunk - 1) / kWinChunk; }
+__host__ __device__ constexpr int window_chunks(int window, int G) {
+  return (window + win_chunk(G) - 1) / win_chunk(G);
+}
 
 struct SlotSet {
   uint64_t mask;   // bit j < topk: selected slot j holds keys
@@ -74,12 +79,13 @@ __device__ __forceinline__ SlotSet row_slots(int v_in, int topk, int64_t pos, in
   return s;
 }
 
-// Whether window chunk s of the row at pos holds keys: some block it
-// overlaps is uncovered.  win as in SlotSet (blocks b0 + w).
-__host__ __device__ inline bool chunk_has_keys(uint32_t win, int64_t pos, int window, int block, int s) {
+// Whether window chunk s (of `chunk` keys) of the row at pos holds keys:
+// some block it overlaps is uncovered.  win as in SlotSet (blocks b0 + w).
+__host__ __device__ inline bool chunk_has_keys(uint32_t win, int64_t pos, int window, int block, int s,
+                                               int chunk) {
   const int64_t w0 = pos - window + 1;                 // unclamped window start
-  int64_t klo = w0 + static_cast<int64_t>(s) * kWinChunk;
-  int64_t khi = w0 + static_cast<int64_t>(s + 1) * kWinChunk - 1;
+  int64_t klo = w0 + static_cast<int64_t>(s) * chunk;
+  int64_t khi = w0 + static_cast<int64_t>(s + 1) * chunk - 1;
   if (khi > pos) khi = pos;
   if (klo < 0) klo = 0;
   if (khi < klo) return false;

@@ -152,12 +152,13 @@ ssa_status from_cuda(cudaError_t e) { return e == cudaSuccess ? SSA_OK : SSA_ERR
 
 // Block-major attention applies to long bf16 problems whose query heads
 // fill a 128-row tensor-core tile in groups of G, whose row slots (selected
-// blocks plus window blocks) fit the 6-bit slot field of an entry, and whose
-// per-block counters fit the inversion's shared memory.
+// blocks plus window chunks) fit the 6-bit slot field of an entry and whose
+// window blocks fit a 32-bit mask, and whose per-block counters fit the
+// inversion's shared memory.
 bool use_block_attn(const ssa_params& p) {
   const int G = p.h_q / p.h_kv;
   const int64_t nb = p.n_kv / p.block;
-  return p.dtype == SSA_BF16 && p.d == 128 && (G == 2 || G == 4 || G == 8) && p.topk * G <= 128 &&
+  return p.dtype == SSA_BF16 && p.d == 128 && (G == 1 || G == 2 || G == 4 || G == 8) && p.topk * G <= 128 &&
          ssa::window_slots(p.window, p.block) <= 32 && nb <= 16384 && p.n_q >= 1024 && p.n_q < (1 << 25);
 }
 
@@ -176,7 +177,7 @@ AttnLayout attn_layout(const ssa_params& p) {
   const size_t G = static_cast<size_t>(p.h_q / p.h_kv);
   const size_t qpt = 128 / G;
   L.nchunk = (p.n_q + ssa::kPlanRows - 1) / ssa::kPlanRows;
-  L.nsl = p.topk + ssa::window_chunks(p.window);
+  L.nsl = p.topk + ssa::window_chunks(p.window, p.h_q / p.h_kv);
   const size_t items = bgs * p.n_q;
   const size_t sel = items * L.nsl;                       // entries, at most
   const size_t max_tiles = (sel + qpt - 1) / qpt + bgs * nb;
@@ -344,7 +345,7 @@ bool encode_attn_maps(AttnMaps& m, const ssa_params& p, const void* Q, const voi
   if (!encode_kv(&m.K, K, p) || !encode_kv(&m.V, V, p) ||
       !encode_rows(&m.Q, Q, p.d, static_cast<uint64_t>(p.batch) * p.n_q * p.h_q, G))
     return false;
-  if (p.d == 128 && (G == 2 || G == 4 || G == 8) && !encode_q_tile(&m.Qw, Q, p, G, 128 / G)) return false;
+  if (p.d == 128 && (G == 1 || G == 2 || G == 4 || G == 8) && !encode_q_tile(&m.Qw, Q, p, G, 128 / G)) return false;
   if (G == 8 && p.d == 128) return encode_q_heads(&m.Qh, Q, p);
   m.Qh = m.Q;
   return true;

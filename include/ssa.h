@@ -186,7 +186,7 @@ SSA_API size_t ssa_attn_workspace_size(const ssa_params* p);
  * (atomically added, not reset).
  * Two evaluations give the same result up to rounding.  With a workspace
  * of ssa_attn_workspace_size(p) bytes (bf16 problems with n_q >= 1024,
- * d = 128, G in {2, 4, 8}, topk * G <= 128, at most 32 key blocks per
+ * d = 128, G in {1, 2, 4, 8}, topk * G <= 128, at most 32 key blocks per
  * window and 16384 key blocks) the evaluation is block-major: every
  * (query, kv-head) row is split into slots, one per used selected block and
  * one per window block not selected, the slots are inverted into per-block

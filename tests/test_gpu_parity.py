@@ -313,18 +313,19 @@ def test_empty_problem_launches_nothing_and_small_workspace_is_rejected():
     assert ssa.ssa_launch_count() == before
 
 
-# Problems the block-major attention takes (bf16, d = 128, G in {2, 4, 8},
+# Problems the block-major attention takes (bf16, d = 128, G in {1, 2, 4, 8},
 # k * G <= 128, at least 1024 query rows) when it is given its workspace.
 BLOCK_MAJOR = [n for n, w in CASES.items()
-               if w.dtype == "bf16" and w.d == 128 and w.h_q // w.h_kv in (2, 4, 8)
+               if w.dtype == "bf16" and w.d == 128 and w.h_q // w.h_kv in (1, 2, 4, 8)
                and w.topk * (w.h_q // w.h_kv) <= 128 and w.n_q >= 1024]
 
 
 def test_block_major_cases_exist():
     assert len(BLOCK_MAJOR) >= 3
+    assert "bf16_mha_d128_b64_k32" in BLOCK_MAJOR          # G = 1: 128 queries per tile
     for n in BLOCK_MAJOR:
         assert ssa.ssa_attn_workspace_size(params(problem_dict(CASES[n]))) > 0
-    assert ssa.ssa_attn_workspace_size(params(problem_dict(CASES["bf16_mha_d128_b64_k32"]))) == 0
+    assert ssa.ssa_attn_workspace_size(params(problem_dict(CASES["bf16_gqa2_d64_b64"]))) == 0   # d = 64
 
 
 @pytest.mark.parametrize("name", BLOCK_MAJOR)

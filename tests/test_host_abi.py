@@ -154,8 +154,8 @@ def test_block_major_workspace_and_stage_checks():
     # the partial outputs dominate: one bf16 row of d per (query, kv-head, slot, head)
     assert aw >= 2048 * 2 * 8 * 4 * 128 * 2
     del base
-    # does not qualify: too few rows, G = 1, d = 64, k * G > 128, float32
-    for kw in (dict(n_q=1000, n_kv=1024), dict(h_q=2, h_kv=2), dict(d=64),
+    # does not qualify: too few rows, d = 64, k * G > 128, float32
+    for kw in (dict(n_q=1000, n_kv=1024), dict(d=64),
                dict(topk=32, h_q=16, h_kv=2), dict(dtype="f32", h_q=2, h_kv=1)):
         q = good(**{**dict(n_q=2048, n_kv=2048), **kw})
         assert ssa.ssa_attn_workspace_size(q) == 0, kw
