@@ -389,7 +389,7 @@ def kernel_report(w, res, peaks, traffic):
         r_tf = wk["route_flops"] / (ms["route"] * 1e-3) / 1e12
         rep["route"] = {"ms": ms["route"], "bound": "alu", "achieved": r_tf, "unit": "TFLOP/s",
                         "frac": r_tf / FP32_TFLOPS, "peak": FP32_TFLOPS, "algorithmic_flops": wk["route_flops"],
-                        "kernel": "route_rowwise_f32_kernel", "traffic": None}
+                        "kernel": "route_qtile_f32_kernel", "traffic": None}
     elif w.n_q < 128:
         # decode: each row streams its (batch, kv-head) table once (row-wise router)
         e = wk["route_table_bytes"] / (ms["route"] * 1e-3) / 1e9

@@ -673,6 +673,127 @@ __global__ void __launch_bounds__(256) route_rowwise_f32_kernel(const float* __r
   select_and_write(keys, nvis, n2, a, out);
 }
 
+// float32 summaries for runs of query rows: a CTA takes 32/G consecutive
+// queries (32 (query, head) pairs) of one kv-head and walks the blocks,
+// staging each block's mu_c and Sigma_c in shared memory once for all of
+// them (the row-wise kernel reads them once per query).  Eight threads share
+// a (query, head) pair, each taking every eighth row of Sigma_c; the block
+// scores of each query stay in shared memory, and a warp per query sorts
+// them and writes its top k.  Sub-block rows are max-pooled per block.
+template <int D, int G, bool FULL>
+__global__ void __launch_bounds__(256) route_qtile_f32_kernel(const float* __restrict__ Q,
+                                                              const float* __restrict__ MU,
+                                                              const float* __restrict__ SG, const RowArgs a,
+                                                              int n2) {
+  constexpr int QT = 32 / G;            // queries per CTA
+  constexpr int SP = FULL ? D + 1 : D;  // padded Sigma row (bank spread)
+  extern __shared__ uint64_t keys[];    // [QT][n2]
+  float* qs = reinterpret_cast<float*>(keys + QT * n2);   // [32][D]
+  float* sgs = qs + 32 * D;                               // [D][SP] or [D]
+  float* mus = sgs + (FULL ? D * SP : D);                 // [D]
+  float* sc = mus + D;                                    // [32] (query, head) scores
+  const int i0 = blockIdx.x * QT, g = blockIdx.y, b = blockIdx.z;
+  const int h_q = a.h_kv * G;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  // the tile's (query, head) rows of Q; rows past n_q are zero
+  for (int e = threadIdx.x; e < 32 * D; e += 256) {
+    const int r = e / D, t = e % D, qq = r / G, h = r % G;
+    const int i = i0 + qq;
+    qs[e] = i < a.n_q ? Q[((static_cast<int64_t>(b) * a.n_q + i) * h_q + static_cast<int64_t>(g) * G + h) * D + t]
+                      : 0.f;
+  }
+  const int64_t last = a.q_offset + min(i0 + QT, a.n_q) - 1;
+  const int ncmax = static_cast<int>(min(static_cast<int64_t>(a.nb), (last + 1) / a.block));
+  const int r = threadIdx.x >> 3, part = threadIdx.x & 7;   // (query, head) row, its eighth
+  const int64_t bgrow = (static_cast<int64_t>(b) * a.h_kv + g) * a.nb * a.S;
+  for (int cb = 0; cb < ncmax; ++cb) {
+    float best = -INFINITY;   // threads < QT: the query's best sub-block score
+    for (int sb = 0; sb < a.S; ++sb) {
+      const int64_t row = bgrow + static_cast<int64_t>(cb) * a.S + sb;
+      __syncthreads();   // the previous summary row is consumed
+      for (int e = threadIdx.x; e < D; e += 256) mus[e] = MU[row * D + e];
+      if (FULL) {
+        for (int e = threadIdx.x; e < D * D; e += 256) sgs[(e / D) * SP + e % D] = SG[row * D * D + e];
+      } else {
+        for (int e = threadIdx.x; e < D; e += 256) sgs[e] = SG[row * D + e];
+      }
+      __syncthreads();
+      const float* q = qs + r * D;
+      float lin = 0.f, quad = 0.f;
+#pragma unroll 4
+      for (int s2 = part; s2 < D; s2 += 8) {
+        const float qv = q[s2];
+        lin = __fmaf_rn(qv, mus[s2], lin);
+        if (FULL) {
+          const float* srow = sgs + s2 * SP;
+          float u = 0.f;
+#pragma unroll 8
+          for (int t = 0; t < D; ++t) u = __fmaf_rn(srow[t], q[t], u);
+          quad = __fmaf_rn(qv, u, quad);
+        } else {
+          quad = __fmaf_rn(qv * qv, sgs[s2], quad);
+        }
+      }
+      float v = lin + a.half_beta * quad;
+#pragma unroll
+      for (int o = 4; o; o >>= 1) v += __shfl_xor_sync(0xFFFFFFFFu, v, o);
+      // the group's score of each query for this summary row: its heads'
+      // scores summed in head order; the block keeps its largest sub-block
+      if (part == 0) sc[r] = v;
+      __syncthreads();
+      if (threadIdx.x < QT) {
+        float acc = 0.f;
+#pragma unroll
+        for (int h = 0; h < G; ++h) acc += sc[threadIdx.x * G + h];
+        best = fmaxf(best, acc);
+      }
+    }
+    if (threadIdx.x < QT) {
+      const int qq = threadIdx.x, i = i0 + qq;
+      const int64_t pos = a.q_offset + i;
+      const bool vis = i < a.n_q && cb < min(static_cast<int64_t>(a.nb), (pos + 1) / a.block);
+      keys[qq * n2 + cb] = vis ? make_key(__float_as_uint(best), cb) : 0ull;
+    }
+  }
+  __syncthreads();
+  for (int e = threadIdx.x; e < QT * n2; e += 256)
+    if (e % n2 >= ncmax) keys[e] = 0ull;
+  __syncthreads();
+  // a warp per query: bitonic sort of its n2 keys (descending), then the top
+  // k in ascending block order
+  for (int qq = warp; qq < QT; qq += 8) {
+    const int i = i0 + qq;
+    if (i >= a.n_q) continue;   // warp-uniform
+    uint64_t* kq = keys + qq * n2;
+    for (int size = 2; size <= n2; size <<= 1) {
+      for (int stride = size >> 1; stride > 0; stride >>= 1) {
+        for (int t = lane; t < n2 / 2; t += 32) {
+          const int x = 2 * t - (t & (stride - 1));
+          const int y = x + stride;
+          const bool desc = (x & size) == 0;
+          const uint64_t kx = kq[x], ky = kq[y];
+          if (desc ? (kx < ky) : (kx > ky)) { kq[x] = ky; kq[y] = kx; }
+        }
+        __syncwarp();
+      }
+    }
+    const uint64_t key = (lane < a.topk && lane < n2) ? kq[lane] : 0ull;
+    const uint32_t blk = key ? key_block(key) : 0xFFFFFFFFu;
+    const uint32_t vmask = __ballot_sync(0xFFFFFFFFu, key != 0);
+    int rank = 0;
+    for (int o = 0; o < 32; ++o) {
+      const uint32_t other = __shfl_sync(0xFFFFFFFFu, blk, o);
+      rank += (other < blk) ? 1 : 0;
+    }
+    if (!key) rank = __popc(vmask) + __popc(~vmask & ((1u << lane) - 1u));
+    const int64_t out = ((static_cast<int64_t>(b) * a.n_q + i) * a.h_kv + g) * a.topk;
+    if (lane < a.topk) {
+      a.block_idx[out + rank] = key ? static_cast<int32_t>(blk) : -1;
+      if (a.top_scores) a.top_scores[out + rank] = key ? key_score(key) : -INFINITY;
+    }
+  }
+}
+
 RowArgs row_args(const ssa_params& p, int32_t* idx, float* scores) {
   RowArgs a;
   a.n_q = p.n_q; a.h_kv = p.h_kv; a.nb = p.n_kv / p.block; a.block = p.block; a.topk = p.topk;
@@ -738,9 +859,32 @@ cudaError_t rowwise_bf16_g(const ssa_params& p, const void* Q, const void* T, in
   return cudaErrorInvalidValue;
 }
 
+// Shared memory of route_qtile_f32_kernel, 0 when it does not fit.
+template <int D, int G, bool FULL>
+int qtile_smem_bytes(const ssa_params& p) {
+  int n2 = 1;
+  while (n2 < p.n_kv / p.block) n2 <<= 1;
+  const int64_t bytes = static_cast<int64_t>(32 / G) * n2 * 8 + 32 * D * 4 +
+                        (FULL ? static_cast<int64_t>(D) * (D + 1) : D) * 4 + D * 4 + 32 * 4;
+  return bytes <= 160 * 1024 ? static_cast<int>(bytes) : 0;
+}
+
 template <int D, int G, bool FULL>
 cudaError_t run_rowwise_f32(const ssa_params& p, const void* Q, const float* mu, const float* sg,
                             int32_t* idx, float* scores, const LaunchCtx& c) {
+  if (const int qs = qtile_smem_bytes<D, G, FULL>(p)) {   // runs of queries share each block's summary
+    int n2 = 1;
+    while (n2 < p.n_kv / p.block) n2 <<= 1;
+    cudaError_t e = cudaFuncSetAttribute(route_qtile_f32_kernel<D, G, FULL>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, qs);
+    if (e != cudaSuccess) return e;
+    constexpr int QT = 32 / G;
+    dim3 grid((p.n_q + QT - 1) / QT, p.h_kv, p.batch);
+    route_qtile_f32_kernel<D, G, FULL><<<grid, 256, qs, c.stream>>>(
+        static_cast<const float*>(Q), mu, sg, row_args(p, idx, scores), n2);
+    note_launch();
+    return cudaGetLastError();
+  }
   const int smem = row_smem_bytes(p);
   cudaError_t e = cudaFuncSetAttribute(route_rowwise_f32_kernel<D, G, FULL>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, smem);

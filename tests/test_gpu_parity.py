@@ -54,6 +54,10 @@ CASES = {
     "f32_full_d64_s2": Workload("c", 120, 1, 768, 1, 1, 64, "f32", 64, "full", 4, 64, 4, "total", subblocks=2),
     "f32_diag_gqa2_d128_b128_s4": Workload("c", 121, 1, 512, 2, 1, 128, "f32", 128, "diag", 2, 100, 2, "total",
                                            subblocks=4),
+    # float32 routing takes runs of 32 (query, head) pairs per CTA unless a
+    # row's 1024 block scores do not fit beside them: then one CTA per row
+    "f32_diag_d64_decode_64k": Workload("c", 122, 1, 65536, 1, 1, 64, "f32", 64, "diag", 8, 64, 2, "per_seq",
+                                        decode=True),
 }
 
 _cache = {}
