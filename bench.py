@@ -5,15 +5,18 @@
 
 One step is one pass of the whole layer over the workload's synthetic input:
 block summaries -> routing features + tensor-core route with fused top-k ->
-gathered exact attention, each a call of the libssa C ABI on the current
-stream (ssa_forward issues the same three calls).  Inputs are resident in HBM
-when the timed region starts; L2 is flushed between steps.  Step time is the
-sum of CUDA-event intervals around the step's kernels, the reported time the
-max over ranks.  With N > 1 every rank runs its own replica of the workload
-(independent problems, no collective on the data path): weak scaling.
+exact attention (block-major: plan, block tiles, window tiles, merge), each a
+call of the libssa C ABI on the current stream (ssa_forward issues the same
+calls).  Inputs are resident in HBM when the timed region starts; L2 is
+flushed between steps.  Step time is the sum of CUDA-event intervals around
+the step's kernels, the reported time the max over ranks.  With N > 1 every
+rank runs its own replica of the workload (independent problems, no
+collective on the data path): weak scaling.
 
 `e2e` repeats the step through ssa_forward_hostio with page-locked host
-inputs and outputs, host<->device copies inside the timed region.
+inputs and outputs, every step's host<->device copies inside the timed
+region; consecutive steps go round-robin to up to three streams (each with its
+own device buffer), so one step's copies overlap the others' compute.
 
 `--impl reference` times the CPU oracle (float64 NumPy) on a bounded sample of
 the same workload on the host cores.
@@ -330,29 +333,51 @@ def run_ours(w, steps, warmup, ws, rank, with_e2e=True):
 
     e2e = None
     if with_e2e:
+        # Through the public host-buffer call, every step copying its inputs in
+        # from pinned host memory and its output back.  Consecutive steps go
+        # round-robin to NS streams, each with its own device buffer and host
+        # output, as a caller pipelining steps would: a step's copies overlap
+        # the other streams' compute (the copy engines run both directions at
+        # once).  As many streams as fit in a third of the device memory, up to 3.
         hQ, hK, hV = Q.cpu().pin_memory(), K.cpu().pin_memory(), V.cpu().pin_memory()
-        hO = torch.empty(Q.shape, dtype=Q.dtype).pin_memory()
-        hl = torch.empty(Q.shape[:3], dtype=torch.float32).pin_memory()
         del O, lse, aws, stages
-        buf = ssa.byte_buffer(ssa.ssa_hostio_buffer_size(p), dev)
-        for _ in range(max(1, warmup)):
-            ssa.ssa_forward_hostio(p, hQ, hK, hV, hO, hl, buf)
+        torch.cuda.empty_cache()
+        hbytes = ssa.ssa_hostio_buffer_size(p)
+        NS = max(1, min(3, int(torch.cuda.mem_get_info(dev)[0] // max(hbytes, 1)) - 1))
+        outs = [(torch.empty(Q.shape, dtype=Q.dtype).pin_memory(),
+                 torch.empty(Q.shape[:3], dtype=torch.float32).pin_memory()) for _ in range(NS)]
+        bufs = [ssa.byte_buffer(hbytes, dev) for _ in range(NS)]
+        streams = [stream] + [torch.cuda.Stream(dev) for _ in range(NS - 1)]
+
+        def e2e_step(k):
+            hO, hl = outs[k % NS]
+            ssa.ssa_forward_hostio(p, hQ, hK, hV, hO, hl, bufs[k % NS], stream=streams[k % NS])
+
+        for k in range(max(NS, warmup)):
+            e2e_step(k)
         torch.cuda.synchronize()
         barrier(ws)
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
-        n_e2e = max(1, min(steps, 5))
-        for _ in range(n_e2e):
-            ssa.ssa_forward_hostio(p, hQ, hK, hV, hO, hl, buf)
-        e1.record(stream)
+        e0.record(streams[0])
+        for st in streams[1:]:
+            st.wait_event(e0)
+        n_e2e = max(2 * NS, min(steps, 3 * NS))
+        for k in range(n_e2e):
+            e2e_step(k)
+        for st in streams[1:]:
+            done = torch.cuda.Event()
+            done.record(st)
+            streams[0].wait_event(done)
+        e1.record(streams[0])
         torch.cuda.synchronize()
         ms_e2e = max_over_ranks(e0.elapsed_time(e1) / n_e2e, ws)
+        hO, hl = outs[0]
         h2d = hQ.numel() * hQ.element_size() + 2 * hK.numel() * hK.element_size()
         d2h = hO.numel() * hO.element_size() + hl.numel() * hl.element_size()
         e2e = {"value": whole_job_rate(w.batch * w.n_q * w.h_q, ws, ms_e2e), "unit": UNIT,
                "ms_per_step": ms_e2e, "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
-               "steps": n_e2e}
-        del buf
+               "steps": n_e2e, "streams": NS}
+        del bufs
     return dict(ms_step=ms_step, ms_kernels=ms_kernels, work=work, launches=int(launches),
                 clocks=clk.summary(), e2e=e2e)
 
