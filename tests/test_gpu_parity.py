@@ -54,6 +54,11 @@ CASES = {
     "f32_full_d64_s2": Workload("c", 120, 1, 768, 1, 1, 64, "f32", 64, "full", 4, 64, 4, "total", subblocks=2),
     "f32_diag_gqa2_d128_b128_s4": Workload("c", 121, 1, 512, 2, 1, 128, "f32", 128, "diag", 2, 100, 2, "total",
                                            subblocks=4),
+    # windows of several chunks on the block-major path: two 128-key chunks
+    # (G = 1) and three 256-key chunks (G = 8)
+    "bf16_mha_d128_b64_w200": Workload("c", 123, 1, 1536, 2, 2, 128, "bf16", 64, "diag", 8, 200, 4, "per_head"),
+    "bf16_gqa8_d128_b64_w600": Workload("c", 124, 1, 2048, 16, 2, 128, "bf16", 64, "diag", 8, 600, 4, "total",
+                                        clustered=True),
     # float32 routing takes runs of 32 (query, head) pairs per CTA unless a
     # row's 1024 block scores do not fit beside them: then one CTA per row
     "f32_diag_d64_decode_64k": Workload("c", 122, 1, 65536, 1, 1, 64, "f32", 64, "diag", 8, 64, 2, "per_seq",
