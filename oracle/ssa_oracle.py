@@ -409,3 +409,149 @@ def recovery_weight(beta: float, delta: float, mu: float) -> float:
     logit margin over each of mu equal distractors is Delta (at inverse
     temperature beta)."""
     return 1.0 / (1.0 + math.exp(-(beta * delta - math.log(mu))))
+
+
+# ---------------------------------------------------------------- hierarchical router
+
+# The page "Subquadratic Sparse Attention (SSA)" names, without defining them,
+# a tree router with a recursive radius (its artifact list, Barnes-Hut style),
+# exact branch-and-bound selection under an admissible bound (same list) and
+# per-query certificates with escalation (the "Certified Causal Cascade"
+# entry).  The reading written out below:
+#
+#   * a node is M consecutive blocks (M = the fan-out); only complete nodes
+#     exist, a trailing group of fewer than M blocks is no node;
+#   * node summary, from the stored bf16 routing rows T_c = [mu_c ; s_c] of its
+#     blocks: centre m_N = bf16(f32(mean_c mu_c)), variance cap
+#     v_N = max_c s_c (per dimension), radius R_N = max_c ||mu_c - m_N||_2
+#     (float64, rounded up to float32);
+#   * admissible bound: for any block c of N and features f = [f_s ; f_q]
+#     with f_q >= 0,  f . T_c <= f . [m_N ; v_N] + ||f_s|| R_N
+#     (Cauchy-Schwarz on the mean part, the cap on the variance part);
+#   * a query row ranks its complete visible nodes by w_N = f . [m_N ; v_N]
+#     (higher first, then lower node index), expands the first p, scores
+#     exactly every block of those nodes and every visible block outside a
+#     complete visible node, and keeps the top-k of those scores;
+#   * certificate: the row is certified when no complete visible node is left
+#     unexpanded, or when its k-th kept score exceeds
+#     w_(p+1) + ||f_s|| R* + margin, with R* the largest radius of the
+#     (batch, kv-head) and margin = 2^-12 ||f|| T*, T* the largest 2-norm of
+#     any of its block or node rows (room for float32 rounding of both
+#     sides).  Every unexpanded block then scores below the k-th kept score,
+#     so the kept set is the exact top-k of all visible blocks;
+#   * escalation: an uncertified row is re-routed over all its visible blocks.
+
+HIER_MARGIN = 2.0 ** -12
+
+
+def round_up_f32(x) -> np.ndarray:
+    """The least float32 >= x (x finite, float64), returned as float64."""
+    x = np.asarray(x, dtype=np.float64)
+    r = x.astype(np.float32)
+    low = r.astype(np.float64) < x
+    r = np.where(low, np.nextafter(r, np.float32(np.inf)), r)
+    return r.astype(np.float64)
+
+
+def hier_nodes(table: np.ndarray, fanout: int):
+    """Node summaries of a bf16 routing table [batch, h_kv, nb, 2d].
+
+    Returns (node_table [batch, h_kv, nn, 2d] bf16 values, radius
+    [batch, h_kv, nn], r_star [batch, h_kv], t_star [batch, h_kv]) with
+    nn = nb // fanout; r_star / t_star are 0 when there are no nodes or rows.
+    """
+    b, h, nb, kf = table.shape
+    d = kf // 2
+    M = fanout
+    nn = nb // M
+    T = np.asarray(table, dtype=np.float64)
+    nodes = T[:, :, :nn * M].reshape(b, h, nn, M, kf)
+    centre = round_bf16(round_f32(nodes[..., :d].sum(axis=3) / M))
+    cap = nodes[..., d:].max(axis=3) if nn else np.zeros((b, h, 0, d))
+    dist = np.sqrt(((nodes[..., :d] - centre[:, :, :, None, :]) ** 2).sum(axis=-1))   # [b, h, nn, M]
+    radius = round_up_f32(dist.max(axis=3)) if nn else np.zeros((b, h, 0))
+    node_table = np.concatenate([centre, cap], axis=-1)
+    r_star = radius.max(axis=2) if nn else np.zeros((b, h))
+    row_norm = np.sqrt((T ** 2).sum(axis=-1))
+    node_norm = np.sqrt((node_table ** 2).sum(axis=-1))
+    t_star = np.zeros((b, h))
+    if nb:
+        t_star = row_norm.max(axis=2)
+    if nn:
+        t_star = np.maximum(t_star, node_norm.max(axis=2))
+    return node_table, radius, round_up_f32(r_star), round_up_f32(t_star)
+
+
+def hier_route_row(f: np.ndarray, table_bg: np.ndarray, nodes_bg, pos: int, p: Problem, fanout: int,
+                   probe: int):
+    """One (query row, kv-head) through the hierarchical router.
+
+    f: the row's features [2d]; table_bg [nb, 2d]; nodes_bg = (node_table
+    [nn, 2d], radius [nn], r_star, t_star) of its (batch, kv-head).
+    Returns (kept block_idx [k] ascending padded with -1, certified,
+    info dict with the expanded nodes, the node gap and the kept-set gap).
+    """
+    node_table, _radius, r_star, t_star = nodes_bg
+    d = p.d
+    M = fanout
+    nn = node_table.shape[0]
+    nv = visible_blocks(pos, p)
+    nvn = max(0, min(nn, (pos + 1) // (M * p.block)))
+    w = node_table[:nvn] @ f
+    order = np.lexsort((np.arange(nvn), -w))
+    expanded = np.sort(order[:probe])
+    cand = [np.arange(N * M, (N + 1) * M) for N in expanded] + [np.arange(nvn * M, nv)]
+    cand = np.concatenate(cand).astype(np.int64)
+    s = table_bg[cand] @ f
+    corder = np.lexsort((cand, -s))
+    take = min(p.topk, cand.size)
+    kept = np.full(p.topk, -1, dtype=np.int64)
+    kept[:take] = np.sort(cand[corder[:take]])
+    tau = s[corder[p.topk - 1]] if cand.size >= p.topk else -np.inf
+    f_s_norm = math.sqrt(float(f[:d] @ f[:d]))
+    margin = HIER_MARGIN * math.sqrt(float(f @ f)) * t_star
+    if nvn <= probe:
+        certified, w_next, node_gap = True, -np.inf, np.inf
+    else:
+        w_next = w[order[probe]]
+        certified = bool(tau > w_next + f_s_norm * r_star + margin)
+        node_gap = w[order[probe - 1]] - w_next
+    kgap = (s[corder[p.topk - 1]] - s[corder[p.topk]]) if cand.size > p.topk else np.inf
+    info = {"expanded": expanded, "tau": tau, "bound": w_next + f_s_norm * r_star + margin,
+            "node_gap": node_gap, "kept_gap": kgap, "scale": math.sqrt(float(f @ f)) * t_star}
+    return kept, certified, info
+
+
+def hier_route(Q: np.ndarray, stored, p: Problem, fanout: int, probe: int, escalate: bool = False,
+               rows=None):
+    """block_idx [batch, n_q, h_kv, k], certified [batch, n_q, h_kv] (bool) and
+    per-row info of the hierarchical router (bf16 problems, S = 1).
+
+    escalate: uncertified rows take the flat top-k of all visible blocks.
+    rows: optional (batch, query row) pairs; other rows stay -2 / False.
+    """
+    if p.dtype != BF16 or p.subblocks != 1:
+        raise ValueError("the hierarchical router is defined on the bf16 routing table, S = 1")
+    _mu32, _sig32, table = stored
+    nodes = hier_nodes(table, fanout)
+    bidx = np.full((p.batch, p.n_q, p.h_kv, p.topk), -2, dtype=np.int64)
+    cert = np.zeros((p.batch, p.n_q, p.h_kv), dtype=bool)
+    info = {}
+    if rows is None:
+        rows = [(bi, i) for bi in range(p.batch) for i in range(p.n_q)]
+    feats = {}
+    for bi, i in rows:
+        if bi not in feats:
+            feats[bi] = route_features(Q[bi:bi + 1], p)[0]          # [h_kv, n_q, 2d]
+        pos = p.q_offset + i
+        for g in range(p.h_kv):
+            f = feats[bi][g, i]
+            nb_g = (nodes[0][bi, g], nodes[1][bi, g], nodes[2][bi, g], nodes[3][bi, g])
+            kept, ok, inf = hier_route_row(f, table[bi, g], nb_g, pos, p, fanout, probe)
+            if escalate and not ok:
+                nv = visible_blocks(pos, p)
+                kept, _gap = select_topk(table[bi, g, :nv] @ f, p.topk)
+            bidx[bi, i, g] = kept
+            cert[bi, i, g] = ok
+            info[(bi, i, g)] = inf
+    return bidx, cert, info

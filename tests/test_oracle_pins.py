@@ -505,3 +505,189 @@ def test_tempered_score_limits_and_cumulant_expansion():
     # non-decreasing in beta (power-mean inequality)
     vals = [O.tempered_block_score(q, Kc, b) for b in (0.0, 0.1, 0.5, 1.0, 2.0, 8.0, 50.0)]
     assert all(a <= b + 1e-12 for a, b in zip(vals, vals[1:]))
+
+
+# ------------------------------------------------------------------ hierarchical router
+
+def _hier_problem(rng, n=512, d=16, block=4, G=2, h_kv=2, topk=4, node_keys=None, spread=4.0):
+    """A bf16 problem and its stored summaries.  node_keys = M * block gives
+    keys drawn around one centre per node (benign geometry: blocks of a node
+    alike, nodes far apart); None gives iid keys."""
+    p = O.Problem(1, n, n, G * h_kv, h_kv, d, block, topk, block, dtype=O.BF16, sigma=O.DIAG)
+    if node_keys is None:
+        K = rng.standard_normal((1, n, h_kv, d))
+    else:
+        cen = spread * rng.standard_normal((1, n // node_keys, h_kv, d))
+        K = np.repeat(cen, node_keys, axis=1) + 0.1 * rng.standard_normal((1, n, h_kv, d))
+    K = O.round_bf16(K)
+    Q = O.round_bf16(rng.standard_normal((1, n, G * h_kv, d)))
+    stored = O.stored_summaries(*O.block_summaries(K, p), p)
+    return p, Q, stored
+
+
+def test_hier_node_bound_is_admissible_and_tight_at_fanout_one():
+    """Every block's score is at most its node's bound f.[m;v] + ||f_s|| R for
+    features with a non-negative variance half, including features aimed at
+    the farthest block; with one block per node the bound is the score."""
+    rng = np.random.default_rng(31)
+    d, nb = 8, 64
+    mu = O.round_bf16(rng.standard_normal((1, 1, nb, d)) * rng.uniform(0.1, 3.0, (1, 1, nb, 1)))
+    sg = O.round_bf16(rng.chisquare(2, (1, 1, nb, d)))
+    table = np.concatenate([mu, sg], axis=-1)
+    for M in (2, 4, 8):
+        nt, rad, r_star, _t = O.hier_nodes(table, M)
+        assert nt.shape == (1, 1, nb // M, 2 * d)
+        assert r_star[0, 0] == rad[0, 0].max()
+        for trial in range(200):
+            fs = O.round_bf16(rng.standard_normal(d) * 2)
+            fq = O.round_bf16(np.abs(rng.standard_normal(d)))
+            if trial % 4 == 0:   # aim the mean half at the block farthest from its centre
+                N = trial % (nb // M)
+                far = np.argmax(np.linalg.norm(mu[0, 0, N * M:(N + 1) * M] - nt[0, 0, N, :d], axis=1))
+                fs = O.round_bf16(mu[0, 0, N * M + far] - nt[0, 0, N, :d])
+                fq = np.zeros(d)
+            f = np.concatenate([fs, fq])
+            bound = nt[0, 0] @ f + np.linalg.norm(fs) * rad[0, 0]
+            score = (table[0, 0] @ f).reshape(nb // M, M)
+            assert np.all(score.max(axis=1) <= bound + 1e-9)
+            if trial % 4 == 0:   # Cauchy-Schwarz is attained in the aimed direction
+                N = trial % (nb // M)
+                assert score[N].max() >= bound[N] - 1e-2 * np.linalg.norm(fs) * rad[0, 0, N]
+    nt1, rad1, r1, _t = O.hier_nodes(table, 1)
+    np.testing.assert_array_equal(nt1, table)
+    np.testing.assert_array_equal(rad1, 0.0)
+    assert r1[0, 0] == 0.0
+
+
+def test_hier_nodes_shift_and_radius_invariants():
+    """Shifting every block mean by a vector shifts the node centres by it and
+    keeps radii and variance caps; the radius is the largest centre distance
+    (rounded up to float32), the cap the per-dimension maximum."""
+    rng = np.random.default_rng(32)
+    d, nb, M = 8, 32, 4
+    mu = rng.integers(-16, 16, (1, 2, nb, d)) / 4.0      # exact in bf16, and so are node means
+    sg = rng.integers(0, 64, (1, 2, nb, d)) / 8.0
+    v = rng.integers(-8, 8, d) / 2.0
+    a = O.hier_nodes(np.concatenate([mu, sg], -1), M)
+    b = O.hier_nodes(np.concatenate([mu + v, sg], -1), M)
+    np.testing.assert_array_equal(b[0][..., :d], a[0][..., :d] + v)
+    np.testing.assert_array_equal(b[0][..., d:], a[0][..., d:])
+    np.testing.assert_array_equal(b[1], a[1])
+    for g in range(2):
+        for N in range(nb // M):
+            blk = mu[0, g, N * M:(N + 1) * M]
+            np.testing.assert_array_equal(a[0][0, g, N, :d], blk.mean(axis=0))
+            np.testing.assert_array_equal(a[0][0, g, N, d:], sg[0, g, N * M:(N + 1) * M].max(axis=0))
+            dist = max(math.sqrt(sum((x - c) ** 2 for x, c in zip(row, blk.mean(axis=0)))) for row in blk)
+            r = a[1][0, g, N]
+            assert dist <= r <= dist * (1 + 2.0 ** -23)
+            assert np.float32(r) == r
+
+
+def _flat(Q, stored, p, bi, i, g):
+    f = O.route_features(Q[bi:bi + 1, i:i + 1], p)[0, g, 0]
+    nv = O.visible_blocks(p.q_offset + i, p)
+    return O.select_topk(stored[2][bi, g, :nv] @ f, p.topk)[0]
+
+
+@pytest.mark.parametrize("benign", [False, True])
+def test_hier_certified_rows_hold_the_exact_topk(benign):
+    """A certified row's kept blocks are the flat top-k of all its visible
+    blocks; on benign geometry the certificate fires on most rows, on iid keys
+    it rarely does (the bound is loose), and uncertified rows occur."""
+    rng = np.random.default_rng(33 + benign)
+    fired = total = 0
+    for M, probe, topk in ((2, 2, 4), (4, 1, 4), (4, 3, 8), (8, 2, 4)):
+        p, Q, stored = _hier_problem(rng, topk=topk, node_keys=(M * 4 if benign else None))
+        rows = [(0, i) for i in range(0, p.n_q, 3)]
+        bidx, cert, info = O.hier_route(Q, stored, p, M, probe, rows=rows)
+        for (bi, i) in rows:
+            for g in range(p.h_kv):
+                total += 1
+                if cert[bi, i, g]:
+                    fired += 1
+                    np.testing.assert_array_equal(bidx[bi, i, g], _flat(Q, stored, p, bi, i, g))
+    if benign:
+        assert fired > 0.6 * total
+    else:
+        assert fired < 0.6 * total
+    assert fired < total
+
+
+def test_hier_ranking_and_kept_set_brute_force():
+    """The expanded nodes are the probe best by w_N (ties to the lower node),
+    and the kept set is the top-k of the expanded nodes' blocks plus the
+    visible blocks outside complete nodes, by explicit enumeration."""
+    rng = np.random.default_rng(35)
+    p, Q, stored = _hier_problem(rng, n=256, topk=3)
+    M, probe = 4, 2
+    nt, rad, r_star, t_star = O.hier_nodes(stored[2], M)
+    f_all = O.route_features(Q, p)[0]
+    for i in range(0, 256, 7):
+        for g in range(p.h_kv):
+            f = f_all[g, i]
+            pos = i
+            nvn = min(nt.shape[2], (pos + 1) // (M * p.block))
+            nv = O.visible_blocks(pos, p)
+            w = [(-(nt[0, g, N] @ f), N) for N in range(nvn)]
+            exp = sorted(N for _, N in sorted(w)[:probe])
+            kept, ok, info = O.hier_route_row(f, stored[2][0, g], (nt[0, g], rad[0, g], r_star[0, g], t_star[0, g]),
+                                              pos, p, M, probe)
+            assert list(info["expanded"]) == exp
+            cand = [c for N in exp for c in range(N * M, N * M + M)] + list(range(nvn * M, nv))
+            ranked = sorted(cand, key=lambda c: (-(stored[2][0, g, c] @ f), c))
+            want = sorted(ranked[:p.topk]) + [-1] * max(0, p.topk - len(cand))
+            assert list(kept) == want
+            if nvn <= probe:
+                assert ok
+
+
+def test_hier_full_probe_and_escalation_equal_flat_and_twins_never_certify():
+    rng = np.random.default_rng(36)
+    p, Q, stored = _hier_problem(rng, n=256, topk=4)
+    flat, _ = O.route_topk(Q, stored, p)
+    M = 4
+    nn = p.nb // M
+    b1, c1, _ = O.hier_route(Q, stored, p, M, nn)            # every node expanded
+    np.testing.assert_array_equal(b1, flat)
+    assert c1.all()
+    b2, c2, _ = O.hier_route(Q, stored, p, M, 1, escalate=True)
+    np.testing.assert_array_equal(b2, flat)
+    assert not c2.all()
+    # two identical nodes: expanding one can never rule out the other
+    tw = stored[2].copy()
+    tw[:, :, 4:8] = tw[:, :, 0:4]
+    st2 = (stored[0], stored[1], tw)
+    _b, c3, info = O.hier_route(Q, st2, p, M, 1, rows=[(0, i) for i in range(64, 256)])
+    for i in range(64, 256):
+        for g in range(p.h_kv):
+            if list(info[(0, i, g)]["expanded"]) in ([0], [1]) and ((i + 1) // (M * p.block)) > 1:
+                assert not c3[0, i, g]
+
+
+def test_hier_certificate_hand_cases_radius_and_margin():
+    """Hand-computed rows (d = 2, one key per block, the whole sequence visible).
+
+    Radius: nodes {b0, b1} with means (1,0), (1,0) and {b2, b3} with (-0.5,0),
+    (1.5,0); f = [1, 0 ; 0, 0].  Node 0: centre (1,0), R = 0, w = 1; node 1:
+    centre (0.5,0), R = 1, w = 0.5.  Probe 1 expands node 0, k = 1 keeps b0 with
+    tau = 1, but the bound of node 1 is 0.5 + 1 * 1 = 1.5 > 1: not certified --
+    rightly, b3 scores 1.5.
+    Margin: one block per node, means (1,1) and (1,0), f = [1, e ; 0, 0]:
+    tau = 1 + e against w_next = 1, R* = 0, margin = 2^-12 ||f|| sqrt(2);
+    e = 2^-12 is inside the margin (not certified), e = 2^-10 outside it."""
+    def row(table, f, M, probe, k):
+        nb = table.shape[0]
+        p = O.Problem(1, nb, nb, 1, 1, 2, 1, k, 1, dtype=O.BF16, sigma=O.DIAG)
+        nt, rad, rs, ts = O.hier_nodes(table[None, None], M)
+        return O.hier_route_row(np.asarray(f, float), table, (nt[0, 0], rad[0, 0], rs[0, 0], ts[0, 0]),
+                                nb - 1, p, M, probe)
+    t = np.array([[1, 0, 0, 0], [1, 0, 0, 0], [-0.5, 0, 0, 0], [1.5, 0, 0, 0]], float)
+    kept, ok, info = row(t, [1, 0, 0, 0], 2, 1, 1)
+    assert list(info["expanded"]) == [0] and list(kept) == [0] and info["tau"] == 1.0
+    assert info["bound"] == pytest.approx(1.5 + 2.0 ** -12 * 1.5)
+    assert not ok
+    t2 = np.array([[1, 1, 0, 0], [1, 0, 0, 0]], float)
+    for e, want in ((2.0 ** -12, False), (2.0 ** -10, True)):
+        kept, ok, info = row(t2, [1, e, 0, 0], 1, 1, 1)
+        assert list(kept) == [0] and ok is want
