@@ -39,12 +39,20 @@ class ssa_params(C.Structure):
 assert C.sizeof(ssa_params) == 72
 
 
+class ssa_hier_params(C.Structure):
+    _fields_ = [("fanout", C.c_int32), ("probe", C.c_int32), ("escalate", C.c_int32), ("reserved", C.c_int32)]
+
+
+assert C.sizeof(ssa_hier_params) == 16
+
+
 def _load():
     if not os.path.exists(_LIB_PATH):
         raise ImportError(f"{_LIB_PATH} is missing: build it with "
                           "`python -m content_routed_block_ssa_b200.build` (nvcc, sm_100a)")
     lib = C.CDLL(_LIB_PATH)
     P = C.POINTER(ssa_params)
+    H = C.POINTER(ssa_hier_params)
     vp, sz, i32 = C.c_void_p, C.c_size_t, C.c_int32
     sig = {
         "ssa_status_string": (C.c_char_p, [i32]),
@@ -65,6 +73,10 @@ def _load():
         "ssa_forward": (i32, [P, vp, vp, vp, vp, vp, vp, sz, vp]),
         "ssa_hostio_buffer_size": (sz, [P]),
         "ssa_forward_hostio": (i32, [P, vp, vp, vp, vp, vp, vp, sz, vp]),
+        "ssa_hier_nodes_size": (sz, [P, H]),
+        "ssa_hier_nodes": (i32, [P, H, vp, vp, vp]),
+        "ssa_route_hier_workspace_size": (sz, [P, H]),
+        "ssa_route_hier": (i32, [P, H, vp, vp, vp, vp, vp, vp, sz, vp]),
     }
     for name, (res, args) in sig.items():
         f = getattr(lib, name)
@@ -79,7 +91,8 @@ EXPORTED = ("ssa_status_string", "ssa_version", "ssa_launch_count", "ssa_device_
             "ssa_block_summary", "ssa_route_workspace_size", "ssa_route_topk", "ssa_route_topk_static",
             "ssa_attn_workspace_size", "ssa_sparse_attn", "ssa_attn_plan", "ssa_attn_blocks",
             "ssa_attn_window", "ssa_attn_merge",
-            "ssa_workspace_size", "ssa_forward", "ssa_hostio_buffer_size", "ssa_forward_hostio")
+            "ssa_workspace_size", "ssa_forward", "ssa_hostio_buffer_size", "ssa_forward_hostio",
+            "ssa_hier_nodes_size", "ssa_hier_nodes", "ssa_route_hier_workspace_size", "ssa_route_hier")
 
 
 def status_string(s: int) -> str:
@@ -227,3 +240,43 @@ def idx_shape(p):
 def byte_buffer(nbytes: int, device="cuda"):
     """A caller-owned uint8 buffer (workspaces are allocated by the caller)."""
     return torch.empty(max(int(nbytes), 16), dtype=torch.uint8, device=device)
+
+
+def make_hier_params(fanout=16, probe=2, escalate=False) -> ssa_hier_params:
+    """An ssa_hier_params struct: nodes of `fanout` blocks, `probe` nodes expanded per row."""
+    return ssa_hier_params(fanout=fanout, probe=probe, escalate=1 if escalate else 0, reserved=0)
+
+
+def ssa_hier_nodes_size(p, hp) -> int:
+    return int(lib.ssa_hier_nodes_size(C.byref(p), C.byref(hp)))
+
+
+def ssa_hier_nodes(p, hp, route_table, nodes, stream=None):
+    _check(lib.ssa_hier_nodes(C.byref(p), C.byref(hp), _ptr(route_table), _ptr(nodes), _stream(stream)),
+           "ssa_hier_nodes")
+
+
+def ssa_route_hier_workspace_size(p, hp) -> int:
+    return int(lib.ssa_route_hier_workspace_size(C.byref(p), C.byref(hp)))
+
+
+def ssa_route_hier(p, hp, Q, route_table, nodes, block_idx, certified=None, ws=None, stream=None):
+    _check(lib.ssa_route_hier(C.byref(p), C.byref(hp), _ptr(Q), _ptr(route_table), _ptr(nodes), _ptr(block_idx),
+                              _ptr(certified), _ptr(ws), _nbytes(ws), _stream(stream)), "ssa_route_hier")
+
+
+def hier_node_views(p, hp, nodes):
+    """(node rows [b, h_kv, nn, 2d] bf16, radii [b, h_kv, nn] f32, bounds [b, h_kv, 2] f32) views of a
+    node store (a uint8 device tensor of ssa_hier_nodes_size bytes)."""
+    nn = (p.n_kv // p.block) // hp.fanout
+    bgs = p.batch * p.h_kv
+
+    def ru(x):
+        return (x + 255) // 256 * 256
+    t_bytes = bgs * nn * 2 * p.d * 2
+    r_off = ru(t_bytes)
+    b_off = r_off + ru(bgs * nn * 4)
+    rows = nodes[:t_bytes].view(torch.bfloat16).view(p.batch, p.h_kv, nn, 2 * p.d)
+    rad = nodes[r_off:r_off + bgs * nn * 4].view(torch.float32).view(p.batch, p.h_kv, nn)
+    bnd = nodes[b_off:b_off + bgs * 8].view(torch.float32).view(p.batch, p.h_kv, 2)
+    return rows, rad, bnd

@@ -1,0 +1,335 @@
+// Hierarchical routing: a tree level of nodes over the block summaries, a
+// per-row probe of the best nodes, and the row's certificate.
+//
+// The page "Subquadratic Sparse Attention (SSA)" names a tree router with a
+// recursive radius (artifact list, Barnes-Hut style), branch-and-bound exact
+// selection under an admissible bound (same list) and per-query certificates
+// with escalation ("Certified Causal Cascade" entry), without fixing their
+// rules.  The rules built here:
+//
+//   node N = blocks N*M .. N*M+M-1 (complete nodes only), summarised from the
+//   blocks' bf16 routing rows T_c = [mu_c ; s_c] by
+//     centre m_N = bf16(f32(mean_c mu_c)),  cap v_N = max_c s_c (per dim),
+//     radius R_N = max_c ||mu_c - m_N||_2   (float64, rounded up to float32);
+//   for features f = [f_s ; f_q] with f_q >= 0 every block of N scores
+//     f . T_c <= f . [m_N ; v_N] + ||f_s|| R_N.
+//
+// A row ranks its complete visible nodes by w_N = f . [m_N ; v_N] (the
+// tensor-core router run over the node table, top probe+1 with scores),
+// scores the blocks of the best `probe` nodes and the visible blocks outside
+// complete nodes exactly, and keeps their top-k.  It is certified when no
+// complete visible node is left, or when the k-th kept score exceeds
+// w_(probe+1) + ||f_s|| R* + 2^-12 ||f|| T* (R*: largest radius, T*: largest
+// row 2-norm of the (batch, kv-head); the last term covers float32 rounding
+// of both scores): every unexpanded block then scores below the kept set, so
+// the kept set is the exact top-k.
+#include <cuda_bf16.h>
+#include <math.h>
+
+#include "common.cuh"
+#include "kernels.h"
+
+namespace ssa {
+namespace {
+
+// Lane l holds elements [FPL*l, FPL*l + FPL) of a 2D-long routing row:
+// lanes 0..15 the mean half, lanes 16..31 the variance half.
+template <int FPL>
+__device__ __forceinline__ void load_slice(const __nv_bfloat16* p, float (&v)[FPL]) {
+  if constexpr (FPL == 8) {
+    const uint4 raw = __ldg(reinterpret_cast<const uint4*>(p));
+    const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      v[2 * j] = __uint_as_float(w[j] << 16);
+      v[2 * j + 1] = __uint_as_float(w[j] & 0xFFFF0000u);
+    }
+  } else {
+    const uint2 raw = __ldg(reinterpret_cast<const uint2*>(p));
+    const uint32_t w[2] = {raw.x, raw.y};
+#pragma unroll
+    for (int j = 0; j < 2; ++j) {
+      v[2 * j] = __uint_as_float(w[j] << 16);
+      v[2 * j + 1] = __uint_as_float(w[j] & 0xFFFF0000u);
+    }
+  }
+}
+
+template <int FPL>
+__device__ __forceinline__ void store_slice(__nv_bfloat16* p, const float (&v)[FPL]) {
+  uint32_t w[FPL / 2];
+#pragma unroll
+  for (int j = 0; j < FPL / 2; ++j)
+    w[j] = static_cast<uint32_t>(__bfloat16_as_ushort(__float2bfloat16_rn(v[2 * j]))) |
+           (static_cast<uint32_t>(__bfloat16_as_ushort(__float2bfloat16_rn(v[2 * j + 1]))) << 16);
+  if constexpr (FPL == 8)
+    *reinterpret_cast<uint4*>(p) = make_uint4(w[0], w[1], w[2], w[3]);
+  else
+    *reinterpret_cast<uint2*>(p) = make_uint2(w[0], w[1]);
+}
+
+__device__ __forceinline__ double warp_sum_d(double x) {
+#pragma unroll
+  for (int o = 16; o; o >>= 1) x += __shfl_xor_sync(0xFFFFFFFFu, x, o);
+  return x;
+}
+
+__device__ __forceinline__ float warp_sum_f(float x) {
+#pragma unroll
+  for (int o = 16; o; o >>= 1) x += __shfl_xor_sync(0xFFFFFFFFu, x, o);
+  return x;
+}
+
+__device__ __forceinline__ uint64_t warp_max_u64(uint64_t x) {
+#pragma unroll
+  for (int o = 16; o; o >>= 1) {
+    const uint64_t y = __shfl_xor_sync(0xFFFFFFFFu, x, o);
+    x = y > x ? y : x;
+  }
+  return x;
+}
+
+__device__ __forceinline__ uint64_t warp_min_u64(uint64_t x) {
+#pragma unroll
+  for (int o = 16; o; o >>= 1) {
+    const uint64_t y = __shfl_xor_sync(0xFFFFFFFFu, x, o);
+    x = y < x ? y : x;
+  }
+  return x;
+}
+
+// ------------------------------------------------------------------ nodes
+
+// One warp per (batch * kv-head, node); node index nn covers the trailing
+// blocks that belong to no complete node (their row norms only).
+template <int D>
+__global__ void __launch_bounds__(256) hier_nodes_kernel(const HierNodeArgs a) {
+  constexpr int FPL = 2 * D / 32;
+  const int lane = threadIdx.x & 31;
+  const int64_t w = static_cast<int64_t>(blockIdx.x) * 8 + threadIdx.x / 32;
+  if (w >= static_cast<int64_t>(a.bgs) * (a.nn + 1)) return;
+  const int bg = static_cast<int>(w / (a.nn + 1)), N = static_cast<int>(w % (a.nn + 1));
+  const bool mean_half = lane < 16;
+  const __nv_bfloat16* trow = a.T + static_cast<int64_t>(bg) * a.nb * (2 * D) + lane * FPL;
+  const int c0 = N * a.M;
+  const int c1 = N < a.nn ? c0 + a.M : a.nb;
+  double sum[FPL];
+  float cap[FPL];
+#pragma unroll
+  for (int e = 0; e < FPL; ++e) { sum[e] = 0.0; cap[e] = -INFINITY; }
+  double row2max = 0.0;
+  for (int c = c0; c < c1; ++c) {
+    float v[FPL];
+    load_slice<FPL>(trow + static_cast<int64_t>(c) * (2 * D), v);
+    double r2 = 0.0;
+#pragma unroll
+    for (int e = 0; e < FPL; ++e) {
+      r2 += static_cast<double>(v[e]) * v[e];
+      sum[e] += v[e];
+      cap[e] = fmaxf(cap[e], v[e]);
+    }
+    row2max = fmax(row2max, warp_sum_d(r2));
+  }
+  if (N < a.nn) {
+    float m[FPL];
+#pragma unroll
+    for (int e = 0; e < FPL; ++e)   // sum / M is exact (M a power of two)
+      m[e] = mean_half ? __bfloat162float(__float2bfloat16_rn(__double2float_rn(sum[e] / a.M))) : cap[e];
+    store_slice<FPL>(a.NT + (static_cast<int64_t>(bg) * a.nn + N) * (2 * D) + lane * FPL, m);
+    double n2 = 0.0;
+#pragma unroll
+    for (int e = 0; e < FPL; ++e) n2 += static_cast<double>(m[e]) * m[e];
+    row2max = fmax(row2max, warp_sum_d(n2));
+    double d2max = 0.0;
+    for (int c = c0; c < c1; ++c) {
+      float v[FPL];
+      load_slice<FPL>(trow + static_cast<int64_t>(c) * (2 * D), v);
+      double d2 = 0.0;
+#pragma unroll
+      for (int e = 0; e < FPL; ++e) {
+        const double t = static_cast<double>(v[e]) - m[e];
+        d2 += mean_half ? t * t : 0.0;
+      }
+      d2max = fmax(d2max, warp_sum_d(d2));
+    }
+    const float R = __double2float_ru(sqrt(d2max));
+    if (lane == 0) {
+      a.radius[static_cast<int64_t>(bg) * a.nn + N] = R;
+      atomicMax(&a.bound[2 * bg], __float_as_uint(R));   // non-negative floats order as their bits
+    }
+  }
+  if (lane == 0) atomicMax(&a.bound[2 * bg + 1], __float_as_uint(__double2float_ru(sqrt(row2max))));
+}
+
+// ------------------------------------------------------------------ probe
+
+constexpr int kProbeMaxCand = 512;   // (probe + 1) * M
+constexpr int kProbeWarps = 8;
+
+// One warp per (batch * kv-head, query row).
+template <int D>
+__global__ void __launch_bounds__(256) hier_probe_kernel(const HierProbeArgs a) {
+  constexpr int FPL = 2 * D / 32;
+  __shared__ uint64_t keys_all[kProbeWarps][kProbeMaxCand];
+  const int lane = threadIdx.x & 31;
+  uint64_t* keys = keys_all[threadIdx.x / 32];
+  const int64_t w = static_cast<int64_t>(blockIdx.x) * kProbeWarps + threadIdx.x / 32;
+  if (w >= static_cast<int64_t>(a.bgs) * a.n_q) return;
+  const int bg = static_cast<int>(w / a.n_q), i = static_cast<int>(w % a.n_q);
+  const int b = bg / a.h_kv, g = bg % a.h_kv;
+  const int64_t pos = a.q_offset + i;
+  const int nv = static_cast<int>(min(static_cast<int64_t>(a.nb), (pos + 1) / a.block));
+  const int nvn = static_cast<int>(min(static_cast<int64_t>(a.nn), (pos + 1) / (static_cast<int64_t>(a.block) * a.M)));
+  const int64_t row = (static_cast<int64_t>(b) * a.n_q + i) * a.h_kv + g;
+
+  float f[FPL];
+  load_slice<FPL>(a.F + (static_cast<int64_t>(bg) * a.n_q + i) * (2 * D) + lane * FPL, f);
+  float f2 = 0.f;
+#pragma unroll
+  for (int e = 0; e < FPL; ++e) f2 = __fmaf_rn(f[e], f[e], f2);
+  const float fs2 = warp_sum_f(lane < 16 ? f2 : 0.f);
+  f2 = warp_sum_f(f2);
+
+  // the node router's probe+1 best nodes (ascending node index, -1 padded)
+  const int P1 = a.probe + 1;
+  int nidx = -1;
+  float nsc = -INFINITY;
+  if (nvn > 0 && lane < P1) {
+    nidx = a.node_idx[row * P1 + lane];
+    nsc = a.node_score[row * P1 + lane];
+  }
+  const bool complete = nvn <= a.probe;   // every complete visible node gets expanded
+  const int nvalid = __popc(__ballot_sync(0xFFFFFFFFu, nidx >= 0 && nidx < nvn));
+  bool list_ok = complete ? nvalid == nvn : nvalid == P1;
+  // when the list is full, its last entry under (score desc, index asc) stays
+  // unexpanded and its score is the largest w_N of all unexpanded nodes
+  const uint64_t k = (nidx >= 0 && nidx < nvn) ? make_key(__float_as_uint(nsc), nidx) : ~0ull;
+  const uint64_t kmin = warp_min_u64(k);
+  const int excl = complete ? -1 : static_cast<int>(key_block(kmin));
+  const float w_next = complete ? -INFINITY : key_score(kmin);
+  const bool expd = nidx >= 0 && nidx < nvn && nidx != excl;
+  const uint32_t emask = __ballot_sync(0xFFFFFFFFu, expd);
+  const int nexp = __popc(emask);
+  int my_exp = 0;   // lane j < nexp: the j-th expanded node (ascending)
+  {
+    uint32_t m = emask;
+    for (int t = 0; t < lane && m; ++t) m &= m - 1u;   // drop the j lowest set bits
+    const int src = (lane < nexp && m) ? __ffs(static_cast<int>(m)) - 1 : 0;
+    my_exp = __shfl_sync(0xFFFFFFFFu, nidx, src);
+  }
+  const int log2M = __ffs(a.M) - 1;
+  const int nexpb = nexp << log2M;
+  const int n_cand = nexpb + (nv - nvn * a.M);
+
+  // exact scores of the candidates, 32 at a time: lane u accumulates its
+  // slice of candidate t0+u, then a transposing butterfly leaves the whole
+  // score of candidate t0+l in lane l
+  const __nv_bfloat16* tb = a.T + static_cast<int64_t>(bg) * a.nb * (2 * D) + lane * FPL;
+  for (int t0 = 0; t0 < n_cand; t0 += 32) {
+    float acc[32];
+#pragma unroll
+    for (int u = 0; u < 32; ++u) {
+      const int t = t0 + u;
+      const int node = __shfl_sync(0xFFFFFFFFu, my_exp, min(t >> log2M, 31));
+      acc[u] = 0.f;
+      if (t < n_cand) {
+        const int c = t < nexpb ? (node << log2M) + (t & (a.M - 1)) : nvn * a.M + (t - nexpb);
+        float v[FPL];
+        load_slice<FPL>(tb + static_cast<int64_t>(c) * (2 * D), v);
+#pragma unroll
+        for (int e = 0; e < FPL; ++e) acc[u] = __fmaf_rn(f[e], v[e], acc[u]);
+      }
+    }
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) {
+      const bool up = (lane & o) != 0;
+#pragma unroll
+      for (int u = 0; u < o; ++u) {
+        const float send = up ? acc[u] : acc[u + o];
+        const float keep = up ? acc[u + o] : acc[u];
+        acc[u] = keep + __shfl_xor_sync(0xFFFFFFFFu, send, o);
+      }
+    }
+    const int t = t0 + lane;
+    const int node = __shfl_sync(0xFFFFFFFFu, my_exp, min(t >> log2M, 31));
+    if (t < n_cand) {
+      const int c = t < nexpb ? (node << log2M) + (t & (a.M - 1)) : nvn * a.M + (t - nexpb);
+      keys[t] = make_key(__float_as_uint(acc[0]), static_cast<uint32_t>(c));
+    }
+  }
+  __syncwarp();
+
+  // top-k under (score desc, block asc): k rounds of a warp arg-max
+  uint64_t kept = 0;
+  int nkept = 0;
+  for (int j = 0; j < a.topk; ++j) {
+    uint64_t m = 0;
+    int at = -1;
+    for (int t = lane; t < n_cand; t += 32) {
+      const uint64_t x = keys[t];
+      if (x > m) { m = x; at = t; }
+    }
+    const uint64_t best = warp_max_u64(m);
+    if (best == 0) break;
+    if (at >= 0 && m == best) keys[at] = 0;
+    __syncwarp();
+    if (lane == j) kept = best;
+    ++nkept;
+  }
+  const uint64_t kth = __shfl_sync(0xFFFFFFFFu, kept, max(a.topk - 1, 0));
+  const float tau = nkept == a.topk ? key_score(kth) : -INFINITY;
+  const float bound = w_next + sqrtf(fs2) * a.bound[2 * bg] + 0x1p-12f * sqrtf(f2) * a.bound[2 * bg + 1];
+  const bool certified = list_ok && (complete || tau > bound);
+
+  // kept blocks in ascending order, -1 padded
+  const uint32_t blk = (lane < nkept) ? key_block(kept) : 0xFFFFFFFFu;
+  int rank = 0;
+#pragma unroll 8
+  for (int o = 0; o < 32; ++o) rank += (__shfl_sync(0xFFFFFFFFu, blk, o) < blk) ? 1 : 0;
+  if (lane < a.topk) {
+    int32_t* out = a.block_idx + row * a.topk;
+    if (lane < nkept)
+      out[rank] = static_cast<int32_t>(blk);
+    else
+      out[lane] = -1;
+  }
+  if (lane == 0) {
+    if (a.cert) a.cert[row] = certified ? 1 : 0;
+    if (!certified && a.unit_need) a.unit_need[static_cast<int64_t>(bg) * a.n_tiles + i / 256] = 1;
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_hier_nodes(const ssa_params& p, const HierNodeArgs& a, const LaunchCtx& c) {
+  const int64_t warps = static_cast<int64_t>(a.bgs) * (a.nn + 1);
+  const int64_t grid = (warps + 7) / 8;
+  if (grid == 0) return cudaSuccess;
+  if (grid > 2147483647) return cudaErrorInvalidValue;
+  if (p.d == 128)
+    hier_nodes_kernel<128><<<static_cast<unsigned>(grid), 256, 0, c.stream>>>(a);
+  else if (p.d == 64)
+    hier_nodes_kernel<64><<<static_cast<unsigned>(grid), 256, 0, c.stream>>>(a);
+  else
+    return cudaErrorInvalidValue;
+  note_launch();
+  return cudaGetLastError();
+}
+
+cudaError_t launch_hier_probe(const ssa_params& p, const HierProbeArgs& a, const LaunchCtx& c) {
+  const int64_t warps = static_cast<int64_t>(a.bgs) * a.n_q;
+  const int64_t grid = (warps + kProbeWarps - 1) / kProbeWarps;
+  if (grid == 0) return cudaSuccess;
+  if (grid > 2147483647) return cudaErrorInvalidValue;
+  if ((a.probe + 1) * a.M > kProbeMaxCand || a.topk > 32 || a.probe + 1 > 32) return cudaErrorInvalidValue;
+  if (p.d == 128)
+    hier_probe_kernel<128><<<static_cast<unsigned>(grid), kProbeWarps * 32, 0, c.stream>>>(a);
+  else if (p.d == 64)
+    hier_probe_kernel<64><<<static_cast<unsigned>(grid), kProbeWarps * 32, 0, c.stream>>>(a);
+  else
+    return cudaErrorInvalidValue;
+  note_launch();
+  return cudaGetLastError();
+}
+
+}  // namespace ssa

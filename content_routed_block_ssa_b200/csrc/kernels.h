@@ -3,6 +3,7 @@
 #pragma once
 
 #include <cuda.h>
+#include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -29,11 +30,13 @@ cudaError_t launch_features(const ssa_params& p, const void* Q, void* F, const L
 
 // step (i): tcgen05 tile router with fused streaming top-k
 cudaError_t launch_route_tiled(const ssa_params& p, const CUtensorMap& tmF, const CUtensorMap& tmT,
-                               int32_t* block_idx, float* top_scores, const LaunchCtx& c);
+                               int32_t* block_idx, float* top_scores, const LaunchCtx& c,
+                               const int32_t* unit_need = nullptr);
 
 // step (i): one CTA per query row (bf16 table)
 cudaError_t launch_route_rowwise_bf16(const ssa_params& p, const void* Q, const void* table,
-                                      int32_t* block_idx, float* top_scores, const LaunchCtx& c);
+                                      int32_t* block_idx, float* top_scores, const LaunchCtx& c,
+                                      const uint8_t* skip = nullptr);
 
 // step (i): one CTA per query row (float32 summaries, diagonal or full)
 cudaError_t launch_route_rowwise_f32(const ssa_params& p, const void* Q, const float* mu,
@@ -98,6 +101,33 @@ cudaError_t launch_attn_window(const ssa_params& p, const BlockPlan& pl, const C
 // Per (query, kv-head): the softmax merge of the slot partials into O, lse.
 cudaError_t launch_attn_merge(const ssa_params& p, const int32_t* block_idx, const void* partO, const void* partL,
                               void* O, float* lse, int32_t* bad, const LaunchCtx& c);
+
+// Hierarchical routing (hier.cu).  Node summaries of the bf16 routing table:
+// one warp per (batch * kv-head, node).
+struct HierNodeArgs {
+  int32_t bgs, nb, nn, M;      // M blocks per node, nn = nb / M complete nodes
+  const __nv_bfloat16* T;      // [bgs, nb, 2d] block routing rows
+  __nv_bfloat16* NT;           // [bgs, nn, 2d] node rows [centre ; cap]
+  float* radius;               // [bgs, nn]
+  uint32_t* bound;             // [bgs, 2] float bits (largest radius, largest row norm); zeroed first
+};
+cudaError_t launch_hier_nodes(const ssa_params& p, const HierNodeArgs& a, const LaunchCtx& c);
+
+// The per-row probe of the best nodes and the certificate: one warp per
+// (batch * kv-head, query row).
+struct HierProbeArgs {
+  int32_t n_q, h_kv, bgs, nb, nn, M, block, topk, probe, n_tiles;
+  int64_t q_offset;
+  const __nv_bfloat16* F;      // [bgs, n_q, 2d] routing features
+  const __nv_bfloat16* T;      // [bgs, nb, 2d] block routing rows
+  const int32_t* node_idx;     // [b, n_q, h_kv, probe+1] best nodes, ascending, -1 padded
+  const float* node_score;     // same layout, their scores f . [centre ; cap]
+  const float* bound;          // [bgs, 2]
+  int32_t* block_idx;          // [b, n_q, h_kv, topk]
+  uint8_t* cert;               // [b, n_q, h_kv] (may be null)
+  int32_t* unit_need;          // [bgs, n_tiles] set to 1 for units holding an uncertified row (may be null)
+};
+cudaError_t launch_hier_probe(const ssa_params& p, const HierProbeArgs& a, const LaunchCtx& c);
 
 int attn_block_smem_bytes(int block);
 

@@ -83,7 +83,14 @@ struct RouteTiledArgs {
   int32_t* block_idx;
   float* top_scores;
   uint32_t* err;
+  // optional [batch * h_kv * n_tiles] flags: units whose flag is 0 are
+  // skipped (every role reads the same flag; no output is written for them)
+  const int32_t* unit_need;
 };
+
+__device__ __forceinline__ bool unit_skipped(const RouteTiledArgs& a, int bg, int row0) {
+  return a.unit_need && a.unit_need[bg * a.n_tiles + row0 / 256] == 0;
+}
 
 template <int KF>
 struct TiledCfg {
@@ -286,7 +293,7 @@ __global__ void __launch_bounds__(TiledCfg<KF>::THREADS, 1)
         if (r >= a.n_units) break;
         int bg, row0, nch;
         route_unit(a, r, bg, row0, nch);
-        if (nch == 0) continue;
+        if (nch == 0 || unit_skipped(a, bg, row0)) continue;
         const int ab = a_cnt % C::NAB;
         if (!mbar_wait(&a_empty[ab], ((a_cnt / C::NAB) & 1) ^ 1, a.err, SITE_ROUTE_PRODUCER)) { ok = false; break; }
         mbar_arrive_expect_tx(&a_full[ab], C::A_BYTES);
@@ -328,7 +335,7 @@ __global__ void __launch_bounds__(TiledCfg<KF>::THREADS, 1)
         if (r >= a.n_units) break;
         int bg, row0, nch;
         route_unit(a, r, bg, row0, nch);
-        if (nch == 0) continue;
+        if (nch == 0 || unit_skipped(a, bg, row0)) continue;
         const int ab = a_cnt % C::NAB;
         if (!mbar_wait(&a_full[ab], (a_cnt / C::NAB) & 1, a.err, SITE_ROUTE_MMA)) { ok = false; break; }
         tc_fence_after();
@@ -381,6 +388,7 @@ __global__ void __launch_bounds__(TiledCfg<KF>::THREADS, 1)
       if (r >= a.n_units) break;
       int bg, row0, nch;
       route_unit(a, r, bg, row0, nch);
+      if (unit_skipped(a, bg, row0)) continue;
       const int i = row0 + grp * 128 + row;
       const bool valid = i < a.n_q;
       const int nvis = valid ? static_cast<int>(min(static_cast<int64_t>(a.nb), (a.q_offset + i + 1) / a.block)) : 0;
@@ -453,7 +461,7 @@ __global__ void __launch_bounds__(TiledCfg<KF>::THREADS, 1)
 
 template <int KF, int KSEL>
 cudaError_t run_tiled(const ssa_params& p, const CUtensorMap& tmF, const CUtensorMap& tmT,
-                      int32_t* idx, float* scores, const LaunchCtx& c) {
+                      int32_t* idx, float* scores, const int32_t* unit_need, const LaunchCtx& c) {
   using C = TiledCfg<KF>;
   RouteTiledArgs a;
   a.batch = p.batch; a.n_q = p.n_q; a.h_kv = p.h_kv; a.nb = p.n_kv / p.block;
@@ -462,6 +470,7 @@ cudaError_t run_tiled(const ssa_params& p, const CUtensorMap& tmF, const CUtenso
   a.n_units = p.batch * p.h_kv * a.n_tiles;
   a.q_offset = p.q_offset;
   a.block_idx = idx; a.top_scores = scores; a.err = c.err;
+  a.unit_need = unit_need;
   cudaError_t e = cudaFuncSetAttribute(route_tiled_kernel<KF, KSEL>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
   if (e != cudaSuccess) return e;
@@ -480,6 +489,7 @@ struct RowArgs {
   float half_beta;
   int32_t* block_idx;
   float* top_scores;
+  const uint8_t* skip;       // optional [b, n_q, h_kv]: rows whose byte is nonzero are skipped
 };
 
 __device__ __forceinline__ int next_pow2(int x) {
@@ -534,6 +544,7 @@ __global__ void __launch_bounds__(256) route_rowwise_bf16_kernel(const __nv_bflo
   constexpr int FPL = 2 * D / 32;   // features per lane: 8 (d=128) or 4 (d=64)
   extern __shared__ uint64_t keys[];
   const int i = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
+  if (a.skip && a.skip[(static_cast<int64_t>(b) * a.n_q + i) * a.h_kv + g]) return;   // whole CTA
   const int lane = threadIdx.x % 32, warp = threadIdx.x / 32;
   const int64_t pos = a.q_offset + i;
   const int nvis = static_cast<int>(min(static_cast<int64_t>(a.nb), (pos + 1) / a.block));
@@ -801,6 +812,7 @@ RowArgs row_args(const ssa_params& p, int32_t* idx, float* scores) {
   a.q_offset = p.q_offset;
   a.half_beta = p.beta * 0.5f;   // exact
   a.block_idx = idx; a.top_scores = scores;
+  a.skip = nullptr;
   return a;
 }
 
@@ -835,26 +847,28 @@ int row_smem_bytes(const ssa_params& p) {
 
 template <int D, int G>
 cudaError_t run_rowwise_bf16(const ssa_params& p, const void* Q, const void* T, int32_t* idx,
-                             float* scores, const LaunchCtx& c) {
+                             float* scores, const uint8_t* skip, const LaunchCtx& c) {
+  RowArgs ra = row_args(p, idx, scores);
+  ra.skip = skip;
   const int smem = row_smem_bytes(p);
   cudaError_t e = cudaFuncSetAttribute(route_rowwise_bf16_kernel<D, G>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   dim3 grid(p.n_q, p.h_kv, p.batch);
   route_rowwise_bf16_kernel<D, G><<<grid, 256, smem, c.stream>>>(
-      static_cast<const __nv_bfloat16*>(Q), static_cast<const __nv_bfloat16*>(T), row_args(p, idx, scores));
+      static_cast<const __nv_bfloat16*>(Q), static_cast<const __nv_bfloat16*>(T), ra);
   note_launch();
   return cudaGetLastError();
 }
 
 template <int D>
 cudaError_t rowwise_bf16_g(const ssa_params& p, const void* Q, const void* T, int32_t* idx,
-                           float* scores, const LaunchCtx& c) {
+                           float* scores, const uint8_t* skip, const LaunchCtx& c) {
   switch (p.h_q / p.h_kv) {
-    case 1: return run_rowwise_bf16<D, 1>(p, Q, T, idx, scores, c);
-    case 2: return run_rowwise_bf16<D, 2>(p, Q, T, idx, scores, c);
-    case 4: return run_rowwise_bf16<D, 4>(p, Q, T, idx, scores, c);
-    case 8: return run_rowwise_bf16<D, 8>(p, Q, T, idx, scores, c);
+    case 1: return run_rowwise_bf16<D, 1>(p, Q, T, idx, scores, skip, c);
+    case 2: return run_rowwise_bf16<D, 2>(p, Q, T, idx, scores, skip, c);
+    case 4: return run_rowwise_bf16<D, 4>(p, Q, T, idx, scores, skip, c);
+    case 8: return run_rowwise_bf16<D, 8>(p, Q, T, idx, scores, skip, c);
   }
   return cudaErrorInvalidValue;
 }
@@ -921,25 +935,25 @@ cudaError_t launch_features(const ssa_params& p, const void* Q, void* F, const L
 }
 
 cudaError_t launch_route_tiled(const ssa_params& p, const CUtensorMap& tmF, const CUtensorMap& tmT,
-                               int32_t* idx, float* scores, const LaunchCtx& c) {
+                               int32_t* idx, float* scores, const LaunchCtx& c, const int32_t* unit_need) {
   const int ksel = p.topk <= 8 ? 8 : (p.topk <= 16 ? 16 : 32);
   if (p.d == 128) {
-    if (ksel == 8) return run_tiled<256, 8>(p, tmF, tmT, idx, scores, c);
-    if (ksel == 16) return run_tiled<256, 16>(p, tmF, tmT, idx, scores, c);
-    return run_tiled<256, 32>(p, tmF, tmT, idx, scores, c);
+    if (ksel == 8) return run_tiled<256, 8>(p, tmF, tmT, idx, scores, unit_need, c);
+    if (ksel == 16) return run_tiled<256, 16>(p, tmF, tmT, idx, scores, unit_need, c);
+    return run_tiled<256, 32>(p, tmF, tmT, idx, scores, unit_need, c);
   }
   if (p.d == 64) {
-    if (ksel == 8) return run_tiled<128, 8>(p, tmF, tmT, idx, scores, c);
-    if (ksel == 16) return run_tiled<128, 16>(p, tmF, tmT, idx, scores, c);
-    return run_tiled<128, 32>(p, tmF, tmT, idx, scores, c);
+    if (ksel == 8) return run_tiled<128, 8>(p, tmF, tmT, idx, scores, unit_need, c);
+    if (ksel == 16) return run_tiled<128, 16>(p, tmF, tmT, idx, scores, unit_need, c);
+    return run_tiled<128, 32>(p, tmF, tmT, idx, scores, unit_need, c);
   }
   return cudaErrorInvalidValue;
 }
 
 cudaError_t launch_route_rowwise_bf16(const ssa_params& p, const void* Q, const void* table,
-                                      int32_t* idx, float* scores, const LaunchCtx& c) {
-  if (p.d == 128) return rowwise_bf16_g<128>(p, Q, table, idx, scores, c);
-  if (p.d == 64) return rowwise_bf16_g<64>(p, Q, table, idx, scores, c);
+                                      int32_t* idx, float* scores, const LaunchCtx& c, const uint8_t* skip) {
+  if (p.d == 128) return rowwise_bf16_g<128>(p, Q, table, idx, scores, skip, c);
+  if (p.d == 64) return rowwise_bf16_g<64>(p, Q, table, idx, scores, skip, c);
   return cudaErrorInvalidValue;
 }
 

@@ -450,6 +450,118 @@ ssa_status forward_impl(const ssa_params& p, const void* Q, const void* K, const
   return do_attn(p, Q, K, V, idx, O, lse, nullptr, aw ? ws + L.attn : nullptr, aw, c);
 }
 
+// ------------------------------------------------------------------ hierarchical routing
+
+struct HierNodeLayout {
+  int64_t nn;
+  size_t table, radius, bound, total;
+};
+
+HierNodeLayout hier_node_layout(const ssa_params& p, const ssa_hier_params& hp) {
+  HierNodeLayout L;
+  const size_t bgs = static_cast<size_t>(p.batch) * p.h_kv;
+  L.nn = nb_of(p) / hp.fanout;
+  size_t off = 0;
+  L.table = off; off += round_up(bgs * L.nn * 2 * p.d * 2);
+  L.radius = off; off += round_up(bgs * L.nn * 4);
+  L.bound = off; off += round_up(bgs * 2 * 4);
+  L.total = off;
+  return L;
+}
+
+struct HierLayout {
+  size_t feat, nidx, nsc, cert, need, total;
+};
+
+int32_t route_tiles(const ssa_params& p) { return (p.n_q + 255) / 256; }
+
+HierLayout hier_layout(const ssa_params& p, const ssa_hier_params& hp) {
+  HierLayout L;
+  const size_t rows = static_cast<size_t>(p.batch) * p.n_q * p.h_kv;
+  const size_t bgs = static_cast<size_t>(p.batch) * p.h_kv;
+  size_t off = 0;
+  L.feat = off; off += round_up(rows * 2 * p.d * 2);
+  L.nidx = off; off += round_up(rows * (hp.probe + 1) * 4);
+  L.nsc = off; off += round_up(rows * (hp.probe + 1) * 4);
+  L.cert = off; off += round_up(rows);
+  L.need = off; off += (hp.escalate && use_tiled(p)) ? round_up(bgs * route_tiles(p) * 4) : 0;
+  L.total = off;
+  return L;
+}
+
+ssa_status check_hier(const ssa_params* p, const ssa_hier_params* hp) {
+  ssa_status st = check_params(p);
+  if (st != SSA_OK) return st;
+  if (!hp || hp->reserved != 0) return SSA_ERR_INVALID_ARG;
+  const int M = hp->fanout;
+  if (M < 1 || M > 64 || (M & (M - 1)) != 0) return SSA_ERR_INVALID_ARG;
+  if (hp->probe < 1 || hp->probe > 31 || (hp->escalate != 0 && hp->escalate != 1)) return SSA_ERR_INVALID_ARG;
+  if ((hp->probe + 1) * M > 512) return SSA_ERR_UNSUPPORTED;   // candidates per row of the probe kernel
+  if (p->dtype != SSA_BF16 || p->subblocks != 1) return SSA_ERR_UNSUPPORTED;
+  if (!use_tiled(*p) && !rowwise_fits(*p)) return SSA_ERR_UNSUPPORTED;
+  return SSA_OK;
+}
+
+// The node problem: nodes of M blocks act as blocks of M * B keys.
+ssa_params node_params(const ssa_params& p, const ssa_hier_params& hp, int64_t nn) {
+  ssa_params pn = p;
+  pn.block = p.block * hp.fanout;
+  pn.n_kv = static_cast<int32_t>(nn * pn.block);
+  pn.topk = hp.probe + 1;
+  pn.subblocks = 1;
+  return pn;
+}
+
+ssa_status do_route_hier(const ssa_params& p, const ssa_hier_params& hp, const void* Q, const void* table,
+                         const void* nodes, int32_t* idx, uint8_t* cert_out, uint8_t* ws, const LaunchCtx& c) {
+  const HierNodeLayout NL = hier_node_layout(p, hp);
+  const HierLayout H = hier_layout(p, hp);
+  const uint8_t* nd = static_cast<const uint8_t*>(nodes);
+  const uint64_t kf = 2 * static_cast<uint64_t>(p.d);
+  const int64_t bgs = static_cast<int64_t>(p.batch) * p.h_kv;
+  void* F = ws + H.feat;
+  int32_t* nidx = reinterpret_cast<int32_t*>(ws + H.nidx);
+  float* nsc = reinterpret_cast<float*>(ws + H.nsc);
+  uint8_t* cert = cert_out ? cert_out : ws + H.cert;
+  const bool tiled = use_tiled(p);
+  ssa_status st = from_cuda(ssa::launch_features(p, Q, F, c));
+  if (st != SSA_OK) return st;
+  CUtensorMap tmF;
+  if (tiled && !encode_2d(&tmF, F, kf, static_cast<uint64_t>(bgs) * p.n_q, 128)) return SSA_ERR_CUDA;
+  if (NL.nn > 0) {   // the best probe+1 nodes of every row, with their scores
+    const ssa_params pn = node_params(p, hp, NL.nn);
+    if (tiled) {
+      CUtensorMap tmN;
+      if (!encode_2d(&tmN, nd + NL.table, kf, static_cast<uint64_t>(bgs * NL.nn), 128)) return SSA_ERR_CUDA;
+      st = from_cuda(ssa::launch_route_tiled(pn, tmF, tmN, nidx, nsc, c));
+    } else {
+      st = from_cuda(ssa::launch_route_rowwise_bf16(pn, Q, nd + NL.table, nidx, nsc, c));
+    }
+    if (st != SSA_OK) return st;
+  }
+  int32_t* need = (hp.escalate && tiled) ? reinterpret_cast<int32_t*>(ws + H.need) : nullptr;
+  if (need && cudaMemsetAsync(need, 0, static_cast<size_t>(bgs) * route_tiles(p) * 4, c.stream) != cudaSuccess)
+    return SSA_ERR_CUDA;
+  ssa::HierProbeArgs a;
+  a.n_q = p.n_q; a.h_kv = p.h_kv; a.bgs = static_cast<int32_t>(bgs);
+  a.nb = static_cast<int32_t>(nb_of(p)); a.nn = static_cast<int32_t>(NL.nn); a.M = hp.fanout;
+  a.block = p.block; a.topk = p.topk; a.probe = hp.probe; a.n_tiles = route_tiles(p);
+  a.q_offset = p.q_offset;
+  a.F = static_cast<const __nv_bfloat16*>(F);
+  a.T = static_cast<const __nv_bfloat16*>(table);
+  a.node_idx = nidx; a.node_score = nsc;
+  a.bound = reinterpret_cast<const float*>(nd + NL.bound);
+  a.block_idx = idx; a.cert = cert; a.unit_need = need;
+  if ((st = from_cuda(ssa::launch_hier_probe(p, a, c))) != SSA_OK) return st;
+  if (!hp.escalate) return SSA_OK;
+  if (tiled) {   // the units holding an uncertified row, over all their visible blocks
+    CUtensorMap tmT;
+    if (!encode_2d(&tmT, table, kf, static_cast<uint64_t>(bgs) * summary_rows(p), 128)) return SSA_ERR_CUDA;
+    return from_cuda(ssa::launch_route_tiled(p, tmF, tmT, idx, nullptr, c, need));
+  }
+  return from_cuda(ssa::launch_route_rowwise_bf16(p, Q, table, idx, nullptr, c, cert));
+}
+
 }  // namespace
 
 extern "C" {
@@ -645,6 +757,59 @@ ssa_status ssa_forward_hostio(const ssa_params* pp, const void* hQ, const void* 
   if (hlse && cudaMemcpyAsync(hlse, d + L.lse, lb, cudaMemcpyDeviceToHost, c.stream) != cudaSuccess)
     return SSA_ERR_CUDA;
   return SSA_OK;
+}
+
+size_t ssa_hier_nodes_size(const ssa_params* p, const ssa_hier_params* hp) {
+  if (check_hier(p, hp) != SSA_OK) return 0;
+  return hier_node_layout(*p, *hp).total;
+}
+
+ssa_status ssa_hier_nodes(const ssa_params* pp, const ssa_hier_params* hp, const void* route_table, void* nodes,
+                          void* stream) {
+  ssa_status st = check_hier(pp, hp);
+  if (st != SSA_OK) return st;
+  const ssa_params& p = *pp;
+  if (p.batch == 0) return SSA_OK;
+  if (!route_table || !nodes || !aligned16(route_table) || !aligned16(nodes)) return SSA_ERR_INVALID_ARG;
+  LaunchCtx c;
+  if ((st = make_ctx(stream, c)) != SSA_OK) return st;
+  const HierNodeLayout L = hier_node_layout(p, *hp);
+  uint8_t* nd = static_cast<uint8_t*>(nodes);
+  const int64_t bgs = static_cast<int64_t>(p.batch) * p.h_kv;
+  if (cudaMemsetAsync(nd + L.bound, 0, static_cast<size_t>(bgs) * 2 * 4, c.stream) != cudaSuccess)
+    return SSA_ERR_CUDA;
+  ssa::HierNodeArgs a;
+  a.bgs = static_cast<int32_t>(bgs);
+  a.nb = static_cast<int32_t>(nb_of(p));
+  a.nn = static_cast<int32_t>(L.nn);
+  a.M = hp->fanout;
+  a.T = static_cast<const __nv_bfloat16*>(route_table);
+  a.NT = reinterpret_cast<__nv_bfloat16*>(nd + L.table);
+  a.radius = reinterpret_cast<float*>(nd + L.radius);
+  a.bound = reinterpret_cast<uint32_t*>(nd + L.bound);
+  return from_cuda(ssa::launch_hier_nodes(p, a, c));
+}
+
+size_t ssa_route_hier_workspace_size(const ssa_params* p, const ssa_hier_params* hp) {
+  if (check_hier(p, hp) != SSA_OK) return 0;
+  return hier_layout(*p, *hp).total;
+}
+
+ssa_status ssa_route_hier(const ssa_params* pp, const ssa_hier_params* hp, const void* Q, const void* route_table,
+                          const void* nodes, int32_t* block_idx, uint8_t* certified, void* ws, size_t ws_bytes,
+                          void* stream) {
+  ssa_status st = check_hier(pp, hp);
+  if (st != SSA_OK) return st;
+  const ssa_params& p = *pp;
+  if (is_empty(p)) return SSA_OK;
+  if (!Q || !route_table || !nodes || !block_idx || !aligned16(Q) || !aligned16(route_table) ||
+      !aligned16(nodes) || !aligned16(block_idx))
+    return SSA_ERR_INVALID_ARG;
+  const HierLayout H = hier_layout(p, *hp);
+  if (!ws || ws_bytes < H.total || !aligned16(ws)) return SSA_ERR_WORKSPACE;
+  LaunchCtx c;
+  if ((st = make_ctx(stream, c)) != SSA_OK) return st;
+  return do_route_hier(p, *hp, Q, route_table, nodes, block_idx, certified, static_cast<uint8_t*>(ws), c);
 }
 
 }  // extern "C"

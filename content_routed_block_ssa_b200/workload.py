@@ -8,7 +8,9 @@ Recipe (one generator per workload, seed = 1000 + workload id):
     the order Q, K noise, V, block centroids (clustered workloads only),
     needle noise;
   * clustered keys: k_j = centroid(block of j) + 0.3 * noise_j, centroids and
-    noise N(0, 1), a centroid per (batch, block, kv-head);
+    noise N(0, 1), a centroid per (batch, block, kv-head), or per run of
+    `cluster_span` consecutive blocks when that is above 1 (keys whose nearby
+    blocks are alike);
   * planted needles: a query row i (query head h) and an earlier key j of the
     kv-head serving h get k_j = 4 * q_i / ||q_i|| * sqrt(d) + N(0, 0.1) noise
     (variance 0.1).  Placement comes from a NumPy generator with the same
@@ -51,6 +53,7 @@ class Workload:
     decode: bool = False
     beta: float = 2.0
     subblocks: int = 1  # summaries per block (sub-block max-pool routing when > 1)
+    cluster_span: int = 1   # consecutive blocks sharing a centroid (clustered keys)
 
     @property
     def n_q(self) -> int:
@@ -143,8 +146,9 @@ def make_inputs(w: Workload, device="cpu", seed: int | None = None):
         Kb = draw((w.n, w.h_kv, w.d))
         V[bi] = draw((w.n, w.h_kv, w.d)).to(out_dt)
         if w.clustered:
-            cent = draw((w.n // w.block, w.h_kv, w.d))
-            Kb = cent.repeat_interleave(w.block, dim=0) + 0.3 * Kb
+            span = w.block * w.cluster_span
+            cent = draw(((w.n + span - 1) // span, w.h_kv, w.d))
+            Kb = cent.repeat_interleave(span, dim=0)[:w.n] + 0.3 * Kb
             del cent
         mine = [p for p in plan if p[0] == bi]
         if mine:

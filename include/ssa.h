@@ -284,6 +284,80 @@ SSA_API ssa_status ssa_forward_hostio(const ssa_params* p, const void* hQ, const
                               const void* hV, void* hO, float* hlse, void* dev_buf,
                               size_t dev_bytes, void* stream);
 
+/*
+ * Hierarchical routing with per-row certificates.  "Subquadratic Sparse
+ * Attention (SSA)" names a tree router with a recursive radius (artifact
+ * list, Barnes-Hut style), exact branch-and-bound selection under an
+ * admissible bound (same list) and sound per-query certificates with
+ * escalation ("Certified Causal Cascade" entry); it does not fix their rules.
+ * The rules here:
+ *
+ *   node N = the M consecutive blocks N*M .. N*M+M-1 (nn = nb / M complete
+ *   nodes per (batch, kv-head); trailing blocks form no node).  From the
+ *   blocks' bf16 routing rows T_c = [mu_c ; s_c]:
+ *     centre m_N = bf16(f32(mean of mu_c)), cap v_N = max of s_c (per dim),
+ *     radius R_N = max_c ||mu_c - m_N||_2 (float64, rounded up to float32).
+ *   For routing features f = [f_s ; f_q] (f_q >= 0) every block c of N has
+ *     f . T_c <= f . [m_N ; v_N] + ||f_s|| R_N.
+ *
+ *   A query row ranks its complete visible nodes by w_N = f . [m_N ; v_N]
+ *   (higher first, then lower index), scores exactly the blocks of its best
+ *   `probe` nodes and every visible block outside a complete visible node,
+ *   and keeps the top-k of those.  The row is certified when no complete
+ *   visible node is left unexpanded, or when its k-th kept score exceeds
+ *   w_(probe+1) + ||f_s|| R* + 2^-12 ||f|| T*, where R* is the largest node
+ *   radius and T* the largest 2-norm of any block or node row of its
+ *   (batch, kv-head) (the last term absorbs float32 rounding).  A certified
+ *   row's kept set is the top-k of all its visible blocks, as
+ *   ssa_route_topk selects it (up to the order of near-equal scores).
+ *   With escalate = 1 every uncertified row is routed again over all its
+ *   visible blocks (by ssa_route_topk's kernels), so block_idx is
+ *   ssa_route_topk's selection for every row.
+ *
+ * bf16 problems with a diagonal Sigma, subblocks = 1 and d in {64, 128}
+ * (else SSA_ERR_UNSUPPORTED).
+ */
+typedef struct {
+  int32_t fanout;    /* M, blocks per node: a power of two, 1..64                 */
+  int32_t probe;     /* nodes expanded per row before the certificate, 1..31      */
+  int32_t escalate;  /* 1: uncertified rows are re-routed over all blocks; or 0   */
+  int32_t reserved;  /* must be 0                                                 */
+} ssa_hier_params;
+
+/*
+ * Bytes of the node store of (p, hp): the node rows (bf16 [b, h_kv, nn, 2d],
+ * at offset 0), the radii (float32 [b, h_kv, nn], at offset
+ * round_up(node row bytes, 256)) and two floats per (batch, kv-head) (largest
+ * radius, largest row norm; after the radii, also 256-byte aligned).
+ * 0 on invalid arguments.
+ */
+SSA_API size_t ssa_hier_nodes_size(const ssa_params* p, const ssa_hier_params* hp);
+
+/*
+ * Builds the node store from a bf16 routing table (ssa_block_summary's
+ * route_table output, device [b, h_kv, nb, 2d]) into the device buffer
+ * `nodes` of ssa_hier_nodes_size bytes (16-byte aligned, caller-owned).
+ */
+SSA_API ssa_status ssa_hier_nodes(const ssa_params* p, const ssa_hier_params* hp, const void* route_table,
+                                  void* nodes, void* stream);
+
+/* Bytes of device workspace ssa_route_hier needs. */
+SSA_API size_t ssa_route_hier_workspace_size(const ssa_params* p, const ssa_hier_params* hp);
+
+/*
+ * Routes every query row through the node store (see above).
+ *   Q            device [b, n_q, h_q, d] bf16
+ *   route_table  device bf16 [b, h_kv, nb, 2d] (the table the nodes were built from)
+ *   nodes        device node store from ssa_hier_nodes
+ *   block_idx    device int32 output [b, n_q, h_kv, k], ascending, -1 padded
+ *   certified    device uint8 output [b, n_q, h_kv]: 1 certified, 0 not
+ *                (rows re-routed by escalation stay 0); may be NULL
+ *   ws, ws_bytes device workspace of at least ssa_route_hier_workspace_size
+ */
+SSA_API ssa_status ssa_route_hier(const ssa_params* p, const ssa_hier_params* hp, const void* Q,
+                                  const void* route_table, const void* nodes, int32_t* block_idx,
+                                  uint8_t* certified, void* ws, size_t ws_bytes, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -171,3 +171,41 @@ def test_block_major_workspace_and_stage_checks():
     # empty problems are no-ops for every stage
     e = good(n_q=0, q_offset=0)
     assert ssa.lib.ssa_attn_merge(C.byref(e), None, None, None, None, None, 0, None) == ssa.SSA_OK
+
+
+def test_hier_params_layout_and_checks():
+    assert C.sizeof(ssa.ssa_hier_params) == 16
+    assert ssa.ssa_hier_params.escalate.offset == 8
+    p = good(n_q=1000, n_kv=4096)
+    dummy = 256
+    ok = ssa.make_hier_params(fanout=8, probe=2, escalate=True)
+    nb, nn, bgs = 4096 // 64, 4096 // 64 // 8, 2
+    rnd = lambda x: (x + 255) // 256 * 256
+    assert ssa.ssa_hier_nodes_size(p, ok) == rnd(bgs * nn * 256 * 2) + rnd(bgs * nn * 4) + rnd(bgs * 8)
+    rows = 1000 * 2
+    tiles = (1000 + 255) // 256
+    assert ssa.ssa_route_hier_workspace_size(p, ok) == (rnd(rows * 256 * 2) + 2 * rnd(rows * 3 * 4) + rnd(rows)
+                                                        + rnd(bgs * tiles * 4))
+    no_esc = ssa.make_hier_params(fanout=8, probe=2, escalate=False)
+    assert ssa.ssa_route_hier_workspace_size(p, ok) - ssa.ssa_route_hier_workspace_size(p, no_esc) == \
+        rnd(bgs * tiles * 4)
+    for hp, code in ((ssa.make_hier_params(fanout=3), ssa.SSA_ERR_INVALID_ARG),      # not a power of two
+                     (ssa.make_hier_params(fanout=128), ssa.SSA_ERR_INVALID_ARG),
+                     (ssa.make_hier_params(probe=0), ssa.SSA_ERR_INVALID_ARG),
+                     (ssa.make_hier_params(probe=32), ssa.SSA_ERR_INVALID_ARG),
+                     (ssa.ssa_hier_params(fanout=8, probe=2, escalate=2, reserved=0), ssa.SSA_ERR_INVALID_ARG),
+                     (ssa.ssa_hier_params(fanout=8, probe=2, escalate=0, reserved=1), ssa.SSA_ERR_INVALID_ARG),
+                     (ssa.make_hier_params(fanout=64, probe=8), ssa.SSA_ERR_UNSUPPORTED)):   # 576 candidates
+        assert ssa.ssa_hier_nodes_size(p, hp) == 0
+        assert ssa.lib.ssa_hier_nodes(C.byref(p), C.byref(hp), dummy, dummy, None) == code
+        assert ssa.lib.ssa_route_hier(C.byref(p), C.byref(hp), dummy, dummy, dummy, dummy, None, dummy,
+                                      1 << 30, None) == code
+    for kw in (dict(dtype="f32", sigma="diag"), dict(subblocks=2)):
+        q = good(**kw)
+        assert ssa.lib.ssa_hier_nodes(C.byref(q), C.byref(ok), dummy, dummy, None) == ssa.SSA_ERR_UNSUPPORTED
+    assert ssa.lib.ssa_hier_nodes(C.byref(p), None, dummy, dummy, None) == ssa.SSA_ERR_INVALID_ARG
+    assert ssa.lib.ssa_hier_nodes(C.byref(p), C.byref(ok), 258, dummy, None) == ssa.SSA_ERR_INVALID_ARG
+    assert ssa.lib.ssa_route_hier(C.byref(p), C.byref(ok), dummy, dummy, dummy, dummy, None, dummy, 16,
+                                  None) == ssa.SSA_ERR_WORKSPACE
+    e = good(batch=0)
+    assert ssa.lib.ssa_route_hier(C.byref(e), C.byref(ok), None, None, None, None, None, None, 0, None) == ssa.SSA_OK
