@@ -236,7 +236,10 @@ def algorithmic_work(w, idx):
     gathered = float(S.sum().item()) * w.d * 2 * es
     qo = 2.0 * w.batch * w.n_q * w.h_q * w.d * es
     attn_flops = 4.0 * float(S.sum().item()) * G * w.d
+    # one pass over the routing table (the node summaries read every block row once)
+    route_table_bytes_once = float(w.batch * w.h_kv * nb) * w.subblocks * 2 * w.d * 2
     out = dict(summary_bytes=summary_bytes, route_flops=route_flops, route_table_bytes=route_table_bytes,
+               route_table_bytes_once=route_table_bytes_once,
                attn_bytes=gathered + qo,
                gathered_bytes=gathered, attn_flops=attn_flops, mean_keys=float(S.float().mean().item()))
     if w.dtype == "bf16":
@@ -264,10 +267,24 @@ def algorithmic_work(w, idx):
 
 # ------------------------------------------------------------------ our arm
 
-def run_ours(w, steps, warmup, ws, rank, with_e2e=True):
+def needle_recall(plan, idx, w):
+    """Fraction of planted needles whose key block the row selected."""
+    if not plan:
+        return None
+    G = w.h_q // w.h_kv
+    b = torch.tensor([p[0] for p in plan], device=idx.device)
+    i = torch.tensor([p[1] for p in plan], device=idx.device)
+    g = torch.tensor([p[2] // G for p in plan], device=idx.device)
+    blk = torch.tensor([p[3] // w.block for p in plan], device=idx.device, dtype=idx.dtype)
+    return float((idx[b, i, g] == blk[:, None]).any(dim=1).float().mean())
+
+
+def run_ours(w, steps, warmup, ws, rank, with_e2e=True, hier=None):
+    """hier: None (the flat router) or (fanout, probe, escalate) for the
+    hierarchical router, whose node summaries are then rebuilt every step."""
     from content_routed_block_ssa_b200 import ssa
     dev = torch.device("cuda", torch.cuda.current_device())
-    Q, K, V, _ = make_inputs(w, dev)
+    Q, K, V, plan = make_inputs(w, dev)
     p = ssa.make_params(**problem_dict(w))
     mu_s, sig_s, tab_s = ssa.summary_shapes(p)
     if w.dtype == "f32":   # float32 problems route on float32 mu / Sigma, no table
@@ -287,17 +304,25 @@ def run_ours(w, steps, warmup, ws, rank, with_e2e=True):
     stream = torch.cuda.current_stream()
 
     # stages of one step, each bracketed by events on the launching stream;
-    # block-major attention runs as its three staged calls
+    # block-major attention runs as its staged calls
+    cert = None
+    if hier is not None:
+        hp = ssa.make_hier_params(*hier)
+        nodes = ssa.byte_buffer(ssa.ssa_hier_nodes_size(p, hp), dev)
+        hws = ssa.byte_buffer(ssa.ssa_route_hier_workspace_size(p, hp), dev)
+        cert = torch.zeros(idx.shape[:3], dtype=torch.uint8, device=dev)
+        route_stages = [("hier_nodes", lambda: ssa.ssa_hier_nodes(p, hp, tab, nodes)),
+                        ("route", lambda: ssa.ssa_route_hier(p, hp, Q, tab, nodes, idx, cert, hws))]
+    else:
+        route_stages = [("route", lambda: ssa.ssa_route_topk(p, Q, mu, sig, tab, idx, None, rws))]
     if aws is not None:
-        stages = [("summary", lambda: ssa.ssa_block_summary(p, K, None, None, tab)),
-                  ("route", lambda: ssa.ssa_route_topk(p, Q, None, None, tab, idx, None, rws)),
+        stages = [("summary", lambda: ssa.ssa_block_summary(p, K, None, None, tab))] + route_stages + [
                   ("attn_plan", lambda: ssa.ssa_attn_plan(p, idx, aws)),
                   ("attn_blocks", lambda: ssa.ssa_attn_blocks(p, Q, K, V, aws)),
                   ("attn_window", lambda: ssa.ssa_attn_window(p, Q, K, V, aws)),
                   ("attn_merge", lambda: ssa.ssa_attn_merge(p, idx, O, lse, None, aws))]
     else:
-        stages = [("summary", lambda: ssa.ssa_block_summary(p, K, mu, sig, tab)),
-                  ("route", lambda: ssa.ssa_route_topk(p, Q, mu, sig, tab, idx, None, rws)),
+        stages = [("summary", lambda: ssa.ssa_block_summary(p, K, mu, sig, tab))] + route_stages + [
                   ("attn_gather", lambda: ssa.ssa_sparse_attn(p, Q, K, V, idx, O, lse))]
     ns = len(stages)
 
@@ -330,6 +355,10 @@ def run_ours(w, steps, warmup, ws, rank, with_e2e=True):
     ms_step_local = float(per.sum(axis=1).mean())
     ms_step = max_over_ranks(ms_step_local, ws)
     work = algorithmic_work(w, idx)
+    selection = {"needle_recall": needle_recall(plan, idx, w)}
+    if cert is not None:
+        selection["certified"] = float(cert.float().mean())
+        selection["router"] = {"fanout": hier[0], "probe": hier[1], "escalate": bool(hier[2])}
 
     e2e = None
     if with_e2e:
@@ -379,10 +408,11 @@ def run_ours(w, steps, warmup, ws, rank, with_e2e=True):
                "steps": n_e2e, "streams": NS}
         del bufs
     return dict(ms_step=ms_step, ms_kernels=ms_kernels, work=work, launches=int(launches),
-                clocks=clk.summary(), e2e=e2e)
+                clocks=clk.summary(), e2e=e2e, selection=selection)
 
 
 KERNEL_NAMES = {"summary": "summary_bf16_warp_kernel", "route": "route_tiled_kernel", "attn_plan": "inv_*_kernel (6)",
+                "hier_nodes": "hier_nodes_kernel",
                 "attn_blocks": "attn_block_kernel", "attn_window": "attn_window_kernel",
                 "attn_merge": "attn_merge_kernel",
                 "attn_gather": "attn_bf16_kernel"}
@@ -408,7 +438,14 @@ def kernel_report(w, res, peaks, traffic):
         rep[name] = e
 
     hbm_entry("summary", wk["summary_bytes"])
-    if w.dtype == "f32":
+    if "hier_nodes" in ms:
+        # node summaries: one pass over the routing table; the hierarchical
+        # route (node router + per-row probe of L2-served table rows + any
+        # escalation) is reported by time, outside the roofline
+        hbm_entry("hier_nodes", wk["route_table_bytes_once"])
+        rep["route"] = {"ms": ms["route"], "kernel": "route_tiled_kernel / route_rowwise_bf16_kernel (nodes) + "
+                                                     "hier_probe_kernel (+ escalation)"}
+    elif w.dtype == "f32":
         rep["summary"]["kernel"] = "summary_diag_kernel" if w.sigma == "diag" else "summary_full_kernel"
         # float32 rows score their blocks with FMA on the CUDA cores (row-wise router)
         r_tf = wk["route_flops"] / (ms["route"] * 1e-3) / 1e12
@@ -520,6 +557,12 @@ def main():
                     help="shorter sequence of the same workload (profiling captures); not a bench line")
     ap.add_argument("--subblocks", type=int, default=1,
                     help="route on S sub-block summaries per block, max-pooled (S in 1, 2, 4; block / S >= 32)")
+    ap.add_argument("--router", default="flat", choices=["flat", "hier"],
+                    help="hier: the hierarchical router (nodes of --fanout blocks, --probe nodes per row); "
+                         "a measurement of that router, not the bench line")
+    ap.add_argument("--fanout", type=int, default=16)
+    ap.add_argument("--probe", type=int, default=2)
+    ap.add_argument("--escalate", action="store_true", help="re-route uncertified rows over all blocks")
     a = ap.parse_args()
     w = WORKLOADS[a.workload]
     if a.n is not None:
@@ -553,7 +596,10 @@ def main():
 
     # the committed DRAM counters were taken with whole-block summaries
     traffic = load_traffic() if w.subblocks == 1 else {}
-    res = run_ours(w, a.steps, a.warmup, ws, rank, with_e2e=not a.no_e2e)
+    hier = (a.fanout, a.probe, a.escalate) if a.router == "hier" else None
+    if hier is not None:
+        config["router"] = {"kind": "hierarchical", "fanout": a.fanout, "probe": a.probe, "escalate": a.escalate}
+    res = run_ours(w, a.steps, a.warmup, ws, rank, with_e2e=not a.no_e2e and hier is None, hier=hier)
     kern = kernel_report(w, res, peaks, traffic)
     value = whole_job_rate(w.batch * w.n_q * w.h_q, ws, res["ms_step"])
     dname, dk = dominant(kern)
@@ -586,7 +632,7 @@ def main():
                 "ms_per_step": res["ms_step"], "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
                 "dtype": w.dtype, "data": "synthetic", "config": config, "roofline": roof, "cpu_baseline": cpu,
                 "e2e": res["e2e"], "gpu_launches": res["launches"], "clocks": res["clocks"], "kernels": kern,
-                "secondary": secondary}
+                "selection": res["selection"], "secondary": secondary}
         print(json.dumps(line), flush=True)
     if ws > 1:
         import torch.distributed as dist
