@@ -55,6 +55,28 @@ __device__ __forceinline__ void load_slice(const __nv_bfloat16* p, float (&v)[FP
   }
 }
 
+// The raw bf16 pairs of a lane's slice (FPL / 2 words; the rest unused).
+template <int FPL>
+__device__ __forceinline__ uint4 load_raw(const __nv_bfloat16* p) {
+  if constexpr (FPL == 8) {
+    return __ldg(reinterpret_cast<const uint4*>(p));
+  } else {
+    const uint2 r = __ldg(reinterpret_cast<const uint2*>(p));
+    return make_uint4(r.x, r.y, 0u, 0u);
+  }
+}
+
+template <int FPL>
+__device__ __forceinline__ float dot_raw(const float (&f)[FPL], uint4 raw, float acc) {
+  const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
+#pragma unroll
+  for (int j = 0; j < FPL / 2; ++j) {
+    acc = __fmaf_rn(f[2 * j], __uint_as_float(w[j] << 16), acc);
+    acc = __fmaf_rn(f[2 * j + 1], __uint_as_float(w[j] & 0xFFFF0000u), acc);
+  }
+  return acc;
+}
+
 template <int FPL>
 __device__ __forceinline__ void store_slice(__nv_bfloat16* p, const float (&v)[FPL]) {
   uint32_t w[FPL / 2];
@@ -77,15 +99,6 @@ __device__ __forceinline__ double warp_sum_d(double x) {
 __device__ __forceinline__ float warp_sum_f(float x) {
 #pragma unroll
   for (int o = 16; o; o >>= 1) x += __shfl_xor_sync(0xFFFFFFFFu, x, o);
-  return x;
-}
-
-__device__ __forceinline__ uint64_t warp_max_u64(uint64_t x) {
-#pragma unroll
-  for (int o = 16; o; o >>= 1) {
-    const uint64_t y = __shfl_xor_sync(0xFFFFFFFFu, x, o);
-    x = y > x ? y : x;
-  }
   return x;
 }
 
@@ -118,6 +131,7 @@ __global__ void __launch_bounds__(256) hier_nodes_kernel(const HierNodeArgs a) {
 #pragma unroll
   for (int e = 0; e < FPL; ++e) { sum[e] = 0.0; cap[e] = -INFINITY; }
   double row2max = 0.0;
+#pragma unroll 4
   for (int c = c0; c < c1; ++c) {
     float v[FPL];
     load_slice<FPL>(trow + static_cast<int64_t>(c) * (2 * D), v);
@@ -141,6 +155,7 @@ __global__ void __launch_bounds__(256) hier_nodes_kernel(const HierNodeArgs a) {
     for (int e = 0; e < FPL; ++e) n2 += static_cast<double>(m[e]) * m[e];
     row2max = fmax(row2max, warp_sum_d(n2));
     double d2max = 0.0;
+#pragma unroll 4
     for (int c = c0; c < c1; ++c) {
       float v[FPL];
       load_slice<FPL>(trow + static_cast<int64_t>(c) * (2 * D), v);
@@ -228,17 +243,20 @@ __global__ void __launch_bounds__(256) hier_probe_kernel(const HierProbeArgs a) 
   for (int t0 = 0; t0 < n_cand; t0 += 32) {
     float acc[32];
 #pragma unroll
-    for (int u = 0; u < 32; ++u) {
-      const int t = t0 + u;
-      const int node = __shfl_sync(0xFFFFFFFFu, my_exp, min(t >> log2M, 31));
-      acc[u] = 0.f;
-      if (t < n_cand) {
-        const int c = t < nexpb ? (node << log2M) + (t & (a.M - 1)) : nvn * a.M + (t - nexpb);
-        float v[FPL];
-        load_slice<FPL>(tb + static_cast<int64_t>(c) * (2 * D), v);
+    for (int u0 = 0; u0 < 32; u0 += 8) {
+      // eight independent row loads in flight; past the last candidate a
+      // lane reads row 0 and the score is discarded
+      uint4 raw[8];
 #pragma unroll
-        for (int e = 0; e < FPL; ++e) acc[u] = __fmaf_rn(f[e], v[e], acc[u]);
+      for (int u = 0; u < 8; ++u) {
+        const int t = t0 + u0 + u;
+        const int node = __shfl_sync(0xFFFFFFFFu, my_exp, min(t >> log2M, 31));
+        int c = t < nexpb ? (node << log2M) + (t & (a.M - 1)) : nvn * a.M + (t - nexpb);
+        c = t < n_cand ? c : 0;
+        raw[u] = load_raw<FPL>(tb + static_cast<int64_t>(c) * (2 * D));
       }
+#pragma unroll
+      for (int u = 0; u < 8; ++u) acc[u0 + u] = dot_raw<FPL>(f, raw[u], 0.f);
     }
 #pragma unroll
     for (int o = 16; o >= 1; o >>= 1) {
@@ -259,22 +277,35 @@ __global__ void __launch_bounds__(256) hier_probe_kernel(const HierProbeArgs a) 
   }
   __syncwarp();
 
-  // top-k under (score desc, block asc): k rounds of a warp arg-max
+  // top-k under (score desc, block asc): k rounds of a warp arg-max, the
+  // score half and the block half of the key each by one warp reduction
+  // (keys are unique: one block each); a lane keeps its best key cached
   uint64_t kept = 0;
   int nkept = 0;
+  uint64_t m = 0;
+  int at = -1;
+  for (int t = lane; t < n_cand; t += 32) {
+    const uint64_t x = keys[t];
+    if (x > m) { m = x; at = t; }
+  }
   for (int j = 0; j < a.topk; ++j) {
-    uint64_t m = 0;
-    int at = -1;
-    for (int t = lane; t < n_cand; t += 32) {
-      const uint64_t x = keys[t];
-      if (x > m) { m = x; at = t; }
-    }
-    const uint64_t best = warp_max_u64(m);
-    if (best == 0) break;
-    if (at >= 0 && m == best) keys[at] = 0;
-    __syncwarp();
+    const uint32_t hi = static_cast<uint32_t>(m >> 32);
+    const uint32_t top = __reduce_max_sync(0xFFFFFFFFu, hi);
+    if (top == 0) break;   // no candidates left
+    const uint32_t lo = __reduce_max_sync(0xFFFFFFFFu, hi == top ? static_cast<uint32_t>(m) : 0u);
+    const uint64_t best = (static_cast<uint64_t>(top) << 32) | lo;
     if (lane == j) kept = best;
     ++nkept;
+    if (m == best) {   // the owner drops it and rescans its candidates
+      keys[at] = 0;
+      m = 0;
+      at = -1;
+      for (int t = lane; t < n_cand; t += 32) {
+        const uint64_t x = keys[t];
+        if (x > m) { m = x; at = t; }
+      }
+    }
+    __syncwarp();
   }
   const uint64_t kth = __shfl_sync(0xFFFFFFFFu, kept, max(a.topk - 1, 0));
   const float tau = nkept == a.topk ? key_score(kth) : -INFINITY;
