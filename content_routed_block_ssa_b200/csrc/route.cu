@@ -498,26 +498,77 @@ __device__ __forceinline__ int next_pow2(int x) {
   return p;
 }
 
-// Sorts keys[0..n2) descending in shared memory (n2 a power of two) and
-// writes the top-k blocks of the row in ascending block order.
-__device__ void select_and_write(uint64_t* keys, int nvis, int n2, const RowArgs& a, int64_t out) {
-  for (int c = nvis + threadIdx.x; c < n2; c += blockDim.x) keys[c] = 0;
-  __syncthreads();
-  for (int size = 2; size <= n2; size <<= 1) {
-    for (int stride = size >> 1; stride > 0; stride >>= 1) {
-      for (int t = threadIdx.x; t < n2 / 2; t += blockDim.x) {
-        const int i = 2 * t - (t & (stride - 1));   // lower index of the pair
-        const int j = i + stride;
-        const bool desc = (i & size) == 0;
-        const uint64_t x = keys[i], y = keys[j];
-        if (desc ? (x < y) : (x > y)) { keys[i] = y; keys[j] = x; }
+// Writes the top-k of keys[0..n) (distinct and nonzero: a block index in
+// the low half) in ascending block order.  A radix select, most significant
+// 8-bit digit first, finds the k-th largest key: per digit, a histogram of
+// the keys that share the digits decided so far (warp-aggregated
+// shared-memory atomics), then one warp finds the digit holding the k-th key.
+// It stops at the first digit whose keys are all needed, so the keys >= the
+// decided prefix (lower digits zero) are exactly the k largest; they are
+// collected and ranked by block index.
+__device__ void select_and_write(const uint64_t* keys, int n, const RowArgs& a, int64_t out) {
+  __shared__ uint32_t hist[256];
+  __shared__ uint64_t s_prefix;
+  __shared__ int s_krem, s_done, s_nsel;
+  __shared__ uint64_t sel[32];
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int k = min(a.topk, n);
+  if (tid == 0) { s_prefix = 0; s_krem = a.topk; s_done = n <= a.topk; s_nsel = 0; }
+  __syncthreads();   // also orders the callers' key writes before the reads below
+  uint64_t mask = 0;
+  for (int shift = 56; shift >= 0 && !s_done; shift -= 8) {
+    for (int j = tid; j < 256; j += blockDim.x) hist[j] = 0;
+    __syncthreads();
+    const uint64_t prefix = s_prefix;
+    for (int c0 = warp * 32; c0 < n; c0 += blockDim.x) {   // warp-uniform trip count
+      const int c = c0 + lane;
+      const uint64_t key = c < n ? keys[c] : 0;
+      const bool in = c < n && (key & mask) == prefix;
+      const uint32_t digit = in ? static_cast<uint32_t>(key >> shift) & 255u : 256u;
+      const uint32_t same = __match_any_sync(0xFFFFFFFFu, digit);
+      if (in && lane == __ffs(static_cast<int>(same)) - 1) atomicAdd(&hist[digit], __popc(same));
+    }
+    __syncthreads();
+    if (warp == 0) {
+      uint32_t h[8], sum = 0;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) { h[j] = hist[lane * 8 + j]; sum += h[j]; }
+      uint32_t suf = sum;   // keys in this lane's digits and all higher ones
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t v = __shfl_down_sync(0xFFFFFFFFu, suf, o);
+        if (lane + o < 32) suf += v;
       }
-      __syncthreads();
+      const uint32_t krem = static_cast<uint32_t>(s_krem);
+      const uint32_t above = suf - sum;
+      if (above < krem && krem <= suf) {   // the k-th key's digit is in this lane's range
+        uint32_t cum = above;
+        int d = lane * 8;
+        uint32_t cnt = 0;
+#pragma unroll
+        for (int j = 7; j >= 0; --j) {
+          if (cnt == 0 && cum + h[j] >= krem) { d = lane * 8 + j; cnt = h[j]; }
+          else if (cnt == 0) cum += h[j];
+        }
+        s_prefix = prefix | (static_cast<uint64_t>(d) << shift);
+        s_krem = static_cast<int>(krem - cum);
+        s_done = cnt == krem - cum;
+      }
+    }
+    __syncthreads();
+    mask |= 0xFFull << shift;
+  }
+  const uint64_t T = s_prefix;   // 0 when every key is taken
+  for (int c = tid; c < n; c += blockDim.x) {
+    const uint64_t key = keys[c];
+    if (key >= T) {
+      const int slot = atomicAdd(&s_nsel, 1);
+      if (slot < 32) sel[slot] = key;
     }
   }
-  if (threadIdx.x < 32) {
-    const int lane = threadIdx.x;
-    const uint64_t key = (lane < a.topk && lane < n2) ? keys[lane] : 0;
+  __syncthreads();
+  if (warp == 0) {
+    const uint64_t key = lane < k ? sel[lane] : 0;
     const uint32_t blk = key ? key_block(key) : 0xFFFFFFFFu;
     // valid entries are ranked by block index; empty slots follow, in lane order
     const uint32_t vmask = __ballot_sync(0xFFFFFFFFu, key != 0);
@@ -572,57 +623,56 @@ __global__ void __launch_bounds__(256) route_rowwise_bf16_kernel(const __nv_bflo
       f[v] = __bfloat162float(__float2bfloat16_rn(raw));
     }
   }
-  // table rows are sub-blocks (S per block); a warp scores 4 consecutive
-  // rows, which hold 4 / S whole blocks
+  // table rows are sub-blocks (S per block); a warp scores two runs of 4
+  // consecutive rows per pass (each run holds 4 / S whole blocks), its eight
+  // row loads issued together: past the last row a lane reads row 0 and the
+  // score is dropped
   const int nrows = nvis * a.S;
   const __nv_bfloat16* trow = T + (static_cast<int64_t>(b) * a.h_kv + g) * a.nb * a.S * (2 * D) + lane * FPL;
-  for (int c0 = warp * 4; c0 < nrows; c0 += 32) {
-    float part[4];
+  for (int c0 = warp * 8; c0 < nrows; c0 += 64) {
+    uint4 raw[8];
 #pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      const int c = c0 + u;
+    for (int u = 0; u < 8; ++u) {
+      const int c = c0 + u < nrows ? c0 + u : 0;
+      const __nv_bfloat16* t = trow + static_cast<int64_t>(c) * (2 * D);
+      if (FPL == 8) {
+        raw[u] = __ldg(reinterpret_cast<const uint4*>(t));
+      } else {
+        const uint2 r2 = __ldg(reinterpret_cast<const uint2*>(t));
+        raw[u] = make_uint4(r2.x, r2.y, 0u, 0u);
+      }
+    }
+    float part[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const uint32_t w[4] = {raw[u].x, raw[u].y, raw[u].z, raw[u].w};
       part[u] = 0.f;
-      if (c < nrows) {
-        const __nv_bfloat16* t = trow + static_cast<int64_t>(c) * (2 * D);
-        float tv[FPL];
-        if (FPL == 8) {
-          const uint4 raw = __ldg(reinterpret_cast<const uint4*>(t));
-          const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
 #pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            tv[2 * j] = __uint_as_float(w[j] << 16);
-            tv[2 * j + 1] = __uint_as_float(w[j] & 0xFFFF0000u);
-          }
-        } else {
-          const uint2 raw = __ldg(reinterpret_cast<const uint2*>(t));
-          const uint32_t w[2] = {raw.x, raw.y};
-#pragma unroll
-          for (int j = 0; j < 2; ++j) {
-            tv[2 * j] = __uint_as_float(w[j] << 16);
-            tv[2 * j + 1] = __uint_as_float(w[j] & 0xFFFF0000u);
-          }
-        }
-#pragma unroll
-        for (int v = 0; v < FPL; ++v) part[u] = __fmaf_rn(f[v], tv[v], part[u]);
+      for (int j = 0; j < FPL / 2; ++j) {
+        part[u] = __fmaf_rn(f[2 * j], __uint_as_float(w[j] << 16), part[u]);
+        part[u] = __fmaf_rn(f[2 * j + 1], __uint_as_float(w[j] & 0xFFFF0000u), part[u]);
       }
     }
 #pragma unroll
-    for (int u = 0; u < 4; ++u) {
+    for (int u = 0; u < 8; ++u) {
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1) part[u] += __shfl_xor_sync(0xFFFFFFFFu, part[u], o);
     }
-    // a block's score is the largest of its sub-blocks' scores
-    if (a.S >= 2) { part[0] = fmaxf(part[0], part[1]); part[1] = fmaxf(part[2], part[3]); }
-    if (a.S == 4) part[0] = fmaxf(part[0], part[1]);
-    const int nper = 4 / a.S;
-    for (int u = 0; u < nper; ++u) {
-      const int c = c0 / a.S + u;
-      if (lane == 0 && c < nvis) keys[c] = make_key(__float_as_uint(part[u]), c);
+#pragma unroll
+    for (int q = 0; q < 2; ++q) {
+      float* pq = part + 4 * q;
+      // a block's score is the largest of its sub-blocks' scores
+      if (a.S >= 2) { pq[0] = fmaxf(pq[0], pq[1]); pq[1] = fmaxf(pq[2], pq[3]); }
+      if (a.S == 4) pq[0] = fmaxf(pq[0], pq[1]);
+      const int nper = 4 / a.S;
+      for (int u = 0; u < nper; ++u) {
+        const int c = (c0 + 4 * q) / a.S + u;
+        if (lane == 0 && c < nvis) keys[c] = make_key(__float_as_uint(pq[u]), c);
+      }
     }
   }
-  const int n2 = next_pow2(max(nvis, 1));
   const int64_t out = ((static_cast<int64_t>(b) * a.n_q + i) * a.h_kv + g) * a.topk;
-  select_and_write(keys, nvis, n2, a, out);
+  select_and_write(keys, nvis, a, out);
 }
 
 // float32 summaries: s_c = sum_h (<q_h, mu_c> + (beta/2) q_h^T Sigma_c q_h).
@@ -678,10 +728,8 @@ __global__ void __launch_bounds__(256) route_rowwise_f32_kernel(const float* __r
     }
     if (lane == 0) keys[cb] = make_key(__float_as_uint(best), cb);
   }
-  const int n2 = next_pow2(max(nvis, 1));
   const int64_t out = ((static_cast<int64_t>(b) * a.n_q + i) * a.h_kv + g) * a.topk;
-  __syncthreads();
-  select_and_write(keys, nvis, n2, a, out);
+  select_and_write(keys, nvis, a, out);
 }
 
 // float32 summaries for runs of query rows: a CTA takes 32/G consecutive
