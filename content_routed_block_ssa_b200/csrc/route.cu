@@ -754,17 +754,106 @@ __global__ void __launch_bounds__(256) route_qtile_f32_kernel(const float* __res
   const int i0 = blockIdx.x * QT, g = blockIdx.y, b = blockIdx.z;
   const int h_q = a.h_kv * G;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  // the tile's (query, head) rows of Q; rows past n_q are zero
+  // the tile's (query, head) rows of Q; rows past n_q are zero.  Full Sigma:
+  // stored transposed, qs[t * 32 + r]
   for (int e = threadIdx.x; e < 32 * D; e += 256) {
     const int r = e / D, t = e % D, qq = r / G, h = r % G;
     const int i = i0 + qq;
-    qs[e] = i < a.n_q ? Q[((static_cast<int64_t>(b) * a.n_q + i) * h_q + static_cast<int64_t>(g) * G + h) * D + t]
-                      : 0.f;
+    const float v = i < a.n_q ? Q[((static_cast<int64_t>(b) * a.n_q + i) * h_q + static_cast<int64_t>(g) * G + h) * D + t]
+                              : 0.f;
+    qs[FULL ? t * 32 + r : e] = v;
   }
   const int64_t last = a.q_offset + min(i0 + QT, a.n_q) - 1;
   const int ncmax = static_cast<int>(min(static_cast<int64_t>(a.nb), (last + 1) / a.block));
-  const int r = threadIdx.x >> 3, part = threadIdx.x & 7;   // (query, head) row, its eighth
   const int64_t bgrow = (static_cast<int64_t>(b) * a.h_kv + g) * a.nb * a.S;
+  if constexpr (FULL) {
+    // Register-tiled: thread (sg, rg) accumulates U[s][r] = sum_t Sigma[t][s] q_r[t]
+    // for its D/16 columns s and two rows r (q^T Sigma^T q = q^T Sigma q), from
+    // contiguous Sigma rows; the next summary row is fetched into registers
+    // while this one is used.
+    constexpr int SPT = D / 16;
+    constexpr int NPF = D * D / 4 / 256;
+    float* red = sc + 32;   // [16][32] partial scores
+    const int sg = threadIdx.x >> 4, r0 = (threadIdx.x & 15) * 2, s0 = sg * SPT;
+    const int nrow = ncmax * a.S;
+    float4 pf[NPF];
+    float4 pm = make_float4(0.f, 0.f, 0.f, 0.f);
+    auto fetch = [&](int u) {
+      const float4* src = reinterpret_cast<const float4*>(SG + (bgrow + u) * D * D);
+#pragma unroll
+      for (int j = 0; j < NPF; ++j) pf[j] = __ldg(src + threadIdx.x + j * 256);
+      if (threadIdx.x < D / 4) pm = __ldg(reinterpret_cast<const float4*>(MU + (bgrow + u) * D) + threadIdx.x);
+    };
+    auto stage = [&]() {
+      float4* dst = reinterpret_cast<float4*>(sgs);
+#pragma unroll
+      for (int j = 0; j < NPF; ++j) dst[threadIdx.x + j * 256] = pf[j];
+      if (threadIdx.x < D / 4) reinterpret_cast<float4*>(mus)[threadIdx.x] = pm;
+    };
+    if (nrow > 0) {
+      fetch(0);
+      stage();
+    }
+    float best = -INFINITY;   // threads < QT: the query's best sub-block score
+    for (int u = 0; u < nrow; ++u) {
+      __syncthreads();   // row u staged, the previous row's scores consumed
+      if (u + 1 < nrow) fetch(u + 1);
+      float acc[SPT][2];
+#pragma unroll
+      for (int i = 0; i < SPT; ++i) { acc[i][0] = 0.f; acc[i][1] = 0.f; }
+#pragma unroll 4
+      for (int t = 0; t < D; ++t) {
+        float sv[SPT];
+#pragma unroll
+        for (int i = 0; i < SPT; i += 4) {
+          const float4 x = *reinterpret_cast<const float4*>(sgs + t * D + s0 + i);
+          sv[i] = x.x; sv[i + 1] = x.y; sv[i + 2] = x.z; sv[i + 3] = x.w;
+        }
+        const float2 qv = *reinterpret_cast<const float2*>(qs + t * 32 + r0);
+#pragma unroll
+        for (int i = 0; i < SPT; ++i) {
+          acc[i][0] = __fmaf_rn(sv[i], qv.x, acc[i][0]);
+          acc[i][1] = __fmaf_rn(sv[i], qv.y, acc[i][1]);
+        }
+      }
+      // this thread's columns of <q, mu> + (beta/2) q^T Sigma q for its two rows
+      float p0 = 0.f, p1 = 0.f;
+#pragma unroll
+      for (int i = 0; i < SPT; ++i) {
+        const float2 qv = *reinterpret_cast<const float2*>(qs + (s0 + i) * 32 + r0);
+        const float m = mus[s0 + i];
+        p0 = __fmaf_rn(qv.x, __fmaf_rn(a.half_beta, acc[i][0], m), p0);
+        p1 = __fmaf_rn(qv.y, __fmaf_rn(a.half_beta, acc[i][1], m), p1);
+      }
+      *reinterpret_cast<float2*>(red + sg * 32 + r0) = make_float2(p0, p1);
+      __syncthreads();   // partials written, row u read
+      if (threadIdx.x < 32) {
+        float v = 0.f;
+#pragma unroll
+        for (int j = 0; j < 16; ++j) v += red[j * 32 + threadIdx.x];
+        sc[threadIdx.x] = v;
+      }
+      if (u + 1 < nrow) stage();
+      __syncthreads();
+      // the group's score of each query for this summary row: its heads'
+      // scores summed in head order; the block keeps its largest sub-block
+      const int cb = u / a.S, sb = u % a.S;
+      if (threadIdx.x < QT) {
+        float gsum = 0.f;
+#pragma unroll
+        for (int h = 0; h < G; ++h) gsum += sc[threadIdx.x * G + h];
+        best = fmaxf(best, gsum);
+        if (sb == a.S - 1) {
+          const int qq = threadIdx.x, i = i0 + qq;
+          const int64_t pos = a.q_offset + i;
+          const bool vis = i < a.n_q && cb < min(static_cast<int64_t>(a.nb), (pos + 1) / a.block);
+          keys[qq * n2 + cb] = vis ? make_key(__float_as_uint(best), cb) : 0ull;
+          best = -INFINITY;
+        }
+      }
+    }
+  } else {
+  const int r = threadIdx.x >> 3, part = threadIdx.x & 7;   // (query, head) row, its eighth
   for (int cb = 0; cb < ncmax; ++cb) {
     float best = -INFINITY;   // threads < QT: the query's best sub-block score
     for (int sb = 0; sb < a.S; ++sb) {
@@ -813,6 +902,7 @@ __global__ void __launch_bounds__(256) route_qtile_f32_kernel(const float* __res
       const bool vis = i < a.n_q && cb < min(static_cast<int64_t>(a.nb), (pos + 1) / a.block);
       keys[qq * n2 + cb] = vis ? make_key(__float_as_uint(best), cb) : 0ull;
     }
+  }
   }
   __syncthreads();
   for (int e = threadIdx.x; e < QT * n2; e += 256)
@@ -927,7 +1017,8 @@ int qtile_smem_bytes(const ssa_params& p) {
   int n2 = 1;
   while (n2 < p.n_kv / p.block) n2 <<= 1;
   const int64_t bytes = static_cast<int64_t>(32 / G) * n2 * 8 + 32 * D * 4 +
-                        (FULL ? static_cast<int64_t>(D) * (D + 1) : D) * 4 + D * 4 + 32 * 4;
+                        (FULL ? static_cast<int64_t>(D) * (D + 1) : D) * 4 + D * 4 + 32 * 4 +
+                        (FULL ? 16 * 32 * 4 : 0);
   return bytes <= 160 * 1024 ? static_cast<int>(bytes) : 0;
 }
 
