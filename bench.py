@@ -474,7 +474,8 @@ def kernel_report(w, res, peaks, traffic):
         e = wk["route_table_bytes"] / (ms["route"] * 1e-3) / 1e9
         rep["route"] = {"ms": ms["route"], "bound": "hbm", "achieved": e, "unit": "GB/s", "frac": e / hbm,
                         "peak": hbm, "algorithmic_bytes": wk["route_table_bytes"],
-                        "kernel": "route_rowwise_bf16_kernel", "traffic": None}
+                        "kernel": "route_rowwise_bf16_kernel",
+                        "traffic": traffic.get(("route_rowwise_bf16_kernel", w.name))}
     else:
         r_tf = wk["route_flops"] / (ms["route"] * 1e-3) / 1e12
         rep["route"] = {"ms": ms["route"], "bound": "tensor", "achieved": r_tf, "unit": "TFLOP/s",
