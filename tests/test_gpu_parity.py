@@ -59,6 +59,12 @@ CASES = {
     "bf16_mha_d128_b64_w200": Workload("c", 123, 1, 1536, 2, 2, 128, "bf16", 64, "diag", 8, 200, 4, "per_head"),
     "bf16_gqa8_d128_b64_w600": Workload("c", 124, 1, 2048, 16, 2, 128, "bf16", 64, "diag", 8, 600, 4, "total",
                                         clustered=True),
+    # the largest windows: 1985 keys (32 window blocks of 64, the most the
+    # block-major path takes: 8 window chunks) and 4032 keys (the API's limit,
+    # 64 window tiles, per-row gather)
+    "bf16_gqa4_d128_b64_w1985": Workload("c", 125, 1, 4096, 8, 2, 128, "bf16", 64, "diag", 8, 1985, 4, "total",
+                                         clustered=True),
+    "bf16_gqa4_d128_b64_w4032": Workload("c", 126, 1, 5120, 8, 2, 128, "bf16", 64, "diag", 8, 4032, 4, "total"),
     # float32 routing takes runs of 32 (query, head) pairs per CTA unless a
     # row's 1024 block scores do not fit beside them: then one CTA per row
     "f32_diag_d64_decode_64k": Workload("c", 122, 1, 65536, 1, 1, 64, "f32", 64, "diag", 8, 64, 2, "per_seq",
@@ -323,10 +329,12 @@ def test_empty_problem_launches_nothing_and_small_workspace_is_rejected():
 
 
 # Problems the block-major attention takes (bf16, d = 128, G in {1, 2, 4, 8},
-# k * G <= 128, at least 1024 query rows) when it is given its workspace.
+# k * G <= 128, at least 1024 query rows, a window over at most 32 key
+# blocks) when it is given its workspace.
 BLOCK_MAJOR = [n for n, w in CASES.items()
                if w.dtype == "bf16" and w.d == 128 and w.h_q // w.h_kv in (1, 2, 4, 8)
-               and w.topk * (w.h_q // w.h_kv) <= 128 and w.n_q >= 1024]
+               and w.topk * (w.h_q // w.h_kv) <= 128 and w.n_q >= 1024
+               and (w.window + w.block - 2) // w.block + 1 <= 32]
 
 
 def test_block_major_cases_exist():
@@ -335,6 +343,8 @@ def test_block_major_cases_exist():
     for n in BLOCK_MAJOR:
         assert ssa.ssa_attn_workspace_size(params(problem_dict(CASES[n]))) > 0
     assert ssa.ssa_attn_workspace_size(params(problem_dict(CASES["bf16_gqa2_d64_b64"]))) == 0   # d = 64
+    assert "bf16_gqa4_d128_b64_w1985" in BLOCK_MAJOR                # 32 window blocks
+    assert ssa.ssa_attn_workspace_size(params(problem_dict(CASES["bf16_gqa4_d128_b64_w4032"]))) == 0
 
 
 @pytest.mark.parametrize("name", BLOCK_MAJOR)
