@@ -407,7 +407,9 @@ def run_ours(w, steps, warmup, ws, rank, with_e2e=True, hier=None):
         e0.record(streams[0])
         for st in streams[1:]:
             st.wait_event(e0)
-        n_e2e = max(2 * NS, min(steps, 3 * NS))
+        # ten steps per stream: the pipeline's fill and drain (one step's
+        # kernels and output copy after the last input copy) are amortised
+        n_e2e = 10 * NS
         for k in range(n_e2e):
             e2e_step(k)
         for st in streams[1:]:
