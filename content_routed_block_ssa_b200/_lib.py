@@ -77,6 +77,7 @@ def _load():
         "ssa_hier_nodes": (i32, [P, H, vp, vp, vp]),
         "ssa_route_hier_workspace_size": (sz, [P, H]),
         "ssa_route_hier": (i32, [P, H, vp, vp, vp, vp, vp, vp, sz, vp]),
+        "ssa_selftest_wait_timeout": (i32, [vp]),
     }
     for name, (res, args) in sig.items():
         f = getattr(lib, name)
@@ -92,7 +93,8 @@ EXPORTED = ("ssa_status_string", "ssa_version", "ssa_launch_count", "ssa_device_
             "ssa_attn_workspace_size", "ssa_sparse_attn", "ssa_attn_plan", "ssa_attn_blocks",
             "ssa_attn_window", "ssa_attn_merge",
             "ssa_workspace_size", "ssa_forward", "ssa_hostio_buffer_size", "ssa_forward_hostio",
-            "ssa_hier_nodes_size", "ssa_hier_nodes", "ssa_route_hier_workspace_size", "ssa_route_hier")
+            "ssa_hier_nodes_size", "ssa_hier_nodes", "ssa_route_hier_workspace_size", "ssa_route_hier",
+            "ssa_selftest_wait_timeout")
 
 
 def status_string(s: int) -> str:
@@ -280,3 +282,11 @@ def hier_node_views(p, hp, nodes):
     rad = nodes[r_off:r_off + bgs * nn * 4].view(torch.float32).view(p.batch, p.h_kv, nn)
     bnd = nodes[b_off:b_off + bgs * 8].view(torch.float32).view(p.batch, p.h_kv, 2)
     return rows, rad, bnd
+
+
+SITE_SELFTEST = 0x7F1
+
+
+def ssa_selftest_wait_timeout(stream=None):
+    """Launches the failure-path self-test kernel (a wait that times out after 1 s)."""
+    _check(lib.ssa_selftest_wait_timeout(_stream(stream)), "ssa_selftest_wait_timeout")

@@ -36,6 +36,7 @@ enum WaitSite : uint32_t {
   SITE_WIN_MMA = 0x502,
   SITE_WIN_SOFTMAX = 0x503,
   SITE_WIN_SMEM = 0x504,       // the aligned shared-memory layout did not fit its allocation
+  SITE_SELFTEST = 0x7F1,       // the failure-path self-test: a wait that nothing completes
 };
 
 // A single wait gives up after this long (legitimate waits last microseconds).

@@ -812,4 +812,11 @@ ssa_status ssa_route_hier(const ssa_params* pp, const ssa_hier_params* hp, const
   return do_route_hier(p, *hp, Q, route_table, nodes, block_idx, certified, static_cast<uint8_t*>(ws), c);
 }
 
+ssa_status ssa_selftest_wait_timeout(void* stream) {
+  LaunchCtx c;
+  ssa_status st = make_ctx(stream, c);
+  if (st != SSA_OK) return st;
+  return from_cuda(ssa::launch_selftest_wait(c));
+}
+
 }  // extern "C"

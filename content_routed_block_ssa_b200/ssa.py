@@ -6,4 +6,4 @@ from ._lib import (SSAError, lib, make_params, ssa_block_summary, ssa_device_err
                    ssa_attn_workspace_size, ssa_attn_plan, ssa_attn_blocks, ssa_attn_window, ssa_attn_merge,
                    ssa_workspace_size, status_string, ssa_hier_params, make_hier_params,
                    ssa_hier_nodes_size, ssa_hier_nodes, ssa_route_hier_workspace_size, ssa_route_hier,
-                   hier_node_views, summary_shapes, idx_shape, byte_buffer, EXPORTED, LIB_PATH)
+                   hier_node_views, ssa_selftest_wait_timeout, SITE_SELFTEST, summary_shapes, idx_shape, byte_buffer, EXPORTED, LIB_PATH)

@@ -358,6 +358,18 @@ SSA_API ssa_status ssa_route_hier(const ssa_params* p, const ssa_hier_params* hp
                                   const void* route_table, const void* nodes, int32_t* block_idx,
                                   uint8_t* certified, void* ws, size_t ws_bytes, void* stream);
 
+/*
+ * Self-test of the failure path (not part of the layer).  Launches on
+ * `stream` one kernel that waits on an mbarrier nothing arrives at, through
+ * the bounded wait every kernel of the library uses: after the wait limit
+ * (1 s) it records SSA_SITE_SELFTEST in the device failure word and returns.
+ * After synchronising, ssa_device_error reports SSA_ERR_DEVICE with that
+ * code (and clears it); the context stays usable.  Returns SSA_OK once the
+ * kernel is launched.
+ */
+#define SSA_SITE_SELFTEST 0x7F1u
+SSA_API ssa_status ssa_selftest_wait_timeout(void* stream);
+
 #ifdef __cplusplus
 }
 #endif

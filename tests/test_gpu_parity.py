@@ -450,3 +450,29 @@ def test_block_major_one_key_window_and_single_block():
     for i in range(63):                          # no full block yet: o = v_i for every head
         for h in range(w.h_q):
             np.testing.assert_allclose(got[0, i, h], Vn[0, i, h // (w.h_q // w.h_kv)], atol=1e-2)
+
+
+def test_bounded_wait_gives_up_reports_its_site_and_leaves_the_context_usable():
+    """A wait that nothing completes (the library's self-test kernel) gives up
+    after the 1 s limit, names its site in the failure word, which reading
+    clears, and the layer still runs correctly on the same context."""
+    import time
+    torch.cuda.synchronize()
+    assert ssa.ssa_device_error() == 0
+    t0 = time.perf_counter()
+    ssa.ssa_selftest_wait_timeout()
+    torch.cuda.synchronize()
+    dt = time.perf_counter() - t0
+    assert 0.9 < dt < 60, dt
+    assert ssa.ssa_device_error() == ssa.SITE_SELFTEST
+    assert ssa.ssa_device_error() == 0
+    c = case("bf16_gqa4_d128_b64")
+    p = params(c["pd"])
+    Q, K, V = to_dev(c["Q"], c["K"], c["V"])
+    ws = ssa.byte_buffer(ssa.ssa_workspace_size(p))
+    O_ = torch.empty_like(Q)
+    ssa.ssa_forward(p, Q, K, V, O_, None, ws)
+    check_no_device_error()
+    keep = np.all(c["ref"]["gaps"] >= NEAR_TIE_BAND, axis=2)
+    max_abs, rel, ok = compare_out(as_np(O_)[keep], c["ref"]["O"][keep], "bf16")
+    assert ok, (max_abs, rel)
