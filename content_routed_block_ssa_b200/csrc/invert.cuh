@@ -52,7 +52,11 @@ struct SlotSet {
 __device__ __forceinline__ SlotSet row_slots(int v_in, int topk, int64_t pos, int nb, int block, int window) {
   const int lane = threadIdx.x & 31;
   const int v = lane < topk ? v_in : -1;
-  const int nvis = static_cast<int>(min(static_cast<int64_t>(nb), (pos + 1) / block));
+  // positions are below 2^31 and the block is a power of two (64 or 128):
+  // 32-bit shifts instead of 64-bit divisions
+  const int p32 = static_cast<int>(pos);
+  const int lb = __ffs(block) - 1;
+  const int nvis = min(nb, (p32 + 1) >> lb);
   const bool inrange = v >= 0 && v < nvis;
   int run = inrange ? v : -1;
 #pragma unroll
@@ -67,9 +71,10 @@ __device__ __forceinline__ SlotSet row_slots(int v_in, int topk, int64_t pos, in
   s.v = v;
   s.mask = __ballot_sync(0xFFFFFFFFu, valid);
   s.n_bad = __popc(__ballot_sync(0xFFFFFFFFu, v != -1 && !valid));
-  s.lo = pos - window + 1 > 0 ? pos - window + 1 : 0;
-  s.b0 = s.lo / block;
-  const int nwb = static_cast<int>(pos / block - s.b0) + 1;
+  const int lo32 = max(p32 - window + 1, 0);
+  s.lo = lo32;
+  s.b0 = lo32 >> lb;
+  const int nwb = (p32 >> lb) - (lo32 >> lb) + 1;
   // window block w is uncovered unless some used entry selects it: each
   // lane marks the window block its own entry covers, OR over the warp
   const int64_t w = static_cast<int64_t>(v) - s.b0;
