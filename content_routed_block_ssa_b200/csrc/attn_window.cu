@@ -314,12 +314,13 @@ __global__ void __launch_bounds__(WinCfg<G>::THREADS, 1)
       if (!valid) { klo = 1; khi = 0; }
       klo -= span0;
       khi -= span0;
-      const int b0 = max(w0, 0) / a.block;
+      const int lbk = __ffs(a.block) - 1;   // the block is a power of two (64 or 128)
+      const int b0 = max(w0, 0) >> lbk;
       const uint32_t win = valid ? __ldg(a.win + static_cast<int64_t>(w.bg) * a.n_q + i) : 0u;
       // columns [c_lo, c_hi] of span block kb hold this row's keys (empty
       // when c_lo > c_hi); a selected block contributes none
       auto cols = [&](int kb, int& c_lo, int& c_hi) {
-        const int wb = (span0 + kb * 64) / a.block - b0;
+        const int wb = ((span0 + kb * 64) >> lbk) - b0;
         const bool open = wb >= 0 && wb < 32 && ((win >> wb) & 1u);
         c_lo = max(klo - kb * 64, 0);
         c_hi = min(khi - kb * 64, 63);

@@ -94,8 +94,14 @@ __host__ __device__ inline bool chunk_has_keys(uint32_t win, int64_t pos, int wi
   if (khi > pos) khi = pos;
   if (klo < 0) klo = 0;
   if (khi < klo) return false;
-  const int64_t b0 = (w0 > 0 ? w0 : 0) / block;
-  const int f = static_cast<int>(klo / block - b0), l = static_cast<int>(khi / block - b0);
+  // non-negative keys below 2^31 and a power-of-two block: shifts
+#ifdef __CUDA_ARCH__
+  const int lb = __ffs(block) - 1;
+#else
+  const int lb = __builtin_ctz(static_cast<unsigned>(block));
+#endif
+  const int b0 = static_cast<int>(w0 > 0 ? w0 : 0) >> lb;
+  const int f = (static_cast<int>(klo) >> lb) - b0, l = (static_cast<int>(khi) >> lb) - b0;
   const uint32_t span = (l - f + 1 >= 32) ? 0xFFFFFFFFu : ((1u << (l - f + 1)) - 1u);
   return ((win >> f) & span) != 0;
 }

@@ -795,6 +795,9 @@ __global__ void __launch_bounds__(256) route_qtile_f32_kernel(const float* __res
       stage();
     }
     float best = -INFINITY;   // threads < QT: the query's best sub-block score
+    const int iq = i0 + static_cast<int>(threadIdx.x);   // threads < QT: their query's visible blocks
+    const int nvq = threadIdx.x < QT && iq < a.n_q
+                        ? static_cast<int>(min(static_cast<int64_t>(a.nb), (a.q_offset + iq + 1) / a.block)) : 0;
     for (int u = 0; u < nrow; ++u) {
       __syncthreads();   // row u staged, the previous row's scores consumed
       if (u + 1 < nrow) fetch(u + 1);
@@ -844,10 +847,8 @@ __global__ void __launch_bounds__(256) route_qtile_f32_kernel(const float* __res
         for (int h = 0; h < G; ++h) gsum += sc[threadIdx.x * G + h];
         best = fmaxf(best, gsum);
         if (sb == a.S - 1) {
-          const int qq = threadIdx.x, i = i0 + qq;
-          const int64_t pos = a.q_offset + i;
-          const bool vis = i < a.n_q && cb < min(static_cast<int64_t>(a.nb), (pos + 1) / a.block);
-          keys[qq * n2 + cb] = vis ? make_key(__float_as_uint(best), cb) : 0ull;
+          const int qq = threadIdx.x;
+          keys[qq * n2 + cb] = cb < nvq ? make_key(__float_as_uint(best), cb) : 0ull;
           best = -INFINITY;
         }
       }
