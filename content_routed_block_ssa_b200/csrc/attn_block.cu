@@ -870,8 +870,9 @@ __global__ void __launch_bounds__(256, (G == 8 ? 2 : (G == 4 ? 3 : 4))) attn_mer
   const int lane = threadIdx.x & 31;
   const int64_t item = static_cast<int64_t>(blockIdx.x) * 8 + (threadIdx.x >> 5);
   if (item >= a.n_items) return;   // warp-uniform
-  const int i = static_cast<int>(item % a.n_q);
-  const int bg = static_cast<int>(item / a.n_q);
+  const int it32 = static_cast<int>(item);   // items (b * h_kv * n_q) fit 31 bits
+  const int i = it32 % a.n_q;
+  const int bg = it32 / a.n_q;
   const int b = bg / a.h_kv, g = bg % a.h_kv;
   const int v = lane < a.topk ? __ldg(a.idx + ((static_cast<int64_t>(b) * a.n_q + i) * a.h_kv + g) * a.topk + lane) : -1;
   SlotSet s = row_slots(v, a.topk, a.q_offset + i, a.nb, a.block, a.window);

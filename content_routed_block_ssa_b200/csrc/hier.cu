@@ -192,9 +192,11 @@ __global__ void __launch_bounds__(256) hier_probe_kernel(const HierProbeArgs a) 
   if (w >= static_cast<int64_t>(a.bgs) * a.n_q) return;
   const int bg = static_cast<int>(w / a.n_q), i = static_cast<int>(w % a.n_q);
   const int b = bg / a.h_kv, g = bg % a.h_kv;
-  const int64_t pos = a.q_offset + i;
-  const int nv = static_cast<int>(min(static_cast<int64_t>(a.nb), (pos + 1) / a.block));
-  const int nvn = static_cast<int>(min(static_cast<int64_t>(a.nn), (pos + 1) / (static_cast<int64_t>(a.block) * a.M)));
+  // key positions fit 31 bits and B, M are powers of two: shifts
+  const int pos1 = static_cast<int>(a.q_offset) + i + 1;
+  const int lbb = __ffs(a.block) - 1;
+  const int nv = min(a.nb, pos1 >> lbb);
+  const int nvn = min(a.nn, pos1 >> (lbb + __ffs(a.M) - 1));
   const int64_t row = (static_cast<int64_t>(b) * a.n_q + i) * a.h_kv + g;
 
   float f[FPL];
