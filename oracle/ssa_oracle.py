@@ -318,6 +318,16 @@ def route_topk(Q: np.ndarray, stored, p: Problem, rows=None):
     return bidx, gaps
 
 
+def route_topk_unquantised(Q: np.ndarray, stored, p: Problem, rows=None):
+    """The selection of a bf16 problem without its bf16 rounding of features
+    and summaries, for information: the same cumulant scores from the float64
+    query heads and the float32 summaries, i.e. exactly what the float32
+    problem computes (``route_topk`` on a float32 copy of the problem)."""
+    mu32, sig32, _table = stored
+    q32 = Problem(**{**p.__dict__, "dtype": F32})
+    return route_topk(Q, (mu32, sig32, None), q32, rows)
+
+
 # ---------------------------------------------------------------- step 4
 
 def key_set(pos: int, sel: np.ndarray, p: Problem) -> np.ndarray:

@@ -691,3 +691,25 @@ def test_hier_certificate_hand_cases_radius_and_margin():
     for e, want in ((2.0 ** -12, False), (2.0 ** -10, True)):
         kept, ok, info = row(t2, [1, e, 0, 0], 1, 1, 1)
         assert list(kept) == [0] and ok is want
+
+
+def test_unquantised_selection_is_the_float32_route_of_the_same_summaries():
+    """The informational unquantised selection of a bf16 problem is the float32
+    problem's selection from the float32 summaries, and its scores are the
+    sum over the group's heads of <q_h, mu> + (beta/2) q_h^2 . sigma^2 from
+    the float64 query heads (checked row by row against a direct sum)."""
+    rng = np.random.default_rng(41)
+    p = O.Problem(1, 96, 96, 4, 2, 8, 4, 3, 4, dtype=O.BF16, sigma=O.DIAG)
+    K = O.round_bf16(rng.standard_normal((1, 96, 2, 8)))
+    Q = O.round_bf16(rng.standard_normal((1, 96, 4, 8)))
+    stored = O.stored_summaries(*O.block_summaries(K, p), p)
+    bidx, gaps = O.route_topk_unquantised(Q, stored, p)
+    mu32, sig32, _ = stored
+    for i in range(0, 96, 5):
+        for g in range(2):
+            nv = O.visible_blocks(i, p)
+            qh = Q[0, i, 2 * g:2 * g + 2]
+            sc = np.array([sum(qh[h] @ mu32[0, g, c] + 1.0 * (qh[h] ** 2) @ sig32[0, g, c] for h in range(2))
+                           for c in range(nv)])
+            want, _ = O.select_topk(sc, p.topk)
+            np.testing.assert_array_equal(bidx[0, i, g], want)
