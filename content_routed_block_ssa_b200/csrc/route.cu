@@ -492,12 +492,6 @@ struct RowArgs {
   const uint8_t* skip;       // optional [b, n_q, h_kv]: rows whose byte is nonzero are skipped
 };
 
-__device__ __forceinline__ int next_pow2(int x) {
-  int p = 1;
-  while (p < x) p <<= 1;
-  return p;
-}
-
 // Writes the top-k of keys[0..n) (distinct and nonzero: a block index in
 // the low half) in ascending block order.  A radix select, most significant
 // 8-bit digit first, finds the k-th largest key: per digit, a histogram of
