@@ -713,3 +713,27 @@ def test_unquantised_selection_is_the_float32_route_of_the_same_summaries():
                            for c in range(nv)])
             want, _ = O.select_topk(sc, p.topk)
             np.testing.assert_array_equal(bidx[0, i, g], want)
+
+
+def test_hier_bound_constants_are_the_largest_radius_and_row_norm():
+    """R* is the largest node radius and T* the largest 2-norm over the block
+    rows and the node rows of each (batch, kv-head), rounded up to float32; a
+    node row can be longer than every block row (its cap takes each
+    dimension's largest variance)."""
+    rng = np.random.default_rng(43)
+    d, nb, M = 4, 16, 4
+    mu = np.zeros((1, 2, nb, d))
+    sg = np.zeros((1, 2, nb, d))
+    for c in range(nb):                       # block c's variance sits in one dimension only
+        sg[0, :, c, c % d] = 4.0
+    mu[0, 1] = O.round_bf16(rng.standard_normal((nb, d)))
+    table = np.concatenate([mu, sg], -1)
+    nt, rad, r_star, t_star = O.hier_nodes(table, M)
+    for g in range(2):
+        assert r_star[0, g] == rad[0, g].max()
+        norms = [np.linalg.norm(table[0, g, c]) for c in range(nb)] + \
+                [np.linalg.norm(nt[0, g, N]) for N in range(nb // M)]
+        assert max(norms) <= t_star[0, g] <= max(norms) * (1 + 2.0 ** -23)
+    # kv-head 0: every block row has norm 4, every node row (cap 4 in all four
+    # dimensions) norm 8
+    assert t_star[0, 0] == 8.0
