@@ -151,7 +151,33 @@ __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity, uint3
 // (lanes past their own count insert -inf, which changes nothing).
 template <int KSEL>
 __device__ __forceinline__ void merge_candidates(float (&Ls)[KSEL], int (&Li)[KSEL], int& cnt, float& thr,
-                                                 const uint2* my_cand, int k) {
+                                                 const uint2* my_cand, int k, bool empty_list) {
+  if constexpr (KSEL == 32) {
+    // the first merge of a row (its list still empty, at most 32 candidates):
+    // one 32-key sorting network instead of 32 insertions; the keys order
+    // (score desc, block asc), the insertions' order
+    if (empty_list) {
+      uint64_t key[32];
+#pragma unroll
+      for (int t = 0; t < 32; ++t) {
+        const uint2 e = t < cnt ? my_cand[t * 128] : make_uint2(0u, 0u);
+        key[t] = t < cnt ? make_key(e.x, e.y) : 0ull;
+      }
+      bitonic_sort_desc<32>(key);
+#pragma unroll
+      for (int j = 0; j < 32; ++j) {
+        Ls[j] = key[j] ? key_score(key[j]) : -INFINITY;
+        Li[j] = key[j] ? static_cast<int>(key_block(key[j])) : -1;
+      }
+      cnt = 0;
+      float kth = INFINITY;
+#pragma unroll
+      for (int j = 0; j < KSEL; ++j)
+        if (j < k) kth = fminf(kth, Ls[j]);
+      thr = kth;
+      return;
+    }
+  }
   int n = cnt;
 #pragma unroll
   for (int o = 16; o; o >>= 1) n = max(n, __shfl_xor_sync(0xFFFFFFFFu, n, o));
@@ -398,6 +424,7 @@ __global__ void __launch_bounds__(TiledCfg<KF>::THREADS, 1)
       for (int j = 0; j < KSEL; ++j) { Ls[j] = -INFINITY; Li[j] = -1; }
       float thr = -INFINITY;
       int cnt = 0;
+      bool empty_list = true;   // warp-uniform: no merge of this unit yet
       for (int j = 0; j < nch; ++j) {
         const int acc = 2 * (ch_cnt & 1) + grp;
         ok = __all_sync(0xFFFFFFFFu, mbar_wait(&acc_full[acc], (ch_cnt >> 1) & 1, a.err, SITE_ROUTE_EPILOGUE));
@@ -421,12 +448,15 @@ __global__ void __launch_bounds__(TiledCfg<KF>::THREADS, 1)
             filter_group<2>(v, c0, nvis, thr, cnt, my_cand);
           else
             filter_group<4>(v, c0, nvis, thr, cnt, my_cand);
-          if (__any_sync(0xFFFFFFFFu, cnt > C::CAP - 16)) merge_candidates<KSEL>(Ls, Li, cnt, thr, my_cand, a.topk);
+          if (__any_sync(0xFFFFFFFFu, cnt > C::CAP - 16)) {
+            merge_candidates<KSEL>(Ls, Li, cnt, thr, my_cand, a.topk, empty_list);
+            empty_list = false;
+          }
         }
         ++ch_cnt;
       }
       if (!ok) break;
-      if (__any_sync(0xFFFFFFFFu, cnt > 0)) merge_candidates<KSEL>(Ls, Li, cnt, thr, my_cand, a.topk);
+      if (__any_sync(0xFFFFFFFFu, cnt > 0)) merge_candidates<KSEL>(Ls, Li, cnt, thr, my_cand, a.topk, empty_list);
       if (valid) {
         uint32_t ob[KSEL];
         float os[KSEL];
