@@ -209,3 +209,23 @@ def test_hier_params_layout_and_checks():
                                   None) == ssa.SSA_ERR_WORKSPACE
     e = good(batch=0)
     assert ssa.lib.ssa_route_hier(C.byref(e), C.byref(ok), None, None, None, None, None, None, 0, None) == ssa.SSA_OK
+
+
+def test_hier_node_views_match_the_node_store_layout():
+    """The binding's views of a node store (rows, radii, bounds) tile the
+    buffer the size call asks for, at the documented 256-byte-aligned offsets."""
+    import torch
+    for kw, M in ((dict(n_q=1000, n_kv=4096), 8), (dict(batch=2, n_kv=4288, n_q=4288, h_q=8, h_kv=2), 16),
+                  (dict(n_kv=8192, n_q=1, q_offset=8191, d=64), 4)):
+        p = good(**kw)
+        hp = ssa.make_hier_params(fanout=M, probe=2)
+        size = ssa.ssa_hier_nodes_size(p, hp)
+        buf = torch.zeros(size, dtype=torch.uint8)
+        rows, rad, bnd = ssa.hier_node_views(p, hp, buf)
+        nn = (p.n_kv // p.block) // M
+        assert rows.shape == (p.batch, p.h_kv, nn, 2 * p.d) and rad.shape == (p.batch, p.h_kv, nn)
+        base = buf.data_ptr()
+        assert rows.data_ptr() == base
+        assert (rad.data_ptr() - base) % 256 == 0 and rad.data_ptr() - base >= rows.numel() * 2
+        assert (bnd.data_ptr() - base) % 256 == 0 and bnd.data_ptr() - base >= rad.data_ptr() - base + rad.numel() * 4
+        assert bnd.data_ptr() - base + bnd.numel() * 4 <= size
