@@ -325,6 +325,18 @@ typedef struct {
 } ssa_hier_params;
 
 /*
+ * Errors of the hierarchical calls, checked before any launch: the
+ * ssa_params checks of the other calls; hp NULL, reserved != 0, fanout not a
+ * power of two in 1..64, probe outside 1..31 or escalate not 0/1 ->
+ * SSA_ERR_INVALID_ARG; (probe + 1) * fanout > 512 (the probe's candidate
+ * capacity), a float32 problem or subblocks != 1 -> SSA_ERR_UNSUPPORTED;
+ * NULL or misaligned (not 16-byte) pointers -> SSA_ERR_INVALID_ARG; a
+ * workspace smaller than ssa_route_hier_workspace_size ->
+ * SSA_ERR_WORKSPACE.  Empty problems (batch or n_q 0) return SSA_OK without
+ * a launch.  The size calls return 0 on any of these.
+ */
+
+/*
  * Bytes of the node store of (p, hp): the node rows (bf16 [b, h_kv, nn, 2d],
  * at offset 0), the radii (float32 [b, h_kv, nn], at offset
  * round_up(node row bytes, 256)) and two floats per (batch, kv-head) (largest
