@@ -332,8 +332,9 @@ typedef struct {
  * capacity), a float32 problem or subblocks != 1 -> SSA_ERR_UNSUPPORTED;
  * NULL or misaligned (not 16-byte) pointers -> SSA_ERR_INVALID_ARG; a
  * workspace smaller than ssa_route_hier_workspace_size ->
- * SSA_ERR_WORKSPACE.  Empty problems (batch or n_q 0) return SSA_OK without
- * a launch.  The size calls return 0 on any of these.
+ * SSA_ERR_WORKSPACE.  ssa_route_hier returns SSA_OK without a launch when
+ * batch or n_q is 0, ssa_hier_nodes when batch is 0.  The size calls return
+ * 0 on any of these errors.
  */
 
 /*
