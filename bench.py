@@ -1,7 +1,8 @@
 """Benchmark of the SSA forward on B200: query-heads/s at 128K (and 1M) tokens.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload NAME] [--no-secondary]
+                    [--workload NAME] [--no-secondary] [--no-cpu-baseline] [--no-e2e]
+                    [--subblocks S] [--router flat|hier [--fanout M] [--probe P] [--escalate]]
 
 One step is one pass of the whole layer over the workload's synthetic input:
 block summaries -> routing features + tensor-core route with fused top-k ->
@@ -11,7 +12,11 @@ calls).  Inputs are resident in HBM when the timed region starts; L2 is
 flushed between steps.  Step time is the sum of CUDA-event intervals around
 the step's kernels, the reported time the max over ranks.  With N > 1 every
 rank runs its own replica of the workload (independent problems, no
-collective on the data path): weak scaling.
+collective on the data path): weak scaling.  The decode workload's block
+summaries (and, with --router hier, its node store) are precomputed state of
+the cache: built once before the timed steps and reported beside them.  The
+line gives the mean and the median step time, and the dominant kernel's
+roofline fraction against the measured peaks and the nominal ones.
 
 `e2e` repeats the step through ssa_forward_hostio with page-locked host
 inputs and outputs, every step's host<->device copies inside the timed
