@@ -15,7 +15,8 @@
 //     f . T_c <= f . [m_N ; v_N] + ||f_s|| R_N.
 //
 // A row ranks its complete visible nodes by w_N = f . [m_N ; v_N] (the
-// tensor-core router run over the node table, top probe+1 with scores),
+// block router run over the node table, tensor-core tiles or one CTA per
+// row, keeping the top probe+1 with their scores),
 // scores the blocks of the best `probe` nodes and the visible blocks outside
 // complete nodes exactly, and keeps their top-k.  It is certified when no
 // complete visible node is left, or when the k-th kept score exceeds
