@@ -51,3 +51,25 @@ def test_block_major_counts_by_direct_count():
                     if 0 <= v < nvis:
                         last = max(last, int(v))
         assert (n_e, n_b) == (used, len(blocks))
+
+
+def test_kernel_report_fractions_and_dominant_stage():
+    """On a synthetic result the report's achieved rates are the algorithmic
+    work over the stage time, its fractions those rates over the peaks, and
+    the dominant stage the longest bounded one (decode state excluded)."""
+    w, p, idx = _case()
+    work = bench.algorithmic_work(w, torch.from_numpy(idx))
+    ms = {"summary": 0.5, "route": 2.0, "attn_plan": 0.1, "attn_blocks": 4.0, "attn_window": 0.3,
+          "attn_merge": 1.0}
+    peaks = {"hbm_gbs": 6000.0, "bf16_tflops": 1600.0, "bf16_tflops_sustained": 1400.0}
+    rep = bench.kernel_report(w, {"ms_kernels": ms, "work": work}, peaks, {})
+    for name in ("summary", "attn_plan", "attn_merge"):
+        e = rep[name]
+        assert abs(e["achieved"] - e["algorithmic_bytes"] / (ms[name] * 1e-3) / 1e9) < 1e-6 * e["achieved"]
+        assert abs(e["frac"] - e["achieved"] / 6000.0) < 1e-12
+    r = rep["route"]
+    assert r["bound"] == "tensor" and abs(r["achieved"] - work["route_flops"] / 2e-3 / 1e12) < 1e-9 * r["achieved"]
+    assert abs(r["frac"] - r["achieved"] / 1400.0) < 1e-12
+    name, d = bench.dominant(rep)
+    assert name == "attn_blocks" and d["ms"] == 4.0
+    assert bench.dominant(rep, exclude=("attn_blocks",))[0] == "route"
