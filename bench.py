@@ -611,7 +611,7 @@ def main():
     if a.impl == "reference":
         if rank != 0:
             return
-        rows = 4
+        rows = 16
         val, sec, info = run_oracle_sample(w, rows, a.steps, a.warmup)
         line = {"impl": "reference", "metric": METRIC, "value": val, "unit": UNIT, "n_gpus": a.gpus,
                 "steps": a.steps, "warmup": a.warmup, "ms_per_step": sec * 1e3, "higher_is_better": True,
@@ -656,7 +656,7 @@ def main():
                      "clocks": r2["clocks"]}
     cpu = None
     if rank == 0 and ws == 1 and not a.no_cpu_baseline:
-        rows = 16
+        rows = 256   # ~10-15 s of host work with the full block summaries
         val, sec, info = run_oracle_sample(w, rows, 2, 1)
         cpu = {"value": val, "unit": UNIT, "cores": cores(), "kind": "oracle",
                "sample": f"{rows} query rows x {w.h_q} heads per step, block summaries of all {w.n} keys "
