@@ -232,6 +232,63 @@ def test_bf16_features_exact_case_equals_group_score():
     np.testing.assert_allclose(S[40, :2], O.route_scores_row(Q, stored, p, 0, 40, 1), rtol=1e-14)
 
 
+def _golden_feature_query(g):
+    """The golden query as a [1, 1, G, d] array (heads by dimension in the file)."""
+    return np.asarray(g["q_heads_by_dim"], dtype=np.float64).T[None, None]
+
+
+def _bf16_torch(x):
+    return torch.from_numpy(np.asarray(x, dtype=np.float32)).to(torch.bfloat16).double().numpy()
+
+
+def _feature_variant(Q, beta, order="forward", acc=np.float32, round_first=False):
+    """Routing features of a wrong-on-purpose variant: heads summed in another
+    order, in another precision, or the squared sum rounded to bf16 before the
+    (beta/2) multiply.  Rounding by torch, so nothing here is the oracle's."""
+    q = np.asarray(Q[0, 0], dtype=acc)                      # [G, d]
+    heads = range(q.shape[0]) if order == "forward" else reversed(range(q.shape[0]))
+    qs = np.zeros(q.shape[1], dtype=acc)
+    qq = np.zeros(q.shape[1], dtype=acc)
+    for h in heads:
+        qs = (qs + q[h]).astype(acc)
+        qq = (qq + q[h] * q[h]).astype(acc)
+    hb = np.float32(beta / 2)
+    if round_first:
+        fq = _bf16_torch((hb * _bf16_torch(qq).astype(np.float32)).astype(np.float32))
+    else:
+        fq = _bf16_torch((hb * qq).astype(np.float32) if acc == np.float32 else hb * qq)
+    return np.concatenate([_bf16_torch(qs), fq])
+
+
+def test_bf16_features_golden_rounding_order():
+    """Hand-derived case (tests/golden/feature_rounding.json) in which the
+    float32 head-order sums, the float32 (beta/2) multiply and the final
+    round-to-nearest-even each decide a feature: the oracle must give the
+    derived values, and summing in float64, summing the heads in reverse
+    order, or rounding the squared sum before the (beta/2) multiply must each
+    give a different (also hand-derived) row."""
+    g = golden("feature_rounding.json")
+    Q = _golden_feature_query(g)
+    d, G = g["d"], g["G"]
+    p = O.Problem(batch=1, n_q=1, n_kv=64, h_q=G, h_kv=1, d=d, block=16, topk=2, window=16,
+                  dtype=O.BF16, sigma=O.DIAG, beta=g["beta"])
+    f = O.route_features(Q, p)[0, 0, 0]
+    assert np.array_equal(f, np.asarray(g["features"]))
+    variants = {
+        "features_reversed_head_order": _feature_variant(Q, g["beta"], order="reversed"),
+        "features_float64_sums": _feature_variant(Q, g["beta"], acc=np.float64),
+        "features_rounded_before_half_beta": _feature_variant(Q, g["beta"], round_first=True),
+    }
+    for key, v in variants.items():
+        assert np.array_equal(v, np.asarray(g[key])), key
+        assert not np.array_equal(v, f), key
+    # the correct variant written the same way reproduces the oracle
+    assert np.array_equal(_feature_variant(Q, g["beta"]), f)
+    # and the routing score against a unit table row reads one feature back
+    table = np.eye(2 * d)
+    assert np.array_equal(table @ f, f)
+
+
 def test_visible_blocks_brute_force():
     p = small_problem(n_kv=64, block=8)
     for pos in range(64):
