@@ -229,3 +229,25 @@ def test_hier_node_views_match_the_node_store_layout():
         assert (rad.data_ptr() - base) % 256 == 0 and rad.data_ptr() - base >= rows.numel() * 2
         assert (bnd.data_ptr() - base) % 256 == 0 and bnd.data_ptr() - base >= rad.data_ptr() - base + rad.numel() * 4
         assert bnd.data_ptr() - base + bnd.numel() * 4 <= size
+
+
+def test_binding_refuses_strided_tensors_before_calling_the_library():
+    """The C ABI reads dense row-major buffers.  A tensor whose memory is in
+    another order (here [b, nb, h_kv, d] memory viewed as [b, h_kv, nb, d],
+    what a reduction over a transposed NumPy array gives) is refused by the
+    binding; nothing reaches the library."""
+    import numpy as np
+    import torch
+    p = good(dtype="f32")
+    mem = torch.zeros(1, 4, 2, 128)                  # [b, nb, h_kv, d] in memory
+    mu = mem.transpose(1, 2)                         # viewed as [b, h_kv, nb, d]
+    assert not mu.is_contiguous()
+    before = ssa.ssa_launch_count()
+    with pytest.raises(ValueError, match="dense row-major"):
+        ssa.ssa_route_topk(p, torch.zeros(1, 256, 4, 128), mu, mu.contiguous(), None,
+                           torch.zeros(1, 256, 2, 4, dtype=torch.int32))
+    assert ssa.ssa_launch_count() == before
+    # the oracle's summaries are such arrays: a reduction keeps the source's order
+    K = np.zeros((1, 256, 2, 128))
+    m = K.reshape(1, 4, 64, 2, 128).transpose(0, 3, 1, 2, 4).sum(axis=3)
+    assert not torch.from_numpy(m).is_contiguous()
