@@ -15,9 +15,16 @@
  * Conventions shared by every call
  * --------------------------------
  *  * All tensors are dense, row-major, caller-owned DEVICE buffers unless a
- *    call says otherwise, and must be 16-byte aligned.  The library allocates
- *    no memory and keeps no per-call state; scratch comes from the caller's
- *    workspace.
+ *    call says otherwise, and must be 16-byte aligned.  No call allocates
+ *    memory and none keeps per-call state; scratch comes from the caller's
+ *    workspace.  The library's own device footprint is fixed: a 4-byte
+ *    failure word and the 16 MiB scratch array of ssa_route_topk_static
+ *    (below), both module globals that exist on a device once the module
+ *    holding them is loaded there.
+ *  * Per device the library caches the addresses of those globals and the
+ *    SM count the first time a call runs on it.  A cudaDeviceReset destroys
+ *    the globals, so the library must not be used on a device after it has
+ *    been reset in the same process.
  *  * Layouts (b = batch, nb = n_kv / block, G = h_q / h_kv):
  *      Q, O        [b, n_q,  h_q,  d]   elements of `dtype`
  *      K, V        [b, n_kv, h_kv, d]   elements of `dtype`
@@ -86,7 +93,7 @@ typedef enum {
   SSA_ROUTE_ROWWISE = 2 /* one CTA per query row (decode-shaped work)          */
 } ssa_route_impl;
 
-/* 64 bytes, no padding: twelve int32, one int64, two float32. */
+/* 72 bytes, no padding: twelve int32, one int64, two float32, two int32. */
 typedef struct {
   int32_t batch;      /* b                                               */
   int32_t n_q;        /* query rows per sequence                         */
@@ -245,11 +252,17 @@ SSA_API ssa_status ssa_attn_merge(const ssa_params* p, const int32_t* block_idx,
  * memory when they route (a host framework whose allocator owns the whole
  * device pool, or a loop that cannot afford cudaMalloc's implicit device
  * synchronisation).  The routing-feature scratch lives in a fixed array of
- * SSA_ROUTE_STATIC_SCRATCH_BYTES inside the library, present on every device
- * that loads it until the process exits; problems that need more return
- * SSA_ERR_WORKSPACE before any launch.  The first call on a device looks up
- * the array's address with that device current; make it before any stream
- * capture.  All calls share the array, so calls whose kernels overlap on the
+ * SSA_ROUTE_STATIC_SCRATCH_BYTES inside the library.  The array occupies
+ * device memory on every device where the module that holds it has been
+ * loaded, until the process exits: with CUDA's lazy module loading (the
+ * default) that is the first call of this function on the device, with
+ * eager loading (CUDA_MODULE_LOADING=EAGER) the first CUDA call of the
+ * process.  Problems that need more than the array return
+ * SSA_ERR_WORKSPACE before any launch: the routing features take
+ * batch * h_kv * n_q * 2d bf16 values (rounded up to 256 bytes), so at
+ * d = 128 at most 32768 (query row, kv-head) pairs fit.  The first call on
+ * a device looks up the array's address with that device current; make it
+ * before any stream capture.  All calls share the array, so calls whose kernels overlap on the
  * GPU race on it and must be serialised.  Arguments and results are those of
  * ssa_route_topk.  Allocates nothing.
  */

@@ -65,6 +65,20 @@ CASES = {
     "bf16_gqa4_d128_b64_w1985": Workload("c", 125, 1, 4096, 8, 2, 128, "bf16", 64, "diag", 8, 1985, 4, "total",
                                          clustered=True),
     "bf16_gqa4_d128_b64_w4032": Workload("c", 126, 1, 5120, 8, 2, 128, "bf16", 64, "diag", 8, 4032, 4, "total"),
+    # routing temperatures other than 2: beta = 0 (centroid routing: the
+    # variance half of every feature is zero), beta = 1 and beta = 3 (the
+    # (beta/2) multiply of the squared sum is then not the identity), on the
+    # tiled and row-wise routers, the block-major attention and float32
+    "bf16_gqa4_d128_b64_beta0": Workload("c", 127, 1, 1536, 8, 2, 128, "bf16", 64, "diag", 16, 256, 6, "total",
+                                         clustered=True, beta=0.0),
+    "bf16_mha_d128_b64_beta1": Workload("c", 128, 1, 1280, 2, 2, 128, "bf16", 64, "diag", 8, 128, 4, "per_head",
+                                        beta=1.0),
+    "bf16_gqa8_d128_b128_beta3": Workload("c", 129, 1, 2048, 8, 1, 128, "bf16", 128, "diag", 8, 256, 6, "total",
+                                          clustered=True, beta=3.0),
+    "bf16_gqa4_d64_b64_beta3": Workload("c", 130, 1, 1024, 8, 2, 64, "bf16", 64, "diag", 8, 64, 4, "total",
+                                        beta=3.0),
+    "f32_full_d64_beta3": Workload("c", 131, 1, 768, 2, 1, 64, "f32", 64, "full", 4, 64, 2, "total", beta=3.0),
+    "f32_diag_d128_beta0": Workload("c", 132, 1, 512, 4, 2, 128, "f32", 64, "diag", 4, 64, 2, "total", beta=0.0),
     # float32 routing takes runs of 32 (query, head) pairs per CTA unless a
     # row's 1024 block scores do not fit beside them: then one CTA per row
     "f32_diag_d64_decode_64k": Workload("c", 122, 1, 65536, 1, 1, 64, "f32", 64, "diag", 8, 64, 2, "per_seq",
@@ -108,10 +122,12 @@ def test_summary_bit_exact(name):
 
 
 def _stored_on_device(c):
+    # the oracle's arrays may keep the strides of a permuted source: the C ABI
+    # reads dense row-major buffers
     mu32, sig32, table = c["ref"]["stored"]
-    mu = torch.from_numpy(mu32.astype(np.float32)).cuda()
-    sig = torch.from_numpy(sig32.astype(np.float32)).cuda()
-    tab = torch.from_numpy(table).to(torch.bfloat16).cuda() if table is not None else None
+    mu = torch.from_numpy(np.ascontiguousarray(mu32, dtype=np.float32)).cuda()
+    sig = torch.from_numpy(np.ascontiguousarray(sig32, dtype=np.float32)).cuda()
+    tab = torch.from_numpy(np.ascontiguousarray(table)).to(torch.bfloat16).cuda() if table is not None else None
     return mu, sig, tab
 
 
@@ -154,6 +170,39 @@ def test_route_matches_oracle_selection(name, impl):
         if nv <= op.topk:
             assert list(gi[0, i, 0, :nv]) == list(range(nv))
             assert np.all(gi[0, i, 0, nv:] == -1)
+
+
+@pytest.mark.parametrize("impl", [ssa.SSA_ROUTE_TILED, ssa.SSA_ROUTE_ROWWISE], ids=["tiled", "rowwise"])
+def test_bf16_features_read_back_equal_golden_rounding(impl):
+    """The GPU's routing features on the hand-derived rounding case
+    (tests/golden/feature_rounding.json: beta = 3, eight query heads whose
+    float32 head-order sums, (beta/2) multiply and bf16 rounding each decide
+    a feature).  A routing table of unit rows e_t turns every score into one
+    feature, f . e_t = f_t, and with all 8 blocks selected top_scores returns
+    them in block order."""
+    import json
+    import os
+    with open(os.path.join(os.path.dirname(__file__), "golden", "feature_rounding.json")) as fh:
+        g = json.load(fh)
+    dg, G, d, B = g["d"], g["G"], 64, 64
+    nb = 2 * dg
+    n = nb * B
+    q = torch.zeros(G, d, dtype=torch.float64)
+    q[:, :dg] = torch.tensor(g["q_heads_by_dim"], dtype=torch.float64).T
+    assert torch.equal(q.to(torch.bfloat16).double(), q)          # every input is a bf16 value
+    Q = q.to(torch.bfloat16).expand(1, n, G, d).contiguous().cuda()
+    tab = torch.zeros(1, 1, nb, 2 * d, dtype=torch.bfloat16)
+    for t in range(dg):
+        tab[0, 0, t, t] = 1.0                 # block t reads f_s[t]
+        tab[0, 0, dg + t, d + t] = 1.0        # block dg + t reads f_q[t]
+    tab = tab.cuda()
+    p = ssa.make_params(batch=1, n_q=n, n_kv=n, h_q=G, h_kv=1, d=d, block=B, topk=nb, window=B,
+                        beta=g["beta"], route_impl=impl)
+    idx, sc = gpu_route(p, Q, None, None, tab)
+    check_no_device_error()
+    last = n - 1                                # the one row that sees all nb blocks
+    assert idx[0, last, 0].tolist() == list(range(nb))
+    assert sc[0, last, 0].double().cpu().tolist() == g["features"]
 
 
 @pytest.mark.parametrize("name", list(CASES))
