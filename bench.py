@@ -202,11 +202,19 @@ def attended_keys(idx, w):
     return n_sel * B + wcount - overlap
 
 
+HOT_BLOCKS = 128   # hot set size of the paired slots (64-key blocks)
+
+
 def block_major_counts(idx, w):
-    """Selected slots of the block-major attention, by the kernels' rule:
-    the used block_idx entries (in range, larger than every earlier in-range
-    entry of the row).  Returns the number of slots and of distinct (batch,
-    kv-head, block) lists they fall in."""
+    """Selected slots of the block-major attention, by the kernels' rules
+    (bookkeeping for the roofline, not part of the layer).  A row's used
+    entries are its in-range block_idx entries larger than every earlier
+    in-range entry.  With 64-key blocks the entries of each (batch, kv-head)'s
+    hot blocks (its at most HOT_BLOCKS most selected blocks: count >= T for
+    the smallest T >= 2 that keeps the set that small) pair up in block
+    order, two per slot; other entries are a slot each.  Returns (used
+    entries, slots, distinct tile keys: blocks, or pairs and single
+    blocks)."""
     nb = w.n // w.block
     B = w.block
     pos = torch.arange(w.n_q, device=idx.device, dtype=torch.int64).view(1, -1, 1, 1) + w.q_offset
@@ -216,12 +224,37 @@ def block_major_counts(idx, w):
     run = torch.cummax(torch.where(inr, v, torch.full_like(v, -1)), dim=-1).values
     prev = torch.cat([torch.full_like(run[..., :1], -1), run[..., :-1]], dim=-1)
     valid = inr & (v > prev)
-    sel = torch.where(valid, v, torch.full_like(v, -1))
+    sel = torch.where(valid, v, torch.zeros_like(v))
     n_entries = int(valid.sum().item())
     bgi = (torch.arange(w.batch, device=idx.device).view(-1, 1, 1, 1) * w.h_kv
-           + torch.arange(w.h_kv, device=idx.device).view(1, 1, -1, 1))
-    n_blocks = int(torch.unique((bgi * nb + sel)[valid]).numel())
-    return n_entries, n_blocks
+           + torch.arange(w.h_kv, device=idx.device).view(1, 1, -1, 1)).expand_as(v)
+    gkey = bgi * nb + sel
+    if w.block != 64:
+        return n_entries, n_entries, int(torch.unique(gkey[valid]).numel())
+    bgs = w.batch * w.h_kv
+    cnt = torch.bincount(gkey[valid], minlength=bgs * nb).view(bgs, nb)
+    srt = cnt.sort(dim=1, descending=True).values
+    c129 = srt[:, HOT_BLOCKS] if nb > HOT_BLOCKS else torch.zeros(bgs, dtype=cnt.dtype, device=cnt.device)
+    T = torch.clamp(c129 + 1, min=2)
+    hot_blk = cnt >= T[:, None]
+    hid_tab = torch.where(hot_blk, torch.cumsum(hot_blk.to(torch.int64), dim=1) - 1, torch.full_like(cnt, -1))
+    hid = torch.where(valid, hid_tab.view(-1)[gkey], torch.full_like(v, -1))
+    hot = hid >= 0
+    nhot = hot.sum(-1, keepdim=True)
+    npair = nhot // 2
+    n_slots = n_entries - int(npair.sum().item())
+    # pair keys: the hot entries in order, taken two at a time
+    order = torch.sort((~hot).to(torch.int8), dim=-1, stable=True).indices
+    hs = hid.gather(-1, order)
+    m = torch.arange(v.shape[-1] // 2, device=v.device)
+    first, second = hs[..., 0::2][..., :m.numel()], hs[..., 1::2][..., :m.numel()]
+    is_pair = m < npair
+    pkey = (bgi[..., :m.numel()] * (nb + HOT_BLOCKS * HOT_BLOCKS) + nb + first * HOT_BLOCKS + second)[is_pair]
+    rank = torch.cumsum(hot.to(torch.int64), dim=-1) - 1
+    single = valid & ~(hot & (rank < 2 * npair))
+    skey = (bgi * (nb + HOT_BLOCKS * HOT_BLOCKS) + sel)[single]
+    n_keys = int(torch.unique(torch.cat([pkey, skey])).numel())
+    return n_entries, n_slots, n_keys
 
 
 def algorithmic_work(w, idx):
@@ -256,19 +289,24 @@ def algorithmic_work(w, idx):
         # once.  Per window chunk of a row the window kernel reads the G query
         # rows and writes G partial rows; it reads the window's K, V once.
         # The merge reads all slot partials and writes O and lse per row.
-        ne, nblk = block_major_counts(idx, w)
+        # (method flops count the keys the row attends, 4 G B d per used
+        # entry; the design's bytes follow its slots: one per entry, or per
+        # pair of hot entries with 64-key blocks, each a 128-key tile)
+        ne, nsl, nkeys = block_major_counts(idx, w)
         items = w.batch * w.n_q * w.h_kv
         nwc = (w.window + 255) // 256
         nwin = items * nwc
         wkeys = float(np.minimum(w.window, pos + 1).sum()) * w.batch * w.h_kv
-        out["blocks_bytes"] = ne * G * (w.d * 2 * 2 + 8) + nblk * 2 * w.block * w.d * 2
+        tile_keys = 128 if w.block == 64 else w.block
+        out["blocks_bytes"] = nsl * G * (w.d * 2 * 2 + 8) + nkeys * 2 * tile_keys * w.d * 2
         out["blocks_flops"] = 4.0 * ne * G * w.block * w.d
         out["window_bytes"] = nwin * G * (w.d * 2 * 2 + 8) + w.batch * w.n * w.h_kv * 2 * w.d * 2
         out["window_flops"] = 4.0 * wkeys * G * w.d
-        out["merge_bytes"] = items * (G * w.d * 2 + G * 4 + w.topk * 4) + (ne + nwin) * G * (w.d * 2 + 8)
-        out["plan_bytes"] = items * w.topk * 4 * 2 + ne * 4 + items * 4
+        out["merge_bytes"] = items * (G * w.d * 2 + G * 4 + w.topk * 4) + (nsl + nwin) * G * (w.d * 2 + 8)
+        out["plan_bytes"] = items * w.topk * 4 * (3 if w.block == 64 else 2) + nsl * 4 + items * 4
         out["n_entries"] = ne
-        out["n_blocks"] = nblk
+        out["n_slots"] = nsl
+        out["n_blocks"] = nkeys
     return out
 
 
@@ -498,16 +536,22 @@ def kernel_report(w, res, peaks, traffic):
             rep["attn_gather"]["kernel"] = "attn_f32_kernel"
     else:
         hbm_entry("attn_plan", wk["plan_bytes"])
-        hbm_entry("attn_blocks", wk["blocks_bytes"], {"n_entries": wk["n_entries"], "n_blocks": wk["n_blocks"]})
-        b_tf = wk["blocks_flops"] / (ms["attn_blocks"] * 1e-3) / 1e12
-        rep["attn_blocks"]["tensor"] = {"achieved": b_tf, "unit": "TFLOP/s", "frac": b_tf / tc, "peak": tc,
-                                        "algorithmic_flops": wk["blocks_flops"]}
-        if b_tf / tc > rep["attn_blocks"]["frac"]:
-            rep["attn_blocks"].update(bound="tensor", achieved=b_tf, unit="TFLOP/s", frac=b_tf / tc, peak=tc)
-        hbm_entry("attn_window", wk["window_bytes"])
-        w_tf = wk["window_flops"] / (ms["attn_window"] * 1e-3) / 1e12
-        rep["attn_window"]["tensor"] = {"achieved": w_tf, "unit": "TFLOP/s", "frac": w_tf / tc, "peak": tc,
-                                        "algorithmic_flops": wk["window_flops"]}
+        # The block and window tiles are rated on the method's work: the
+        # attention's flops (QK^T and PV, 4 G B d per selected slot; 4 G d
+        # per window key), against the tensor-core peak.  Their HBM figure
+        # counts the block-major design's own traffic (query rows re-read
+        # per slot, partial outputs written for the merge), so it is kept
+        # beside the headline as `design_traffic`, not as the bound.
+        for name, fl_key in (("attn_blocks", "blocks_flops"), ("attn_window", "window_flops")):
+            hbm_entry(name, wk[name.replace("attn_", "") + "_bytes"])
+            e = rep[name]
+            design = {"achieved": e["achieved"], "unit": "GB/s", "frac": e["frac"], "peak": hbm,
+                      "algorithmic_bytes": e["algorithmic_bytes"], "traffic": e["traffic"]}
+            t_f = wk[fl_key] / (ms[name] * 1e-3) / 1e12
+            e.update(bound="tensor", achieved=t_f, unit="TFLOP/s", frac=t_f / tc, peak=tc,
+                     algorithmic_flops=wk[fl_key], design_traffic=design)
+            del e["algorithmic_bytes"]
+        rep["attn_blocks"].update(n_entries=wk["n_entries"], n_slots=wk["n_slots"], n_tile_keys=wk["n_blocks"])
         hbm_entry("attn_merge", wk["merge_bytes"])
     # the pages' attention figure: algorithmic gathered K+V (+ q, o) bytes over
     # the whole attention time, whichever way it is evaluated
@@ -516,6 +560,30 @@ def kernel_report(w, res, peaks, traffic):
                                           "unit": "GB/s", "algorithmic_bytes": wk["attn_bytes"],
                                           "mean_keys_per_row": wk["mean_keys"]}
     return rep
+
+
+def layer_report(w, wk, ms_step, peaks):
+    """The whole layer against both roofs: the method's flops (routing scores
+    and exact attention over the attended keys) per step over the step time,
+    against the sustained tensor-core peak; and its compulsory HBM bytes (Q,
+    K, V read once, O and lse written once, the routing table and block_idx
+    each written and read once) over the step time, against the copy
+    bandwidth."""
+    es = 4 if w.dtype == "f32" else 2
+    nb = w.n // w.block
+    flops = wk["route_flops"] + wk["attn_flops"]
+    io = (w.batch * w.n_q * w.h_q * w.d * es * 2 + w.batch * w.n * w.h_kv * w.d * es * 2
+          + w.batch * w.n_q * w.h_q * 4)
+    table = w.batch * w.h_kv * nb * w.subblocks * 2 * w.d * (2 if w.dtype == "bf16" else 4)
+    idx = w.batch * w.n_q * w.h_kv * w.topk * 4
+    nbytes = io + 2 * table + 2 * idx
+    t = ms_step * 1e-3
+    tf = flops / t / 1e12
+    gbs = nbytes / t / 1e9
+    return {"ms": ms_step, "method_flops": flops, "achieved_tflops": tf,
+            "frac_tensor": tf / peaks["bf16_tflops_sustained"], "tensor_peak": peaks["bf16_tflops_sustained"],
+            "compulsory_bytes": nbytes, "achieved_gbs": gbs, "frac_hbm": gbs / peaks["hbm_gbs"],
+            "hbm_peak": peaks["hbm_gbs"], "mean_keys_per_row": wk["mean_keys"]}
 
 
 def dominant(rep, exclude=()):
@@ -642,6 +710,9 @@ def main():
             "frac_nominal": dk["achieved"] / NOMINAL[dk["unit"]] if dk["bound"] in ("hbm", "tensor") else None,
             "algorithmic_per_launch": dk.get("algorithmic_flops") if dk["bound"] in ("tensor", "alu")
             else dk["algorithmic_bytes"]}
+    if "design_traffic" in dk:
+        roof["design_traffic"] = dk["design_traffic"]
+    roof["layer"] = layer_report(w, res["work"], res["ms_step"], peaks)
     secondary = None
     if not a.no_secondary and w.name == PRIMARY and a.n is None:
         torch.cuda.empty_cache()

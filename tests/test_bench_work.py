@@ -32,25 +32,63 @@ def test_attended_keys_is_the_key_set_size():
             assert got[0, i, g] == len(O.key_set(p.q_offset + i, idx[0, i, g], p)), (i, g)
 
 
+def _direct_slots(arr, w, p):
+    """The slot rule written out row by row: used entries; with 64-key blocks
+    the hot blocks of each kv-head (count >= the smallest T >= 2 that leaves
+    at most 128 of them) are paired two at a time in block order."""
+    from collections import Counter
+    used_rows = {}
+    cnt = Counter()
+    for i in range(w.n_q):
+        nvis = O.visible_blocks(p.q_offset + i, p)
+        for g in range(w.h_kv):
+            last, used = -1, []
+            for v in arr[0, i, g]:
+                if 0 <= v < nvis and v > last:
+                    used.append(int(v))
+                if 0 <= v < nvis:
+                    last = max(last, int(v))
+            used_rows[(i, g)] = used
+            cnt.update((g, c) for c in used)
+    n_e = sum(len(u) for u in used_rows.values())
+    if w.block != 64:
+        return n_e, n_e, len(cnt)
+    hot = {}
+    for g in range(w.h_kv):
+        counts = [cnt[(g, c)] for c in range(w.n // w.block)]
+        T = 2
+        while sum(x >= T for x in counts) > 128:
+            T += 1
+        hot[g] = [c for c, x in enumerate(counts) if x >= T]
+    n_s, keys = 0, set()
+    for (i, g), used in used_rows.items():
+        hs = [c for c in used if c in hot[g]]
+        npair = len(hs) // 2
+        pairs = [(hs[2 * m], hs[2 * m + 1]) for m in range(npair)]
+        paired = set(hs[:2 * npair])
+        singles = [c for c in used if c not in paired]
+        n_s += npair + len(singles)
+        keys.update((g, "p", a, b) for a, b in pairs)
+        keys.update((g, "s", c) for c in singles)
+    return n_e, n_s, len(keys)
+
+
 def test_block_major_counts_by_direct_count():
     w, p, idx = _case()
     bad = idx.copy()
-    bad[0, 100, 0, 3] = bad[0, 100, 0, 2]       # a repeat and an out-of-range entry are not used
-    bad[0, 200, 1, 5] = p.nb + 3
+    rng = np.random.default_rng(5)
+    bad[rng.random(bad.shape) < 0.05] = 10 ** 6
+    bad[rng.random(bad.shape) < 0.05] = 0
     for arr in (idx, bad):
-        n_e, n_b = bench.block_major_counts(torch.from_numpy(arr), w)
-        used, blocks = 0, set()
-        for i in range(w.n_q):
-            nvis = O.visible_blocks(p.q_offset + i, p)
-            for g in range(w.h_kv):
-                last = -1
-                for v in arr[0, i, g]:
-                    if 0 <= v < nvis and v > last:
-                        used += 1
-                        blocks.add((g, int(v)))
-                    if 0 <= v < nvis:
-                        last = max(last, int(v))
-        assert (n_e, n_b) == (used, len(blocks))
+        got = bench.block_major_counts(torch.from_numpy(arr), w)
+        assert got == _direct_slots(arr, w, p)
+        assert got[1] < got[0]          # some entries pair up
+    # 128-key blocks: one slot per used entry
+    w2 = w.scaled(block=128)
+    p2 = O.Problem(**problem_dict(w2))
+    arr2 = np.where(idx >= 0, idx // 2, idx)
+    got2 = bench.block_major_counts(torch.from_numpy(arr2), w2)
+    assert got2 == _direct_slots(arr2, w2, p2) and got2[0] == got2[1]
 
 
 def test_kernel_report_fractions_and_dominant_stage():
@@ -70,6 +108,38 @@ def test_kernel_report_fractions_and_dominant_stage():
     r = rep["route"]
     assert r["bound"] == "tensor" and abs(r["achieved"] - work["route_flops"] / 2e-3 / 1e12) < 1e-9 * r["achieved"]
     assert abs(r["frac"] - r["achieved"] / 1400.0) < 1e-12
+    # the tiles are rated on the method's flops; the design's bytes ride along
+    for name, key in (("attn_blocks", "blocks_flops"), ("attn_window", "window_flops")):
+        e = rep[name]
+        assert e["bound"] == "tensor" and e["algorithmic_flops"] == work[key]
+        assert abs(e["achieved"] - work[key] / (ms[name] * 1e-3) / 1e12) < 1e-9 * e["achieved"]
+        assert abs(e["frac"] - e["achieved"] / 1400.0) < 1e-12
+        dt = e["design_traffic"]
+        assert abs(dt["achieved"] - dt["algorithmic_bytes"] / (ms[name] * 1e-3) / 1e9) < 1e-6 * dt["achieved"]
+    # per selected slot the block tiles do 4 G B d flops (S = Q K^T, O = P V)
+    G = w.h_q // w.h_kv
+    assert work["blocks_flops"] == 4.0 * work["n_entries"] * G * w.block * w.d
     name, d = bench.dominant(rep)
     assert name == "attn_blocks" and d["ms"] == 4.0
     assert bench.dominant(rep, exclude=("attn_blocks",))[0] == "route"
+
+
+def test_layer_report_against_both_roofs():
+    """The layer line: method flops (route scores + attention over the
+    attended keys) and compulsory bytes over the step time, recomputed here
+    from the definitions."""
+    w, p, idx = _case()
+    work = bench.algorithmic_work(w, torch.from_numpy(idx))
+    peaks = {"hbm_gbs": 6000.0, "bf16_tflops": 1600.0, "bf16_tflops_sustained": 1400.0}
+    lay = bench.layer_report(w, work, 2.0, peaks)
+    S = bench.attended_keys(torch.from_numpy(idx), w).sum().item()
+    G = w.h_q // w.h_kv
+    nvis = sum(min(w.n // w.block, (i + 1) // w.block) for i in range(w.n_q))
+    flops = 4.0 * S * G * w.d + 2.0 * 2 * w.d * nvis * w.h_kv
+    assert abs(lay["method_flops"] - flops) < 1e-9 * flops
+    assert abs(lay["frac_tensor"] - flops / 2e-3 / 1e12 / 1400.0) < 1e-12
+    nb = w.n // w.block
+    nbytes = (2 * w.n_q * w.h_q * w.d * 2 + 2 * w.n * w.h_kv * w.d * 2 + w.n_q * w.h_q * 4
+              + 2 * w.h_kv * nb * 2 * w.d * 2 + 2 * w.n_q * w.h_kv * w.topk * 4)
+    assert lay["compulsory_bytes"] == nbytes
+    assert abs(lay["frac_hbm"] - nbytes / 2e-3 / 1e9 / 6000.0) < 1e-12
