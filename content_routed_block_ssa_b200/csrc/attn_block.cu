@@ -40,10 +40,21 @@ namespace {
 
 constexpr int kPlanThreads = 512;
 
+// Hot number of this lane's entry (-1 when unused or not hot).
+__device__ __forceinline__ int lane_hot_id(const BlockPlan& pl, const SlotSet& s, int bg) {
+  const int lane = threadIdx.x & 31;
+  return ((s.mask >> lane) & 1) ? __ldg(pl.hot_id + static_cast<int64_t>(bg) * pl.nb + s.v) : -1;
+}
+
+// keyed = false: counts per key block (the first pass in pair mode, the only
+// one otherwise) and each row's uncovered window blocks; chist columns are
+// blocks.  keyed = true (pair mode): counts per tile key; columns are keys.
+template <bool KEYED>
 __global__ void __launch_bounds__(kPlanThreads) inv_hist_kernel(const BlockPlan pl, const int32_t* __restrict__ idx) {
   extern __shared__ int32_t hist[];
+  const int ncol = KEYED ? pl.nkey : pl.nb;
   const int k = blockIdx.x, bg = blockIdx.y;
-  for (int c = threadIdx.x; c < pl.nb; c += blockDim.x) hist[c] = 0;
+  for (int c = threadIdx.x; c < ncol; c += blockDim.x) hist[c] = 0;
   __syncthreads();
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
   const int b = bg / pl.h_kv, g = bg % pl.h_kv;
@@ -51,51 +62,129 @@ __global__ void __launch_bounds__(kPlanThreads) inv_hist_kernel(const BlockPlan 
   for (int i = k * kPlanRows + warp; i < r1; i += nw) {
     const int v = lane < pl.topk ? __ldg(idx + ((static_cast<int64_t>(b) * pl.n_q + i) * pl.h_kv + g) * pl.topk + lane) : -1;
     const SlotSet s = row_slots(v, pl.topk, pl.q_offset + i, pl.nb, pl.block, pl.window);
-    if ((s.mask >> lane) & 1) atomicAdd(&hist[s.v], 1);
-    if (lane == 0) pl.win[static_cast<int64_t>(bg) * pl.n_q + i] = s.win;
+    if (KEYED) {
+      const PairSlot ps = pair_slots(s, lane_hot_id(pl, s, bg), pl.nb);
+      if (ps.emit) atomicAdd(&hist[ps.key], 1);
+    } else {
+      if ((s.mask >> lane) & 1) atomicAdd(&hist[s.v], 1);
+      if (lane == 0) pl.win[static_cast<int64_t>(bg) * pl.n_q + i] = s.win;
+    }
   }
   __syncthreads();
-  int32_t* out = pl.chist + (static_cast<int64_t>(bg) * pl.nchunk + k) * pl.nb;
-  for (int c = threadIdx.x; c < pl.nb; c += blockDim.x) out[c] = hist[c];
+  int32_t* out = pl.chist + (static_cast<int64_t>(bg) * pl.nchunk + k) * ncol;
+  for (int c = threadIdx.x; c < ncol; c += blockDim.x) out[c] = hist[c];
 }
 
-// Thread per (batch, kv-head, block): exclusive scan of the chunk counts in
-// place, and the block's total.
+// One CTA per (batch, kv-head), pair mode: each block's selections summed
+// over the chunks of the first pass; the hot set is the largest set
+// {c : count_c >= T} (T >= 2) of at most kHotBlocks blocks, numbered in
+// block order.
+__global__ void __launch_bounds__(1024) inv_hot_kernel(const BlockPlan pl) {
+  extern __shared__ int32_t tot[];   // [nb]
+  __shared__ int32_t red[32];
+  __shared__ int32_t s_lo, s_hi;
+  const int bg = blockIdx.x;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int32_t* ch = pl.chist + static_cast<int64_t>(bg) * pl.nchunk * pl.nb;
+  for (int c = threadIdx.x; c < pl.nb; c += blockDim.x) {
+    int v = 0;
+    for (int k = 0; k < pl.nchunk; ++k) v += ch[static_cast<int64_t>(k) * pl.nb + c];
+    tot[c] = v;
+  }
+  // block-wide count of blocks with tot >= T
+  auto count_ge = [&](int T) {
+    int n = 0;
+    for (int c = threadIdx.x; c < pl.nb; c += blockDim.x) n += tot[c] >= T ? 1 : 0;
+#pragma unroll
+    for (int o = 16; o; o >>= 1) n += __shfl_xor_sync(0xFFFFFFFFu, n, o);
+    __syncthreads();   // red is free (also orders the tot writes before the first reads)
+    if (lane == 0) red[warp] = n;
+    __syncthreads();
+    int t = 0;
+    for (int w = 0; w < 32; ++w) t += red[w];
+    return t;
+  };
+  // smallest T in [2, n_q + 1] with count_ge(T) <= kHotBlocks (count_ge(n_q + 1) = 0)
+  if (threadIdx.x == 0) { s_lo = 2; s_hi = pl.n_q + 1; }
+  __syncthreads();
+  while (true) {
+    const int lo = s_lo, hi = s_hi;   // uniform
+    if (lo >= hi) break;
+    const int mid = lo + ((hi - lo) >> 1);
+    const int n = count_ge(mid);
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      if (n <= kHotBlocks) s_hi = mid; else s_lo = mid + 1;
+    }
+    __syncthreads();
+  }
+  const int T = s_lo;
+  // hot numbers in block order: a block-wide exclusive scan of the flags
+  const int per = (pl.nb + 1023) / 1024;
+  const int c0 = threadIdx.x * per;
+  int mine = 0;
+  for (int c = c0; c < min(c0 + per, pl.nb); ++c) mine += tot[c] >= T ? 1 : 0;
+  int inc = mine;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xFFFFFFFFu, inc, o);
+    if (lane >= o) inc += y;
+  }
+  __syncthreads();
+  if (lane == 31) red[warp] = inc;
+  __syncthreads();
+  int base = inc - mine;
+  for (int w = 0; w < warp; ++w) base += red[w];
+  int32_t* hid = pl.hot_id + static_cast<int64_t>(bg) * pl.nb;
+  int32_t* hb = pl.hot_blk + static_cast<int64_t>(bg) * kHotBlocks;
+  for (int c = c0; c < min(c0 + per, pl.nb); ++c) {
+    if (tot[c] >= T) {
+      hid[c] = base;
+      hb[base] = c;
+      ++base;
+    } else {
+      hid[c] = -1;
+    }
+  }
+}
+
+// Thread per (batch, kv-head, key): exclusive scan of the chunk counts in
+// place, and the key's total.
 __global__ void __launch_bounds__(256) inv_colscan_kernel(const BlockPlan pl) {
   const int64_t x = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
-  if (x >= static_cast<int64_t>(pl.bgs) * pl.nb) return;
-  const int bg = static_cast<int>(x / pl.nb), c = static_cast<int>(x % pl.nb);
-  int32_t* col = pl.chist + static_cast<int64_t>(bg) * pl.nchunk * pl.nb + c;
+  if (x >= static_cast<int64_t>(pl.bgs) * pl.nkey) return;
+  const int bg = static_cast<int>(x / pl.nkey), c = static_cast<int>(x % pl.nkey);
+  int32_t* col = pl.chist + static_cast<int64_t>(bg) * pl.nchunk * pl.nkey + c;
   int run = 0;
   int k = 0;
   for (; k + 8 <= pl.nchunk; k += 8) {   // eight loads in flight per thread
     int v[8];
 #pragma unroll
-    for (int u = 0; u < 8; ++u) v[u] = col[static_cast<int64_t>(k + u) * pl.nb];
+    for (int u = 0; u < 8; ++u) v[u] = col[static_cast<int64_t>(k + u) * pl.nkey];
 #pragma unroll
     for (int u = 0; u < 8; ++u) {
-      col[static_cast<int64_t>(k + u) * pl.nb] = run;
+      col[static_cast<int64_t>(k + u) * pl.nkey] = run;
       run += v[u];
     }
   }
   for (; k < pl.nchunk; ++k) {
-    const int v = col[static_cast<int64_t>(k) * pl.nb];
-    col[static_cast<int64_t>(k) * pl.nb] = run;
+    const int v = col[static_cast<int64_t>(k) * pl.nkey];
+    col[static_cast<int64_t>(k) * pl.nkey] = run;
     run += v;
   }
   pl.count[x] = run;
 }
 
-// One CTA per (batch, kv-head): exclusive scans of the per-block entry and
+// One CTA per (batch, kv-head): exclusive scans of the per-key entry and
 // tile counts.
 __global__ void __launch_bounds__(1024) inv_scan_kernel(const BlockPlan pl) {
   __shared__ int32_t wsum_e[32], wsum_t[32];
   const int bg = blockIdx.x;
-  const int32_t* cnt = pl.count + static_cast<int64_t>(bg) * pl.nb;
-  const int per = (pl.nb + 1023) / 1024;
+  const int32_t* cnt = pl.count + static_cast<int64_t>(bg) * pl.nkey;
+  const int per = (pl.nkey + 1023) / 1024;
   const int c0 = threadIdx.x * per;
   int se = 0, st = 0;
-  for (int c = c0; c < min(c0 + per, pl.nb); ++c) {
+  for (int c = c0; c < min(c0 + per, pl.nkey); ++c) {
     se += cnt[c];
     st += (cnt[c] + pl.qpt - 1) / pl.qpt;
   }
@@ -122,9 +211,9 @@ __global__ void __launch_bounds__(1024) inv_scan_kernel(const BlockPlan pl) {
   __syncthreads();
   int base_e = (warp ? wsum_e[warp - 1] : 0) + ie - se;
   int base_t = (warp ? wsum_t[warp - 1] : 0) + it - st;
-  for (int c = c0; c < min(c0 + per, pl.nb); ++c) {
-    pl.blk_off[static_cast<int64_t>(bg) * pl.nb + c] = base_e;
-    pl.tile_off[static_cast<int64_t>(bg) * pl.nb + c] = base_t;
+  for (int c = c0; c < min(c0 + per, pl.nkey); ++c) {
+    pl.blk_off[static_cast<int64_t>(bg) * pl.nkey + c] = base_e;
+    pl.tile_off[static_cast<int64_t>(bg) * pl.nkey + c] = base_t;
     base_e += cnt[c];
     base_t += (cnt[c] + pl.qpt - 1) / pl.qpt;
   }
@@ -148,15 +237,15 @@ __global__ void __launch_bounds__(32) inv_scan_bg_kernel(const BlockPlan pl) {
   pl.tile_base[pl.bgs] = t;
 }
 
-// Same rows as inv_hist_kernel: every used selected slot becomes the entry
-// make_entry(query row, slot) in its block's list.
+// Same rows as inv_hist_kernel: every selected slot becomes the entry
+// make_entry(query row, slot) in its key's list.
 __global__ void __launch_bounds__(kPlanThreads) inv_scatter_kernel(const BlockPlan pl, const int32_t* __restrict__ idx) {
   extern __shared__ int32_t cur[];
   const int k = blockIdx.x, bg = blockIdx.y;
-  const int32_t* col = pl.chist + (static_cast<int64_t>(bg) * pl.nchunk + k) * pl.nb;
-  const int32_t* boff = pl.blk_off + static_cast<int64_t>(bg) * pl.nb;
+  const int32_t* col = pl.chist + (static_cast<int64_t>(bg) * pl.nchunk + k) * pl.nkey;
+  const int32_t* boff = pl.blk_off + static_cast<int64_t>(bg) * pl.nkey;
   const int ebase = pl.ent_base[bg];
-  for (int c = threadIdx.x; c < pl.nb; c += blockDim.x) cur[c] = ebase + boff[c] + col[c];
+  for (int c = threadIdx.x; c < pl.nkey; c += blockDim.x) cur[c] = ebase + boff[c] + col[c];
   __syncthreads();
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
   const int b = bg / pl.h_kv, g = bg % pl.h_kv;
@@ -164,23 +253,40 @@ __global__ void __launch_bounds__(kPlanThreads) inv_scatter_kernel(const BlockPl
   for (int i = k * kPlanRows + warp; i < r1; i += nw) {
     const int v = lane < pl.topk ? __ldg(idx + ((static_cast<int64_t>(b) * pl.n_q + i) * pl.h_kv + g) * pl.topk + lane) : -1;
     const SlotSet s = row_slots(v, pl.topk, pl.q_offset + i, pl.nb, pl.block, pl.window);
-    if ((s.mask >> lane) & 1) pl.entries[atomicAdd(&cur[s.v], 1)] = make_entry(i, lane);
+    if (pl.pair) {
+      const PairSlot ps = pair_slots(s, lane_hot_id(pl, s, bg), pl.nb);
+      if (ps.emit) pl.entries[atomicAdd(&cur[ps.key], 1)] = make_entry(i, ps.slot);
+    } else {
+      if ((s.mask >> lane) & 1) pl.entries[atomicAdd(&cur[s.v], 1)] = make_entry(i, lane);
+    }
   }
 }
 
-// A warp per (batch, kv-head, block): its tiles written lane-strided (a
-// block chosen by nearly every query has tens of thousands of tiles).
+// A warp per (batch, kv-head, key): its tiles written lane-strided (a
+// block chosen by nearly every query has tens of thousands of tiles).  The
+// tile's block field is the block, or in pair mode pair_tile_y(c1, c2).
 __global__ void __launch_bounds__(256) inv_tiles_kernel(const BlockPlan pl) {
   const int64_t x = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
-  if (x >= static_cast<int64_t>(pl.bgs) * pl.nb) return;   // warp-uniform
+  if (x >= static_cast<int64_t>(pl.bgs) * pl.nkey) return;   // warp-uniform
   const int lane = threadIdx.x & 31;
-  const int bg = static_cast<int>(x / pl.nb), c = static_cast<int>(x % pl.nb);
+  const int bg = static_cast<int>(x / pl.nkey), c = static_cast<int>(x % pl.nkey);
   const int n = pl.count[x];
+  if (n == 0) return;
+  int y = c;
+  if (pl.pair) {
+    if (c < pl.nb) {
+      y = pair_tile_y(c, -1);
+    } else {
+      const int hh = c - pl.nb;
+      const int32_t* hb = pl.hot_blk + static_cast<int64_t>(bg) * kHotBlocks;
+      y = pair_tile_y(hb[hh / kHotBlocks], hb[hh % kHotBlocks]);
+    }
+  }
   const int e0 = pl.ent_base[bg] + pl.blk_off[x];
   const int t0 = pl.tile_base[bg] + pl.tile_off[x];
   const int nt = (n + pl.qpt - 1) / pl.qpt;
   for (int t = lane; t < nt; t += 32)
-    pl.tiles[t0 + t] = make_int4(bg, c, e0 + t * pl.qpt, min(pl.qpt, n - t * pl.qpt));
+    pl.tiles[t0 + t] = make_int4(bg, y, e0 + t * pl.qpt, min(pl.qpt, n - t * pl.qpt));
 }
 
 // Work estimate of each tile for the split over CTAs (units of a quarter of
@@ -372,10 +478,16 @@ __device__ __forceinline__ void tmem_ld64(uint32_t taddr, uint32_t (&r)[64]) {
 //   SW0 .. softmax and epilogue in two groups of four warps that take
 //          alternate tiles (S, P and O are double-buffered by tile parity),
 //          one tensor-core row = one (query, head) pair per thread.
-template <int G, int BLK>
+//
+// PAIR (64-key blocks, BLK = 128): a tile's 128 keys are the two blocks of
+// a pair, pair_tile_c1/c2 of its block field, loaded into the two 64-key
+// halves; a single-block tile loads its block into both halves and its
+// softmax leaves the second half out (P = 0 there).
+template <int G, int BLK, bool PAIR>
 __global__ void __maxnreg__((BlkCfg<G, BLK>::MAXREG))
     attn_block_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                       const __grid_constant__ CUtensorMap tmQ, const BlkArgs a) {
+  static_assert(!PAIR || BLK == 128, "pairs fill 128-key tiles");
   using C = BlkCfg<G, BLK>;
   constexpr int D = C::D;
   constexpr int QPT = 128 / G;
@@ -449,13 +561,23 @@ __global__ void __maxnreg__((BlkCfg<G, BLK>::MAXREG))
         const int b = td.x / a.h_kv, g = td.x % a.h_kv;
         uint8_t* kv = sKV + kb * C::KV_BYTES;
         mbar_arrive_expect_tx(&kv_full[kb], C::KV_BYTES);
-        const int z = static_cast<int>(static_cast<int64_t>(b) * a.n_kv + static_cast<int64_t>(td.y) * BLK);
+        // first key of each 64-key half of the tile
+        int zs[BLK / 64];
+        if (PAIR) {
+          const int c1 = pair_tile_c1(td.y), c2 = pair_tile_c2(td.y);
+          zs[0] = static_cast<int>(static_cast<int64_t>(b) * a.n_kv + static_cast<int64_t>(c1) * 64);
+          zs[BLK / 64 - 1] = static_cast<int>(static_cast<int64_t>(b) * a.n_kv + static_cast<int64_t>(c2 >= 0 ? c2 : c1) * 64);
+        } else {
+#pragma unroll
+          for (int sub = 0; sub < BLK / 64; ++sub)
+            zs[sub] = static_cast<int>(static_cast<int64_t>(b) * a.n_kv + static_cast<int64_t>(td.y) * BLK + sub * 64);
+        }
 #pragma unroll
         for (int sub = 0; sub < BLK / 64; ++sub) {
 #pragma unroll
           for (int hf = 0; hf < 2; ++hf) {
-            tma_load_3d(kv + hf * C::KV_HALF + sub * 64 * C::ROW, &tmK, &kv_full[kb], hf * 64, g, z + sub * 64);
-            tma_load_3d(kv + (2 + hf) * C::KV_HALF + sub * 64 * C::ROW, &tmV, &kv_full[kb], hf * 64, g, z + sub * 64);
+            tma_load_3d(kv + hf * C::KV_HALF + sub * 64 * C::ROW, &tmK, &kv_full[kb], hf * 64, g, zs[sub]);
+            tma_load_3d(kv + (2 + hf) * C::KV_HALF + sub * 64 * C::ROW, &tmV, &kv_full[kb], hf * 64, g, zs[sub]);
           }
         }
         ++kv_loads;
@@ -592,6 +714,9 @@ __global__ void __maxnreg__((BlkCfg<G, BLK>::MAXREG))
         tc_fence_after();
         const uint32_t scol = tmem_base + lane_base + C::S_COL + sb * BLK;
         auto load_half = [&](int hf, uint32_t (&r)[64]) { tmem_ld64(scol + hf * 64, r); };
+        // pair mode: a single-block tile holds keys in its first half only
+        // (tile-uniform)
+        const int nhalf = (PAIR && pair_tile_c2(tile_at(ts).y) < 0) ? 1 : BLK / 64;
         // maxima and sums in eight independent chains
         float mx[8] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY, -INFINITY, -INFINITY, -INFINITY, -INFINITY};
         float ls[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
@@ -599,6 +724,7 @@ __global__ void __maxnreg__((BlkCfg<G, BLK>::MAXREG))
         if (BLK > 64) {   // first pass: the maximum over both halves
 #pragma unroll
           for (int hf = 0; hf < BLK / 64; ++hf) {
+            if (hf >= nhalf) break;
             uint32_t r[64];
             load_half(hf, r);
 #pragma unroll
@@ -610,6 +736,14 @@ __global__ void __maxnreg__((BlkCfg<G, BLK>::MAXREG))
         // covers are already in registers (half 0) or consumed (half 1)
 #pragma unroll
         for (int hf = 0; hf < BLK / 64; ++hf) {
+          if (hf >= nhalf) {   // no keys: P = 0 over this half's 32 columns
+            uint32_t pw[16];
+#pragma unroll
+            for (int u = 0; u < 16; ++u) pw[u] = 0u;
+            tmem_st16(scol + hf * 32, pw);
+            tmem_st16(scol + hf * 32 + 16, pw);
+            continue;
+          }
           uint32_t r[64];
           load_half(hf, r);
           if (BLK == 64) {
@@ -853,6 +987,7 @@ __global__ void __maxnreg__((BlkCfg<G, BLK>::MAXREG))
 
 struct MergeArgs {
   const int32_t* idx;
+  const int32_t* hot_id;     // pair mode: [bgs][nb] hot numbers (else NULL)
   const __half* partO;
   const float2* partL;
   __nv_bfloat16* O;
@@ -877,6 +1012,11 @@ __global__ void __launch_bounds__(256, (G == 8 ? 2 : (G == 4 ? 3 : 4))) attn_mer
   const int v = lane < a.topk ? __ldg(a.idx + ((static_cast<int64_t>(b) * a.n_q + i) * a.h_kv + g) * a.topk + lane) : -1;
   SlotSet s = row_slots(v, a.topk, a.q_offset + i, a.nb, a.block, a.window);
   if (lane == 0 && a.bad && s.n_bad) atomicAdd(a.bad, s.n_bad);
+  if (a.hot_id) {   // pair mode: the selected slots are 0 .. nsel - 1
+    const int hid = ((s.mask >> lane) & 1) ? __ldg(a.hot_id + static_cast<int64_t>(bg) * a.nb + s.v) : -1;
+    const PairSlot ps = pair_slots(s, hid, a.nb);
+    s.mask = (1ull << ps.nsel) - 1ull;
+  }
   // the window chunks (slots topk + c) that hold keys, one lane each
   const uint32_t wch = __ballot_sync(0xFFFFFFFFu, lane < a.nsl - a.topk &&
                                                       chunk_has_keys(s.win, a.q_offset + i, a.window, a.block, lane,
@@ -957,13 +1097,14 @@ __global__ void __launch_bounds__(256, (G == 8 ? 2 : (G == 4 ? 3 : 4))) attn_mer
   }
 }
 
-template <int G, int BLK>
+template <int G, int BLK, bool PAIR = false>
 cudaError_t run_block(const BlockPlan& pl, const CUtensorMap& tmK, const CUtensorMap& tmV, const CUtensorMap& tmQ,
                       const BlkArgs& a, const LaunchCtx& c) {
   using C = BlkCfg<G, BLK>;
-  cudaError_t e = cudaFuncSetAttribute(attn_block_kernel<G, BLK>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+  cudaError_t e = cudaFuncSetAttribute(attn_block_kernel<G, BLK, PAIR>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       C::SMEM);
   if (e != cudaSuccess) return e;
-  attn_block_kernel<G, BLK><<<c.sm_count, C::THREADS, C::SMEM, c.stream>>>(tmK, tmV, tmQ, a);
+  attn_block_kernel<G, BLK, PAIR><<<c.sm_count, C::THREADS, C::SMEM, c.stream>>>(tmK, tmV, tmQ, a);
   note_launch();
   (void)pl;
   return cudaGetLastError();
@@ -971,10 +1112,12 @@ cudaError_t run_block(const BlockPlan& pl, const CUtensorMap& tmK, const CUtenso
 
 }  // namespace
 
-cudaError_t launch_attn_merge(const ssa_params& p, const int32_t* block_idx, const void* partO, const void* partL,
-                              void* O, float* lse, int32_t* bad, const LaunchCtx& c) {
+cudaError_t launch_attn_merge(const ssa_params& p, const int32_t* block_idx, const int32_t* hot_id,
+                              const void* partO, const void* partL, void* O, float* lse, int32_t* bad,
+                              const LaunchCtx& c) {
   MergeArgs a;
   a.idx = block_idx;
+  a.hot_id = hot_id;
   a.partO = static_cast<const __half*>(partO);
   a.partL = static_cast<const float2*>(partL);
   a.O = static_cast<__nv_bfloat16*>(O);
@@ -1002,34 +1145,45 @@ int attn_block_smem_bytes(int block) { return block == 64 ? BlkCfg<4, 64>::SMEM 
 
 cudaError_t launch_block_plan(const ssa_params& p, const int32_t* block_idx, const BlockPlan& pl,
                               const LaunchCtx& c) {
-  const size_t hist_smem = static_cast<size_t>(pl.nb) * sizeof(int32_t);
-  cudaError_t e = cudaFuncSetAttribute(inv_hist_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       static_cast<int>(hist_smem));
+  const int blk_smem = pl.nb * static_cast<int>(sizeof(int32_t));
+  const int key_smem = pl.nkey * static_cast<int>(sizeof(int32_t));
+  cudaError_t e = cudaFuncSetAttribute(inv_hist_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, blk_smem);
   if (e == cudaSuccess)
-    e = cudaFuncSetAttribute(inv_scatter_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(hist_smem));
+    e = cudaFuncSetAttribute(inv_hist_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, key_smem);
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(inv_hot_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, blk_smem);
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(inv_scatter_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, key_smem);
   if (e != cudaSuccess) return e;
   const dim3 rows(static_cast<unsigned>(pl.nchunk), static_cast<unsigned>(pl.bgs));
-  const unsigned cols = static_cast<unsigned>((static_cast<int64_t>(pl.bgs) * pl.nb + 255) / 256);
-  inv_hist_kernel<<<rows, kPlanThreads, hist_smem, c.stream>>>(pl, block_idx);
+  const unsigned cols = static_cast<unsigned>((static_cast<int64_t>(pl.bgs) * pl.nkey + 255) / 256);
+  // per-block counts and window blocks; in pair mode then the hot sets and
+  // the counts per tile key
+  inv_hist_kernel<false><<<rows, kPlanThreads, blk_smem, c.stream>>>(pl, block_idx);
   note_launch();
+  if (pl.pair) {
+    inv_hot_kernel<<<pl.bgs, 1024, blk_smem, c.stream>>>(pl);
+    note_launch();
+    inv_hist_kernel<true><<<rows, kPlanThreads, key_smem, c.stream>>>(pl, block_idx);
+    note_launch();
+  }
   inv_colscan_kernel<<<cols, 256, 0, c.stream>>>(pl);
   note_launch();
   inv_scan_kernel<<<pl.bgs, 1024, 0, c.stream>>>(pl);
   note_launch();
   inv_scan_bg_kernel<<<1, 32, 0, c.stream>>>(pl);
   note_launch();
-  inv_scatter_kernel<<<rows, kPlanThreads, hist_smem, c.stream>>>(pl, block_idx);
+  inv_scatter_kernel<<<rows, kPlanThreads, key_smem, c.stream>>>(pl, block_idx);
   note_launch();
-  inv_tiles_kernel<<<static_cast<unsigned>((static_cast<int64_t>(pl.bgs) * pl.nb * 32 + 255) / 256), 256, 0,
+  inv_tiles_kernel<<<static_cast<unsigned>((static_cast<int64_t>(pl.bgs) * pl.nkey * 32 + 255) / 256), 256, 0,
                      c.stream>>>(pl);
   note_launch();
   if (pl.grid < 1 || pl.grid > kMaxBlockGrid) return cudaErrorInvalidValue;
   const int n_chunks = (pl.max_tiles + 255) / 256;
-  // 64-key blocks (two K/V buffers): every tile alike — equal counts were
-  // measured as fast as any weighting; 128-key blocks (one K/V buffer): a
-  // new block costs two tiles
-  inv_cost_kernel<<<n_chunks, 256, 0, c.stream>>>(pl, p.block == 64 ? 0 : 8);
+  // 64-key tiles (two K/V buffers): every tile alike — equal counts were
+  // measured as fast as any weighting; 128-key tiles (128-key blocks or
+  // pairs; one K/V buffer): a new block costs two tiles
+  inv_cost_kernel<<<n_chunks, 256, 0, c.stream>>>(pl, (p.block == 64 && !pl.pair) ? 0 : 8);
   note_launch();
   inv_split_kernel<<<1, 1024, 0, c.stream>>>(pl, n_chunks);
   note_launch();
@@ -1053,7 +1207,12 @@ cudaError_t launch_attn_block(const ssa_params& p, const BlockPlan& pl, const vo
   a.err = c.err;
   const int G = p.h_q / p.h_kv;
   if (p.d != 128) return cudaErrorInvalidValue;
-  if (p.block == 64) {
+  if (p.block == 64 && pl.pair) {
+    if (G == 1) return run_block<1, 128, true>(pl, tmK, tmV, tmQ, a, c);
+    if (G == 2) return run_block<2, 128, true>(pl, tmK, tmV, tmQ, a, c);
+    if (G == 4) return run_block<4, 128, true>(pl, tmK, tmV, tmQ, a, c);
+    if (G == 8) return run_block<8, 128, true>(pl, tmK, tmV, tmQ, a, c);
+  } else if (p.block == 64) {
     if (G == 1) return run_block<1, 64>(pl, tmK, tmV, tmQ, a, c);
     if (G == 2) return run_block<2, 64>(pl, tmK, tmV, tmQ, a, c);
     if (G == 4) return run_block<4, 64>(pl, tmK, tmV, tmQ, a, c);

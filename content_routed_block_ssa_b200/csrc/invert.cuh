@@ -84,6 +84,63 @@ __device__ __forceinline__ SlotSet row_slots(int v_in, int topk, int64_t pos, in
   return s;
 }
 
+// Paired slots (64-key blocks).  Each (batch, kv-head) has a hot set of at
+// most kHotBlocks blocks, its most selected ones, numbered in block order.
+// A row's used entries that select hot blocks are taken two at a time in
+// ascending block order: each pair is one selected slot of 128 keys (the
+// two blocks' keys), evaluated for all rows that chose the same two blocks
+// together.  Every other used entry (a block outside the hot set, or the
+// last hot one when their number is odd) is a single slot of its block's 64
+// keys.  Slots are numbered pairs first, then singles, both in block order.
+// Tiles are keyed per (batch, kv-head): single block c -> key c; pair of hot
+// numbers (h1, h2) -> key nb + h1 * kHotBlocks + h2.
+constexpr int kHotBlocks = 128;
+
+struct PairSlot {
+  bool emit;       // this lane's entry starts a slot
+  int key;         // its tile key
+  int slot;        // its slot number
+  int nsel;        // selected slots of the row
+};
+
+// Warp-collective.  s from row_slots; hid = hot number of this lane's entry
+// (-1 when it is not hot or not used).  Every lane gets nsel.
+__device__ __forceinline__ PairSlot pair_slots(const SlotSet& s, int hid, int nb) {
+  const int lane = threadIdx.x & 31;
+  const uint32_t lt = (1u << lane) - 1u;
+  const bool used = (s.mask >> lane) & 1;
+  const uint32_t used_m = static_cast<uint32_t>(s.mask);
+  const uint32_t hot_m = __ballot_sync(0xFFFFFFFFu, used && hid >= 0);
+  const int nhot = __popc(hot_m), npair = nhot >> 1;
+  const int r = __popc(hot_m & lt);                       // rank among hot entries
+  const bool hot = (hot_m >> lane) & 1;
+  const bool paired = hot && r < 2 * npair;
+  const uint32_t paired_m = __ballot_sync(0xFFFFFFFFu, paired);
+  const uint32_t single_m = used_m & ~paired_m;
+  // the next hot lane above this one (the partner of a pair's first entry)
+  const uint32_t above = hot_m & ~(lt | (1u << lane));
+  const int partner = above ? __ffs(static_cast<int>(above)) - 1 : lane;
+  const int hid2 = __shfl_sync(0xFFFFFFFFu, hid, partner);
+  PairSlot o;
+  o.nsel = __popc(used_m) - npair;
+  if (paired) {
+    o.emit = (r & 1) == 0;
+    o.key = nb + hid * kHotBlocks + hid2;
+    o.slot = r >> 1;
+  } else {
+    o.emit = used;
+    o.key = s.v;
+    o.slot = npair + __popc(single_m & lt);
+  }
+  return o;
+}
+
+// Tile block field for a pair mode tile: first block in bits 0..14, second
+// block + 1 above (0 for a single block).
+__host__ __device__ constexpr int pair_tile_y(int c1, int c2) { return c1 | ((c2 + 1) << 15); }
+__host__ __device__ constexpr int pair_tile_c1(int y) { return y & 0x7FFF; }
+__host__ __device__ constexpr int pair_tile_c2(int y) { return (y >> 15) - 1; }
+
 // Whether window chunk s (of `chunk` keys) of the row at pos holds keys:
 // some block it overlaps is uncovered.  win as in SlotSet (blocks b0 + w).
 __host__ __device__ inline bool chunk_has_keys(uint32_t win, int64_t pos, int window, int block, int s,

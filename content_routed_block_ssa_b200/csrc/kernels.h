@@ -28,10 +28,30 @@ cudaError_t launch_summary(const ssa_params& p, const void* K, float* mu, float*
 // step (i): routing features for the tiled router, [b, h_kv, n_q, 2d] bf16
 cudaError_t launch_features(const ssa_params& p, const void* Q, void* F, const LaunchCtx& c);
 
-// step (i): tcgen05 tile router with fused streaming top-k
+// Seeds of the tile router (one summary row per block): after every 32
+// blocks of a (batch, kv-head), snapshot s holds the topk blocks of largest
+// variance sum among blocks 0 .. 32 (s + 1) - 1 (ties to the lower block)
+// and their routing rows.  A unit of query rows whose first row sees
+// snapshot s scores those rows first: the least of the scores is a lower
+// bound on every row's k-th best score, the filter's starting threshold.
+struct RouteSeeds {
+  int32_t n_snap;            // snapshots per (batch, kv-head): nb / 32
+  float* var;                // [bgs][nb] variance sums of the routing rows
+  int32_t* blk;              // [bgs][n_snap][topk] seed blocks
+  void* tab;                 // [max(bgs * n_snap * topk, 128)][2d] bf16 seed rows
+};
+size_t route_seed_bytes(const ssa_params& p);
+// The feature rows alone: the least workspace of ssa_route_topk's tiled router.
+size_t route_min_workspace(const ssa_params& p);   // workspace of the three arrays, 256-byte aligned each
+RouteSeeds route_seed_layout(const ssa_params& p, void* base);
+cudaError_t launch_route_seeds(const ssa_params& p, const void* table, const RouteSeeds& s, const LaunchCtx& c);
+
+// step (i): tcgen05 tile router with fused streaming top-k; tmS (when not
+// NULL) maps the seed rows of `seeds`
 cudaError_t launch_route_tiled(const ssa_params& p, const CUtensorMap& tmF, const CUtensorMap& tmT,
                                int32_t* block_idx, float* top_scores, const LaunchCtx& c,
-                               const int32_t* unit_need = nullptr);
+                               const int32_t* unit_need = nullptr, const CUtensorMap* tmS = nullptr,
+                               int n_snap = 0);
 
 // step (i): one CTA per query row (bf16 table)
 cudaError_t launch_route_rowwise_bf16(const ssa_params& p, const void* Q, const void* table,
@@ -58,11 +78,20 @@ cudaError_t launch_attn_f32(const ssa_params& p, const void* Q, const void* K, c
 // Query rows per CTA of the selection inversion.
 constexpr int kPlanRows = 1024;
 
+// Summary rows per block: the S sub-blocks, plus the outlier row.
+inline int rows_per_block(const ssa_params& p) { return p.subblocks + (p.outlier ? 1 : 0); }
+
 struct BlockPlan {
   int32_t bgs, n_q, h_kv, nb, block, topk, window, qpt, nchunk;
+  // paired slots (64-key blocks): tile keys are single blocks (0 .. nb-1)
+  // and pairs of hot blocks (nb + h1 * kHotBlocks + h2); otherwise the key
+  // is the block and nkey = nb
+  int32_t pair, nkey;
+  int32_t* hot_id;     // [bgs][nb] hot number of each block, -1 when not hot (pair mode)
+  int32_t* hot_blk;    // [bgs][kHotBlocks] block of each hot number (pair mode)
   int64_t q_offset;
-  int32_t* chist;      // [bgs][nchunk][nb] slot counts, then their column scans
-  int32_t *count, *blk_off, *tile_off;   // [bgs][nb]
+  int32_t* chist;      // [bgs][nchunk][nkey] slot counts, then their column scans
+  int32_t *count, *blk_off, *tile_off;   // [bgs][nkey]
   int32_t *bg_ents, *bg_tiles;           // [bgs]
   int32_t *ent_base, *tile_base;         // [bgs + 1]
   int32_t* entries;                      // make_entry(query row, slot)
@@ -99,8 +128,10 @@ cudaError_t launch_attn_window(const ssa_params& p, const BlockPlan& pl, const C
                                const LaunchCtx& c);
 
 // Per (query, kv-head): the softmax merge of the slot partials into O, lse.
-cudaError_t launch_attn_merge(const ssa_params& p, const int32_t* block_idx, const void* partO, const void* partL,
-                              void* O, float* lse, int32_t* bad, const LaunchCtx& c);
+// hot_id: the plan's hot numbers in pair mode (64-key blocks), else NULL.
+cudaError_t launch_attn_merge(const ssa_params& p, const int32_t* block_idx, const int32_t* hot_id,
+                              const void* partO, const void* partL, void* O, float* lse, int32_t* bad,
+                              const LaunchCtx& c);
 
 // Hierarchical routing (hier.cu).  Node summaries of the bf16 routing table:
 // one warp per (batch * kv-head, node).

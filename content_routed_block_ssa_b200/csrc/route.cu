@@ -86,7 +86,18 @@ struct RouteTiledArgs {
   // optional [batch * h_kv * n_tiles] flags: units whose flag is 0 are
   // skipped (every role reads the same flag; no output is written for them)
   const int32_t* unit_need;
+  // seeds (0 snapshots: none): a unit whose first row sees snapshot s first
+  // scores that snapshot's topk seed rows, at row (bg * n_snap + s) * topk
+  int32_t n_snap;
 };
+
+// The unit's seed snapshot, or -1: the last snapshot whose 32 (s + 1)
+// blocks are all visible to the unit's first row (and so to all its rows).
+__device__ __forceinline__ int unit_snap(const RouteTiledArgs& a, int row0) {
+  if (a.n_snap == 0) return -1;
+  const int64_t nv0 = min(static_cast<int64_t>(a.nb), (a.q_offset + row0 + 1) / a.block);
+  return static_cast<int>(nv0 / 32) - 1;
+}
 
 __device__ __forceinline__ bool unit_skipped(const RouteTiledArgs& a, int bg, int row0) {
   return a.unit_need && a.unit_need[bg * a.n_tiles + row0 / 256] == 0;
@@ -274,7 +285,7 @@ __device__ __forceinline__ void filter_group(const uint32_t (&v)[16], int c0, in
 template <int KF, int KSEL>
 __global__ void __launch_bounds__(TiledCfg<KF>::THREADS, 1)
     route_tiled_kernel(const __grid_constant__ CUtensorMap tmF, const __grid_constant__ CUtensorMap tmT,
-                       const RouteTiledArgs a) {
+                       const __grid_constant__ CUtensorMap tmS, const RouteTiledArgs a) {
   using C = TiledCfg<KF>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -300,6 +311,7 @@ __global__ void __launch_bounds__(TiledCfg<KF>::THREADS, 1)
     fence_barrier_init();
     tma_prefetch_desc(&tmF);
     tma_prefetch_desc(&tmT);
+    if (a.n_snap) tma_prefetch_desc(&tmS);
   }
   if (warp == 1) {
     tmem_alloc(tmem_slot, 512);
@@ -332,13 +344,18 @@ __global__ void __launch_bounds__(TiledCfg<KF>::THREADS, 1)
                         frow + rt * 128);
         ++a_cnt;
         const int trow = bg * a.nb * a.S;
-        for (int j = 0; j < nch && ok; ++j) {
+        const int snap = unit_snap(a, row0);
+        // chunk -1: the unit's seed rows (when it has a snapshot)
+        for (int j = (snap >= 0 ? -1 : 0); j < nch && ok; ++j) {
 #pragma unroll
           for (int ks = 0; ks < C::A_BOXES; ++ks) {
             const int s = b_cnt % C::NS;
             if (!mbar_wait(&b_empty[s], ((b_cnt / C::NS) & 1) ^ 1, a.err, SITE_ROUTE_PRODUCER)) { ok = false; break; }
             mbar_arrive_expect_tx(&b_full[s], C::BOX_BYTES);
-            tma_load_2d(sB + s * C::BOX_BYTES, &tmT, &b_full[s], ks * 64, trow + j * 128);
+            if (j < 0)
+              tma_load_2d(sB + s * C::BOX_BYTES, &tmS, &b_full[s], ks * 64, (bg * a.n_snap + snap) * a.topk);
+            else
+              tma_load_2d(sB + s * C::BOX_BYTES, &tmT, &b_full[s], ks * 64, trow + j * 128);
             ++b_cnt;
           }
         }
@@ -365,7 +382,7 @@ __global__ void __launch_bounds__(TiledCfg<KF>::THREADS, 1)
         const int ab = a_cnt % C::NAB;
         if (!mbar_wait(&a_full[ab], (a_cnt / C::NAB) & 1, a.err, SITE_ROUTE_MMA)) { ok = false; break; }
         tc_fence_after();
-        for (int j = 0; j < nch && ok; ++j) {
+        for (int j = (unit_snap(a, row0) >= 0 ? -1 : 0); j < nch && ok; ++j) {
           // chunk slot: accumulators 2 slot + rt, one per tile
           const int slot = ch_cnt & 1;
           const uint32_t par = ((ch_cnt >> 1) & 1) ^ 1;
@@ -423,8 +440,37 @@ __global__ void __launch_bounds__(TiledCfg<KF>::THREADS, 1)
 #pragma unroll
       for (int j = 0; j < KSEL; ++j) { Ls[j] = -INFINITY; Li[j] = -1; }
       float thr = -INFINITY;
+      float floor_thr = -INFINITY;   // the seeds' lower bound on the k-th best score
       int cnt = 0;
       bool empty_list = true;   // warp-uniform: no merge of this unit yet
+      const int snap = unit_snap(a, row0);
+      if (snap >= 0) {
+        // chunk -1: the topk seed blocks' scores (columns 0 .. topk-1); all
+        // are visible to every row of the unit, so the least of them is at
+        // most the row's k-th best score.  The threshold sits a little
+        // below it, so a block scoring exactly that much still passes.
+        const int acc = 2 * (ch_cnt & 1) + grp;
+        ok = __all_sync(0xFFFFFFFFu, mbar_wait(&acc_full[acc], (ch_cnt >> 1) & 1, a.err, SITE_ROUTE_EPILOGUE));
+        if (!ok) break;
+        tc_fence_after();
+        const uint32_t taddr = tmem_base + (static_cast<uint32_t>(eq * 32) << 16) + acc * 128;
+        uint32_t v0[16], v1[16];
+        tmem_ld16(taddr, v0);
+        tmem_ld16(taddr + 16, v1);
+        tmem_wait_ld();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&acc_empty[acc]);
+        float mn = INFINITY;
+#pragma unroll
+        for (int t = 0; t < 16; ++t) {
+          if (t < a.topk) mn = fminf(mn, __uint_as_float(v0[t]));
+          if (t + 16 < a.topk) mn = fminf(mn, __uint_as_float(v1[t]));
+        }
+        floor_thr = mn - (fabsf(mn) * 0x1p-16f + 0x1p-24f);
+        thr = floor_thr;
+        ++ch_cnt;
+      }
       for (int j = 0; j < nch; ++j) {
         const int acc = 2 * (ch_cnt & 1) + grp;
         ok = __all_sync(0xFFFFFFFFu, mbar_wait(&acc_full[acc], (ch_cnt >> 1) & 1, a.err, SITE_ROUTE_EPILOGUE));
@@ -450,6 +496,7 @@ __global__ void __launch_bounds__(TiledCfg<KF>::THREADS, 1)
             filter_group<4>(v, c0, nvis, thr, cnt, my_cand);
           if (__any_sync(0xFFFFFFFFu, cnt > C::CAP - 16)) {
             merge_candidates<KSEL>(Ls, Li, cnt, thr, my_cand, a.topk, empty_list);
+            thr = fmaxf(thr, floor_thr);
             empty_list = false;
           }
         }
@@ -490,22 +537,23 @@ __global__ void __launch_bounds__(TiledCfg<KF>::THREADS, 1)
 }
 
 template <int KF, int KSEL>
-cudaError_t run_tiled(const ssa_params& p, const CUtensorMap& tmF, const CUtensorMap& tmT,
-                      int32_t* idx, float* scores, const int32_t* unit_need, const LaunchCtx& c) {
+cudaError_t run_tiled(const ssa_params& p, const CUtensorMap& tmF, const CUtensorMap& tmT, const CUtensorMap* tmS,
+                      int n_snap, int32_t* idx, float* scores, const int32_t* unit_need, const LaunchCtx& c) {
   using C = TiledCfg<KF>;
   RouteTiledArgs a;
   a.batch = p.batch; a.n_q = p.n_q; a.h_kv = p.h_kv; a.nb = p.n_kv / p.block;
-  a.block = p.block; a.topk = p.topk; a.S = p.subblocks;
+  a.block = p.block; a.topk = p.topk; a.S = rows_per_block(p);
   a.n_tiles = (p.n_q + 255) / 256;   // 256-row units per (batch, kv-head)
   a.n_units = p.batch * p.h_kv * a.n_tiles;
   a.q_offset = p.q_offset;
   a.block_idx = idx; a.top_scores = scores; a.err = c.err;
   a.unit_need = unit_need;
+  a.n_snap = tmS ? n_snap : 0;
   cudaError_t e = cudaFuncSetAttribute(route_tiled_kernel<KF, KSEL>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
   if (e != cudaSuccess) return e;
   const int grid = a.n_units < c.sm_count ? a.n_units : c.sm_count;
-  route_tiled_kernel<KF, KSEL><<<grid, C::THREADS, C::SMEM, c.stream>>>(tmF, tmT, a);
+  route_tiled_kernel<KF, KSEL><<<grid, C::THREADS, C::SMEM, c.stream>>>(tmF, tmT, tmS ? *tmS : tmT, a);
   note_launch();
   return cudaGetLastError();
 }
@@ -971,7 +1019,7 @@ __global__ void __launch_bounds__(256) route_qtile_f32_kernel(const float* __res
 RowArgs row_args(const ssa_params& p, int32_t* idx, float* scores) {
   RowArgs a;
   a.n_q = p.n_q; a.h_kv = p.h_kv; a.nb = p.n_kv / p.block; a.block = p.block; a.topk = p.topk;
-  a.S = p.subblocks;
+  a.S = rows_per_block(p);
   a.q_offset = p.q_offset;
   a.half_beta = p.beta * 0.5f;   // exact
   a.block_idx = idx; a.top_scores = scores;
@@ -1099,19 +1147,146 @@ cudaError_t launch_features(const ssa_params& p, const void* Q, void* F, const L
 }
 
 cudaError_t launch_route_tiled(const ssa_params& p, const CUtensorMap& tmF, const CUtensorMap& tmT,
-                               int32_t* idx, float* scores, const LaunchCtx& c, const int32_t* unit_need) {
+                               int32_t* idx, float* scores, const LaunchCtx& c, const int32_t* unit_need,
+                               const CUtensorMap* tmS, int n_snap) {
   const int ksel = p.topk <= 8 ? 8 : (p.topk <= 16 ? 16 : 32);
+  if (rows_per_block(p) != 1) tmS = nullptr;   // seeds are whole-block rows
   if (p.d == 128) {
-    if (ksel == 8) return run_tiled<256, 8>(p, tmF, tmT, idx, scores, unit_need, c);
-    if (ksel == 16) return run_tiled<256, 16>(p, tmF, tmT, idx, scores, unit_need, c);
-    return run_tiled<256, 32>(p, tmF, tmT, idx, scores, unit_need, c);
+    if (ksel == 8) return run_tiled<256, 8>(p, tmF, tmT, tmS, n_snap, idx, scores, unit_need, c);
+    if (ksel == 16) return run_tiled<256, 16>(p, tmF, tmT, tmS, n_snap, idx, scores, unit_need, c);
+    return run_tiled<256, 32>(p, tmF, tmT, tmS, n_snap, idx, scores, unit_need, c);
   }
   if (p.d == 64) {
-    if (ksel == 8) return run_tiled<128, 8>(p, tmF, tmT, idx, scores, unit_need, c);
-    if (ksel == 16) return run_tiled<128, 16>(p, tmF, tmT, idx, scores, unit_need, c);
-    return run_tiled<128, 32>(p, tmF, tmT, idx, scores, unit_need, c);
+    if (ksel == 8) return run_tiled<128, 8>(p, tmF, tmT, tmS, n_snap, idx, scores, unit_need, c);
+    if (ksel == 16) return run_tiled<128, 16>(p, tmF, tmT, tmS, n_snap, idx, scores, unit_need, c);
+    return run_tiled<128, 32>(p, tmF, tmT, tmS, n_snap, idx, scores, unit_need, c);
   }
   return cudaErrorInvalidValue;
+}
+
+// ------------------------------------------------------------------ seeds
+
+size_t route_seed_bytes(const ssa_params& p) {
+  if (rows_per_block(p) != 1 || p.dtype != SSA_BF16) return 0;
+  const size_t bgs = static_cast<size_t>(p.batch) * p.h_kv;
+  const size_t nb = static_cast<size_t>(p.n_kv / p.block);
+  const size_t n_snap = nb / 32;
+  if (n_snap == 0) return 0;
+  auto ru = [](size_t x) { return (x + 255) & ~size_t(255); };
+  const size_t rows = bgs * n_snap * p.topk > 128 ? bgs * n_snap * p.topk : 128;
+  return ru(bgs * nb * 4) + ru(bgs * n_snap * p.topk * 4) + ru(rows * 2 * p.d * 2);
+}
+
+RouteSeeds route_seed_layout(const ssa_params& p, void* base) {
+  RouteSeeds s{};
+  const size_t bgs = static_cast<size_t>(p.batch) * p.h_kv;
+  const size_t nb = static_cast<size_t>(p.n_kv / p.block);
+  s.n_snap = static_cast<int32_t>(nb / 32);
+  auto ru = [](size_t x) { return (x + 255) & ~size_t(255); };
+  uint8_t* b = static_cast<uint8_t*>(base);
+  s.var = reinterpret_cast<float*>(b);
+  s.blk = reinterpret_cast<int32_t*>(b + ru(bgs * nb * 4));
+  s.tab = b + ru(bgs * nb * 4) + ru(bgs * s.n_snap * p.topk * 4);
+  return s;
+}
+
+namespace {
+
+// Warp per routing row: the sum of its variance half (any order: the seeds
+// only need some blocks, and every choice of them gives a valid bound).
+template <int D>
+__global__ void __launch_bounds__(256) seed_var_kernel(const __nv_bfloat16* __restrict__ T, float* __restrict__ var,
+                                                       int64_t rows) {
+  const int64_t row = (static_cast<int64_t>(blockIdx.x) * 256 + threadIdx.x) >> 5;
+  if (row >= rows) return;   // warp-uniform
+  const int lane = threadIdx.x & 31;
+  const __nv_bfloat16* v = T + row * (2 * D) + D;
+  float acc = 0.f;
+#pragma unroll
+  for (int t = lane; t < D; t += 32) acc += __bfloat162float(v[t]);
+#pragma unroll
+  for (int o = 16; o; o >>= 1) acc += __shfl_xor_sync(0xFFFFFFFFu, acc, o);
+  if (lane == 0) var[row] = acc;
+}
+
+// Lane l of the warp ends with the l-th largest of the warp's 32 keys.
+__device__ __forceinline__ uint64_t warp_sort_desc(uint64_t key) {
+  const int lane = threadIdx.x & 31;
+#pragma unroll
+  for (int size = 2; size <= 32; size <<= 1) {
+#pragma unroll
+    for (int stride = size >> 1; stride > 0; stride >>= 1) {
+      const uint64_t other = __shfl_xor_sync(0xFFFFFFFFu, key, stride);
+      const bool desc = (lane & size) == 0 || size == 32;
+      const bool low = (lane & stride) == 0;
+      key = (low == desc) ? (key > other ? key : other) : (key < other ? key : other);
+    }
+  }
+  return key;
+}
+
+// Warp per (batch, kv-head): the running 32 blocks of largest variance sum
+// (key: variance desc, then block asc), and after every full batch of 32
+// blocks the first topk of them as snapshot s.
+__global__ void __launch_bounds__(256) seed_prefix_kernel(const float* __restrict__ var, int32_t* __restrict__ blk,
+                                                          int bgs, int nb, int n_snap, int topk) {
+  const int bg = (blockIdx.x * 256 + threadIdx.x) >> 5;
+  if (bg >= bgs) return;   // warp-uniform
+  const int lane = threadIdx.x & 31;
+  uint64_t best = 0;       // lane l: the l-th best so far (0: none)
+  for (int s = 0; s < n_snap; ++s) {
+    const int c = s * 32 + lane;
+    const uint64_t key = make_key(__float_as_uint(var[static_cast<int64_t>(bg) * nb + c]), static_cast<uint32_t>(c));
+    const uint64_t fresh = warp_sort_desc(key);
+    // the larger 32 of two descending runs: best[l] against fresh[31 - l]
+    // gives a bitonic sequence holding them; sort it
+    const uint64_t rev = __shfl_sync(0xFFFFFFFFu, fresh, 31 - lane);
+    best = warp_sort_desc(best > rev ? best : rev);
+    if (lane < topk) blk[(static_cast<int64_t>(bg) * n_snap + s) * topk + lane] = static_cast<int32_t>(key_block(best));
+  }
+}
+
+// Warp per seed row: copies the routing row of its block.
+template <int D>
+__global__ void __launch_bounds__(256) seed_gather_kernel(const __nv_bfloat16* __restrict__ T,
+                                                          const int32_t* __restrict__ blk,
+                                                          __nv_bfloat16* __restrict__ tab, int64_t rows, int nb,
+                                                          int per_bg) {
+  const int64_t r = (static_cast<int64_t>(blockIdx.x) * 256 + threadIdx.x) >> 5;
+  if (r >= rows) return;   // warp-uniform
+  const int lane = threadIdx.x & 31;
+  const int64_t bg = r / per_bg;
+  const int c = blk[r];
+  constexpr int PER = 2 * D / 32;   // bf16 values per lane
+  const __nv_bfloat16* src = T + (bg * nb + c) * (2 * D) + lane * PER;
+  __nv_bfloat16* dst = tab + r * (2 * D) + lane * PER;
+  if constexpr (PER == 8)
+    *reinterpret_cast<uint4*>(dst) = *reinterpret_cast<const uint4*>(src);
+  else
+    *reinterpret_cast<uint2*>(dst) = *reinterpret_cast<const uint2*>(src);
+}
+
+}  // namespace
+
+cudaError_t launch_route_seeds(const ssa_params& p, const void* table, const RouteSeeds& s, const LaunchCtx& c) {
+  const int bgs = p.batch * p.h_kv;
+  const int nb = p.n_kv / p.block;
+  const __nv_bfloat16* T = static_cast<const __nv_bfloat16*>(table);
+  const int64_t rows = static_cast<int64_t>(bgs) * nb;
+  const unsigned g1 = static_cast<unsigned>((rows * 32 + 255) / 256);
+  if (p.d == 128) seed_var_kernel<128><<<g1, 256, 0, c.stream>>>(T, s.var, rows);
+  else seed_var_kernel<64><<<g1, 256, 0, c.stream>>>(T, s.var, rows);
+  note_launch();
+  seed_prefix_kernel<<<static_cast<unsigned>((bgs * 32 + 255) / 256), 256, 0, c.stream>>>(s.var, s.blk, bgs, nb,
+                                                                                          s.n_snap, p.topk);
+  note_launch();
+  const int64_t srows = static_cast<int64_t>(bgs) * s.n_snap * p.topk;
+  const unsigned g3 = static_cast<unsigned>((srows * 32 + 255) / 256);
+  __nv_bfloat16* tab = static_cast<__nv_bfloat16*>(s.tab);
+  if (p.d == 128) seed_gather_kernel<128><<<g3, 256, 0, c.stream>>>(T, s.blk, tab, srows, nb, s.n_snap * p.topk);
+  else seed_gather_kernel<64><<<g3, 256, 0, c.stream>>>(T, s.blk, tab, srows, nb, s.n_snap * p.topk);
+  note_launch();
+  return cudaGetLastError();
 }
 
 cudaError_t launch_route_rowwise_bf16(const ssa_params& p, const void* Q, const void* table,

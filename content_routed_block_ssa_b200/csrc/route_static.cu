@@ -25,6 +25,7 @@
 
 #include <mutex>
 
+#include "kernels.h"
 #include "ssa.h"
 
 namespace {
@@ -55,7 +56,9 @@ extern "C" ssa_status ssa_route_topk_static(const ssa_params* p, const void* Q, 
                                             const float* sigma, const void* route_table,
                                             int32_t* block_idx, float* top_scores, void* stream) {
   if (!p) return SSA_ERR_INVALID_ARG;
-  const size_t need = ssa_route_workspace_size(p);
+  // the feature rows must fit; the router's seed arrays are used when they
+  // fit beside them
+  const size_t need = ssa::route_min_workspace(*p);
   if (need > SSA_ROUTE_STATIC_SCRATCH_BYTES) return SSA_ERR_WORKSPACE;
   void* scratch = nullptr;
   if (need > 0) {

@@ -81,7 +81,7 @@ inline size_t round_up(size_t x) { return (x + 255) & ~size_t(255); }
 
 int64_t nb_of(const ssa_params& p) { return p.block > 0 ? p.n_kv / p.block : 0; }
 // Summary rows per (batch, kv-head): one per sub-block.
-int64_t summary_rows(const ssa_params& p) { return nb_of(p) * p.subblocks; }
+int64_t summary_rows(const ssa_params& p) { return nb_of(p) * ssa::rows_per_block(p); }
 size_t esize(const ssa_params& p) { return p.dtype == SSA_BF16 ? 2 : 4; }
 
 bool is_empty(const ssa_params& p) { return p.batch == 0 || p.n_q == 0; }
@@ -94,7 +94,8 @@ ssa_status check_params(const ssa_params* pp) {
       p.topk < 1 || p.window < 1)
     return SSA_ERR_INVALID_ARG;
   if (p.h_q % p.h_kv != 0 || p.n_kv % p.block != 0) return SSA_ERR_INVALID_ARG;
-  if (p.subblocks < 1 || p.block % p.subblocks != 0 || p.reserved != 0) return SSA_ERR_INVALID_ARG;
+  if (p.subblocks < 1 || p.block % p.subblocks != 0 || (p.outlier != 0 && p.outlier != 1))
+    return SSA_ERR_INVALID_ARG;
   if (p.q_offset < 0 || p.q_offset + p.n_q > p.n_kv) return SSA_ERR_INVALID_ARG;
   if ((p.dtype != SSA_F32 && p.dtype != SSA_BF16) || (p.sigma != SSA_SIGMA_DIAG && p.sigma != SSA_SIGMA_FULL) ||
       p.route_impl < SSA_ROUTE_AUTO || p.route_impl > SSA_ROUTE_ROWWISE)
@@ -105,6 +106,7 @@ ssa_status check_params(const ssa_params* pp) {
   if (p.block != 64 && p.block != 128) return SSA_ERR_UNSUPPORTED;
   if ((p.subblocks != 1 && p.subblocks != 2 && p.subblocks != 4) || p.block / p.subblocks < 32)
     return SSA_ERR_UNSUPPORTED;
+  if (p.outlier && p.subblocks != 1) return SSA_ERR_UNSUPPORTED;
   if (G != 1 && G != 2 && G != 4 && G != 8) return SSA_ERR_UNSUPPORTED;
   if (p.topk > 32 || p.window > 4032) return SSA_ERR_UNSUPPORTED;
   if (p.dtype == SSA_BF16 && p.sigma != SSA_SIGMA_DIAG) return SSA_ERR_UNSUPPORTED;
@@ -132,6 +134,11 @@ bool rowwise_fits(const ssa_params& p) {
 
 size_t features_bytes(const ssa_params& p) {
   return use_tiled(p) ? round_up(static_cast<size_t>(p.batch) * p.h_kv * p.n_q * 2 * p.d * 2) : 0;
+}
+// Route workspace: the feature rows (required by the tiled router), then
+// the router's seed arrays (used when the caller's workspace holds them).
+size_t route_ws_bytes(const ssa_params& p) {
+  return features_bytes(p) + (use_tiled(p) ? ssa::route_seed_bytes(p) : 0);
 }
 size_t table_bytes(const ssa_params& p) {
   return p.dtype == SSA_BF16 ? round_up(static_cast<size_t>(p.batch) * p.h_kv * summary_rows(p) * 2 * p.d * 2) : 0;
@@ -162,10 +169,14 @@ bool use_block_attn(const ssa_params& p) {
          ssa::window_slots(p.window, p.block) <= 32 && nb <= 16384 && p.n_q >= 1024 && p.n_q < (1 << 25);
 }
 
+// Paired slots: the block-major attention of 64-key blocks evaluates two
+// selected blocks per slot (128-key tiles).
+bool pair_mode(const ssa_params& p) { return p.block == 64; }
+
 struct AttnLayout {
   size_t chist, count, blk_off, tile_off, bg_ents, bg_tiles, ent_base, tile_base, entries, tiles, tcost, csum,
-      t_start, win, part_o, part_l, total;
-  int nchunk, nsl;
+      t_start, win, hot_id, hot_blk, part_o, part_l, total;
+  int nchunk, nsl, nkey;
   size_t max_tiles;
 };
 
@@ -180,12 +191,14 @@ AttnLayout attn_layout(const ssa_params& p) {
   L.nsl = p.topk + ssa::window_chunks(p.window, p.h_q / p.h_kv);
   const size_t items = bgs * p.n_q;
   const size_t sel = items * L.nsl;                       // entries, at most
-  const size_t max_tiles = (sel + qpt - 1) / qpt + bgs * nb;
+  const size_t nkey = nb + (pair_mode(p) ? static_cast<size_t>(ssa::kHotBlocks) * ssa::kHotBlocks : 0);
+  L.nkey = static_cast<int>(nkey);
+  const size_t max_tiles = (sel + qpt - 1) / qpt + bgs * nkey;
   size_t off = 0;
-  L.chist = off; off += round_up(bgs * L.nchunk * nb * 4);
-  L.count = off; off += round_up(bgs * nb * 4);
-  L.blk_off = off; off += round_up(bgs * nb * 4);
-  L.tile_off = off; off += round_up(bgs * nb * 4);
+  L.chist = off; off += round_up(bgs * L.nchunk * nkey * 4);
+  L.count = off; off += round_up(bgs * nkey * 4);
+  L.blk_off = off; off += round_up(bgs * nkey * 4);
+  L.tile_off = off; off += round_up(bgs * nkey * 4);
   L.bg_ents = off; off += round_up(bgs * 4);
   L.bg_tiles = off; off += round_up(bgs * 4);
   L.ent_base = off; off += round_up((bgs + 1) * 4);
@@ -197,6 +210,8 @@ AttnLayout attn_layout(const ssa_params& p) {
   L.csum = off; off += round_up((max_tiles + 255) / 256 * 4);
   L.t_start = off; off += round_up((ssa::kMaxBlockGrid + 1) * 4);
   L.win = off; off += round_up(items * 4);
+  L.hot_id = off; off += pair_mode(p) ? round_up(bgs * nb * 4) : 0;
+  L.hot_blk = off; off += pair_mode(p) ? round_up(bgs * ssa::kHotBlocks * 4) : 0;
   L.part_o = off; off += round_up(sel * G * p.d * 2);
   L.part_l = off; off += round_up(sel * G * 8);
   L.total = off;
@@ -301,6 +316,15 @@ ssa_status do_route(const ssa_params& p, const void* Q, const float* mu, const f
   if (!encode_2d(&tmF, ws, kf, static_cast<uint64_t>(p.batch) * p.h_kv * p.n_q, 128) ||
       !encode_2d(&tmT, table, kf, static_cast<uint64_t>(p.batch) * p.h_kv * summary_rows(p), 128))
     return SSA_ERR_CUDA;
+  const size_t sb = ssa::route_seed_bytes(p);
+  if (sb && ws_bytes >= need + sb) {
+    const ssa::RouteSeeds S = ssa::route_seed_layout(p, static_cast<uint8_t*>(ws) + need);
+    if ((st = from_cuda(ssa::launch_route_seeds(p, table, S, c))) != SSA_OK) return st;
+    const uint64_t srows = static_cast<uint64_t>(p.batch) * p.h_kv * S.n_snap * p.topk;
+    CUtensorMap tmS;
+    if (!encode_2d(&tmS, S.tab, kf, srows > 128 ? srows : 128, 128)) return SSA_ERR_CUDA;
+    return from_cuda(ssa::launch_route_tiled(p, tmF, tmT, idx, scores, c, nullptr, &tmS, S.n_snap));
+  }
   return from_cuda(ssa::launch_route_tiled(p, tmF, tmT, idx, scores, c));
 }
 
@@ -315,6 +339,10 @@ ssa::BlockPlan block_plan(const ssa_params& p, const AttnLayout& L, uint8_t* w) 
   pl.window = p.window;
   pl.qpt = 128 / (p.h_q / p.h_kv);
   pl.nchunk = L.nchunk;
+  pl.pair = pair_mode(p) ? 1 : 0;
+  pl.nkey = L.nkey;
+  pl.hot_id = pl.pair ? reinterpret_cast<int32_t*>(w + L.hot_id) : nullptr;
+  pl.hot_blk = pl.pair ? reinterpret_cast<int32_t*>(w + L.hot_blk) : nullptr;
   pl.q_offset = p.q_offset;
   pl.chist = reinterpret_cast<int32_t*>(w + L.chist);
   pl.count = reinterpret_cast<int32_t*>(w + L.count);
@@ -377,7 +405,8 @@ ssa_status attn_stage_window(const ssa_params& p, const AttnMaps& m, uint8_t* w,
 ssa_status attn_stage_merge(const ssa_params& p, const int32_t* idx, void* O, float* lse, int32_t* bad,
                             const uint8_t* w, const LaunchCtx& c) {
   const AttnLayout L = attn_layout(p);
-  return from_cuda(ssa::launch_attn_merge(p, idx, w + L.part_o, w + L.part_l, O, lse, bad, c));
+  const int32_t* hot_id = pair_mode(p) ? reinterpret_cast<const int32_t*>(w + L.hot_id) : nullptr;
+  return from_cuda(ssa::launch_attn_merge(p, idx, hot_id, w + L.part_o, w + L.part_l, O, lse, bad, c));
 }
 
 ssa_status do_attn(const ssa_params& p, const void* Q, const void* K, const void* V,
@@ -408,7 +437,7 @@ ForwardLayout forward_layout(const ssa_params& p) {
   L.table = off; off += table_bytes(p);
   L.mu = off; off += mu_bytes(p);
   L.sigma = off; off += sigma_bytes(p);
-  L.feat = off; off += features_bytes(p);
+  L.feat = off; off += route_ws_bytes(p);
   L.idx = off; off += idx_bytes(p);
   L.attn = off; off += attn_layout(p).total;
   L.total = off;
@@ -443,8 +472,8 @@ ssa_status forward_impl(const ssa_params& p, const void* Q, const void* K, const
   int32_t* idx = reinterpret_cast<int32_t*>(ws + L.idx);
   ssa_status st = do_summary(p, K, mu, sg, table, c);
   if (st != SSA_OK) return st;
-  st = do_route(p, Q, mu, sg, table, idx, nullptr, features_bytes(p) ? ws + L.feat : nullptr,
-                features_bytes(p), c);
+  st = do_route(p, Q, mu, sg, table, idx, nullptr, route_ws_bytes(p) ? ws + L.feat : nullptr,
+                route_ws_bytes(p), c);
   if (st != SSA_OK) return st;
   const size_t aw = attn_layout(p).total;
   return do_attn(p, Q, K, V, idx, O, lse, nullptr, aw ? ws + L.attn : nullptr, aw, c);
@@ -497,7 +526,7 @@ ssa_status check_hier(const ssa_params* p, const ssa_hier_params* hp) {
   if (M < 1 || M > 64 || (M & (M - 1)) != 0) return SSA_ERR_INVALID_ARG;
   if (hp->probe < 1 || hp->probe > 31 || (hp->escalate != 0 && hp->escalate != 1)) return SSA_ERR_INVALID_ARG;
   if ((hp->probe + 1) * M > 512) return SSA_ERR_UNSUPPORTED;   // candidates per row of the probe kernel
-  if (p->dtype != SSA_BF16 || p->subblocks != 1) return SSA_ERR_UNSUPPORTED;
+  if (p->dtype != SSA_BF16 || p->subblocks != 1 || p->outlier) return SSA_ERR_UNSUPPORTED;
   if (!use_tiled(*p) && !rowwise_fits(*p)) return SSA_ERR_UNSUPPORTED;
   return SSA_OK;
 }
@@ -564,6 +593,10 @@ ssa_status do_route_hier(const ssa_params& p, const ssa_hier_params& hp, const v
 
 }  // namespace
 
+namespace ssa {
+size_t route_min_workspace(const ssa_params& p) { return check_params(&p) == SSA_OK ? features_bytes(p) : 0; }
+}  // namespace ssa
+
 extern "C" {
 
 const char* ssa_status_string(int32_t s) {
@@ -610,7 +643,7 @@ ssa_status ssa_block_summary(const ssa_params* pp, const void* K, float* mu, flo
 
 size_t ssa_route_workspace_size(const ssa_params* p) {
   if (check_params(p) != SSA_OK) return 0;
-  return features_bytes(*p);
+  return route_ws_bytes(*p);
 }
 
 ssa_status ssa_route_topk(const ssa_params* pp, const void* Q, const float* mu, const float* sigma,

@@ -35,7 +35,7 @@ def test_params_layout_matches_header():
     assert ssa.ssa_params.beta.offset == 56
     assert ssa.ssa_params.scale.offset == 60
     assert ssa.ssa_params.subblocks.offset == 64
-    assert ssa.ssa_params.reserved.offset == 68
+    assert ssa.ssa_params.outlier.offset == 68
     text = open(HEADER).read()
     body = text[text.index("typedef struct {"):text.index("} ssa_params;")]
     fields = re.findall(r"\b(int32_t|int64_t|float)\s+(\w+);", body)
@@ -88,12 +88,22 @@ def test_invalid_and_unsupported_params(kw, code):
     assert ssa.lib.ssa_workspace_size(C.byref(p)) == 0
 
 
-def test_reserved_field_must_be_zero():
-    p = good()
-    p.reserved = 1
+def test_outlier_field_is_a_flag():
     dummy = 256
-    assert ssa.lib.ssa_block_summary(C.byref(p), dummy, None, None, dummy, None) == ssa.SSA_ERR_INVALID_ARG
-    assert ssa.ssa_workspace_size(p) == 0
+    for v in (2, -1):
+        p = good()
+        p.outlier = v
+        assert ssa.lib.ssa_block_summary(C.byref(p), dummy, None, None, dummy, None) == ssa.SSA_ERR_INVALID_ARG
+        assert ssa.ssa_workspace_size(p) == 0
+    # the outlier row is not combined with sub-block summaries, nor with the
+    # hierarchical router
+    p = good(subblocks=2, outlier=True)
+    assert ssa.lib.ssa_block_summary(C.byref(p), dummy, None, None, dummy, None) == ssa.SSA_ERR_UNSUPPORTED
+    p = good(outlier=True)
+    assert ssa.ssa_hier_nodes_size(p, ssa.make_hier_params()) == 0
+    # two summary rows per block
+    mu, sig, tab = ssa.summary_shapes(p)
+    assert mu == (1, 2, 2 * (256 // 64), 128) and tab == (1, 2, 2 * (256 // 64), 256)
 
 
 def test_null_and_misaligned_pointers_rejected():
@@ -128,6 +138,12 @@ def test_workspace_sizes():
     rnd = lambda x: (x + 255) // 256 * 256
     assert ssa.ssa_route_workspace_size(p) == rnd(feat)
     assert ssa.ssa_workspace_size(p) == rnd(tab) + rnd(feat) + rnd(idx)
+    # with at least 32 blocks the tiled router also takes its seed arrays:
+    # variance sums [bgs, nb] f32, seed blocks [bgs, nb/32, k] i32 and the
+    # seed rows [max(bgs * nb/32 * k, 128), 2d] bf16
+    sp = good(n_q=1000, n_kv=4096)
+    feat4 = 1 * 2 * 1000 * 256 * 2
+    assert ssa.ssa_route_workspace_size(sp) == rnd(feat4) + rnd(2 * 64 * 4) + rnd(2 * 2 * 4 * 4) + rnd(128 * 256 * 2)
     row = good(n_q=1, n_kv=1024, q_offset=1023)           # decode routes per row: no features
     assert ssa.ssa_route_workspace_size(row) == 0
     f32 = good(dtype="f32", sigma="full", d=64, h_q=2, n_q=128, n_kv=128)
