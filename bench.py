@@ -2,7 +2,7 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
                     [--workload NAME] [--no-secondary] [--no-cpu-baseline] [--no-e2e]
-                    [--subblocks S] [--router flat|hier [--fanout M] [--probe P] [--escalate]]
+                    [--subblocks S] [--outlier] [--router flat|hier [--fanout M] [--probe P] [--escalate]]
 
 One step is one pass of the whole layer over the workload's synthetic input:
 block summaries -> routing features + tensor-core route with fused top-k ->
@@ -265,19 +265,20 @@ def algorithmic_work(w, idx):
     nvis = np.minimum(nb, (pos + 1) // w.block).sum()
     # one summary row and one routing dot product per sub-block (float32:
     # mu and Sigma rows, d + d^2 for a full Sigma)
-    summary_bytes = w.batch * w.n * w.h_kv * w.d * es + w.batch * w.h_kv * nb * w.subblocks * 2 * w.d * 2
-    route_flops = 2.0 * (2 * w.d) * float(nvis) * w.subblocks * w.h_kv * w.batch
+    R = w.subblocks + (1 if w.outlier else 0)      # summary rows per block
+    summary_bytes = w.batch * w.n * w.h_kv * w.d * es + w.batch * w.h_kv * nb * R * 2 * w.d * 2
+    route_flops = 2.0 * (2 * w.d) * float(nvis) * R * w.h_kv * w.batch
     if w.dtype == "f32":
         per = w.d + (w.d * w.d if w.sigma == "full" else w.d)
-        route_flops = 2.0 * per * float(nvis) * w.subblocks * w.h_q * w.batch
+        route_flops = 2.0 * per * float(nvis) * R * w.h_q * w.batch
         summary_bytes = w.batch * w.n * w.h_kv * w.d * es + w.batch * w.h_kv * nb * per * 4
-    route_table_bytes = float(nvis) * w.subblocks * w.h_kv * w.batch * 2 * w.d * 2
+    route_table_bytes = float(nvis) * R * w.h_kv * w.batch * 2 * w.d * 2
     S = attended_keys(idx, w)
     gathered = float(S.sum().item()) * w.d * 2 * es
     qo = 2.0 * w.batch * w.n_q * w.h_q * w.d * es
     attn_flops = 4.0 * float(S.sum().item()) * G * w.d
     # one pass over the routing table (the node summaries read every block row once)
-    route_table_bytes_once = float(w.batch * w.h_kv * nb) * w.subblocks * 2 * w.d * 2
+    route_table_bytes_once = float(w.batch * w.h_kv * nb) * R * 2 * w.d * 2
     out = dict(summary_bytes=summary_bytes, route_flops=route_flops, route_table_bytes=route_table_bytes,
                route_table_bytes_once=route_table_bytes_once,
                attn_bytes=gathered + qo,
@@ -574,7 +575,7 @@ def layer_report(w, wk, ms_step, peaks):
     flops = wk["route_flops"] + wk["attn_flops"]
     io = (w.batch * w.n_q * w.h_q * w.d * es * 2 + w.batch * w.n * w.h_kv * w.d * es * 2
           + w.batch * w.n_q * w.h_q * 4)
-    table = w.batch * w.h_kv * nb * w.subblocks * 2 * w.d * (2 if w.dtype == "bf16" else 4)
+    table = w.batch * w.h_kv * nb * (w.subblocks + (1 if w.outlier else 0)) * 2 * w.d * (2 if w.dtype == "bf16" else 4)
     idx = w.batch * w.n_q * w.h_kv * w.topk * 4
     nbytes = io + 2 * table + 2 * idx
     t = ms_step * 1e-3
@@ -654,6 +655,8 @@ def main():
                     help="shorter sequence of the same workload (profiling captures); not a bench line")
     ap.add_argument("--subblocks", type=int, default=1,
                     help="route on S sub-block summaries per block, max-pooled (S in 1, 2, 4; block / S >= 32)")
+    ap.add_argument("--outlier", action="store_true",
+                    help="route with the outlier-channel row per block (largest-norm key, max-pooled)")
     ap.add_argument("--router", default="flat", choices=["flat", "hier"],
                     help="hier: the hierarchical router (nodes of --fanout blocks, --probe nodes per row); "
                          "a measurement of that router, not the bench line")
@@ -666,12 +669,14 @@ def main():
         w = w.scaled(n=a.n, needles=max(1, w.needles * a.n // w.n))
     if a.subblocks != 1:
         w = w.scaled(subblocks=a.subblocks)
+    if a.outlier:
+        w = w.scaled(outlier=True)
     ws, rank, local = dist_setup(a.gpus)
     peaks, peak_src = load_peaks()
 
     config = {"workload": w.name, "batch": w.batch, "n": w.n, "n_q": w.n_q, "h_q": w.h_q, "h_kv": w.h_kv,
               "d": w.d, "block": w.block, "topk": w.topk, "window": w.window, "sigma": w.sigma,
-              "subblocks": w.subblocks,
+              "subblocks": w.subblocks, "outlier": w.outlier,
               "beta": w.beta, "keys": "block-clustered + planted needles" if w.clustered else "iid + planted needles",
               "l2": "flushed between steps (256 MiB write); inputs larger than L2",
               "parallelism": f"replicas x{ws} (independent problems)"}
@@ -692,7 +697,7 @@ def main():
         return
 
     # the committed DRAM counters were taken with whole-block summaries
-    traffic = load_traffic() if w.subblocks == 1 else {}
+    traffic = load_traffic() if w.subblocks == 1 and not w.outlier else {}
     hier = (a.fanout, a.probe, a.escalate) if a.router == "hier" else None
     if w.decode:
         config["state"] = "block summaries precomputed (built once, untimed; kernels.summary times one build)"
@@ -719,9 +724,12 @@ def main():
         w2 = WORKLOADS[SECONDARY]
         if w.subblocks != 1 and w2.block // w.subblocks >= 32:
             w2 = w2.scaled(subblocks=w.subblocks)
+        if w.outlier:
+            w2 = w2.scaled(outlier=True)
         r2 = run_ours(w2, max(3, a.steps // 2), a.warmup, ws, rank, with_e2e=False)
         k2 = kernel_report(w2, r2, peaks, traffic)
-        secondary = {"workload": w2.name, "subblocks": w2.subblocks,
+        secondary = {"workload": w2.name, "subblocks": w2.subblocks, "outlier": w2.outlier,
+                     "selection": r2["selection"],
                      "value": whole_job_rate(w2.batch * w2.n_q * w2.h_q, ws, r2["ms_step"]),
                      "unit": UNIT, "ms_per_step": r2["ms_step"], "kernels": k2, "gpu_launches": r2["launches"],
                      "clocks": r2["clocks"]}

@@ -1,4 +1,5 @@
-// Step (i) of the layer: per-block key summaries.
+// Step (i) of the layer: per-block key summaries (and the outlier channel's
+// rows).
 //
 // "routes ... using only per-block summary statistics"
 // [Subquadratic Sparse Attention (SSA), opening section]; the routing score
@@ -48,7 +49,7 @@ __global__ void __launch_bounds__(256) summary_diag_kernel(const T* __restrict__
                                                            float* __restrict__ mu,
                                                            float* __restrict__ sig,
                                                            __nv_bfloat16* __restrict__ table,
-                                                           int n_kv, int h_kv, int nb) {
+                                                           int n_kv, int h_kv, int nb, int rstride) {
   constexpr int VEC = 16 / sizeof(T);
   constexpr int CG = D / VEC;
   constexpr int RG = 256 / CG;
@@ -100,7 +101,7 @@ __global__ void __launch_bounds__(256) summary_diag_kernel(const T* __restrict__
     for (int r = 0; r < RG; ++r) s += red[r][threadIdx.x];
     const float m32 = __double2float_rn(mean_s[threadIdx.x]);
     const float v32 = __double2float_rn(s / BLK);
-    const int64_t row = (static_cast<int64_t>(b) * h_kv + g) * nb + c;
+    const int64_t row = ((static_cast<int64_t>(b) * h_kv + g) * nb + c) * rstride;
     if (mu) mu[row * D + threadIdx.x] = m32;
     if (sig) sig[row * D + threadIdx.x] = v32;
     if (table) {
@@ -120,12 +121,12 @@ template <int D, int BLK>
 __global__ void __launch_bounds__(256) summary_bf16_warp_kernel(const __nv_bfloat16* __restrict__ K,
                                                                  float* __restrict__ mu, float* __restrict__ sig,
                                                                  __nv_bfloat16* __restrict__ table, int n_kv,
-                                                                 int h_kv, int nu, int64_t units) {
+                                                                 int h_kv, int nu, int64_t units, int rstride) {
   constexpr int VPL = D / 32;   // dimensions per lane: 4 (d = 128) or 2 (d = 64)
   constexpr int UNROLL = 16;    // rows loaded before they are summed
   static_assert(BLK % UNROLL == 0, "unit size");
   const int lane = threadIdx.x & 31;
-  const int64_t x = static_cast<int64_t>(blockIdx.x) * 8 + (threadIdx.x >> 5);   // output row
+  int64_t x = static_cast<int64_t>(blockIdx.x) * 8 + (threadIdx.x >> 5);   // unit
   if (x >= units) return;   // warp-uniform
   const int c = static_cast<int>(x % nu);
   const int64_t bg = x / nu;
@@ -171,6 +172,8 @@ __global__ void __launch_bounds__(256) summary_bf16_warp_kernel(const __nv_bfloa
     m32[v] = __double2float_rn(s0[v] / BLK);
     v32[v] = __double2float_rn((s2[v] - s1[v] * s1[v] / BLK) / BLK);
   }
+  const int64_t x_in = x;
+  x = x_in * rstride;   // output row
   if (mu) {
 #pragma unroll
     for (int v = 0; v < VPL; ++v) mu[x * D + lane * VPL + v] = m32[v];
@@ -194,7 +197,7 @@ template <int D, int BLK>
 __global__ void __launch_bounds__(256) summary_full_kernel(const float* __restrict__ K,
                                                            float* __restrict__ mu,
                                                            float* __restrict__ sig,
-                                                           int n_kv, int h_kv, int nb) {
+                                                           int n_kv, int h_kv, int nb, int rstride) {
   extern __shared__ double xs[];   // [BLK][D]
   __shared__ double mean_s[D];
   const int c = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
@@ -213,7 +216,7 @@ __global__ void __launch_bounds__(256) summary_full_kernel(const float* __restri
   __syncthreads();
   for (int e = threadIdx.x; e < BLK * D; e += 256) xs[e] -= mean_s[e % D];
   __syncthreads();
-  const int64_t row = (static_cast<int64_t>(b) * h_kv + g) * nb + c;
+  const int64_t row = ((static_cast<int64_t>(b) * h_kv + g) * nb + c) * rstride;
   if (mu && threadIdx.x < D) mu[row * D + threadIdx.x] = __double2float_rn(mean_s[threadIdx.x]);
   if (sig) {
     for (int e = threadIdx.x; e < D * D; e += 256) {
@@ -223,6 +226,68 @@ __global__ void __launch_bounds__(256) summary_full_kernel(const float* __restri
       sig[row * D * D + e] = __double2float_rn(acc / BLK);
     }
   }
+}
+
+// Outlier rows, a warp per (batch, kv-head, block): the block's key of
+// largest 2-norm — squared norms summed in float64 (exact for bf16 keys;
+// float32 keys' squares are exact too), equal norms to the earlier key —
+// written as summary row 2c + 1: mu = the key, sigma = 0 (d values, or the
+// d x d zero matrix), route table [bf16(key) ; 0].
+template <typename T, int D>
+__global__ void __launch_bounds__(256) outlier_kernel(const T* __restrict__ K, float* __restrict__ mu,
+                                                      float* __restrict__ sig, __nv_bfloat16* __restrict__ table,
+                                                      int n_kv, int h_kv, int nb, int B, int full, int64_t units) {
+  constexpr int VPL = D / 32;
+  const int lane = threadIdx.x & 31;
+  const int64_t x = static_cast<int64_t>(blockIdx.x) * 8 + (threadIdx.x >> 5);
+  if (x >= units) return;   // warp-uniform
+  const int c = static_cast<int>(x % nb);
+  const int64_t bg = x / nb;
+  const int g = static_cast<int>(bg % h_kv), b = static_cast<int>(bg / h_kv);
+  const int64_t row_stride = static_cast<int64_t>(h_kv) * D;
+  const T* base = K + ((static_cast<int64_t>(b) * n_kv + static_cast<int64_t>(c) * B) * h_kv + g) * D + lane * VPL;
+  double best = -1.0;
+  int brow = 0;
+#pragma unroll 4
+  for (int r = 0; r < B; ++r) {
+    double n2 = 0.0;
+#pragma unroll
+    for (int v = 0; v < VPL; ++v) {
+      const double kv = static_cast<double>(static_cast<float>(base[r * row_stride + v]));
+      n2 = fma(kv, kv, n2);
+    }
+#pragma unroll
+    for (int o = 16; o; o >>= 1) n2 += __shfl_xor_sync(0xFFFFFFFFu, n2, o);
+    if (n2 > best) { best = n2; brow = r; }   // the same on every lane
+  }
+  const int64_t row = x * 2 + 1;
+#pragma unroll
+  for (int v = 0; v < VPL; ++v) {
+    const float kv = static_cast<float>(base[brow * row_stride + v]);
+    const int t = lane * VPL + v;
+    if (mu) mu[row * D + t] = kv;
+    if (sig && !full) sig[row * D + t] = 0.f;
+    if (table) {
+      table[row * 2 * D + t] = __float2bfloat16_rn(kv);
+      table[row * 2 * D + D + t] = __float2bfloat16_rn(0.f);
+    }
+  }
+  if (sig && full)
+    for (int e = lane; e < D * D; e += 32) sig[row * D * D + e] = 0.f;
+}
+
+template <typename T, int D>
+cudaError_t run_outlier(const ssa_params& p, const void* K, float* mu, float* sig, void* table,
+                        const LaunchCtx& c) {
+  const int nb = p.n_kv / p.block;
+  const int64_t units = static_cast<int64_t>(p.batch) * p.h_kv * nb;
+  const int64_t grid = (units + 7) / 8;
+  if (grid > 2147483647) return cudaErrorInvalidValue;
+  outlier_kernel<T, D><<<static_cast<unsigned>(grid), 256, 0, c.stream>>>(
+      static_cast<const T*>(K), mu, sig, static_cast<__nv_bfloat16*>(table), p.n_kv, p.h_kv, nb, p.block,
+      p.sigma == SSA_SIGMA_FULL ? 1 : 0, units);
+  note_launch();
+  return cudaGetLastError();
 }
 
 // A launch summarises units of BLK keys: whole blocks, or the sub-blocks of
@@ -238,13 +303,14 @@ cudaError_t run_diag(const ssa_params& p, const void* K, float* mu, float* sig, 
     if (grid > 2147483647) return cudaErrorInvalidValue;
     summary_bf16_warp_kernel<D, BLK><<<static_cast<unsigned>(grid), 256, 0, c.stream>>>(
         reinterpret_cast<const __nv_bfloat16*>(K), mu, sig, static_cast<__nv_bfloat16*>(table), p.n_kv, p.h_kv, nu,
-        units);
+        units, p.outlier ? 2 : 1);
     note_launch();
     return cudaGetLastError();
   } else {   // float32: a CTA per unit
     dim3 grid(nu, p.h_kv, p.batch);
     summary_diag_kernel<T, D, BLK><<<grid, 256, 0, c.stream>>>(
-        static_cast<const T*>(K), mu, sig, static_cast<__nv_bfloat16*>(table), p.n_kv, p.h_kv, nu);
+        static_cast<const T*>(K), mu, sig, static_cast<__nv_bfloat16*>(table), p.n_kv, p.h_kv, nu,
+        p.outlier ? 2 : 1);
     note_launch();
     return cudaGetLastError();
   }
@@ -259,7 +325,7 @@ cudaError_t run_full(const ssa_params& p, const void* K, float* mu, float* sig, 
   if (e != cudaSuccess) return e;
   dim3 grid(nu, p.h_kv, p.batch);
   summary_full_kernel<D, BLK><<<grid, 256, smem, c.stream>>>(static_cast<const float*>(K), mu, sig,
-                                                             p.n_kv, p.h_kv, nu);
+                                                             p.n_kv, p.h_kv, nu, p.outlier ? 2 : 1);
   note_launch();
   return cudaGetLastError();
 }
@@ -283,8 +349,31 @@ cudaError_t diag_u(int unit, const ssa_params& p, const void* K, float* mu, floa
 
 }  // namespace
 
+namespace {
+cudaError_t launch_block_rows(const ssa_params& p, const void* K, float* mu, float* sigma, void* table,
+                              const LaunchCtx& c);
+}  // namespace
+
+// The block (or sub-block) summary rows, then with the outlier channel each
+// block's outlier row after its summary row.
 cudaError_t launch_summary(const ssa_params& p, const void* K, float* mu, float* sigma,
                            void* table, const LaunchCtx& c) {
+  cudaError_t e = launch_block_rows(p, K, mu, sigma, table, c);
+  if (e != cudaSuccess || !p.outlier) return e;
+  if (p.subblocks != 1) return cudaErrorInvalidValue;
+  if (p.dtype == SSA_BF16) {
+    if (p.d == 128) return run_outlier<__nv_bfloat16, 128>(p, K, mu, sigma, table, c);
+    if (p.d == 64) return run_outlier<__nv_bfloat16, 64>(p, K, mu, sigma, table, c);
+  } else {
+    if (p.d == 128) return run_outlier<float, 128>(p, K, mu, sigma, nullptr, c);
+    if (p.d == 64) return run_outlier<float, 64>(p, K, mu, sigma, nullptr, c);
+  }
+  return cudaErrorInvalidValue;
+}
+
+namespace {
+cudaError_t launch_block_rows(const ssa_params& p, const void* K, float* mu, float* sigma, void* table,
+                              const LaunchCtx& c) {
   if (p.subblocks < 1 || p.block % p.subblocks != 0) return cudaErrorInvalidValue;
   const int unit = p.block / p.subblocks;
   if (p.sigma == SSA_SIGMA_FULL) {
@@ -301,5 +390,6 @@ cudaError_t launch_summary(const ssa_params& p, const void* K, float* mu, float*
   }
   return cudaErrorInvalidValue;
 }
+}  // namespace
 
 }  // namespace ssa

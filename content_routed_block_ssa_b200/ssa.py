@@ -33,7 +33,7 @@ class ssa_params(C.Structure):
                 ("h_kv", C.c_int32), ("d", C.c_int32), ("block", C.c_int32), ("topk", C.c_int32),
                 ("window", C.c_int32), ("dtype", C.c_int32), ("sigma", C.c_int32),
                 ("route_impl", C.c_int32), ("q_offset", C.c_int64), ("beta", C.c_float),
-                ("scale", C.c_float), ("subblocks", C.c_int32), ("reserved", C.c_int32)]
+                ("scale", C.c_float), ("subblocks", C.c_int32), ("outlier", C.c_int32)]
 
 
 assert C.sizeof(ssa_params) == 72
@@ -102,13 +102,16 @@ def status_string(s: int) -> str:
 
 
 def make_params(batch, n_q, n_kv, h_q, h_kv, d, block, topk, window, q_offset=0, beta=2.0,
-                scale=None, dtype="bf16", sigma="diag", route_impl=SSA_ROUTE_AUTO, subblocks=1) -> ssa_params:
-    """An ssa_params struct from plain values (dtype 'f32'|'bf16', sigma 'diag'|'full')."""
+                scale=None, dtype="bf16", sigma="diag", route_impl=SSA_ROUTE_AUTO, subblocks=1,
+                outlier=False) -> ssa_params:
+    """An ssa_params struct from plain values (dtype 'f32'|'bf16', sigma 'diag'|'full';
+    outlier: add the outlier-channel row to every block's summaries)."""
     return ssa_params(batch=batch, n_q=n_q, n_kv=n_kv, h_q=h_q, h_kv=h_kv, d=d, block=block, topk=topk,
                       window=window, dtype={"f32": SSA_F32, "bf16": SSA_BF16}.get(dtype, dtype),
                       sigma={"diag": SSA_SIGMA_DIAG, "full": SSA_SIGMA_FULL}.get(sigma, sigma),
                       route_impl=route_impl, q_offset=q_offset, beta=beta,
-                      scale=(1.0 / math.sqrt(d)) if scale is None else scale, subblocks=subblocks, reserved=0)
+                      scale=(1.0 / math.sqrt(d)) if scale is None else scale, subblocks=subblocks,
+                      outlier=1 if outlier else 0)
 
 
 def _ptr(t):
@@ -234,8 +237,9 @@ def ssa_forward_hostio(p, hQ, hK, hV, hO, hlse=None, dev_buf=None, stream=None):
 # ---------------------------------------------------------------- buffers
 
 def summary_shapes(p):
-    """Shapes of mu, Sigma and the route table: one row per sub-block."""
-    rows = (p.n_kv // p.block) * max(p.subblocks, 1)
+    """Shapes of mu, Sigma and the route table: one row per sub-block (and
+    one more per block with the outlier channel)."""
+    rows = (p.n_kv // p.block) * (max(p.subblocks, 1) + (1 if p.outlier else 0))
     mu = (p.batch, p.h_kv, rows, p.d)
     sig = mu + ((p.d,) if p.sigma == SSA_SIGMA_FULL else ())
     tab = (p.batch, p.h_kv, rows, 2 * p.d)

@@ -54,6 +54,7 @@ class Workload:
     beta: float = 2.0
     subblocks: int = 1  # summaries per block (sub-block max-pool routing when > 1)
     cluster_span: int = 1   # consecutive blocks sharing a centroid (clustered keys)
+    outlier: bool = False   # route with the outlier-channel row per block
 
     @property
     def n_q(self) -> int:
@@ -168,4 +169,4 @@ def problem_dict(w: Workload) -> dict:
     return dict(batch=w.batch, n_q=w.n_q, n_kv=w.n, h_q=w.h_q, h_kv=w.h_kv, d=w.d,
                 block=w.block, topk=w.topk, window=w.window, q_offset=w.q_offset,
                 beta=w.beta, scale=1.0 / math.sqrt(w.d), dtype=w.dtype, sigma=w.sigma,
-                subblocks=w.subblocks)
+                subblocks=w.subblocks, outlier=w.outlier)

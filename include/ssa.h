@@ -111,7 +111,7 @@ typedef struct {
   float beta;         /* routing inverse temperature                      */
   float scale;        /* attention logit scale (normally 1/sqrt(d))        */
   int32_t subblocks;  /* S in {1, 2, 4}: summaries per block (see below)  */
-  int32_t reserved;   /* must be 0                                        */
+  int32_t outlier;    /* 1: outlier-channel row per block (see below); 0  */
 } ssa_params;
 
 /*
@@ -125,6 +125,17 @@ typedef struct {
  * (SSA)", artifact list: sub-block max-pool).  Selection, the window and the
  * attention still work on whole blocks.  Summary outputs then have nb * S
  * rows per (batch, kv-head), sub-block s of block c at row c * S + s.
+ *
+ * Outlier channel (outlier = 1, with subblocks = 1): the same page names an
+ * outlier channel beside the sub-block max-pool, without a rule.  Here every
+ * block gets a second summary row: its key of largest 2-norm k*_c (squared
+ * norms in float64, equal norms to the earlier key) with a zero covariance,
+ * so the row's score is the exact group logit sum_h <q_h, k*_c>; a block
+ * scores the larger of its two rows.  Summary outputs then have 2 nb rows
+ * per (batch, kv-head): row 2c the block's (mu, Sigma), row 2c + 1 the
+ * outlier key (sigma rows zero; route_table row [k*_c ; 0]).  outlier = 1
+ * with subblocks > 1 is SSA_ERR_UNSUPPORTED; any value other than 0 or 1 is
+ * SSA_ERR_INVALID_ARG.
  */
 
 /* Human-readable name of a status code (static string, never NULL). */
@@ -327,7 +338,7 @@ SSA_API ssa_status ssa_forward_hostio(const ssa_params* p, const void* hQ, const
  *   visible blocks (by ssa_route_topk's kernels), so block_idx is
  *   ssa_route_topk's selection for every row.
  *
- * bf16 problems with a diagonal Sigma, subblocks = 1 and d in {64, 128}
+ * bf16 problems with a diagonal Sigma, subblocks = 1, outlier = 0 and d in {64, 128}
  * (else SSA_ERR_UNSUPPORTED).
  */
 typedef struct {
@@ -342,7 +353,7 @@ typedef struct {
  * ssa_params checks of the other calls; hp NULL, reserved != 0, fanout not a
  * power of two in 1..64, probe outside 1..31 or escalate not 0/1 ->
  * SSA_ERR_INVALID_ARG; (probe + 1) * fanout > 512 (the probe's candidate
- * capacity), a float32 problem or subblocks != 1 -> SSA_ERR_UNSUPPORTED;
+ * capacity), a float32 problem, subblocks != 1 or outlier != 0 -> SSA_ERR_UNSUPPORTED;
  * NULL or misaligned (not 16-byte) pointers -> SSA_ERR_INVALID_ARG; a
  * workspace smaller than ssa_route_hier_workspace_size ->
  * SSA_ERR_WORKSPACE.  ssa_route_hier returns SSA_OK without a launch when

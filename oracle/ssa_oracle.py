@@ -41,7 +41,12 @@ the repository's design notes):
   * grouped-query attention: one selection per (token, kv-head), ranked by
     the sum over the group's query heads of r_c(q_h);
   * bf16 problems route on bf16 features and bf16 summaries whose rounding
-    is part of the definition (``route_features`` / ``stored_summaries``).
+    is part of the definition (``route_features`` / ``stored_summaries``);
+  * the cascade's outlier channel (named on the same page, artifact list,
+    without a rule): each block gets one more summary row, its key of
+    largest 2-norm with a zero covariance, so the row scores that key's
+    exact group logit; a block scores the larger of its two rows
+    (``outlier_keys`` / ``with_outlier_rows``).
 
 Parity status: every function here is pinned by ``tests/test_oracle_pins.py``
 (closed forms, brute force, invariants and hand-computed golden cases).
@@ -77,6 +82,7 @@ class Problem:
     dtype: str = BF16
     sigma: str = DIAG
     subblocks: int = 1          # sub-block summaries per block (max-pooled routing)
+    outlier: bool = False       # one more summary row per block: its largest-norm key
 
     def __post_init__(self):
         if not math.isfinite(self.scale):
@@ -94,6 +100,11 @@ class Problem:
     def unit(self) -> int:
         """Keys per summary: the block, or its sub-block when subblocks > 1."""
         return self.block // self.subblocks
+
+    @property
+    def rows_per_block(self) -> int:
+        """Summary rows per block: the S sub-blocks, plus the outlier row."""
+        return self.subblocks + (1 if self.outlier else 0)
 
 
 # ---------------------------------------------------------------- rounding
@@ -131,6 +142,8 @@ def block_summaries(K: np.ndarray, p: Problem):
       sig [batch, h_kv, nb, d, d]    full:     (1/B) sum_j (k_j - mu_c)(k_j - mu_c)^T
     With p.subblocks = S > 1 the summaries are taken per sub-block of B/S
     consecutive keys instead (nb * S rows, sub-block s of block c at c*S + s).
+    With p.outlier each block gets a second row, its largest-norm key with a
+    zero covariance (row 2c+1; see with_outlier_rows).
     """
     b, n, h, d = K.shape
     B = p.unit
@@ -142,7 +155,37 @@ def block_summaries(K: np.ndarray, p: Problem):
         sig = np.einsum("xhcjs,xhcjt->xhcst", dev, dev) / B
     else:
         sig = (dev * dev).sum(axis=3) / B
+    if p.outlier:
+        mu, sig = with_outlier_rows(K, mu, sig, p)
     return mu, sig
+
+
+def outlier_keys(K: np.ndarray, p: Problem) -> np.ndarray:
+    """The outlier channel's key of every block: the key of largest 2-norm
+    (squared norms in float64; equal norms go to the earlier key).
+    Returns [batch, h_kv, nb, d] float64."""
+    b, n, h, d = K.shape
+    nb = n // p.block
+    Kb = np.asarray(K, dtype=np.float64).reshape(b, nb, p.block, h, d).transpose(0, 3, 1, 2, 4)
+    norm2 = (Kb * Kb).sum(axis=-1)                       # [b, h, nb, B]
+    j = np.argmax(norm2, axis=-1)                        # first of equal maxima
+    return np.take_along_axis(Kb, j[..., None, None], axis=3)[:, :, :, 0, :]
+
+
+def with_outlier_rows(K: np.ndarray, mu: np.ndarray, sig: np.ndarray, p: Problem):
+    """Interleaves the outlier rows after each block's summary row: row 2c is
+    block c's (mean, covariance), row 2c+1 its largest-norm key k*_c with a
+    zero covariance, so that the row's score is the group logit of k*_c
+    (sub-block summaries are not combined with the outlier row)."""
+    if p.subblocks != 1:
+        raise ValueError("the outlier row is defined for whole-block summaries")
+    ko = outlier_keys(K, p)
+    b, h, nb, d = mu.shape
+    mu2 = np.empty((b, h, 2 * nb, d))
+    mu2[:, :, 0::2], mu2[:, :, 1::2] = mu, ko
+    sig2 = np.zeros((b, h, 2 * nb) + sig.shape[3:])
+    sig2[:, :, 0::2] = sig
+    return mu2, sig2
 
 
 def stored_summaries(mu: np.ndarray, sig: np.ndarray, p: Problem):
@@ -197,9 +240,10 @@ def visible_blocks(pos: int, p: Problem) -> int:
 # ---------------------------------------------------------------- step 2 (scores)
 
 def pool_subblocks(scores: np.ndarray, p: Problem) -> np.ndarray:
-    """Block scores from sub-block scores (last axis nb * S): the maximum
-    over each block's S sub-blocks (identity for S = 1)."""
-    S = p.subblocks
+    """Block scores from summary-row scores (last axis nb * R, R rows per
+    block: the S sub-blocks and the outlier row): the maximum over each
+    block's rows (identity for R = 1)."""
+    S = p.rows_per_block
     if S == 1:
         return scores
     sh = scores.shape
@@ -217,7 +261,7 @@ def route_scores_row(Q: np.ndarray, stored, p: Problem, bi: int, i: int, g: int)
     """
     mu32, sig32, table = stored
     nv = visible_blocks(p.q_offset + i, p)
-    nu = nv * p.subblocks                      # visible summary rows
+    nu = nv * p.rows_per_block                 # visible summary rows
     if p.dtype == BF16:
         f = route_features(Q[bi:bi + 1, i:i + 1], p)[0, g, 0]
         return pool_subblocks(table[bi, g, :nu] @ f, p)
@@ -540,7 +584,7 @@ def hier_route(Q: np.ndarray, stored, p: Problem, fanout: int, probe: int, escal
     escalate: uncertified rows take the flat top-k of all visible blocks.
     rows: optional (batch, query row) pairs; other rows stay -2 / False.
     """
-    if p.dtype != BF16 or p.subblocks != 1:
+    if p.dtype != BF16 or p.subblocks != 1 or p.outlier:
         raise ValueError("the hierarchical router is defined on the bf16 routing table, S = 1")
     _mu32, _sig32, table = stored
     nodes = hier_nodes(table, fanout)

@@ -79,6 +79,19 @@ CASES = {
                                         beta=3.0),
     "f32_full_d64_beta3": Workload("c", 131, 1, 768, 2, 1, 64, "f32", 64, "full", 4, 64, 2, "total", beta=3.0),
     "f32_diag_d128_beta0": Workload("c", 132, 1, 512, 4, 2, 128, "f32", 64, "diag", 4, 64, 2, "total", beta=0.0),
+    # the outlier channel: a second summary row per block (its largest-norm
+    # key, zero covariance), max-pooled with the block's cumulant score, on
+    # the tiled and row-wise bf16 routers and the float32 routers
+    "bf16_gqa4_d128_b64_outlier": Workload("c", 133, 1, 1536, 8, 2, 128, "bf16", 64, "diag", 8, 256, 6, "total",
+                                           clustered=True, outlier=True),
+    "bf16_gqa8_d128_b128_outlier": Workload("c", 134, 1, 2048, 8, 1, 128, "bf16", 128, "diag", 8, 256, 6,
+                                            "total", outlier=True),
+    "bf16_mha_d64_b64_outlier_beta0": Workload("c", 135, 1, 1024, 2, 2, 64, "bf16", 64, "diag", 4, 64, 4,
+                                               "per_head", outlier=True, beta=0.0),
+    "f32_diag_d128_outlier": Workload("c", 136, 1, 512, 4, 2, 128, "f32", 64, "diag", 4, 64, 2, "total",
+                                      outlier=True),
+    "f32_full_d64_outlier": Workload("c", 137, 1, 768, 2, 1, 64, "f32", 64, "full", 4, 64, 2, "total",
+                                     outlier=True),
     # float32 routing takes runs of 32 (query, head) pairs per CTA unless a
     # row's 1024 block scores do not fit beside them: then one CTA per row
     "f32_diag_d64_decode_64k": Workload("c", 122, 1, 65536, 1, 1, 64, "f32", 64, "diag", 8, 64, 2, "per_seq",
@@ -203,6 +216,33 @@ def test_bf16_features_read_back_equal_golden_rounding(impl):
     last = n - 1                                # the one row that sees all nb blocks
     assert idx[0, last, 0].tolist() == list(range(nb))
     assert sc[0, last, 0].double().cpu().tolist() == g["features"]
+
+
+@pytest.mark.parametrize("impl", [ssa.SSA_ROUTE_TILED, ssa.SSA_ROUTE_ROWWISE], ids=["tiled", "rowwise"])
+def test_route_all_blocks_equal_takes_the_first_k(impl):
+    """Every block holds the same keys, so every visible block scores the
+    same: the selection is the k lowest visible blocks.  With the tile
+    router's seeds the seed bound equals the k-th best score exactly here,
+    so this also checks that a block scoring exactly the bound is kept."""
+    B, n, k = 64, 64 * 96, 16
+    blk = torch.randn(B, 2, 128, generator=torch.Generator().manual_seed(9)).to(torch.bfloat16)
+    K = blk.repeat(n // B, 1, 1).unsqueeze(0).contiguous()
+    Q = torch.randn(1, n, 8, 128, generator=torch.Generator().manual_seed(10)).to(torch.bfloat16)
+    p = ssa.make_params(batch=1, n_q=n, n_kv=n, h_q=8, h_kv=2, d=128, block=B, topk=k, window=B,
+                        route_impl=impl)
+    (Qd, Kd) = to_dev(Q, K)
+    _, _, tab = gpu_summary(p, Kd)
+    assert torch.equal(tab[0, :, :1].expand_as(tab[0]), tab[0])   # identical rows
+    idx, sc = gpu_route(p, Qd, None, None, tab)
+    check_no_device_error()
+    gi = idx.cpu().numpy()
+    for i in (63, 64 * 16 - 1, 64 * 40, n - 1):
+        nv = min(n // B, (i + 1) // B)
+        want = list(range(min(k, nv))) + [-1] * (k - min(k, nv))
+        for g in range(2):
+            assert gi[0, i, g].tolist() == want, (i, g)
+            s = sc[0, i, g, :min(k, nv)].cpu()
+            assert torch.all(s == s[0])
 
 
 @pytest.mark.parametrize("name", list(CASES))

@@ -794,3 +794,86 @@ def test_hier_bound_constants_are_the_largest_radius_and_row_norm():
     # kv-head 0: every block row has norm 4, every node row (cap 4 in all four
     # dimensions) norm 8
     assert t_star[0, 0] == 8.0
+
+
+# ------------------------------------------------------------------ outlier channel
+
+def test_outlier_channel_golden_block():
+    """Hand case (tests/golden/outlier_channel.json): cumulant routing ranks
+    the block of four moderate keys first; the outlier row (the largest-norm
+    key, zero covariance) recovers the block holding the largest logit.
+    Checked through both the float32 and the bf16 routing rows."""
+    g = golden("outlier_channel.json")
+    K = np.asarray(g["keys"], dtype=np.float64)[None, :, None, :]      # [1, 8, 1, 2]
+    q = np.asarray(g["q"], dtype=np.float64)
+    for dtype in (O.F32, O.BF16):
+        kw = dict(batch=1, n_q=8, n_kv=8, h_q=1, h_kv=1, d=2, block=4, topk=1, window=1,
+                  dtype=dtype, sigma=O.DIAG, beta=g["beta"])
+        base = O.Problem(**kw)
+        out = O.Problem(**kw, outlier=True)
+        mu, sig = O.block_summaries(K, base)
+        np.testing.assert_array_equal(mu[0, 0], g["mu"])
+        np.testing.assert_array_equal(sig[0, 0], g["var"])
+        mu2, sig2 = O.block_summaries(K, out)
+        np.testing.assert_array_equal(mu2[0, 0, 1::2], g["outlier_key"])
+        np.testing.assert_array_equal(sig2[0, 0, 1::2], np.zeros((2, 2)))
+        Q = np.zeros((1, 8, 1, 2))
+        Q[0, 7, 0] = q
+        s0 = O.route_scores_row(Q, O.stored_summaries(mu, sig, base), base, 0, 7, 0)
+        s1 = O.route_scores_row(Q, O.stored_summaries(mu2, sig2, out), out, 0, 7, 0)
+        np.testing.assert_array_equal(s0, g["r_cumulant"])
+        np.testing.assert_array_equal(s1, g["r_pooled"])
+        assert O.select_topk(s0, 1)[0][0] == g["top1_cumulant"]
+        assert O.select_topk(s1, 1)[0][0] == g["top1_with_outlier"]
+
+
+def test_outlier_keys_brute_force_with_ties():
+    """The outlier key is the first key of largest squared norm, by a direct
+    scan; small integer keys make equal norms common."""
+    rng = np.random.default_rng(21)
+    p = O.Problem(batch=2, n_q=32, n_kv=32, h_q=2, h_kv=2, d=3, block=8, topk=2, window=8,
+                  dtype=O.F32, sigma=O.FULL, outlier=True)
+    for _ in range(20):
+        K = rng.integers(-2, 3, size=(2, 32, 2, 3)).astype(np.float64)
+        ko = O.outlier_keys(K, p)
+        for b in range(2):
+            for h in range(2):
+                for c in range(4):
+                    best, arg = -1.0, None
+                    for j in range(8):
+                        k = K[b, c * 8 + j, h]
+                        n2 = float(k @ k)
+                        if n2 > best:
+                            best, arg = n2, k
+                    np.testing.assert_array_equal(ko[b, h, c], arg)
+        # the full-Sigma rows of the outlier channel are zero matrices, and the
+        # block rows are the plain block summaries
+        mu2, sig2 = O.block_summaries(K, p)
+        mu1, sig1 = O.block_summaries(K, O.Problem(**{**p.__dict__, "outlier": False}))
+        np.testing.assert_array_equal(mu2[:, :, 0::2], mu1)
+        np.testing.assert_array_equal(sig2[:, :, 0::2], sig1)
+        assert not sig2[:, :, 1::2].any()
+
+
+def test_outlier_score_is_the_exact_group_logit_of_the_max_norm_key():
+    """A block's outlier-row score equals sum_h q_h . k*_c computed directly
+    from the keys, and the pooled score is the larger of it and the
+    cumulant score."""
+    rng = np.random.default_rng(22)
+    p = O.Problem(batch=1, n_q=64, n_kv=64, h_q=4, h_kv=2, d=8, block=16, topk=2, window=16,
+                  dtype=O.F32, sigma=O.DIAG, beta=2.0, outlier=True)
+    K = rng.standard_normal((1, 64, 2, 8))
+    Q = rng.standard_normal((1, 64, 4, 8))
+    stored = O.stored_summaries(*O.block_summaries(K, p), p)
+    base = O.Problem(**{**p.__dict__, "outlier": False})
+    stored0 = O.stored_summaries(*O.block_summaries(K, base), base)
+    for g in range(2):
+        s = O.route_scores_row(Q, stored, p, 0, 63, g)
+        s0 = O.route_scores_row(Q, stored0, base, 0, 63, g)
+        for c in range(4):
+            Kc = K[0, c * 16:(c + 1) * 16, g]
+            ks = O.round_f32(Kc[np.argmax((Kc * Kc).sum(axis=1))])
+            logit = sum(O.round_f32(Q[0, 63, h]) @ ks for h in (2 * g, 2 * g + 1))
+            assert abs(s[c] - max(s0[c], logit)) <= 1e-12 * max(1.0, abs(s[c]))
+    with pytest.raises(ValueError):
+        O.block_summaries(K, O.Problem(**{**p.__dict__, "subblocks": 2}))
