@@ -46,37 +46,43 @@ __device__ __forceinline__ int lane_hot_id(const BlockPlan& pl, const SlotSet& s
   return ((s.mask >> lane) & 1) ? __ldg(pl.hot_id + static_cast<int64_t>(bg) * pl.nb + s.v) : -1;
 }
 
-// keyed = false: counts per key block (the first pass in pair mode, the only
-// one otherwise) and each row's uncovered window blocks; chist columns are
-// blocks.  keyed = true (pair mode): counts per tile key; columns are keys.
-template <bool KEYED>
+// Counting passes over the rows of one chunk.  MODE 0: counts per key block
+// and each row's uncovered window blocks (the only pass without pairs).
+// MODE 1 (pair mode, first pass): counts per key block over every
+// kHotSample-th row only — they choose the hot set, and any hot set gives
+// the same attention.  MODE 2 (pair mode): counts per tile key and the
+// window blocks, every row.  chist columns: blocks (0, 1) or keys (2).
+constexpr int kHotSample = 8;
+
+template <int MODE>
 __global__ void __launch_bounds__(kPlanThreads) inv_hist_kernel(const BlockPlan pl, const int32_t* __restrict__ idx) {
   extern __shared__ int32_t hist[];
-  const int ncol = KEYED ? pl.nkey : pl.nb;
+  const int ncol = MODE == 2 ? pl.nkey : pl.nb;
+  const int step = MODE == 1 ? kHotSample : 1;
   const int k = blockIdx.x, bg = blockIdx.y;
   for (int c = threadIdx.x; c < ncol; c += blockDim.x) hist[c] = 0;
   __syncthreads();
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
   const int b = bg / pl.h_kv, g = bg % pl.h_kv;
   const int r1 = min((k + 1) * kPlanRows, pl.n_q);
-  for (int i = k * kPlanRows + warp; i < r1; i += nw) {
+  for (int i = k * kPlanRows + warp * step; i < r1; i += nw * step) {
     const int v = lane < pl.topk ? __ldg(idx + ((static_cast<int64_t>(b) * pl.n_q + i) * pl.h_kv + g) * pl.topk + lane) : -1;
     const SlotSet s = row_slots(v, pl.topk, pl.q_offset + i, pl.nb, pl.block, pl.window);
-    if (KEYED) {
+    if (MODE == 2) {
       const PairSlot ps = pair_slots(s, lane_hot_id(pl, s, bg), pl.nb);
       if (ps.emit) atomicAdd(&hist[ps.key], 1);
     } else {
       if ((s.mask >> lane) & 1) atomicAdd(&hist[s.v], 1);
-      if (lane == 0) pl.win[static_cast<int64_t>(bg) * pl.n_q + i] = s.win;
     }
+    if (MODE != 1 && lane == 0) pl.win[static_cast<int64_t>(bg) * pl.n_q + i] = s.win;
   }
   __syncthreads();
   int32_t* out = pl.chist + (static_cast<int64_t>(bg) * pl.nchunk + k) * ncol;
   for (int c = threadIdx.x; c < ncol; c += blockDim.x) out[c] = hist[c];
 }
 
-// One CTA per (batch, kv-head), pair mode: each block's selections summed
-// over the chunks of the first pass; the hot set is the largest set
+// One CTA per (batch, kv-head), pair mode: each block's (sampled) selections
+// summed over the chunks of the first pass; the hot set is the largest set
 // {c : count_c >= T} (T >= 2) of at most kHotBlocks blocks, numbered in
 // block order.
 __global__ void __launch_bounds__(1024) inv_hot_kernel(const BlockPlan pl) {
@@ -277,9 +283,10 @@ __global__ void __launch_bounds__(256) inv_tiles_kernel(const BlockPlan pl) {
     if (c < pl.nb) {
       y = pair_tile_y(c, -1);
     } else {
-      const int hh = c - pl.nb;
+      int h1, h2;
+      pair_of_index(c - pl.nb, h1, h2);
       const int32_t* hb = pl.hot_blk + static_cast<int64_t>(bg) * kHotBlocks;
-      y = pair_tile_y(hb[hh / kHotBlocks], hb[hh % kHotBlocks]);
+      y = pair_tile_y(hb[h1], hb[h2]);
     }
   }
   const int e0 = pl.ent_base[bg] + pl.blk_off[x];
@@ -396,7 +403,7 @@ struct BlkCfg {
   // Q tile buffers: with G = 8 one warp fills them all by TMA; otherwise one
   // cp.async warp per buffer
   static constexpr bool TMA_Q = (G == 8);
-  static constexpr int NA = (BLK == 64) ? 4 : (TMA_Q ? 3 : 2);
+  static constexpr int NA = (BLK == 128 && TMA_Q) ? 3 : 4;
   static constexpr int NGW = TMA_Q ? 1 : NA;            // gather warps
   static constexpr int KV_HALF = BLK * ROW;             // BLK keys x 64 dims
   static constexpr int KV_BYTES = 4 * KV_HALF;          // K lo, K hi, V lo, V hi
@@ -407,7 +414,10 @@ struct BlkCfg {
   // spare TMEM columns with 64-key blocks, else in shared memory
   static constexpr bool ML_TMEM = (BLK == 64);
   static constexpr int ML_BYTES = ML_TMEM ? 0 : 2 * 128 * 8;
-  static constexpr int SMEM = 1024 + NA * A_BYTES + NKV * KV_BYTES + 2 * STG_BYTES + ML_BYTES + NBAR * 8 + 16;
+  static constexpr int USED = NA * A_BYTES + NKV * KV_BYTES + 2 * STG_BYTES + ML_BYTES + NBAR * 8 + 16;
+  // room to align the base to 1024 bytes, up to the 227 KB limit (the
+  // kernel checks that the aligned layout fits)
+  static constexpr int SMEM = USED + 1024 < 232448 ? USED + 1024 : 232448;
   static constexpr int SW0 = 2 + NGW;                   // first softmax warp
   static constexpr int THREADS = 32 * (SW0 + 8);        // KV, MMA, gather, 2 x 4 softmax warps
   // registers per thread: a sub-partition (SMSP) holds ceil(warps / 4) warps
@@ -417,7 +427,7 @@ struct BlkCfg {
   static constexpr int O_COL = 2 * BLK;                 // columns of its S), O[2], (m, l)[2]
   static constexpr int ML_COL = O_COL + 2 * 128;
   static_assert(!ML_TMEM || ML_COL + 4 <= 512, "tensor memory");
-  static_assert(SMEM <= 232448, "shared memory");
+  static_assert(USED <= 232448, "shared memory");
 };
 
 struct BlkArgs {
@@ -492,8 +502,12 @@ __global__ void __maxnreg__((BlkCfg<G, BLK>::MAXREG))
   constexpr int D = C::D;
   constexpr int QPT = 128 / G;
   constexpr int NA = C::NA;
-  extern __shared__ uint8_t smem_raw[];
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  if (static_cast<int>(smem - smem_raw) + C::USED > C::SMEM) {   // never with a 1024-aligned base
+    if (threadIdx.x == 0) atomicCAS(a.err, 0u, static_cast<uint32_t>(SITE_BLK_SMEM));
+    return;
+  }
   uint8_t* sA = smem;                                   // [NA][A_BYTES]
   uint8_t* sKV = sA + NA * C::A_BYTES;                  // [NKV][KV_BYTES]
   uint8_t* sStg = sKV + C::NKV * C::KV_BYTES;           // [2][STG_BYTES] epilogue staging
@@ -1147,9 +1161,11 @@ cudaError_t launch_block_plan(const ssa_params& p, const int32_t* block_idx, con
                               const LaunchCtx& c) {
   const int blk_smem = pl.nb * static_cast<int>(sizeof(int32_t));
   const int key_smem = pl.nkey * static_cast<int>(sizeof(int32_t));
-  cudaError_t e = cudaFuncSetAttribute(inv_hist_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, blk_smem);
+  cudaError_t e = cudaFuncSetAttribute(inv_hist_kernel<0>, cudaFuncAttributeMaxDynamicSharedMemorySize, blk_smem);
   if (e == cudaSuccess)
-    e = cudaFuncSetAttribute(inv_hist_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, key_smem);
+    e = cudaFuncSetAttribute(inv_hist_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, blk_smem);
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(inv_hist_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, key_smem);
   if (e == cudaSuccess)
     e = cudaFuncSetAttribute(inv_hot_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, blk_smem);
   if (e == cudaSuccess)
@@ -1157,14 +1173,17 @@ cudaError_t launch_block_plan(const ssa_params& p, const int32_t* block_idx, con
   if (e != cudaSuccess) return e;
   const dim3 rows(static_cast<unsigned>(pl.nchunk), static_cast<unsigned>(pl.bgs));
   const unsigned cols = static_cast<unsigned>((static_cast<int64_t>(pl.bgs) * pl.nkey + 255) / 256);
-  // per-block counts and window blocks; in pair mode then the hot sets and
-  // the counts per tile key
-  inv_hist_kernel<false><<<rows, kPlanThreads, blk_smem, c.stream>>>(pl, block_idx);
-  note_launch();
+  // per-block counts and window blocks; in pair mode sampled per-block
+  // counts, the hot sets, then the counts per tile key and window blocks
   if (pl.pair) {
+    inv_hist_kernel<1><<<rows, kPlanThreads, blk_smem, c.stream>>>(pl, block_idx);
+    note_launch();
     inv_hot_kernel<<<pl.bgs, 1024, blk_smem, c.stream>>>(pl);
     note_launch();
-    inv_hist_kernel<true><<<rows, kPlanThreads, key_smem, c.stream>>>(pl, block_idx);
+    inv_hist_kernel<2><<<rows, kPlanThreads, key_smem, c.stream>>>(pl, block_idx);
+    note_launch();
+  } else {
+    inv_hist_kernel<0><<<rows, kPlanThreads, blk_smem, c.stream>>>(pl, block_idx);
     note_launch();
   }
   inv_colscan_kernel<<<cols, 256, 0, c.stream>>>(pl);

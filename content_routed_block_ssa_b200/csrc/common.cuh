@@ -32,6 +32,7 @@ enum WaitSite : uint32_t {
   SITE_BLK_ML_EMPTY = 0x423,   // softmax: the epilogue two tiles back has not read (m, l)
   SITE_BLK_MMA_STALL = 0x416,  // the MMA issuer saw no progress
   SITE_BLK_BAD_ENTRY = 0x431,  // an entry outside the query rows (inconsistent plan)
+  SITE_BLK_SMEM = 0x432,       // the aligned shared-memory layout did not fit its allocation
   SITE_WIN_PRODUCER = 0x501,   // sliding-window tiles
   SITE_WIN_MMA = 0x502,
   SITE_WIN_SOFTMAX = 0x503,

@@ -93,8 +93,22 @@ __device__ __forceinline__ SlotSet row_slots(int v_in, int topk, int64_t pos, in
 // last hot one when their number is odd) is a single slot of its block's 64
 // keys.  Slots are numbered pairs first, then singles, both in block order.
 // Tiles are keyed per (batch, kv-head): single block c -> key c; pair of hot
-// numbers (h1, h2) -> key nb + h1 * kHotBlocks + h2.
+// numbers h1 < h2 -> key nb + pair_index(h1, h2), the pairs numbered row by
+// row of the upper triangle.
 constexpr int kHotBlocks = 128;
+constexpr int kPairKeys = kHotBlocks * (kHotBlocks - 1) / 2;
+
+__host__ __device__ constexpr int pair_index(int h1, int h2) {
+  return h1 * (2 * kHotBlocks - h1 - 1) / 2 + (h2 - h1 - 1);
+}
+
+// Inverse of pair_index: the pair of pair number t (0 <= t < kPairKeys).
+__host__ __device__ inline void pair_of_index(int t, int& h1, int& h2) {
+  int a = 0;
+  while (pair_index(a + 1, a + 2) <= t) ++a;   // first pair of row a+1 is past t
+  h1 = a;
+  h2 = t - pair_index(a, a + 1) + a + 1;
+}
 
 struct PairSlot {
   bool emit;       // this lane's entry starts a slot
@@ -125,7 +139,7 @@ __device__ __forceinline__ PairSlot pair_slots(const SlotSet& s, int hid, int nb
   o.nsel = __popc(used_m) - npair;
   if (paired) {
     o.emit = (r & 1) == 0;
-    o.key = nb + hid * kHotBlocks + hid2;
+    o.key = nb + pair_index(hid, hid2);
     o.slot = r >> 1;
   } else {
     o.emit = used;

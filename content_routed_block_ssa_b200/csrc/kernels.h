@@ -84,7 +84,7 @@ inline int rows_per_block(const ssa_params& p) { return p.subblocks + (p.outlier
 struct BlockPlan {
   int32_t bgs, n_q, h_kv, nb, block, topk, window, qpt, nchunk;
   // paired slots (64-key blocks): tile keys are single blocks (0 .. nb-1)
-  // and pairs of hot blocks (nb + h1 * kHotBlocks + h2); otherwise the key
+  // and pairs of hot blocks (nb + pair_index(h1, h2)); otherwise the key
   // is the block and nkey = nb
   int32_t pair, nkey;
   int32_t* hot_id;     // [bgs][nb] hot number of each block, -1 when not hot (pair mode)

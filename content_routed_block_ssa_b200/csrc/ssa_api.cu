@@ -191,7 +191,7 @@ AttnLayout attn_layout(const ssa_params& p) {
   L.nsl = p.topk + ssa::window_chunks(p.window, p.h_q / p.h_kv);
   const size_t items = bgs * p.n_q;
   const size_t sel = items * L.nsl;                       // entries, at most
-  const size_t nkey = nb + (pair_mode(p) ? static_cast<size_t>(ssa::kHotBlocks) * ssa::kHotBlocks : 0);
+  const size_t nkey = nb + (pair_mode(p) ? static_cast<size_t>(ssa::kPairKeys) : 0);
   L.nkey = static_cast<int>(nkey);
   const size_t max_tiles = (sel + qpt - 1) / qpt + bgs * nkey;
   size_t off = 0;

@@ -34,8 +34,9 @@ def test_attended_keys_is_the_key_set_size():
 
 def _direct_slots(arr, w, p):
     """The slot rule written out row by row: used entries; with 64-key blocks
-    the hot blocks of each kv-head (count >= the smallest T >= 2 that leaves
-    at most 128 of them) are paired two at a time in block order."""
+    the hot blocks of each kv-head (count over every 8th row >= the smallest
+    T >= 2 that leaves at most 128 of them) are paired two at a time in
+    block order."""
     from collections import Counter
     used_rows = {}
     cnt = Counter()
@@ -49,10 +50,11 @@ def _direct_slots(arr, w, p):
                 if 0 <= v < nvis:
                     last = max(last, int(v))
             used_rows[(i, g)] = used
-            cnt.update((g, c) for c in used)
+            if i % 8 == 0:
+                cnt.update((g, c) for c in used)
     n_e = sum(len(u) for u in used_rows.values())
     if w.block != 64:
-        return n_e, n_e, len(cnt)
+        return n_e, n_e, len({(g, c) for (i, g), u in used_rows.items() for c in u})
     hot = {}
     for g in range(w.h_kv):
         counts = [cnt[(g, c)] for c in range(w.n // w.block)]
