@@ -202,19 +202,20 @@ def attended_keys(idx, w):
     return n_sel * B + wcount - overlap
 
 
-HOT_BLOCKS = 128   # hot set size of the paired slots (64-key blocks)
+HOT_BLOCKS = 128   # hot set size of the paired slots
+HOT_SAMPLE = 8     # the hot set is counted over every 8th query row
 
 
 def block_major_counts(idx, w):
     """Selected slots of the block-major attention, by the kernels' rules
     (bookkeeping for the roofline, not part of the layer).  A row's used
     entries are its in-range block_idx entries larger than every earlier
-    in-range entry.  With 64-key blocks the entries of each (batch, kv-head)'s
-    hot blocks (its at most HOT_BLOCKS most selected blocks: count >= T for
-    the smallest T >= 2 that keeps the set that small) pair up in block
-    order, two per slot; other entries are a slot each.  Returns (used
-    entries, slots, distinct tile keys: blocks, or pairs and single
-    blocks)."""
+    in-range entry.  The entries of each (batch, kv-head)'s hot blocks (its
+    at most HOT_BLOCKS most selected blocks, counted over every
+    HOT_SAMPLE-th query row: count >= T for the smallest T >= 2 that keeps
+    the set that small) pair up in block order, two per slot; other entries
+    are a slot each.  Returns (used entries, slots, distinct tile keys: pairs
+    and single blocks)."""
     nb = w.n // w.block
     B = w.block
     pos = torch.arange(w.n_q, device=idx.device, dtype=torch.int64).view(1, -1, 1, 1) + w.q_offset
@@ -229,10 +230,10 @@ def block_major_counts(idx, w):
     bgi = (torch.arange(w.batch, device=idx.device).view(-1, 1, 1, 1) * w.h_kv
            + torch.arange(w.h_kv, device=idx.device).view(1, 1, -1, 1)).expand_as(v)
     gkey = bgi * nb + sel
-    if w.block != 64:
-        return n_entries, n_entries, int(torch.unique(gkey[valid]).numel())
     bgs = w.batch * w.h_kv
-    cnt = torch.bincount(gkey[valid], minlength=bgs * nb).view(bgs, nb)
+    rows = torch.arange(w.n_q, device=idx.device).view(1, -1, 1, 1)
+    sampled = valid & (rows % HOT_SAMPLE == 0)
+    cnt = torch.bincount(gkey[sampled], minlength=bgs * nb).view(bgs, nb)
     srt = cnt.sort(dim=1, descending=True).values
     c129 = srt[:, HOT_BLOCKS] if nb > HOT_BLOCKS else torch.zeros(bgs, dtype=cnt.dtype, device=cnt.device)
     T = torch.clamp(c129 + 1, min=2)
@@ -291,20 +292,20 @@ def algorithmic_work(w, idx):
         # rows and writes G partial rows; it reads the window's K, V once.
         # The merge reads all slot partials and writes O and lse per row.
         # (method flops count the keys the row attends, 4 G B d per used
-        # entry; the design's bytes follow its slots: one per entry, or per
-        # pair of hot entries with 64-key blocks, each a 128-key tile)
+        # entry; the design's bytes follow its slots: one per pair of hot
+        # entries or per other entry, each a tile of twice the block's keys)
         ne, nsl, nkeys = block_major_counts(idx, w)
         items = w.batch * w.n_q * w.h_kv
         nwc = (w.window + 255) // 256
         nwin = items * nwc
         wkeys = float(np.minimum(w.window, pos + 1).sum()) * w.batch * w.h_kv
-        tile_keys = 128 if w.block == 64 else w.block
+        tile_keys = 2 * w.block
         out["blocks_bytes"] = nsl * G * (w.d * 2 * 2 + 8) + nkeys * 2 * tile_keys * w.d * 2
         out["blocks_flops"] = 4.0 * ne * G * w.block * w.d
         out["window_bytes"] = nwin * G * (w.d * 2 * 2 + 8) + w.batch * w.n * w.h_kv * 2 * w.d * 2
         out["window_flops"] = 4.0 * wkeys * G * w.d
         out["merge_bytes"] = items * (G * w.d * 2 + G * 4 + w.topk * 4) + (nsl + nwin) * G * (w.d * 2 + 8)
-        out["plan_bytes"] = items * w.topk * 4 * (3 if w.block == 64 else 2) + nsl * 4 + items * 4
+        out["plan_bytes"] = items * w.topk * 4 * 3 + nsl * 4 + items * 12
         out["n_entries"] = ne
         out["n_slots"] = nsl
         out["n_blocks"] = nkeys

@@ -49,9 +49,10 @@ __device__ __forceinline__ int lane_hot_id(const BlockPlan& pl, const SlotSet& s
 // Counting passes over the rows of one chunk.  MODE 0: counts per key block
 // and each row's uncovered window blocks (the only pass without pairs).
 // MODE 1 (pair mode, first pass): counts per key block over every
-// kHotSample-th row only — they choose the hot set, and any hot set gives
-// the same attention.  MODE 2 (pair mode): counts per tile key and the
-// window blocks, every row.  chist columns: blocks (0, 1) or keys (2).
+// kHotSample-th row only, added into per-block totals — they choose the hot
+// set, and any hot set gives the same attention.  MODE 2 (pair mode):
+// counts per tile key and the window blocks, every row.  chist columns:
+// blocks (0) or keys (2).
 constexpr int kHotSample = 8;
 
 template <int MODE>
@@ -68,21 +69,33 @@ __global__ void __launch_bounds__(kPlanThreads) inv_hist_kernel(const BlockPlan 
   for (int i = k * kPlanRows + warp * step; i < r1; i += nw * step) {
     const int v = lane < pl.topk ? __ldg(idx + ((static_cast<int64_t>(b) * pl.n_q + i) * pl.h_kv + g) * pl.topk + lane) : -1;
     const SlotSet s = row_slots(v, pl.topk, pl.q_offset + i, pl.nb, pl.block, pl.window);
+    uint32_t selmask = static_cast<uint32_t>(s.mask);
     if (MODE == 2) {
       const PairSlot ps = pair_slots(s, lane_hot_id(pl, s, bg), pl.nb);
       if (ps.emit) atomicAdd(&hist[ps.key], 1);
+      selmask = ps.nsel >= 32 ? 0xFFFFFFFFu : ((1u << ps.nsel) - 1u);   // slots 0 .. nsel-1
     } else {
       if ((s.mask >> lane) & 1) atomicAdd(&hist[s.v], 1);
     }
-    if (MODE != 1 && lane == 0) pl.win[static_cast<int64_t>(bg) * pl.n_q + i] = s.win;
+    if (MODE != 1 && lane == 0) {
+      const int64_t it = static_cast<int64_t>(bg) * pl.n_q + i;
+      pl.win[it] = s.win;
+      pl.rowinfo[it] = make_uint2(selmask, static_cast<uint32_t>(s.n_bad));
+    }
   }
   __syncthreads();
+  if (MODE == 1) {   // sampled block totals, summed over the chunks (pl.count zeroed)
+    int32_t* tot = pl.count + static_cast<int64_t>(bg) * pl.nb;
+    for (int c = threadIdx.x; c < ncol; c += blockDim.x)
+      if (hist[c]) atomicAdd(&tot[c], hist[c]);
+    return;
+  }
   int32_t* out = pl.chist + (static_cast<int64_t>(bg) * pl.nchunk + k) * ncol;
   for (int c = threadIdx.x; c < ncol; c += blockDim.x) out[c] = hist[c];
 }
 
-// One CTA per (batch, kv-head), pair mode: each block's (sampled) selections
-// summed over the chunks of the first pass; the hot set is the largest set
+// One CTA per (batch, kv-head), pair mode: from each block's sampled
+// selections (totals of the first pass), the hot set is the largest set
 // {c : count_c >= T} (T >= 2) of at most kHotBlocks blocks, numbered in
 // block order.
 __global__ void __launch_bounds__(1024) inv_hot_kernel(const BlockPlan pl) {
@@ -91,12 +104,8 @@ __global__ void __launch_bounds__(1024) inv_hot_kernel(const BlockPlan pl) {
   __shared__ int32_t s_lo, s_hi;
   const int bg = blockIdx.x;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int32_t* ch = pl.chist + static_cast<int64_t>(bg) * pl.nchunk * pl.nb;
-  for (int c = threadIdx.x; c < pl.nb; c += blockDim.x) {
-    int v = 0;
-    for (int k = 0; k < pl.nchunk; ++k) v += ch[static_cast<int64_t>(k) * pl.nb + c];
-    tot[c] = v;
-  }
+  const int32_t* cnt = pl.count + static_cast<int64_t>(bg) * pl.nb;
+  for (int c = threadIdx.x; c < pl.nb; c += blockDim.x) tot[c] = cnt[c];
   // block-wide count of blocks with tot >= T
   auto count_ge = [&](int T) {
     int n = 0;
@@ -403,7 +412,9 @@ struct BlkCfg {
   // Q tile buffers: with G = 8 one warp fills them all by TMA; otherwise one
   // cp.async warp per buffer
   static constexpr bool TMA_Q = (G == 8);
-  static constexpr int NA = (BLK == 128 && TMA_Q) ? 3 : 4;
+  // 256-key tiles (pairs of 128-key blocks) fit two Q buffers beside their
+  // 128 KB of K and V
+  static constexpr int NA = BLK == 256 ? 2 : ((BLK == 128 && TMA_Q) ? 3 : 4);
   static constexpr int NGW = TMA_Q ? 1 : NA;            // gather warps
   static constexpr int KV_HALF = BLK * ROW;             // BLK keys x 64 dims
   static constexpr int KV_BYTES = 4 * KV_HALF;          // K lo, K hi, V lo, V hi
@@ -423,9 +434,13 @@ struct BlkCfg {
   // registers per thread: a sub-partition (SMSP) holds ceil(warps / 4) warps
   // of its 16384 registers
   static constexpr int MAXREG = (16384 / (32 * ((SW0 + 8 + 3) / 4))) & ~7;
-  static constexpr int S_COL = 0;                       // TMEM: S[2] (P over the first BLK/2
-  static constexpr int O_COL = 2 * BLK;                 // columns of its S), O[2], (m, l)[2]
+  // TMEM: S[NSB] (P over the first BLK/2 columns of its S), O[2], (m, l)[2];
+  // a 256-key tile's S takes half of the 512 columns, so it has one buffer
+  static constexpr int NSB = BLK == 256 ? 1 : 2;
+  static constexpr int S_COL = 0;
+  static constexpr int O_COL = NSB * BLK;
   static constexpr int ML_COL = O_COL + 2 * 128;
+  static_assert(O_COL + 2 * 128 <= 512, "tensor memory");
   static_assert(!ML_TMEM || ML_COL + 4 <= 512, "tensor memory");
   static_assert(USED <= 232448, "shared memory");
 };
@@ -489,15 +504,17 @@ __device__ __forceinline__ void tmem_ld64(uint32_t taddr, uint32_t (&r)[64]) {
 //          alternate tiles (S, P and O are double-buffered by tile parity),
 //          one tensor-core row = one (query, head) pair per thread.
 //
-// PAIR (64-key blocks, BLK = 128): a tile's 128 keys are the two blocks of
-// a pair, pair_tile_c1/c2 of its block field, loaded into the two 64-key
-// halves; a single-block tile loads its block into both halves and its
-// softmax leaves the second half out (P = 0 there).
+// PAIR (BLK = 2 x the block size: 128 for 64-key blocks, 256 for 128-key
+// blocks): a tile's keys are the two blocks of a pair, pair_tile_c1/c2 of
+// its block field, loaded into the two halves; a single-block tile loads its
+// block into both halves and its softmax leaves the second half out (P = 0
+// there).
 template <int G, int BLK, bool PAIR>
 __global__ void __maxnreg__((BlkCfg<G, BLK>::MAXREG))
     attn_block_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                       const __grid_constant__ CUtensorMap tmQ, const BlkArgs a) {
-  static_assert(!PAIR || BLK == 128, "pairs fill 128-key tiles");
+  static_assert(!PAIR || BLK == 128 || BLK == 256, "pairs fill 128- or 256-key tiles");
+  static_assert(PAIR || BLK != 256, "256-key tiles are pairs");
   using C = BlkCfg<G, BLK>;
   constexpr int D = C::D;
   constexpr int QPT = 128 / G;
@@ -578,9 +595,14 @@ __global__ void __maxnreg__((BlkCfg<G, BLK>::MAXREG))
         // first key of each 64-key half of the tile
         int zs[BLK / 64];
         if (PAIR) {
+          constexpr int KPB = BLK / 2;   // keys per block of the pair
           const int c1 = pair_tile_c1(td.y), c2 = pair_tile_c2(td.y);
-          zs[0] = static_cast<int>(static_cast<int64_t>(b) * a.n_kv + static_cast<int64_t>(c1) * 64);
-          zs[BLK / 64 - 1] = static_cast<int>(static_cast<int64_t>(b) * a.n_kv + static_cast<int64_t>(c2 >= 0 ? c2 : c1) * 64);
+#pragma unroll
+          for (int sub = 0; sub < BLK / 64; ++sub) {
+            const int src = sub * 64 < KPB ? c1 : (c2 >= 0 ? c2 : c1);
+            zs[sub] = static_cast<int>(static_cast<int64_t>(b) * a.n_kv + static_cast<int64_t>(src) * KPB +
+                                       (sub * 64) % KPB);
+          }
         } else {
 #pragma unroll
           for (int sub = 0; sub < BLK / 64; ++sub)
@@ -605,7 +627,8 @@ __global__ void __maxnreg__((BlkCfg<G, BLK>::MAXREG))
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      constexpr uint32_t IDESC1 = umma_idesc_bf16(128, BLK);
+      constexpr int SN = BLK;
+      constexpr uint32_t IDESC1 = umma_idesc_bf16(128, SN);
       constexpr uint32_t IDESC2 = umma_idesc_bf16(128, D) | (1u << 16);   // B (V) is MN-major
       const uint32_t sA_u = smem_u32(sA), sKV_u = smem_u32(sKV);
       int n1 = 0, n2 = 0;               // tiles whose S = Q K^T / O = P V are issued
@@ -626,15 +649,23 @@ __global__ void __maxnreg__((BlkCfg<G, BLK>::MAXREG))
           const int ab = n1 % NA;
           const int ord = kv_ord + (fresh ? 1 : 0);
           if ((!fresh || mbar_test_wait(&kv_full[kb], (ord / C::NKV) & 1)) &&
-              mbar_test_wait(&a_full[ab], (n1 / NA) & 1) && mbar_test_wait(&s_empty[n1 & 1], ((n1 >> 1) & 1) ^ 1)) {
+              mbar_test_wait(&a_full[ab], (n1 / NA) & 1) &&
+              // S(n1) reuses the S columns of tile n1 - NSB once its P V has
+              // read them; barriers go by tile parity, each waited on in order
+              (n1 < C::NSB ||
+               mbar_test_wait(&s_empty[(n1 - C::NSB) & 1], ((n1 - C::NSB) >> 1) & 1))) {
             tc_fence_after();
-            const uint32_t s_tmem = tmem_base + C::S_COL + (n1 & 1) * BLK;
+            const uint32_t s_tmem = tmem_base + C::S_COL + (n1 % C::NSB) * BLK;
             const uint32_t kbase = sKV_u + kb * C::KV_BYTES;
 #pragma unroll
             for (int ks = 0; ks < D / 16; ++ks) {
               const uint64_t ad = umma_desc_sw128(sA_u + ab * C::A_BYTES + (ks >> 2) * C::A_HALF + (ks & 3) * 32);
-              const uint64_t bd = umma_desc_sw128(kbase + (ks >> 2) * C::KV_HALF + (ks & 3) * 32);
-              umma_bf16(s_tmem, ad, bd, IDESC1, ks != 0 ? 1u : 0u);
+#pragma unroll
+              for (int np = 0; np < BLK / SN; ++np) {
+                const uint64_t bd =
+                    umma_desc_sw128(kbase + (ks >> 2) * C::KV_HALF + np * SN * C::ROW + (ks & 3) * 32);
+                umma_bf16(s_tmem + np * SN, ad, bd, IDESC1, ks != 0 ? 1u : 0u);
+              }
             }
             umma_commit(&s_full[n1 & 1]);
             umma_commit(&a_empty[ab]);
@@ -659,7 +690,7 @@ __global__ void __maxnreg__((BlkCfg<G, BLK>::MAXREG))
             const uint32_t d_tmem = tmem_base + C::O_COL + ob * D;
             // P (bf16, two per column) sits over the first BLK/2 columns of
             // this tile's S; 16 keys = 8 columns per step
-            const uint32_t p_tmem = tmem_base + C::S_COL + ob * BLK;
+            const uint32_t p_tmem = tmem_base + C::S_COL + (n2 % C::NSB) * BLK;
             const uint32_t vbase = sKV_u + kb2 * C::KV_BYTES + 2 * C::KV_HALF;
 #pragma unroll
             for (int kk = 0; kk < BLK / 16; ++kk) {
@@ -667,7 +698,7 @@ __global__ void __maxnreg__((BlkCfg<G, BLK>::MAXREG))
               umma_bf16_tmem_a(d_tmem, p_tmem + kk * 8, bd, IDESC2, kk != 0 ? 1u : 0u);
             }
             umma_commit(&o_full[ob]);
-            umma_commit(&s_empty[ob]);   // P read: the S / P columns take the next tile
+            umma_commit(&s_empty[n2 & 1]);   // P read: the S / P columns may take tile n2 + NSB
             if ((ring_last >> (n2 & 3)) & 1) umma_commit(&kv_empty[kb2]);
             ++n2;
             progressed = true;
@@ -722,15 +753,17 @@ __global__ void __maxnreg__((BlkCfg<G, BLK>::MAXREG))
       e_ent = entry_of(e_td);
       if (ts < T) {
         // ---------------- softmax of tile ts: P = 2^(s - m) in bf16 over S
+        // barriers and the (m, l) slot by tile parity (each group waits on
+        // its own barriers, in order); the S columns by buffer
         const int sb = ts & 1, use = ts >> 1;
         ok = __all_sync(0xFFFFFFFFu, mbar_wait(&s_full[sb], use & 1, a.err, SITE_BLK_S_FULL));
         if (!ok) break;
         tc_fence_after();
-        const uint32_t scol = tmem_base + lane_base + C::S_COL + sb * BLK;
+        const uint32_t scol = tmem_base + lane_base + C::S_COL + (ts % C::NSB) * BLK;
         auto load_half = [&](int hf, uint32_t (&r)[64]) { tmem_ld64(scol + hf * 64, r); };
         // pair mode: a single-block tile holds keys in its first half only
         // (tile-uniform)
-        const int nhalf = (PAIR && pair_tile_c2(tile_at(ts).y) < 0) ? 1 : BLK / 64;
+        const int nhalf = (PAIR && pair_tile_c2(tile_at(ts).y) < 0) ? BLK / 128 : BLK / 64;
         // maxima and sums in eight independent chains
         float mx[8] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY, -INFINITY, -INFINITY, -INFINITY, -INFINITY};
         float ls[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
@@ -1000,8 +1033,8 @@ __global__ void __maxnreg__((BlkCfg<G, BLK>::MAXREG))
 // lse = (M + log2 sum_j 2^(L_j - M)) ln 2, with M the largest L_j.
 
 struct MergeArgs {
-  const int32_t* idx;
-  const int32_t* hot_id;     // pair mode: [bgs][nb] hot numbers (else NULL)
+  const uint32_t* win;       // [items] uncovered window blocks (from the plan)
+  const uint2* rowinfo;      // [items] {selected-slot mask, skipped block_idx entries}
   const __half* partO;
   const float2* partL;
   __nv_bfloat16* O;
@@ -1023,19 +1056,17 @@ __global__ void __launch_bounds__(256, (G == 8 ? 2 : (G == 4 ? 3 : 4))) attn_mer
   const int i = it32 % a.n_q;
   const int bg = it32 / a.n_q;
   const int b = bg / a.h_kv, g = bg % a.h_kv;
-  const int v = lane < a.topk ? __ldg(a.idx + ((static_cast<int64_t>(b) * a.n_q + i) * a.h_kv + g) * a.topk + lane) : -1;
-  SlotSet s = row_slots(v, a.topk, a.q_offset + i, a.nb, a.block, a.window);
-  if (lane == 0 && a.bad && s.n_bad) atomicAdd(a.bad, s.n_bad);
-  if (a.hot_id) {   // pair mode: the selected slots are 0 .. nsel - 1
-    const int hid = ((s.mask >> lane) & 1) ? __ldg(a.hot_id + static_cast<int64_t>(bg) * a.nb + s.v) : -1;
-    const PairSlot ps = pair_slots(s, hid, a.nb);
-    s.mask = (1ull << ps.nsel) - 1ull;
-  }
-  // the window chunks (slots topk + c) that hold keys, one lane each
+  // the row's slots as the plan recorded them: selected slots (bit j) and,
+  // from its uncovered window blocks, the window chunks (slots topk + c)
+  // that hold keys, one lane each
+  const uint2 ri = __ldg(a.rowinfo + item);
+  const uint32_t win = __ldg(a.win + item);
+  if (lane == 0 && a.bad && ri.y) atomicAdd(a.bad, static_cast<int>(ri.y));
   const uint32_t wch = __ballot_sync(0xFFFFFFFFu, lane < a.nsl - a.topk &&
-                                                      chunk_has_keys(s.win, a.q_offset + i, a.window, a.block, lane,
+                                                      chunk_has_keys(win, a.q_offset + i, a.window, a.block, lane,
                                                                      win_chunk(G)));
-  s.mask |= static_cast<uint64_t>(wch) << a.topk;
+  struct { uint64_t mask; } s;
+  s.mask = static_cast<uint64_t>(ri.x) | (static_cast<uint64_t>(wch) << a.topk);
   const float2* pl = a.partL + item * a.nsl * G;
   const __half* po = a.partO + item * a.nsl * G * D;
   // per head: this lane's slots lane and lane + 32, their weights 2^(L-M) 2^e
@@ -1126,12 +1157,12 @@ cudaError_t run_block(const BlockPlan& pl, const CUtensorMap& tmK, const CUtenso
 
 }  // namespace
 
-cudaError_t launch_attn_merge(const ssa_params& p, const int32_t* block_idx, const int32_t* hot_id,
+cudaError_t launch_attn_merge(const ssa_params& p, const uint32_t* win, const uint2* rowinfo,
                               const void* partO, const void* partL, void* O, float* lse, int32_t* bad,
                               const LaunchCtx& c) {
   MergeArgs a;
-  a.idx = block_idx;
-  a.hot_id = hot_id;
+  a.win = win;
+  a.rowinfo = rowinfo;
   a.partO = static_cast<const __half*>(partO);
   a.partL = static_cast<const float2*>(partL);
   a.O = static_cast<__nv_bfloat16*>(O);
@@ -1176,6 +1207,8 @@ cudaError_t launch_block_plan(const ssa_params& p, const int32_t* block_idx, con
   // per-block counts and window blocks; in pair mode sampled per-block
   // counts, the hot sets, then the counts per tile key and window blocks
   if (pl.pair) {
+    e = cudaMemsetAsync(pl.count, 0, static_cast<size_t>(pl.bgs) * pl.nb * sizeof(int32_t), c.stream);
+    if (e != cudaSuccess) return e;
     inv_hist_kernel<1><<<rows, kPlanThreads, blk_smem, c.stream>>>(pl, block_idx);
     note_launch();
     inv_hot_kernel<<<pl.bgs, 1024, blk_smem, c.stream>>>(pl);
@@ -1231,6 +1264,11 @@ cudaError_t launch_attn_block(const ssa_params& p, const BlockPlan& pl, const vo
     if (G == 2) return run_block<2, 128, true>(pl, tmK, tmV, tmQ, a, c);
     if (G == 4) return run_block<4, 128, true>(pl, tmK, tmV, tmQ, a, c);
     if (G == 8) return run_block<8, 128, true>(pl, tmK, tmV, tmQ, a, c);
+  } else if (p.block == 128 && pl.pair) {
+    if (G == 1) return run_block<1, 256, true>(pl, tmK, tmV, tmQ, a, c);
+    if (G == 2) return run_block<2, 256, true>(pl, tmK, tmV, tmQ, a, c);
+    if (G == 4) return run_block<4, 256, true>(pl, tmK, tmV, tmQ, a, c);
+    if (G == 8) return run_block<8, 256, true>(pl, tmK, tmV, tmQ, a, c);
   } else if (p.block == 64) {
     if (G == 1) return run_block<1, 64>(pl, tmK, tmV, tmQ, a, c);
     if (G == 2) return run_block<2, 64>(pl, tmK, tmV, tmQ, a, c);

@@ -29,16 +29,18 @@ cudaError_t launch_summary(const ssa_params& p, const void* K, float* mu, float*
 cudaError_t launch_features(const ssa_params& p, const void* Q, void* F, const LaunchCtx& c);
 
 // Seeds of the tile router (one summary row per block): after every 32
-// blocks of a (batch, kv-head), snapshot s holds the topk blocks of largest
-// variance sum among blocks 0 .. 32 (s + 1) - 1 (ties to the lower block)
-// and their routing rows.  A unit of query rows whose first row sees
-// snapshot s scores those rows first: the least of the scores is a lower
-// bound on every row's k-th best score, the filter's starting threshold.
+// blocks of a (batch, kv-head), snapshot s holds 128 blocks among blocks
+// 0 .. 32 (s + 1) - 1 — the 32 of largest variance sum (ties to the lower
+// block) in each of four disjoint sets of 32-block batches — and their
+// routing rows.  A unit of query rows whose first row sees snapshot s
+// scores those rows first: the least of the maxima over disjoint groups of
+// them is a lower bound on every row's k-th best score, the filter's
+// starting threshold.
 struct RouteSeeds {
   int32_t n_snap;            // snapshots per (batch, kv-head): nb / 32
   float* var;                // [bgs][nb] variance sums of the routing rows
-  int32_t* blk;              // [bgs][n_snap][topk] seed blocks
-  void* tab;                 // [max(bgs * n_snap * topk, 128)][2d] bf16 seed rows
+  int32_t* blk;              // [bgs][n_snap][128] seed blocks
+  void* tab;                 // [bgs * n_snap * 128][2d] bf16 seed rows
 };
 size_t route_seed_bytes(const ssa_params& p);
 // The feature rows alone: the least workspace of ssa_route_topk's tiled router.
@@ -97,6 +99,7 @@ struct BlockPlan {
   int32_t* entries;                      // make_entry(query row, slot)
   int4* tiles;                           // {bg, block, first entry, entries}
   uint32_t* win;                         // [bgs * n_q] uncovered window blocks of each row
+  uint2* rowinfo;                        // [bgs * n_q] {selected-slot mask, skipped block_idx entries}
   // balanced split of the tiles over the block kernel's CTAs
   int32_t max_tiles, grid;               // tile capacity; CTAs (<= kMaxBlockGrid)
   uint8_t* tcost;                        // [max_tiles] estimated cost of each tile
@@ -128,8 +131,8 @@ cudaError_t launch_attn_window(const ssa_params& p, const BlockPlan& pl, const C
                                const LaunchCtx& c);
 
 // Per (query, kv-head): the softmax merge of the slot partials into O, lse.
-// hot_id: the plan's hot numbers in pair mode (64-key blocks), else NULL.
-cudaError_t launch_attn_merge(const ssa_params& p, const int32_t* block_idx, const int32_t* hot_id,
+// win, rowinfo: the plan's per-row window blocks and slot records.
+cudaError_t launch_attn_merge(const ssa_params& p, const uint32_t* win, const uint2* rowinfo,
                               const void* partO, const void* partL, void* O, float* lse, int32_t* bad,
                               const LaunchCtx& c);
 

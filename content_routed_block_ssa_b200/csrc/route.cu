@@ -87,9 +87,11 @@ struct RouteTiledArgs {
   // skipped (every role reads the same flag; no output is written for them)
   const int32_t* unit_need;
   // seeds (0 snapshots: none): a unit whose first row sees snapshot s first
-  // scores that snapshot's topk seed rows, at row (bg * n_snap + s) * topk
+  // scores that snapshot's kSeedRows seed rows, at row (bg * n_snap + s) * kSeedRows
   int32_t n_snap;
 };
+
+constexpr int kSeedRows = 128;   // seed rows per snapshot: one chunk of columns
 
 // The unit's seed snapshot, or -1: the last snapshot whose 32 (s + 1)
 // blocks are all visible to the unit's first row (and so to all its rows).
@@ -273,6 +275,13 @@ __device__ __forceinline__ void filter_group(const uint32_t (&v)[16], int c0, in
   } else {
     pool_columns<S>(v, w);
   }
+  // the group's largest score against the threshold first: most groups of
+  // most rows hold no candidate once the threshold is high (the scores are
+  // finite, so fmaxf is the maximum)
+  float mx = __uint_as_float(w[0]);
+#pragma unroll
+  for (int t = 1; t < N; ++t) mx = fmaxf(mx, __uint_as_float(w[t]));
+  if (!__any_sync(0xFFFFFFFFu, mx > thr)) return;
   if (__all_sync(0xFFFFFFFFu, b0 + N <= nvis))
     filter_n<N, false>(w, b0, nvis, thr, cnt, my_cand);
   else
@@ -353,7 +362,7 @@ __global__ void __launch_bounds__(TiledCfg<KF>::THREADS, 1)
             if (!mbar_wait(&b_empty[s], ((b_cnt / C::NS) & 1) ^ 1, a.err, SITE_ROUTE_PRODUCER)) { ok = false; break; }
             mbar_arrive_expect_tx(&b_full[s], C::BOX_BYTES);
             if (j < 0)
-              tma_load_2d(sB + s * C::BOX_BYTES, &tmS, &b_full[s], ks * 64, (bg * a.n_snap + snap) * a.topk);
+              tma_load_2d(sB + s * C::BOX_BYTES, &tmS, &b_full[s], ks * 64, (bg * a.n_snap + snap) * kSeedRows);
             else
               tma_load_2d(sB + s * C::BOX_BYTES, &tmT, &b_full[s], ks * 64, trow + j * 128);
             ++b_cnt;
@@ -445,28 +454,36 @@ __global__ void __launch_bounds__(TiledCfg<KF>::THREADS, 1)
       bool empty_list = true;   // warp-uniform: no merge of this unit yet
       const int snap = unit_snap(a, row0);
       if (snap >= 0) {
-        // chunk -1: the topk seed blocks' scores (columns 0 .. topk-1); all
-        // are visible to every row of the unit, so the least of them is at
-        // most the row's k-th best score.  The threshold sits a little
+        // chunk -1: the scores of the snapshot's 128 seed blocks, all visible
+        // to every row of the unit, in ng = 128 / gs disjoint groups of gs
+        // consecutive columns (ng the least power of two >= topk).  Each
+        // group's largest score belongs to a distinct block, so at least ng
+        // >= topk blocks score at least the least of the ng maxima: a lower
+        // bound on the row's k-th best score.  The threshold sits a little
         // below it, so a block scoring exactly that much still passes.
         const int acc = 2 * (ch_cnt & 1) + grp;
         ok = __all_sync(0xFFFFFFFFu, mbar_wait(&acc_full[acc], (ch_cnt >> 1) & 1, a.err, SITE_ROUTE_EPILOGUE));
         if (!ok) break;
         tc_fence_after();
         const uint32_t taddr = tmem_base + (static_cast<uint32_t>(eq * 32) << 16) + acc * 128;
-        uint32_t v0[16], v1[16];
-        tmem_ld16(taddr, v0);
-        tmem_ld16(taddr + 16, v1);
-        tmem_wait_ld();
+        int ng = 1;
+        while (ng < a.topk) ng <<= 1;
+        const int gs = kSeedRows / ng;
+        float mn = INFINITY, gmax = -INFINITY;
+#pragma unroll 1
+        for (int sub = 0; sub < kSeedRows / 16; ++sub) {
+          uint32_t v[16];
+          tmem_ld16(taddr + sub * 16, v);
+          tmem_wait_ld();
+#pragma unroll
+          for (int t = 0; t < 16; ++t) {
+            gmax = fmaxf(gmax, __uint_as_float(v[t]));
+            if (((sub * 16 + t + 1) & (gs - 1)) == 0) { mn = fminf(mn, gmax); gmax = -INFINITY; }
+          }
+        }
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&acc_empty[acc]);
-        float mn = INFINITY;
-#pragma unroll
-        for (int t = 0; t < 16; ++t) {
-          if (t < a.topk) mn = fminf(mn, __uint_as_float(v0[t]));
-          if (t + 16 < a.topk) mn = fminf(mn, __uint_as_float(v1[t]));
-        }
         floor_thr = mn - (fabsf(mn) * 0x1p-16f + 0x1p-24f);
         thr = floor_thr;
         ++ch_cnt;
@@ -1166,15 +1183,20 @@ cudaError_t launch_route_tiled(const ssa_params& p, const CUtensorMap& tmF, cons
 
 // ------------------------------------------------------------------ seeds
 
+// Snapshots per (batch, kv-head) the prefix scan holds in shared memory
+// (2 x 512 lists of 32 keys = 256 KB would not fit; 2 x 384 = 192 KB does):
+// problems with more blocks route without seeds.
+constexpr size_t kMaxSnap = 384;
+
 size_t route_seed_bytes(const ssa_params& p) {
   if (rows_per_block(p) != 1 || p.dtype != SSA_BF16) return 0;
   const size_t bgs = static_cast<size_t>(p.batch) * p.h_kv;
   const size_t nb = static_cast<size_t>(p.n_kv / p.block);
   const size_t n_snap = nb / 32;
-  if (n_snap == 0) return 0;
+  if (n_snap == 0 || n_snap > kMaxSnap) return 0;
   auto ru = [](size_t x) { return (x + 255) & ~size_t(255); };
-  const size_t rows = bgs * n_snap * p.topk > 128 ? bgs * n_snap * p.topk : 128;
-  return ru(bgs * nb * 4) + ru(bgs * n_snap * p.topk * 4) + ru(rows * 2 * p.d * 2);
+  const size_t rows = bgs * n_snap * kSeedRows;
+  return ru(bgs * nb * 4) + ru(rows * 4) + ru(rows * 2 * p.d * 2);
 }
 
 RouteSeeds route_seed_layout(const ssa_params& p, void* base) {
@@ -1186,7 +1208,7 @@ RouteSeeds route_seed_layout(const ssa_params& p, void* base) {
   uint8_t* b = static_cast<uint8_t*>(base);
   s.var = reinterpret_cast<float*>(b);
   s.blk = reinterpret_cast<int32_t*>(b + ru(bgs * nb * 4));
-  s.tab = b + ru(bgs * nb * 4) + ru(bgs * s.n_snap * p.topk * 4);
+  s.tab = b + ru(bgs * nb * 4) + ru(bgs * s.n_snap * kSeedRows * 4);
   return s;
 }
 
@@ -1225,24 +1247,71 @@ __device__ __forceinline__ uint64_t warp_sort_desc(uint64_t key) {
   return key;
 }
 
-// Warp per (batch, kv-head): the running 32 blocks of largest variance sum
-// (key: variance desc, then block asc), and after every full batch of 32
-// blocks the first topk of them as snapshot s.
-__global__ void __launch_bounds__(256) seed_prefix_kernel(const float* __restrict__ var, int32_t* __restrict__ blk,
-                                                          int bgs, int nb, int n_snap, int topk) {
-  const int bg = (blockIdx.x * 256 + threadIdx.x) >> 5;
-  if (bg >= bgs) return;   // warp-uniform
+// CTA per (batch, kv-head): every 32-block batch's keys (variance desc,
+// then block asc) sorted by one warp, then a Hillis-Steele prefix scan over
+// the batches of each residue class mod 4, each step keeping the larger 32
+// of two sorted lists (an associative merge): list s ends as the 32 best
+// keys of batches s, s-4, s-8, ...  Snapshot s (blocks 0 .. 32 (s+1) - 1)
+// takes lists s, s-1, s-2, s-3 — four disjoint sets of blocks — as its 128
+// seeds, ordered so that every group of 4 consecutive seeds holds one of the
+// 32 largest variance sums (below).  Two shared buffers of n_snap lists of
+// 32 keys (n_snap <= kMaxSnap).
+__device__ __forceinline__ uint64_t merge_top32(uint64_t a, uint64_t b_desc) {
+  // a, b: descending runs held one element per lane; the larger 32 of the
+  // 64 form a bitonic sequence a[l] max b[31 - l], sorted once more
   const int lane = threadIdx.x & 31;
-  uint64_t best = 0;       // lane l: the l-th best so far (0: none)
-  for (int s = 0; s < n_snap; ++s) {
+  const uint64_t rev = __shfl_sync(0xFFFFFFFFu, b_desc, 31 - lane);
+  return warp_sort_desc(a > rev ? a : rev);
+}
+
+__global__ void __launch_bounds__(1024) seed_prefix_kernel(const float* __restrict__ var, int32_t* __restrict__ blk,
+                                                           int nb, int n_snap) {
+  extern __shared__ uint64_t lists[];   // [2][n_snap][32]
+  const int bg = blockIdx.x;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+  uint64_t* cur = lists;
+  uint64_t* nxt = lists + n_snap * 32;
+  for (int s = warp; s < n_snap; s += nw) {
     const int c = s * 32 + lane;
-    const uint64_t key = make_key(__float_as_uint(var[static_cast<int64_t>(bg) * nb + c]), static_cast<uint32_t>(c));
-    const uint64_t fresh = warp_sort_desc(key);
-    // the larger 32 of two descending runs: best[l] against fresh[31 - l]
-    // gives a bitonic sequence holding them; sort it
-    const uint64_t rev = __shfl_sync(0xFFFFFFFFu, fresh, 31 - lane);
-    best = warp_sort_desc(best > rev ? best : rev);
-    if (lane < topk) blk[(static_cast<int64_t>(bg) * n_snap + s) * topk + lane] = static_cast<int32_t>(key_block(best));
+    cur[s * 32 + lane] = warp_sort_desc(
+        make_key(__float_as_uint(var[static_cast<int64_t>(bg) * nb + c]), static_cast<uint32_t>(c)));
+  }
+  __syncthreads();
+  for (int off = 4; off < n_snap; off <<= 1) {
+    for (int s = warp; s < n_snap; s += nw) {
+      const uint64_t mine = cur[s * 32 + lane];
+      nxt[s * 32 + lane] = s >= off ? merge_top32(mine, cur[(s - off) * 32 + lane]) : mine;
+    }
+    __syncthreads();
+    uint64_t* t = cur; cur = nxt; nxt = t;
+  }
+  // snapshot s: the nl = min(4, s + 1) lists s, s-1, .. ranked together by
+  // key (the keys are distinct); seed column 4 j + t holds rank j + 32 t, or
+  // rank j again when that rank does not exist, so group j of 4 consecutive
+  // columns holds rank j, one of the 32 largest variances
+  for (int s = warp; s < n_snap; s += nw) {
+    const int nl = s + 1 < 4 ? s + 1 : 4;
+    int32_t* out = blk + (static_cast<int64_t>(bg) * n_snap + s) * kSeedRows;
+#pragma unroll
+    for (int r = 0; r < 4; ++r) {
+      if (r >= nl) break;   // warp-uniform
+      const uint64_t key = cur[(s - r) * 32 + lane];
+      int rank = lane;
+      for (int q = 0; q < nl; ++q) {
+        if (q == r) continue;
+        const uint64_t* L = cur + (s - q) * 32;   // descending: count the keys above `key`
+        int lo = 0, hi = 32;
+        while (lo < hi) {
+          const int mid = (lo + hi) >> 1;
+          if (L[mid] > key) lo = mid + 1; else hi = mid;
+        }
+        rank += lo;
+      }
+      const int32_t b = static_cast<int32_t>(key_block(key));
+      out[(rank & 31) * 4 + (rank >> 5)] = b;
+      if (rank < 32)
+        for (int t = nl; t < 4; ++t) out[rank * 4 + t] = b;
+    }
   }
 }
 
@@ -1277,14 +1346,16 @@ cudaError_t launch_route_seeds(const ssa_params& p, const void* table, const Rou
   if (p.d == 128) seed_var_kernel<128><<<g1, 256, 0, c.stream>>>(T, s.var, rows);
   else seed_var_kernel<64><<<g1, 256, 0, c.stream>>>(T, s.var, rows);
   note_launch();
-  seed_prefix_kernel<<<static_cast<unsigned>((bgs * 32 + 255) / 256), 256, 0, c.stream>>>(s.var, s.blk, bgs, nb,
-                                                                                          s.n_snap, p.topk);
+  const int psmem = 2 * s.n_snap * 32 * static_cast<int>(sizeof(uint64_t));
+  cudaError_t e = cudaFuncSetAttribute(seed_prefix_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, psmem);
+  if (e != cudaSuccess) return e;
+  seed_prefix_kernel<<<static_cast<unsigned>(bgs), 1024, psmem, c.stream>>>(s.var, s.blk, nb, s.n_snap);
   note_launch();
-  const int64_t srows = static_cast<int64_t>(bgs) * s.n_snap * p.topk;
+  const int64_t srows = static_cast<int64_t>(bgs) * s.n_snap * kSeedRows;
   const unsigned g3 = static_cast<unsigned>((srows * 32 + 255) / 256);
   __nv_bfloat16* tab = static_cast<__nv_bfloat16*>(s.tab);
-  if (p.d == 128) seed_gather_kernel<128><<<g3, 256, 0, c.stream>>>(T, s.blk, tab, srows, nb, s.n_snap * p.topk);
-  else seed_gather_kernel<64><<<g3, 256, 0, c.stream>>>(T, s.blk, tab, srows, nb, s.n_snap * p.topk);
+  if (p.d == 128) seed_gather_kernel<128><<<g3, 256, 0, c.stream>>>(T, s.blk, tab, srows, nb, s.n_snap * kSeedRows);
+  else seed_gather_kernel<64><<<g3, 256, 0, c.stream>>>(T, s.blk, tab, srows, nb, s.n_snap * kSeedRows);
   note_launch();
   return cudaGetLastError();
 }

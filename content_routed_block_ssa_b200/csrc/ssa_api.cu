@@ -169,13 +169,13 @@ bool use_block_attn(const ssa_params& p) {
          ssa::window_slots(p.window, p.block) <= 32 && nb <= 16384 && p.n_q >= 1024 && p.n_q < (1 << 25);
 }
 
-// Paired slots: the block-major attention of 64-key blocks evaluates two
-// selected blocks per slot (128-key tiles).
-bool pair_mode(const ssa_params& p) { return p.block == 64; }
+// Paired slots: the block-major attention evaluates two selected blocks per
+// slot (128-key tiles for 64-key blocks, 256-key tiles for 128-key blocks).
+bool pair_mode(const ssa_params& p) { return p.block == 64 || p.block == 128; }
 
 struct AttnLayout {
   size_t chist, count, blk_off, tile_off, bg_ents, bg_tiles, ent_base, tile_base, entries, tiles, tcost, csum,
-      t_start, win, hot_id, hot_blk, part_o, part_l, total;
+      t_start, win, rowinfo, hot_id, hot_blk, part_o, part_l, total;
   int nchunk, nsl, nkey;
   size_t max_tiles;
 };
@@ -210,6 +210,7 @@ AttnLayout attn_layout(const ssa_params& p) {
   L.csum = off; off += round_up((max_tiles + 255) / 256 * 4);
   L.t_start = off; off += round_up((ssa::kMaxBlockGrid + 1) * 4);
   L.win = off; off += round_up(items * 4);
+  L.rowinfo = off; off += round_up(items * 8);
   L.hot_id = off; off += pair_mode(p) ? round_up(bgs * nb * 4) : 0;
   L.hot_blk = off; off += pair_mode(p) ? round_up(bgs * ssa::kHotBlocks * 4) : 0;
   L.part_o = off; off += round_up(sel * G * p.d * 2);
@@ -320,9 +321,9 @@ ssa_status do_route(const ssa_params& p, const void* Q, const float* mu, const f
   if (sb && ws_bytes >= need + sb) {
     const ssa::RouteSeeds S = ssa::route_seed_layout(p, static_cast<uint8_t*>(ws) + need);
     if ((st = from_cuda(ssa::launch_route_seeds(p, table, S, c))) != SSA_OK) return st;
-    const uint64_t srows = static_cast<uint64_t>(p.batch) * p.h_kv * S.n_snap * p.topk;
+    const uint64_t srows = static_cast<uint64_t>(p.batch) * p.h_kv * S.n_snap * 128;   // 128 seed rows each
     CUtensorMap tmS;
-    if (!encode_2d(&tmS, S.tab, kf, srows > 128 ? srows : 128, 128)) return SSA_ERR_CUDA;
+    if (!encode_2d(&tmS, S.tab, kf, srows, 128)) return SSA_ERR_CUDA;
     return from_cuda(ssa::launch_route_tiled(p, tmF, tmT, idx, scores, c, nullptr, &tmS, S.n_snap));
   }
   return from_cuda(ssa::launch_route_tiled(p, tmF, tmT, idx, scores, c));
@@ -355,6 +356,7 @@ ssa::BlockPlan block_plan(const ssa_params& p, const AttnLayout& L, uint8_t* w) 
   pl.entries = reinterpret_cast<int32_t*>(w + L.entries);
   pl.tiles = reinterpret_cast<int4*>(w + L.tiles);
   pl.win = reinterpret_cast<uint32_t*>(w + L.win);
+  pl.rowinfo = reinterpret_cast<uint2*>(w + L.rowinfo);
   pl.max_tiles = static_cast<int32_t>(L.max_tiles);
   pl.grid = 0;   // set by the caller from the device's SM count
   pl.tcost = w + L.tcost;
@@ -405,8 +407,10 @@ ssa_status attn_stage_window(const ssa_params& p, const AttnMaps& m, uint8_t* w,
 ssa_status attn_stage_merge(const ssa_params& p, const int32_t* idx, void* O, float* lse, int32_t* bad,
                             const uint8_t* w, const LaunchCtx& c) {
   const AttnLayout L = attn_layout(p);
-  const int32_t* hot_id = pair_mode(p) ? reinterpret_cast<const int32_t*>(w + L.hot_id) : nullptr;
-  return from_cuda(ssa::launch_attn_merge(p, idx, hot_id, w + L.part_o, w + L.part_l, O, lse, bad, c));
+  (void)idx;   // the plan recorded each row's slots from block_idx
+  return from_cuda(ssa::launch_attn_merge(p, reinterpret_cast<const uint32_t*>(w + L.win),
+                                          reinterpret_cast<const uint2*>(w + L.rowinfo), w + L.part_o,
+                                          w + L.part_l, O, lse, bad, c));
 }
 
 ssa_status do_attn(const ssa_params& p, const void* Q, const void* K, const void* V,

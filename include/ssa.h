@@ -206,12 +206,15 @@ SSA_API size_t ssa_attn_workspace_size(const ssa_params* p);
  * of ssa_attn_workspace_size(p) bytes (bf16 problems with n_q >= 1024,
  * d = 128, G in {1, 2, 4, 8}, topk * G <= 128, at most 32 key blocks per
  * window and 16384 key blocks) the evaluation is block-major: every
- * (query, kv-head) row is split into slots, one per used selected block and
- * one per window block not selected, the slots are inverted into per-block
- * lists, each key block is multiplied once against all its slots' queries on
- * the tensor cores (window slots masked to the window), and the slot
- * partials are merged per row.  With ws NULL (or too small) every
- * (query, kv-head) gathers its own keys.
+ * (query, kv-head) row is split into slots — its used selected blocks of
+ * the (batch, kv-head)'s hot set (its at most 128 most selected blocks)
+ * taken two at a time in block order, one slot per pair; every other used
+ * block a slot of its own; and the chunks of the window outside them — the
+ * slots are inverted into per-key lists, each block or pair of blocks is
+ * multiplied once against all its slots' queries on the tensor cores, the
+ * window chunks run as dense sliding-window tiles, and the slot partials are
+ * merged per row.  With ws NULL (or too small) every (query, kv-head)
+ * gathers its own keys.
  *   O            device output [b, n_q, h_q, d] of dtype
  *   lse          device float32 output, may be NULL
  *   ws, ws_bytes device workspace, may be NULL / 0
@@ -226,22 +229,26 @@ SSA_API ssa_status ssa_sparse_attn(const ssa_params* p, const void* Q, const voi
  * stream with one workspace (ssa_attn_workspace_size(p) bytes, 16-byte
  * aligned; its contents are private to the library and live from the plan
  * call to the merge call), they give exactly the bytes ssa_sparse_attn gives
- * with that workspace.  A row's keys fall in "slots": each used selected
- * block, and each 256-key chunk of the window (pos-W+1 .. pos) minus the
- * keys of its used selected blocks.
- *   ssa_attn_plan    inverts block_idx: the used selected blocks of every
- *                    row as per-(batch, kv-head, key block) lists, in tiles
- *                    of 128 / G queries, and each row's window blocks that
- *                    no used entry selects;
- *   ssa_attn_blocks  per tile, S = Q_tile K_c^T and O = P V_c on the tensor
- *                    cores; writes each selected slot's normalised partial
- *                    output and base-2 log-sum-exp into the workspace;
+ * with that workspace.  A row's keys fall in "slots": each pair of used
+ * selected hot blocks (or used selected block outside the pairs), and each
+ * 256-key chunk of the window (pos-W+1 .. pos; 128 keys when G = 1) minus
+ * the keys of its used selected blocks.
+ *   ssa_attn_plan    inverts block_idx: the selected slots of every row as
+ *                    per-(batch, kv-head, block or pair) lists, in tiles of
+ *                    128 / G queries, and each row's window blocks that no
+ *                    used entry selects;
+ *   ssa_attn_blocks  per tile, S = Q_tile K^T and O = P V over the block's
+ *                    or pair's keys on the tensor cores; writes each selected
+ *                    slot's normalised partial output and base-2 log-sum-exp
+ *                    into the workspace;
  *   ssa_attn_window  per run of 128 / G consecutive queries and window
  *                    chunk, the same over the chunk's keys (dense tensor-core
  *                    tiles masked per row); writes the window slots' partials;
  *   ssa_attn_merge   per (query, kv-head): the softmax merge of the row's
  *                    slot partials into O and lse; counts skipped block_idx
- *                    entries as ssa_sparse_attn does.
+ *                    entries as ssa_sparse_attn does.  It reads each row's
+ *                    slots as the plan call recorded them, so block_idx
+ *                    must be the array that call was given.
  * ssa_attn_blocks and ssa_attn_window write disjoint parts of the workspace
  * and may run in either order (or on two streams ordered after the plan and
  * before the merge).

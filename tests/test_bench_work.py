@@ -33,8 +33,8 @@ def test_attended_keys_is_the_key_set_size():
 
 
 def _direct_slots(arr, w, p):
-    """The slot rule written out row by row: used entries; with 64-key blocks
-    the hot blocks of each kv-head (count over every 8th row >= the smallest
+    """The slot rule written out row by row: used entries; the hot blocks of
+    each kv-head (count over every 8th row >= the smallest
     T >= 2 that leaves at most 128 of them) are paired two at a time in
     block order."""
     from collections import Counter
@@ -53,8 +53,6 @@ def _direct_slots(arr, w, p):
             if i % 8 == 0:
                 cnt.update((g, c) for c in used)
     n_e = sum(len(u) for u in used_rows.values())
-    if w.block != 64:
-        return n_e, n_e, len({(g, c) for (i, g), u in used_rows.items() for c in u})
     hot = {}
     for g in range(w.h_kv):
         counts = [cnt[(g, c)] for c in range(w.n // w.block)]
@@ -85,12 +83,26 @@ def test_block_major_counts_by_direct_count():
         got = bench.block_major_counts(torch.from_numpy(arr), w)
         assert got == _direct_slots(arr, w, p)
         assert got[1] < got[0]          # some entries pair up
-    # 128-key blocks: one slot per used entry
+    # 128-key blocks pair the same way
     w2 = w.scaled(block=128)
     p2 = O.Problem(**problem_dict(w2))
     arr2 = np.where(idx >= 0, idx // 2, idx)
     got2 = bench.block_major_counts(torch.from_numpy(arr2), w2)
-    assert got2 == _direct_slots(arr2, w2, p2) and got2[0] == got2[1]
+    assert got2 == _direct_slots(arr2, w2, p2) and got2[1] < got2[0]
+    # a block chosen only by rows the hot-set count skips is not hot: sampled
+    # and full counts give different slot totals here
+    arr3 = idx.copy()
+    arr3[:, :, :, :] = -1
+    arr3[0, 700:720, 0, 0] = 3          # rows 700..719 (704, 712 sampled): blocks 3 and 5
+    arr3[0, 700:720, 0, 1] = 5
+    arr3[0, 701, 0, 2] = 7              # blocks 7 and 9: rows 701 and 703, never sampled
+    arr3[0, 703, 0, 2] = 7
+    arr3[0, 701, 0, 3] = 9
+    arr3[0, 703, 0, 3] = 9
+    got3 = bench.block_major_counts(torch.from_numpy(arr3), w)
+    assert got3 == _direct_slots(arr3, w, p)
+    # 3 and 5 are hot (two sampled rows each), 7 and 9 are not: 20 pairs + 4 singles
+    assert got3 == (44, 24, 3)
 
 
 def test_kernel_report_fractions_and_dominant_stage():

@@ -92,6 +92,15 @@ CASES = {
                                       outlier=True),
     "f32_full_d64_outlier": Workload("c", 137, 1, 768, 2, 1, 64, "f32", 64, "full", 4, 64, 2, "total",
                                      outlier=True),
+    # paired slots at their edges: k = 1 (every tile a single block, its
+    # second half masked) and k = 2 (one pair or two singles per row), with
+    # 64-key blocks (128-key tiles) and 128-key blocks (256-key tiles)
+    "bf16_gqa4_d128_b64_k1": Workload("c", 138, 1, 2048, 8, 2, 128, "bf16", 64, "diag", 1, 128, 4, "total",
+                                      clustered=True),
+    "bf16_gqa8_d128_b128_k1": Workload("c", 139, 1, 3072, 8, 1, 128, "bf16", 128, "diag", 1, 256, 6, "total",
+                                       clustered=True),
+    "bf16_gqa4_d128_b128_k2": Workload("c", 140, 1, 3072, 8, 2, 128, "bf16", 128, "diag", 2, 256, 6, "total",
+                                       clustered=True),
     # float32 routing takes runs of 32 (query, head) pairs per CTA unless a
     # row's 1024 block scores do not fit beside them: then one CTA per row
     "f32_diag_d64_decode_64k": Workload("c", 122, 1, 65536, 1, 1, 64, "f32", 64, "diag", 8, 64, 2, "per_seq",

@@ -139,11 +139,12 @@ def test_workspace_sizes():
     assert ssa.ssa_route_workspace_size(p) == rnd(feat)
     assert ssa.ssa_workspace_size(p) == rnd(tab) + rnd(feat) + rnd(idx)
     # with at least 32 blocks the tiled router also takes its seed arrays:
-    # variance sums [bgs, nb] f32, seed blocks [bgs, nb/32, k] i32 and the
-    # seed rows [max(bgs * nb/32 * k, 128), 2d] bf16
+    # variance sums [bgs, nb] f32, seed blocks [bgs, nb/32, 128] i32 and the
+    # seed rows [bgs * nb/32 * 128, 2d] bf16
     sp = good(n_q=1000, n_kv=4096)
     feat4 = 1 * 2 * 1000 * 256 * 2
-    assert ssa.ssa_route_workspace_size(sp) == rnd(feat4) + rnd(2 * 64 * 4) + rnd(2 * 2 * 4 * 4) + rnd(128 * 256 * 2)
+    assert ssa.ssa_route_workspace_size(sp) == (rnd(feat4) + rnd(2 * 64 * 4) + rnd(2 * 2 * 128 * 4)
+                                                + rnd(2 * 2 * 128 * 256 * 2))
     row = good(n_q=1, n_kv=1024, q_offset=1023)           # decode routes per row: no features
     assert ssa.ssa_route_workspace_size(row) == 0
     f32 = good(dtype="f32", sigma="full", d=64, h_q=2, n_q=128, n_kv=128)
