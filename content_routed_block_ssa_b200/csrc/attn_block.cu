@@ -403,29 +403,40 @@ __global__ void __launch_bounds__(1024) inv_split_kernel(const BlockPlan pl, int
 
 // ------------------------------------------------------------------ block tiles
 
+// The second 128-key sub-tile of a 256-key tile keeps the softmax's running
+// maximum while its own maximum exceeds it by at most this many powers of
+// two (P <= 2^16 then).  Pairs of selected blocks differ in their largest
+// logit by more than 8 powers of two in a few percent of rows, by more than
+// 16 in about one in a thousand.
+constexpr float kStaleMax = 16.f;
+
 template <int G, int BLK>
 struct BlkCfg {
+  static_assert(BLK == 128 || BLK == 256, "tiles hold pairs of 64- or 128-key blocks");
   static constexpr int D = 128;
   static constexpr int ROW = 128;                       // bytes per 64-wide swizzled row
   static constexpr int A_HALF = 128 * ROW;              // 128 rows x 64 dims
   static constexpr int A_BYTES = 2 * A_HALF;            // Q tile
   // Q tile buffers: with G = 8 one warp fills them all by TMA; otherwise one
-  // cp.async warp per buffer
+  // cp.async warp per buffer.  256-key tiles fit two beside their 128 KB of
+  // K and V.
   static constexpr bool TMA_Q = (G == 8);
-  // 256-key tiles (pairs of 128-key blocks) fit two Q buffers beside their
-  // 128 KB of K and V
-  static constexpr int NA = BLK == 256 ? 2 : ((BLK == 128 && TMA_Q) ? 3 : 4);
+  static constexpr int NA = BLK == 256 ? 2 : 4;
   static constexpr int NGW = TMA_Q ? 1 : NA;            // gather warps
   static constexpr int KV_HALF = BLK * ROW;             // BLK keys x 64 dims
   static constexpr int KV_BYTES = 4 * KV_HALF;          // K lo, K hi, V lo, V hi
-  static constexpr int NKV = (BLK == 64) ? 2 : 1;       // K/V buffers (at most 2)
-  static constexpr int STG_BYTES = 128 * ROW;           // epilogue staging: 128 rows x 64 dims
-  static constexpr int NBAR = 2 * NA + 2 * NKV + 2 * 6 + 1;
-  // (m, l) of each row from the softmax to the epilogue, by tile parity: in
-  // spare TMEM columns with 64-key blocks, else in shared memory
-  static constexpr bool ML_TMEM = (BLK == 64);
-  static constexpr int ML_BYTES = ML_TMEM ? 0 : 2 * 128 * 8;
-  static constexpr int USED = NA * A_BYTES + NKV * KV_BYTES + 2 * STG_BYTES + ML_BYTES + NBAR * 8 + 16;
+  static constexpr int NKV = 1;                         // K/V buffers
+  static constexpr int STG_WARP = 32 * 64;              // epilogue staging per softmax warp: 32 rows x 32 dims
+  // S sub-tiles: a 256-key tile runs as two 128-key sub-tiles that share its
+  // Q rows and its O accumulator
+  static constexpr int SK = 128;                        // keys per sub-tile
+  static constexpr int SUB = BLK / SK;                  // sub-tiles per tile
+  // barriers: a[NA] x 2, kv[NKV] x 2, s_full and p_full [2][SUB], s_empty,
+  // o_full, o_empty, ml_empty, pa_done [2], mma_done
+  static constexpr int NBAR = 2 * NA + 2 * NKV + 4 * SUB + 10 + 1;
+  // (m, l, lr) of each row from the softmax to the epilogue, by tile parity
+  static constexpr int ML_BYTES = 2 * 128 * 16;
+  static constexpr int USED = NA * A_BYTES + NKV * KV_BYTES + 8 * STG_WARP + ML_BYTES + NBAR * 8 + 16;
   // room to align the base to 1024 bytes, up to the 227 KB limit (the
   // kernel checks that the aligned layout fits)
   static constexpr int SMEM = USED + 1024 < 232448 ? USED + 1024 : 232448;
@@ -434,14 +445,12 @@ struct BlkCfg {
   // registers per thread: a sub-partition (SMSP) holds ceil(warps / 4) warps
   // of its 16384 registers
   static constexpr int MAXREG = (16384 / (32 * ((SW0 + 8 + 3) / 4))) & ~7;
-  // TMEM: S[NSB] (P over the first BLK/2 columns of its S), O[2], (m, l)[2];
-  // a 256-key tile's S takes half of the 512 columns, so it has one buffer
-  static constexpr int NSB = BLK == 256 ? 1 : 2;
+  // TMEM: S[2] by sub-tile parity (P over the first SK/2 columns of its S),
+  // O[2] by tile parity
+  static constexpr int NSB = 2;
   static constexpr int S_COL = 0;
-  static constexpr int O_COL = NSB * BLK;
-  static constexpr int ML_COL = O_COL + 2 * 128;
-  static_assert(O_COL + 2 * 128 <= 512, "tensor memory");
-  static_assert(!ML_TMEM || ML_COL + 4 <= 512, "tensor memory");
+  static constexpr int O_COL = NSB * SK;
+  static_assert(O_COL + 2 * D <= 512, "tensor memory");
   static_assert(USED <= 232448, "shared memory");
 };
 
@@ -453,8 +462,8 @@ struct BlkArgs {
   int32_t n_q, n_kv, h_q, h_kv, topk, window, nsl;
   int64_t q_offset;
   float scale_log2;
-  __half* partO;             // [items][nsl][G][D], o / 2^e
-  float2* partL;             // [items][nsl][G]: (log2-sum-exp, 2^e)
+  __half* partO;             // [items][nsl][G][D], o / 2^e per 64-dim half
+  float2* partL;             // [items][nsl][G]: (log2-sum-exp, e0 | e1 << 16 as int16s)
   uint32_t* err;
 };
 
@@ -509,12 +518,10 @@ __device__ __forceinline__ void tmem_ld64(uint32_t taddr, uint32_t (&r)[64]) {
 // its block field, loaded into the two halves; a single-block tile loads its
 // block into both halves and its softmax leaves the second half out (P = 0
 // there).
-template <int G, int BLK, bool PAIR>
+template <int G, int BLK>
 __global__ void __maxnreg__((BlkCfg<G, BLK>::MAXREG))
     attn_block_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                       const __grid_constant__ CUtensorMap tmQ, const BlkArgs a) {
-  static_assert(!PAIR || BLK == 128 || BLK == 256, "pairs fill 128- or 256-key tiles");
-  static_assert(PAIR || BLK != 256, "256-key tiles are pairs");
   using C = BlkCfg<G, BLK>;
   constexpr int D = C::D;
   constexpr int QPT = 128 / G;
@@ -527,30 +534,33 @@ __global__ void __maxnreg__((BlkCfg<G, BLK>::MAXREG))
   }
   uint8_t* sA = smem;                                   // [NA][A_BYTES]
   uint8_t* sKV = sA + NA * C::A_BYTES;                  // [NKV][KV_BYTES]
-  uint8_t* sStg = sKV + C::NKV * C::KV_BYTES;           // [2][STG_BYTES] epilogue staging
-  float2* sML = reinterpret_cast<float2*>(sStg + 2 * C::STG_BYTES);   // [2][128] when not in TMEM
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sStg + 2 * C::STG_BYTES + C::ML_BYTES);
+  uint8_t* sStg = sKV + C::NKV * C::KV_BYTES;           // [8][STG_WARP] epilogue staging
+  float4* sML = reinterpret_cast<float4*>(sStg + 8 * C::STG_WARP);   // [2][128]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sStg + 8 * C::STG_WARP + C::ML_BYTES);
   uint64_t* a_full = bars;                  // [NA] gather warp arrives once its copies landed
   uint64_t* a_empty = a_full + NA;          // [NA]
   uint64_t* kv_full = a_empty + NA;         // [NKV]
   uint64_t* kv_empty = kv_full + C::NKV;    // [NKV]
-  uint64_t* s_full = kv_empty + C::NKV;     // [2]
-  uint64_t* s_empty = s_full + 2;           // [2]
-  uint64_t* p_full = s_empty + 2;           // [2]
-  uint64_t* o_full = p_full + 2;            // [2]
+  uint64_t* s_full = kv_empty + C::NKV;     // [2][SUB]
+  uint64_t* p_full = s_full + 2 * C::SUB;   // [2][SUB]
+  uint64_t* s_empty = p_full + 2 * C::SUB;  // [2] by S buffer
+  uint64_t* o_full = s_empty + 2;           // [2]
   uint64_t* o_empty = o_full + 2;           // [2]
-  uint64_t* ml_empty = o_empty + 2;         // [2] the epilogue has read a tile's (m, l)
-  uint64_t* mma_done = ml_empty + 2;
+  uint64_t* ml_empty = o_empty + 2;         // [2]
+  uint64_t* pa_done = ml_empty + 2;         // [2]
+  uint64_t* mma_done = pa_done + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   if (threadIdx.x == 0) {
     for (int i = 0; i < NA; ++i) { mbar_init(&a_full[i], 1); mbar_init(&a_empty[i], 1); }
     for (int i = 0; i < C::NKV; ++i) { mbar_init(&kv_full[i], 1); mbar_init(&kv_empty[i], 1); }
+    for (int i = 0; i < 2 * C::SUB; ++i) { mbar_init(&s_full[i], 1); mbar_init(&p_full[i], 4); }
     for (int i = 0; i < 2; ++i) {
-      mbar_init(&s_full[i], 1); mbar_init(&s_empty[i], 1);
-      mbar_init(&p_full[i], 4); mbar_init(&o_full[i], 1); mbar_init(&o_empty[i], 4);
+      mbar_init(&s_empty[i], 1);
+      mbar_init(&o_full[i], 1); mbar_init(&o_empty[i], 4);
       mbar_init(&ml_empty[i], 4);
+      mbar_init(&pa_done[i], 1);
     }
     mbar_init(mma_done, 1);
     fence_barrier_init();
@@ -594,19 +604,13 @@ __global__ void __maxnreg__((BlkCfg<G, BLK>::MAXREG))
         mbar_arrive_expect_tx(&kv_full[kb], C::KV_BYTES);
         // first key of each 64-key half of the tile
         int zs[BLK / 64];
-        if (PAIR) {
-          constexpr int KPB = BLK / 2;   // keys per block of the pair
-          const int c1 = pair_tile_c1(td.y), c2 = pair_tile_c2(td.y);
+        constexpr int KPB = BLK / 2;   // keys per block of the pair
+        const int c1 = pair_tile_c1(td.y), c2 = pair_tile_c2(td.y);
 #pragma unroll
-          for (int sub = 0; sub < BLK / 64; ++sub) {
-            const int src = sub * 64 < KPB ? c1 : (c2 >= 0 ? c2 : c1);
-            zs[sub] = static_cast<int>(static_cast<int64_t>(b) * a.n_kv + static_cast<int64_t>(src) * KPB +
-                                       (sub * 64) % KPB);
-          }
-        } else {
-#pragma unroll
-          for (int sub = 0; sub < BLK / 64; ++sub)
-            zs[sub] = static_cast<int>(static_cast<int64_t>(b) * a.n_kv + static_cast<int64_t>(td.y) * BLK + sub * 64);
+        for (int sub = 0; sub < BLK / 64; ++sub) {
+          const int src = sub * 64 < KPB ? c1 : (c2 >= 0 ? c2 : c1);
+          zs[sub] = static_cast<int>(static_cast<int64_t>(b) * a.n_kv + static_cast<int64_t>(src) * KPB +
+                                     (sub * 64) % KPB);
         }
 #pragma unroll
         for (int sub = 0; sub < BLK / 64; ++sub) {
@@ -627,14 +631,16 @@ __global__ void __maxnreg__((BlkCfg<G, BLK>::MAXREG))
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      constexpr int SN = BLK;
-      constexpr uint32_t IDESC1 = umma_idesc_bf16(128, SN);
+      constexpr int SK = C::SK, SUB = C::SUB;
+      constexpr uint32_t IDESC1 = umma_idesc_bf16(128, SK);
       constexpr uint32_t IDESC2 = umma_idesc_bf16(128, D) | (1u << 16);   // B (V) is MN-major
       const uint32_t sA_u = smem_u32(sA), sKV_u = smem_u32(sKV);
-      int n1 = 0, n2 = 0;               // tiles whose S = Q K^T / O = P V are issued
+      // sub-tiles u = SUB tile + sub whose S = Q K^T / O += P V are issued
+      int u1 = 0, u2 = 0;
+      const int U = T * SUB;
       int kv_ord = -1;
       int64_t prev = -1;
-      uint32_t ring_kb = 0, ring_last = 0;   // bit (n & 3) per issued S, read by its P V
+      uint32_t ring_kb = 0, ring_last = 0;   // bit (n & 3) per tile in flight, read by its P V
       int4 cur = T > 0 ? a.tiles[t0] : none;
       int4 nxt = T > 1 ? a.tiles[t0 + 1] : none;
       int4 nxt2 = T > 2 ? a.tiles[t0 + 2] : none;
@@ -643,64 +649,72 @@ __global__ void __maxnreg__((BlkCfg<G, BLK>::MAXREG))
       uint64_t last_progress = global_timer_ns();
       uint32_t spins = 0;
       bool ok = true;
-      while (n2 < T) {
+      while (u2 < U) {
         bool progressed = false;
-        if (n1 < T && n1 - n2 < 4) {
+        const int n1 = u1 / SUB, s1 = u1 % SUB;
+        if (u1 < U && n1 - u2 / SUB < 4) {
           const int ab = n1 % NA;
           const int ord = kv_ord + (fresh ? 1 : 0);
-          if ((!fresh || mbar_test_wait(&kv_full[kb], (ord / C::NKV) & 1)) &&
-              mbar_test_wait(&a_full[ab], (n1 / NA) & 1) &&
-              // S(n1) reuses the S columns of tile n1 - NSB once its P V has
-              // read them; barriers go by tile parity, each waited on in order
-              (n1 < C::NSB ||
-               mbar_test_wait(&s_empty[(n1 - C::NSB) & 1], ((n1 - C::NSB) >> 1) & 1))) {
+          // a tile's first sub-tile waits for its K, V and Q rows; S(u1)
+          // reuses the S columns of sub-tile u1 - NSB once its P V has read
+          // them (each barrier waited on in order)
+          if ((s1 > 0 || ((!fresh || mbar_test_wait(&kv_full[kb], (ord / C::NKV) & 1)) &&
+                          mbar_test_wait(&a_full[ab], (n1 / NA) & 1))) &&
+              (u1 < C::NSB ||
+               mbar_test_wait(&s_empty[(u1 - C::NSB) & 1], ((u1 - C::NSB) >> 1) & 1))) {
             tc_fence_after();
-            const uint32_t s_tmem = tmem_base + C::S_COL + (n1 % C::NSB) * BLK;
-            const uint32_t kbase = sKV_u + kb * C::KV_BYTES;
+            const uint32_t s_tmem = tmem_base + C::S_COL + (u1 & 1) * SK;
+            const uint32_t kbase = sKV_u + kb * C::KV_BYTES + s1 * SK * C::ROW;
 #pragma unroll
             for (int ks = 0; ks < D / 16; ++ks) {
               const uint64_t ad = umma_desc_sw128(sA_u + ab * C::A_BYTES + (ks >> 2) * C::A_HALF + (ks & 3) * 32);
-#pragma unroll
-              for (int np = 0; np < BLK / SN; ++np) {
-                const uint64_t bd =
-                    umma_desc_sw128(kbase + (ks >> 2) * C::KV_HALF + np * SN * C::ROW + (ks & 3) * 32);
-                umma_bf16(s_tmem + np * SN, ad, bd, IDESC1, ks != 0 ? 1u : 0u);
-              }
+              const uint64_t bd = umma_desc_sw128(kbase + (ks >> 2) * C::KV_HALF + (ks & 3) * 32);
+              umma_bf16(s_tmem, ad, bd, IDESC1, ks != 0 ? 1u : 0u);
             }
-            umma_commit(&s_full[n1 & 1]);
-            umma_commit(&a_empty[ab]);
-            if (fresh) { kv_ord = ord; prev = tile_key(cur); }
-            const uint32_t bit = 1u << (n1 & 3);
-            ring_kb = kb ? (ring_kb | bit) : (ring_kb & ~bit);
-            ring_last = (n1 + 1 == T || tile_key(nxt) != tile_key(cur)) ? (ring_last | bit) : (ring_last & ~bit);
-            ++n1;
-            cur = nxt;
-            nxt = nxt2;
-            nxt2 = n1 + 2 < T ? a.tiles[t0 + n1 + 2] : none;
-            fresh = tile_key(cur) != prev;
-            kb = (kv_ord + (fresh ? 1 : 0)) % C::NKV;
+            umma_commit(&s_full[(n1 & 1) * SUB + s1]);
+            if (s1 == 0) {   // the tile's K/V buffer, and whether it is the buffer's last tile
+              const uint32_t bit = 1u << (n1 & 3);
+              ring_kb = kb ? (ring_kb | bit) : (ring_kb & ~bit);
+              ring_last = (n1 + 1 == T || tile_key(nxt) != tile_key(cur)) ? (ring_last | bit) : (ring_last & ~bit);
+            }
+            if (s1 == SUB - 1) {   // the tile's Q rows are read
+              umma_commit(&a_empty[ab]);
+              if (fresh) { kv_ord = ord; prev = tile_key(cur); }
+              cur = nxt;
+              nxt = nxt2;
+              nxt2 = n1 + 3 < T ? a.tiles[t0 + n1 + 3] : none;
+              fresh = tile_key(cur) != prev;
+              kb = (kv_ord + (fresh ? 1 : 0)) % C::NKV;
+            }
+            ++u1;
             progressed = true;
           }
         }
-        if (n2 < n1) {
+        if (u2 < u1) {
+          const int n2 = u2 / SUB, s2 = u2 % SUB;
           const int ob = n2 & 1;
-          if (mbar_test_wait(&p_full[ob], (n2 >> 1) & 1) && mbar_test_wait(&o_empty[ob], ((n2 >> 1) & 1) ^ 1)) {
+          if (mbar_test_wait(&p_full[ob * SUB + s2], (n2 >> 1) & 1) &&
+              (s2 > 0 || mbar_test_wait(&o_empty[ob], ((n2 >> 1) & 1) ^ 1))) {
             tc_fence_after();
             const int kb2 = (ring_kb >> (n2 & 3)) & 1;
             const uint32_t d_tmem = tmem_base + C::O_COL + ob * D;
-            // P (bf16, two per column) sits over the first BLK/2 columns of
-            // this tile's S; 16 keys = 8 columns per step
-            const uint32_t p_tmem = tmem_base + C::S_COL + (n2 % C::NSB) * BLK;
-            const uint32_t vbase = sKV_u + kb2 * C::KV_BYTES + 2 * C::KV_HALF;
+            // P (bf16, two per column) sits over the first SK/2 columns of
+            // this sub-tile's S; 16 keys = 8 columns per step
+            const uint32_t p_tmem = tmem_base + C::S_COL + (u2 & 1) * SK;
+            const uint32_t vbase = sKV_u + kb2 * C::KV_BYTES + 2 * C::KV_HALF + s2 * SK * C::ROW;
 #pragma unroll
-            for (int kk = 0; kk < BLK / 16; ++kk) {
+            for (int kk = 0; kk < SK / 16; ++kk) {
               const uint64_t bd = umma_desc_sw128_mn(vbase + kk * 16 * C::ROW, C::KV_HALF, 1024);
-              umma_bf16_tmem_a(d_tmem, p_tmem + kk * 8, bd, IDESC2, kk != 0 ? 1u : 0u);
+              umma_bf16_tmem_a(d_tmem, p_tmem + kk * 8, bd, IDESC2, (s2 != 0 || kk != 0) ? 1u : 0u);
             }
-            umma_commit(&o_full[ob]);
-            umma_commit(&s_empty[n2 & 1]);   // P read: the S / P columns may take tile n2 + NSB
-            if ((ring_last >> (n2 & 3)) & 1) umma_commit(&kv_empty[kb2]);
-            ++n2;
+            umma_commit(&s_empty[u2 & 1]);   // P read: the S / P columns may take sub-tile u2 + NSB
+            if (s2 == SUB - 1) {
+              umma_commit(&o_full[ob]);
+              if ((ring_last >> (n2 & 3)) & 1) umma_commit(&kv_empty[kb2]);
+            } else {
+              umma_commit(&pa_done[ob]);
+            }
+            ++u2;
             progressed = true;
           }
         }
@@ -734,8 +748,8 @@ __global__ void __maxnreg__((BlkCfg<G, BLK>::MAXREG))
     const int row = eq * 32 + lane;
     const int e = row / G, h = row % G;
     const uint32_t lane_base = static_cast<uint32_t>(eq * 32) << 16;
-    // this warp's 32 staging rows (a 64-dim half of each)
-    uint8_t* stage = sStg + grp * C::STG_BYTES + eq * 32 * C::ROW;
+    // this warp's 32 staging rows (32 dims of each)
+    uint8_t* stage = sStg + (grp * 4 + eq) * C::STG_WARP;
     auto tile_at = [&](int x) { return (x >= 0 && x < T) ? a.tiles[t0 + x] : none; };
     auto entry_of = [&](const int4& td) { return e < td.w ? __ldg(a.entries + td.z + e) : 0; };
     // the epilogue's tile descriptors two tiles ahead and this thread's entry
@@ -752,82 +766,115 @@ __global__ void __maxnreg__((BlkCfg<G, BLK>::MAXREG))
       e_td = e_td2; e_td2 = tile_at(te + 4);
       e_ent = entry_of(e_td);
       if (ts < T) {
-        // ---------------- softmax of tile ts: P = 2^(s - m) in bf16 over S
-        // barriers and the (m, l) slot by tile parity (each group waits on
-        // its own barriers, in order); the S columns by buffer
+        // ---------------- softmax of tile ts: P = 2^(x - m) in bf16 of the
+        // scaled scores x over the S columns, one 128-key sub-tile after the
+        // other.  A sub-tile's maximum over its two 64-key halves comes
+        // first (one pass over S), then the powers and the row sums (a
+        // second).  Barriers and the (m, l) slot go by tile parity (each
+        // group waits on its own barriers, in order), S columns by sub-tile
+        // parity.  A second sub-tile keeps the first one's maximum m unless
+        // its own exceeds m by more than kStaleMax: then that row's m moves
+        // up, and its O (complete for the first sub-tile) and l are rescaled.
         const int sb = ts & 1, use = ts >> 1;
-        ok = __all_sync(0xFFFFFFFFu, mbar_wait(&s_full[sb], use & 1, a.err, SITE_BLK_S_FULL));
-        if (!ok) break;
-        tc_fence_after();
-        const uint32_t scol = tmem_base + lane_base + C::S_COL + (ts % C::NSB) * BLK;
-        auto load_half = [&](int hf, uint32_t (&r)[64]) { tmem_ld64(scol + hf * 64, r); };
-        // pair mode: a single-block tile holds keys in its first half only
-        // (tile-uniform)
-        const int nhalf = (PAIR && pair_tile_c2(tile_at(ts).y) < 0) ? BLK / 128 : BLK / 64;
-        // maxima and sums in eight independent chains
-        float mx[8] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY, -INFINITY, -INFINITY, -INFINITY, -INFINITY};
-        float ls[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-        float m = -INFINITY;
-        if (BLK > 64) {   // first pass: the maximum over both halves
+        const bool single = pair_tile_c2(tile_at(ts).y) < 0;   // keys in the first BLK / 2 only
+        // l sums P in float32 (the tile's log-sum-exp).  lr, the normaliser
+        // of O, adds to it the bf16 rounding of each sub-tile's largest P:
+        // P V multiplies the rounded P, so a key that dominates the row
+        // divides out exactly (its P is 1 unless a kept maximum leaves it
+        // anywhere in (1, 2^kStaleMax]); the other keys' roundings stay
+        // below 2^-9 of their weights either way.
+        float m = -INFINITY, l = 0.f, lr = 0.f;
+        for (int s = 0; s < C::SUB; ++s) {
+          ok = __all_sync(0xFFFFFFFFu, mbar_wait(&s_full[sb * C::SUB + s], use & 1, a.err, SITE_BLK_S_FULL));
+          if (!ok) break;
+          tc_fence_after();
+          const uint32_t scol = tmem_base + lane_base + C::S_COL + ((ts * C::SUB + s) & 1) * C::SK;
+          const int nhalf = !single ? 2 : (C::SUB == 2 ? (s == 0 ? 2 : 0) : 1);   // halves holding keys
+          // maxima and sums in independent chains
+          float mx[8] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY, -INFINITY, -INFINITY, -INFINITY, -INFINITY};
+          float ls[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-          for (int hf = 0; hf < BLK / 64; ++hf) {
+          for (int hf = 0; hf < 2; ++hf) {
             if (hf >= nhalf) break;
             uint32_t r[64];
-            load_half(hf, r);
+            tmem_ld64(scol + hf * 64, r);
 #pragma unroll
             for (int u = 0; u < 64; ++u) mx[u & 7] = fmaxf(mx[u & 7], __uint_as_float(r[u]));
           }
-          m = max8(mx) * a.scale_log2;
-        }
-        // P of half hf goes to columns hf*32 .. hf*32+31: the S columns it
-        // covers are already in registers (half 0) or consumed (half 1)
+          const float raw_max = max8(mx);
+          const float mt = raw_max * a.scale_log2;
+          if (s == 0) {
+            m = mt;
+          } else {
+            const bool up = mt > m + kStaleMax;
+            if (__any_sync(0xFFFFFFFFu, up)) {   // warp-uniform: the TMEM accesses are collective
+              const float alpha = up ? fast_exp2(m - mt) : 1.f;
+              if (up) m = mt;
+              l *= alpha;
+              lr *= alpha;
+              ok = __all_sync(0xFFFFFFFFu, mbar_wait(&pa_done[sb], use & 1, a.err, SITE_BLK_O_FULL));
+              if (!ok) break;
+              tc_fence_after();
+              const uint32_t ocol = tmem_base + lane_base + C::O_COL + sb * D;
 #pragma unroll
-        for (int hf = 0; hf < BLK / 64; ++hf) {
-          if (hf >= nhalf) {   // no keys: P = 0 over this half's 32 columns
-            uint32_t pw[16];
+              for (int hf = 0; hf < D / 64; ++hf) {
+                uint32_t r[64];
+                tmem_ld64(ocol + hf * 64, r);
 #pragma unroll
-            for (int u = 0; u < 16; ++u) pw[u] = 0u;
-            tmem_st16(scol + hf * 32, pw);
-            tmem_st16(scol + hf * 32 + 16, pw);
-            continue;
-          }
-          uint32_t r[64];
-          load_half(hf, r);
-          if (BLK == 64) {
+                for (int u = 0; u < 64; ++u) r[u] = __float_as_uint(__uint_as_float(r[u]) * alpha);
 #pragma unroll
-            for (int u = 0; u < 64; ++u) mx[u & 7] = fmaxf(mx[u & 7], __uint_as_float(r[u]));
-            m = max8(mx) * a.scale_log2;
-          }
-#pragma unroll
-          for (int qq = 0; qq < 2; ++qq) {   // 32 keys = 16 columns of P per store
-            uint32_t pw[16];
-#pragma unroll
-            for (int u = 0; u < 16; ++u) {
-              const int c = qq * 32 + 2 * u;
-              const float p0 = fast_exp2(fmaf(__uint_as_float(r[c]), a.scale_log2, -m));
-              const float p1 = fast_exp2(fmaf(__uint_as_float(r[c + 1]), a.scale_log2, -m));
-              ls[c & 7] += p0;
-              ls[(c + 1) & 7] += p1;
-              pw[u] = pack_bf16(p0, p1);
+                for (int q = 0; q < 4; ++q)
+                  tmem_st16(ocol + hf * 64 + q * 16, *reinterpret_cast<const uint32_t(*)[16]>(&r[q * 16]));
+              }
             }
-            tmem_st16(scol + hf * 32 + qq * 16, pw);
           }
+          // P of half hf goes to columns hf*32 .. hf*32+31: the S columns it
+          // covers are already in registers (half 0) or consumed (half 1)
+#pragma unroll
+          for (int hf = 0; hf < 2; ++hf) {
+            if (hf >= nhalf) {   // no keys: P = 0 over this half's 32 columns
+              uint32_t pw[16];
+#pragma unroll
+              for (int u = 0; u < 16; ++u) pw[u] = 0u;
+              tmem_st16(scol + hf * 32, pw);
+              tmem_st16(scol + hf * 32 + 16, pw);
+              continue;
+            }
+            uint32_t r[64];
+            tmem_ld64(scol + hf * 64, r);
+#pragma unroll
+            for (int qq = 0; qq < 2; ++qq) {   // 32 keys = 16 columns of P per store
+              uint32_t pw[16];
+#pragma unroll
+              for (int u = 0; u < 16; ++u) {
+                const int c = qq * 32 + 2 * u;
+                const float p0 = fast_exp2(fmaf(__uint_as_float(r[c]), a.scale_log2, -m));
+                const float p1 = fast_exp2(fmaf(__uint_as_float(r[c + 1]), a.scale_log2, -m));
+                ls[c & 7] += p0;
+                ls[(c + 1) & 7] += p1;
+                pw[u] = pack_bf16(p0, p1);
+              }
+              tmem_st16(scol + hf * 32 + qq * 16, pw);
+            }
+          }
+          const float ps = ((ls[0] + ls[1]) + (ls[2] + ls[3])) + ((ls[4] + ls[5]) + (ls[6] + ls[7]));
+          // the sub-tile's largest P, computed as its element's own was
+          const float pmax = nhalf > 0 ? fast_exp2(fmaf(raw_max, a.scale_log2, -m)) : 0.f;
+          l += ps;
+          lr += ps + (__bfloat162float(__float2bfloat16_rn(pmax)) - pmax);
+          if (s == C::SUB - 1) {
+            // (m, l) into this parity's slot once the epilogue two tiles back read it
+            ok = __all_sync(0xFFFFFFFFu, mbar_wait(&ml_empty[sb], (use & 1) ^ 1, a.err, SITE_BLK_ML_EMPTY));
+            if (!ok) break;
+            tc_fence_after();
+            sML[sb * 128 + row] = make_float4(m, l, lr, 0.f);
+          }
+          tmem_wait_st();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&p_full[sb * C::SUB + s]);
         }
-        const float l = ((ls[0] + ls[1]) + (ls[2] + ls[3])) + ((ls[4] + ls[5]) + (ls[6] + ls[7]));
-        // (m, l) into this parity's slot once the epilogue two tiles back read it
-        ok = __all_sync(0xFFFFFFFFu, mbar_wait(&ml_empty[sb], (use & 1) ^ 1, a.err, SITE_BLK_ML_EMPTY));
         if (!ok) break;
-        tc_fence_after();
-        if (C::ML_TMEM) {
-          const uint32_t mlv[2] = {__float_as_uint(m), __float_as_uint(l)};
-          tmem_st2(tmem_base + lane_base + C::ML_COL + sb * 2, mlv);
-        } else {
-          sML[sb * 128 + row] = make_float2(m, l);
-        }
-        tmem_wait_st();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&p_full[sb]);
       }
       if (te >= 0 && te < T) {
         // ---------------- epilogue of tile te: o = O / l as scaled float16
@@ -836,53 +883,37 @@ __global__ void __maxnreg__((BlkCfg<G, BLK>::MAXREG))
         const int i = entry_row(eent), j = entry_slot(eent);
         const bool valid = e < ne && static_cast<unsigned>(i) < static_cast<unsigned>(a.n_q) && j < a.topk;
         // the softmax's (m, l) are published with P (p_full); O follows P V
-        ok = __all_sync(0xFFFFFFFFu, mbar_wait(&p_full[ob], use & 1, a.err, SITE_BLK_O_FULL) &&
+        ok = __all_sync(0xFFFFFFFFu, mbar_wait(&p_full[ob * C::SUB + C::SUB - 1], use & 1, a.err, SITE_BLK_O_FULL) &&
                                          mbar_wait(&o_full[ob], use & 1, a.err, SITE_BLK_O_FULL));
         if (!ok) break;
         tc_fence_after();
-        float m, l;
-        if (C::ML_TMEM) {
-          uint32_t mlv[2];
-          tmem_ld2(tmem_base + lane_base + C::ML_COL + ob * 2, mlv);
-          tmem_wait_ld();
-          tmem_regs_ready(mlv);
-          m = __uint_as_float(mlv[0]);
-          l = __uint_as_float(mlv[1]);
-        } else {
-          const float2 ml = sML[ob * 128 + row];
-          m = ml.x;
-          l = ml.y;
-        }
+        const float4 ml = sML[ob * 128 + row];
+        const float m = ml.x, l = ml.y, lr = ml.z;
         // (m, l) read: its slot may take the next tile of this parity
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&ml_empty[ob]);
-        // two passes over the row in halves of 64 columns: its largest
-        // magnitude, then the scaled float16 conversion
-        const uint32_t ocol = tmem_base + lane_base + C::O_COL + ob * D;
-        float am[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-        for (int hf = 0; hf < D / 64; ++hf) {
-          uint32_t r[64];
-          tmem_ld64(ocol + hf * 64, r);
-#pragma unroll
-          for (int u = 0; u < 64; ++u) am[u & 7] = fmaxf(am[u & 7], fabsf(__uint_as_float(r[u])));
-        }
-        const float amax = max8(am);
-        // the normalised row o = O / l, stored as float16 times 2^-e with the
-        // power of two 2^e chosen so the row's largest entry lands in
+        // One pass over the row in halves of 64 dims: the normalised
+        // o = O / lr of each half stored as float16 times 2^-e, the power of
+        // two 2^e chosen per half so its largest entry lands in
         // [2^14, 2^15): 11 significant bits whatever the scale of V.  Every
         // lane runs the (warp-collective) TMEM loads; only valid rows store.
-        const float inv_l = 1.f / l;
-        const float x = amax * inv_l;
-        int ex = x > 0.f ? static_cast<int>((__float_as_uint(x) >> 23) & 0xFFu) - 127 - 14 : 0;
-        ex = min(max(ex, -100), 100);
-        const float mul = inv_l * __uint_as_float(static_cast<uint32_t>(127 - ex) << 23);
+        const uint32_t ocol = tmem_base + lane_base + C::O_COL + ob * D;
+        const float inv_l = 1.f / lr;
         const int64_t slot = ((static_cast<int64_t>(bg) * a.n_q + i) * a.nsl + j) * G + h;
-        // Coalesced stores: each warp passes its 32 rows through its own 32
-        // staging rows, 16-byte chunks XOR-swizzled by row against bank
-        // conflicts, then writes four whole 128-byte half-rows per instruction.
-        const int srow = lane >> 3, sch = lane & 7;   // store phase: row k*4 + srow, chunk sch
+        // Coalesced stores: the warp's 32 rows pass through its staging rows
+        // 32 dims at a time (16-byte chunk c of row r at r * 64 +
+        // 16 (c ^ ((r >> 1) & 3)), free of bank conflicts), then eight rows of
+        // 64 bytes go out per instruction.  Lane l stores rows 8 k + l / 4.
+        const int srow = lane >> 2, sch = lane & 3;
+        int64_t rslot[4];
+        bool rvalid[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          rslot[k] = __shfl_sync(0xFFFFFFFFu, slot, k * 8 + srow);
+          rvalid[k] = __shfl_sync(0xFFFFFFFFu, valid ? 1 : 0, k * 8 + srow) != 0;
+        }
+        uint32_t exs = 0;   // the two halves' exponents, 16 bits each
 #pragma unroll
         for (int hf = 0; hf < D / 64; ++hf) {
           uint32_t r[64];
@@ -892,29 +923,39 @@ __global__ void __maxnreg__((BlkCfg<G, BLK>::MAXREG))
             __syncwarp();
             if (lane == 0) mbar_arrive(&o_empty[ob]);
           }
+          float am[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-          for (int q = 0; q < 8; ++q) {
-            uint32_t w[4];
+          for (int x = 0; x < 64; ++x) am[x & 7] = fmaxf(am[x & 7], fabsf(__uint_as_float(r[x])));
+          const float xm = max8(am) * inv_l;
+          int ex = xm > 0.f ? static_cast<int>((__float_as_uint(xm) >> 23) & 0xFFu) - 127 - 14 : 0;
+          ex = min(max(ex, -100), 100);
+          exs |= (static_cast<uint32_t>(ex) & 0xFFFFu) << (16 * hf);
+          const float mul = inv_l * __uint_as_float(static_cast<uint32_t>(127 - ex) << 23);
 #pragma unroll
-            for (int u = 0; u < 4; ++u) {
-              const __half2 hv = __floats2half2_rn(__uint_as_float(r[q * 8 + 2 * u]) * mul,
-                                                   __uint_as_float(r[q * 8 + 2 * u + 1]) * mul);
-              w[u] = *reinterpret_cast<const uint32_t*>(&hv);
+          for (int qh = 0; qh < 2; ++qh) {
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {   // 8 dims = 16 bytes
+              uint32_t w[4];
+#pragma unroll
+              for (int u = 0; u < 4; ++u) {
+                const int c = qh * 32 + q * 8 + 2 * u;
+                const __half2 hv = __floats2half2_rn(__uint_as_float(r[c]) * mul, __uint_as_float(r[c + 1]) * mul);
+                w[u] = *reinterpret_cast<const uint32_t*>(&hv);
+              }
+              *reinterpret_cast<uint4*>(stage + lane * 64 + ((q ^ ((lane >> 1) & 3)) << 4)) =
+                  make_uint4(w[0], w[1], w[2], w[3]);
             }
-            *reinterpret_cast<uint4*>(stage + lane * C::ROW + ((q ^ (lane & 7)) << 4)) = make_uint4(w[0], w[1], w[2], w[3]);
-          }
-          __syncwarp();
+            __syncwarp();
 #pragma unroll
-          for (int k = 0; k < 8; ++k) {
-            const int rr = k * 4 + srow;   // the warp lane whose row this is
-            const int64_t rslot = __shfl_sync(0xFFFFFFFFu, slot, rr);
-            const bool rvalid = __shfl_sync(0xFFFFFFFFu, valid ? 1 : 0, rr) != 0;
-            const uint4 v = *reinterpret_cast<const uint4*>(stage + rr * C::ROW + ((sch ^ (rr & 7)) << 4));
-            if (rvalid) reinterpret_cast<uint4*>(a.partO + rslot * D + hf * 64)[sch] = v;
+            for (int k = 0; k < 4; ++k) {
+              const int rr = k * 8 + srow;
+              const uint4 v = *reinterpret_cast<const uint4*>(stage + rr * 64 + ((sch ^ ((rr >> 1) & 3)) << 4));
+              if (rvalid[k]) reinterpret_cast<uint4*>(a.partO + rslot[k] * D + hf * 64 + qh * 32)[sch] = v;
+            }
+            __syncwarp();
           }
-          __syncwarp();
         }
-        if (valid) a.partL[slot] = make_float2(m + log2f(l), __uint_as_float(static_cast<uint32_t>(127 + ex) << 23));
+        if (valid) a.partL[slot] = make_float2(m + log2f(l), __uint_as_float(exs));
       }
     }
   } else {
@@ -1069,28 +1110,43 @@ __global__ void __launch_bounds__(256, (G == 8 ? 2 : (G == 4 ? 3 : 4))) attn_mer
   s.mask = static_cast<uint64_t>(ri.x) | (static_cast<uint64_t>(wch) << a.topk);
   const float2* pl = a.partL + item * a.nsl * G;
   const __half* po = a.partO + item * a.nsl * G * D;
-  // per head: this lane's slots lane and lane + 32, their weights 2^(L-M) 2^e
-  float w0[G], w1[G], inv_den[G], lse2[G];
-  const bool has0 = (s.mask >> lane) & 1, has1 = (s.mask >> (lane + 32)) & 1;
+  // Per head, the slots' weights 2^(L - M) 2^e, e the slot's exponent for
+  // the 64-dim half this lane accumulates (lanes 0-15: dims 0-63, lanes
+  // 16-31: dims 64-127): lane i of each 16-lane half holds slots i, i + 16,
+  // i + 32, i + 48, so one 16-wide shuffle hands every lane the weight of
+  // its own half.
+  const int li = lane & 15, eshift = (lane >> 4) * 16;
+  float w[4][G], inv_den[G], lse2[G];
 #pragma unroll
   for (int h = 0; h < G; ++h) {
-    const float2 l0 = has0 ? pl[lane * G + h] : make_float2(-INFINITY, 0.f);
-    const float2 l1 = has1 ? pl[(lane + 32) * G + h] : make_float2(-INFINITY, 0.f);
-    float M = fmaxf(l0.x, l1.x);
+    float2 lv[4];
+    bool hv[4];
+    float M = -INFINITY;
 #pragma unroll
-    for (int o = 16; o; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xFFFFFFFFu, M, o));
-    const float f0 = has0 ? fast_exp2(l0.x - M) : 0.f, f1 = has1 ? fast_exp2(l1.x - M) : 0.f;
-    float den = f0 + f1;
+    for (int k = 0; k < 4; ++k) {
+      const int j = li + 16 * k;
+      hv[k] = (s.mask >> j) & 1;
+      lv[k] = hv[k] ? pl[j * G + h] : make_float2(-INFINITY, 0.f);
+      M = fmaxf(M, lv[k].x);
+    }
 #pragma unroll
-    for (int o = 16; o; o >>= 1) den += __shfl_xor_sync(0xFFFFFFFFu, den, o);
-    w0[h] = f0 * l0.y;
-    w1[h] = f1 * l1.y;
+    for (int o = 8; o; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xFFFFFFFFu, M, o));
+    float den = 0.f;
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const float f = hv[k] ? fast_exp2(lv[k].x - M) : 0.f;
+      den += f;
+      const int e = static_cast<int16_t>((__float_as_uint(lv[k].y) >> eshift) & 0xFFFFu);   // |e| <= 100
+      w[k][h] = f * __uint_as_float(static_cast<uint32_t>(127 + e) << 23);
+    }
+#pragma unroll
+    for (int o = 8; o; o >>= 1) den += __shfl_xor_sync(0xFFFFFFFFu, den, o);
     inv_den[h] = 1.f / den;
     lse2[h] = M + log2f(den);
   }
   // every lane accumulates dims 4 lane .. 4 lane + 3 of every head, SU
   // slots at a time (loads of SU x G rows in flight)
-  constexpr int SU = G == 8 ? 2 : 4;
+  constexpr int SU = G == 8 ? 2 : (G == 4 ? 3 : 4);
   float acc[G][4];
 #pragma unroll
   for (int h = 0; h < G; ++h)
@@ -1114,10 +1170,13 @@ __global__ void __launch_bounds__(256, (G == 8 ? 2 : (G == 4 ? 3 : 4))) attn_mer
 #pragma unroll
     for (int q = 0; q < SU; ++q) {
       if (js[q] < 0) break;   // warp-uniform
-      const int src = js[q] & 31;
+      const int src = js[q] & 15, grp16 = js[q] >> 4;   // warp-uniform
 #pragma unroll
       for (int h = 0; h < G; ++h) {
-        const float wj = __shfl_sync(0xFFFFFFFFu, js[q] < 32 ? w0[h] : w1[h], src);
+        float wg = w[0][h];
+#pragma unroll
+        for (int k = 1; k < 4; ++k) wg = grp16 == k ? w[k][h] : wg;
+        const float wj = __shfl_sync(0xFFFFFFFFu, wg, src, 16);
         const float2 o01 = __half22float2(*reinterpret_cast<const __half2*>(&raw[q][h].x));
         const float2 o23 = __half22float2(*reinterpret_cast<const __half2*>(&raw[q][h].y));
         acc[h][0] += wj * o01.x;
@@ -1142,16 +1201,15 @@ __global__ void __launch_bounds__(256, (G == 8 ? 2 : (G == 4 ? 3 : 4))) attn_mer
   }
 }
 
-template <int G, int BLK, bool PAIR = false>
-cudaError_t run_block(const BlockPlan& pl, const CUtensorMap& tmK, const CUtensorMap& tmV, const CUtensorMap& tmQ,
-                      const BlkArgs& a, const LaunchCtx& c) {
+template <int G, int BLK>
+cudaError_t run_block(const CUtensorMap& tmK, const CUtensorMap& tmV, const CUtensorMap& tmQ, const BlkArgs& a,
+                      const LaunchCtx& c) {
   using C = BlkCfg<G, BLK>;
-  cudaError_t e = cudaFuncSetAttribute(attn_block_kernel<G, BLK, PAIR>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  cudaError_t e = cudaFuncSetAttribute(attn_block_kernel<G, BLK>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        C::SMEM);
   if (e != cudaSuccess) return e;
-  attn_block_kernel<G, BLK, PAIR><<<c.sm_count, C::THREADS, C::SMEM, c.stream>>>(tmK, tmV, tmQ, a);
+  attn_block_kernel<G, BLK><<<c.sm_count, C::THREADS, C::SMEM, c.stream>>>(tmK, tmV, tmQ, a);
   note_launch();
-  (void)pl;
   return cudaGetLastError();
 }
 
@@ -1186,7 +1244,6 @@ cudaError_t launch_attn_merge(const ssa_params& p, const uint32_t* win, const ui
   return cudaGetLastError();
 }
 
-int attn_block_smem_bytes(int block) { return block == 64 ? BlkCfg<4, 64>::SMEM : BlkCfg<4, 128>::SMEM; }
 
 cudaError_t launch_block_plan(const ssa_params& p, const int32_t* block_idx, const BlockPlan& pl,
                               const LaunchCtx& c) {
@@ -1232,10 +1289,8 @@ cudaError_t launch_block_plan(const ssa_params& p, const int32_t* block_idx, con
   note_launch();
   if (pl.grid < 1 || pl.grid > kMaxBlockGrid) return cudaErrorInvalidValue;
   const int n_chunks = (pl.max_tiles + 255) / 256;
-  // 64-key tiles (two K/V buffers): every tile alike — equal counts were
-  // measured as fast as any weighting; 128-key tiles (128-key blocks or
-  // pairs; one K/V buffer): a new block costs two tiles
-  inv_cost_kernel<<<n_chunks, 256, 0, c.stream>>>(pl, (p.block == 64 && !pl.pair) ? 0 : 8);
+  // one K/V buffer: a new tile key costs two tiles
+  inv_cost_kernel<<<n_chunks, 256, 0, c.stream>>>(pl, 8);
   note_launch();
   inv_split_kernel<<<1, 1024, 0, c.stream>>>(pl, n_chunks);
   note_launch();
@@ -1259,26 +1314,18 @@ cudaError_t launch_attn_block(const ssa_params& p, const BlockPlan& pl, const vo
   a.err = c.err;
   const int G = p.h_q / p.h_kv;
   if (p.d != 128) return cudaErrorInvalidValue;
-  if (p.block == 64 && pl.pair) {
-    if (G == 1) return run_block<1, 128, true>(pl, tmK, tmV, tmQ, a, c);
-    if (G == 2) return run_block<2, 128, true>(pl, tmK, tmV, tmQ, a, c);
-    if (G == 4) return run_block<4, 128, true>(pl, tmK, tmV, tmQ, a, c);
-    if (G == 8) return run_block<8, 128, true>(pl, tmK, tmV, tmQ, a, c);
-  } else if (p.block == 128 && pl.pair) {
-    if (G == 1) return run_block<1, 256, true>(pl, tmK, tmV, tmQ, a, c);
-    if (G == 2) return run_block<2, 256, true>(pl, tmK, tmV, tmQ, a, c);
-    if (G == 4) return run_block<4, 256, true>(pl, tmK, tmV, tmQ, a, c);
-    if (G == 8) return run_block<8, 256, true>(pl, tmK, tmV, tmQ, a, c);
-  } else if (p.block == 64) {
-    if (G == 1) return run_block<1, 64>(pl, tmK, tmV, tmQ, a, c);
-    if (G == 2) return run_block<2, 64>(pl, tmK, tmV, tmQ, a, c);
-    if (G == 4) return run_block<4, 64>(pl, tmK, tmV, tmQ, a, c);
-    if (G == 8) return run_block<8, 64>(pl, tmK, tmV, tmQ, a, c);
+  // tiles hold pairs of blocks: 128 keys for 64-key blocks, 256 for 128-key blocks
+  if (!pl.pair) return cudaErrorInvalidValue;
+  if (p.block == 64) {
+    if (G == 1) return run_block<1, 128>(tmK, tmV, tmQ, a, c);
+    if (G == 2) return run_block<2, 128>(tmK, tmV, tmQ, a, c);
+    if (G == 4) return run_block<4, 128>(tmK, tmV, tmQ, a, c);
+    if (G == 8) return run_block<8, 128>(tmK, tmV, tmQ, a, c);
   } else if (p.block == 128) {
-    if (G == 1) return run_block<1, 128>(pl, tmK, tmV, tmQ, a, c);
-    if (G == 2) return run_block<2, 128>(pl, tmK, tmV, tmQ, a, c);
-    if (G == 4) return run_block<4, 128>(pl, tmK, tmV, tmQ, a, c);
-    if (G == 8) return run_block<8, 128>(pl, tmK, tmV, tmQ, a, c);
+    if (G == 1) return run_block<1, 256>(tmK, tmV, tmQ, a, c);
+    if (G == 2) return run_block<2, 256>(tmK, tmV, tmQ, a, c);
+    if (G == 4) return run_block<4, 256>(tmK, tmV, tmQ, a, c);
+    if (G == 8) return run_block<8, 256>(tmK, tmV, tmQ, a, c);
   }
   return cudaErrorInvalidValue;
 }

@@ -55,8 +55,8 @@ struct WinArgs {
   int64_t q_offset;
   int32_t n_tiles;           // bgs * n_qt * nwc
   float scale_log2;
-  __half* partO;             // [items][nsl][G][D], o / 2^e
-  float2* partL;             // [items][nsl][G]: (log2-sum-exp, 2^e)
+  __half* partO;             // [items][nsl][G][D], o / 2^e per 64-dim half
+  float2* partL;             // [items][nsl][G]: (log2-sum-exp, e0 | e1 << 16 as int16s)
   uint32_t* err;
 };
 
@@ -448,24 +448,14 @@ __global__ void __launch_bounds__(WinCfg<G>::THREADS, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(ml_read);
       const float m = __uint_as_float(mlv[0]), l = __uint_as_float(mlv[1]);
-      float am[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-      for (int hf = 0; hf < D / 64; ++hf) {
-        uint32_t r[64];
-        win_ld64(ocol + hf * 64, r);
-#pragma unroll
-        for (int u2 = 0; u2 < 64; ++u2) am[u2 & 7] = fmaxf(am[u2 & 7], fabsf(__uint_as_float(r[u2])));
-      }
-      const float amax = fmaxf(fmaxf(fmaxf(am[0], am[1]), fmaxf(am[2], am[3])), fmaxf(fmaxf(am[4], am[5]), fmaxf(am[6], am[7])));
-      // o = O / l as float16 times 2^-e; a row with no keys in this chunk
-      // (never read by the merge) stores zeros
+      // one pass over O in halves of 64 dims: o = O / l of each half as
+      // float16 times 2^-e, e chosen per half so its largest entry lands in
+      // [2^14, 2^15); a row with no keys in this chunk (never read by the
+      // merge) stores zeros
       const float inv_l = l > 0.f ? 1.f / l : 0.f;
-      const float x = amax * inv_l;
-      int ex = x > 0.f ? static_cast<int>((__float_as_uint(x) >> 23) & 0xFFu) - 127 - 14 : 0;
-      ex = min(max(ex, -100), 100);
-      const float mul = inv_l * __uint_as_float(static_cast<uint32_t>(127 - ex) << 23);
       const int64_t slot = ((static_cast<int64_t>(w.bg) * a.n_q + i) * a.nsl + a.topk + w.s) * G + h;
       const int srow = lane >> 3, sch = lane & 7;
+      uint32_t exs = 0;   // the two halves' exponents, 16 bits each
       // the staging rows are free once the previous tile's stores have read them
 #pragma unroll
       for (int hf = 0; hf < D / 64; ++hf) {
@@ -476,6 +466,15 @@ __global__ void __launch_bounds__(WinCfg<G>::THREADS, 1)
           __syncwarp();
           if (lane == 0) mbar_arrive(o_empty);
         }
+        float am[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int u2 = 0; u2 < 64; ++u2) am[u2 & 7] = fmaxf(am[u2 & 7], fabsf(__uint_as_float(r[u2])));
+        const float x = fmaxf(fmaxf(fmaxf(am[0], am[1]), fmaxf(am[2], am[3])),
+                              fmaxf(fmaxf(am[4], am[5]), fmaxf(am[6], am[7]))) * inv_l;
+        int ex = x > 0.f ? static_cast<int>((__float_as_uint(x) >> 23) & 0xFFu) - 127 - 14 : 0;
+        ex = min(max(ex, -100), 100);
+        exs |= (static_cast<uint32_t>(ex) & 0xFFFFu) << (16 * hf);
+        const float mul = inv_l * __uint_as_float(static_cast<uint32_t>(127 - ex) << 23);
 #pragma unroll
         for (int q = 0; q < 8; ++q) {
           uint32_t wv[4];
@@ -499,9 +498,7 @@ __global__ void __launch_bounds__(WinCfg<G>::THREADS, 1)
         }
         __syncwarp();
       }
-      if (valid)
-        a.partL[slot] = make_float2(l > 0.f ? m + log2f(l) : -INFINITY,
-                                    __uint_as_float(static_cast<uint32_t>(127 + ex) << 23));
+      if (valid) a.partL[slot] = make_float2(l > 0.f ? m + log2f(l) : -INFINITY, __uint_as_float(exs));
       if (lane == 0) mbar_arrive(stg_done);
       ++u;
     }

@@ -166,7 +166,6 @@ cudaError_t launch_hier_probe(const ssa_params& p, const HierProbeArgs& a, const
 // One CTA whose bounded wait never completes (the failure-path self-test).
 cudaError_t launch_selftest_wait(const LaunchCtx& c);
 
-int attn_block_smem_bytes(int block);
 
 // Shared-memory bytes of the tiled router / gather attention (for checks).
 int route_tiled_smem_bytes(int d, int topk);

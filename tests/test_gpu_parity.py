@@ -550,6 +550,60 @@ def test_block_major_one_key_window_and_single_block():
             np.testing.assert_allclose(got[0, i, h], Vn[0, i, h // (w.h_q // w.h_kv)], atol=1e-2)
 
 
+def test_pair_tiles_when_one_block_of_the_pair_dominates():
+    """256-key pair tiles (128-key blocks, G = 8) where one block's logits
+    stand far above the other's: keys of one block of every pair are scaled
+    by 8 (exact in bf16).  When the second block dominates, the softmax of
+    the tile's second 128-key sub-tile must raise the running maximum and
+    rescale the first sub-tile's O and row sum; when the first dominates,
+    the second sub-tile's P stays far below 1.  Both against the oracle."""
+    w = Workload("c", 141, 1, 3072, 8, 1, 128, "bf16", 128, "diag", 2, 256, 4, "total")
+    Q, K, V, _ = make_inputs(w, "cpu")
+    pd = problem_dict(w)
+    op = O.Problem(**pd)
+    nb = w.n // w.block
+    Kf = K.float()
+    for c in range(nb):
+        # pairs (2j, 2j + 1): the second block dominates in the first half of
+        # the sequence, the first block in the second half
+        big = (c % 2 == 1) if c < nb // 2 else (c % 2 == 0)
+        if big:
+            Kf[:, c * w.block:(c + 1) * w.block] *= 8.0
+    K = Kf.to(torch.bfloat16)
+    idx = np.full((1, w.n, 1, 2), -1, dtype=np.int32)
+    for i in range(w.n):
+        npair = ((i + 1) // w.block) // 2          # fully visible pairs
+        if npair:
+            j = (i * 7) % npair
+            idx[0, i, 0] = (2 * j, 2 * j + 1)
+    Qn, Kn, Vn = Q.float().numpy(), K.float().numpy(), V.float().numpy()
+    # the rescale is really exercised: for many rows the second block's
+    # largest logit is more than 8 powers of two above the first block's
+    log2e = 1.0 / np.log(2.0)
+    up = down = rows = 0
+    for i in range(0, w.n, 16):
+        c1, c2 = idx[0, i, 0]
+        if c1 < 0:
+            continue
+        s1 = Qn[0, i] @ Kn[0, c1 * w.block:(c1 + 1) * w.block, 0].T * op.scale * log2e
+        s2 = Qn[0, i] @ Kn[0, c2 * w.block:(c2 + 1) * w.block, 0].T * op.scale * log2e
+        jump = s2.max(axis=1) - s1.max(axis=1)       # per head
+        rows += 1
+        up += bool(jump.max() > 8)
+        down += bool(jump.min() < -8)
+    assert up > 0.25 * rows and down > 0.05 * rows, (up, down, rows)
+    Oref, Lref = O.attention(Qn, Kn, Vn, idx, op)
+    p = params(pd)
+    assert ssa.ssa_attn_workspace_size(p) > 0
+    Qd, Kd, Vd = to_dev(Q, K, V)
+    O_, lse, bad = gpu_attn(p, Qd, Kd, Vd, torch.from_numpy(idx).cuda())
+    check_no_device_error()
+    assert int(bad.item()) == 0
+    max_abs, rel, ok = compare_out(as_np(O_), Oref, "bf16")
+    assert ok, (max_abs, rel)
+    np.testing.assert_allclose(lse.cpu().numpy(), Lref, rtol=0, atol=2e-3)
+
+
 def test_bounded_wait_gives_up_reports_its_site_and_leaves_the_context_usable():
     """A wait that nothing completes (the library's self-test kernel) gives up
     after the 1 s limit, names its site in the failure word, which reading
