@@ -162,6 +162,24 @@ __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity, uint3
 // lower block index wins ties.  Each insertion is a branchless shift over the
 // list with independent compares; the loop runs to the warp's largest count
 // (lanes past their own count insert -inf, which changes nothing).
+// Inserts (x, xi) into the descending list at its place among entries
+// J0 .. KSEL-1 (x not above entry J0 - 1): the entries from the insertion
+// point shift down by one, the last drops out; an equal score goes after
+// the entries already held.
+template <int KSEL, int J0>
+__device__ __forceinline__ void insert_tail(float (&Ls)[KSEL], int (&Li)[KSEL], float x, int xi) {
+  bool gt[KSEL];
+#pragma unroll
+  for (int j = J0; j < KSEL; ++j) gt[j] = x > Ls[j];
+#pragma unroll
+  for (int j = KSEL - 1; j > J0; --j) {
+    Ls[j] = gt[j - 1] ? Ls[j - 1] : (gt[j] ? x : Ls[j]);
+    Li[j] = gt[j - 1] ? Li[j - 1] : (gt[j] ? xi : Li[j]);
+  }
+  Ls[J0] = gt[J0] ? x : Ls[J0];
+  Li[J0] = gt[J0] ? xi : Li[J0];
+}
+
 template <int KSEL>
 __device__ __forceinline__ void merge_candidates(float (&Ls)[KSEL], int (&Li)[KSEL], int& cnt, float& thr,
                                                  const uint2* my_cand, int k, bool empty_list) {
@@ -203,16 +221,7 @@ __device__ __forceinline__ void merge_candidates(float (&Ls)[KSEL], int (&Li)[KS
       x = __uint_as_float(e.x);
       xi = static_cast<int>(e.y);
     }
-    bool gt[KSEL];
-#pragma unroll
-    for (int j = 0; j < KSEL; ++j) gt[j] = x > Ls[j];
-#pragma unroll
-    for (int j = KSEL - 1; j >= 1; --j) {
-      Ls[j] = gt[j - 1] ? Ls[j - 1] : (gt[j] ? x : Ls[j]);
-      Li[j] = gt[j - 1] ? Li[j - 1] : (gt[j] ? xi : Li[j]);
-    }
-    Ls[0] = gt[0] ? x : Ls[0];
-    Li[0] = gt[0] ? xi : Li[0];
+    insert_tail<KSEL, 0>(Ls, Li, x, xi);
   }
   cnt = 0;
   // the k-th best (the list is descending: the least of its first k)
@@ -533,11 +542,29 @@ __global__ void __launch_bounds__(TiledCfg<KF>::THREADS, 1)
         bitonic_sort_asc_u32<KSEL>(ob, os);
         const int b = bg / a.h_kv, g = bg % a.h_kv;
         const int64_t o = ((static_cast<int64_t>(b) * a.n_q + i) * a.h_kv + g) * a.topk;
+        // four entries per store when the row's entries are 16-byte aligned
+        if ((a.topk & 3) == 0 && (reinterpret_cast<uintptr_t>(a.block_idx) & 15) == 0 &&
+            (reinterpret_cast<uintptr_t>(a.top_scores) & 15) == 0) {
 #pragma unroll
-        for (int j = 0; j < KSEL; ++j) {
-          if (j < a.topk) {
-            a.block_idx[o + j] = ob[j] == 0xFFFFFFFFu ? -1 : static_cast<int32_t>(ob[j]);
-            if (a.top_scores) a.top_scores[o + j] = os[j];
+          for (int j = 0; j < KSEL; j += 4) {
+            if (j < a.topk) {
+              int4 w;
+              w.x = ob[j] == 0xFFFFFFFFu ? -1 : static_cast<int32_t>(ob[j]);
+              w.y = ob[j + 1] == 0xFFFFFFFFu ? -1 : static_cast<int32_t>(ob[j + 1]);
+              w.z = ob[j + 2] == 0xFFFFFFFFu ? -1 : static_cast<int32_t>(ob[j + 2]);
+              w.w = ob[j + 3] == 0xFFFFFFFFu ? -1 : static_cast<int32_t>(ob[j + 3]);
+              *reinterpret_cast<int4*>(a.block_idx + o + j) = w;
+              if (a.top_scores)
+                *reinterpret_cast<float4*>(a.top_scores + o + j) = make_float4(os[j], os[j + 1], os[j + 2], os[j + 3]);
+            }
+          }
+        } else {
+#pragma unroll
+          for (int j = 0; j < KSEL; ++j) {
+            if (j < a.topk) {
+              a.block_idx[o + j] = ob[j] == 0xFFFFFFFFu ? -1 : static_cast<int32_t>(ob[j]);
+              if (a.top_scores) a.top_scores[o + j] = os[j];
+            }
           }
         }
       }
