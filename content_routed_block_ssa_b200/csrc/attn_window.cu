@@ -238,12 +238,17 @@ __global__ void __launch_bounds__(WinCfg<G>::THREADS, 1)
             !mbar_wait(q_full, par, a.err, SITE_WIN_MMA) || !mbar_wait(k_full, par, a.err, SITE_WIN_MMA))
           break;
         tc_fence_after();
-        for (int n0 = 0; n0 < w.nkb; n0 += 4) {
-          const int nn = min(4, w.nkb - n0);
-          const uint32_t idesc = umma_idesc_bf16(128, 64 * nn);
+        // the span's first four blocks (N = 256) and the rest (N = 64 or
+        // 128) go to separate accumulators: their K-steps alternate, so one
+        // product runs while the other waits for its previous step
+        const uint32_t idesc_hi = umma_idesc_bf16(128, 64 * max(w.nkb - 4, 1));
 #pragma unroll
-          for (int ks = 0; ks < D / 16; ++ks) {
-            const uint64_t ad = umma_desc_sw128(sQ_u + (ks >> 2) * C::Q_HALF + (ks & 3) * 32);
+        for (int ks = 0; ks < D / 16; ++ks) {
+          const uint64_t ad = umma_desc_sw128(sQ_u + (ks >> 2) * C::Q_HALF + (ks & 3) * 32);
+#pragma unroll
+          for (int n0 = 0; n0 < C::KB; n0 += 4) {
+            if (n0 >= w.nkb) break;
+            const uint32_t idesc = n0 == 0 ? umma_idesc_bf16(128, 64 * min(4, w.nkb)) : idesc_hi;
             const uint64_t bd = umma_desc_sw128(sK_u + (ks >> 2) * C::K_HALF + n0 * C::K_BLK + (ks & 3) * 32);
             umma_bf16(tmem_base + C::S_COL + n0 * 64, ad, bd, idesc, ks != 0 ? 1u : 0u);
           }
