@@ -536,6 +536,36 @@ def hier_nodes(table: np.ndarray, fanout: int):
     return node_table, radius, round_up_f32(r_star), round_up_f32(t_star)
 
 
+def hier_super_nodes(node_table: np.ndarray, radius: np.ndarray, t_star: np.ndarray, fanout: int):
+    """The tree's second level over the node table [batch, h_kv, nn, 2d].
+
+    Super-node S = nodes S*M .. S*M+M-1 (complete super-nodes only): centre
+    bf16(f32(mean of the nodes' centres)), cap = per-dimension maximum of the
+    nodes' caps, and the recursive radius max_N (||m_N - m_S|| + R_N) (float64,
+    rounded up to float32): by the triangle inequality every block mean of
+    S lies within it of m_S.  Returns (super_table [batch, h_kv, ns, 2d],
+    super_radius [batch, h_kv, ns], r2_star [batch, h_kv] (0 without
+    super-nodes), t_star raised to the super-node rows' largest 2-norm).
+    """
+    b, h, nn, kf = node_table.shape
+    d = kf // 2
+    M = fanout
+    ns = nn // M
+    N = np.asarray(node_table, dtype=np.float64)
+    kids = N[:, :, :ns * M].reshape(b, h, ns, M, kf)
+    centre = round_bf16(round_f32(kids[..., :d].sum(axis=3) / M))
+    cap = kids[..., d:].max(axis=3) if ns else np.zeros((b, h, 0, d))
+    kid_r = np.asarray(radius, dtype=np.float64)[:, :, :ns * M].reshape(b, h, ns, M)
+    dist = np.sqrt(((kids[..., :d] - centre[:, :, :, None, :]) ** 2).sum(axis=-1))   # [b, h, ns, M]
+    sradius = round_up_f32((dist + kid_r).max(axis=3)) if ns else np.zeros((b, h, 0))
+    stable = np.concatenate([centre, cap], axis=-1)
+    r2_star = round_up_f32(sradius.max(axis=2)) if ns else np.zeros((b, h))
+    t2 = np.asarray(t_star, dtype=np.float64)
+    if ns:
+        t2 = np.maximum(t2, round_up_f32(np.sqrt((stable ** 2).sum(axis=-1)).max(axis=2)))
+    return stable, sradius, r2_star, t2
+
+
 def hier_route_row(f: np.ndarray, table_bg: np.ndarray, nodes_bg, pos: int, p: Problem, fanout: int,
                    probe: int):
     """One (query row, kv-head) through the hierarchical router.
@@ -576,18 +606,71 @@ def hier_route_row(f: np.ndarray, table_bg: np.ndarray, nodes_bg, pos: int, p: P
     return kept, certified, info
 
 
+def hier_route_row2(f: np.ndarray, table_bg: np.ndarray, nodes_bg, supers_bg, pos: int, p: Problem,
+                    fanout: int, probe: int):
+    """One (query row, kv-head) through the two-level tree.
+
+    supers_bg = (super_table [ns, 2d], super_radius [ns], r2_star, t_star)
+    of its (batch, kv-head); nodes_bg as for hier_route_row (its t_star is
+    replaced by the one covering the super-node rows).  The row ranks its
+    complete visible super-nodes by w_S = f . [m_S ; v_S] and expands the best
+    `probe`; their nodes and the complete visible nodes outside complete
+    super-nodes are ranked by w_N, the best `probe` of them expanded; the
+    blocks of those and the visible blocks outside complete nodes are scored
+    exactly and their top-k kept.  Certified when neither level leaves an
+    unexpanded entry whose bound (w + ||f_s|| R* + margin, R* the level's
+    largest radius) reaches the k-th kept score.
+    """
+    node_table, _radius, r_star, _t1 = nodes_bg
+    stable, _sradius, r2_star, t_star = supers_bg
+    d = p.d
+    M = fanout
+    nn = node_table.shape[0]
+    ns = stable.shape[0]
+    nv = visible_blocks(pos, p)
+    nvn = max(0, min(nn, (pos + 1) // (M * p.block)))
+    nvs = max(0, min(ns, (pos + 1) // (M * M * p.block)))
+    w2 = stable[:nvs] @ f
+    order2 = np.lexsort((np.arange(nvs), -w2))
+    sexp = np.sort(order2[:probe])
+    ncand = np.concatenate([np.arange(S * M, (S + 1) * M) for S in sexp] +
+                           [np.arange(nvs * M, nvn)]).astype(np.int64)
+    w1 = node_table[ncand] @ f
+    order1 = np.lexsort((ncand, -w1))
+    expanded = np.sort(ncand[order1[:probe]])
+    cand = np.concatenate([np.arange(N * M, (N + 1) * M) for N in expanded] +
+                          [np.arange(nvn * M, nv)]).astype(np.int64)
+    s = table_bg[cand] @ f
+    corder = np.lexsort((cand, -s))
+    take = min(p.topk, cand.size)
+    kept = np.full(p.topk, -1, dtype=np.int64)
+    kept[:take] = np.sort(cand[corder[:take]])
+    tau = s[corder[p.topk - 1]] if cand.size >= p.topk else -np.inf
+    f_s_norm = math.sqrt(float(f[:d] @ f[:d]))
+    margin = HIER_MARGIN * math.sqrt(float(f @ f)) * t_star
+    bound1 = w1[order1[probe]] + f_s_norm * r_star + margin if ncand.size > probe else -np.inf
+    bound2 = w2[order2[probe]] + f_s_norm * r2_star + margin if nvs > probe else -np.inf
+    certified = bool(tau > bound1 and tau > bound2) if max(bound1, bound2) > -np.inf else True
+    info = {"super_expanded": sexp, "expanded": expanded, "tau": tau, "bound": max(bound1, bound2)}
+    return kept, certified, info
+
+
 def hier_route(Q: np.ndarray, stored, p: Problem, fanout: int, probe: int, escalate: bool = False,
-               rows=None):
+               rows=None, levels: int = 1):
     """block_idx [batch, n_q, h_kv, k], certified [batch, n_q, h_kv] (bool) and
     per-row info of the hierarchical router (bf16 problems, S = 1).
 
     escalate: uncertified rows take the flat top-k of all visible blocks.
     rows: optional (batch, query row) pairs; other rows stay -2 / False.
+    levels: 1 (nodes over blocks) or 2 (super-nodes over the nodes as well).
     """
     if p.dtype != BF16 or p.subblocks != 1 or p.outlier:
         raise ValueError("the hierarchical router is defined on the bf16 routing table, S = 1")
+    if levels not in (1, 2):
+        raise ValueError("one or two tree levels")
     _mu32, _sig32, table = stored
     nodes = hier_nodes(table, fanout)
+    supers = hier_super_nodes(nodes[0], nodes[1], nodes[3], fanout) if levels == 2 else None
     bidx = np.full((p.batch, p.n_q, p.h_kv, p.topk), -2, dtype=np.int64)
     cert = np.zeros((p.batch, p.n_q, p.h_kv), dtype=bool)
     info = {}
@@ -601,7 +684,11 @@ def hier_route(Q: np.ndarray, stored, p: Problem, fanout: int, probe: int, escal
         for g in range(p.h_kv):
             f = feats[bi][g, i]
             nb_g = (nodes[0][bi, g], nodes[1][bi, g], nodes[2][bi, g], nodes[3][bi, g])
-            kept, ok, inf = hier_route_row(f, table[bi, g], nb_g, pos, p, fanout, probe)
+            if levels == 1:
+                kept, ok, inf = hier_route_row(f, table[bi, g], nb_g, pos, p, fanout, probe)
+            else:
+                sb_g = (supers[0][bi, g], supers[1][bi, g], supers[2][bi, g], supers[3][bi, g])
+                kept, ok, inf = hier_route_row2(f, table[bi, g], nb_g, sb_g, pos, p, fanout, probe)
             if escalate and not ok:
                 nv = visible_blocks(pos, p)
                 kept, _gap = select_topk(table[bi, g, :nv] @ f, p.topk)

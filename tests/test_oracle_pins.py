@@ -877,3 +877,103 @@ def test_outlier_score_is_the_exact_group_logit_of_the_max_norm_key():
             assert abs(s[c] - max(s0[c], logit)) <= 1e-12 * max(1.0, abs(s[c]))
     with pytest.raises(ValueError):
         O.block_summaries(K, O.Problem(**{**p.__dict__, "subblocks": 2}))
+
+
+# ------------------------------------------------------------------ two-level tree
+
+def test_hier_super_node_bound_is_admissible_and_radius_recursive():
+    """Every block's score is at most its super-node's bound f.[m_S;v_S] +
+    ||f_s|| R_S (features aimed at the farthest block included); R_S is the
+    largest ||m_N - m_S|| + R_N over its nodes, rounded up to float32, so it
+    covers the true largest distance of a block mean from m_S."""
+    rng = np.random.default_rng(41)
+    d, nb = 8, 128
+    mu = O.round_bf16(rng.standard_normal((1, 1, nb, d)) * rng.uniform(0.1, 3.0, (1, 1, nb, 1)))
+    sg = O.round_bf16(rng.chisquare(2, (1, 1, nb, d)))
+    table = np.concatenate([mu, sg], axis=-1)
+    for M in (2, 4):
+        nt, rad, _r1, t1 = O.hier_nodes(table, M)
+        st, srad, r2, t2 = O.hier_super_nodes(nt, rad, t1, M)
+        ns = nb // (M * M)
+        assert st.shape == (1, 1, ns, 2 * d) and r2[0, 0] == srad[0, 0].max() and t2[0, 0] >= t1[0, 0]
+        for S in range(ns):
+            kids = nt[0, 0, S * M:(S + 1) * M]
+            rec = max(float(np.linalg.norm(kids[j, :d] - st[0, 0, S, :d])) + float(rad[0, 0, S * M + j])
+                      for j in range(M))
+            assert rec <= srad[0, 0, S] <= rec * (1 + 2.0 ** -22)
+            true = np.linalg.norm(mu[0, 0, S * M * M:(S + 1) * M * M] - st[0, 0, S, :d], axis=1).max()
+            assert true <= srad[0, 0, S]
+            np.testing.assert_array_equal(st[0, 0, S, d:], kids[:, d:].max(axis=0))
+        for trial in range(200):
+            fs = O.round_bf16(rng.standard_normal(d) * 2)
+            fq = O.round_bf16(np.abs(rng.standard_normal(d)))
+            if trial % 4 == 0:
+                S = trial % ns
+                blk = mu[0, 0, S * M * M:(S + 1) * M * M]
+                far = np.argmax(np.linalg.norm(blk - st[0, 0, S, :d], axis=1))
+                fs = O.round_bf16(blk[far] - st[0, 0, S, :d])
+                fq = np.zeros(d)
+            f = np.concatenate([fs, fq])
+            bound = st[0, 0] @ f + np.linalg.norm(fs) * srad[0, 0]
+            score = (table[0, 0, :ns * M * M] @ f).reshape(ns, M * M)
+            assert np.all(score.max(axis=1) <= bound + 1e-9)
+
+
+def test_hier_two_levels_brute_force_ranking():
+    """Both levels by explicit enumeration: the probe best super-nodes by w_S
+    (ties to the lower index), then the probe best of their nodes and the
+    nodes outside complete super-nodes by w_N, then the top-k of the expanded
+    nodes' blocks and the blocks outside complete nodes."""
+    rng = np.random.default_rng(42)
+    p, Q, stored = _hier_problem(rng, n=512, topk=3)
+    M, probe = 2, 2
+    nt, rad, r1, t1 = O.hier_nodes(stored[2], M)
+    st, srad, r2, t2 = O.hier_super_nodes(nt, rad, t1, M)
+    f_all = O.route_features(Q, p)[0]
+    T = stored[2]
+    for i in range(0, 512, 11):
+        for g in range(p.h_kv):
+            f = f_all[g, i]
+            nv = O.visible_blocks(i, p)
+            nvn = min(nt.shape[2], (i + 1) // (M * p.block))
+            nvs = min(st.shape[2], (i + 1) // (M * M * p.block))
+            sexp = sorted(sorted(range(nvs), key=lambda S: (-(st[0, g, S] @ f), S))[:probe])
+            ncand = [N for S in sexp for N in range(S * M, S * M + M)] + list(range(nvs * M, nvn))
+            nexp = sorted(sorted(ncand, key=lambda N: (-(nt[0, g, N] @ f), N))[:probe])
+            cand = [c for N in nexp for c in range(N * M, N * M + M)] + list(range(nvn * M, nv))
+            ranked = sorted(cand, key=lambda c: (-(T[0, g, c] @ f), c))
+            want = sorted(ranked[:p.topk]) + [-1] * max(0, p.topk - len(cand))
+            kept, ok, info = O.hier_route_row2(f, T[0, g], (nt[0, g], rad[0, g], r1[0, g], t1[0, g]),
+                                               (st[0, g], srad[0, g], r2[0, g], t2[0, g]), i, p, M, probe)
+            assert list(info["super_expanded"]) == sexp and list(info["expanded"]) == nexp
+            assert list(kept) == want
+            if nvs <= probe and len(ncand) <= probe:
+                assert ok
+
+
+@pytest.mark.parametrize("benign", [False, True])
+def test_hier_two_levels_certified_rows_hold_the_exact_topk(benign):
+    """A certified row of the two-level tree keeps the flat top-k of all its
+    visible blocks; probing every super-node and node gives the flat router;
+    escalation gives the flat router on every row."""
+    rng = np.random.default_rng(43 + benign)
+    fired = total = 0
+    for M, probe, topk in ((2, 2, 4), (4, 2, 4), (2, 3, 8)):
+        p, Q, stored = _hier_problem(rng, n=512, topk=topk, node_keys=(M * 4 if benign else None))
+        rows = [(0, i) for i in range(0, p.n_q, 5)]
+        bidx, cert, _ = O.hier_route(Q, stored, p, M, probe, rows=rows, levels=2)
+        for (bi, i) in rows:
+            for g in range(p.h_kv):
+                total += 1
+                if cert[bi, i, g]:
+                    fired += 1
+                    np.testing.assert_array_equal(bidx[bi, i, g], _flat(Q, stored, p, bi, i, g))
+    assert 0 < fired < total
+    p, Q, stored = _hier_problem(rng, n=256, topk=4)
+    flat, _ = O.route_topk(Q, stored, p)
+    M = 2
+    b1, c1, _ = O.hier_route(Q, stored, p, M, p.nb // M, levels=2)   # everything expanded
+    np.testing.assert_array_equal(b1, flat)
+    assert c1.all()
+    b2, _c2, _ = O.hier_route(Q, stored, p, M, 1, escalate=True, levels=2)
+    np.testing.assert_array_equal(b2, flat)
