@@ -2,7 +2,7 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
                     [--workload NAME] [--no-secondary] [--no-cpu-baseline] [--no-e2e]
-                    [--subblocks S] [--outlier] [--router flat|hier [--fanout M] [--probe P] [--escalate]]
+                    [--subblocks S] [--outlier] [--router flat|hier [--fanout M] [--probe P] [--escalate] [--levels L]]
 
 One step is one pass of the whole layer over the workload's synthetic input:
 block summaries -> routing features + tensor-core route with fused top-k ->
@@ -327,8 +327,8 @@ def needle_recall(plan, idx, w):
 
 
 def run_ours(w, steps, warmup, ws, rank, with_e2e=True, hier=None):
-    """hier: None (the flat router) or (fanout, probe, escalate) for the
-    hierarchical router, whose node summaries are then rebuilt every step."""
+    """hier: None (the flat router) or (fanout, probe, escalate, levels) for
+    the hierarchical router, whose node summaries are then rebuilt every step."""
     from content_routed_block_ssa_b200 import ssa
     dev = torch.device("cuda", torch.cuda.current_device())
     Q, K, V, plan = make_inputs(w, dev)
@@ -423,7 +423,7 @@ def run_ours(w, steps, warmup, ws, rank, with_e2e=True, hier=None):
     selection = {"needle_recall": needle_recall(plan, idx, w)}
     if cert is not None:
         selection["certified"] = float(cert.float().mean())
-        selection["router"] = {"fanout": hier[0], "probe": hier[1], "escalate": bool(hier[2])}
+        selection["router"] = {"fanout": hier[0], "probe": hier[1], "escalate": bool(hier[2]), "levels": hier[3]}
 
     e2e = None
     if with_e2e:
@@ -511,7 +511,8 @@ def kernel_report(w, res, peaks, traffic):
         # route (node router + per-row probe of L2-served table rows + any
         # escalation) is reported by time, outside the roofline
         hbm_entry("hier_nodes", wk["route_table_bytes_once"])
-        rep["route"] = {"ms": ms["route"], "kernel": "route_tiled_kernel / route_rowwise_bf16_kernel (nodes) + "
+        rep["route"] = {"ms": ms["route"], "kernel": "route_tiled_kernel / route_rowwise_bf16_kernel (nodes or "
+                                                     "super-nodes) + hier_probe2_kernel (two levels) + "
                                                      "hier_probe_kernel (+ escalation)"}
     elif w.dtype == "f32":
         rep["summary"]["kernel"] = "summary_diag_kernel" if w.sigma == "diag" else "summary_full_kernel"
@@ -664,6 +665,7 @@ def main():
     ap.add_argument("--fanout", type=int, default=16)
     ap.add_argument("--probe", type=int, default=2)
     ap.add_argument("--escalate", action="store_true", help="re-route uncertified rows over all blocks")
+    ap.add_argument("--levels", type=int, default=1, choices=[1, 2], help="tree levels of the hierarchical router")
     a = ap.parse_args()
     w = WORKLOADS[a.workload]
     if a.n is not None:
@@ -699,11 +701,12 @@ def main():
 
     # the committed DRAM counters were taken with whole-block summaries
     traffic = load_traffic() if w.subblocks == 1 and not w.outlier else {}
-    hier = (a.fanout, a.probe, a.escalate) if a.router == "hier" else None
+    hier = (a.fanout, a.probe, a.escalate, a.levels) if a.router == "hier" else None
     if w.decode:
         config["state"] = "block summaries precomputed (built once, untimed; kernels.summary times one build)"
     if hier is not None:
-        config["router"] = {"kind": "hierarchical", "fanout": a.fanout, "probe": a.probe, "escalate": a.escalate}
+        config["router"] = {"kind": "hierarchical", "fanout": a.fanout, "probe": a.probe, "escalate": a.escalate,
+                            "levels": a.levels}
     res = run_ours(w, a.steps, a.warmup, ws, rank, with_e2e=not a.no_e2e and hier is None, hier=hier)
     kern = kernel_report(w, res, peaks, traffic)
     value = whole_job_rate(w.batch * w.n_q * w.h_q, ws, res["ms_step"])

@@ -147,6 +147,37 @@ struct HierNodeArgs {
 };
 cudaError_t launch_hier_nodes(const ssa_params& p, const HierNodeArgs& a, const LaunchCtx& c);
 
+// The tree's second level: one warp per (batch * kv-head, super-node) of M
+// consecutive nodes.
+struct HierSuperArgs {
+  int32_t bgs, nn, ns, M;      // ns = nn / M complete super-nodes
+  const __nv_bfloat16* NT;     // [bgs, nn, 2d] node rows
+  const float* radius;         // [bgs, nn] node radii
+  __nv_bfloat16* ST;           // [bgs, ns, 2d] super-node rows [centre ; cap]
+  float* sradius;              // [bgs, ns] recursive radii
+  uint32_t* sbound;            // [bgs] float bits: largest super-node radius; zeroed first
+  uint32_t* bound;             // [bgs, 2] of the nodes: the row-norm half is raised to the super rows'
+};
+cudaError_t launch_hier_supers(const ssa_params& p, const HierSuperArgs& a, const LaunchCtx& c);
+
+// Two-level routing, first probe: one warp per (batch * kv-head, query row)
+// expands the row's best super-nodes and ranks their nodes (and the nodes
+// outside complete super-nodes) by their exact node scores, keeping the best
+// probe+1 in the layout the node router gives the block probe.
+struct HierProbe2Args {
+  int32_t n_q, h_kv, bgs, nn, ns, M, block, probe;
+  int64_t q_offset;
+  const __nv_bfloat16* F;      // [bgs, n_q, 2d] routing features
+  const __nv_bfloat16* NT;     // [bgs, nn, 2d] node rows
+  const int32_t* sup_idx;      // [b, n_q, h_kv, probe+1] best super-nodes, ascending, -1 padded (null: none)
+  const float* sup_score;      // same layout, their scores
+  int32_t* node_idx;           // [b, n_q, h_kv, probe+1] out: best candidate nodes, ascending, -1 padded
+  float* node_score;           // same layout, their scores
+  int32_t* n_cand;             // [b, n_q, h_kv] out: candidate nodes of the row
+  float* w2_next;              // [b, n_q, h_kv] out: best unexpanded super-node score, -inf if none
+};
+cudaError_t launch_hier_probe2(const ssa_params& p, const HierProbe2Args& a, const LaunchCtx& c);
+
 // The per-row probe of the best nodes and the certificate: one warp per
 // (batch * kv-head, query row).
 struct HierProbeArgs {
@@ -160,6 +191,12 @@ struct HierProbeArgs {
   int32_t* block_idx;          // [b, n_q, h_kv, topk]
   uint8_t* cert;               // [b, n_q, h_kv] (may be null)
   int32_t* unit_need;          // [bgs, n_tiles] set to 1 for units holding an uncertified row (may be null)
+  // two levels (null for one): the row's candidate nodes and best
+  // unexpanded super-node score from the first probe, and the largest
+  // super-node radius of each (batch * kv-head)
+  const int32_t* n_cand;       // [b, n_q, h_kv]
+  const float* w2_next;        // [b, n_q, h_kv]
+  const float* sbound;         // [bgs]
 };
 cudaError_t launch_hier_probe(const ssa_params& p, const HierProbeArgs& a, const LaunchCtx& c);
 

@@ -485,25 +485,31 @@ ssa_status forward_impl(const ssa_params& p, const void* Q, const void* K, const
 
 // ------------------------------------------------------------------ hierarchical routing
 
+int hier_levels(const ssa_hier_params& hp) { return hp.levels == 2 ? 2 : 1; }
+
 struct HierNodeLayout {
-  int64_t nn;
-  size_t table, radius, bound, total;
+  int64_t nn, ns;   // nodes; super-nodes (second level, else 0)
+  size_t table, radius, bound, stable, sradius, sbound, total;
 };
 
 HierNodeLayout hier_node_layout(const ssa_params& p, const ssa_hier_params& hp) {
   HierNodeLayout L;
   const size_t bgs = static_cast<size_t>(p.batch) * p.h_kv;
   L.nn = nb_of(p) / hp.fanout;
+  L.ns = hier_levels(hp) == 2 ? L.nn / hp.fanout : 0;
   size_t off = 0;
   L.table = off; off += round_up(bgs * L.nn * 2 * p.d * 2);
   L.radius = off; off += round_up(bgs * L.nn * 4);
   L.bound = off; off += round_up(bgs * 2 * 4);
+  L.stable = off; off += round_up(bgs * L.ns * 2 * p.d * 2);
+  L.sradius = off; off += round_up(bgs * L.ns * 4);
+  L.sbound = off; off += hier_levels(hp) == 2 ? round_up(bgs * 4) : 0;
   L.total = off;
   return L;
 }
 
 struct HierLayout {
-  size_t feat, nidx, nsc, cert, need, total;
+  size_t feat, nidx, nsc, cert, need, sidx, ssc, ncand, w2n, total;
 };
 
 int32_t route_tiles(const ssa_params& p) { return (p.n_q + 255) / 256; }
@@ -518,6 +524,11 @@ HierLayout hier_layout(const ssa_params& p, const ssa_hier_params& hp) {
   L.nsc = off; off += round_up(rows * (hp.probe + 1) * 4);
   L.cert = off; off += round_up(rows);
   L.need = off; off += (hp.escalate && use_tiled(p)) ? round_up(bgs * route_tiles(p) * 4) : 0;
+  const bool two = hier_levels(hp) == 2;
+  L.sidx = off; off += two ? round_up(rows * (hp.probe + 1) * 4) : 0;
+  L.ssc = off; off += two ? round_up(rows * (hp.probe + 1) * 4) : 0;
+  L.ncand = off; off += two ? round_up(rows * 4) : 0;
+  L.w2n = off; off += two ? round_up(rows * 4) : 0;
   L.total = off;
   return L;
 }
@@ -525,7 +536,7 @@ HierLayout hier_layout(const ssa_params& p, const ssa_hier_params& hp) {
 ssa_status check_hier(const ssa_params* p, const ssa_hier_params* hp) {
   ssa_status st = check_params(p);
   if (st != SSA_OK) return st;
-  if (!hp || hp->reserved != 0) return SSA_ERR_INVALID_ARG;
+  if (!hp || hp->levels < 0 || hp->levels > 2) return SSA_ERR_INVALID_ARG;
   const int M = hp->fanout;
   if (M < 1 || M > 64 || (M & (M - 1)) != 0) return SSA_ERR_INVALID_ARG;
   if (hp->probe < 1 || hp->probe > 31 || (hp->escalate != 0 && hp->escalate != 1)) return SSA_ERR_INVALID_ARG;
@@ -535,10 +546,11 @@ ssa_status check_hier(const ssa_params* p, const ssa_hier_params* hp) {
   return SSA_OK;
 }
 
-// The node problem: nodes of M blocks act as blocks of M * B keys.
-ssa_params node_params(const ssa_params& p, const ssa_hier_params& hp, int64_t nn) {
+// The node problem: nodes of M blocks act as blocks of M * B keys (and
+// super-nodes of M nodes as blocks of M * M * B keys: span = M * M).
+ssa_params node_params(const ssa_params& p, const ssa_hier_params& hp, int64_t nn, int span) {
   ssa_params pn = p;
-  pn.block = p.block * hp.fanout;
+  pn.block = p.block * span;
   pn.n_kv = static_cast<int32_t>(nn * pn.block);
   pn.topk = hp.probe + 1;
   pn.subblocks = 1;
@@ -561,16 +573,39 @@ ssa_status do_route_hier(const ssa_params& p, const ssa_hier_params& hp, const v
   if (st != SSA_OK) return st;
   CUtensorMap tmF;
   if (tiled && !encode_2d(&tmF, F, kf, static_cast<uint64_t>(bgs) * p.n_q, 128)) return SSA_ERR_CUDA;
-  if (NL.nn > 0) {   // the best probe+1 nodes of every row, with their scores
-    const ssa_params pn = node_params(p, hp, NL.nn);
+  // the best probe+1 entries of every row, with their scores, from the
+  // block router run over a node or super-node table
+  auto rank_rows = [&](const uint8_t* rows_table, int64_t n_rows, int span, int32_t* out_idx,
+                       float* out_sc) -> ssa_status {
+    const ssa_params pn = node_params(p, hp, n_rows, span);
     if (tiled) {
       CUtensorMap tmN;
-      if (!encode_2d(&tmN, nd + NL.table, kf, static_cast<uint64_t>(bgs * NL.nn), 128)) return SSA_ERR_CUDA;
-      st = from_cuda(ssa::launch_route_tiled(pn, tmF, tmN, nidx, nsc, c));
-    } else {
-      st = from_cuda(ssa::launch_route_rowwise_bf16(pn, Q, nd + NL.table, nidx, nsc, c));
+      if (!encode_2d(&tmN, rows_table, kf, static_cast<uint64_t>(bgs * n_rows), 128)) return SSA_ERR_CUDA;
+      return from_cuda(ssa::launch_route_tiled(pn, tmF, tmN, out_idx, out_sc, c));
     }
-    if (st != SSA_OK) return st;
+    return from_cuda(ssa::launch_route_rowwise_bf16(pn, Q, rows_table, out_idx, out_sc, c));
+  };
+  const bool two = hier_levels(hp) == 2;
+  if (two) {
+    // super-nodes first; the first probe ranks the candidate nodes exactly
+    int32_t* sidx = reinterpret_cast<int32_t*>(ws + H.sidx);
+    float* ssc = reinterpret_cast<float*>(ws + H.ssc);
+    if (NL.ns > 0 && (st = rank_rows(nd + NL.stable, NL.ns, hp.fanout * hp.fanout, sidx, ssc)) != SSA_OK)
+      return st;
+    ssa::HierProbe2Args a2;
+    a2.n_q = p.n_q; a2.h_kv = p.h_kv; a2.bgs = static_cast<int32_t>(bgs);
+    a2.nn = static_cast<int32_t>(NL.nn); a2.ns = static_cast<int32_t>(NL.ns); a2.M = hp.fanout;
+    a2.block = p.block; a2.probe = hp.probe; a2.q_offset = p.q_offset;
+    a2.F = static_cast<const __nv_bfloat16*>(F);
+    a2.NT = reinterpret_cast<const __nv_bfloat16*>(nd + NL.table);
+    a2.sup_idx = NL.ns > 0 ? sidx : nullptr;
+    a2.sup_score = NL.ns > 0 ? ssc : nullptr;
+    a2.node_idx = nidx; a2.node_score = nsc;
+    a2.n_cand = reinterpret_cast<int32_t*>(ws + H.ncand);
+    a2.w2_next = reinterpret_cast<float*>(ws + H.w2n);
+    if ((st = from_cuda(ssa::launch_hier_probe2(p, a2, c))) != SSA_OK) return st;
+  } else if (NL.nn > 0 && (st = rank_rows(nd + NL.table, NL.nn, hp.fanout, nidx, nsc)) != SSA_OK) {
+    return st;
   }
   int32_t* need = (hp.escalate && tiled) ? reinterpret_cast<int32_t*>(ws + H.need) : nullptr;
   if (need && cudaMemsetAsync(need, 0, static_cast<size_t>(bgs) * route_tiles(p) * 4, c.stream) != cudaSuccess)
@@ -585,6 +620,9 @@ ssa_status do_route_hier(const ssa_params& p, const ssa_hier_params& hp, const v
   a.node_idx = nidx; a.node_score = nsc;
   a.bound = reinterpret_cast<const float*>(nd + NL.bound);
   a.block_idx = idx; a.cert = cert; a.unit_need = need;
+  a.n_cand = two ? reinterpret_cast<const int32_t*>(ws + H.ncand) : nullptr;
+  a.w2_next = two ? reinterpret_cast<const float*>(ws + H.w2n) : nullptr;
+  a.sbound = two ? reinterpret_cast<const float*>(nd + NL.sbound) : nullptr;
   if ((st = from_cuda(ssa::launch_hier_probe(p, a, c))) != SSA_OK) return st;
   if (!hp.escalate) return SSA_OK;
   if (tiled) {   // the units holding an uncertified row, over all their visible blocks
@@ -815,6 +853,8 @@ ssa_status ssa_hier_nodes(const ssa_params* pp, const ssa_hier_params* hp, const
   const int64_t bgs = static_cast<int64_t>(p.batch) * p.h_kv;
   if (cudaMemsetAsync(nd + L.bound, 0, static_cast<size_t>(bgs) * 2 * 4, c.stream) != cudaSuccess)
     return SSA_ERR_CUDA;
+  if (hier_levels(*hp) == 2 && cudaMemsetAsync(nd + L.sbound, 0, static_cast<size_t>(bgs) * 4, c.stream) != cudaSuccess)
+    return SSA_ERR_CUDA;
   ssa::HierNodeArgs a;
   a.bgs = static_cast<int32_t>(bgs);
   a.nb = static_cast<int32_t>(nb_of(p));
@@ -824,7 +864,19 @@ ssa_status ssa_hier_nodes(const ssa_params* pp, const ssa_hier_params* hp, const
   a.NT = reinterpret_cast<__nv_bfloat16*>(nd + L.table);
   a.radius = reinterpret_cast<float*>(nd + L.radius);
   a.bound = reinterpret_cast<uint32_t*>(nd + L.bound);
-  return from_cuda(ssa::launch_hier_nodes(p, a, c));
+  if ((st = from_cuda(ssa::launch_hier_nodes(p, a, c))) != SSA_OK || hier_levels(*hp) != 2) return st;
+  ssa::HierSuperArgs s2;
+  s2.bgs = static_cast<int32_t>(bgs);
+  s2.nn = static_cast<int32_t>(L.nn);
+  s2.ns = static_cast<int32_t>(L.ns);
+  s2.M = hp->fanout;
+  s2.NT = reinterpret_cast<const __nv_bfloat16*>(nd + L.table);
+  s2.radius = reinterpret_cast<const float*>(nd + L.radius);
+  s2.ST = reinterpret_cast<__nv_bfloat16*>(nd + L.stable);
+  s2.sradius = reinterpret_cast<float*>(nd + L.sradius);
+  s2.sbound = reinterpret_cast<uint32_t*>(nd + L.sbound);
+  s2.bound = reinterpret_cast<uint32_t*>(nd + L.bound);
+  return from_cuda(ssa::launch_hier_supers(p, s2, c));
 }
 
 size_t ssa_route_hier_workspace_size(const ssa_params* p, const ssa_hier_params* hp) {

@@ -40,7 +40,7 @@ assert C.sizeof(ssa_params) == 72
 
 
 class ssa_hier_params(C.Structure):
-    _fields_ = [("fanout", C.c_int32), ("probe", C.c_int32), ("escalate", C.c_int32), ("reserved", C.c_int32)]
+    _fields_ = [("fanout", C.c_int32), ("probe", C.c_int32), ("escalate", C.c_int32), ("levels", C.c_int32)]
 
 
 assert C.sizeof(ssa_hier_params) == 16
@@ -255,9 +255,10 @@ def byte_buffer(nbytes: int, device="cuda"):
     return torch.empty(max(int(nbytes), 16), dtype=torch.uint8, device=device)
 
 
-def make_hier_params(fanout=16, probe=2, escalate=False) -> ssa_hier_params:
-    """An ssa_hier_params struct: nodes of `fanout` blocks, `probe` nodes expanded per row."""
-    return ssa_hier_params(fanout=fanout, probe=probe, escalate=1 if escalate else 0, reserved=0)
+def make_hier_params(fanout=16, probe=2, escalate=False, levels=1) -> ssa_hier_params:
+    """An ssa_hier_params struct: nodes of `fanout` blocks (and with levels=2
+    super-nodes of `fanout` nodes), `probe` entries expanded per row and level."""
+    return ssa_hier_params(fanout=fanout, probe=probe, escalate=1 if escalate else 0, levels=levels)
 
 
 def ssa_hier_nodes_size(p, hp) -> int:
@@ -292,6 +293,25 @@ def hier_node_views(p, hp, nodes):
     rows = nodes[:t_bytes].view(torch.bfloat16).view(p.batch, p.h_kv, nn, 2 * p.d)
     rad = nodes[r_off:r_off + bgs * nn * 4].view(torch.float32).view(p.batch, p.h_kv, nn)
     bnd = nodes[b_off:b_off + bgs * 8].view(torch.float32).view(p.batch, p.h_kv, 2)
+    return rows, rad, bnd
+
+
+def hier_super_views(p, hp, nodes):
+    """(super-node rows [b, h_kv, ns, 2d] bf16, radii [b, h_kv, ns] f32, largest radius [b, h_kv] f32)
+    views of a two-level node store."""
+    nn = (p.n_kv // p.block) // hp.fanout
+    ns = nn // hp.fanout
+    bgs = p.batch * p.h_kv
+
+    def ru(x):
+        return (x + 255) // 256 * 256
+    off = ru(bgs * nn * 2 * p.d * 2) + ru(bgs * nn * 4) + ru(bgs * 8)
+    t_bytes = bgs * ns * 2 * p.d * 2
+    r_off = off + ru(t_bytes)
+    b_off = r_off + ru(bgs * ns * 4)
+    rows = nodes[off:off + t_bytes].view(torch.bfloat16).view(p.batch, p.h_kv, ns, 2 * p.d)
+    rad = nodes[r_off:r_off + bgs * ns * 4].view(torch.float32).view(p.batch, p.h_kv, ns)
+    bnd = nodes[b_off:b_off + bgs * 4].view(torch.float32).view(p.batch, p.h_kv)
     return rows, rad, bnd
 
 

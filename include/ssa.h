@@ -345,6 +345,19 @@ SSA_API ssa_status ssa_forward_hostio(const ssa_params* p, const void* hQ, const
  *   visible blocks (by ssa_route_topk's kernels), so block_idx is
  *   ssa_route_topk's selection for every row.
  *
+ *   levels = 2 adds a tree level: super-node S = nodes S*M .. S*M+M-1
+ *   (complete super-nodes only) with centre bf16(f32(mean of m_N)), cap the
+ *   per-dimension max of v_N and the recursive radius
+ *   R_S = max_N (||m_N - m_S||_2 + R_N) (float64, rounded up to float32),
+ *   so every block of S has f . T_c <= f . [m_S ; v_S] + ||f_s|| R_S.  A row
+ *   ranks its complete visible super-nodes, scores exactly the nodes of its
+ *   best `probe` and the complete visible nodes outside complete super-
+ *   nodes, and probes the best `probe` of those nodes as above; certified
+ *   when the k-th kept score also exceeds the best unexpanded super-node's
+ *   w_S + ||f_s|| R2* + 2^-12 ||f|| T* (R2*: largest super-node radius;
+ *   T* then also covers the super-node rows), or no complete visible
+ *   super-node is left unexpanded.
+ *
  * bf16 problems with a diagonal Sigma, subblocks = 1, outlier = 0 and d in {64, 128}
  * (else SSA_ERR_UNSUPPORTED).
  */
@@ -352,12 +365,12 @@ typedef struct {
   int32_t fanout;    /* M, blocks per node: a power of two, 1..64                 */
   int32_t probe;     /* nodes expanded per row before the certificate, 1..31      */
   int32_t escalate;  /* 1: uncertified rows are re-routed over all blocks; or 0   */
-  int32_t reserved;  /* must be 0                                                 */
+  int32_t levels;    /* tree levels: 2, or 1 (0 reads as 1)                       */
 } ssa_hier_params;
 
 /*
  * Errors of the hierarchical calls, checked before any launch: the
- * ssa_params checks of the other calls; hp NULL, reserved != 0, fanout not a
+ * ssa_params checks of the other calls; hp NULL, levels outside 0..2, fanout not a
  * power of two in 1..64, probe outside 1..31 or escalate not 0/1 ->
  * SSA_ERR_INVALID_ARG; (probe + 1) * fanout > 512 (the probe's candidate
  * capacity), a float32 problem, subblocks != 1 or outlier != 0 -> SSA_ERR_UNSUPPORTED;
@@ -372,8 +385,10 @@ typedef struct {
  * Bytes of the node store of (p, hp): the node rows (bf16 [b, h_kv, nn, 2d],
  * at offset 0), the radii (float32 [b, h_kv, nn], at offset
  * round_up(node row bytes, 256)) and two floats per (batch, kv-head) (largest
- * radius, largest row norm; after the radii, also 256-byte aligned).
- * 0 on invalid arguments.
+ * radius, largest row norm; after the radii, also 256-byte aligned); with
+ * levels = 2 then the super-node rows (bf16 [b, h_kv, nn / M, 2d]), their
+ * radii and one float per (batch, kv-head) (largest super-node radius), each
+ * part 256-byte aligned.  0 on invalid arguments.
  */
 SSA_API size_t ssa_hier_nodes_size(const ssa_params* p, const ssa_hier_params* hp);
 

@@ -651,7 +651,14 @@ def hier_route_row2(f: np.ndarray, table_bg: np.ndarray, nodes_bg, supers_bg, po
     bound1 = w1[order1[probe]] + f_s_norm * r_star + margin if ncand.size > probe else -np.inf
     bound2 = w2[order2[probe]] + f_s_norm * r2_star + margin if nvs > probe else -np.inf
     certified = bool(tau > bound1 and tau > bound2) if max(bound1, bound2) > -np.inf else True
-    info = {"super_expanded": sexp, "expanded": expanded, "tau": tau, "bound": max(bound1, bound2)}
+    # the gaps that float32 rounding could flip: each level's probe-th /
+    # (probe+1)-th score, the kept set's k-th / (k+1)-th
+    super_gap = w2[order2[probe - 1]] - w2[order2[probe]] if nvs > probe else np.inf
+    node_gap = w1[order1[probe - 1]] - w1[order1[probe]] if ncand.size > probe else np.inf
+    kgap = (s[corder[p.topk - 1]] - s[corder[p.topk]]) if cand.size > p.topk else np.inf
+    info = {"super_expanded": sexp, "expanded": expanded, "tau": tau, "bound": max(bound1, bound2),
+            "bounds": (bound1, bound2), "super_gap": super_gap, "node_gap": node_gap, "kept_gap": kgap,
+            "scale": math.sqrt(float(f @ f)) * t_star}
     return kept, certified, info
 
 

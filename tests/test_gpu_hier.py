@@ -163,3 +163,120 @@ def test_hier_certificates_fire_on_alike_blocks_and_not_on_block_clusters():
         fired[name] = float(late.mean())
     assert fired["gqa4_d128_b64_span16_M16_p2"] > 0.3
     assert fired["gqa4_d128_b64_blockclusters_M8_p3"] < fired["gqa4_d128_b64_span16_M16_p2"]
+
+
+# ------------------------------------------------------------------ two levels
+
+# name: (workload, fanout, probe); nodes of M blocks, super-nodes of M nodes
+CASES2 = {
+    # keys alike over runs of 16 blocks: a super-node of 4 x 4 blocks is one run
+    "gqa4_d128_b64_span16_M4_p2": (Workload("h", 141, 1, 4096, 8, 2, 128, "bf16", 64, "diag", 8, 256, 6,
+                                            "total", clustered=True, cluster_span=16), 4, 2),
+    # a centroid per block: loose bounds at both levels
+    "gqa4_d128_b64_blockclusters_M4_p3": (Workload("h", 142, 1, 3072, 8, 2, 128, "bf16", 64, "diag", 16, 128, 6,
+                                                   "total", clustered=True), 4, 3),
+    # 70 blocks of 128 keys at M = 2: 35 nodes, 17 super-nodes and a trailing node
+    "gqa8_d128_b128_ragged_M2_p2": (Workload("h", 143, 1, 8960, 8, 1, 128, "bf16", 128, "diag", 8, 256, 8,
+                                             "total", clustered=True, cluster_span=4), 2, 2),
+    "decode_gqa4_d128_span16_M4_p2": (Workload("h", 144, 4, 16384, 8, 2, 128, "bf16", 64, "diag", 16, 256, 2,
+                                               "per_seq", clustered=True, cluster_span=16, decode=True), 4, 2),
+}
+
+_cache2 = {}
+
+
+def case2(name):
+    if name not in _cache2:
+        w, M, probe = CASES2[name]
+        Q, K, V, _plan = make_inputs(w, "cpu")
+        pd = problem_dict(w)
+        op = O.Problem(**pd)
+        Qn, Kn = Q.float().numpy(), K.float().numpy()
+        stored = O.stored_summaries(*O.block_summaries(Kn, op), op)
+        flat, gaps = O.route_topk(Qn, stored, op)
+        hb, hc, info = O.hier_route(Qn, stored, op, M, probe, levels=2)
+        nodes = O.hier_nodes(stored[2], M)
+        _cache2[name] = dict(w=w, M=M, probe=probe, pd=pd, op=op, Q=Q, Qn=Qn, stored=stored, flat=flat,
+                             gaps=gaps, hb=hb, hc=hc, info=info, nodes=nodes,
+                             supers=O.hier_super_nodes(nodes[0], nodes[1], nodes[3], M))
+    return _cache2[name]
+
+
+def impls2(name):
+    return (ssa.SSA_ROUTE_ROWWISE,) if CASES2[name][0].decode else (ssa.SSA_ROUTE_TILED, ssa.SSA_ROUTE_ROWWISE)
+
+
+PAIRS2 = [(n, i) for n in CASES2 for i in impls2(n)]
+IDS2 = [f"{n}-{'tiled' if i == ssa.SSA_ROUTE_TILED else 'rowwise'}" for n, i in PAIRS2]
+
+
+def _ulps(a, b):
+    a = np.asarray(a, np.float32)
+    b = np.asarray(b, np.float32)
+    return np.abs(a.view(np.int32).astype(np.int64) - b.view(np.int32).astype(np.int64))
+
+
+@pytest.mark.parametrize("name", list(CASES2))
+def test_hier_super_nodes_match_oracle(name):
+    """Second level: super-node rows bit-exact; recursive radii, the largest
+    radius and the row-norm bound (now over the super-node rows too) within a
+    float32 ulp; the node level is unchanged by the second."""
+    c = case2(name)
+    p = params(c["pd"])
+    hp = ssa.make_hier_params(c["M"], c["probe"], levels=2)
+    _tab, nodes = gpu_nodes(c, p, hp)
+    check_no_device_error()
+    rows, rad, bnd = ssa.hier_node_views(p, hp, nodes)
+    nt, radius, r_star, _t1 = c["nodes"]
+    st, srad, r2, t2 = c["supers"]
+    assert np.array_equal(rows.float().cpu().numpy().astype(np.float64), nt)
+    assert _ulps(rad.cpu().numpy(), radius).max(initial=0) <= 1
+    g = bnd.cpu().numpy()
+    assert _ulps(g[..., 0], r_star).max() <= 1 and _ulps(g[..., 1], t2).max() <= 1
+    srows, sr, sb = ssa.hier_super_views(p, hp, nodes)
+    assert np.array_equal(srows.float().cpu().numpy().astype(np.float64), st)
+    assert _ulps(sr.cpu().numpy(), srad).max(initial=0) <= 1
+    assert _ulps(sb.cpu().numpy(), r2).max() <= 1
+
+
+def _decidable2(c, bi, i, g):
+    inf = c["info"][(bi, i, g)]
+    band = HIER_BAND * inf["scale"]
+    return (inf["super_gap"] >= band and inf["node_gap"] >= band and inf["kept_gap"] >= band
+            and all(not np.isfinite(b) or abs(inf["tau"] - b) >= band for b in inf["bounds"]))
+
+
+@pytest.mark.parametrize("name,impl", PAIRS2, ids=IDS2)
+def test_hier_two_levels_probe_and_certificates_match_oracle(name, impl):
+    c = case2(name)
+    op = c["op"]
+    p = params(c["pd"], impl)
+    hp = ssa.make_hier_params(c["M"], c["probe"], escalate=False, levels=2)
+    tab, nodes = gpu_nodes(c, p, hp)
+    gi, gc = gpu_hier(c, p, hp, tab, nodes)
+    assert set(np.unique(gc)) <= {0, 1}
+    checked = mism = cmis = 0
+    for bi in range(op.batch):
+        for i in range(op.n_q):
+            for g in range(op.h_kv):
+                if gc[bi, i, g] and c["gaps"][bi, i, g] >= 1e-5:   # a certified row holds the flat top-k
+                    assert np.array_equal(gi[bi, i, g], c["flat"][bi, i, g]), (bi, i, g)
+                if not _decidable2(c, bi, i, g):
+                    continue
+                checked += 1
+                mism += int(not np.array_equal(gi[bi, i, g], c["hb"][bi, i, g]))
+                cmis += int(bool(gc[bi, i, g]) != bool(c["hc"][bi, i, g]))
+    total = op.batch * op.n_q * op.h_kv
+    assert checked >= 0.8 * total, (checked, total)
+    assert mism == 0 and cmis == 0, (mism, cmis, checked)
+
+
+@pytest.mark.parametrize("name,impl", PAIRS2, ids=IDS2)
+def test_hier_two_levels_escalation_gives_the_flat_selection(name, impl):
+    c = case2(name)
+    p = params(c["pd"], impl)
+    hp = ssa.make_hier_params(c["M"], c["probe"], escalate=True, levels=2)
+    tab, nodes = gpu_nodes(c, p, hp)
+    gi, _gc = gpu_hier(c, p, hp, tab, nodes)
+    n, strict, _lit, _band = compare_idx(gi, c["flat"], c["gaps"])
+    assert strict == 0, f"{strict} of {n} rows differ from the flat top-k outside the near-tie band"

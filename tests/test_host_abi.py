@@ -206,12 +206,24 @@ def test_hier_params_layout_and_checks():
     no_esc = ssa.make_hier_params(fanout=8, probe=2, escalate=False)
     assert ssa.ssa_route_hier_workspace_size(p, ok) - ssa.ssa_route_hier_workspace_size(p, no_esc) == \
         rnd(bgs * tiles * 4)
+    # two levels: the super-node rows, radii and largest radius after the
+    # nodes; per row the super-node list (probe+1 entries and scores), the
+    # candidate-node count and the best unexpanded super-node score
+    two = ssa.make_hier_params(fanout=8, probe=2, escalate=True, levels=2)
+    ns = nn // 8
+    assert ssa.ssa_hier_nodes_size(p, two) == (ssa.ssa_hier_nodes_size(p, ok) + rnd(bgs * ns * 256 * 2)
+                                               + rnd(bgs * ns * 4) + rnd(bgs * 4))
+    assert ssa.ssa_route_hier_workspace_size(p, two) == (ssa.ssa_route_hier_workspace_size(p, ok)
+                                                         + 2 * rnd(rows * 3 * 4) + 2 * rnd(rows * 4))
+    assert ssa.ssa_hier_nodes_size(p, ssa.make_hier_params(fanout=8, probe=2, levels=0)) == \
+        ssa.ssa_hier_nodes_size(p, ssa.make_hier_params(fanout=8, probe=2, levels=1))
     for hp, code in ((ssa.make_hier_params(fanout=3), ssa.SSA_ERR_INVALID_ARG),      # not a power of two
                      (ssa.make_hier_params(fanout=128), ssa.SSA_ERR_INVALID_ARG),
                      (ssa.make_hier_params(probe=0), ssa.SSA_ERR_INVALID_ARG),
                      (ssa.make_hier_params(probe=32), ssa.SSA_ERR_INVALID_ARG),
-                     (ssa.ssa_hier_params(fanout=8, probe=2, escalate=2, reserved=0), ssa.SSA_ERR_INVALID_ARG),
-                     (ssa.ssa_hier_params(fanout=8, probe=2, escalate=0, reserved=1), ssa.SSA_ERR_INVALID_ARG),
+                     (ssa.ssa_hier_params(fanout=8, probe=2, escalate=2, levels=0), ssa.SSA_ERR_INVALID_ARG),
+                     (ssa.ssa_hier_params(fanout=8, probe=2, escalate=0, levels=3), ssa.SSA_ERR_INVALID_ARG),
+                     (ssa.ssa_hier_params(fanout=8, probe=2, escalate=0, levels=-1), ssa.SSA_ERR_INVALID_ARG),
                      (ssa.make_hier_params(fanout=64, probe=8), ssa.SSA_ERR_UNSUPPORTED)):   # 576 candidates
         assert ssa.ssa_hier_nodes_size(p, hp) == 0
         assert ssa.lib.ssa_hier_nodes(C.byref(p), C.byref(hp), dummy, dummy, None) == code
