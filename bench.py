@@ -3,6 +3,7 @@
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
                     [--workload NAME] [--no-secondary] [--no-cpu-baseline] [--no-e2e]
                     [--subblocks S] [--outlier] [--router flat|hier [--fanout M] [--probe P] [--escalate] [--levels L]]
+                    [--cluster-span S]
 
 One step is one pass of the whole layer over the workload's synthetic input:
 block summaries -> routing features + tensor-core route with fused top-k ->
@@ -666,6 +667,9 @@ def main():
     ap.add_argument("--probe", type=int, default=2)
     ap.add_argument("--escalate", action="store_true", help="re-route uncertified rows over all blocks")
     ap.add_argument("--levels", type=int, default=1, choices=[1, 2], help="tree levels of the hierarchical router")
+    ap.add_argument("--cluster-span", type=int, default=1,
+                    help="clustered keys: S consecutive blocks share a centroid (nearby blocks alike); "
+                         "a measurement of the routers on that structure, not the bench line")
     a = ap.parse_args()
     w = WORKLOADS[a.workload]
     if a.n is not None:
@@ -674,6 +678,10 @@ def main():
         w = w.scaled(subblocks=a.subblocks)
     if a.outlier:
         w = w.scaled(outlier=True)
+    if a.cluster_span != 1:
+        if not w.clustered or a.cluster_span < 1:
+            raise SystemExit("--cluster-span needs a clustered workload and S >= 1")
+        w = w.scaled(cluster_span=a.cluster_span)
     ws, rank, local = dist_setup(a.gpus)
     peaks, peak_src = load_peaks()
 
@@ -681,6 +689,7 @@ def main():
               "d": w.d, "block": w.block, "topk": w.topk, "window": w.window, "sigma": w.sigma,
               "subblocks": w.subblocks, "outlier": w.outlier,
               "beta": w.beta, "keys": "block-clustered + planted needles" if w.clustered else "iid + planted needles",
+              "cluster_span": w.cluster_span,
               "l2": "flushed between steps (256 MiB write); inputs larger than L2",
               "parallelism": f"replicas x{ws} (independent problems)"}
 
