@@ -17,7 +17,10 @@ collective on the data path): weak scaling.  The decode workload's block
 summaries (and, with --router hier, its node store) are precomputed state of
 the cache: built once before the timed steps and reported beside them.  The
 line gives the mean and the median step time, and the dominant kernel's
-roofline fraction against the measured peaks and the nominal ones.
+roofline fraction against the measured peaks and the nominal ones.  SM
+clocks and throttle reasons are sampled by nvidia-smi every 200 ms during
+the timed steps, on the GPU whose UUID is the CUDA device's (nvidia-smi's
+index can differ from the CUDA ordinal under CUDA_VISIBLE_DEVICES).
 
 `e2e` repeats the step through ssa_forward_hostio with page-locked host
 inputs and outputs, every step's host<->device copies inside the timed
@@ -131,6 +134,26 @@ def whole_job_rate(units_per_rank, ws, ms_max):
 
 # ------------------------------------------------------------------ clocks
 
+def smi_index(device, listing=None):
+    """The nvidia-smi index of CUDA device `device` (which may differ from
+    the CUDA ordinal when CUDA_VISIBLE_DEVICES remaps devices): matched by
+    UUID against `nvidia-smi --query-gpu=index,uuid` (or `listing`, its
+    output, for tests); the CUDA ordinal when nothing matches."""
+    try:
+        uuid = str(torch.cuda.get_device_properties(device).uuid).lower()
+        uuid = uuid[4:] if uuid.startswith("gpu-") else uuid
+        if listing is None:
+            listing = subprocess.run(["nvidia-smi", "--query-gpu=index,uuid", "--format=csv,noheader"],
+                                     capture_output=True, text=True, timeout=20).stdout
+        for line in listing.splitlines():
+            f = [x.strip() for x in line.split(",")]
+            if len(f) == 2 and uuid and f[1].lower().removeprefix("gpu-") == uuid:
+                return int(f[0])
+    except Exception:
+        pass
+    return int(device)
+
+
 class ClockSampler:
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
@@ -180,9 +203,9 @@ class ClockSampler:
                 if v.lower().startswith("active"):
                     reasons.add(n)
         if not sm:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0, "smi_index": self.gpu}
         return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
-                "samples": len(sm)}
+                "samples": len(sm), "smi_index": self.gpu}
 
 
 # ------------------------------------------------------------------ algorithmic work
@@ -406,7 +429,7 @@ def run_ours(w, steps, warmup, ws, rank, with_e2e=True, hier=None):
     barrier(ws)
     torch.cuda.synchronize()
     l0 = ssa.ssa_launch_count()
-    with ClockSampler(torch.cuda.current_device()) as clk:
+    with ClockSampler(smi_index(torch.cuda.current_device())) as clk:
         for k in range(steps):
             flush.zero_()
             step(evs[k])

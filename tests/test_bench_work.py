@@ -157,3 +157,22 @@ def test_layer_report_against_both_roofs():
               + 2 * w.h_kv * nb * 2 * w.d * 2 + 2 * w.n_q * w.h_kv * w.topk * 4)
     assert lay["compulsory_bytes"] == nbytes
     assert abs(lay["frac_hbm"] - nbytes / 2e-3 / 1e9 / 6000.0) < 1e-12
+
+
+def test_clock_sampler_follows_the_device_uuid(monkeypatch):
+    """With CUDA_VISIBLE_DEVICES remapping, CUDA device 0 may be nvidia-smi's
+    GPU 5: the sampler is pointed at the index whose UUID matches; with no
+    match (or no properties) it keeps the CUDA ordinal."""
+    class Props:
+        uuid = "0f1e2d3c-4b5a-6978-8796-a5b4c3d2e1f0"
+    listing = ("0, GPU-11111111-2222-3333-4444-555555555555\n"
+               "5, GPU-0F1E2D3C-4B5A-6978-8796-A5B4C3D2E1F0\n")
+    monkeypatch.setattr(torch.cuda, "get_device_properties", lambda d: Props())
+    assert bench.smi_index(0, listing) == 5
+    assert bench.smi_index(0, "0, GPU-11111111-2222-3333-4444-555555555555\n") == 0
+    assert bench.smi_index(2, "") == 2
+
+    def fail(d):
+        raise RuntimeError("no device")
+    monkeypatch.setattr(torch.cuda, "get_device_properties", fail)
+    assert bench.smi_index(1, listing) == 1
