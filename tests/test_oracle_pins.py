@@ -750,6 +750,55 @@ def test_hier_certificate_hand_cases_radius_and_margin():
         assert list(kept) == [0] and ok is want
 
 
+def test_hier_two_levels_hand_cases_recursive_radius_and_row_norm():
+    """Hand-computed two-level rows (d = 2, one key per block, M = 2, probe 1,
+    k = 1, f = [1, 0 ; 0, 0], the whole sequence visible).
+
+    Nodes are tight (two equal blocks each, R_N = 0, so R* = 0) and the
+    super-nodes' spread is all in the recursive radius.  Super-node 0 = nodes
+    {2, 2}, {0, 0}: centre 1, R_S = max(|2 - 1| + 0, |0 - 1| + 0) = 1.
+    (A) super-node 1 = nodes {-1, -1}, {2.5, 2.5}: centre 0.75,
+    R_S = 1.75.  The row expands super-node 0 (w 1 > 0.75), then node 0, and
+    keeps b0 with tau = 2; the node level holds (tau > 0 + 0 + margin) but the
+    super level's bound 0.75 + 1.75 = 2.5 does not -- rightly, b6 scores 2.5.
+    (B) super-node 1 = nodes {0.25, 0.25}, {1.25, 1.25}: centre 0.75,
+    R_S = 0.5, R2* = 1; bound 0.75 + 1 = 1.75 < 2: certified, and b0 is the
+    flat top-1.
+    Row norm: a super-node's cap takes each dimension's largest node cap, so
+    its row can be the longest one, and T* covers it."""
+    def run(means):
+        nb = len(means)
+        table = np.zeros((nb, 4))
+        table[:, 0] = means
+        p = O.Problem(1, nb, nb, 1, 1, 2, 1, 1, 1, dtype=O.BF16, sigma=O.DIAG)
+        nt, rad, rs, t1 = O.hier_nodes(table[None, None], 2)
+        st, srad, r2, t2 = O.hier_super_nodes(nt, rad, t1, 2)
+        kept, ok, info = O.hier_route_row2(np.array([1.0, 0, 0, 0]), table, (nt[0, 0], rad[0, 0], rs[0, 0], t1[0, 0]),
+                                           (st[0, 0], srad[0, 0], r2[0, 0], t2[0, 0]), nb - 1, p, 2, 1)
+        return kept, ok, info, rs[0, 0], srad[0, 0], r2[0, 0], t2[0, 0]
+    kept, ok, info, r1, srad, r2, t2 = run([2, 2, 0, 0, -1, -1, 2.5, 2.5])
+    assert r1 == 0.0 and list(srad) == [1.0, 1.75] and r2 == 1.75 and t2 == 2.5
+    assert list(info["super_expanded"]) == [0] and list(info["expanded"]) == [0]
+    assert list(kept) == [0] and info["tau"] == 2.0
+    m = 2.0 ** -12 * 1.0 * 2.5
+    assert info["bounds"][0] == pytest.approx(0.0 + m) and info["bounds"][1] == pytest.approx(2.5 + m)
+    assert not ok
+    kept, ok, info, r1, srad, r2, t2 = run([2, 2, 0, 0, 0.25, 0.25, 1.25, 1.25])
+    assert list(srad) == [1.0, 0.5] and r2 == 1.0
+    assert list(kept) == [0] and info["bounds"][1] == pytest.approx(1.75 + 2.0 ** -12 * 2.0)
+    assert ok
+    # the longest row is a super-node's: caps 1 in dimension 0 (node 0) and
+    # in dimension 1 (node 1) give the super row (0, 0 ; 1, 1), norm sqrt(2),
+    # against 1 for every block and node row
+    table = np.zeros((1, 1, 8, 4))
+    table[0, 0, 0:2, 2] = 1.0
+    table[0, 0, 2:4, 3] = 1.0
+    nt, rad, rs, t1 = O.hier_nodes(table, 2)
+    st, srad, r2, t2 = O.hier_super_nodes(nt, rad, t1, 2)
+    assert t1[0, 0] == 1.0
+    assert math.sqrt(2) <= t2[0, 0] <= math.sqrt(2) * (1 + 2.0 ** -23)
+
+
 def test_unquantised_selection_is_the_float32_route_of_the_same_summaries():
     """The informational unquantised selection of a bf16 problem is the float32
     problem's selection from the float32 summaries, and its scores are the
