@@ -494,6 +494,18 @@ def recovery_weight(beta: float, delta: float, mu: float) -> float:
 #     sides).  Every unexpanded block then scores below the k-th kept score,
 #     so the kept set is the exact top-k of all visible blocks;
 #   * escalation: an uncertified row is re-routed over all its visible blocks.
+#
+# Listed outlier blocks (optional, parameter lambda >= 1): block c of a
+# complete node N is listed when the 2-norm of its variance half s_c exceeds
+# lambda times the node's lower median of those norms (the (M/2)-th
+# smallest).  The node's centre, cap and radius then come from its unlisted
+# blocks only (the mean divides by their count; at least half of the blocks
+# are unlisted), and a row scores exactly every listed block of its complete
+# visible nodes beside the blocks of its expanded nodes and the tail.  The
+# bound and the certificate are unchanged: they now cover the unlisted
+# blocks, and every listed block is a candidate.  (A block whose variance
+# stands far above its neighbours' -- a block holding one extreme key --
+# would otherwise lift the node's cap in every dimension.)
 
 HIER_MARGIN = 2.0 ** -12
 
@@ -507,12 +519,32 @@ def round_up_f32(x) -> np.ndarray:
     return r.astype(np.float64)
 
 
-def hier_nodes(table: np.ndarray, fanout: int):
+def hier_listed_blocks(table: np.ndarray, fanout: int, factor: float) -> np.ndarray:
+    """listed [batch, h_kv, nb] (bool): block c of complete node N is listed
+    when ||s_c||_2 > factor * (the (M/2)-th smallest ||s||_2 of N's blocks),
+    s_c the variance half of its stored row; blocks outside complete nodes
+    are never listed."""
+    b, h, nb, kf = table.shape
+    d = kf // 2
+    M = fanout
+    nn = nb // M
+    vn = np.sqrt((np.asarray(table, dtype=np.float64)[..., d:] ** 2).sum(axis=-1))   # [b, h, nb]
+    listed = np.zeros((b, h, nb), dtype=bool)
+    if nn:
+        node_vn = vn[:, :, :nn * M].reshape(b, h, nn, M)
+        lower_median = np.sort(node_vn, axis=3)[..., M // 2 - 1] if M > 1 else node_vn[..., 0]
+        listed[:, :, :nn * M] = (node_vn > factor * lower_median[..., None]).reshape(b, h, nn * M)
+    return listed
+
+
+def hier_nodes(table: np.ndarray, fanout: int, listed=None):
     """Node summaries of a bf16 routing table [batch, h_kv, nb, 2d].
 
     Returns (node_table [batch, h_kv, nn, 2d] bf16 values, radius
     [batch, h_kv, nn], r_star [batch, h_kv], t_star [batch, h_kv]) with
     nn = nb // fanout; r_star / t_star are 0 when there are no nodes or rows.
+    listed [batch, h_kv, nb] (optional): blocks left out of their node's
+    centre, cap and radius.
     """
     b, h, nb, kf = table.shape
     d = kf // 2
@@ -520,10 +552,14 @@ def hier_nodes(table: np.ndarray, fanout: int):
     nn = nb // M
     T = np.asarray(table, dtype=np.float64)
     nodes = T[:, :, :nn * M].reshape(b, h, nn, M, kf)
-    centre = round_bf16(round_f32(nodes[..., :d].sum(axis=3) / M))
-    cap = nodes[..., d:].max(axis=3) if nn else np.zeros((b, h, 0, d))
+    keep = np.ones((b, h, nn, M), dtype=bool)
+    if listed is not None:
+        keep = ~np.asarray(listed, dtype=bool)[:, :, :nn * M].reshape(b, h, nn, M)
+    count = keep.sum(axis=3)
+    centre = round_bf16(round_f32((nodes[..., :d] * keep[..., None]).sum(axis=3) / np.maximum(count, 1)[..., None]))
+    cap = np.where(keep[..., None], nodes[..., d:], -np.inf).max(axis=3) if nn else np.zeros((b, h, 0, d))
     dist = np.sqrt(((nodes[..., :d] - centre[:, :, :, None, :]) ** 2).sum(axis=-1))   # [b, h, nn, M]
-    radius = round_up_f32(dist.max(axis=3)) if nn else np.zeros((b, h, 0))
+    radius = round_up_f32(np.where(keep, dist, 0.0).max(axis=3)) if nn else np.zeros((b, h, 0))
     node_table = np.concatenate([centre, cap], axis=-1)
     r_star = radius.max(axis=2) if nn else np.zeros((b, h))
     row_norm = np.sqrt((T ** 2).sum(axis=-1))
@@ -567,11 +603,13 @@ def hier_super_nodes(node_table: np.ndarray, radius: np.ndarray, t_star: np.ndar
 
 
 def hier_route_row(f: np.ndarray, table_bg: np.ndarray, nodes_bg, pos: int, p: Problem, fanout: int,
-                   probe: int):
+                   probe: int, listed_bg=None):
     """One (query row, kv-head) through the hierarchical router.
 
     f: the row's features [2d]; table_bg [nb, 2d]; nodes_bg = (node_table
-    [nn, 2d], radius [nn], r_star, t_star) of its (batch, kv-head).
+    [nn, 2d], radius [nn], r_star, t_star) of its (batch, kv-head);
+    listed_bg [nb] (optional): listed blocks, candidates of every row that
+    sees their node and no part of an expanded node's candidates.
     Returns (kept block_idx [k] ascending padded with -1, certified,
     info dict with the expanded nodes, the node gap and the kept-set gap).
     """
@@ -586,6 +624,10 @@ def hier_route_row(f: np.ndarray, table_bg: np.ndarray, nodes_bg, pos: int, p: P
     expanded = np.sort(order[:probe])
     cand = [np.arange(N * M, (N + 1) * M) for N in expanded] + [np.arange(nvn * M, nv)]
     cand = np.concatenate(cand).astype(np.int64)
+    if listed_bg is not None:
+        lst = np.asarray(listed_bg, dtype=bool)
+        in_nodes = cand < nvn * M
+        cand = np.concatenate([cand[~(in_nodes & lst[cand])], np.flatnonzero(lst[:nvn * M])]).astype(np.int64)
     s = table_bg[cand] @ f
     corder = np.lexsort((cand, -s))
     take = min(p.topk, cand.size)
@@ -663,20 +705,24 @@ def hier_route_row2(f: np.ndarray, table_bg: np.ndarray, nodes_bg, supers_bg, po
 
 
 def hier_route(Q: np.ndarray, stored, p: Problem, fanout: int, probe: int, escalate: bool = False,
-               rows=None, levels: int = 1):
+               rows=None, levels: int = 1, list_factor=None):
     """block_idx [batch, n_q, h_kv, k], certified [batch, n_q, h_kv] (bool) and
     per-row info of the hierarchical router (bf16 problems, S = 1).
 
     escalate: uncertified rows take the flat top-k of all visible blocks.
     rows: optional (batch, query row) pairs; other rows stay -2 / False.
     levels: 1 (nodes over blocks) or 2 (super-nodes over the nodes as well).
+    list_factor: lambda of the listed outlier blocks (one level only), or None.
     """
     if p.dtype != BF16 or p.subblocks != 1 or p.outlier:
         raise ValueError("the hierarchical router is defined on the bf16 routing table, S = 1")
     if levels not in (1, 2):
         raise ValueError("one or two tree levels")
+    if list_factor is not None and (levels != 1 or not list_factor >= 1.0):
+        raise ValueError("listed blocks: one tree level and a factor >= 1")
     _mu32, _sig32, table = stored
-    nodes = hier_nodes(table, fanout)
+    listed = hier_listed_blocks(table, fanout, list_factor) if list_factor is not None else None
+    nodes = hier_nodes(table, fanout, listed)
     supers = hier_super_nodes(nodes[0], nodes[1], nodes[3], fanout) if levels == 2 else None
     bidx = np.full((p.batch, p.n_q, p.h_kv, p.topk), -2, dtype=np.int64)
     cert = np.zeros((p.batch, p.n_q, p.h_kv), dtype=bool)
@@ -692,7 +738,8 @@ def hier_route(Q: np.ndarray, stored, p: Problem, fanout: int, probe: int, escal
             f = feats[bi][g, i]
             nb_g = (nodes[0][bi, g], nodes[1][bi, g], nodes[2][bi, g], nodes[3][bi, g])
             if levels == 1:
-                kept, ok, inf = hier_route_row(f, table[bi, g], nb_g, pos, p, fanout, probe)
+                kept, ok, inf = hier_route_row(f, table[bi, g], nb_g, pos, p, fanout, probe,
+                                               None if listed is None else listed[bi, g])
             else:
                 sb_g = (supers[0][bi, g], supers[1][bi, g], supers[2][bi, g], supers[3][bi, g])
                 kept, ok, inf = hier_route_row2(f, table[bi, g], nb_g, sb_g, pos, p, fanout, probe)

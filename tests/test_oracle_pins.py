@@ -799,6 +799,85 @@ def test_hier_two_levels_hand_cases_recursive_radius_and_row_norm():
     assert math.sqrt(2) <= t2[0, 0] <= math.sqrt(2) * (1 + 2.0 ** -23)
 
 
+def test_hier_listed_blocks_and_the_summaries_of_the_rest():
+    """Listed blocks by explicit enumeration (the variance half's 2-norm above
+    lambda times the node's (M/2)-th smallest); the node's centre, cap and
+    radius over its unlisted blocks written out; the node bound is
+    admissible for those blocks (features aimed at the farthest included);
+    a very large lambda lists nothing and gives the plain node summaries."""
+    rng = np.random.default_rng(47)
+    d, nb = 8, 64
+    mu = O.round_bf16(rng.standard_normal((1, 1, nb, d)))
+    sg = O.round_bf16(rng.chisquare(2, (1, 1, nb, d)) * rng.choice([1.0, 1.0, 1.0, 9.0], (1, 1, nb, 1)))
+    table = np.concatenate([mu, sg], axis=-1)
+    for M, lam in ((4, 1.5), (8, 2.0), (8, 1.0), (16, 3.0)):
+        listed = O.hier_listed_blocks(table, M, lam)
+        nt, rad, r_star, _t = O.hier_nodes(table, M, listed)
+        for N in range(nb // M):
+            ids = list(range(N * M, (N + 1) * M))
+            norms = [math.sqrt(float(sum(x * x for x in table[0, 0, c, d:]))) for c in ids]
+            lm = sorted(norms)[M // 2 - 1]
+            want = [norms[j] > lam * lm for j in range(M)]
+            assert [bool(listed[0, 0, c]) for c in ids] == want
+            keep = [c for c, lst in zip(ids, want) if not lst]
+            assert len(keep) >= M // 2
+            centre = O.round_bf16(O.round_f32(sum(table[0, 0, c, :d] for c in keep) / len(keep)))
+            np.testing.assert_array_equal(nt[0, 0, N, :d], centre)
+            np.testing.assert_array_equal(nt[0, 0, N, d:], np.max([table[0, 0, c, d:] for c in keep], axis=0))
+            far = max(float(np.linalg.norm(table[0, 0, c, :d] - centre)) for c in keep)
+            assert far <= rad[0, 0, N] <= far * (1 + 2.0 ** -23)
+            for trial in range(40):
+                fs = O.round_bf16(rng.standard_normal(d))
+                fq = O.round_bf16(np.abs(rng.standard_normal(d)))
+                if trial % 4 == 0:
+                    c = max(keep, key=lambda c: np.linalg.norm(table[0, 0, c, :d] - centre))
+                    fs, fq = O.round_bf16(table[0, 0, c, :d] - centre), np.zeros(d)
+                f = np.concatenate([fs, fq])
+                bound = nt[0, 0, N] @ f + np.linalg.norm(fs) * rad[0, 0, N]
+                assert max(table[0, 0, c] @ f for c in keep) <= bound + 1e-9
+    assert not O.hier_listed_blocks(table, 4, 1e30).any()
+    plain = O.hier_nodes(table, 4)
+    none = O.hier_nodes(table, 4, O.hier_listed_blocks(table, 4, 1e30))
+    for a, b in zip(plain, none):
+        np.testing.assert_array_equal(a, b)
+
+
+def test_hier_listed_blocks_certify_nodes_with_one_extreme_key():
+    """Nodes of alike blocks, a third of them holding one extreme key (its
+    block's variance is large in every dimension).  Without listing those
+    blocks lift their nodes' caps and the certificate rarely fires; listed
+    (lambda = 2), they are scored exactly and it fires on most rows.  Either
+    way a certified row holds the flat top-k, and escalation gives the flat
+    router on every row."""
+    rng = np.random.default_rng(48)
+    M, probe, topk = 4, 2, 4
+    p, Q, _ = _hier_problem(rng, n=512, topk=topk)      # the problem and its queries
+    # keys around one centre per node, then the extreme keys planted
+    n, h_kv, d, block = 512, 2, 16, 4
+    cen = 4.0 * rng.standard_normal((1, n // (M * block), h_kv, d))
+    K = np.repeat(cen, M * block, axis=1) + 0.1 * rng.standard_normal((1, n, h_kv, d))
+    for node in range(0, n // (M * block), 3):
+        j = node * M * block + int(rng.integers(0, M * block))
+        K[0, j] = 12.0 * rng.choice([-1.0, 1.0], (h_kv, d))
+    K = O.round_bf16(K)
+    stored = O.stored_summaries(*O.block_summaries(K, p), p)
+    rows = [(0, i) for i in range(64, p.n_q, 3)]
+    rates = {}
+    for lam in (None, 2.0):
+        bidx, cert, _ = O.hier_route(Q, stored, p, M, probe, rows=rows, list_factor=lam)
+        fired = 0
+        for (bi, i) in rows:
+            for g in range(p.h_kv):
+                if cert[bi, i, g]:
+                    fired += 1
+                    np.testing.assert_array_equal(bidx[bi, i, g], _flat(Q, stored, p, bi, i, g))
+        rates[lam] = fired / (len(rows) * p.h_kv)
+    assert rates[2.0] > 0.6 and rates[None] < 0.5 * rates[2.0]
+    flat, _ = O.route_topk(Q, stored, p)
+    b2, _c, _ = O.hier_route(Q, stored, p, M, 1, escalate=True, list_factor=2.0)
+    np.testing.assert_array_equal(b2, flat)
+
+
 def test_unquantised_selection_is_the_float32_route_of_the_same_summaries():
     """The informational unquantised selection of a bf16 problem is the float32
     problem's selection from the float32 summaries, and its scores are the
