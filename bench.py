@@ -18,7 +18,7 @@ summaries (and, with --router hier, its node store) are precomputed state of
 the cache: built once before the timed steps and reported beside them.  The
 line gives the mean and the median step time, and the dominant kernel's
 roofline fraction against the measured peaks and the nominal ones.  SM
-clocks and throttle reasons are sampled by nvidia-smi every 200 ms during
+clocks and throttle reasons are sampled by nvidia-smi every 100 ms during
 the timed steps, on the GPU whose UUID is the CUDA device's (nvidia-smi's
 index can differ from the CUDA ordinal under CUDA_VISIBLE_DEVICES).
 
@@ -168,7 +168,7 @@ class ClockSampler:
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                 "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
             self.t = threading.Thread(target=self._read, daemon=True)
             self.t.start()
         except Exception:
